@@ -1,0 +1,194 @@
+/*
+ * ra.h -- C ABI of the B200 (sm_100a) ring-chunked attention and Ulysses
+ * layout-transform library (libra_b200.so).
+ *
+ * Sources, cited by page title and section:
+ *   [SP-QA]   "Как работает sequence parallelism в контексте LLM?" (Q&A page on
+ *             sequence parallelism): section 2 "Базовый принцип: разрезание
+ *             последовательности" (contiguous chunking), section 3 "Ring
+ *             Attention — эффективная коммуникация" (the P-step ring), section 5
+ *             "Практическая реализация: псевдокод ring attention" (per-chunk
+ *             scores, online-softmax / log-sum-exp merge, final normalisation).
+ *   [ULYSSES] "Метод контекстного параллелизма Ulysses" (post on Ulysses context
+ *             parallelism): the all-to-all from [local_seqlen, global_heads,
+ *             head_dim] to [global_seqlen, local_heads, head_dim] and back, and
+ *             the GQA rule that KV heads are copied up to the CP-group size.
+ *   [ACCEL-SP] "Paralelismo de secuencias en 🤗 accelerate", section "En qué se
+ *             diferencia Ulysses SP de FSDP CP": Ulysses needs the head count
+ *             divisible by the number of ranks; ring attention does not.
+ *
+ * The P "ranks" of the ring are virtual: P chunk partitions held in the memory
+ * of one GPU. Nothing here communicates between devices.
+ *
+ * Conventions shared by every entry point
+ *   - Every tensor pointer is a DEVICE pointer into memory the caller owns and
+ *     keeps alive until the work queued on `stream` has finished.  The library
+ *     allocates no device memory and keeps no reference after the call returns.
+ *   - Arrays of chunk pointers (k_chunks, v_chunks) are HOST arrays of device
+ *     pointers; they are read during the call only.
+ *   - Every tensor is dense, row-major, in the element type named by its dtype
+ *     argument, unless a stride argument says otherwise.  Every device pointer
+ *     must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Work is enqueued asynchronously; the return status covers argument
+ *     validation and the launch only.  A kernel that gives up on a bounded
+ *     internal wait records that in a per-device error word, which
+ *     ra_sync_status() reads back.
+ *   - On any status other than RA_OK nothing has been enqueued, except for
+ *     RA_ERR_CUDA after a failed launch, and ra_last_error() returns a message
+ *     describing the problem (thread-local, valid until the next call on the
+ *     same thread).
+ *   - Outputs must not alias inputs unless an entry point says so.
+ */
+#ifndef RA_B200_H
+#define RA_B200_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RA_OK = 0,
+    RA_ERR_INVALID = 1,      /* bad argument: null/misaligned pointer, bad size or divisibility */
+    RA_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement (e.g. D not in {32,64,128}) */
+    RA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed; see ra_last_error() */
+    RA_ERR_TIMEOUT = 4       /* a kernel gave up on a bounded internal wait; outputs are undefined */
+} ra_status;
+
+typedef enum {
+    RA_BF16 = 0,  /* bfloat16, 2 bytes */
+    RA_FP32 = 1   /* IEEE binary32, 4 bytes */
+} ra_dtype;
+
+/*
+ * ra_ring_attn_fwd -- exact attention of every query row against P K/V chunks,
+ * computed chunk by chunk in ring order with an online-softmax (log-sum-exp)
+ * merge after each chunk step.  [SP-QA] sections 2, 3 and 5.
+ *
+ * Sequence: global length L = P*Lc.  Virtual rank i owns the contiguous tokens
+ * [i*Lc, (i+1)*Lc) ([SP-QA] section 2).  For the queries of rank i, chunk step s
+ * (s = 0..P-1) attends to the K/V chunk j = (i - s) mod P ([SP-QA] section 3:
+ * each rank passes its chunk to the next rank, so at step s it holds the chunk
+ * of rank i-s), and merges the partial result into the running one by the
+ * log-sum-exp rule of [SP-QA] section 5.
+ *
+ * Result, per batch b, query position t, query head h (kv head g = h/(H_q/H_kv)):
+ *   s_j      = scale * sum_d q[b,t,h,d] * k[b,j,g,d]   for visible j
+ *   lse      = log(sum_j exp(s_j))                       (natural log)
+ *   out[...] = sum_j exp(s_j - lse) * v[b,j,g,:]
+ * Visible keys: all j < L, or with causal != 0 the keys j <= t (global
+ * positions in rank order).  Chunk pairs whose keys are all invisible issue no
+ * work.  Every query row sees at least one key.
+ *
+ * Arguments
+ *   q          device, in_dtype, [B][P*Lc][H_q][D]; batch b starts at
+ *              q + b*q_bstride elements (q_bstride >= P*Lc*H_q*D).
+ *   k_chunks   host array of P device pointers; chunk j is [B][Lc][H_kv][D]
+ *              in_dtype, batch b of chunk j starts at k_chunks[j] + b*kv_bstride
+ *              elements (kv_bstride >= Lc*H_kv*D).
+ *   v_chunks   as k_chunks, same kv_bstride.
+ *   P          number of virtual ranks, 1 <= P <= RA_MAX_P.
+ *   B, H_q, H_kv, Lc, D   sizes; H_q % H_kv == 0 (grouped-query attention).
+ *   scale      multiplier of the raw scores (typically 1/sqrt(D)).
+ *   causal     0 or 1.
+ *   in_dtype   RA_BF16 (tcgen05 tensor-core path; D in {64,128}) or RA_FP32
+ *              (CUDA-core fp32 path; D in {32,64,128}).
+ *   out_dtype  RA_FP32 or RA_BF16 (BF16 only with in_dtype RA_BF16).
+ *   out        device, out_dtype, dense [B][P*Lc][H_q][D] (normalised output).
+ *   lse        device, fp32, dense [B][H_q][P*Lc], natural-log log-sum-exp.
+ *   stream     cudaStream_t.
+ * Errors: RA_ERR_INVALID for null or misaligned pointers, P < 1 or P > RA_MAX_P,
+ *   B/H_q/H_kv/Lc < 1, H_q % H_kv != 0, strides below the dense size, causal
+ *   not in {0,1}, out_dtype BF16 with fp32 input; RA_ERR_UNSUPPORTED for D
+ *   outside the lists above.
+ */
+#define RA_MAX_P 64
+ra_status ra_ring_attn_fwd(const void* q, const void* const* k_chunks, const void* const* v_chunks,
+                           int P, int B, int H_q, int H_kv, int Lc, int D,
+                           long long q_bstride, long long kv_bstride,
+                           float scale, int causal, ra_dtype in_dtype, ra_dtype out_dtype,
+                           void* out, float* lse, void* stream);
+
+/*
+ * ra_lse_merge -- merge two partial attention results over disjoint key sets
+ * into one, in place into (o_a, lse_a).  [SP-QA] section 5 (the merge step of
+ * the ring loop, read as the exact log-sum-exp combination):
+ *   lse      = log(exp(lse_a) + exp(lse_b))
+ *   o_a[...] = exp(lse_a - lse) * o_a + exp(lse_b - lse) * o_b
+ * A partial over no visible key is (o = anything finite, lse = -inf); merging
+ * with it leaves the other side unchanged, and two such partials merge to
+ * (0, -inf).
+ *   o_a, o_b     device fp32, [B][L][H][D]  (o_a is read and overwritten)
+ *   lse_a, lse_b device fp32, [B][H][L]     (lse_a is read and overwritten)
+ * o_b/lse_b must not alias o_a/lse_a.  Errors: RA_ERR_INVALID for null or
+ * misaligned pointers or sizes < 1; RA_ERR_UNSUPPORTED if D % 4 != 0.
+ */
+ra_status ra_lse_merge(float* o_a, float* lse_a, const float* o_b, const float* lse_b,
+                       int B, int H, long long L, int D, void* stream);
+
+/*
+ * ra_ulysses_seq2head -- the Ulysses layout transform from sequence-sharded to
+ * head-sharded activations, for all P virtual ranks at once.  [ULYSSES]: the
+ * all-to-all that turns [local_seqlen, global_heads, head_dim] into
+ * [global_seqlen, local_heads, head_dim]; with GQA the KV heads are first
+ * copied up so that every rank gets one ([ULYSSES], [ACCEL-SP]).
+ *
+ *   in   device, dt, [P][B][Lc][H_in][D]   (rank s holds tokens s*Lc .. s*Lc+Lc-1)
+ *   out  device, dt, [P][B][P*Lc][H_out/P][D]
+ *   out[r][b][s*Lc+t][h'][:] = in[s][b][t][ ((r*H_out/P + h') * H_in) / H_out ][:]
+ * Rank r receives the contiguous head block [r*H_out/P, (r+1)*H_out/P) of the
+ * H_out (replicated) heads; replica j of the H_out heads is a copy of source
+ * head floor(j*H_in/H_out) (repeat-interleave).  H_out == H_in is the plain
+ * transform.  The copy is bit-exact.
+ * Errors: RA_ERR_INVALID for null/misaligned pointers, sizes < 1,
+ *   H_out % P != 0 (heads must divide among ranks), H_out % H_in != 0,
+ *   D*sizeof(dt) % 16 != 0.
+ */
+ra_status ra_ulysses_seq2head(const void* in, void* out, int P, int B, int Lc,
+                              int H_in, int H_out, int D, ra_dtype dt, void* stream);
+
+/*
+ * ra_ulysses_head2seq -- the inverse transform, after attention and before the
+ * output projection ([ULYSSES]):
+ *   in   device, dt, [P][B][P*Lc][H/P][D]
+ *   out  device, dt, [P][B][Lc][H][D]
+ *   out[s][b][t][r*H/P + h'][:] = in[r][b][s*Lc+t][h'][:]
+ * Bit-exact.  Errors as ra_ulysses_seq2head (H % P != 0 is RA_ERR_INVALID).
+ */
+ra_status ra_ulysses_head2seq(const void* in, void* out, int P, int B, int Lc,
+                              int H, int D, ra_dtype dt, void* stream);
+
+/*
+ * ra_sync_status -- synchronise `stream`, then read and clear this device's
+ * kernel error word.  Returns RA_ERR_TIMEOUT if a kernel launched since the
+ * last call gave up on a bounded wait, RA_ERR_CUDA if the synchronisation
+ * itself failed, RA_OK otherwise.
+ */
+ra_status ra_sync_status(void* stream);
+
+/* Thread-local description of the last non-OK status returned on this thread. */
+const char* ra_last_error(void);
+
+/*
+ * ra_set_wait_limit_ns -- bound, in nanoseconds, on every internal spin-wait of
+ * the tensor-core attention kernel (default 4e9).  Takes effect at the next
+ * launch.  Returns the previous value.  ns == 0 restores the default.
+ */
+unsigned long long ra_set_wait_limit_ns(unsigned long long ns);
+
+/*
+ * ra_debug_inject_stall -- test hook.  With on != 0 the next tensor-core
+ * attention launch on this thread withholds one K tile load, so the consumer's
+ * bounded wait expires, the kernel drains and exits, and ra_sync_status()
+ * returns RA_ERR_TIMEOUT.  No fault and no unbounded wait is involved.  The
+ * hook disarms itself after that launch.
+ */
+void ra_debug_inject_stall(int on);
+
+/* Library version string. */
+const char* ra_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RA_B200_H */

@@ -1,0 +1,170 @@
+"""fp64 CPU oracle for ring-chunked attention, the log-sum-exp merge and the
+Ulysses layout transforms.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` are the only callers.  The oracle shares no code
+with the CUDA library (``sequence_parallelism_attn_b200``) and neither imports
+the other.  The arithmetic lives in ``ra_oracle.cpp`` (plain loops, fp64); this
+module only builds it and marshals numpy arrays.
+
+Sources: "Как работает sequence parallelism в контексте LLM?" sections 2, 3, 5
+(chunking, the ring, the per-chunk softmax and its merge) and "Метод
+контекстного параллелизма Ulysses" (the seq<->head all-to-all and the GQA copy).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ra_oracle.cpp")
+_LIB_PATH = os.path.join(_HERE, "libra_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ra_oracle.cpp into libra_oracle.so (plain g++, IEEE fp64, no fast-math)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + ".tmp"
+    cmd = ["g++", "-O2", "-std=c++17", "-fPIC", "-shared", "-pthread", "-ffp-contract=off",
+           "-o", tmp, _SRC]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    build()
+    lib = ctypes.CDLL(_LIB_PATH)
+    P = ctypes.c_void_p
+    i32, i64, f64 = ctypes.c_int, ctypes.c_longlong, ctypes.c_double
+    lib.ora_attention.argtypes = [P, P, P, i32, i64, i32, i32, i32, f64, i32, P, P, i32]
+    lib.ora_attention_rows.argtypes = [P, P, P, P, i64, P, P, i32, i64, i32, i32, i32, f64, i32,
+                                       P, P, i32]
+    lib.ora_ring_attention.argtypes = [P, P, P, i32, i32, i64, i32, i32, i32, f64, i32, P, P, P,
+                                       i32]
+    lib.ora_lse_merge.argtypes = [P, P, P, P, i32, i32, i64, i32]
+    lib.ora_seq2head.argtypes = [P, P, i32, i32, i64, i32, i32, i32, i32]
+    lib.ora_head2seq.argtypes = [P, P, i32, i32, i64, i32, i32, i32]
+    for f in ("ora_attention", "ora_attention_rows", "ora_ring_attention", "ora_lse_merge",
+              "ora_seq2head", "ora_head2seq"):
+        getattr(lib, f).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise ValueError(f"oracle {what}: invalid arguments")
+
+
+def attention(q, k, v, scale: float, causal: bool, nthreads: int = 0):
+    """Plain attention.  q [B,L,H_q,D], k/v [B,L,H_kv,D] -> (out [B,L,H_q,D], lse [B,H_q,L])."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, L, H_q, D = q.shape
+    H_kv = k.shape[2]
+    assert k.shape == (B, L, H_kv, D) and v.shape == k.shape
+    out = np.empty((B, L, H_q, D), np.float64)
+    lse = np.empty((B, H_q, L), np.float64)
+    rc = _load().ora_attention(_ptr(q), _ptr(k), _ptr(v), B, L, H_q, H_kv, D, float(scale),
+                               int(bool(causal)), _ptr(out), _ptr(lse), nthreads)
+    _check(rc, "attention")
+    return out, lse
+
+
+def attention_rows(q_rows, rb, rt, rh, k, v, H_q: int, scale: float, causal: bool,
+                   nthreads: int = 0):
+    """Plain attention for sampled query rows.
+
+    q_rows [n,D] are the query vectors of rows (rb[i], rt[i], rh[i]); k/v [B,L,H_kv,D].
+    Returns (out [n,D], lse [n]).
+    """
+    q_rows, k, v = _f64(q_rows), _f64(k), _f64(v)
+    rb = np.ascontiguousarray(rb, dtype=np.int32)
+    rt = np.ascontiguousarray(rt, dtype=np.int64)
+    rh = np.ascontiguousarray(rh, dtype=np.int32)
+    n, D = q_rows.shape
+    B, L, H_kv, Dk = k.shape
+    assert Dk == D and v.shape == k.shape and rb.shape == rt.shape == rh.shape == (n,)
+    out = np.empty((n, D), np.float64)
+    lse = np.empty((n,), np.float64)
+    rc = _load().ora_attention_rows(_ptr(q_rows), _ptr(rb), _ptr(rt), _ptr(rh), n, _ptr(k),
+                                    _ptr(v), B, L, H_q, H_kv, D, float(scale), int(bool(causal)),
+                                    _ptr(out), _ptr(lse), nthreads)
+    _check(rc, "attention_rows")
+    return out, lse
+
+
+def ring_attention(q, k_chunks, v_chunks, scale: float, causal: bool, step_offset=None,
+                   nthreads: int = 0):
+    """Ring form.  q [B,P*Lc,H_q,D]; k_chunks/v_chunks [P,B,Lc,H_kv,D] -> (out, lse).
+
+    Rank i visits chunk (i - step_offset[s]) mod P at step s (default: ring order s)."""
+    q, kc, vc = _f64(q), _f64(k_chunks), _f64(v_chunks)
+    P, B, Lc, H_kv, D = kc.shape
+    H_q = q.shape[2]
+    assert q.shape == (B, P * Lc, H_q, D) and vc.shape == kc.shape
+    so = None
+    if step_offset is not None:
+        so = np.ascontiguousarray(step_offset, dtype=np.int32)
+        assert so.shape == (P,)
+    out = np.empty((B, P * Lc, H_q, D), np.float64)
+    lse = np.empty((B, H_q, P * Lc), np.float64)
+    rc = _load().ora_ring_attention(_ptr(q), _ptr(kc), _ptr(vc), P, B, Lc, H_q, H_kv, D,
+                                    float(scale), int(bool(causal)),
+                                    _ptr(so) if so is not None else None, _ptr(out), _ptr(lse),
+                                    nthreads)
+    _check(rc, "ring_attention")
+    return out, lse
+
+
+def lse_merge(o_a, lse_a, o_b, lse_b):
+    """Merge of two partials.  o [B,L,H,D], lse [B,H,L] -> new (o, lse) (inputs untouched)."""
+    o = _f64(o_a).copy()
+    l = _f64(lse_a).copy()
+    ob, lb = _f64(o_b), _f64(lse_b)
+    B, L, H, D = o.shape
+    assert l.shape == (B, H, L) and ob.shape == o.shape and lb.shape == l.shape
+    _check(_load().ora_lse_merge(_ptr(o), _ptr(l), _ptr(ob), _ptr(lb), B, H, L, D), "lse_merge")
+    return o, l
+
+
+def seq2head(x: np.ndarray, H_out: int) -> np.ndarray:
+    """[P,B,Lc,H_in,D] -> [P,B,P*Lc,H_out/P,D], any dtype, bit-exact."""
+    x = np.ascontiguousarray(x)
+    P, B, Lc, H_in, D = x.shape
+    if H_out % P or H_out % H_in:
+        raise ValueError("seq2head: H_out must divide by P and by H_in")
+    out = np.empty((P, B, P * Lc, H_out // P, D), x.dtype)
+    _check(_load().ora_seq2head(_ptr(x), _ptr(out), P, B, Lc, H_in, H_out, D, x.itemsize),
+           "seq2head")
+    return out
+
+
+def head2seq(x: np.ndarray) -> np.ndarray:
+    """[P,B,P*Lc,H/P,D] -> [P,B,Lc,H,D], any dtype, bit-exact."""
+    x = np.ascontiguousarray(x)
+    P, B, L, Hl, D = x.shape
+    if L % P:
+        raise ValueError("head2seq: global length must divide by P")
+    Lc = L // P
+    out = np.empty((P, B, Lc, Hl * P, D), x.dtype)
+    _check(_load().ora_head2seq(_ptr(x), _ptr(out), P, B, Lc, Hl * P, D, x.itemsize),
+           "head2seq")
+    return out

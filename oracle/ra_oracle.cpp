@@ -1,0 +1,316 @@
+// ra_oracle.cpp -- plain, slow fp64 CPU oracle for ring-chunked attention, the
+// log-sum-exp merge and the Ulysses layout transforms.
+//
+// TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU
+// baseline leg of the benchmark load this library.  It shares no code, header,
+// table or helper with the CUDA library; the two see the same inputs only.
+//
+// Sources (cited by page title and section):
+//   [SP-QA]    "Как работает sequence parallelism в контексте LLM?":
+//              section 2 (contiguous chunking: rank i owns tokens
+//              i*L/P .. (i+1)*L/P-1), section 3 (the ring: each step a rank
+//              attends its queries to the K/V chunk it holds, passes that chunk
+//              on and receives the previous rank's; P-1 exchanges), section 5
+//              (per-chunk scores, row max, exp, sum, the online-softmax merge,
+//              final division by the normaliser).
+//   [ULYSSES]  "Метод контекстного параллелизма Ulysses": all-to-all from
+//              [local_seqlen, global_heads, head_dim] to
+//              [global_seqlen, local_heads, head_dim] and back; GQA KV heads
+//              copied up to the CP-group size.
+//
+// Readings taken where the pages are silent or inconsistent (each is listed
+// with its reason in the design notes of the repository):
+//   * scores are multiplied by an explicit `scale` (the pseudocode has none);
+//   * "lse" is the true natural-log log-sum-exp of the scaled scores, not the
+//     row max the pseudocode stores under that name;
+//   * the merge of two partials is the exact log-sum-exp combination
+//       lse = log(e^lse_a + e^lse_b), o = e^(lse_a-lse) o_a + e^(lse_b-lse) o_b
+//     (the pseudocode's update reuses the first step's weights and drops the
+//     factor on the new term);
+//   * at ring step s, rank i holds chunk (i - s) mod P (the stated intent of
+//     section 3; the pseudocode re-sends its own chunk every step);
+//   * causal masking, absent from the pages, is the global mask over the
+//     concatenation of chunks in rank order, key position <= query position;
+//   * GQA: query head h reads kv head h / (H_q / H_kv);
+//   * Ulysses rank r receives the contiguous head block [r*H/P, (r+1)*H/P),
+//     the global sequence is source-rank-major, and KV replica j of H_out is
+//     source head floor(j * H_in / H_out).
+//
+// Everything is fp64.  Inputs arrive as fp64 arrays holding the exact values
+// of the bf16/fp32 inputs.  Threads (std::thread) split independent query rows;
+// each row is computed by the same sequential loop whatever the thread count.
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <limits>
+#include <thread>
+#include <vector>
+#include <algorithm>
+
+namespace {
+
+const double NEG_INF = -std::numeric_limits<double>::infinity();
+
+int pick_threads(int requested, long long work_items) {
+    int n = requested > 0 ? requested : (int)std::thread::hardware_concurrency();
+    if (n < 1) n = 1;
+    if ((long long)n > work_items) n = (int)std::max<long long>(1, work_items);
+    return n;
+}
+
+template <class F>
+void parallel_for(long long n_items, int nthreads, F body) {
+    int nt = pick_threads(nthreads, n_items);
+    if (nt == 1) {
+        for (long long i = 0; i < n_items; ++i) body(i);
+        return;
+    }
+    std::vector<std::thread> pool;
+    pool.reserve(nt);
+    for (int w = 0; w < nt; ++w) {
+        pool.emplace_back([=]() {
+            for (long long i = w; i < n_items; i += nt) body(i);
+        });
+    }
+    for (auto& th : pool) th.join();
+}
+
+// Attention of one query vector against keys [key_begin, key_end) of one
+// (batch, kv head) sequence, by the plain definition ([SP-QA] section 5,
+// read with the true log-sum-exp):
+//   s_j = scale * <q, k_j>;  lse = log sum_j exp(s_j);  o = sum_j exp(s_j - lse) v_j
+// `key_visible(j)` decides the mask.  With no visible key: o = 0, lse = -inf.
+// k, v point at token 0 of the sequence, consecutive tokens `tok_stride` apart.
+template <class Visible>
+void attend_one(const double* qv, const double* k, const double* v, long long tok_stride,
+                long long key_begin, long long key_end, int D, double scale, Visible key_visible,
+                std::vector<double>& s, double* o, double* lse_out) {
+    s.assign((size_t)std::max<long long>(0, key_end - key_begin), NEG_INF);
+    double m = NEG_INF;
+    for (long long j = key_begin; j < key_end; ++j) {
+        if (!key_visible(j)) continue;
+        const double* kj = k + j * tok_stride;
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d) dot += qv[d] * kj[d];
+        double sj = scale * dot;
+        s[(size_t)(j - key_begin)] = sj;
+        if (sj > m) m = sj;
+    }
+    for (int d = 0; d < D; ++d) o[d] = 0.0;
+    if (m == NEG_INF) {  // no visible key
+        *lse_out = NEG_INF;
+        return;
+    }
+    double sum = 0.0;
+    for (long long j = key_begin; j < key_end; ++j) {
+        double sj = s[(size_t)(j - key_begin)];
+        if (sj == NEG_INF) continue;
+        sum += std::exp(sj - m);
+    }
+    double lse = m + std::log(sum);
+    for (long long j = key_begin; j < key_end; ++j) {
+        double sj = s[(size_t)(j - key_begin)];
+        if (sj == NEG_INF) continue;
+        double w = std::exp(sj - lse);
+        const double* vj = v + j * tok_stride;
+        for (int d = 0; d < D; ++d) o[d] += w * vj[d];
+    }
+    *lse_out = lse;
+}
+
+// The exact merge of two partials over disjoint key sets ([SP-QA] section 5,
+// merge step).  (o_a, lse_a) <- (o_a, lse_a) (+) (o_b, lse_b).
+void merge_into(double* o_a, double* lse_a, const double* o_b, double lse_b, int D) {
+    double la = *lse_a;
+    if (lse_b == NEG_INF) {
+        if (la == NEG_INF)
+            for (int d = 0; d < D; ++d) o_a[d] = 0.0;
+        return;
+    }
+    if (la == NEG_INF) {
+        for (int d = 0; d < D; ++d) o_a[d] = o_b[d];
+        *lse_a = lse_b;
+        return;
+    }
+    double mx = std::max(la, lse_b);
+    double lse = mx + std::log(std::exp(la - mx) + std::exp(lse_b - mx));
+    double wa = std::exp(la - lse), wb = std::exp(lse_b - lse);
+    for (int d = 0; d < D; ++d) o_a[d] = wa * o_a[d] + wb * o_b[d];
+    *lse_a = lse;
+}
+
+}  // namespace
+
+extern "C" {
+
+// Plain (unchunked) attention, the definition every other form must equal.
+//   q   [B][L][H_q][D]     k, v [B][L][H_kv][D]
+//   out [B][L][H_q][D]     lse  [B][H_q][L]
+int ora_attention(const double* q, const double* k, const double* v, int B, long long L, int H_q,
+                  int H_kv, int D, double scale, int causal, double* out, double* lse,
+                  int nthreads) {
+    if (B < 1 || L < 1 || H_q < 1 || H_kv < 1 || D < 1 || H_q % H_kv != 0) return 1;
+    const int group = H_q / H_kv;
+    const long long n_rows = (long long)B * H_q * L;
+    parallel_for(n_rows, nthreads, [&](long long row) {
+        thread_local std::vector<double> s;
+        const long long t = row % L;
+        const int h = (int)((row / L) % H_q);
+        const int b = (int)(row / L / H_q);
+        const int g = h / group;
+        const double* qv = q + (((long long)b * L + t) * H_q + h) * D;
+        const double* kb = k + ((long long)b * L * H_kv + g) * D;
+        const double* vb = v + ((long long)b * L * H_kv + g) * D;
+        double* o = out + (((long long)b * L + t) * H_q + h) * D;
+        auto visible = [&](long long j) { return !causal || j <= t; };
+        attend_one(qv, kb, vb, (long long)H_kv * D, 0, L, D, scale, visible, s, o,
+                   lse + ((long long)b * H_q + h) * L + t);
+    });
+    return 0;
+}
+
+// The same definition for a sample of query rows (b_i, t_i, h_i), for parity
+// checks at sizes where computing every row is too slow.
+//   q_rows [n][D] (the sampled query vectors)   k, v [B][L][H_kv][D]
+//   out [n][D]   lse [n]
+int ora_attention_rows(const double* q_rows, const int* rb, const long long* rt, const int* rh,
+                       long long n, const double* k, const double* v, int B, long long L, int H_q,
+                       int H_kv, int D, double scale, int causal, double* out, double* lse,
+                       int nthreads) {
+    if (B < 1 || L < 1 || H_q < 1 || H_kv < 1 || D < 1 || H_q % H_kv != 0) return 1;
+    for (long long i = 0; i < n; ++i)
+        if (rb[i] < 0 || rb[i] >= B || rt[i] < 0 || rt[i] >= L || rh[i] < 0 || rh[i] >= H_q)
+            return 1;
+    const int group = H_q / H_kv;
+    parallel_for(n, nthreads, [&](long long i) {
+        thread_local std::vector<double> s;
+        const long long t = rt[i];
+        const int g = rh[i] / group;
+        const double* kb = k + ((long long)rb[i] * L * H_kv + g) * D;
+        const double* vb = v + ((long long)rb[i] * L * H_kv + g) * D;
+        auto visible = [&](long long j) { return !causal || j <= t; };
+        attend_one(q_rows + i * D, kb, vb, (long long)H_kv * D, 0, L, D, scale, visible, s,
+                   out + i * D, lse + i);
+    });
+    return 0;
+}
+
+// The ring form ([SP-QA] sections 2, 3, 5): queries of rank i attend, at step
+// s = 0..P-1, to the chunk j = (i - step_offset[s]) mod P, and each partial is
+// merged into the running result.  step_offset == NULL means the ring order
+// step_offset[s] = s.  Any permutation of 0..P-1 gives another visiting order.
+//   q  [B][P*Lc][H_q][D]    k, v [P][B][Lc][H_kv][D] (chunk j = rank j's K/V)
+//   out [B][P*Lc][H_q][D]   lse [B][H_q][P*Lc]
+int ora_ring_attention(const double* q, const double* k_chunks, const double* v_chunks, int P,
+                       int B, long long Lc, int H_q, int H_kv, int D, double scale, int causal,
+                       const int* step_offset, double* out, double* lse, int nthreads) {
+    if (P < 1 || B < 1 || Lc < 1 || H_q < 1 || H_kv < 1 || D < 1 || H_q % H_kv != 0) return 1;
+    if (step_offset) {
+        std::vector<int> seen(P, 0);
+        for (int s = 0; s < P; ++s) {
+            if (step_offset[s] < 0 || step_offset[s] >= P || seen[step_offset[s]]) return 1;
+            seen[step_offset[s]] = 1;
+        }
+    }
+    const long long L = (long long)P * Lc;
+    const int group = H_q / H_kv;
+    const long long chunk_elems = (long long)B * Lc * H_kv * D;
+    const long long n_rows = (long long)B * H_q * L;
+    parallel_for(n_rows, nthreads, [&](long long row) {
+        thread_local std::vector<double> s;
+        thread_local std::vector<double> o_part;
+        const long long t = row % L;
+        const int h = (int)((row / L) % H_q);
+        const int b = (int)(row / L / H_q);
+        const int g = h / group;
+        const int i = (int)(t / Lc);  // rank owning this query
+        const double* qv = q + (((long long)b * L + t) * H_q + h) * D;
+        double* o = out + (((long long)b * L + t) * H_q + h) * D;
+        double* l = lse + ((long long)b * H_q + h) * L + t;
+        for (int d = 0; d < D; ++d) o[d] = 0.0;
+        *l = NEG_INF;
+        o_part.assign(D, 0.0);
+        for (int step = 0; step < P; ++step) {
+            const int off = step_offset ? step_offset[step] : step;
+            const int j = ((i - off) % P + P) % P;
+            const double* kc = k_chunks + j * chunk_elems + ((long long)b * Lc * H_kv + g) * D;
+            const double* vc = v_chunks + j * chunk_elems + ((long long)b * Lc * H_kv + g) * D;
+            const long long key0 = (long long)j * Lc;  // global position of the chunk's first key
+            auto visible = [&](long long c) { return !causal || key0 + c <= t; };
+            double lse_part;
+            attend_one(qv, kc, vc, (long long)H_kv * D, 0, Lc, D, scale, visible, s,
+                       o_part.data(), &lse_part);
+            merge_into(o, l, o_part.data(), lse_part, D);
+        }
+    });
+    return 0;
+}
+
+// Elementwise merge, in place into a ([SP-QA] section 5, merge step).
+//   o_a, o_b [B][L][H][D]   lse_a, lse_b [B][H][L]
+int ora_lse_merge(double* o_a, double* lse_a, const double* o_b, const double* lse_b, int B,
+                  int H, long long L, int D) {
+    if (B < 1 || H < 1 || L < 1 || D < 1) return 1;
+    for (int b = 0; b < B; ++b)
+        for (long long t = 0; t < L; ++t)
+            for (int h = 0; h < H; ++h) {
+                const long long oi = (((long long)b * L + t) * H + h) * D;
+                const long long li = ((long long)b * H + h) * L + t;
+                merge_into(o_a + oi, lse_a + li, o_b + oi, lse_b[li], D);
+            }
+    return 0;
+}
+
+// Ulysses sequence-sharded -> head-sharded ([ULYSSES]), one element at a time.
+//   in  [P][B][Lc][H_in][D]  ->  out [P][B][P*Lc][H_out/P][D], elements of esize bytes
+//   out[r][b][s*Lc+t][hh][:] = in[s][b][t][((r*Hl + hh) * H_in) / H_out][:],  Hl = H_out/P
+int ora_seq2head(const void* in, void* out, int P, int B, long long Lc, int H_in, int H_out,
+                 int D, int esize) {
+    if (P < 1 || B < 1 || Lc < 1 || H_in < 1 || H_out < 1 || D < 1 || esize < 1) return 1;
+    if (H_out % P != 0 || H_out % H_in != 0) return 1;
+    const int Hl = H_out / P;
+    const unsigned char* src = (const unsigned char*)in;
+    unsigned char* dst = (unsigned char*)out;
+    for (int r = 0; r < P; ++r)
+        for (int b = 0; b < B; ++b)
+            for (int s = 0; s < P; ++s)
+                for (long long t = 0; t < Lc; ++t)
+                    for (int hh = 0; hh < Hl; ++hh) {
+                        const int j = r * Hl + hh;                       // replicated head index
+                        const int hs = (int)(((long long)j * H_in) / H_out);  // its source head
+                        for (int d = 0; d < D; ++d) {
+                            const long long di =
+                                ((((long long)r * B + b) * (P * Lc) + (s * Lc + t)) * Hl + hh) * D + d;
+                            const long long si =
+                                ((((long long)s * B + b) * Lc + t) * H_in + hs) * D + d;
+                            std::memcpy(dst + di * esize, src + si * esize, (size_t)esize);
+                        }
+                    }
+    return 0;
+}
+
+// Ulysses head-sharded -> sequence-sharded ([ULYSSES]), the inverse transform.
+//   in  [P][B][P*Lc][H/P][D]  ->  out [P][B][Lc][H][D]
+//   out[s][b][t][r*Hl + hh][:] = in[r][b][s*Lc+t][hh][:],  Hl = H/P
+int ora_head2seq(const void* in, void* out, int P, int B, long long Lc, int H, int D, int esize) {
+    if (P < 1 || B < 1 || Lc < 1 || H < 1 || D < 1 || esize < 1 || H % P != 0) return 1;
+    const int Hl = H / P;
+    const unsigned char* src = (const unsigned char*)in;
+    unsigned char* dst = (unsigned char*)out;
+    for (int s = 0; s < P; ++s)
+        for (int b = 0; b < B; ++b)
+            for (long long t = 0; t < Lc; ++t)
+                for (int r = 0; r < P; ++r)
+                    for (int hh = 0; hh < Hl; ++hh)
+                        for (int d = 0; d < D; ++d) {
+                            const long long di =
+                                ((((long long)s * B + b) * Lc + t) * H + (r * Hl + hh)) * D + d;
+                            const long long si =
+                                ((((long long)r * B + b) * (P * Lc) + (s * Lc + t)) * Hl + hh) * D + d;
+                            std::memcpy(dst + di * esize, src + si * esize, (size_t)esize);
+                        }
+    return 0;
+}
+
+}  // extern "C"

@@ -1,0 +1,333 @@
+"""Pins of the fp64 oracle against facts the pages and the mathematics fix.
+
+Nothing here compares the oracle with itself by retyping its formulas: the pins
+are a hand-derived worked example (tests/golden), closed forms, the float64
+library routine torch.nn.functional.scaled_dot_product_attention, brute force
+in 50-digit decimal arithmetic on tiny inputs, and invariants that a dropped
+term, a wrong sign or index, or a transposed operand would break.
+
+Sources: "Как работает sequence parallelism в контексте LLM?" sections 2, 3, 5
+(chunking, ring order, the per-chunk softmax merged across steps) and "Метод
+контекстного параллелизма Ulysses" (the seq<->head transform and the GQA copy).
+"""
+import math
+import os
+from decimal import Decimal, getcontext
+
+import numpy as np
+import pytest
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def rnd(shape, seed, scale=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * scale
+
+
+def torch_sdpa(q, k, v, scale, causal):
+    """float64 library attention; q [B,L,H_q,D], k/v [B,L,H_kv,D] -> out, lse."""
+    tq = torch.from_numpy(q).permute(0, 2, 1, 3)
+    tk = torch.from_numpy(k).permute(0, 2, 1, 3)
+    tv = torch.from_numpy(v).permute(0, 2, 1, 3)
+    out = torch.nn.functional.scaled_dot_product_attention(
+        tq, tk, tv, scale=scale, is_causal=causal, enable_gqa=True)
+    rep = q.shape[2] // k.shape[2]
+    s = torch.matmul(tq, tk.repeat_interleave(rep, dim=1).transpose(-1, -2)) * scale
+    if causal:
+        L = q.shape[1]
+        s = s.masked_fill(torch.ones(L, L, dtype=torch.bool).triu(1), float("-inf"))
+    lse = torch.logsumexp(s, dim=-1)
+    return out.permute(0, 2, 1, 3).numpy(), lse.numpy()
+
+
+# ---------------------------------------------------------------- worked example
+def test_golden_three_keys(oracle_mod):
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "attention_three_keys.txt"))
+            if l.strip() and not l.startswith("#")]
+    q = np.tile(np.array([math.log(3.0), math.log(2.0)]), (1, 3, 1, 1))
+    k = np.array([[0, 0], [1, 0], [0, 1]], np.float64).reshape(1, 3, 1, 2)
+    v = np.array([[6, 0], [0, 6], [3, 3]], np.float64).reshape(1, 3, 1, 2)
+    for causal in (0, 1):
+        out, lse = oracle_mod.attention(q, k, v, 1.0, bool(causal))
+        for r in rows:
+            if int(r[0]) != causal:
+                continue
+            t = int(r[1])
+            np.testing.assert_allclose(out[0, t, 0], [float(r[2]), float(r[3])], atol=1e-13)
+            np.testing.assert_allclose(lse[0, 0, t], math.log(float(r[4])), atol=1e-13)
+
+
+# ---------------------------------------------------------------- library routine
+@pytest.mark.parametrize("B,L,H_q,H_kv,D,causal", [
+    (1, 37, 2, 2, 8, False), (2, 64, 4, 2, 16, True), (1, 50, 6, 3, 32, True),
+    (1, 129, 8, 1, 4, False), (1, 33, 4, 4, 64, True)])
+def test_plain_matches_torch_sdpa_fp64(oracle_mod, B, L, H_q, H_kv, D, causal):
+    q = rnd((B, L, H_q, D), 1, 2.0)
+    k = rnd((B, L, H_kv, D), 2)
+    v = rnd((B, L, H_kv, D), 3)
+    scale = 1.0 / math.sqrt(D)
+    out, lse = oracle_mod.attention(q, k, v, scale, causal)
+    ref_o, ref_l = torch_sdpa(q, k, v, scale, causal)
+    np.testing.assert_allclose(out, ref_o, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, ref_l, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- closed forms
+@pytest.mark.parametrize("causal", [False, True])
+def test_constant_scores_give_mean_of_v(oracle_mod, causal):
+    B, L, H_q, H_kv, D = 2, 40, 4, 2, 8
+    q = np.zeros((B, L, H_q, D))
+    k = rnd((B, L, H_kv, D), 5)
+    v = rnd((B, L, H_kv, D), 6)
+    out, lse = oracle_mod.attention(q, k, v, 0.3, causal)
+    for h in range(H_q):
+        g = h // (H_q // H_kv)
+        for t in range(L):
+            n = t + 1 if causal else L
+            np.testing.assert_allclose(out[:, t, h], v[:, :n, g].mean(axis=1), atol=1e-13)
+            np.testing.assert_allclose(lse[:, h, t], math.log(n), atol=1e-13)
+
+
+def test_one_dominant_key(oracle_mod):
+    B, L, H, D = 1, 24, 2, 4
+    q = rnd((B, L, H, D), 7)
+    k = rnd((B, L, H, D), 8) * 0.1
+    v = rnd((B, L, H, D), 9)
+    j = 11
+    k[0, j] = 200.0 * q[0, 5]  # row 5's score with key j dominates by a huge margin
+    out, lse = oracle_mod.attention(q, k, v, 1.0, False)
+    np.testing.assert_allclose(out[0, 5], v[0, j], atol=1e-12)
+    s = 200.0 * np.sum(q[0, 5] ** 2, axis=-1)  # per head
+    np.testing.assert_allclose(lse[0, :, 5], s, rtol=1e-12)
+
+
+def test_first_causal_row_is_v0(oracle_mod):
+    q, k, v = rnd((2, 16, 4, 8), 10), rnd((2, 16, 2, 8), 11), rnd((2, 16, 2, 8), 12)
+    out, lse = oracle_mod.attention(q, k, v, 0.5, True)
+    for h in range(4):
+        np.testing.assert_allclose(out[:, 0, h], v[:, 0, h // 2], atol=1e-14)
+        np.testing.assert_allclose(lse[:, h, 0],
+                                   0.5 * np.sum(q[:, 0, h] * k[:, 0, h // 2], -1), atol=1e-14)
+
+
+def test_causal_row_equals_prefix_attention(oracle_mod):
+    q, k, v = rnd((1, 30, 2, 8), 13), rnd((1, 30, 2, 8), 14), rnd((1, 30, 2, 8), 15)
+    out, lse = oracle_mod.attention(q, k, v, 0.4, True)
+    for t in (0, 7, 29):
+        o2, l2 = oracle_mod.attention(q[:, :t + 1], k[:, :t + 1], v[:, :t + 1], 0.4, False)
+        np.testing.assert_allclose(out[:, t], o2[:, t], atol=1e-13)
+        np.testing.assert_allclose(lse[:, :, t], l2[:, :, t], atol=1e-13)
+
+
+# ---------------------------------------------------------------- brute force
+def _decimal_attention(q, k, v, scale, causal):
+    getcontext().prec = 50
+    B, L, H_q, D = q.shape
+    H_kv = k.shape[2]
+    out = np.zeros(q.shape)
+    lse = np.zeros((B, H_q, L))
+    for b in range(B):
+        for h in range(H_q):
+            g = h // (H_q // H_kv)
+            for t in range(L):
+                keys = range(t + 1) if causal else range(L)
+                s = [Decimal(scale) * sum(Decimal(q[b, t, h, d]) * Decimal(k[b, j, g, d])
+                                          for d in range(D)) for j in keys]
+                e = [x.exp() for x in s]
+                z = sum(e)
+                lse[b, h, t] = float(z.ln())
+                for d in range(D):
+                    out[b, t, h, d] = float(sum(ei * Decimal(v[b, j, g, d])
+                                                for ei, j in zip(e, keys)) / z)
+    return out, lse
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_brute_force_decimal(oracle_mod, causal):
+    q, k, v = rnd((1, 9, 4, 3), 16, 3.0), rnd((1, 9, 2, 3), 17), rnd((1, 9, 2, 3), 18)
+    out, lse = oracle_mod.attention(q, k, v, 0.7, causal)
+    ref_o, ref_l = _decimal_attention(q, k, v, 0.7, causal)
+    np.testing.assert_allclose(out, ref_o, atol=1e-13)
+    np.testing.assert_allclose(lse, ref_l, atol=1e-13)
+
+
+# ---------------------------------------------------------------- invariants
+def test_noncausal_invariant_to_joint_kv_permutation(oracle_mod):
+    q, k, v = rnd((1, 45, 4, 8), 19), rnd((1, 45, 2, 8), 20), rnd((1, 45, 2, 8), 21)
+    perm = np.random.default_rng(22).permutation(45)
+    o1, l1 = oracle_mod.attention(q, k, v, 0.3, False)
+    o2, l2 = oracle_mod.attention(q, k[:, perm], v[:, perm], 0.3, False)
+    np.testing.assert_allclose(o1, o2, atol=1e-13)
+    np.testing.assert_allclose(l1, l2, atol=1e-13)
+
+
+def _chunks(x, P):
+    B, L, H, D = x.shape
+    return np.ascontiguousarray(x.reshape(B, P, L // P, H, D).transpose(1, 0, 2, 3, 4))
+
+
+@pytest.mark.parametrize("P", [1, 2, 4, 8, 16])
+@pytest.mark.parametrize("causal", [False, True])
+def test_ring_merge_equals_plain_attention(oracle_mod, P, causal):
+    """Merging per-chunk partials in ring order gives exactly the unchunked result."""
+    L = 16 * 6
+    q, k, v = rnd((2, L, 4, 8), 23, 2.0), rnd((2, L, 2, 8), 24), rnd((2, L, 2, 8), 25)
+    o_ref, l_ref = oracle_mod.attention(q, k, v, 0.35, causal)
+    o, l = oracle_mod.ring_attention(q, _chunks(k, P), _chunks(v, P), 0.35, causal)
+    np.testing.assert_allclose(o, o_ref, atol=1e-12)
+    np.testing.assert_allclose(l, l_ref, atol=1e-12)
+
+
+@pytest.mark.parametrize("order", ["reversed", "shuffled"])
+@pytest.mark.parametrize("causal", [False, True])
+def test_ring_order_does_not_matter(oracle_mod, order, causal):
+    P, L = 8, 64
+    q, k, v = rnd((1, L, 2, 8), 26), rnd((1, L, 2, 8), 27), rnd((1, L, 2, 8), 28)
+    offs = list(range(P))[::-1] if order == "reversed" else \
+        list(np.random.default_rng(29).permutation(P))
+    o_ref, l_ref = oracle_mod.attention(q, k, v, 0.5, causal)
+    o, l = oracle_mod.ring_attention(q, _chunks(k, P), _chunks(v, P), 0.5, causal, offs)
+    np.testing.assert_allclose(o, o_ref, atol=1e-12)
+    np.testing.assert_allclose(l, l_ref, atol=1e-12)
+
+
+def test_ring_single_rank_is_plain(oracle_mod):
+    q, k, v = rnd((1, 20, 2, 4), 30), rnd((1, 20, 1, 4), 31), rnd((1, 20, 1, 4), 32)
+    o, l = oracle_mod.ring_attention(q, k[None], v[None], 0.5, True)
+    ref_o, ref_l = torch_sdpa(q, k, v, 0.5, True)
+    np.testing.assert_allclose(o, ref_o, atol=1e-12)
+    np.testing.assert_allclose(l, ref_l, atol=1e-12)
+
+
+def test_attention_rows_sample(oracle_mod):
+    q, k, v = rnd((2, 40, 4, 8), 33), rnd((2, 40, 2, 8), 34), rnd((2, 40, 2, 8), 35)
+    rb, rt, rh = [0, 1, 1, 0], [0, 39, 17, 5], [3, 0, 2, 1]
+    o, l = oracle_mod.attention_rows(q[rb, rt, rh], rb, rt, rh, k, v, 4, 0.3, True)
+    ref_o, ref_l = torch_sdpa(q, k, v, 0.3, True)
+    np.testing.assert_allclose(o, ref_o[rb, rt, rh], atol=1e-12)
+    np.testing.assert_allclose(l, ref_l[rb, rh, rt], atol=1e-12)
+
+
+def test_invalid_arguments_rejected(oracle_mod):
+    with pytest.raises(ValueError):
+        oracle_mod.seq2head(np.zeros((2, 1, 4, 3, 8)), 3)  # 3 heads over 2 ranks
+    with pytest.raises(ValueError):
+        oracle_mod.attention_rows(np.zeros((1, 4)), [0], [99], [0], np.zeros((1, 8, 1, 4)),
+                                  np.zeros((1, 8, 1, 4)), 1, 1.0, False)
+
+
+# ---------------------------------------------------------------- merge
+def test_merge_of_key_halves_equals_whole(oracle_mod):
+    """Attention over keys [0,m) merged with attention over [m,L) is attention over [0,L)."""
+    q, k, v = rnd((2, 33, 4, 8), 36, 2.0), rnd((2, 33, 4, 8), 37), rnd((2, 33, 4, 8), 38)
+    m = 13
+    o_full, l_full = oracle_mod.attention(q, k, v, 0.4, False)
+    oa, la = _attend_subset(oracle_mod, q, k, v, 0.4, 0, m)
+    ob, lb = _attend_subset(oracle_mod, q, k, v, 0.4, m, 33)
+    o, l = oracle_mod.lse_merge(oa, la, ob, lb)
+    np.testing.assert_allclose(o, o_full, atol=1e-12)
+    np.testing.assert_allclose(l, l_full, atol=1e-12)
+
+
+def _attend_subset(oracle_mod, q, k, v, scale, lo, hi):
+    """Attention of every query row against keys [lo, hi) only, via attention_rows."""
+    B, L, H, D = q.shape
+    rb, rt, rh = np.meshgrid(np.arange(B), np.arange(L), np.arange(H), indexing="ij")
+    rb, rt, rh = rb.ravel(), rt.ravel(), rh.ravel()
+    o, l = oracle_mod.attention_rows(q[rb, rt, rh], rb, np.zeros_like(rt), rh,
+                                     k[:, lo:hi], v[:, lo:hi], H, scale, False)
+    return o.reshape(B, L, H, D), l.reshape(B, L, H).transpose(0, 2, 1).copy()
+
+
+def test_merge_identities(oracle_mod):
+    B, L, H, D = 1, 6, 2, 4
+    oa, ob = rnd((B, L, H, D), 39), rnd((B, L, H, D), 40)
+    la, lb = rnd((B, H, L), 41), rnd((B, H, L), 42)
+    ninf = np.full((B, H, L), -np.inf)
+    # (x) (+) empty = x, empty (+) (x) = x
+    o, l = oracle_mod.lse_merge(oa, la, np.zeros_like(ob), ninf)
+    np.testing.assert_array_equal(o, oa)
+    np.testing.assert_array_equal(l, la)
+    o, l = oracle_mod.lse_merge(np.zeros_like(oa), ninf, ob, lb)
+    np.testing.assert_array_equal(o, ob)
+    np.testing.assert_array_equal(l, lb)
+    # empty (+) empty = (0, -inf), no NaN
+    o, l = oracle_mod.lse_merge(oa, ninf, ob, ninf)
+    assert np.all(o == 0) and np.all(l == -np.inf)
+    # equal lse: the average, lse + ln 2
+    o, l = oracle_mod.lse_merge(oa, la, ob, la)
+    np.testing.assert_allclose(o, 0.5 * (oa + ob), atol=1e-15)
+    np.testing.assert_allclose(l, la + math.log(2), atol=1e-15)
+    # weights e^(la-l), e^(lb-l) with l = log(e^la + e^lb): closed form for lb = la + ln 3
+    o, l = oracle_mod.lse_merge(oa, la, ob, la + math.log(3))
+    np.testing.assert_allclose(o, 0.25 * oa + 0.75 * ob, atol=1e-14)
+    np.testing.assert_allclose(l, la + math.log(4), atol=1e-14)
+    # commutative
+    o1, l1 = oracle_mod.lse_merge(oa, la, ob, lb)
+    o2, l2 = oracle_mod.lse_merge(ob, lb, oa, la)
+    np.testing.assert_allclose(o1, o2, atol=1e-15)
+    np.testing.assert_allclose(l1, l2, atol=1e-15)
+
+
+def test_merge_large_lse_no_overflow(oracle_mod):
+    oa, ob = np.ones((1, 1, 1, 4)), 3 * np.ones((1, 1, 1, 4))
+    o, l = oracle_mod.lse_merge(oa, np.array([[[1000.0]]]), ob, np.array([[[1000.0]]]))
+    np.testing.assert_allclose(o, 2 * np.ones((1, 1, 1, 4)))
+    np.testing.assert_allclose(l, 1000 + math.log(2))
+
+
+# ---------------------------------------------------------------- Ulysses permute
+def _golden_ulysses():
+    cases = {}
+    for line in open(os.path.join(GOLDEN, "ulysses_tiny.txt")):
+        if not line.strip() or line.startswith("#"):
+            continue
+        head, vals = line.split(":")
+        case, h_in, h_out, r = head.split()
+        cases.setdefault((case, int(h_in), int(h_out)), {})[int(r)] = [int(x) for x in vals.split()]
+    return cases
+
+
+def test_seq2head_golden(oracle_mod):
+    P, Lc = 2, 2
+    for (case, H_in, H_out), per_rank in _golden_ulysses().items():
+        x = np.zeros((P, 1, Lc, H_in, 1), np.int32)
+        for s in range(P):
+            for t in range(Lc):
+                for h in range(H_in):
+                    x[s, 0, t, h, 0] = 100 * s + 10 * t + h
+        y = oracle_mod.seq2head(x, H_out)
+        assert y.shape == (P, 1, P * Lc, H_out // P, 1)
+        for r, vals in per_rank.items():
+            assert y[r].ravel().tolist() == vals, (case, r)
+
+
+@pytest.mark.parametrize("dtype", [np.float32, np.uint16, np.float64])
+def test_seq2head_head2seq_round_trip(oracle_mod, dtype):
+    P, B, Lc, H, D = 4, 2, 6, 8, 5
+    x = (np.random.default_rng(43).integers(0, 60000, (P, B, Lc, H, D))).astype(dtype)
+    y = oracle_mod.seq2head(x, H)
+    assert y.size == x.size  # memory unchanged by the transform
+    z = oracle_mod.head2seq(y)
+    assert z.dtype == x.dtype and np.array_equal(z, x)
+
+
+def test_seq2head_is_a_permutation_of_elements(oracle_mod):
+    P, B, Lc, H, D = 4, 1, 3, 4, 2
+    x = np.arange(P * B * Lc * H * D, dtype=np.int64).reshape(P, B, Lc, H, D)
+    y = oracle_mod.seq2head(x, H)
+    assert sorted(y.ravel().tolist()) == list(range(x.size))
+
+
+def test_seq2head_gqa_replicas_copy_their_source(oracle_mod):
+    P, B, Lc, H_in, H_out, D = 8, 1, 5, 4, 8, 3
+    x = np.random.default_rng(44).standard_normal((P, B, Lc, H_in, D))
+    y = oracle_mod.seq2head(x, H_out)  # [P, B, P*Lc, 1, D]
+    glob = x.transpose(1, 0, 2, 3, 4).reshape(B, P * Lc, H_in, D)
+    for r in range(P):
+        np.testing.assert_array_equal(y[r, :, :, 0], glob[:, :, (r * H_in) // H_out])
+    # each replicated rank pair then sees the kv head its query-head block needs:
+    # with 32 query heads on 8 ranks, rank r's heads 4r..4r+3 use kv head (4r)//(32//4)
+    for r in range(P):
+        assert (r * H_in) // H_out == (4 * r) // (32 // H_in)

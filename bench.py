@@ -1,0 +1,470 @@
+"""Benchmark of the ring-chunked attention / Ulysses hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+  seq2head(Q), seq2head(K), seq2head(V) (GQA copy of 4 KV heads to 8 ranks)
+  -> causal ring-chunked attention over L = 131072 (8 virtual ranks x 16384 tokens,
+     per-rank head group of 4 query heads, tcgen05 tensor cores)
+  -> head2seq(O)
+i.e. the Ulysses layer of "Метод контекстного параллелизма Ulysses" with the ring
+attention of "Как работает sequence parallelism в контексте LLM?" as its local kernel.
+
+value = attention FLOPs (4*B*H*L^2*D / 2, causal) of all ranks' steps / device time of
+the steps (max over ranks), in TFLOP/s.  With --gpus N every rank runs its own replica
+(weak scaling: the path has no data-path exchange between independent replicas).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload ulysses_e2e|long_128k|llama8b_32k|small_4k]
+"""
+from __future__ import annotations
+
+import argparse
+import faulthandler
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "ring-chunked attention TFLOP/s & % BF16 tensor peak (1 B200); permute GB/s"
+UNIT = "TFLOP/s"
+DATASHEET_BF16_TFLOPS = 2250.0
+DATASHEET_HBM_GBS = 8000.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ workloads
+def workloads():
+    from sequence_parallelism_attn_b200 import synth
+    return {
+        "ulysses_e2e": ("ulysses", synth.ULYSSES_128K),
+        "long_128k": ("attn", synth.LONG_128K),
+        "llama8b_32k": ("attn", synth.LLAMA8B_GQA),
+        "small_4k": ("attn", synth.SMALL_BF16),
+    }
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons every 100 ms through NVML."""
+
+    BAD = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown"}
+    NAMES = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+             0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+             0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self._stop = threading.Event()
+        self._thread = None
+        self.max_mhz = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            prop = torch.cuda.get_device_properties(device_index)
+            # torch gives the PCI location as three integers; NVML wants the string form
+            bus = "%08X:%02X:%02X.0" % (int(prop.pci_domain_id), int(prop.pci_bus_id),
+                                        int(prop.pci_device_id))
+            assert isinstance(bus, str)
+            self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: fall back to nvidia-smi
+            self._nv = None
+            self.error = str(e)
+            self._bus = locals().get("bus")
+
+    def _run_smi(self):
+        import subprocess
+        q = "clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active"
+        cmd = ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self._bus:
+            cmd += ["-i", self._bus]
+        try:
+            proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, text=True)
+        except Exception:
+            return
+        for line in proc.stdout:
+            if self._stop.is_set():
+                break
+            try:
+                sm, mx, pw, rs = [x.strip() for x in line.split(",")]
+                self.max_mhz = float(mx)
+                self.samples.append((float(sm), int(rs, 16), float(pw)))
+            except Exception:
+                pass
+        proc.terminate()
+
+    def _run(self):
+        nv = self._nv
+        if nv is None:
+            return self._run_smi()
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                try:
+                    reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                except Exception:
+                    reasons = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                power = nv.nvmlDeviceGetPowerUsage(self._h) / 1000.0
+                self.samples.append((sm, reasons, power))
+            except Exception:
+                pass
+            self._stop.wait(0.1)
+
+    def __enter__(self):
+        if True:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        sm = [s[0] for s in self.samples]
+        bits = 0
+        for s in self.samples:
+            bits |= s[1]
+        reasons = [n for b, n in self.NAMES.items() if bits & b and b != 0x1]
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "power_w_max": max(s[2] for s in self.samples),
+                "samples": len(sm)}
+
+    def rejected(self) -> bool:
+        if not self.samples:
+            return False
+        bits = 0
+        for s in self.samples:
+            bits |= s[1]
+        if any(bits & b for b in self.BAD):
+            return True
+        med = statistics.median(s[0] for s in self.samples)
+        no_reason = not (bits & ~0x1)
+        return bool(self.max_mhz and no_reason and med < 0.6 * self.max_mhz)
+
+
+# ------------------------------------------------------------------ our path
+class Path:
+    """Device buffers and the per-step launches of one workload."""
+
+    def __init__(self, kind, w, device):
+        import torch
+        from sequence_parallelism_attn_b200 import ra, synth
+        self.ra, self.kind, self.w, self.dev = ra, kind, w, device
+        if kind == "ulysses":
+            a = w.attn()
+            self.a = a
+            self.q, self.k, self.v = synth.ulysses_inputs(w, device=device)
+            self.qh = torch.empty((w.P, w.B, a.L, a.H_q, a.D), dtype=w.dtype, device=device)
+            self.kh = torch.empty((w.P, w.B, a.L, a.H_kv, a.D), dtype=w.dtype, device=device)
+            self.vh = torch.empty_like(self.kh)
+            self.o = torch.empty((a.B, a.L, a.H_q, a.D), dtype=torch.bfloat16, device=device)
+            self.lse = torch.empty((a.B, a.H_q, a.L), dtype=torch.float32, device=device)
+            self.o_seq = torch.empty_like(self.q)
+            kvv = lambda x: [x.view(a.B, a.P, a.Lc, a.H_kv, a.D)[:, j] for j in range(a.P)]
+            self.k_chunks, self.v_chunks = kvv(self.kh), kvv(self.vh)
+            self.qa = self.qh.view(a.B, a.L, a.H_q, a.D)
+            self.launches_per_step = 5
+            self.flops = a.flops()
+            self.permute_bytes = w.permute_bytes()
+            self.in_bytes = sum(t.numel() * t.element_size() for t in (self.q, self.k, self.v))
+            self.out_bytes = self.o_seq.numel() * self.o_seq.element_size()
+        else:
+            self.a = w
+            q, k, v = synth.attention_inputs(w, device=device)
+            self.q, self.k, self.v = q, k, v
+            self.o = torch.empty((w.B, w.L, w.H_q, w.D), dtype=torch.bfloat16, device=device)
+            self.lse = torch.empty((w.B, w.H_q, w.L), dtype=torch.float32, device=device)
+            self.launches_per_step = 1
+            self.flops = w.flops()
+            self.permute_bytes = 0
+            self.in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
+            self.out_bytes = self.o.numel() * self.o.element_size()
+
+    def step(self, ev=None):
+        """One pass of the path.  ev: optional dict of CUDA event pairs per stage."""
+        ra = self.ra
+        rec = (lambda name, i: ev[name][i].record()) if ev is not None else (lambda *_: None)
+        if self.kind == "ulysses":
+            w, a = self.w, self.a
+            rec("permute_in", 0)
+            ra.ra_ulysses_seq2head(self.q, w.H_q, out=self.qh)
+            ra.ra_ulysses_seq2head(self.k, w.H_kv_rep, out=self.kh)
+            ra.ra_ulysses_seq2head(self.v, w.H_kv_rep, out=self.vh)
+            rec("permute_in", 1)
+            rec("attn", 0)
+            ra.ring_attn_fwd(self.qa, self.k_chunks, self.v_chunks, True, a.scale,
+                             out=self.o, lse=self.lse)
+            rec("attn", 1)
+            rec("permute_out", 0)
+            ra.ra_ulysses_head2seq(self.o.view(w.P, w.B, a.L, a.H_q, a.D), out=self.o_seq)
+            rec("permute_out", 1)
+        else:
+            w = self.w
+            rec("attn", 0)
+            ra.ring_attn_fwd(self.q, self.k, self.v, w.causal, w.scale, out=self.o, lse=self.lse)
+            rec("attn", 1)
+
+    def result(self):
+        return self.o_seq if self.kind == "ulysses" else self.o
+
+
+def time_region(path, steps, torch, dist, ev_stages):
+    """Time exactly `steps` steps between barrier+synchronize; returns (ms_total, stage_ms)."""
+    events = {k: [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+              for k in ev_stages}
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record()
+    for i in range(steps):
+        path.step({k: events[k][i] for k in ev_stages})
+    end.record()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    total = start.elapsed_time(end)
+    stage = {k: [events[k][i][0].elapsed_time(events[k][i][1]) for i in range(steps)]
+             for k in ev_stages}
+    return total, stage
+
+
+def max_over_ranks(x, dist, torch, device):
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def e2e_region(path, steps, torch, dist, device):
+    """The same step through the public API with inputs copied from pinned host memory each
+    step and the result read back to pinned host memory; returns ms per step (max ranks)."""
+    host_in = [t.cpu().pin_memory() for t in (path.q, path.k, path.v)]
+    res = path.result()
+    host_out = torch.empty(res.shape, dtype=res.dtype, pin_memory=True)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record()
+    for _ in range(steps):
+        for h, d in zip(host_in, (path.q, path.k, path.v)):
+            d.copy_(h, non_blocking=True)
+        path.step()
+        host_out.copy_(res, non_blocking=True)
+    end.record()
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end) / steps
+    return max_over_ranks(ms, dist, torch, device)
+
+
+def attn_traffic(path_kind):
+    """DRAM bytes per attention launch from the committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    import hashlib
+    src = os.path.join(ROOT, "sequence_parallelism_attn_b200", "csrc", "attn_sm100.cu")
+    prof = os.path.join(ROOT, "profiles", "attn_sm100_traffic.json")
+    if not os.path.exists(prof):
+        return None
+    with open(prof) as f:
+        d = json.load(f)
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if d.get("kernel_sha") != sha:
+        return None
+    return d.get("bytes_per_launch", {}).get(path_kind)
+
+
+# ------------------------------------------------------------------ CPU baseline (oracle)
+def oracle_sample(w_attn, n_rows, seed=4242):
+    """A bounded sample of the attention workload for the oracle: n query rows of one
+    (batch, kv-head) sequence of the same length and distribution, against all their keys."""
+    import numpy as np
+    import torch
+    g = torch.Generator().manual_seed(seed)
+    L, D = w_attn.L, w_attn.D
+    k = torch.randn(1, L, 1, D, generator=g).to(w_attn.dtype).double().numpy()
+    v = torch.randn(1, L, 1, D, generator=g).to(w_attn.dtype).double().numpy()
+    rt = torch.randint(0, L, (n_rows,), generator=g).numpy().astype(np.int64)
+    q = (torch.randn(n_rows, D, generator=g) * w_attn.q_mult).to(w_attn.dtype).double().numpy()
+    vis = (rt + 1) if w_attn.causal else np.full(n_rows, L)
+    flops = float(np.sum(4.0 * vis * D))
+    return q, np.zeros(n_rows, np.int32), rt, np.zeros(n_rows, np.int32), k, v, flops
+
+
+def run_oracle_sample(w_attn, target_s=15.0, max_rows=4096):
+    """Time the oracle as it stands on a bounded sample; returns (TFLOP/s, rows, seconds)."""
+    import oracle
+    oracle.build()
+    cores = os.cpu_count() or 1
+    n = 8 * cores
+    while True:
+        q, rb, rt, rh, k, v, flops = oracle_sample(w_attn, n)
+        t0 = time.perf_counter()
+        oracle.attention_rows(q, rb, rt, rh, k, v, 1, w_attn.scale, w_attn.causal)
+        dt = time.perf_counter() - t0
+        if dt >= target_s * 0.5 or n >= max_rows:
+            return flops / dt / 1e12, n, dt, cores
+        n = min(max_rows, max(n * 2, int(n * target_s / max(dt, 1e-3))))
+
+
+# ------------------------------------------------------------------ main
+def main():
+    faulthandler.enable()
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="ulysses_e2e")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    kind, w = workloads()[args.workload]
+    w_attn = w.attn() if kind == "ulysses" else w
+
+    if args.impl == "reference":
+        return reference_arm(args, kind, w, w_attn, rank, world)
+
+    import torch
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    peaks, peaks_src = load_peaks()
+
+    path = Path(kind, w, device)
+    for _ in range(args.warmup):
+        path.step()
+    torch.cuda.synchronize()
+    stages = ["attn"] + (["permute_in", "permute_out"] if kind == "ulysses" else [])
+    for attempt in range(2):
+        with ClockSampler(local_rank) as clk:
+            total_ms, stage_ms = time_region(path, args.steps, torch, dist, stages)
+        if not clk.rejected():
+            break
+    st = path.ra.ra_sync_status()
+    if st != 0:
+        raise RuntimeError(f"kernel status {st}: {path.ra.ra_last_error()}")
+    ms_step = max_over_ranks(total_ms / args.steps, dist, torch, device)
+    attn_ms = max_over_ranks(statistics.mean(stage_ms["attn"]), dist, torch, device)
+    value = path.flops * world / (ms_step * 1e-3) / 1e12
+    attn_tflops = path.flops / (attn_ms * 1e-3) / 1e12
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "global_batch": w_attn.B * world, "seq_len": w_attn.L,
+                   "heads_q": w_attn.H_q, "heads_kv": w_attn.H_kv, "head_dim": w_attn.D,
+                   "virtual_ranks": w_attn.P, "chunk_len": w_attn.Lc, "causal": w_attn.causal,
+                   "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (126 MB); no flush between steps"},
+    }
+    sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    traffic = attn_traffic(args.workload)
+    out["roofline"] = {"bound": "tensor", "achieved": round(attn_tflops, 2),
+                       "peak": sustained, "unit": "TFLOP/s",
+                       "frac": round(attn_tflops / sustained, 4),
+                       "traffic": traffic,
+                       "kernel": "attn_fwd_sm100<128>",
+                       "peak_source": f"{peaks_src} bf16_tflops_sustained",
+                       "frac_of_burst": round(attn_tflops / peaks.get("bf16_tflops", 1590.0), 4),
+                       "frac_of_datasheet": round(attn_tflops / DATASHEET_BF16_TFLOPS, 4)}
+    if kind == "ulysses":
+        perm_ms = max_over_ranks(statistics.mean(
+            a + b for a, b in zip(stage_ms["permute_in"], stage_ms["permute_out"])),
+            dist, torch, device)
+        perm_gbs = path.permute_bytes / (perm_ms * 1e-3) / 1e9
+        out["permute"] = {"gbs": round(perm_gbs, 1), "bytes_per_step": path.permute_bytes,
+                          "ms_per_step": round(perm_ms, 4),
+                          "frac_of_measured_hbm": round(perm_gbs / peaks.get("hbm_gbs", 6650.0), 4),
+                          "frac_of_datasheet_hbm": round(perm_gbs / DATASHEET_HBM_GBS, 4)}
+    out["gpu_launches"] = path.launches_per_step * args.steps
+    out["clocks"] = clk.summary()
+    if not args.no_e2e:
+        e2e_ms = e2e_region(path, max(2, min(args.steps, 5)), torch, dist, device)
+        out["e2e"] = {"value": round(path.flops * world / (e2e_ms * 1e-3) / 1e12, 2),
+                      "unit": UNIT, "h2d_bytes_per_step": path.in_bytes,
+                      "d2h_bytes_per_step": path.out_bytes, "ms_per_step": round(e2e_ms, 3)}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, n, dt, cores = run_oracle_sample(w_attn)
+        out["cpu_baseline"] = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle",
+                               "sample": f"{n} query rows x all visible keys of one "
+                                         f"{w_attn.L}-token sequence (D={w_attn.D}), fp64 "
+                                         f"oracle, {dt:.1f} s"}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def reference_arm(args, kind, w, w_attn, rank, world):
+    """The oracle timed on the host cores as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    cores = os.cpu_count() or 1
+    # size one step's sample so that warmup + steps end within a few minutes
+    per_step_s = max(2.0, min(20.0, 150.0 / (args.steps + args.warmup)))
+    tf, n, dt, _ = run_oracle_sample(w_attn, target_s=per_step_s)
+    import numpy as np
+    q, rb, rt, rh, k, v, flops = oracle_sample(w_attn, n)
+    for _ in range(args.warmup):
+        pass  # the oracle has no warm state; the calibration run above served as warm-up
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.attention_rows(q, rb, rt, rh, k, v, 1, w_attn.scale, w_attn.causal)
+        times.append(time.perf_counter() - t0)
+    sec = sum(times) / len(times)
+    value = flops / sec / 1e12
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic",
+           "config": {"workload": w.name, "seq_len": w_attn.L, "head_dim": w_attn.D,
+                      "causal": w_attn.causal, "parallelism": "cpu-oracle"},
+           "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                            "sample": f"{n} query rows x all visible keys of one {w_attn.L}-token "
+                                      f"sequence per step, fp64 oracle"},
+           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -43,6 +43,12 @@
 #ifndef RA_B200_H
 #define RA_B200_H
 
+#if defined(__GNUC__)
+#define RA_API __attribute__((visibility("default")))
+#else
+#define RA_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -103,7 +109,7 @@ typedef enum {
  *   outside the lists above.
  */
 #define RA_MAX_P 64
-ra_status ra_ring_attn_fwd(const void* q, const void* const* k_chunks, const void* const* v_chunks,
+RA_API ra_status ra_ring_attn_fwd(const void* q, const void* const* k_chunks, const void* const* v_chunks,
                            int P, int B, int H_q, int H_kv, int Lc, int D,
                            long long q_bstride, long long kv_bstride,
                            float scale, int causal, ra_dtype in_dtype, ra_dtype out_dtype,
@@ -123,7 +129,7 @@ ra_status ra_ring_attn_fwd(const void* q, const void* const* k_chunks, const voi
  * o_b/lse_b must not alias o_a/lse_a.  Errors: RA_ERR_INVALID for null or
  * misaligned pointers or sizes < 1; RA_ERR_UNSUPPORTED if D % 4 != 0.
  */
-ra_status ra_lse_merge(float* o_a, float* lse_a, const float* o_b, const float* lse_b,
+RA_API ra_status ra_lse_merge(float* o_a, float* lse_a, const float* o_b, const float* lse_b,
                        int B, int H, long long L, int D, void* stream);
 
 /*
@@ -144,7 +150,7 @@ ra_status ra_lse_merge(float* o_a, float* lse_a, const float* o_b, const float* 
  *   H_out % P != 0 (heads must divide among ranks), H_out % H_in != 0,
  *   D*sizeof(dt) % 16 != 0.
  */
-ra_status ra_ulysses_seq2head(const void* in, void* out, int P, int B, int Lc,
+RA_API ra_status ra_ulysses_seq2head(const void* in, void* out, int P, int B, int Lc,
                               int H_in, int H_out, int D, ra_dtype dt, void* stream);
 
 /*
@@ -155,7 +161,7 @@ ra_status ra_ulysses_seq2head(const void* in, void* out, int P, int B, int Lc,
  *   out[s][b][t][r*H/P + h'][:] = in[r][b][s*Lc+t][h'][:]
  * Bit-exact.  Errors as ra_ulysses_seq2head (H % P != 0 is RA_ERR_INVALID).
  */
-ra_status ra_ulysses_head2seq(const void* in, void* out, int P, int B, int Lc,
+RA_API ra_status ra_ulysses_head2seq(const void* in, void* out, int P, int B, int Lc,
                               int H, int D, ra_dtype dt, void* stream);
 
 /*
@@ -164,17 +170,17 @@ ra_status ra_ulysses_head2seq(const void* in, void* out, int P, int B, int Lc,
  * last call gave up on a bounded wait, RA_ERR_CUDA if the synchronisation
  * itself failed, RA_OK otherwise.
  */
-ra_status ra_sync_status(void* stream);
+RA_API ra_status ra_sync_status(void* stream);
 
 /* Thread-local description of the last non-OK status returned on this thread. */
-const char* ra_last_error(void);
+RA_API const char* ra_last_error(void);
 
 /*
  * ra_set_wait_limit_ns -- bound, in nanoseconds, on every internal spin-wait of
  * the tensor-core attention kernel (default 4e9).  Takes effect at the next
  * launch.  Returns the previous value.  ns == 0 restores the default.
  */
-unsigned long long ra_set_wait_limit_ns(unsigned long long ns);
+RA_API unsigned long long ra_set_wait_limit_ns(unsigned long long ns);
 
 /*
  * ra_debug_inject_stall -- test hook.  With on != 0 the next tensor-core
@@ -183,10 +189,10 @@ unsigned long long ra_set_wait_limit_ns(unsigned long long ns);
  * returns RA_ERR_TIMEOUT.  No fault and no unbounded wait is involved.  The
  * hook disarms itself after that launch.
  */
-void ra_debug_inject_stall(int on);
+RA_API void ra_debug_inject_stall(int on);
 
 /* Library version string. */
-const char* ra_version(void);
+RA_API const char* ra_version(void);
 
 #ifdef __cplusplus
 }

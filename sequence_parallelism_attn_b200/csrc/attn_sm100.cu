@@ -1,0 +1,681 @@
+// attn_sm100.cu -- ring-chunked exact attention on the Blackwell tensor cores (sm_100a).
+//
+// What it computes ("Как работает sequence parallelism в контексте LLM?"):
+//   section 2  -- the sequence of length L = P*Lc is split into P contiguous chunks, rank i
+//                 owning tokens [i*Lc, (i+1)*Lc);
+//   section 3  -- ring attention: at step s the queries of rank i attend to the K/V chunk
+//                 it holds then, chunk j = (i - s) mod P, for s = 0..P-1;
+//   section 5  -- per chunk: scores Q.K^T, row max, exp, row sum, and the merge of the new
+//                 partial into the running one by rescaling with exp(lse_old - lse_new);
+//                 finally the division by the normaliser.
+// Here the P ranks are virtual chunk partitions in one GPU's memory.  The merge across
+// chunk steps is carried in registers and tensor memory as the running (max, normaliser,
+// output) state of an online softmax: rescaling the running output by
+// exp2(m_old - m_new) whenever a tile of a new chunk raises the row maximum is exactly the
+// ring's log-sum-exp merge, applied at 128-key granularity.  Causal masking (a reading:
+// global positions in rank order, key <= query) skips chunk pairs and 128-key tiles that
+// lie wholly after the CTA's last query row -- no MMA is issued for them -- and masks
+// elements only in tiles that straddle the diagonal or a ragged chunk end.
+//
+// Kernel organisation (one CTA per 256 query rows of one (batch, head); 384 threads):
+//   warps 0-3  softmax for query tile A (rows r0 .. r0+127), one TMEM lane (= row) each
+//   warps 4-7  softmax for query tile B (rows r0+128 .. r0+255)
+//   warp 8     TMA producer: Q tiles once, then K and V tiles into NS-deep rings
+//   warp 9     MMA issuer (one thread) and TMEM owner
+//   warps 10-11 idle (they complete the third warpgroup for the register split)
+// Registers: launched at 168 per thread (3 warps per SM sub-partition); the softmax
+// warpgroups raise their budget to 216 and the third warpgroup drops to 72
+// (216 + 216 + 72 = 504 <= 512 per sub-partition; 256*216 + 128*72 = 384*168).
+// Tensor memory (512 columns x 128 lanes x 32 bit):
+//   S_A [0,128) S_B [128,256) fp32 scores; P_A/P_B (bf16 probabilities) overwrite the
+//   first 64 columns of S_A/S_B; O_A at 256, O_B at 256+D (fp32 accumulators).
+// Per KV tile j the MMA thread issues, in this order,
+//   PV_A(j) = P_A V(j);  S_A(j+1) = Q_A K(j+1)^T;  PV_B(j);  S_B(j+1)
+// so the tensor core works on one query tile while the softmax warps of the other
+// tile turn its scores into probabilities.  tcgen05.commit after S_A(j+1) signals both
+// "S_A(j+1) ready" and "PV_A(j) done", which is what the softmax needs before it may
+// rescale O_A.  The O rescale is skipped unless the row max grew by more than 2^8
+// (exact: the final normalisation uses the same stale max as the probabilities).
+//
+// Every wait is bounded (a time limit on %globaltimer): a role that gives up sets a CTA
+// abort flag and the per-device error word; every role then stops issuing, the producer
+// waits for its own copies in flight, the MMA thread waits for its own MMAs, and the CTA
+// frees its tensor memory and exits.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <cmath>
+#include <cstdint>
+#include "ra_internal.h"
+#include "sm100_ptx.cuh"
+#include "../../include/ra.h"
+
+namespace ra {
+
+__device__ unsigned int g_ra_error_word = 0;
+
+namespace {
+
+constexpr int kThreads = 384;
+constexpr uint32_t kRegsSoftmax = 216, kRegsOther = 72;
+constexpr int kWarpLoad = 8;
+constexpr int kWarpMma = 9;
+constexpr int kBM = 128;  // query rows per tile
+constexpr int kBN = 128;  // keys per tile
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+// error-word bits
+constexpr unsigned kErrProducer = 1u, kErrMma = 2u, kErrSoftmax = 4u, kErrDrain = 8u;
+
+struct __align__(64) AttnParams {
+    CUtensorMap tm_q;
+    CUtensorMap tm_k[RA_MAX_P];
+    CUtensorMap tm_v[RA_MAX_P];
+    void* out;
+    float* lse;
+    int P, B, H_q, H_kv, Lc, L;
+    int causal, out_bf16, group, n_row_blocks;
+    float scale_log2;
+    int inject_stall;
+    unsigned long long wait_limit_ns;
+};
+
+template <int D>
+struct Cfg {
+    static constexpr int TILE = kBM * D * 2;  // bytes of a 128 x D bf16 tile
+    static constexpr int NKB = D / 64;        // 64-column (128-byte) swizzle blocks per tile
+    static constexpr int BLK = kBM * 128;     // bytes of one swizzle block (16 KB)
+    static constexpr int NS = (D == 128) ? 2 : 4;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = 2 * TILE;
+    static constexpr int OFF_V = OFF_K + NS * TILE;
+    static constexpr int OFF_BAR = OFF_V + NS * TILE;
+    // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2],
+    // p_full[2], o_full[2], drain
+    static constexpr int N_BARS = 1 + 4 * NS + 2 + 2 + 2 + 1;
+    static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem base (4 B), abort flag (4 B)
+    static constexpr int SMEM = OFF_MISC + 16 + 1024;      // + slack for 1024-B alignment
+    static constexpr int BAR_Q = 0;
+    __host__ __device__ static constexpr int bar_kf(int s) { return 1 + s; }
+    __host__ __device__ static constexpr int bar_ke(int s) { return 1 + NS + s; }
+    __host__ __device__ static constexpr int bar_vf(int s) { return 1 + 2 * NS + s; }
+    __host__ __device__ static constexpr int bar_ve(int s) { return 1 + 3 * NS + s; }
+    __host__ __device__ static constexpr int bar_sf(int w) { return 1 + 4 * NS + w; }
+    __host__ __device__ static constexpr int bar_pf(int w) { return 3 + 4 * NS + w; }
+    __host__ __device__ static constexpr int bar_of(int w) { return 5 + 4 * NS + w; }
+    static constexpr int BAR_DRAIN = 7 + 4 * NS;
+    static constexpr uint32_t S_COL0 = 0, S_COL1 = 128;
+    static constexpr uint32_t O_COL0 = 256, O_COL1 = 256 + D;
+};
+
+// The chunk/tile visiting order of one CTA (all roles derive the same sequence).
+struct Sched {
+    int P, Lc, ntc, i0, causal;
+    long long last_row;  // last query row of the CTA that exists (< L)
+    __device__ int chunk_at(int s) const {
+        int j = (i0 - s) % P;
+        return j < 0 ? j + P : j;
+    }
+    // 128-key tiles of chunk j with at least one key <= last_row (all of them if not causal)
+    __device__ int tiles_in(int j) const {
+        if (!causal) return ntc;
+        const long long k0 = (long long)j * Lc;
+        if (k0 > last_row) return 0;
+        const long long t = (last_row - k0) / kBN + 1;
+        return t < ntc ? (int)t : ntc;
+    }
+    __device__ int count() const {
+        int n = 0;
+        for (int s = 0; s < P; ++s) n += tiles_in(chunk_at(s));
+        return n;
+    }
+};
+
+struct SchedIter {
+    const Sched* S;
+    int s, t, nt;
+    __device__ void begin(const Sched* sched) {
+        S = sched;
+        s = 0;
+        t = 0;
+        nt = S->tiles_in(S->chunk_at(0));
+        skip_empty();
+    }
+    __device__ void skip_empty() {
+        while (s < S->P && t >= nt) {
+            ++s;
+            t = 0;
+            if (s < S->P) nt = S->tiles_in(S->chunk_at(s));
+        }
+    }
+    __device__ void next() {
+        ++t;
+        skip_empty();
+    }
+    __device__ int chunk() const { return S->chunk_at(s); }
+};
+
+__device__ __forceinline__ void raise_abort(volatile int* abort_flag, unsigned code) {
+    *abort_flag = 1;
+    atomicOr(&g_ra_error_word, code);
+}
+
+// Single-thread bounded wait.  Gives up when the CTA aborted or after `limit` ns.
+__device__ __forceinline__ bool wait1(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                   unsigned long long limit, unsigned code) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 15u) == 0) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > limit) {
+                raise_abort(abort_flag, code);
+                return false;
+            }
+        }
+    }
+}
+
+// Bounded wait that ignores the abort flag: used to drain work this thread started.
+__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                        unsigned long long limit) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 15u) == 0 && global_timer_ns() - t0 > limit) {
+            raise_abort(abort_flag, kErrDrain);
+            return false;
+        }
+    }
+}
+
+// Warp-uniform bounded wait (every lane polls; the give-up decision is lane 0's).
+__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                       unsigned long long limit) {
+    const unsigned FULL = 0xffffffffu;
+    bool done = mbar_try_wait(bar, parity);
+    if (__all_sync(FULL, done)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (!done) done = mbar_try_wait(bar, parity);
+        if (__all_sync(FULL, done)) return true;
+        if ((it & 15u) == 0) {
+            int stop = 0;
+            if ((threadIdx.x & 31) == 0) {
+                if (*abort_flag) stop = 1;
+                else if (global_timer_ns() - t0 > limit) {
+                    raise_abort(abort_flag, kErrSoftmax);
+                    stop = 1;
+                }
+            }
+            if (__shfl_sync(FULL, stop, 0)) return false;
+        }
+    }
+}
+
+template <int D>
+__device__ __forceinline__ void producer(const AttnParams& p, uint32_t base, const Sched& sched,
+                                         int n, int b, int h, int g, int r0,
+                                         volatile int* abort_flag) {
+    using C = Cfg<D>;
+    auto bar = [&](int i) { return base + C::OFF_BAR + 8u * (uint32_t)i; };
+    const unsigned long long lim = p.wait_limit_ns;
+    int k_armed[C::NS], v_armed[C::NS];
+#pragma unroll
+    for (int s = 0; s < C::NS; ++s) k_armed[s] = v_armed[s] = -1;
+
+    mbar_arrive_expect_tx(bar(C::BAR_Q), 2 * C::TILE);
+#pragma unroll
+    for (int kb = 0; kb < C::NKB; ++kb) {
+        tma_load_4d(base + C::OFF_Q + kb * C::BLK, &p.tm_q, bar(C::BAR_Q), kb * 64, h, r0, b);
+        tma_load_4d(base + C::OFF_Q + C::TILE + kb * C::BLK, &p.tm_q, bar(C::BAR_Q), kb * 64, h,
+                    r0 + kBM, b);
+    }
+    SchedIter it;
+    it.begin(&sched);
+    for (int jt = 0; jt < n; ++jt, it.next()) {
+        const int slot = jt % C::NS;
+        const int j = it.chunk();
+        const int row0 = it.t * kBN;
+        if (jt >= C::NS && !wait1(bar(C::bar_ke(slot)), ((jt / C::NS) - 1) & 1, abort_flag, lim,
+                                  kErrProducer))
+            break;
+        // Test hook: withhold the last K tile so the consumer's bounded wait expires.
+        if (!(p.inject_stall && jt == n - 1)) {
+            mbar_arrive_expect_tx(bar(C::bar_kf(slot)), C::TILE);
+#pragma unroll
+            for (int kb = 0; kb < C::NKB; ++kb)
+                tma_load_4d(base + C::OFF_K + slot * C::TILE + kb * C::BLK, &p.tm_k[j],
+                            bar(C::bar_kf(slot)), kb * 64, g, row0, b);
+            k_armed[slot] = jt;
+        }
+        if (jt >= C::NS && !wait1(bar(C::bar_ve(slot)), ((jt / C::NS) - 1) & 1, abort_flag, lim,
+                                  kErrProducer))
+            break;
+        mbar_arrive_expect_tx(bar(C::bar_vf(slot)), C::TILE);
+#pragma unroll
+        for (int kb = 0; kb < C::NKB; ++kb)
+            tma_load_4d(base + C::OFF_V + slot * C::TILE + kb * C::BLK, &p.tm_v[j],
+                        bar(C::bar_vf(slot)), kb * 64, g, row0, b);
+        v_armed[slot] = jt;
+    }
+    // Drain: every copy this thread started must have landed before the CTA exits.
+    wait_drain(bar(C::BAR_Q), 0, abort_flag, lim);
+#pragma unroll
+    for (int s = 0; s < C::NS; ++s) {
+        if (k_armed[s] >= 0) wait_drain(bar(C::bar_kf(s)), (k_armed[s] / C::NS) & 1, abort_flag, lim);
+        if (v_armed[s] >= 0) wait_drain(bar(C::bar_vf(s)), (v_armed[s] / C::NS) & 1, abort_flag, lim);
+    }
+}
+
+template <int D>
+__device__ __forceinline__ void mma_issuer(const AttnParams& p, uint32_t base, uint32_t tmem,
+                                           int n, volatile int* abort_flag) {
+    using C = Cfg<D>;
+    auto bar = [&](int i) { return base + C::OFF_BAR + 8u * (uint32_t)i; };
+    const unsigned long long lim = p.wait_limit_ns;
+    constexpr uint32_t IDESC_S = idesc_bf16_f32(kBM, kBN, 0);  // K-major Q and K
+    constexpr uint32_t IDESC_O = idesc_bf16_f32(kBM, D, 1);    // V is MN-major (D contiguous)
+    const uint32_t s_col[2] = {C::S_COL0, C::S_COL1};
+    const uint32_t o_col[2] = {C::O_COL0, C::O_COL1};
+
+    // Descriptors are built once per operand tile; a K step only moves the start address,
+    // which lives in the low 14 bits (address >> 4) and never carries out of them here
+    // (shared memory < 256 KB).
+    const uint64_t dq[2] = {desc_sw128(base + C::OFF_Q, 16, 1024),
+                            desc_sw128(base + C::OFF_Q + C::TILE, 16, 1024)};
+    const uint64_t dk0 = desc_sw128(base + C::OFF_K, 16, 1024);
+    const uint64_t dv0 = desc_sw128(base + C::OFF_V, C::BLK, 1024);
+    // S_w = Q_w K^T over D in steps of 16: step kk lives in swizzle block kk/4 at byte 32*(kk%4).
+    auto issue_s = [&](int w, int slot) {
+        const uint64_t dk = dk0 + (uint64_t)((slot * C::TILE) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = ((kk / 4) * C::BLK + (kk % 4) * 32) >> 4;
+            mma_ss(tmem + s_col[w], dq[w] + off, dk + off, IDESC_S, kk > 0 ? 1u : 0u);
+        }
+    };
+    // O_w (+)= P_w V over 128 keys in steps of 16: P from TMEM (8 columns of bf16 pairs per
+    // step), V rows at 128-byte pitch (16 keys = 2048 B), 64-wide D blocks 16 KB apart.
+    auto issue_pv = [&](int w, int slot, bool acc) {
+        const uint64_t dv = dv0 + (uint64_t)((slot * C::TILE) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+            mma_ts(tmem + o_col[w], tmem + s_col[w] + kk * 8, dv + (uint64_t)((kk * 2048) >> 4),
+                   IDESC_O, (acc || kk > 0) ? 1u : 0u);
+    };
+
+    bool issued = false;
+    if (wait1(bar(C::BAR_Q), 0, abort_flag, lim, kErrMma) &&
+        wait1(bar(C::bar_kf(0)), 0, abort_flag, lim, kErrMma)) {
+        tc_fence_after();
+        issue_s(0, 0);
+        tc_commit(bar(C::bar_sf(0)));
+        issue_s(1, 0);
+        tc_commit(bar(C::bar_sf(1)));
+        tc_commit(bar(C::bar_ke(0)));
+        issued = true;
+        for (int jt = 0; jt < n; ++jt) {
+            const int slot_v = jt % C::NS;
+            const int slot_k = (jt + 1) % C::NS;
+            const bool more = jt + 1 < n;
+            if (!wait1(bar(C::bar_vf(slot_v)), (jt / C::NS) & 1, abort_flag, lim, kErrMma)) break;
+            if (!wait1(bar(C::bar_pf(0)), jt & 1, abort_flag, lim, kErrMma)) break;
+            tc_fence_after();
+            issue_pv(0, slot_v, jt > 0);
+            if (more) {
+                if (!wait1(bar(C::bar_kf(slot_k)), ((jt + 1) / C::NS) & 1, abort_flag, lim, kErrMma))
+                    break;
+                tc_fence_after();
+                issue_s(0, slot_k);
+                tc_commit(bar(C::bar_sf(0)));
+            } else {
+                tc_commit(bar(C::bar_of(0)));
+            }
+            if (!wait1(bar(C::bar_pf(1)), jt & 1, abort_flag, lim, kErrMma)) break;
+            tc_fence_after();
+            issue_pv(1, slot_v, jt > 0);
+            tc_commit(bar(C::bar_ve(slot_v)));
+            if (more) {
+                issue_s(1, slot_k);
+                tc_commit(bar(C::bar_sf(1)));
+                tc_commit(bar(C::bar_ke(slot_k)));
+            } else {
+                tc_commit(bar(C::bar_of(1)));
+            }
+        }
+    }
+    if (issued) {  // every MMA this thread issued completes before TMEM is released
+        tc_commit(bar(C::BAR_DRAIN));
+        wait_drain(bar(C::BAR_DRAIN), 0, abort_flag, lim);
+    }
+}
+
+template <int D>
+__device__ __forceinline__ void softmax_wg(const AttnParams& p, uint32_t base, uint32_t tmem,
+                                           const Sched& sched, int n, int wg, int b, int h,
+                                           int r0, volatile int* abort_flag) {
+    using C = Cfg<D>;
+    auto bar = [&](int i) { return base + C::OFF_BAR + 8u * (uint32_t)i; };
+    const unsigned long long lim = p.wait_limit_ns;
+    const unsigned FULL = 0xffffffffu;
+    const int wr = (threadIdx.x >> 5) & 3;  // warp within the warpgroup = TMEM lane quarter
+    const int lane = threadIdx.x & 31;
+    const int q_lo = r0 + wg * kBM;
+    const long long my_row = (long long)q_lo + wr * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(wr * 32) << 16;
+    const uint32_t tS = tmem + lane_off + (wg ? C::S_COL1 : C::S_COL0);
+    const uint32_t tO = tmem + lane_off + (wg ? C::O_COL1 : C::O_COL0);
+    const float sl2 = p.scale_log2;
+
+    // l_run: normaliser of the fp32 probabilities (gives the LSE); l_used: normaliser of
+    // the bf16-rounded probabilities that enter P.V (divides O, so that the weights applied
+    // to V sum to one exactly as used).
+    float m_run = -INFINITY, l_run = 0.f, l_used = 0.f;
+    bool ok = true;
+    SchedIter it;
+    it.begin(&sched);
+    for (int jt = 0; jt < n; ++jt, it.next()) {
+        if (!wait_warp(bar(C::bar_sf(wg)), jt & 1, abort_flag, lim)) {
+            ok = false;
+            break;
+        }
+        __syncwarp();
+        tc_fence_after();
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, sr[q]);
+        tmem_wait_ld();
+        float s[128];
+#pragma unroll
+        for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c / 32][c % 32]);
+
+        const long long k0 = (long long)it.chunk() * p.Lc + (long long)it.t * kBN;
+        const int kvalid = min(kBN, p.Lc - it.t * kBN);
+        const bool need_mask = (kvalid < kBN) || (p.causal && k0 + kBN - 1 > q_lo);
+        if (need_mask) {
+            const long long lim_c = p.causal ? my_row - k0 : (long long)kBN;  // keys c <= lim_c
+#pragma unroll
+            for (int c = 0; c < 128; ++c)
+                if (c >= kvalid || c > lim_c) s[c] = -INFINITY;
+        }
+        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+        for (int c = 4; c < 128; c += 4) {
+            mx0 = fmaxf(mx0, s[c]);
+            mx1 = fmaxf(mx1, s[c + 1]);
+            mx2 = fmaxf(mx2, s[c + 2]);
+            mx3 = fmaxf(mx3, s[c + 3]);
+        }
+        const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        const float m_new = fmaxf(m_run, mx * sl2);
+        float alpha = 1.f;
+        bool resc = false;
+        if (jt == 0) {
+            m_run = m_new;
+        } else if (m_new - m_run > kRescaleThreshold) {
+            alpha = ex2_approx(m_run - m_new);
+            m_run = m_new;
+            resc = true;
+        }
+        const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
+        float sum0 = 0.f, sum1 = 0.f, rsum0 = 0.f, rsum1 = 0.f;
+        // P = 2^(s*scale*log2e - m) in bf16 pairs, written over the first 64 columns of S
+        // (all of S is already in registers), one 64-key half at a time.
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            uint32_t pk[32];
+#pragma unroll
+            for (int c2 = 0; c2 < 32; ++c2) {
+                const int c = half * 64 + 2 * c2;
+                const float p0 = ex2_approx(fmaf(s[c], sl2, neg_m));
+                const float p1 = ex2_approx(fmaf(s[c + 1], sl2, neg_m));
+                sum0 += p0;
+                sum1 += p1;
+                const uint32_t pp = pack_bf16x2(p0, p1);
+                pk[c2] = pp;
+                // the bf16 values the P.V product actually uses
+                rsum0 += __uint_as_float(pp << 16);
+                rsum1 += __uint_as_float(pp & 0xffff0000u);
+            }
+            tmem_st32(tS + half * 32, pk);
+        }
+        l_run = l_run * alpha + (sum0 + sum1);
+        l_used = l_used * alpha + (rsum0 + rsum1);
+        if (__any_sync(FULL, resc)) {
+            // PV of the previous tile is complete: its commit preceded this tile's S commit.
+#pragma unroll
+            for (int cb = 0; cb < D / 32; ++cb) {
+                uint32_t o[32];
+                tmem_ld32(tO + cb * 32, o);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                tmem_st32(tO + cb * 32, o);
+            }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(C::bar_pf(wg)));
+    }
+    if (ok && !wait_warp(bar(C::bar_of(wg)), 0, abort_flag, lim)) ok = false;
+    if (!ok) return;
+    __syncwarp();
+    tc_fence_after();
+
+    const bool row_ok = my_row < p.L;
+    const float inv_l = 1.f / l_used;
+    const long long orow = ((long long)b * p.L + my_row) * p.H_q + h;
+#pragma unroll
+    for (int cb = 0; cb < D / 32; ++cb) {
+        uint32_t o[32];
+        tmem_ld32(tO + cb * 32, o);
+        tmem_wait_ld();
+        if (row_ok) {
+            if (!p.out_bf16) {
+                float4* dst = reinterpret_cast<float4*>((float*)p.out + orow * D + cb * 32);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv_l,
+                                         __uint_as_float(o[4 * i + 1]) * inv_l,
+                                         __uint_as_float(o[4 * i + 2]) * inv_l,
+                                         __uint_as_float(o[4 * i + 3]) * inv_l);
+            } else {
+                uint4* dst = reinterpret_cast<uint4*>((uint16_t*)p.out + orow * D + cb * 32);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dst[i] = make_uint4(
+                        pack_bf16x2(__uint_as_float(o[8 * i]) * inv_l, __uint_as_float(o[8 * i + 1]) * inv_l),
+                        pack_bf16x2(__uint_as_float(o[8 * i + 2]) * inv_l, __uint_as_float(o[8 * i + 3]) * inv_l),
+                        pack_bf16x2(__uint_as_float(o[8 * i + 4]) * inv_l, __uint_as_float(o[8 * i + 5]) * inv_l),
+                        pack_bf16x2(__uint_as_float(o[8 * i + 6]) * inv_l, __uint_as_float(o[8 * i + 7]) * inv_l));
+            }
+        }
+    }
+    if (row_ok)
+        p.lse[((long long)b * p.H_q + h) * p.L + my_row] =
+            (m_run + lg2_approx(l_run)) * 0.69314718055994530942f;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100(const __grid_constant__ AttnParams p) {
+    using C = Cfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint32_t base = smem_u32(smem_raw);
+    const uint32_t pad = (1024u - (base & 1023u)) & 1023u;
+    base += pad;
+    uint8_t* smem = smem_raw + pad;
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+    auto bar = [&](int i) { return base + C::OFF_BAR + 8u * (uint32_t)i; };
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int BH = p.B * p.H_q;
+    const int bh = blockIdx.x % BH;
+    const int rb = p.n_row_blocks - 1 - (int)(blockIdx.x / BH);  // heaviest row blocks first
+    const int b = bh / p.H_q, h = bh % p.H_q, g = h / p.group;
+    const int r0 = rb * 2 * kBM;
+
+    Sched sched;
+    sched.P = p.P;
+    sched.Lc = p.Lc;
+    sched.ntc = (p.Lc + kBN - 1) / kBN;
+    sched.i0 = r0 / p.Lc;
+    sched.causal = p.causal;
+    sched.last_row = min((long long)r0 + 2 * kBM - 1, (long long)p.L - 1);
+    const int n = sched.count();
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(C::BAR_Q), 1);
+        for (int s = 0; s < C::NS; ++s) {
+            mbar_init(bar(C::bar_kf(s)), 1);
+            mbar_init(bar(C::bar_ke(s)), 1);
+            mbar_init(bar(C::bar_vf(s)), 1);
+            mbar_init(bar(C::bar_ve(s)), 1);
+        }
+        for (int w = 0; w < 2; ++w) {
+            mbar_init(bar(C::bar_sf(w)), 1);
+            mbar_init(bar(C::bar_pf(w)), 4 * 32);
+            mbar_init(bar(C::bar_of(w)), 1);
+        }
+        mbar_init(bar(C::BAR_DRAIN), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == kWarpLoad && lane == 0) {
+        tma_prefetch_desc(&p.tm_q);
+    }
+    if (warp == kWarpMma) {
+        __syncwarp();
+        tmem_alloc(base + C::OFF_MISC, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp >= 8) {
+        regs_decrease<kRegsOther>();
+        if (warp == kWarpLoad) {
+            if (lane == 0) producer<D>(p, base, sched, n, b, h, g, r0, abort_flag);
+        } else if (warp == kWarpMma) {
+            if (lane == 0) mma_issuer<D>(p, base, tmem, n, abort_flag);
+        }
+    } else {
+        regs_increase<kRegsSoftmax>();
+        softmax_wg<D>(p, base, tmem, sched, n, warp >> 2, b, h, r0, abort_flag);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kWarpMma) {
+        __syncwarp();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// [D][H][rows][B] bf16 tensor, 128-row x 64-column boxes, 128-byte swizzle, zero fill.
+bool encode_tile_map(CUtensorMap* m, const void* ptr, int D, int H, long long rows, int B,
+                     long long bstride_elems) {
+    auto enc = get_encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)bstride_elems * 2};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)kBM, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch_d(const AttnParams& p, int grid, cudaStream_t stream) {
+    using C = Cfg<D>;
+    static int configured_for = -1;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (configured_for != dev) {
+        e = cudaFuncSetAttribute(attn_fwd_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM);
+        if (e != cudaSuccess) return e;
+        configured_for = dev;
+    }
+    attn_fwd_sm100<D><<<grid, kThreads, C::SMEM, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_sm100(const AttnArgs& a, unsigned long long wait_limit_ns,
+                              int inject_stall, const char** why) {
+    static thread_local AttnParams p;  // ~16.6 KB of tensor maps: kept off the stack
+    const long long L = (long long)a.P * a.Lc;
+    if (!encode_tile_map(&p.tm_q, a.q, a.D, a.H_q, L, a.B, a.q_bstride)) {
+        *why = "cuTensorMapEncodeTiled failed for q";
+        return cudaErrorInvalidValue;
+    }
+    for (int j = 0; j < a.P; ++j) {
+        if (!encode_tile_map(&p.tm_k[j], a.k_chunks[j], a.D, a.H_kv, a.Lc, a.B, a.kv_bstride) ||
+            !encode_tile_map(&p.tm_v[j], a.v_chunks[j], a.D, a.H_kv, a.Lc, a.B, a.kv_bstride)) {
+            *why = "cuTensorMapEncodeTiled failed for a K/V chunk";
+            return cudaErrorInvalidValue;
+        }
+    }
+    p.out = a.out;
+    p.lse = a.lse;
+    p.P = a.P;
+    p.B = a.B;
+    p.H_q = a.H_q;
+    p.H_kv = a.H_kv;
+    p.Lc = a.Lc;
+    p.L = (int)L;
+    p.causal = a.causal;
+    p.out_bf16 = a.out_bf16;
+    p.group = a.H_q / a.H_kv;
+    p.n_row_blocks = (int)((L + 2 * kBM - 1) / (2 * kBM));
+    p.scale_log2 = (float)((double)a.scale * 1.4426950408889634);
+    p.inject_stall = inject_stall;
+    p.wait_limit_ns = wait_limit_ns;
+    const long long grid = (long long)p.n_row_blocks * a.B * a.H_q;
+    if (grid > 0x7fffffffLL) {
+        *why = "problem too large for one launch";
+        return cudaErrorInvalidValue;
+    }
+    if (a.D == 128) return launch_d<128>(p, (int)grid, a.stream);
+    if (a.D == 64) return launch_d<64>(p, (int)grid, a.stream);
+    *why = "head dimension not supported by the tensor-core path";
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t read_and_clear_error_word(unsigned int* value) {
+    cudaError_t e = cudaMemcpyFromSymbol(value, g_ra_error_word, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    if (*value) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_ra_error_word, &zero, sizeof(unsigned int));
+    }
+    return e;
+}
+
+}  // namespace ra

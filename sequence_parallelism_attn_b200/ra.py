@@ -1,0 +1,187 @@
+"""ctypes binding of libra_b200.so (the C ABI of include/ra.h), entry point for entry point.
+
+Argument marshalling only: torch tensors are turned into device pointers, sizes and
+the current CUDA stream; every step of the computation runs in the library's CUDA
+kernels.  Loading fails loudly if the library has not been built -- there is no
+fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libra_b200.so")
+
+RA_OK, RA_ERR_INVALID, RA_ERR_UNSUPPORTED, RA_ERR_CUDA, RA_ERR_TIMEOUT = 0, 1, 2, 3, 4
+RA_BF16, RA_FP32 = 0, 1
+RA_MAX_P = 64
+EXPORTED = ("ra_ring_attn_fwd", "ra_lse_merge", "ra_ulysses_seq2head", "ra_ulysses_head2seq",
+            "ra_sync_status", "ra_last_error", "ra_set_wait_limit_ns", "ra_debug_inject_stall",
+            "ra_version")
+
+
+class RaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"ra status {status}: {message}")
+        self.status = status
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libra_b200.so (built by sequence_parallelism_attn_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m sequence_parallelism_attn_b200.build` (no fallback path)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_float
+    lib.ra_ring_attn_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i64, i64, f32, i32,
+                                     i32, i32, vp, vp, vp]
+    lib.ra_lse_merge.argtypes = [vp, vp, vp, vp, i32, i32, i64, i32, vp]
+    lib.ra_ulysses_seq2head.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, vp]
+    lib.ra_ulysses_head2seq.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp]
+    lib.ra_sync_status.argtypes = [vp]
+    for f in ("ra_ring_attn_fwd", "ra_lse_merge", "ra_ulysses_seq2head", "ra_ulysses_head2seq",
+              "ra_sync_status"):
+        getattr(lib, f).restype = ctypes.c_int
+    lib.ra_last_error.restype = ctypes.c_char_p
+    lib.ra_version.restype = ctypes.c_char_p
+    lib.ra_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+    lib.ra_set_wait_limit_ns.restype = ctypes.c_ulonglong
+    lib.ra_debug_inject_stall.argtypes = [i32]
+    lib.ra_debug_inject_stall.restype = None
+    _lib = lib
+    return lib
+
+
+def _check(status: int):
+    if status != RA_OK:
+        raise RaError(status, load().ra_last_error().decode())
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dt(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return RA_BF16
+    if t == torch.float32:
+        return RA_FP32
+    raise ValueError(f"unsupported dtype {t}")
+
+
+def version() -> str:
+    return load().ra_version().decode()
+
+
+# ------------------------------------------------------------------ raw entry points
+def ra_ring_attn_fwd(q_ptr, k_ptrs, v_ptrs, P, B, H_q, H_kv, Lc, D, q_bstride, kv_bstride, scale,
+                     causal, in_dtype, out_dtype, out_ptr, lse_ptr, stream):
+    """The C entry point with raw pointers (k_ptrs/v_ptrs: sequences of P device pointers)."""
+    arr = ctypes.c_void_p * P
+    ks, vs = arr(*k_ptrs), arr(*v_ptrs)
+    _check(load().ra_ring_attn_fwd(q_ptr, ks, vs, P, B, H_q, H_kv, Lc, D, q_bstride, kv_bstride,
+                                   scale, int(causal), in_dtype, out_dtype, out_ptr, lse_ptr,
+                                   stream))
+
+
+def ra_lse_merge(o_a: torch.Tensor, lse_a: torch.Tensor, o_b: torch.Tensor, lse_b: torch.Tensor,
+                 stream=None):
+    """In-place merge into (o_a, lse_a).  o [B,L,H,D] fp32, lse [B,H,L] fp32."""
+    B, L, H, D = o_a.shape
+    for t in (o_a, lse_a, o_b, lse_b):
+        assert t.is_cuda and t.dtype == torch.float32 and t.is_contiguous()
+    assert o_b.shape == o_a.shape and lse_a.shape == lse_b.shape == (B, H, L)
+    _check(load().ra_lse_merge(o_a.data_ptr(), lse_a.data_ptr(), o_b.data_ptr(), lse_b.data_ptr(),
+                               B, H, L, D, _stream(stream)))
+
+
+def ra_ulysses_seq2head(x: torch.Tensor, H_out: int | None = None, out: torch.Tensor | None = None,
+                        stream=None) -> torch.Tensor:
+    """[P,B,Lc,H_in,D] -> [P,B,P*Lc,H_out/P,D] (H_out defaults to H_in)."""
+    assert x.is_cuda and x.is_contiguous() and x.dim() == 5
+    P, B, Lc, H_in, D = x.shape
+    H_out = H_in if H_out is None else H_out
+    if out is None:
+        out = torch.empty((P, B, P * Lc, max(H_out // P, 1), D), dtype=x.dtype, device=x.device)
+    _check(load().ra_ulysses_seq2head(x.data_ptr(), out.data_ptr(), P, B, Lc, H_in, H_out, D,
+                                      _dt(x.dtype), _stream(stream)))
+    return out
+
+
+def ra_ulysses_head2seq(x: torch.Tensor, out: torch.Tensor | None = None,
+                        stream=None) -> torch.Tensor:
+    """[P,B,P*Lc,H/P,D] -> [P,B,Lc,H,D]."""
+    assert x.is_cuda and x.is_contiguous() and x.dim() == 5
+    P, B, L, Hl, D = x.shape
+    Lc = L // P
+    if out is None:
+        out = torch.empty((P, B, Lc, Hl * P, D), dtype=x.dtype, device=x.device)
+    _check(load().ra_ulysses_head2seq(x.data_ptr(), out.data_ptr(), P, B, Lc, Hl * P, D,
+                                      _dt(x.dtype), _stream(stream)))
+    return out
+
+
+def ra_sync_status(stream=None) -> int:
+    """Synchronise the stream and return the kernel status (RA_OK or RA_ERR_TIMEOUT)."""
+    return load().ra_sync_status(_stream(stream))
+
+
+def ra_last_error() -> str:
+    return load().ra_last_error().decode()
+
+
+def ra_set_wait_limit_ns(ns: int) -> int:
+    return load().ra_set_wait_limit_ns(ns)
+
+
+def ra_debug_inject_stall(on: bool):
+    load().ra_debug_inject_stall(1 if on else 0)
+
+
+# ------------------------------------------------------------------ tensor-level helper
+def ring_attn_fwd(q: torch.Tensor, k_chunks, v_chunks, causal: bool, scale: float | None = None,
+                  out_dtype: torch.dtype = torch.float32, out: torch.Tensor | None = None,
+                  lse: torch.Tensor | None = None, stream=None):
+    """Ring-chunked attention of q [B, P*Lc, H_q, D] against P K/V chunks.
+
+    k_chunks / v_chunks: a tensor [P, B, Lc, H_kv, D] (chunk j = k_chunks[j]) or a list
+    of P tensors [B, Lc, H_kv, D], each batch-contiguous with the same batch stride.
+    Returns (out [B, P*Lc, H_q, D] in out_dtype, lse [B, H_q, P*Lc] fp32).
+    """
+    if isinstance(k_chunks, torch.Tensor):
+        k_list = [k_chunks[j] for j in range(k_chunks.shape[0])]
+        v_list = [v_chunks[j] for j in range(v_chunks.shape[0])]
+    else:
+        k_list, v_list = list(k_chunks), list(v_chunks)
+    P = len(k_list)
+    B, L, H_q, D = q.shape
+    _, Lc, H_kv, _ = k_list[0].shape
+    assert L == P * Lc, "q length must equal P * Lc"
+    assert q.stride(3) == 1 and q.stride(2) == D and q.stride(1) == H_q * D
+    kv_bstride = k_list[0].stride(0)
+    for t in k_list + v_list:
+        assert t.shape == (B, Lc, H_kv, D) and t.dtype == q.dtype and t.is_cuda
+        assert t.stride(3) == 1 and t.stride(2) == D and t.stride(1) == H_kv * D
+        assert B == 1 or t.stride(0) == kv_bstride
+    if scale is None:
+        scale = D ** -0.5
+    if out is None:
+        out = torch.empty((B, L, H_q, D), dtype=out_dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H_q, L), dtype=torch.float32, device=q.device)
+    ra_ring_attn_fwd(q.data_ptr(), [t.data_ptr() for t in k_list], [t.data_ptr() for t in v_list],
+                     P, B, H_q, H_kv, Lc, D, q.stride(0) if B > 1 else L * H_q * D,
+                     kv_bstride if B > 1 else Lc * H_kv * D, float(scale), int(bool(causal)),
+                     _dt(q.dtype), _dt(out.dtype), out.data_ptr(), lse.data_ptr(), _stream(stream))
+    return out, lse

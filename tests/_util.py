@@ -1,0 +1,42 @@
+"""Helpers for the GPU parity tests: tolerances, comparisons and the oracle call shapes."""
+import numpy as np
+import torch
+
+# Tolerances fixed for this path: bf16 inputs with fp32 accumulation -> max-abs 1e-2 on O
+# and 1e-3 on LSE; fp32 inputs -> 1e-4 on both.
+TOL = {torch.bfloat16: (1e-2, 1e-3), torch.float32: (1e-4, 1e-4)}
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    """Exact fp64 copy of a (bf16 or fp32) tensor."""
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def chunks_to_seq(x: torch.Tensor) -> torch.Tensor:
+    """[P, B, Lc, H, D] chunk-major K/V -> [B, P*Lc, H, D] in global token order."""
+    P, B, Lc, H, D = x.shape
+    return x.permute(1, 0, 2, 3, 4).reshape(B, P * Lc, H, D)
+
+
+def max_abs(a, b) -> float:
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    assert a.shape == b.shape, (a.shape, b.shape)
+    if a.size == 0:
+        return 0.0
+    assert np.all(np.isfinite(a)), "non-finite values in the GPU result"
+    return float(np.max(np.abs(a - b)))
+
+
+def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
+    """Half a bf16 unit in the last place at |x| (8 significand bits)."""
+    ax = np.maximum(np.abs(x), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(ax)) - 8)
+
+
+def rows_oracle(oracle_mod, q, k_seq, v_seq, rows, scale, causal):
+    """Oracle output for sampled (b, t, h) rows; q [B,L,H_q,D], k/v [B,L,H_kv,D] tensors."""
+    rb, rt, rh = rows
+    qn = f64(q[torch.tensor(rb), torch.tensor(rt), torch.tensor(rh)])
+    return oracle_mod.attention_rows(qn, rb, rt, rh, f64(k_seq), f64(v_seq), q.shape[2], scale,
+                                     causal)

@@ -1,0 +1,110 @@
+"""Host-side tests of the C ABI: the library builds, loads without a GPU, exports every
+entry point include/ra.h declares, and rejects bad arguments before launching anything
+(no compute call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sequence_parallelism_attn_b200 import build, ra
+    build.build()
+    return ra.load()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "ra.h")).read()
+    return sorted(set(re.findall(r"RA_API\s+[\w\s\*]+?\b(ra_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_symbols()
+    for required in ("ra_ring_attn_fwd", "ra_lse_merge", "ra_ulysses_seq2head",
+                     "ra_ulysses_head2seq", "ra_sync_status", "ra_last_error"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    from sequence_parallelism_attn_b200 import ra
+    assert sorted(ra.EXPORTED) == declared_symbols()
+
+
+def test_only_ra_symbols_are_exported(lib):
+    import subprocess
+    from sequence_parallelism_attn_b200 import ra
+    out = subprocess.run(["nm", "-D", "--defined-only", ra.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    names = sorted(l.split()[-1] for l in out.splitlines() if l.strip())
+    assert names == declared_symbols()
+
+
+def test_version(lib):
+    from sequence_parallelism_attn_b200 import ra
+    assert "sm_100a" in ra.version()
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: every call below fails validation
+
+
+def _attn(lib, **kw):
+    a = dict(q=FAKE, k=[FAKE], v=[FAKE], P=1, B=1, H_q=2, H_kv=1, Lc=128, D=128,
+             qb=None, kvb=None, scale=0.1, causal=1, ind=0, outd=1, out=FAKE, lse=FAKE)
+    a.update(kw)
+    P = a["P"]
+    arr = ctypes.c_void_p * max(P, 1)
+    ks = arr(*(a["k"] * P)[:P]) if P > 0 else None
+    vs = arr(*(a["v"] * P)[:P]) if P > 0 else None
+    L = max(P, 1) * a["Lc"]
+    qb = a["qb"] if a["qb"] is not None else L * a["H_q"] * a["D"]
+    kvb = a["kvb"] if a["kvb"] is not None else a["Lc"] * a["H_kv"] * a["D"]
+    return lib.ra_ring_attn_fwd(a["q"], ks, vs, P, a["B"], a["H_q"], a["H_kv"], a["Lc"], a["D"],
+                                qb, kvb, a["scale"], a["causal"], a["ind"], a["outd"], a["out"],
+                                a["lse"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(P=0), 1), (dict(P=65), 1), (dict(B=0), 1), (dict(H_q=3, H_kv=2), 1),
+    (dict(causal=2), 1), (dict(scale=0.0), 1), (dict(scale=float("nan")), 1),
+    (dict(ind=1, outd=0), 1), (dict(D=32), 2), (dict(D=96), 2), (dict(ind=1, D=48), 2),
+    (dict(q=FAKE + 8), 1), (dict(q=0), 1), (dict(out=FAKE + 4), 1), (dict(lse=0), 1),
+    (dict(k=[0]), 1), (dict(v=[FAKE + 2]), 1), (dict(qb=5), 1), (dict(B=2, kvb=128 * 128 + 3), 1),
+    (dict(ind=5), 1),
+])
+def test_attention_argument_validation(lib, kw, status):
+    assert _attn(lib, **kw) == status
+    assert lib.ra_last_error()
+
+
+def test_permute_argument_validation(lib):
+    s2h, h2s = lib.ra_ulysses_seq2head, lib.ra_ulysses_head2seq
+    # heads not divisible by ranks ("heads divisible by the number of GPUs")
+    assert s2h(FAKE, FAKE * 2, 4, 1, 16, 6, 6, 64, 0, None) == 1
+    assert b"divisible" in lib.ra_last_error()
+    assert s2h(FAKE, FAKE * 2, 4, 1, 16, 3, 8, 64, 0, None) == 1   # H_out % H_in
+    assert s2h(FAKE, FAKE * 2, 2, 1, 16, 2, 2, 4, 0, None) == 1    # D*2 bytes % 16
+    assert s2h(FAKE + 2, FAKE * 2, 2, 1, 16, 2, 2, 64, 0, None) == 1
+    assert s2h(FAKE, FAKE, 2, 1, 16, 2, 2, 64, 0, None) == 1        # aliasing
+    assert s2h(FAKE, FAKE * 2, 2, 1, 0, 2, 2, 64, 0, None) == 1
+    assert h2s(FAKE, FAKE * 2, 3, 1, 16, 4, 64, 0, None) == 1
+    assert h2s(FAKE, FAKE * 2, 2, 1, 16, 4, 64, 7, None) == 1       # bad dtype
+
+
+def test_merge_argument_validation(lib):
+    m = lib.ra_lse_merge
+    assert m(FAKE, FAKE * 2, FAKE * 3, FAKE * 4, 1, 1, 8, 6, None) == 2  # D % 4
+    assert m(FAKE, FAKE * 2, FAKE, FAKE * 4, 1, 1, 8, 8, None) == 1      # o_b aliases o_a
+    assert m(0, FAKE * 2, FAKE * 3, FAKE * 4, 1, 1, 8, 8, None) == 1
+    assert m(FAKE, FAKE * 2, FAKE * 3, FAKE * 4, 1, 0, 8, 8, None) == 1
+
+
+def test_wait_limit_roundtrip(lib):
+    old = lib.ra_set_wait_limit_ns(12345)
+    assert lib.ra_set_wait_limit_ns(0) == 12345
+    assert lib.ra_set_wait_limit_ns(old) == 4000000000

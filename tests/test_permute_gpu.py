@@ -1,0 +1,77 @@
+"""GPU parity of the Ulysses transforms: bit-exact against the oracle's index loops.
+
+Source: "Метод контекстного параллелизма Ulysses" (seq-sharded [local_seqlen,
+global_heads, head_dim] <-> head-sharded [global_seqlen, local_heads, head_dim], KV heads
+copied up under GQA)."""
+import numpy as np
+import pytest
+import torch
+
+from sequence_parallelism_attn_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    """The raw bits of a tensor (uint16 for bf16, uint32 for fp32)."""
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    return t.view(torch.int32).numpy().view(np.uint32)
+
+
+@pytest.mark.parametrize("P,B,Lc,H_in,H_out,D,dtype", [
+    (2, 1, 64, 2, 2, 32, torch.float32),       # the tiny fp32 workload
+    (4, 1, 1024, 8, 8, 64, torch.bfloat16),    # [4 x 1024, 8, 64] -> [4096, 2/rank, 64]
+    (8, 1, 1000, 4, 8, 128, torch.bfloat16),   # GQA copy: 4 kv heads over 8 ranks
+    (4, 2, 37, 8, 8, 64, torch.bfloat16),      # ragged token count, B > 1
+    (2, 3, 5, 2, 4, 8, torch.bfloat16),        # 16-byte heads (one vector): unvectorised path
+    (3, 2, 11, 3, 6, 32, torch.float32),       # odd rank count, replication 2
+    (1, 1, 9, 4, 4, 64, torch.bfloat16),       # one rank: identity layout
+    (8, 1, 16, 1, 8, 128, torch.bfloat16),     # one kv head copied to every rank
+])
+def test_seq2head_bit_exact(ra_lib, oracle_mod, P, B, Lc, H_in, H_out, D, dtype):
+    g = torch.Generator().manual_seed(P * 1000 + Lc)
+    x = torch.randn(P, B, Lc, H_in, D, generator=g).to(dtype)
+    y = ra_lib.ra_ulysses_seq2head(x.cuda(), H_out)
+    torch.cuda.synchronize()
+    want = oracle_mod.seq2head(_bits(x), H_out)
+    assert np.array_equal(_bits(y), want)
+
+
+@pytest.mark.parametrize("P,B,Lc,H,D,dtype", [
+    (2, 1, 64, 2, 32, torch.float32), (4, 1, 1024, 8, 64, torch.bfloat16),
+    (4, 2, 37, 8, 64, torch.bfloat16), (2, 3, 5, 4, 8, torch.bfloat16),
+    (3, 2, 11, 6, 32, torch.float32), (8, 1, 300, 32, 128, torch.bfloat16)])
+def test_head2seq_bit_exact(ra_lib, oracle_mod, P, B, Lc, H, D, dtype):
+    g = torch.Generator().manual_seed(P * 7 + Lc)
+    x = torch.randn(P, B, P * Lc, H // P, D, generator=g).to(dtype)
+    y = ra_lib.ra_ulysses_head2seq(x.cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(_bits(y), oracle_mod.head2seq(_bits(x)))
+
+
+def test_round_trip_is_identity(ra_lib):
+    w = synth.SMALL_PERMUTE
+    q, _, _ = synth.ulysses_inputs(w)
+    x = q.cuda()
+    z = ra_lib.ra_ulysses_head2seq(ra_lib.ra_ulysses_seq2head(x))
+    torch.cuda.synchronize()
+    assert torch.equal(z.view(torch.int16), x.view(torch.int16))
+
+
+def test_full_size_ulysses_transforms_bit_exact(ra_lib, oracle_mod):
+    """The 128k-token Ulysses workload: Q [8 x 16384, 32, 128] and the GQA copy of
+    K [8 x 16384, 4 -> 8, 128], each against the oracle over every element."""
+    w = synth.ULYSSES_128K
+    q, k, _ = synth.ulysses_inputs(w)
+    for x, h_out in ((q, w.H_q), (k, w.H_kv_rep)):
+        y = ra_lib.ra_ulysses_seq2head(x.cuda(), h_out)
+        torch.cuda.synchronize()
+        assert np.array_equal(_bits(y), oracle_mod.seq2head(_bits(x), h_out))
+        del y
+    yq = oracle_mod.seq2head(_bits(q), w.H_q)
+    back = ra_lib.ra_ulysses_head2seq(
+        torch.from_numpy(yq.view(np.int16)).view(torch.bfloat16).cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(_bits(back), _bits(q))

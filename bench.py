@@ -13,7 +13,7 @@ the steps (max over ranks), in TFLOP/s.  With --gpus N every rank runs its own r
 (weak scaling: the path has no data-path exchange between independent replicas).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload ulysses_e2e|long_128k|llama8b_32k|small_4k]
+                  [--workload ulysses_e2e|ulysses_32k|long_128k|llama8b_32k|small_4k]
 """
 from __future__ import annotations
 
@@ -52,6 +52,7 @@ def workloads():
     from sequence_parallelism_attn_b200 import synth
     return {
         "ulysses_e2e": ("ulysses", synth.ULYSSES_128K),
+        "ulysses_32k": ("ulysses", synth.ULYSSES_32K),
         "long_128k": ("attn", synth.LONG_128K),
         "llama8b_32k": ("attn", synth.LLAMA8B_GQA),
         "small_4k": ("attn", synth.SMALL_BF16),
@@ -342,6 +343,8 @@ def main():
     ap.add_argument("--workload", default="ulysses_e2e")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-step-seconds", type=float, default=None,
+                    help="reference arm: target seconds of oracle work per step")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -440,7 +443,7 @@ def reference_arm(args, kind, w, w_attn, rank, world):
     oracle.build()
     cores = os.cpu_count() or 1
     # size one step's sample so that warmup + steps end within a few minutes
-    per_step_s = max(2.0, min(20.0, 150.0 / (args.steps + args.warmup)))
+    per_step_s = args.ref_step_seconds or max(2.0, min(20.0, 150.0 / (args.steps + args.warmup)))
     tf, n, dt, _ = run_oracle_sample(w_attn, target_s=per_step_s)
     import numpy as np
     q, rb, rt, rh, k, v, flops = oracle_sample(w_attn, n)

@@ -140,7 +140,7 @@ ra_status ra_ulysses_seq2head(const void* in, void* out, int P, int B, int Lc, i
     ra_status s = check_permute(in, out, P, B, Lc, H_in, H_out, D, dt);
     if (s != RA_OK) return s;
     cudaError_t e = ra::launch_seq2head(in, out, P, B, Lc, H_in, H_out, D, elem_size(dt),
-                                        (cudaStream_t)stream);
+                                        (cudaStream_t)stream, g_wait_limit_ns.load());
     if (e != cudaSuccess) return cuda_fail(e, "seq2head launch");
     return RA_OK;
 }
@@ -149,8 +149,8 @@ ra_status ra_ulysses_head2seq(const void* in, void* out, int P, int B, int Lc, i
                               ra_dtype dt, void* stream) {
     ra_status s = check_permute(in, out, P, B, Lc, H, H, D, dt);
     if (s != RA_OK) return s;
-    cudaError_t e =
-        ra::launch_head2seq(in, out, P, B, Lc, H, D, elem_size(dt), (cudaStream_t)stream);
+    cudaError_t e = ra::launch_head2seq(in, out, P, B, Lc, H, D, elem_size(dt),
+                                        (cudaStream_t)stream, g_wait_limit_ns.load());
     if (e != cudaSuccess) return cuda_fail(e, "head2seq launch");
     return RA_OK;
 }
@@ -158,14 +158,16 @@ ra_status ra_ulysses_head2seq(const void* in, void* out, int P, int B, int Lc, i
 ra_status ra_sync_status(void* stream) {
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
-    unsigned int word = 0;
+    unsigned int word = 0, pword = 0;
     e = ra::read_and_clear_error_word(&word);
+    if (e == cudaSuccess) e = ra::read_and_clear_permute_error(&pword);
     if (e != cudaSuccess) return cuda_fail(e, "reading the kernel error word");
+    word |= pword ? 16u : 0u;
     if (word) {
         char buf[128];
         std::snprintf(buf, sizeof buf,
                       "a kernel gave up on a bounded wait (error bits 0x%x: 1 load, 2 mma, "
-                      "4 softmax, 8 drain)", word);
+                      "4 softmax, 8 drain, 16 permute)", word);
         return fail(RA_ERR_TIMEOUT, buf);
     }
     return RA_OK;

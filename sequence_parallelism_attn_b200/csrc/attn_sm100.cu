@@ -20,9 +20,10 @@
 // Kernel organisation (one CTA per 256 query rows of one (batch, head); 384 threads):
 //   warps 0-3  softmax for query tile A (rows r0 .. r0+127), one TMEM lane (= row) each
 //   warps 4-7  softmax for query tile B (rows r0+128 .. r0+255)
-//   warp 8     TMA producer: Q tiles once, then K and V tiles into NS-deep rings
+//   warp 8     TMA producer of the Q tiles (once) and the K tiles (NSK-deep ring)
 //   warp 9     MMA issuer (one thread) and TMEM owner
-//   warps 10-11 idle (they complete the third warpgroup for the register split)
+//   warp 10    TMA producer of the V tiles (NSV-deep ring)
+//   warp 11    idle (it completes the third warpgroup for the register split)
 // Registers: launched at 168 per thread (3 warps per SM sub-partition); the softmax
 // warpgroups raise their budget to 216 and the third warpgroup drops to 72
 // (216 + 216 + 72 = 504 <= 512 per sub-partition; 256*216 + 128*72 = 384*168).
@@ -57,9 +58,10 @@ __device__ unsigned int g_ra_error_word = 0;
 namespace {
 
 constexpr int kThreads = 384;
-constexpr uint32_t kRegsSoftmax = 216, kRegsOther = 72;
+constexpr uint32_t kRegsSoftmax = 208, kRegsOther = 88;
 constexpr int kWarpLoad = 8;
 constexpr int kWarpMma = 9;
+constexpr int kWarpLoadV = 10;
 constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 128;  // keys per tile
 constexpr uint32_t kTmemCols = 512;
@@ -86,27 +88,31 @@ struct Cfg {
     static constexpr int TILE = kBM * D * 2;  // bytes of a 128 x D bf16 tile
     static constexpr int NKB = D / 64;        // 64-column (128-byte) swizzle blocks per tile
     static constexpr int BLK = kBM * 128;     // bytes of one swizzle block (16 KB)
-    static constexpr int NS = (D == 128) ? 2 : 4;
+    // K is needed first in each step (S = Q K^T right after the previous P V), so its ring
+    // is the deeper one.  D = 128: 64 KB Q + 3 x 32 KB K + 2 x 32 KB V = 224 KB.
+    static constexpr int NSK = (D == 128) ? 3 : 4;
+    static constexpr int NSV = (D == 128) ? 2 : 4;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = 2 * TILE;
-    static constexpr int OFF_V = OFF_K + NS * TILE;
-    static constexpr int OFF_BAR = OFF_V + NS * TILE;
-    // barriers: q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2],
+    static constexpr int OFF_V = OFF_K + NSK * TILE;
+    static constexpr int OFF_BAR = OFF_V + NSV * TILE;
+    // barriers: q_full, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV], s_full[2],
     // p_full[2], o_full[2], drain
-    static constexpr int N_BARS = 1 + 4 * NS + 2 + 2 + 2 + 1;
+    static constexpr int N_BARS = 1 + 2 * NSK + 2 * NSV + 2 + 2 + 2 + 1;
     static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem base (4 B), abort flag (4 B)
     static constexpr int SMEM = OFF_MISC + 16 + 1024;      // + slack for 1024-B alignment
     static constexpr int BAR_Q = 0;
     __host__ __device__ static constexpr int bar_kf(int s) { return 1 + s; }
-    __host__ __device__ static constexpr int bar_ke(int s) { return 1 + NS + s; }
-    __host__ __device__ static constexpr int bar_vf(int s) { return 1 + 2 * NS + s; }
-    __host__ __device__ static constexpr int bar_ve(int s) { return 1 + 3 * NS + s; }
-    __host__ __device__ static constexpr int bar_sf(int w) { return 1 + 4 * NS + w; }
-    __host__ __device__ static constexpr int bar_pf(int w) { return 3 + 4 * NS + w; }
-    __host__ __device__ static constexpr int bar_of(int w) { return 5 + 4 * NS + w; }
-    static constexpr int BAR_DRAIN = 7 + 4 * NS;
+    __host__ __device__ static constexpr int bar_ke(int s) { return 1 + NSK + s; }
+    __host__ __device__ static constexpr int bar_vf(int s) { return 1 + 2 * NSK + s; }
+    __host__ __device__ static constexpr int bar_ve(int s) { return 1 + 2 * NSK + NSV + s; }
+    __host__ __device__ static constexpr int bar_sf(int w) { return 1 + 2 * NSK + 2 * NSV + w; }
+    __host__ __device__ static constexpr int bar_pf(int w) { return 3 + 2 * NSK + 2 * NSV + w; }
+    __host__ __device__ static constexpr int bar_of(int w) { return 5 + 2 * NSK + 2 * NSV + w; }
+    static constexpr int BAR_DRAIN = 7 + 2 * NSK + 2 * NSV;
     static constexpr uint32_t S_COL0 = 0, S_COL1 = 128;
     static constexpr uint32_t O_COL0 = 256, O_COL1 = 256 + D;
+    static_assert(SMEM <= 232448, "shared memory budget");
 };
 
 // The chunk/tile visiting order of one CTA (all roles derive the same sequence).
@@ -216,59 +222,53 @@ __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatil
     }
 }
 
-template <int D>
+// K/V producer: one thread streams either the K tiles (and first the two Q tiles) or the
+// V tiles of the CTA's schedule through its ring, each with its own bounded waits.
+template <int D, bool IS_K>
 __device__ __forceinline__ void producer(const AttnParams& p, uint32_t base, const Sched& sched,
                                          int n, int b, int h, int g, int r0,
                                          volatile int* abort_flag) {
     using C = Cfg<D>;
+    constexpr int NS = IS_K ? C::NSK : C::NSV;
     auto bar = [&](int i) { return base + C::OFF_BAR + 8u * (uint32_t)i; };
+    auto bar_full = [&](int s) { return bar(IS_K ? C::bar_kf(s) : C::bar_vf(s)); };
+    auto bar_empty = [&](int s) { return bar(IS_K ? C::bar_ke(s) : C::bar_ve(s)); };
+    const uint32_t ring = base + (IS_K ? C::OFF_K : C::OFF_V);
+    const CUtensorMap* maps = IS_K ? p.tm_k : p.tm_v;
     const unsigned long long lim = p.wait_limit_ns;
-    int k_armed[C::NS], v_armed[C::NS];
+    int armed[NS];
 #pragma unroll
-    for (int s = 0; s < C::NS; ++s) k_armed[s] = v_armed[s] = -1;
+    for (int s = 0; s < NS; ++s) armed[s] = -1;
 
-    mbar_arrive_expect_tx(bar(C::BAR_Q), 2 * C::TILE);
+    if (IS_K) {
+        mbar_arrive_expect_tx(bar(C::BAR_Q), 2 * C::TILE);
 #pragma unroll
-    for (int kb = 0; kb < C::NKB; ++kb) {
-        tma_load_4d(base + C::OFF_Q + kb * C::BLK, &p.tm_q, bar(C::BAR_Q), kb * 64, h, r0, b);
-        tma_load_4d(base + C::OFF_Q + C::TILE + kb * C::BLK, &p.tm_q, bar(C::BAR_Q), kb * 64, h,
-                    r0 + kBM, b);
+        for (int kb = 0; kb < C::NKB; ++kb) {
+            tma_load_4d(base + C::OFF_Q + kb * C::BLK, &p.tm_q, bar(C::BAR_Q), kb * 64, h, r0, b);
+            tma_load_4d(base + C::OFF_Q + C::TILE + kb * C::BLK, &p.tm_q, bar(C::BAR_Q), kb * 64,
+                        h, r0 + kBM, b);
+        }
     }
     SchedIter it;
     it.begin(&sched);
     for (int jt = 0; jt < n; ++jt, it.next()) {
-        const int slot = jt % C::NS;
-        const int j = it.chunk();
-        const int row0 = it.t * kBN;
-        if (jt >= C::NS && !wait1(bar(C::bar_ke(slot)), ((jt / C::NS) - 1) & 1, abort_flag, lim,
-                                  kErrProducer))
+        const int slot = jt % NS;
+        if (jt >= NS && !wait1(bar_empty(slot), ((jt / NS) - 1) & 1, abort_flag, lim, kErrProducer))
             break;
         // Test hook: withhold the last K tile so the consumer's bounded wait expires.
-        if (!(p.inject_stall && jt == n - 1)) {
-            mbar_arrive_expect_tx(bar(C::bar_kf(slot)), C::TILE);
-#pragma unroll
-            for (int kb = 0; kb < C::NKB; ++kb)
-                tma_load_4d(base + C::OFF_K + slot * C::TILE + kb * C::BLK, &p.tm_k[j],
-                            bar(C::bar_kf(slot)), kb * 64, g, row0, b);
-            k_armed[slot] = jt;
-        }
-        if (jt >= C::NS && !wait1(bar(C::bar_ve(slot)), ((jt / C::NS) - 1) & 1, abort_flag, lim,
-                                  kErrProducer))
-            break;
-        mbar_arrive_expect_tx(bar(C::bar_vf(slot)), C::TILE);
+        if (IS_K && p.inject_stall && jt == n - 1) continue;
+        mbar_arrive_expect_tx(bar_full(slot), C::TILE);
 #pragma unroll
         for (int kb = 0; kb < C::NKB; ++kb)
-            tma_load_4d(base + C::OFF_V + slot * C::TILE + kb * C::BLK, &p.tm_v[j],
-                        bar(C::bar_vf(slot)), kb * 64, g, row0, b);
-        v_armed[slot] = jt;
+            tma_load_4d(ring + slot * C::TILE + kb * C::BLK, &maps[it.chunk()], bar_full(slot),
+                        kb * 64, g, it.t * kBN, b);
+        armed[slot] = jt;
     }
     // Drain: every copy this thread started must have landed before the CTA exits.
-    wait_drain(bar(C::BAR_Q), 0, abort_flag, lim);
+    if (IS_K) wait_drain(bar(C::BAR_Q), 0, abort_flag, lim);
 #pragma unroll
-    for (int s = 0; s < C::NS; ++s) {
-        if (k_armed[s] >= 0) wait_drain(bar(C::bar_kf(s)), (k_armed[s] / C::NS) & 1, abort_flag, lim);
-        if (v_armed[s] >= 0) wait_drain(bar(C::bar_vf(s)), (v_armed[s] / C::NS) & 1, abort_flag, lim);
-    }
+    for (int s = 0; s < NS; ++s)
+        if (armed[s] >= 0) wait_drain(bar_full(s), (armed[s] / NS) & 1, abort_flag, lim);
 }
 
 template <int D>
@@ -319,15 +319,16 @@ __device__ __forceinline__ void mma_issuer(const AttnParams& p, uint32_t base, u
         tc_commit(bar(C::bar_ke(0)));
         issued = true;
         for (int jt = 0; jt < n; ++jt) {
-            const int slot_v = jt % C::NS;
-            const int slot_k = (jt + 1) % C::NS;
+            const int slot_v = jt % C::NSV;
+            const int slot_k = (jt + 1) % C::NSK;
             const bool more = jt + 1 < n;
-            if (!wait1(bar(C::bar_vf(slot_v)), (jt / C::NS) & 1, abort_flag, lim, kErrMma)) break;
+            if (!wait1(bar(C::bar_vf(slot_v)), (jt / C::NSV) & 1, abort_flag, lim, kErrMma)) break;
             if (!wait1(bar(C::bar_pf(0)), jt & 1, abort_flag, lim, kErrMma)) break;
             tc_fence_after();
             issue_pv(0, slot_v, jt > 0);
             if (more) {
-                if (!wait1(bar(C::bar_kf(slot_k)), ((jt + 1) / C::NS) & 1, abort_flag, lim, kErrMma))
+                if (!wait1(bar(C::bar_kf(slot_k)), ((jt + 1) / C::NSK) & 1, abort_flag, lim,
+                           kErrMma))
                     break;
                 tc_fence_after();
                 issue_s(0, slot_k);
@@ -402,15 +403,17 @@ __device__ __forceinline__ void softmax_wg(const AttnParams& p, uint32_t base, u
             for (int c = 0; c < 128; ++c)
                 if (c >= kvalid || c > lim_c) s[c] = -INFINITY;
         }
-        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+        // row max over all 128 columns: four chains of three-input max, 8 columns per step
+        float mx0 = fmaxf(s[0], s[1]), mx1 = fmaxf(s[2], s[3]);
+        float mx2 = fmaxf(s[4], s[5]), mx3 = fmaxf(s[6], s[7]);
 #pragma unroll
-        for (int c = 4; c < 128; c += 4) {
-            mx0 = fmaxf(mx0, s[c]);
-            mx1 = fmaxf(mx1, s[c + 1]);
-            mx2 = fmaxf(mx2, s[c + 2]);
-            mx3 = fmaxf(mx3, s[c + 3]);
+        for (int c = 8; c < 128; c += 8) {
+            mx0 = fmax3(mx0, s[c], s[c + 1]);
+            mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
+            mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
+            mx3 = fmax3(mx3, s[c + 6], s[c + 7]);
         }
-        const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        const float mx = fmaxf(fmax3(mx0, mx1, mx2), mx3);
         const float m_new = fmaxf(m_run, mx * sl2);
         float alpha = 1.f;
         bool resc = false;
@@ -422,29 +425,41 @@ __device__ __forceinline__ void softmax_wg(const AttnParams& p, uint32_t base, u
             resc = true;
         }
         const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
-        float sum0 = 0.f, sum1 = 0.f, rsum0 = 0.f, rsum1 = 0.f;
         // P = 2^(s*scale*log2e - m) in bf16 pairs, written over the first 64 columns of S
-        // (all of S is already in registers), one 64-key half at a time.
+        // (all of S is already in registers), one 64-key half at a time.  Pairs of columns
+        // go through the packed f32x2 pipe: one FMA and two adds per pair.
+        const uint64_t sl2x2 = f2_pack(sl2, sl2), negm_x2 = f2_pack(neg_m, neg_m);
+        uint64_t sum_a = 0, sum_b = 0, used_a = 0, used_b = 0;  // (0.f, 0.f) pairs
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
             uint32_t pk[32];
 #pragma unroll
             for (int c2 = 0; c2 < 32; ++c2) {
                 const int c = half * 64 + 2 * c2;
-                const float p0 = ex2_approx(fmaf(s[c], sl2, neg_m));
-                const float p1 = ex2_approx(fmaf(s[c + 1], sl2, neg_m));
-                sum0 += p0;
-                sum1 += p1;
+                float x0, x1;
+                f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), sl2x2, negm_x2), x0, x1);
+                const float p0 = ex2_approx(x0);
+                const float p1 = ex2_approx(x1);
                 const uint32_t pp = pack_bf16x2(p0, p1);
                 pk[c2] = pp;
-                // the bf16 values the P.V product actually uses
-                rsum0 += __uint_as_float(pp << 16);
-                rsum1 += __uint_as_float(pp & 0xffff0000u);
+                // fp32 sum (for the LSE) and the sum of the bf16 values P.V actually uses
+                const uint64_t pr = f2_pack(p0, p1);
+                const uint64_t ur = f2_pack(__uint_as_float(pp << 16), __uint_as_float(pp & 0xffff0000u));
+                if (c2 & 1) {
+                    sum_b = f2_add(sum_b, pr);
+                    used_b = f2_add(used_b, ur);
+                } else {
+                    sum_a = f2_add(sum_a, pr);
+                    used_a = f2_add(used_a, ur);
+                }
             }
             tmem_st32(tS + half * 32, pk);
         }
-        l_run = l_run * alpha + (sum0 + sum1);
-        l_used = l_used * alpha + (rsum0 + rsum1);
+        float s0, s1, u0, u1;
+        f2_unpack(f2_add(sum_a, sum_b), s0, s1);
+        f2_unpack(f2_add(used_a, used_b), u0, u1);
+        l_run = l_run * alpha + (s0 + s1);
+        l_used = l_used * alpha + (u0 + u1);
         if (__any_sync(FULL, resc)) {
             // PV of the previous tile is complete: its commit preceded this tile's S commit.
 #pragma unroll
@@ -513,10 +528,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100(const __grid_const
     auto bar = [&](int i) { return base + C::OFF_BAR + 8u * (uint32_t)i; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int BH = p.B * p.H_q;
-    const int bh = blockIdx.x % BH;
-    const int rb = p.n_row_blocks - 1 - (int)(blockIdx.x / BH);  // heaviest row blocks first
-    const int b = bh / p.H_q, h = bh % p.H_q, g = h / p.group;
+    // Grid order: (batch, kv head) outermost, then 256-row blocks heaviest first (the last
+    // rows see the most keys when causal), then the query heads sharing that kv head.  The
+    // CTAs resident at any time then stream the same K/V tiles in near lockstep, so K/V are
+    // read from HBM about once per (batch, kv head) and served from L2 after that.
+    const int per_bg = p.n_row_blocks * p.group;
+    const int bg = (int)(blockIdx.x / per_bg);
+    const int rem = (int)(blockIdx.x % per_bg);
+    const int rb = p.n_row_blocks - 1 - rem / p.group;
+    const int b = bg / p.H_kv, g = bg % p.H_kv;
+    const int h = g * p.group + rem % p.group;
     const int r0 = rb * 2 * kBM;
 
     Sched sched;
@@ -530,9 +551,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100(const __grid_const
 
     if (threadIdx.x == 0) {
         mbar_init(bar(C::BAR_Q), 1);
-        for (int s = 0; s < C::NS; ++s) {
+        for (int s = 0; s < C::NSK; ++s) {
             mbar_init(bar(C::bar_kf(s)), 1);
             mbar_init(bar(C::bar_ke(s)), 1);
+        }
+        for (int s = 0; s < C::NSV; ++s) {
             mbar_init(bar(C::bar_vf(s)), 1);
             mbar_init(bar(C::bar_ve(s)), 1);
         }
@@ -562,7 +585,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100(const __grid_const
     if (warp >= 8) {
         regs_decrease<kRegsOther>();
         if (warp == kWarpLoad) {
-            if (lane == 0) producer<D>(p, base, sched, n, b, h, g, r0, abort_flag);
+            if (lane == 0) producer<D, true>(p, base, sched, n, b, h, g, r0, abort_flag);
+        } else if (warp == kWarpLoadV) {
+            if (lane == 0) producer<D, false>(p, base, sched, n, b, h, g, r0, abort_flag);
         } else if (warp == kWarpMma) {
             if (lane == 0) mma_issuer<D>(p, base, tmem, n, abort_flag);
         }

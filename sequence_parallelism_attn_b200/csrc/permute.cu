@@ -8,10 +8,15 @@
 // source (D * element size contiguous bytes).  The grid is a multiple of the SM count and
 // strides over the output.  HBM-bound: algorithmic bytes = input read once per output
 // byte that needs it + output written once.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include "ra_internal.h"
 #include "permute_index.cuh"
+#include "sm100_ptx.cuh"
 
 namespace ra {
+
+__device__ unsigned int g_permute_error_word = 0;
 
 namespace {
 
@@ -61,6 +66,186 @@ __global__ void __launch_bounds__(256) head2seq_kernel(const int4* __restrict__ 
     }
 }
 
+
+// ---------------------------------------------------------------- TMA bulk-tensor path
+// The sequence-sharded side is viewed as a 4-D tensor of 32-bit words
+//   {W = D*elem/4, H, Lc, P*B}              (token t of rank s, batch b at (.., t, s*B + b))
+// and the head-sharded side as a 5-D tensor
+//   {W, Hl, Lc, P, P*B}                      (rank r, batch b, global token s*Lc + t at
+//                                             (.., t, s, r*B + b))
+// so a box of T tokens never crosses a chunk boundary: loads past Lc read zeros and stores
+// past Lc are clipped.  One thread per CTA runs a ring of NS shared-memory stages: a tiled
+// TMA load fills a stage, a tiled TMA store drains it, and a stage is refilled once the
+// store that read it is done.  Each thread issues a handful of instructions per 32 KB.
+constexpr int kPermStages = 3;
+constexpr int kPermStageBytes = 32 * 1024;
+constexpr int kPermSmem = kPermStages * kPermStageBytes + 128 + 64;
+
+struct __align__(64) PermTmaParams {
+    CUtensorMap src;
+    CUtensorMap dst;
+    int P, B, Lc, Hl, H_in, H_out, T, n_tblk, per_head;
+    int box_bytes;
+    long long n_blocks;
+    unsigned long long wait_limit_ns;
+};
+
+__device__ __forceinline__ bool perm_wait(uint32_t bar, uint32_t parity, unsigned long long limit) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 15u) == 0 && global_timer_ns() - t0 > limit) {
+            atomicOr(&g_permute_error_word, 1u);
+            return false;
+        }
+    }
+}
+
+// MODE 0: seq2head, MODE 1: head2seq
+template <int MODE>
+__global__ void __launch_bounds__(32) permute_tma_kernel(const __grid_constant__ PermTmaParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    if (threadIdx.x != 0) return;
+    uint32_t base = smem_u32(smem_raw);
+    base = (base + 127u) & ~127u;
+    const uint32_t bars = base + kPermStages * kPermStageBytes;
+    for (int i = 0; i < kPermStages; ++i) mbar_init(bars + 8 * i, 1);
+    fence_mbar_init();
+    fence_proxy_async_smem();
+
+    const long long n_my =
+        p.n_blocks > blockIdx.x ? (p.n_blocks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const int nh = p.per_head ? p.Hl : 1;
+
+    // block -> coordinates.  seq2head order: (r, b, s, t-block, head); head2seq: (s, b,
+    // t-block, r), so that consecutive blocks write neighbouring destination bytes.
+    auto issue_load = [&](long long i) {
+        const long long blk = blockIdx.x + i * gridDim.x;
+        const uint32_t stage = base + (uint32_t)(i % kPermStages) * kPermStageBytes;
+        const uint32_t bar = bars + 8 * (uint32_t)(i % kPermStages);
+        mbar_arrive_expect_tx(bar, (uint32_t)p.box_bytes);
+        if (MODE == 0) {
+            long long x = blk;
+            const int hh = (int)(x % nh); x /= nh;
+            const int tb = (int)(x % p.n_tblk); x /= p.n_tblk;
+            const int s = (int)(x % p.P); x /= p.P;
+            const int b = (int)(x % p.B);
+            const int r = (int)(x / p.B);
+            const int h_src = p.per_head ? ((r * p.Hl + hh) * p.H_in) / p.H_out : r * p.Hl;
+            tma_load_4d(stage, &p.src, bar, 0, h_src, tb * p.T, s * p.B + b);
+        } else {
+            long long x = blk;
+            const int r = (int)(x % p.P); x /= p.P;
+            const int tb = (int)(x % p.n_tblk); x /= p.n_tblk;
+            const int b = (int)(x % p.B);
+            const int s = (int)(x / p.B);
+            tma_load_5d(stage, &p.src, bar, 0, 0, tb * p.T, s, r * p.B + b);
+        }
+    };
+    auto issue_store = [&](long long i) {
+        const long long blk = blockIdx.x + i * gridDim.x;
+        const uint32_t stage = base + (uint32_t)(i % kPermStages) * kPermStageBytes;
+        if (MODE == 0) {
+            long long x = blk;
+            const int hh = (int)(x % nh); x /= nh;
+            const int tb = (int)(x % p.n_tblk); x /= p.n_tblk;
+            const int s = (int)(x % p.P); x /= p.P;
+            const int b = (int)(x % p.B);
+            const int r = (int)(x / p.B);
+            tma_store_5d(&p.dst, stage, 0, p.per_head ? hh : 0, tb * p.T, s, r * p.B + b);
+        } else {
+            long long x = blk;
+            const int r = (int)(x % p.P); x /= p.P;
+            const int tb = (int)(x % p.n_tblk); x /= p.n_tblk;
+            const int b = (int)(x % p.B);
+            const int s = (int)(x / p.B);
+            tma_store_4d(&p.dst, stage, 0, r * p.Hl, tb * p.T, s * p.B + b);
+        }
+    };
+
+    long long issued = 0;
+    for (; issued < kPermStages - 1 && issued < n_my; ++issued) issue_load(issued);
+    long long n = 0;
+    for (; n < n_my; ++n) {
+        const uint32_t bar = bars + 8 * (uint32_t)(n % kPermStages);
+        if (!perm_wait(bar, (uint32_t)((n / kPermStages) & 1), p.wait_limit_ns)) break;
+        issue_store(n);
+        bulk_commit();
+        if (issued < n_my) {
+            bulk_wait_read<1>();  // the store that last read stage (issued % NS) is done
+            issue_load(issued);
+            ++issued;
+        }
+    }
+    bulk_wait_all();
+    // loads issued but never consumed (only after a timeout) must land before exit
+    for (long long i = n; i < issued; ++i)
+        perm_wait(bars + 8 * (uint32_t)(i % kPermStages), (uint32_t)((i / kPermStages) & 1),
+                  p.wait_limit_ns);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 perm_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// rank-4 {W, H, Lc, PB} or rank-5 {W, Hl, Lc, P, PB} tensor of 32-bit words
+bool encode_words(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
+                  const uint32_t* box) {
+    auto enc = perm_encode_fn();
+    if (!enc) return false;
+    cuuint64_t d[5], st[4];
+    cuuint32_t bx[5], es[5] = {1, 1, 1, 1, 1};
+    uint64_t stride = 4;
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        bx[i] = box[i];
+        if (i > 0) st[i - 1] = stride;
+        stride *= dims[i];
+    }
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, rank, const_cast<void*>(ptr), d, st, bx, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE>
+cudaError_t launch_perm_tma(const PermTmaParams& p, cudaStream_t s) {
+    static int configured_for = -1;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (configured_for != dev) {
+        e = cudaFuncSetAttribute(permute_tma_kernel<MODE>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kPermSmem);
+        if (e != cudaSuccess) return e;
+        configured_for = dev;
+    }
+    long long grid = (long long)sm_count() * 2;
+    if (grid > p.n_blocks) grid = p.n_blocks;
+    if (grid < 1) grid = 1;
+    permute_tma_kernel<MODE><<<(unsigned)grid, 32, kPermSmem, s>>>(p);
+    return cudaGetLastError();
+}
+
+// TMA path usable: a head segment is at most 256 words (the box limit)
+bool tma_ok(int D, int esize) { return (D * esize) % 16 == 0 && (D * esize) / 4 <= 256; }
+
+int tokens_per_box(int words, int heads_per_box) {
+    int t = kPermStageBytes / (words * 4 * heads_per_box);
+    if (t > 256) t = 256;
+    return t < 1 ? 1 : t;
+}
+
 unsigned grid_for(uint32_t n_groups) {
     const uint32_t per_wave = (uint32_t)sm_count() * 8u;  // 8 resident 256-thread CTAs per SM
     uint32_t blocks = (n_groups + 255u) / 256u;
@@ -71,7 +256,28 @@ unsigned grid_for(uint32_t n_groups) {
 }  // namespace
 
 cudaError_t launch_seq2head(const void* in, void* out, int P, int B, int Lc, int H_in, int H_out,
-                            int D, int esize, cudaStream_t s) {
+                            int D, int esize, cudaStream_t s, unsigned long long wait_limit_ns) {
+    const int Hl = H_out / P;
+    if (tma_ok(D, esize) && Hl <= 256 && Hl * (D * esize) <= kPermStageBytes) {
+        static thread_local PermTmaParams p;
+        const int W = D * esize / 4;
+        p.per_head = H_in != H_out;
+        const int hbox = p.per_head ? 1 : Hl;
+        p.T = tokens_per_box(W, hbox);
+        const uint64_t sdims[4] = {(uint64_t)W, (uint64_t)H_in, (uint64_t)Lc, (uint64_t)P * B};
+        const uint32_t sbox[4] = {(uint32_t)W, (uint32_t)hbox, (uint32_t)p.T, 1};
+        const uint64_t ddims[5] = {(uint64_t)W, (uint64_t)Hl, (uint64_t)Lc, (uint64_t)P,
+                                   (uint64_t)P * B};
+        const uint32_t dbox[5] = {(uint32_t)W, (uint32_t)hbox, (uint32_t)p.T, 1, 1};
+        if (encode_words(&p.src, in, 4, sdims, sbox) && encode_words(&p.dst, out, 5, ddims, dbox)) {
+            p.P = P; p.B = B; p.Lc = Lc; p.Hl = Hl; p.H_in = H_in; p.H_out = H_out;
+            p.n_tblk = (Lc + p.T - 1) / p.T;
+            p.box_bytes = W * 4 * hbox * p.T;
+            p.n_blocks = (long long)P * B * P * p.n_tblk * (p.per_head ? Hl : 1);
+            p.wait_limit_ns = wait_limit_ns;
+            return launch_perm_tma<0>(p, s);
+        }
+    }
     PermuteGeom geo = make_seq2head_geom(P, B, Lc, H_in, H_out, D, esize);
     const uint64_t n_vec = (uint64_t)P * B * P * Lc * (uint64_t)(H_out / P) * geo.VD.div;
     if (geo.VD.div % 4 == 0) {
@@ -87,7 +293,27 @@ cudaError_t launch_seq2head(const void* in, void* out, int P, int B, int Lc, int
 }
 
 cudaError_t launch_head2seq(const void* in, void* out, int P, int B, int Lc, int H, int D,
-                            int esize, cudaStream_t s) {
+                            int esize, cudaStream_t s, unsigned long long wait_limit_ns) {
+    const int Hl = H / P;
+    if (tma_ok(D, esize) && Hl <= 256 && Hl * (D * esize) <= kPermStageBytes) {
+        static thread_local PermTmaParams p;
+        const int W = D * esize / 4;
+        p.per_head = 0;
+        p.T = tokens_per_box(W, Hl);
+        const uint64_t sdims[5] = {(uint64_t)W, (uint64_t)Hl, (uint64_t)Lc, (uint64_t)P,
+                                   (uint64_t)P * B};
+        const uint32_t sbox[5] = {(uint32_t)W, (uint32_t)Hl, (uint32_t)p.T, 1, 1};
+        const uint64_t ddims[4] = {(uint64_t)W, (uint64_t)H, (uint64_t)Lc, (uint64_t)P * B};
+        const uint32_t dbox[4] = {(uint32_t)W, (uint32_t)Hl, (uint32_t)p.T, 1};
+        if (encode_words(&p.src, in, 5, sdims, sbox) && encode_words(&p.dst, out, 4, ddims, dbox)) {
+            p.P = P; p.B = B; p.Lc = Lc; p.Hl = Hl; p.H_in = H; p.H_out = H;
+            p.n_tblk = (Lc + p.T - 1) / p.T;
+            p.box_bytes = W * 4 * Hl * p.T;
+            p.n_blocks = (long long)P * B * p.n_tblk * P;
+            p.wait_limit_ns = wait_limit_ns;
+            return launch_perm_tma<1>(p, s);
+        }
+    }
     PermuteGeom geo = make_head2seq_geom(P, B, Lc, H, D, esize);
     const uint64_t n_vec = (uint64_t)P * B * Lc * (uint64_t)H * geo.VD.div;
     if (geo.VD.div % 4 == 0) {
@@ -100,6 +326,16 @@ cudaError_t launch_head2seq(const void* in, void* out, int P, int B, int Lc, int
                                                               n_groups, geo);
     }
     return cudaGetLastError();
+}
+
+cudaError_t read_and_clear_permute_error(unsigned int* value) {
+    cudaError_t e = cudaMemcpyFromSymbol(value, g_permute_error_word, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    if (*value) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_permute_error_word, &zero, sizeof(unsigned int));
+    }
+    return e;
 }
 
 }  // namespace ra

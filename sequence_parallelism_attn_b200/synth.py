@@ -95,6 +95,8 @@ LONG_128K = AttnWorkload("causal_L131072_H8_D128", B=1, H_q=8, H_kv=8, D=128, P=
                          dtype=torch.bfloat16, causal=True, seed=1004)
 ULYSSES_128K = UlyssesWorkload("ulysses_e2e_L131072", P=8, B=1, Lc=16384, H_q=32, H_kv=4,
                                D=128, dtype=torch.bfloat16, causal=True, seed=1005)
+ULYSSES_32K = UlyssesWorkload("ulysses_e2e_L32768", P=8, B=1, Lc=4096, H_q=32, H_kv=4,
+                              D=128, dtype=torch.bfloat16, causal=True, seed=1006)
 TINY_PERMUTE = UlyssesWorkload("tiny_permute", P=2, B=1, Lc=64, H_q=2, H_kv=2, D=32,
                                dtype=torch.float32, causal=False, seed=1001)
 SMALL_PERMUTE = UlyssesWorkload("small_permute", P=4, B=1, Lc=1024, H_q=8, H_kv=8, D=64,

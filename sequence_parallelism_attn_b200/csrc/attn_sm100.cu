@@ -58,7 +58,7 @@ __device__ unsigned int g_ra_error_word = 0;
 namespace {
 
 constexpr int kThreads = 384;
-constexpr uint32_t kRegsSoftmax = 208, kRegsOther = 88;
+constexpr uint32_t kRegsSoftmax = 200, kRegsOther = 104;
 constexpr int kWarpLoad = 8;
 constexpr int kWarpMma = 9;
 constexpr int kWarpLoadV = 10;
@@ -322,15 +322,16 @@ __device__ __forceinline__ void mma_issuer(const AttnParams& p, uint32_t base, u
             const int slot_v = jt % C::NSV;
             const int slot_k = (jt + 1) % C::NSK;
             const bool more = jt + 1 < n;
+            // V(j) and K(j+1) are awaited before P_A(j): the loads have long landed by then,
+            // so the waits cost nothing on the path from P_A(j) to S_A(j+1).
             if (!wait1(bar(C::bar_vf(slot_v)), (jt / C::NSV) & 1, abort_flag, lim, kErrMma)) break;
+            if (more && !wait1(bar(C::bar_kf(slot_k)), ((jt + 1) / C::NSK) & 1, abort_flag, lim,
+                               kErrMma))
+                break;
             if (!wait1(bar(C::bar_pf(0)), jt & 1, abort_flag, lim, kErrMma)) break;
             tc_fence_after();
             issue_pv(0, slot_v, jt > 0);
             if (more) {
-                if (!wait1(bar(C::bar_kf(slot_k)), ((jt + 1) / C::NSK) & 1, abort_flag, lim,
-                           kErrMma))
-                    break;
-                tc_fence_after();
                 issue_s(0, slot_k);
                 tc_commit(bar(C::bar_sf(0)));
             } else {
@@ -386,13 +387,8 @@ __device__ __forceinline__ void softmax_wg(const AttnParams& p, uint32_t base, u
         }
         __syncwarp();
         tc_fence_after();
-        uint32_t sr[4][32];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, sr[q]);
-        tmem_wait_ld();
-        float s[128];
-#pragma unroll
-        for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c / 32][c % 32]);
+        uint64_t s2[64];  // the row's 128 scores as pairs (2i, 2i+1)
+        tmem_ld128_pairs(tS, s2);
 
         const long long k0 = (long long)it.chunk() * p.Lc + (long long)it.t * kBN;
         const int kvalid = min(kBN, p.Lc - it.t * kBN);
@@ -400,18 +396,29 @@ __device__ __forceinline__ void softmax_wg(const AttnParams& p, uint32_t base, u
         if (need_mask) {
             const long long lim_c = p.causal ? my_row - k0 : (long long)kBN;  // keys c <= lim_c
 #pragma unroll
-            for (int c = 0; c < 128; ++c)
-                if (c >= kvalid || c > lim_c) s[c] = -INFINITY;
+            for (int i = 0; i < 64; ++i) {
+                float a, b;
+                f2_unpack(s2[i], a, b);
+                if (2 * i >= kvalid || 2 * i > lim_c) a = -INFINITY;
+                if (2 * i + 1 >= kvalid || 2 * i + 1 > lim_c) b = -INFINITY;
+                s2[i] = f2_pack(a, b);
+            }
         }
         // row max over all 128 columns: four chains of three-input max, 8 columns per step
-        float mx0 = fmaxf(s[0], s[1]), mx1 = fmaxf(s[2], s[3]);
-        float mx2 = fmaxf(s[4], s[5]), mx3 = fmaxf(s[6], s[7]);
+        float mx0, mx1, mx2, mx3;
+        {
+            float a, b;
+            f2_unpack(s2[0], a, b); mx0 = fmaxf(a, b);
+            f2_unpack(s2[1], a, b); mx1 = fmaxf(a, b);
+            f2_unpack(s2[2], a, b); mx2 = fmaxf(a, b);
+            f2_unpack(s2[3], a, b); mx3 = fmaxf(a, b);
 #pragma unroll
-        for (int c = 8; c < 128; c += 8) {
-            mx0 = fmax3(mx0, s[c], s[c + 1]);
-            mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
-            mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
-            mx3 = fmax3(mx3, s[c + 6], s[c + 7]);
+            for (int i = 4; i < 64; i += 4) {
+                f2_unpack(s2[i], a, b); mx0 = fmax3(mx0, a, b);
+                f2_unpack(s2[i + 1], a, b); mx1 = fmax3(mx1, a, b);
+                f2_unpack(s2[i + 2], a, b); mx2 = fmax3(mx2, a, b);
+                f2_unpack(s2[i + 3], a, b); mx3 = fmax3(mx3, a, b);
+            }
         }
         const float mx = fmaxf(fmax3(mx0, mx1, mx2), mx3);
         const float m_new = fmaxf(m_run, mx * sl2);
@@ -426,8 +433,7 @@ __device__ __forceinline__ void softmax_wg(const AttnParams& p, uint32_t base, u
         }
         const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
         // P = 2^(s*scale*log2e - m) in bf16 pairs, written over the first 64 columns of S
-        // (all of S is already in registers), one 64-key half at a time.  Pairs of columns
-        // go through the packed f32x2 pipe: one FMA and two adds per pair.
+        // (all of S is already in registers), one 64-key half at a time.
         const uint64_t sl2x2 = f2_pack(sl2, sl2), negm_x2 = f2_pack(neg_m, neg_m);
         uint64_t sum_a = 0, sum_b = 0, used_a = 0, used_b = 0;  // (0.f, 0.f) pairs
 #pragma unroll
@@ -435,23 +441,10 @@ __device__ __forceinline__ void softmax_wg(const AttnParams& p, uint32_t base, u
             uint32_t pk[32];
 #pragma unroll
             for (int c2 = 0; c2 < 32; ++c2) {
-                const int c = half * 64 + 2 * c2;
-                float x0, x1;
-                f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), sl2x2, negm_x2), x0, x1);
-                const float p0 = ex2_approx(x0);
-                const float p1 = ex2_approx(x1);
-                const uint32_t pp = pack_bf16x2(p0, p1);
-                pk[c2] = pp;
-                // fp32 sum (for the LSE) and the sum of the bf16 values P.V actually uses
-                const uint64_t pr = f2_pack(p0, p1);
-                const uint64_t ur = f2_pack(__uint_as_float(pp << 16), __uint_as_float(pp & 0xffff0000u));
-                if (c2 & 1) {
-                    sum_b = f2_add(sum_b, pr);
-                    used_b = f2_add(used_b, ur);
-                } else {
-                    sum_a = f2_add(sum_a, pr);
-                    used_a = f2_add(used_a, ur);
-                }
+                if (c2 & 1)
+                    pk[c2] = softmax_pair(s2[half * 32 + c2], sl2x2, negm_x2, sum_b, used_b);
+                else
+                    pk[c2] = softmax_pair(s2[half * 32 + c2], sl2x2, negm_x2, sum_a, used_a);
             }
             tmem_st32(tS + half * 32, pk);
         }

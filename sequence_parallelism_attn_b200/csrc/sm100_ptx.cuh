@@ -179,6 +179,112 @@ __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+
+// All 128 fp32 columns of this thread's TMEM lane as 64 register pairs (column 2i in the
+// low half of pair i), loaded and waited for in one block so that every pair is an
+// aligned 64-bit register ready for the packed f32x2 instructions.
+__device__ __forceinline__ void tmem_ld128_pairs(uint32_t taddr, uint64_t (&o)[64]) {
+    asm volatile(
+        "{\n\t.reg .b32 r0, r1, r2, r3, r4, r5, r6, r7, r8, r9, r10, r11, r12, r13, r14, r15, r16, r17, r18, r19, r20, r21, r22, r23, r24, r25, r26, r27, r28, r29, r30, r31, r32, r33, r34, r35, r36, r37, r38, r39, r40, r41, r42, r43, r44, r45, r46, r47, r48, r49, r50, r51, r52, r53, r54, r55, r56, r57, r58, r59, r60, r61, r62, r63, r64, r65, r66, r67, r68, r69, r70, r71, r72, r73, r74, r75, r76, r77, r78, r79, r80, r81, r82, r83, r84, r85, r86, r87, r88, r89, r90, r91, r92, r93, r94, r95, r96, r97, r98, r99, r100, r101, r102, r103, r104, r105, r106, r107, r108, r109, r110, r111, r112, r113, r114, r115, r116, r117, r118, r119, r120, r121, r122, r123, r124, r125, r126, r127;\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {r0, r1, r2, r3, r4, r5, r6, r7, r8, r9, r10, r11, r12, r13, r14, r15, r16, r17, r18, r19, r20, r21, r22, r23, r24, r25, r26, r27, r28, r29, r30, r31}, [%64];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {r32, r33, r34, r35, r36, r37, r38, r39, r40, r41, r42, r43, r44, r45, r46, r47, r48, r49, r50, r51, r52, r53, r54, r55, r56, r57, r58, r59, r60, r61, r62, r63}, [%65];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {r64, r65, r66, r67, r68, r69, r70, r71, r72, r73, r74, r75, r76, r77, r78, r79, r80, r81, r82, r83, r84, r85, r86, r87, r88, r89, r90, r91, r92, r93, r94, r95}, [%66];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {r96, r97, r98, r99, r100, r101, r102, r103, r104, r105, r106, r107, r108, r109, r110, r111, r112, r113, r114, r115, r116, r117, r118, r119, r120, r121, r122, r123, r124, r125, r126, r127}, [%67];\n\t"
+        "tcgen05.wait::ld.sync.aligned;\n\t"
+        "mov.b64 %0, {r0, r1};\n\t"
+        "mov.b64 %1, {r2, r3};\n\t"
+        "mov.b64 %2, {r4, r5};\n\t"
+        "mov.b64 %3, {r6, r7};\n\t"
+        "mov.b64 %4, {r8, r9};\n\t"
+        "mov.b64 %5, {r10, r11};\n\t"
+        "mov.b64 %6, {r12, r13};\n\t"
+        "mov.b64 %7, {r14, r15};\n\t"
+        "mov.b64 %8, {r16, r17};\n\t"
+        "mov.b64 %9, {r18, r19};\n\t"
+        "mov.b64 %10, {r20, r21};\n\t"
+        "mov.b64 %11, {r22, r23};\n\t"
+        "mov.b64 %12, {r24, r25};\n\t"
+        "mov.b64 %13, {r26, r27};\n\t"
+        "mov.b64 %14, {r28, r29};\n\t"
+        "mov.b64 %15, {r30, r31};\n\t"
+        "mov.b64 %16, {r32, r33};\n\t"
+        "mov.b64 %17, {r34, r35};\n\t"
+        "mov.b64 %18, {r36, r37};\n\t"
+        "mov.b64 %19, {r38, r39};\n\t"
+        "mov.b64 %20, {r40, r41};\n\t"
+        "mov.b64 %21, {r42, r43};\n\t"
+        "mov.b64 %22, {r44, r45};\n\t"
+        "mov.b64 %23, {r46, r47};\n\t"
+        "mov.b64 %24, {r48, r49};\n\t"
+        "mov.b64 %25, {r50, r51};\n\t"
+        "mov.b64 %26, {r52, r53};\n\t"
+        "mov.b64 %27, {r54, r55};\n\t"
+        "mov.b64 %28, {r56, r57};\n\t"
+        "mov.b64 %29, {r58, r59};\n\t"
+        "mov.b64 %30, {r60, r61};\n\t"
+        "mov.b64 %31, {r62, r63};\n\t"
+        "mov.b64 %32, {r64, r65};\n\t"
+        "mov.b64 %33, {r66, r67};\n\t"
+        "mov.b64 %34, {r68, r69};\n\t"
+        "mov.b64 %35, {r70, r71};\n\t"
+        "mov.b64 %36, {r72, r73};\n\t"
+        "mov.b64 %37, {r74, r75};\n\t"
+        "mov.b64 %38, {r76, r77};\n\t"
+        "mov.b64 %39, {r78, r79};\n\t"
+        "mov.b64 %40, {r80, r81};\n\t"
+        "mov.b64 %41, {r82, r83};\n\t"
+        "mov.b64 %42, {r84, r85};\n\t"
+        "mov.b64 %43, {r86, r87};\n\t"
+        "mov.b64 %44, {r88, r89};\n\t"
+        "mov.b64 %45, {r90, r91};\n\t"
+        "mov.b64 %46, {r92, r93};\n\t"
+        "mov.b64 %47, {r94, r95};\n\t"
+        "mov.b64 %48, {r96, r97};\n\t"
+        "mov.b64 %49, {r98, r99};\n\t"
+        "mov.b64 %50, {r100, r101};\n\t"
+        "mov.b64 %51, {r102, r103};\n\t"
+        "mov.b64 %52, {r104, r105};\n\t"
+        "mov.b64 %53, {r106, r107};\n\t"
+        "mov.b64 %54, {r108, r109};\n\t"
+        "mov.b64 %55, {r110, r111};\n\t"
+        "mov.b64 %56, {r112, r113};\n\t"
+        "mov.b64 %57, {r114, r115};\n\t"
+        "mov.b64 %58, {r116, r117};\n\t"
+        "mov.b64 %59, {r118, r119};\n\t"
+        "mov.b64 %60, {r120, r121};\n\t"
+        "mov.b64 %61, {r122, r123};\n\t"
+        "mov.b64 %62, {r124, r125};\n\t"
+        "mov.b64 %63, {r126, r127};\n\t"
+        "}"
+        : "=l"(o[0]), "=l"(o[1]), "=l"(o[2]), "=l"(o[3]), "=l"(o[4]), "=l"(o[5]), "=l"(o[6]), "=l"(o[7]), "=l"(o[8]), "=l"(o[9]), "=l"(o[10]), "=l"(o[11]), "=l"(o[12]), "=l"(o[13]), "=l"(o[14]), "=l"(o[15]), "=l"(o[16]), "=l"(o[17]), "=l"(o[18]), "=l"(o[19]), "=l"(o[20]), "=l"(o[21]), "=l"(o[22]), "=l"(o[23]), "=l"(o[24]), "=l"(o[25]), "=l"(o[26]), "=l"(o[27]), "=l"(o[28]), "=l"(o[29]), "=l"(o[30]), "=l"(o[31]), "=l"(o[32]), "=l"(o[33]), "=l"(o[34]), "=l"(o[35]), "=l"(o[36]), "=l"(o[37]), "=l"(o[38]), "=l"(o[39]), "=l"(o[40]), "=l"(o[41]), "=l"(o[42]), "=l"(o[43]), "=l"(o[44]), "=l"(o[45]), "=l"(o[46]), "=l"(o[47]), "=l"(o[48]), "=l"(o[49]), "=l"(o[50]), "=l"(o[51]), "=l"(o[52]), "=l"(o[53]), "=l"(o[54]), "=l"(o[55]), "=l"(o[56]), "=l"(o[57]), "=l"(o[58]), "=l"(o[59]), "=l"(o[60]), "=l"(o[61]), "=l"(o[62]), "=l"(o[63])
+        : "r"(taddr), "r"(taddr + 32), "r"(taddr + 64), "r"(taddr + 96)
+        : "memory");
+}
+
+// One column pair of the softmax: x = s * scale_log2 - m (packed), p = 2^x (two MUFU ops),
+// pp = bf16x2(p) (the P.V operand), sum += p (fp32, packed) and used += (float)pp (the
+// bf16 values as used, packed).  All pair traffic stays in 64-bit registers.
+__device__ __forceinline__ uint32_t softmax_pair(uint64_t s2, uint64_t scale2, uint64_t negm2,
+                                                 uint64_t& sum, uint64_t& used) {
+    uint32_t pp;
+    asm("{\n\t.reg .b32 x0, x1, p0, p1, lo, hi;\n\t.reg .b64 x, p, u;\n\t"
+        "fma.rn.f32x2 x, %3, %4, %5;\n\t"
+        "mov.b64 {x0, x1}, x;\n\t"
+        "ex2.approx.ftz.f32 p0, x0;\n\t"
+        "ex2.approx.ftz.f32 p1, x1;\n\t"
+        "cvt.rn.bf16x2.f32 %0, p1, p0;\n\t"
+        "mov.b64 p, {p0, p1};\n\t"
+        "add.rn.f32x2 %1, %1, p;\n\t"
+        "shl.b32 lo, %0, 16;\n\t"
+        "and.b32 hi, %0, -65536;\n\t"
+        "mov.b64 u, {lo, hi};\n\t"
+        "add.rn.f32x2 %2, %2, u;\n\t}"
+        : "=r"(pp), "+l"(sum), "+l"(used)
+        : "l"(s2), "l"(scale2), "l"(negm2));
+    return pp;
+}
+
+
 // ------------------------------------------------------------------ register split
 // Per-warpgroup register budget change (all 4 warps of the warpgroup execute it).  The
 // sum over the block must stay within what the block was launched with.

@@ -116,7 +116,6 @@ __global__ void __launch_bounds__(32) permute_tma_kernel(const __grid_constant__
 
     const long long n_my =
         p.n_blocks > blockIdx.x ? (p.n_blocks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    const int nh = p.per_head ? p.Hl : 1;
 
     // block -> coordinates.  seq2head order: (r, b, s, t-block, head); head2seq: (s, b,
     // t-block, r), so that consecutive blocks write neighbouring destination bytes.
@@ -125,15 +124,22 @@ __global__ void __launch_bounds__(32) permute_tma_kernel(const __grid_constant__
         const uint32_t stage = base + (uint32_t)(i % kPermStages) * kPermStageBytes;
         const uint32_t bar = bars + 8 * (uint32_t)(i % kPermStages);
         mbar_arrive_expect_tx(bar, (uint32_t)p.box_bytes);
-        if (MODE == 0) {
+        if (MODE == 0 && p.per_head) {
+            // GQA copy: one block per (source head, rank s, batch, token block); the
+            // source box is read once and stored to every replica of that head.
             long long x = blk;
-            const int hh = (int)(x % nh); x /= nh;
+            const int tb = (int)(x % p.n_tblk); x /= p.n_tblk;
+            const int s = (int)(x % p.P); x /= p.P;
+            const int b = (int)(x % p.B);
+            const int hs = (int)(x / p.B);
+            tma_load_4d(stage, &p.src, bar, 0, hs, tb * p.T, s * p.B + b);
+        } else if (MODE == 0) {
+            long long x = blk;
             const int tb = (int)(x % p.n_tblk); x /= p.n_tblk;
             const int s = (int)(x % p.P); x /= p.P;
             const int b = (int)(x % p.B);
             const int r = (int)(x / p.B);
-            const int h_src = p.per_head ? ((r * p.Hl + hh) * p.H_in) / p.H_out : r * p.Hl;
-            tma_load_4d(stage, &p.src, bar, 0, h_src, tb * p.T, s * p.B + b);
+            tma_load_4d(stage, &p.src, bar, 0, r * p.Hl, tb * p.T, s * p.B + b);
         } else {
             long long x = blk;
             const int r = (int)(x % p.P); x /= p.P;
@@ -146,14 +152,26 @@ __global__ void __launch_bounds__(32) permute_tma_kernel(const __grid_constant__
     auto issue_store = [&](long long i) {
         const long long blk = blockIdx.x + i * gridDim.x;
         const uint32_t stage = base + (uint32_t)(i % kPermStages) * kPermStageBytes;
-        if (MODE == 0) {
+        if (MODE == 0 && p.per_head) {
             long long x = blk;
-            const int hh = (int)(x % nh); x /= nh;
+            const int tb = (int)(x % p.n_tblk); x /= p.n_tblk;
+            const int s = (int)(x % p.P); x /= p.P;
+            const int b = (int)(x % p.B);
+            const int hs = (int)(x / p.B);
+            // replicas j = hs*rep .. hs*rep+rep-1 of the H_out heads copy source head hs
+            const int rep = p.H_out / p.H_in;
+            for (int jr = 0; jr < rep; ++jr) {
+                const int j = hs * rep + jr;
+                const int r = j / p.Hl, hh = j % p.Hl;
+                tma_store_5d(&p.dst, stage, 0, hh, tb * p.T, s, r * p.B + b);
+            }
+        } else if (MODE == 0) {
+            long long x = blk;
             const int tb = (int)(x % p.n_tblk); x /= p.n_tblk;
             const int s = (int)(x % p.P); x /= p.P;
             const int b = (int)(x % p.B);
             const int r = (int)(x / p.B);
-            tma_store_5d(&p.dst, stage, 0, p.per_head ? hh : 0, tb * p.T, s, r * p.B + b);
+            tma_store_5d(&p.dst, stage, 0, 0, tb * p.T, s, r * p.B + b);
         } else {
             long long x = blk;
             const int r = (int)(x % p.P); x /= p.P;
@@ -273,7 +291,8 @@ cudaError_t launch_seq2head(const void* in, void* out, int P, int B, int Lc, int
             p.P = P; p.B = B; p.Lc = Lc; p.Hl = Hl; p.H_in = H_in; p.H_out = H_out;
             p.n_tblk = (Lc + p.T - 1) / p.T;
             p.box_bytes = W * 4 * hbox * p.T;
-            p.n_blocks = (long long)P * B * P * p.n_tblk * (p.per_head ? Hl : 1);
+            // per_head: one block per source head (its replicas are stored from one load)
+            p.n_blocks = (long long)(p.per_head ? H_in : P) * B * P * p.n_tblk;
             p.wait_limit_ns = wait_limit_ns;
             return launch_perm_tma<0>(p, s);
         }

@@ -25,8 +25,8 @@
 //   warp 10    TMA producer of the V tiles (NSV-deep ring)
 //   warp 11    idle (it completes the third warpgroup for the register split)
 // Registers: launched at 168 per thread (3 warps per SM sub-partition); the softmax
-// warpgroups raise their budget to 216 and the third warpgroup drops to 72
-// (216 + 216 + 72 = 504 <= 512 per sub-partition; 256*216 + 128*72 = 384*168).
+// warpgroups raise their budget to 192 and the third warpgroup drops to 120
+// (192 + 192 + 120 = 504 <= 512 per sub-partition; 256*192 + 128*120 = 384*168).
 // Tensor memory (512 columns x 128 lanes x 32 bit):
 //   S_A [0,128) S_B [128,256) fp32 scores; P_A/P_B (bf16 probabilities) overwrite the
 //   first 64 columns of S_A/S_B; O_A at 256, O_B at 256+D (fp32 accumulators).
@@ -58,7 +58,7 @@ __device__ unsigned int g_ra_error_word = 0;
 namespace {
 
 constexpr int kThreads = 384;
-constexpr uint32_t kRegsSoftmax = 200, kRegsOther = 104;
+constexpr uint32_t kRegsSoftmax = 192, kRegsOther = 120;
 constexpr int kWarpLoad = 8;
 constexpr int kWarpMma = 9;
 constexpr int kWarpLoadV = 10;
@@ -138,28 +138,34 @@ struct Sched {
     }
 };
 
+// Walks the schedule tile by tile; the chunk index is recomputed only when the step s
+// changes, so a tile costs no integer division.
 struct SchedIter {
     const Sched* S;
-    int s, t, nt;
+    int s, t, nt, j;
     __device__ void begin(const Sched* sched) {
         S = sched;
         s = 0;
         t = 0;
-        nt = S->tiles_in(S->chunk_at(0));
+        j = S->chunk_at(0);
+        nt = S->tiles_in(j);
         skip_empty();
     }
     __device__ void skip_empty() {
         while (s < S->P && t >= nt) {
             ++s;
             t = 0;
-            if (s < S->P) nt = S->tiles_in(S->chunk_at(s));
+            if (s < S->P) {
+                j = S->chunk_at(s);
+                nt = S->tiles_in(j);
+            }
         }
     }
     __device__ void next() {
         ++t;
         skip_empty();
     }
-    __device__ int chunk() const { return S->chunk_at(s); }
+    __device__ int chunk() const { return j; }
 };
 
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag, unsigned code) {

@@ -263,11 +263,12 @@ __device__ __forceinline__ void tmem_ld128_pairs(uint32_t taddr, uint64_t (&o)[6
 
 // One column pair of the softmax: x = s * scale_log2 - m (packed), p = 2^x (two MUFU ops),
 // pp = bf16x2(p) (the P.V operand), sum += p (fp32, packed) and used += (float)pp (the
-// bf16 values as used, packed).  All pair traffic stays in 64-bit registers.
+// bf16 values as used, each added to its fp32 lane by a mixed-precision add).  All pair
+// traffic stays in 64-bit registers.
 __device__ __forceinline__ uint32_t softmax_pair(uint64_t s2, uint64_t scale2, uint64_t negm2,
                                                  uint64_t& sum, uint64_t& used) {
     uint32_t pp;
-    asm("{\n\t.reg .b32 x0, x1, p0, p1, lo, hi;\n\t.reg .b64 x, p, u;\n\t"
+    asm("{\n\t.reg .b32 x0, x1, p0, p1, u0, u1;\n\t.reg .b16 h0, h1;\n\t.reg .b64 x, p;\n\t"
         "fma.rn.f32x2 x, %3, %4, %5;\n\t"
         "mov.b64 {x0, x1}, x;\n\t"
         "ex2.approx.ftz.f32 p0, x0;\n\t"
@@ -275,10 +276,11 @@ __device__ __forceinline__ uint32_t softmax_pair(uint64_t s2, uint64_t scale2, u
         "cvt.rn.bf16x2.f32 %0, p1, p0;\n\t"
         "mov.b64 p, {p0, p1};\n\t"
         "add.rn.f32x2 %1, %1, p;\n\t"
-        "shl.b32 lo, %0, 16;\n\t"
-        "and.b32 hi, %0, -65536;\n\t"
-        "mov.b64 u, {lo, hi};\n\t"
-        "add.rn.f32x2 %2, %2, u;\n\t}"
+        "mov.b32 {h0, h1}, %0;\n\t"
+        "mov.b64 {u0, u1}, %2;\n\t"
+        "add.rn.f32.bf16 u0, h0, u0;\n\t"
+        "add.rn.f32.bf16 u1, h1, u1;\n\t"
+        "mov.b64 %2, {u0, u1};\n\t}"
         : "=r"(pp), "+l"(sum), "+l"(used)
         : "l"(s2), "l"(scale2), "l"(negm2));
     return pp;

@@ -107,6 +107,37 @@ def test_bf16_output(ra_lib, oracle_mod):
     assert max_abs(f64(l), want_l) <= 1e-3
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_padded_batch_strides(ra_lib, oracle_mod, dtype):
+    """q_bstride and kv_bstride above the dense size: each batch of Q and of every K/V chunk
+    is followed by padding rows filled with NaN, which must never be read."""
+    w = wl(f"padded_{dtype}", B=2, H_q=4, H_kv=2, D=128, P=3, Lc=200, causal=True,
+           dtype=dtype, q_mult=2.0)
+    q, k, v = synth.attention_inputs(w)
+    L, pad_q, pad_kv = w.L, 37, 19
+    qp = torch.full((w.B, L + pad_q, w.H_q, w.D), float("nan"), dtype=dtype, device="cuda")
+    qp[:, :L] = q.cuda()
+    kp = torch.full((w.P, w.B, w.Lc + pad_kv, w.H_kv, w.D), float("nan"), dtype=dtype,
+                    device="cuda")
+    vp = kp.clone()
+    kp[:, :, :w.Lc] = k.cuda()
+    vp[:, :, :w.Lc] = v.cuda()
+    out = torch.empty((w.B, L, w.H_q, w.D), dtype=torch.float32, device="cuda")
+    lse = torch.empty((w.B, w.H_q, L), dtype=torch.float32, device="cuda")
+    in_dt = ra_lib.RA_BF16 if dtype == torch.bfloat16 else ra_lib.RA_FP32
+    ra_lib.ra_ring_attn_fwd(qp.data_ptr(), [kp[j].data_ptr() for j in range(w.P)],
+                            [vp[j].data_ptr() for j in range(w.P)], w.P, w.B, w.H_q, w.H_kv,
+                            w.Lc, w.D, (L + pad_q) * w.H_q * w.D,
+                            (w.Lc + pad_kv) * w.H_kv * w.D, w.scale, 1, in_dt, ra_lib.RA_FP32,
+                            out.data_ptr(), lse.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    assert ra_lib.ra_sync_status() == 0, ra_lib.ra_last_error()
+    want_o, want_l = oracle_mod.ring_attention(f64(q), f64(k), f64(v), w.scale, True)
+    tol_o, tol_l = TOL[dtype]
+    eo, el = max_abs(f64(out), want_o), max_abs(f64(lse), want_l)
+    print(f"[parity] {w.name}: max|dO|={eo:.3e} max|dLSE|={el:.3e}")
+    assert eo <= tol_o and el <= tol_l
+
+
 # ---------------------------------------------------------------- fp32 path
 def test_tiny_fp32_workload_every_row(ra_lib, oracle_mod):
     """B=1, H=2, D=32, 2 ranks x 64 tokens, fp32, non-causal."""

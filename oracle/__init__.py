@@ -49,13 +49,14 @@ def _load():
     lib.ora_attention.argtypes = [P, P, P, i32, i64, i32, i32, i32, f64, i32, P, P, i32]
     lib.ora_attention_rows.argtypes = [P, P, P, P, i64, P, P, i32, i64, i32, i32, i32, f64, i32,
                                        P, P, i32]
-    lib.ora_ring_attention.argtypes = [P, P, P, i32, i32, i64, i32, i32, i32, f64, i32, P, P, P,
+    lib.ora_ring_attention.argtypes = [P, P, P, i32, i32, i64, i32, i32, i32, f64, i32, P, P, P, P,
                                        i32]
     lib.ora_lse_merge.argtypes = [P, P, P, P, i32, i32, i64, i32]
     lib.ora_seq2head.argtypes = [P, P, i32, i32, i64, i32, i32, i32, i32]
     lib.ora_head2seq.argtypes = [P, P, i32, i32, i64, i32, i32, i32]
+    lib.ora_zigzag_positions.argtypes = [i32, i64, P]
     for f in ("ora_attention", "ora_attention_rows", "ora_ring_attention", "ora_lse_merge",
-              "ora_seq2head", "ora_head2seq"):
+              "ora_seq2head", "ora_head2seq", "ora_zigzag_positions"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -112,10 +113,12 @@ def attention_rows(q_rows, rb, rt, rh, k, v, H_q: int, scale: float, causal: boo
 
 
 def ring_attention(q, k_chunks, v_chunks, scale: float, causal: bool, step_offset=None,
-                   nthreads: int = 0):
+                   positions=None, nthreads: int = 0):
     """Ring form.  q [B,P*Lc,H_q,D]; k_chunks/v_chunks [P,B,Lc,H_kv,D] -> (out, lse).
 
-    Rank i visits chunk (i - step_offset[s]) mod P at step s (default: ring order s)."""
+    Rank i visits chunk (i - step_offset[s]) mod P at step s (default: ring order s).
+    positions [P*Lc]: sequence position of each rank-major token (default: contiguous,
+    position = index); the causal mask compares positions."""
     q, kc, vc = _f64(q), _f64(k_chunks), _f64(v_chunks)
     P, B, Lc, H_kv, D = kc.shape
     H_q = q.shape[2]
@@ -124,14 +127,34 @@ def ring_attention(q, k_chunks, v_chunks, scale: float, causal: bool, step_offse
     if step_offset is not None:
         so = np.ascontiguousarray(step_offset, dtype=np.int32)
         assert so.shape == (P,)
+    pos = None
+    if positions is not None:
+        pos = np.ascontiguousarray(positions, dtype=np.int64)
+        assert pos.shape == (P * Lc,)
     out = np.empty((B, P * Lc, H_q, D), np.float64)
     lse = np.empty((B, H_q, P * Lc), np.float64)
     rc = _load().ora_ring_attention(_ptr(q), _ptr(kc), _ptr(vc), P, B, Lc, H_q, H_kv, D,
                                     float(scale), int(bool(causal)),
-                                    _ptr(so) if so is not None else None, _ptr(out), _ptr(lse),
+                                    _ptr(so) if so is not None else None,
+                                    _ptr(pos) if pos is not None else None, _ptr(out), _ptr(lse),
                                     nthreads)
     _check(rc, "ring_attention")
     return out, lse
+
+
+def zigzag_positions(P: int, Lc: int) -> np.ndarray:
+    """Sequence position of each rank-major token in the zigzag layout: rank i holds
+    segment i and segment 2P-1-i of the 2P segments of Lc/2 tokens ([P*Lc] int64)."""
+    pos = np.empty((P * Lc,), np.int64)
+    _check(_load().ora_zigzag_positions(P, Lc, _ptr(pos)), "zigzag_positions")
+    return pos
+
+
+def ring_attention_zigzag(q, k_chunks, v_chunks, scale: float, causal: bool, nthreads: int = 0):
+    """The ring form over shards in the zigzag layout (see zigzag_positions)."""
+    P, _, Lc = np.shape(k_chunks)[:3]
+    return ring_attention(q, k_chunks, v_chunks, scale, causal,
+                          positions=zigzag_positions(P, Lc), nthreads=nthreads)
 
 
 def lse_merge(o_a, lse_a, o_b, lse_b):

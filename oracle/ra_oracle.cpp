@@ -32,6 +32,9 @@
 //   * causal masking, absent from the pages, is the global mask over the
 //     concatenation of chunks in rank order, key position <= query position;
 //   * GQA: query head h reads kv head h / (H_q / H_kv);
+//   * the zigzag layout, only named in [ULYSSES] (introduction), is 2P segments of
+//     Lc/2 tokens with rank i holding segment i then segment 2P-1-i; the causal mask
+//     compares sequence positions, not rank-major indices;
 //   * Ulysses rank r receives the contiguous head block [r*H/P, (r+1)*H/P),
 //     the global sequence is source-rank-major, and KV replica j of H_out is
 //     source head floor(j * H_in / H_out).
@@ -200,11 +203,17 @@ int ora_attention_rows(const double* q_rows, const int* rb, const long long* rt,
 // s = 0..P-1, to the chunk j = (i - step_offset[s]) mod P, and each partial is
 // merged into the running result.  step_offset == NULL means the ring order
 // step_offset[s] = s.  Any permutation of 0..P-1 gives another visiting order.
+// `pos` gives the global sequence position of each of the P*Lc tokens in rank-major
+// order (rank j's shard is tokens j*Lc .. j*Lc+Lc-1 of q and chunk j of k/v); the causal
+// mask is pos[key] <= pos[query].  pos == NULL is the contiguous layout of [SP-QA]
+// section 2 (pos[t] = t); any permutation of 0..P*Lc-1 is another assignment of
+// sequence positions to shards (the zigzag layout is one, see ora_zigzag_positions).
 //   q  [B][P*Lc][H_q][D]    k, v [P][B][Lc][H_kv][D] (chunk j = rank j's K/V)
 //   out [B][P*Lc][H_q][D]   lse [B][H_q][P*Lc]
 int ora_ring_attention(const double* q, const double* k_chunks, const double* v_chunks, int P,
                        int B, long long Lc, int H_q, int H_kv, int D, double scale, int causal,
-                       const int* step_offset, double* out, double* lse, int nthreads) {
+                       const int* step_offset, const long long* pos, double* out, double* lse,
+                       int nthreads) {
     if (P < 1 || B < 1 || Lc < 1 || H_q < 1 || H_kv < 1 || D < 1 || H_q % H_kv != 0) return 1;
     if (step_offset) {
         std::vector<int> seen(P, 0);
@@ -214,6 +223,14 @@ int ora_ring_attention(const double* q, const double* k_chunks, const double* v_
         }
     }
     const long long L = (long long)P * Lc;
+    if (pos) {
+        std::vector<char> seen(L, 0);
+        for (long long t = 0; t < L; ++t) {
+            if (pos[t] < 0 || pos[t] >= L || seen[pos[t]]) return 1;
+            seen[pos[t]] = 1;
+        }
+    }
+    auto position = [&](long long t) { return pos ? pos[t] : t; };
     const int group = H_q / H_kv;
     const long long chunk_elems = (long long)B * Lc * H_kv * D;
     const long long n_rows = (long long)B * H_q * L;
@@ -236,14 +253,29 @@ int ora_ring_attention(const double* q, const double* k_chunks, const double* v_
             const int j = ((i - off) % P + P) % P;
             const double* kc = k_chunks + j * chunk_elems + ((long long)b * Lc * H_kv + g) * D;
             const double* vc = v_chunks + j * chunk_elems + ((long long)b * Lc * H_kv + g) * D;
-            const long long key0 = (long long)j * Lc;  // global position of the chunk's first key
-            auto visible = [&](long long c) { return !causal || key0 + c <= t; };
+            const long long key0 = (long long)j * Lc;  // rank-major index of the chunk's first key
+            const long long qpos = position(t);
+            auto visible = [&](long long c) { return !causal || position(key0 + c) <= qpos; };
             double lse_part;
             attend_one(qv, kc, vc, (long long)H_kv * D, 0, Lc, D, scale, visible, s,
                        o_part.data(), &lse_part);
             merge_into(o, l, o_part.data(), lse_part, D);
         }
     });
+    return 0;
+}
+
+// The zigzag layout (named beside the plain ring in [ULYSSES], introduction; the layout
+// is a reading): the sequence of P*Lc tokens (Lc even) is cut into 2P segments of
+// h = Lc/2 tokens and rank i holds segment i followed by segment 2P-1-i, so that under a
+// causal mask every rank has the same work.  pos[i*Lc + t] is the sequence position of
+// rank i's local token t.
+int ora_zigzag_positions(int P, long long Lc, long long* pos) {
+    if (P < 1 || Lc < 2 || Lc % 2 != 0) return 1;
+    const long long h = Lc / 2;
+    for (int i = 0; i < P; ++i)
+        for (long long t = 0; t < Lc; ++t)
+            pos[i * Lc + t] = t < h ? i * h + t : (2LL * P - 1 - i) * h + (t - h);
     return 0;
 }
 

@@ -200,6 +200,74 @@ def test_ring_single_rank_is_plain(oracle_mod):
     np.testing.assert_allclose(l, ref_l, atol=1e-12)
 
 
+# ---------------------------------------------------------------- zigzag layout
+# The pages name ZigZag beside the plain ring ("Метод контекстного параллелизма Ulysses",
+# introduction) without describing it; the reading taken: 2P segments of Lc/2 tokens,
+# rank i holding segment i then segment 2P-1-i.
+
+def test_zigzag_positions_hand_written(oracle_mod):
+    # P=2, Lc=4: segments of 2 tokens {0,1} {2,3} {4,5} {6,7}; rank 0 holds segments 0 and
+    # 3, rank 1 holds segments 1 and 2.
+    assert list(oracle_mod.zigzag_positions(2, 4)) == [0, 1, 6, 7, 2, 3, 4, 5]
+    # P=3, Lc=2: single-token segments 0..5; ranks hold (0,5), (1,4), (2,3).
+    assert list(oracle_mod.zigzag_positions(3, 2)) == [0, 5, 1, 4, 2, 3]
+    # one rank holds both segments in order: the identity
+    assert list(oracle_mod.zigzag_positions(1, 6)) == [0, 1, 2, 3, 4, 5]
+
+
+@pytest.mark.parametrize("P,Lc", [(1, 2), (2, 6), (4, 8), (5, 10), (8, 256), (16, 2)])
+def test_zigzag_positions_are_a_permutation(oracle_mod, P, Lc):
+    pos = oracle_mod.zigzag_positions(P, Lc)
+    assert sorted(pos.tolist()) == list(range(P * Lc))
+
+
+@pytest.mark.parametrize("P,Lc", [(2, 4), (4, 8), (8, 64)])
+def test_zigzag_balances_causal_work(oracle_mod, P, Lc):
+    """Under a causal mask a token at position p sees p+1 keys; zigzag gives every rank
+    the same total, h*(2P*h+1) with h = Lc/2, while the contiguous layout does not."""
+    h = Lc // 2
+    pos = oracle_mod.zigzag_positions(P, Lc).reshape(P, Lc)
+    work = (pos + 1).sum(axis=1)
+    assert np.all(work == h * (2 * P * h + 1))
+    contiguous = (np.arange(P * Lc).reshape(P, Lc) + 1).sum(axis=1)
+    assert len(set(contiguous.tolist())) == P
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_ring_identity_positions_equal_contiguous(oracle_mod, causal):
+    P, L = 4, 48
+    q, k, v = rnd((2, L, 4, 8), 60, 2.0), rnd((2, L, 2, 8), 61), rnd((2, L, 2, 8), 62)
+    o0, l0 = oracle_mod.ring_attention(q, _chunks(k, P), _chunks(v, P), 0.4, causal)
+    o1, l1 = oracle_mod.ring_attention(q, _chunks(k, P), _chunks(v, P), 0.4, causal,
+                                       positions=np.arange(L))
+    assert np.array_equal(o0, o1) and np.array_equal(l0, l1)
+
+
+@pytest.mark.parametrize("P,Lc", [(2, 4), (3, 6), (4, 10)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_ring_zigzag_equals_natural_order_sdpa(oracle_mod, P, Lc, causal):
+    """Shards in the zigzag layout: the result of rank-major token R equals the float64
+    library attention over the sequence in natural order, at position pos[R]."""
+    L = P * Lc
+    q, k, v = rnd((2, L, 4, 8), 63, 2.0), rnd((2, L, 2, 8), 64), rnd((2, L, 2, 8), 65)
+    pos = oracle_mod.zigzag_positions(P, Lc)
+    o, l = oracle_mod.ring_attention_zigzag(q, _chunks(k, P), _chunks(v, P), 0.4, causal)
+    nat = np.empty(L, np.int64)
+    nat[pos] = np.arange(L)  # rank-major index of each natural position
+    ref_o, ref_l = torch_sdpa(q[:, nat], k[:, nat], v[:, nat], 0.4, causal)
+    np.testing.assert_allclose(o, ref_o[:, pos], atol=1e-12)
+    np.testing.assert_allclose(l, ref_l[:, :, pos], atol=1e-12)
+
+
+def test_ring_positions_must_be_a_permutation(oracle_mod):
+    q, k, v = rnd((1, 8, 2, 4), 66), rnd((1, 8, 2, 4), 67), rnd((1, 8, 2, 4), 68)
+    with pytest.raises(ValueError):
+        oracle_mod.ring_attention(q, _chunks(k, 2), _chunks(v, 2), 0.5, True,
+                                  positions=[0, 1, 2, 3, 4, 5, 6, 6])
+    with pytest.raises(ValueError):
+        oracle_mod.zigzag_positions(2, 3)  # odd chunk length
+
+
 def test_attention_rows_sample(oracle_mod):
     q, k, v = rnd((2, 40, 4, 8), 33), rnd((2, 40, 2, 8), 34), rnd((2, 40, 2, 8), 35)
     rb, rt, rh = [0, 1, 1, 0], [0, 39, 17, 5], [3, 0, 2, 1]

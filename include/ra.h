@@ -116,6 +116,30 @@ RA_API ra_status ra_ring_attn_fwd(const void* q, const void* const* k_chunks, co
                            void* out, float* lse, void* stream);
 
 /*
+ * ra_ring_attn_fwd_zigzag -- ra_ring_attn_fwd for shards in the zigzag layout.
+ * [ULYSSES] names ZigZag beside the plain ring among the context-parallel
+ * methods (introduction) without describing it; the layout taken here is the
+ * load-balanced one for causal attention: the sequence of L = P*Lc tokens (Lc
+ * even) is cut into 2P segments of Lc/2 tokens and rank i holds segment i
+ * followed by segment 2P-1-i, so under a causal mask every rank has the same
+ * work.  The ring schedule, the merge and the result formula are those of
+ * ra_ring_attn_fwd; only the sequence position of each token changes:
+ *   local token u of rank j's shard (row j*Lc + u of q and of out/lse, row u
+ *   of chunk j) sits at position u < Lc/2 ? j*Lc/2 + u : (2P-1-j)*Lc/2 + u - Lc/2,
+ * and with causal != 0 a key is visible to a query when its position is not
+ * after the query's.  Without causal masking the result equals
+ * ra_ring_attn_fwd's (positions then play no role).
+ * Arguments, layout, ownership and errors: as ra_ring_attn_fwd, plus
+ *   RA_ERR_INVALID when Lc is odd.
+ */
+RA_API ra_status ra_ring_attn_fwd_zigzag(const void* q, const void* const* k_chunks,
+                                         const void* const* v_chunks, int P, int B, int H_q,
+                                         int H_kv, int Lc, int D, long long q_bstride,
+                                         long long kv_bstride, float scale, int causal,
+                                         ra_dtype in_dtype, ra_dtype out_dtype, void* out,
+                                         float* lse, void* stream);
+
+/*
  * ra_lse_merge -- merge two partial attention results over disjoint key sets
  * into one, in place into (o_a, lse_a).  [SP-QA] section 5 (the merge step of
  * the ring loop, read as the exact log-sum-exp combination):

@@ -30,7 +30,7 @@ struct Fp32Params {
     float* out;
     float* lse;
     long long q_bstride, kv_bstride;
-    int P, B, H_q, H_kv, Lc, L, causal;
+    int P, B, H_q, H_kv, Lc, L, causal, zigzag;
     float scale;
 };
 
@@ -48,6 +48,10 @@ __global__ void __launch_bounds__(kRows * 32) attn_fwd_fp32(const __grid_constan
     const int row = r0 + warp;
     const bool active = row < p.L;
     const int last_row = min(r0 + kRows - 1, p.L - 1);
+    // sequence positions (the shard layout): this warp's row and the CTA's largest
+    const long long my_pos = active ? shard_pos(p.zigzag, p.P, p.Lc, row / p.Lc, row % p.Lc) : 0;
+    long long qmin, qmax;
+    row_pos_range(p.zigzag, p.P, p.Lc, r0, last_row, qmin, qmax);
 
     for (int i = threadIdx.x; i < kRows * D; i += blockDim.x) {
         const int rr = r0 + i / D;
@@ -62,12 +66,11 @@ __global__ void __launch_bounds__(kRows * 32) attn_fwd_fp32(const __grid_constan
     const int i0 = r0 / p.Lc;  // rank owning the CTA's first query
     for (int s = 0; s < p.P; ++s) {
         const int j = ((i0 - s) % p.P + p.P) % p.P;
-        const long long key0 = (long long)j * p.Lc;
-        if (p.causal && key0 > last_row) continue;  // chunk wholly after every query: skipped
+        // keys of chunk j at a position <= qmax: a prefix of the chunk (all if not causal)
+        const int n_keys = p.causal ? (int)shard_prefix(p.zigzag, p.P, p.Lc, j, qmax) : p.Lc;
+        if (n_keys == 0) continue;  // chunk wholly after every query: skipped
         const float* kc = p.k[j] + b * p.kv_bstride;
         const float* vc = p.v[j] + b * p.kv_bstride;
-        int n_keys = p.Lc;
-        if (p.causal) n_keys = (int)min((long long)p.Lc, (long long)last_row - key0 + 1);
         for (int c0 = 0; c0 < n_keys; c0 += kKeys) {
             __syncthreads();  // previous tile fully consumed (and qs written, first time)
             for (int i = threadIdx.x; i < kKeys * D; i += blockDim.x) {
@@ -78,8 +81,8 @@ __global__ void __launch_bounds__(kRows * 32) attn_fwd_fp32(const __grid_constan
                 vs[c][d] = in ? vc[off] : 0.f;
             }
             __syncthreads();
-            const long long key = key0 + c0 + lane;
-            const bool vis = active && (c0 + lane < n_keys) && (!p.causal || key <= row);
+            const bool vis = active && (c0 + lane < n_keys) &&
+                             (!p.causal || shard_pos(p.zigzag, p.P, p.Lc, j, c0 + lane) <= my_pos);
             float sc = -INFINITY;
             if (vis) {
                 float dot = 0.f;
@@ -138,6 +141,7 @@ cudaError_t launch_attn_fp32(const AttnArgs& a) {
     p.Lc = a.Lc;
     p.L = a.P * a.Lc;
     p.causal = a.causal;
+    p.zigzag = a.zigzag;
     p.scale = a.scale;
     dim3 grid((p.L + kRows - 1) / kRows, a.B * a.H_q);
     switch (a.D) {

@@ -77,7 +77,7 @@ struct __align__(64) AttnParams {
     void* out;
     float* lse;
     int P, B, H_q, H_kv, Lc, L;
-    int causal, out_bf16, group, n_row_blocks;
+    int causal, zigzag, out_bf16, group, n_row_blocks;
     float scale_log2;
     int inject_stall;
     unsigned long long wait_limit_ns;
@@ -117,18 +117,18 @@ struct Cfg {
 
 // The chunk/tile visiting order of one CTA (all roles derive the same sequence).
 struct Sched {
-    int P, Lc, ntc, i0, causal;
-    long long last_row;  // last query row of the CTA that exists (< L)
+    int P, Lc, ntc, i0, causal, zigzag;
+    long long qmax;  // largest sequence position among the CTA's rows that exist (< L)
     __device__ int chunk_at(int s) const {
         int j = (i0 - s) % P;
         return j < 0 ? j + P : j;
     }
-    // 128-key tiles of chunk j with at least one key <= last_row (all of them if not causal)
+    // 128-key tiles of chunk j holding a key at a position <= qmax (all of them if not
+    // causal).  Positions increase along a shard, so those tiles are a prefix of the chunk.
     __device__ int tiles_in(int j) const {
         if (!causal) return ntc;
-        const long long k0 = (long long)j * Lc;
-        if (k0 > last_row) return 0;
-        const long long t = (last_row - k0) / kBN + 1;
+        const long long nk = shard_prefix(zigzag, P, Lc, j, qmax);
+        const long long t = (nk + kBN - 1) / kBN;
         return t < ntc ? (int)t : ntc;
     }
     __device__ int count() const {
@@ -374,6 +374,15 @@ __device__ __forceinline__ void softmax_wg(const AttnParams& p, uint32_t base, u
     const int lane = threadIdx.x & 31;
     const int q_lo = r0 + wg * kBM;
     const long long my_row = (long long)q_lo + wr * 32 + lane;
+    // Sequence positions: this thread's row, and the smallest among the tile's rows (a
+    // key tile needs a mask only if some key comes after it).
+    const long long my_pos =
+        my_row < p.L ? shard_pos(p.zigzag, p.P, p.Lc, (int)(my_row / p.Lc), my_row % p.Lc)
+                     : (long long)p.L;
+    long long tile_qmin = (long long)p.L, tile_qmax = -1;
+    if (q_lo < p.L)
+        row_pos_range(p.zigzag, p.P, p.Lc, q_lo, min((long long)q_lo + kBM - 1, (long long)p.L - 1),
+                      tile_qmin, tile_qmax);
     const uint32_t lane_off = (uint32_t)(wr * 32) << 16;
     const uint32_t tS = tmem + lane_off + (wg ? C::S_COL1 : C::S_COL0);
     const uint32_t tO = tmem + lane_off + (wg ? C::O_COL1 : C::O_COL0);
@@ -396,17 +405,31 @@ __device__ __forceinline__ void softmax_wg(const AttnParams& p, uint32_t base, u
         uint64_t s2[64];  // the row's 128 scores as pairs (2i, 2i+1)
         tmem_ld128_pairs(tS, s2);
 
-        const long long k0 = (long long)it.chunk() * p.Lc + (long long)it.t * kBN;
-        const int kvalid = min(kBN, p.Lc - it.t * kBN);
-        const bool need_mask = (kvalid < kBN) || (p.causal && k0 + kBN - 1 > q_lo);
+        const int j = it.chunk(), key0 = it.t * kBN;  // chunk and first local key of the tile
+        const int kvalid = min(kBN, p.Lc - key0);
+        const bool need_mask =
+            (kvalid < kBN) ||
+            (p.causal && shard_pos(p.zigzag, p.P, p.Lc, j, key0 + kvalid - 1) > tile_qmin);
         if (need_mask) {
-            const long long lim_c = p.causal ? my_row - k0 : (long long)kBN;  // keys c <= lim_c
+            // Key c of the tile sits at position kpos0 + c; a zigzag tile that straddles
+            // the shard's two segments continues from c = cs at the second segment's start.
+            // Keys c <= lim1 (c < cs) and c <= lim2 (c >= cs) are visible.
+            const long long kpos0 = shard_pos(p.zigzag, p.P, p.Lc, j, key0);
+            const long long lim1 = p.causal ? my_pos - kpos0 : (long long)kBN;
+            int cs = kBN;
+            long long lim2 = lim1;
+            const int hseg = p.Lc / 2;
+            if (p.zigzag && key0 < hseg && key0 + kBN > hseg) {
+                cs = hseg - key0;
+                lim2 = p.causal ? my_pos - shard_pos(1, p.P, p.Lc, j, hseg) + cs : (long long)kBN;
+            }
 #pragma unroll
             for (int i = 0; i < 64; ++i) {
                 float a, b;
                 f2_unpack(s2[i], a, b);
-                if (2 * i >= kvalid || 2 * i > lim_c) a = -INFINITY;
-                if (2 * i + 1 >= kvalid || 2 * i + 1 > lim_c) b = -INFINITY;
+                const long long la = 2 * i < cs ? lim1 : lim2, lb = 2 * i + 1 < cs ? lim1 : lim2;
+                if (2 * i >= kvalid || 2 * i > la) a = -INFINITY;
+                if (2 * i + 1 >= kvalid || 2 * i + 1 > lb) b = -INFINITY;
                 s2[i] = f2_pack(a, b);
             }
         }
@@ -545,7 +568,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100(const __grid_const
     sched.ntc = (p.Lc + kBN - 1) / kBN;
     sched.i0 = r0 / p.Lc;
     sched.causal = p.causal;
-    sched.last_row = min((long long)r0 + 2 * kBM - 1, (long long)p.L - 1);
+    sched.zigzag = p.zigzag;
+    {
+        long long qmin;
+        row_pos_range(p.zigzag, p.P, p.Lc, r0, min((long long)r0 + 2 * kBM - 1, (long long)p.L - 1),
+                      qmin, sched.qmax);
+    }
     const int n = sched.count();
 
     if (threadIdx.x == 0) {
@@ -675,6 +703,7 @@ cudaError_t launch_attn_sm100(const AttnArgs& a, unsigned long long wait_limit_n
     p.Lc = a.Lc;
     p.L = (int)L;
     p.causal = a.causal;
+    p.zigzag = a.zigzag;
     p.out_bf16 = a.out_bf16;
     p.group = a.H_q / a.H_kv;
     p.n_row_blocks = (int)((L + 2 * kBM - 1) / (2 * kBM));

@@ -31,11 +31,64 @@ struct AttnArgs {
     long long q_bstride, kv_bstride;  // elements
     float scale;
     int causal;
+    int zigzag;  // shard layout: 0 contiguous, 1 zigzag (Lc even)
     int out_bf16;
     void* out;
     float* lse;
     cudaStream_t stream;
 };
+
+// ---- sequence positions of the shard layouts ("Как работает sequence parallelism в
+// контексте LLM?", section 2: rank i owns the contiguous tokens i*Lc .. i*Lc+Lc-1; the
+// zigzag layout, named beside the ring in "Метод контекстного параллелизма Ulysses",
+// introduction: 2P segments of h = Lc/2 tokens, rank i holding segment i then segment
+// 2P-1-i).  Within one shard positions increase with the local index in both layouts,
+// which is what lets a causal schedule keep a prefix of each K/V chunk.
+
+// Sequence position of local token u of rank j's shard.
+__host__ __device__ inline long long shard_pos(int zigzag, int P, int Lc, int j, long long u) {
+    if (!zigzag) return (long long)j * Lc + u;
+    const long long h = Lc / 2;
+    return u < h ? (long long)j * h + u : (2LL * P - 1 - j) * h + (u - h);
+}
+
+// Number of leading tokens of rank j's shard whose position is <= qmax (0 .. Lc).
+__host__ __device__ inline long long shard_prefix(int zigzag, int P, int Lc, int j,
+                                                  long long qmax) {
+    long long n;
+    if (!zigzag) {
+        n = qmax - (long long)j * Lc + 1;
+    } else {
+        const long long h = Lc / 2;
+        const long long lo = (long long)j * h, hi = (2LL * P - 1 - j) * h;
+        n = qmax < hi ? qmax - lo + 1 : h + (qmax - hi + 1);
+        if (qmax >= hi) n = n > Lc ? Lc : n;
+        else n = n > h ? h : n;
+    }
+    return n < 0 ? 0 : (n > Lc ? Lc : n);
+}
+
+// Smallest and largest position among the rank-major rows a .. b (a <= b), one shard
+// slice at a time (positions increase within a slice).
+__host__ __device__ inline void row_pos_range(int zigzag, int P, int Lc, long long a, long long b,
+                                              long long& pmin, long long& pmax) {
+    if (!zigzag) {
+        pmin = a;
+        pmax = b;
+        return;
+    }
+    pmin = shard_pos(1, P, Lc, (int)(a / Lc), a % Lc);
+    pmax = pmin;
+    for (long long r = a; r <= b;) {
+        const int i = (int)(r / Lc);
+        const long long t0 = r - (long long)i * Lc;
+        const long long t1 = (b - r) < (Lc - 1 - t0) ? t0 + (b - r) : Lc - 1;
+        const long long p0 = shard_pos(1, P, Lc, i, t0), p1 = shard_pos(1, P, Lc, i, t1);
+        pmin = p0 < pmin ? p0 : pmin;
+        pmax = p1 > pmax ? p1 : pmax;
+        r += t1 - t0 + 1;
+    }
+}
 
 // Tensor-core (tcgen05) attention for bf16 inputs, D in {64, 128}.
 cudaError_t launch_attn_sm100(const AttnArgs& a, unsigned long long wait_limit_ns,

@@ -18,7 +18,8 @@ LIB_PATH = os.path.join(_HERE, "libra_b200.so")
 RA_OK, RA_ERR_INVALID, RA_ERR_UNSUPPORTED, RA_ERR_CUDA, RA_ERR_TIMEOUT = 0, 1, 2, 3, 4
 RA_BF16, RA_FP32 = 0, 1
 RA_MAX_P = 64
-EXPORTED = ("ra_ring_attn_fwd", "ra_lse_merge", "ra_ulysses_seq2head", "ra_ulysses_head2seq",
+EXPORTED = ("ra_ring_attn_fwd", "ra_ring_attn_fwd_zigzag", "ra_lse_merge", "ra_ulysses_seq2head",
+            "ra_ulysses_head2seq",
             "ra_sync_status", "ra_last_error", "ra_set_wait_limit_ns", "ra_debug_inject_stall",
             "ra_version")
 
@@ -44,12 +45,13 @@ def load() -> ctypes.CDLL:
     vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_float
     lib.ra_ring_attn_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i64, i64, f32, i32,
                                      i32, i32, vp, vp, vp]
+    lib.ra_ring_attn_fwd_zigzag.argtypes = lib.ra_ring_attn_fwd.argtypes
     lib.ra_lse_merge.argtypes = [vp, vp, vp, vp, i32, i32, i64, i32, vp]
     lib.ra_ulysses_seq2head.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, vp]
     lib.ra_ulysses_head2seq.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp]
     lib.ra_sync_status.argtypes = [vp]
-    for f in ("ra_ring_attn_fwd", "ra_lse_merge", "ra_ulysses_seq2head", "ra_ulysses_head2seq",
-              "ra_sync_status"):
+    for f in ("ra_ring_attn_fwd", "ra_ring_attn_fwd_zigzag", "ra_lse_merge",
+              "ra_ulysses_seq2head", "ra_ulysses_head2seq", "ra_sync_status"):
         getattr(lib, f).restype = ctypes.c_int
     lib.ra_last_error.restype = ctypes.c_char_p
     lib.ra_version.restype = ctypes.c_char_p
@@ -93,6 +95,16 @@ def ra_ring_attn_fwd(q_ptr, k_ptrs, v_ptrs, P, B, H_q, H_kv, Lc, D, q_bstride, k
     _check(load().ra_ring_attn_fwd(q_ptr, ks, vs, P, B, H_q, H_kv, Lc, D, q_bstride, kv_bstride,
                                    scale, int(causal), in_dtype, out_dtype, out_ptr, lse_ptr,
                                    stream))
+
+
+def ra_ring_attn_fwd_zigzag(q_ptr, k_ptrs, v_ptrs, P, B, H_q, H_kv, Lc, D, q_bstride, kv_bstride,
+                            scale, causal, in_dtype, out_dtype, out_ptr, lse_ptr, stream):
+    """The zigzag-layout C entry point with raw pointers (arguments as ra_ring_attn_fwd)."""
+    arr = ctypes.c_void_p * P
+    ks, vs = arr(*k_ptrs), arr(*v_ptrs)
+    _check(load().ra_ring_attn_fwd_zigzag(q_ptr, ks, vs, P, B, H_q, H_kv, Lc, D, q_bstride,
+                                          kv_bstride, scale, int(causal), in_dtype, out_dtype,
+                                          out_ptr, lse_ptr, stream))
 
 
 def ra_lse_merge(o_a: torch.Tensor, lse_a: torch.Tensor, o_b: torch.Tensor, lse_b: torch.Tensor,
@@ -152,13 +164,18 @@ def ra_debug_inject_stall(on: bool):
 # ------------------------------------------------------------------ tensor-level helper
 def ring_attn_fwd(q: torch.Tensor, k_chunks, v_chunks, causal: bool, scale: float | None = None,
                   out_dtype: torch.dtype = torch.float32, out: torch.Tensor | None = None,
-                  lse: torch.Tensor | None = None, stream=None):
+                  lse: torch.Tensor | None = None, stream=None, layout: str = "contiguous"):
     """Ring-chunked attention of q [B, P*Lc, H_q, D] against P K/V chunks.
 
     k_chunks / v_chunks: a tensor [P, B, Lc, H_kv, D] (chunk j = k_chunks[j]) or a list
     of P tensors [B, Lc, H_kv, D], each batch-contiguous with the same batch stride.
+    layout: "contiguous" (rank i holds tokens i*Lc .. i*Lc+Lc-1) or "zigzag" (rank i holds
+    segments i and 2P-1-i of 2P segments of Lc/2 tokens; see ra_ring_attn_fwd_zigzag).
     Returns (out [B, P*Lc, H_q, D] in out_dtype, lse [B, H_q, P*Lc] fp32).
     """
+    if layout not in ("contiguous", "zigzag"):
+        raise ValueError(f"unknown layout {layout!r}")
+    entry = ra_ring_attn_fwd_zigzag if layout == "zigzag" else ra_ring_attn_fwd
     if isinstance(k_chunks, torch.Tensor):
         k_list = [k_chunks[j] for j in range(k_chunks.shape[0])]
         v_list = [v_chunks[j] for j in range(v_chunks.shape[0])]
@@ -180,8 +197,8 @@ def ring_attn_fwd(q: torch.Tensor, k_chunks, v_chunks, causal: bool, scale: floa
         out = torch.empty((B, L, H_q, D), dtype=out_dtype, device=q.device)
     if lse is None:
         lse = torch.empty((B, H_q, L), dtype=torch.float32, device=q.device)
-    ra_ring_attn_fwd(q.data_ptr(), [t.data_ptr() for t in k_list], [t.data_ptr() for t in v_list],
-                     P, B, H_q, H_kv, Lc, D, q.stride(0) if B > 1 else L * H_q * D,
-                     kv_bstride if B > 1 else Lc * H_kv * D, float(scale), int(bool(causal)),
-                     _dt(q.dtype), _dt(out.dtype), out.data_ptr(), lse.data_ptr(), _stream(stream))
+    entry(q.data_ptr(), [t.data_ptr() for t in k_list], [t.data_ptr() for t in v_list],
+          P, B, H_q, H_kv, Lc, D, q.stride(0) if B > 1 else L * H_q * D,
+          kv_bstride if B > 1 else Lc * H_kv * D, float(scale), int(bool(causal)),
+          _dt(q.dtype), _dt(out.dtype), out.data_ptr(), lse.data_ptr(), _stream(stream))
     return out, lse

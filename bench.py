@@ -13,7 +13,7 @@ the steps (max over ranks), in TFLOP/s.  With --gpus N every rank runs its own r
 (weak scaling: the path has no data-path exchange between independent replicas).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload ulysses_e2e|ulysses_32k|long_128k|llama8b_32k|small_4k]
+                  [--workload ulysses_e2e|ulysses_32k|long_128k|long_128k_zigzag|llama8b_32k|small_4k]
 """
 from __future__ import annotations
 
@@ -54,6 +54,7 @@ def workloads():
         "ulysses_e2e": ("ulysses", synth.ULYSSES_128K),
         "ulysses_32k": ("ulysses", synth.ULYSSES_32K),
         "long_128k": ("attn", synth.LONG_128K),
+        "long_128k_zigzag": ("attn_zigzag", synth.LONG_128K),
         "llama8b_32k": ("attn", synth.LLAMA8B_GQA),
         "small_4k": ("attn", synth.SMALL_BF16),
     }
@@ -172,6 +173,9 @@ class Path:
         import torch
         from sequence_parallelism_attn_b200 import ra, synth
         self.ra, self.kind, self.w, self.dev = ra, kind, w, device
+        # shard layout of the plain attention workloads (zigzag: rank i holds segments i and
+        # 2P-1-i of 2P segments of Lc/2 tokens)
+        self.layout = "zigzag" if kind == "attn_zigzag" else "contiguous"
         if kind == "ulysses":
             a = w.attn()
             self.a = a
@@ -223,7 +227,8 @@ class Path:
         else:
             w = self.w
             rec("attn", 0)
-            ra.ring_attn_fwd(self.q, self.k, self.v, w.causal, w.scale, out=self.o, lse=self.lse)
+            ra.ring_attn_fwd(self.q, self.k, self.v, w.causal, w.scale, out=self.o, lse=self.lse,
+                             layout=self.layout)
             rec("attn", 1)
 
     def result(self):
@@ -422,7 +427,8 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": w.name, "global_batch": w_attn.B * world, "seq_len": w_attn.L,
+        "config": {"workload": w.name + ("_zigzag" if kind == "attn_zigzag" else ""),
+                   "global_batch": w_attn.B * world, "seq_len": w_attn.L,
                    "heads_q": w_attn.H_q, "heads_kv": w_attn.H_kv, "head_dim": w_attn.D,
                    "virtual_ranks": w_attn.P, "chunk_len": w_attn.Lc, "causal": w_attn.causal,
                    "parallelism": f"replicas{world}",
@@ -496,7 +502,8 @@ def reference_arm(args, kind, w, w_attn, rank, world):
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
            "data": "synthetic",
-           "config": {"workload": w.name, "seq_len": w_attn.L, "head_dim": w_attn.D,
+           "config": {"workload": w.name + ("_zigzag" if kind == "attn_zigzag" else ""),
+                      "seq_len": w_attn.L, "head_dim": w_attn.D,
                       "causal": w_attn.causal, "parallelism": "cpu-oracle"},
            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                             "sample": f"{n} query rows x all visible keys of one {w_attn.L}-token "

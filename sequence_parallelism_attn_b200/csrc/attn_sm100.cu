@@ -25,8 +25,8 @@
 //   warp 10    TMA producer of the V tiles (NSV-deep ring)
 //   warp 11    idle (it completes the third warpgroup for the register split)
 // Registers: launched at 168 per thread (3 warps per SM sub-partition); the softmax
-// warpgroups raise their budget to 192 and the third warpgroup drops to 120
-// (192 + 192 + 120 = 504 <= 512 per sub-partition; 256*192 + 128*120 = 384*168).
+// warpgroups raise their budget to 184 and the third warpgroup drops to 136
+// (184 + 184 + 136 = 504 <= 512 per sub-partition; 256*184 + 128*136 = 384*168).
 // Tensor memory (512 columns x 128 lanes x 32 bit):
 //   S_A [0,128) S_B [128,256) fp32 scores; P_A/P_B (bf16 probabilities) overwrite the
 //   first 64 columns of S_A/S_B; O_A at 256, O_B at 256+D (fp32 accumulators).
@@ -58,7 +58,7 @@ __device__ unsigned int g_ra_error_word = 0;
 namespace {
 
 constexpr int kThreads = 384;
-constexpr uint32_t kRegsSoftmax = 192, kRegsOther = 120;
+constexpr uint32_t kRegsSoftmax = 184, kRegsOther = 136;
 constexpr int kWarpLoad = 8;
 constexpr int kWarpMma = 9;
 constexpr int kWarpLoadV = 10;
@@ -78,6 +78,7 @@ struct __align__(64) AttnParams {
     float* lse;
     int P, B, H_q, H_kv, Lc, L;
     int causal, zigzag, out_bf16, group, n_row_blocks;
+    int position_order;  // visit row blocks by descending sequence position (zigzag, see below)
     float scale_log2;
     int inject_stall;
     unsigned long long wait_limit_ns;
@@ -550,17 +551,29 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100(const __grid_const
     auto bar = [&](int i) { return base + C::OFF_BAR + 8u * (uint32_t)i; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // Grid order: (batch, kv head) outermost, then 256-row blocks heaviest first (the last
-    // rows see the most keys when causal), then the query heads sharing that kv head.  The
-    // CTAs resident at any time then stream the same K/V tiles in near lockstep, so K/V are
-    // read from HBM about once per (batch, kv head) and served from L2 after that.
+    // Grid order: (batch, kv head) outermost, then 256-row blocks heaviest first (the rows
+    // at the latest sequence positions see the most keys when causal), then the query heads
+    // sharing that kv head.  The CTAs resident at any time then stream the same K/V tiles
+    // in near lockstep, so K/V are read from HBM about once per (batch, kv head) and served
+    // from L2 after that.  In the contiguous layout the latest positions are the last rows;
+    // in the zigzag layout (when each Lc/2-token segment holds whole blocks) the k-th block
+    // visited is the one at the k-th latest position: segments 2P-1 down to 0, segment
+    // s >= P being the second half of rank 2P-1-s and segment s < P the first half of
+    // rank s.
     const int per_bg = p.n_row_blocks * p.group;
     const int bg = (int)(blockIdx.x / per_bg);
     const int rem = (int)(blockIdx.x % per_bg);
-    const int rb = p.n_row_blocks - 1 - rem / p.group;
+    const int kvis = rem / p.group;  // 0 = visited first
     const int b = bg / p.H_kv, g = bg % p.H_kv;
     const int h = g * p.group + rem % p.group;
-    const int r0 = rb * 2 * kBM;
+    int r0 = (p.n_row_blocks - 1 - kvis) * 2 * kBM;
+    if (p.position_order) {
+        const int hseg = p.Lc / 2, seg_blocks = hseg / (2 * kBM);
+        const int seg = 2 * p.P - 1 - kvis / seg_blocks;
+        const int bis = seg_blocks - 1 - kvis % seg_blocks;
+        const int rank = seg < p.P ? seg : 2 * p.P - 1 - seg;
+        r0 = rank * p.Lc + (seg < p.P ? 0 : hseg) + bis * 2 * kBM;
+    }
 
     Sched sched;
     sched.P = p.P;
@@ -704,6 +717,7 @@ cudaError_t launch_attn_sm100(const AttnArgs& a, unsigned long long wait_limit_n
     p.L = (int)L;
     p.causal = a.causal;
     p.zigzag = a.zigzag;
+    p.position_order = a.zigzag && a.causal && a.Lc % (4 * kBM) == 0;
     p.out_bf16 = a.out_bf16;
     p.group = a.H_q / a.H_kv;
     p.n_row_blocks = (int)((L + 2 * kBM - 1) / (2 * kBM));

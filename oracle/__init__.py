@@ -49,14 +49,15 @@ def _load():
     lib.ora_attention.argtypes = [P, P, P, i32, i64, i32, i32, i32, f64, i32, P, P, i32]
     lib.ora_attention_rows.argtypes = [P, P, P, P, i64, P, P, i32, i64, i32, i32, i32, f64, i32,
                                        P, P, i32]
-    lib.ora_ring_attention.argtypes = [P, P, P, i32, i32, i64, i32, i32, i32, f64, i32, P, P, P, P,
+    lib.ora_ring_attention.argtypes = [P, P, P, i32, i32, i64, i32, i32, i32, f64, i32, P, P, P, P, P,
                                        i32]
     lib.ora_lse_merge.argtypes = [P, P, P, P, i32, i32, i64, i32]
     lib.ora_seq2head.argtypes = [P, P, i32, i32, i64, i32, i32, i32, i32]
     lib.ora_head2seq.argtypes = [P, P, i32, i32, i64, i32, i32, i32]
     lib.ora_zigzag_positions.argtypes = [i32, i64, P]
+    lib.ora_packed_lower_bounds.argtypes = [P, i32, i64, P]
     for f in ("ora_attention", "ora_attention_rows", "ora_ring_attention", "ora_lse_merge",
-              "ora_seq2head", "ora_head2seq", "ora_zigzag_positions"):
+              "ora_seq2head", "ora_head2seq", "ora_zigzag_positions", "ora_packed_lower_bounds"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -113,12 +114,13 @@ def attention_rows(q_rows, rb, rt, rh, k, v, H_q: int, scale: float, causal: boo
 
 
 def ring_attention(q, k_chunks, v_chunks, scale: float, causal: bool, step_offset=None,
-                   positions=None, nthreads: int = 0):
+                   positions=None, lower_bounds=None, nthreads: int = 0):
     """Ring form.  q [B,P*Lc,H_q,D]; k_chunks/v_chunks [P,B,Lc,H_kv,D] -> (out, lse).
 
     Rank i visits chunk (i - step_offset[s]) mod P at step s (default: ring order s).
     positions [P*Lc]: sequence position of each rank-major token (default: contiguous,
-    position = index); the causal mask compares positions."""
+    position = index); the causal mask compares positions.
+    lower_bounds [B, P*Lc]: smallest key position each query may see (packed samples)."""
     q, kc, vc = _f64(q), _f64(k_chunks), _f64(v_chunks)
     P, B, Lc, H_kv, D = kc.shape
     H_q = q.shape[2]
@@ -131,12 +133,17 @@ def ring_attention(q, k_chunks, v_chunks, scale: float, causal: bool, step_offse
     if positions is not None:
         pos = np.ascontiguousarray(positions, dtype=np.int64)
         assert pos.shape == (P * Lc,)
+    lo = None
+    if lower_bounds is not None:
+        lo = np.ascontiguousarray(lower_bounds, dtype=np.int64)
+        assert lo.shape == (B, P * Lc)
     out = np.empty((B, P * Lc, H_q, D), np.float64)
     lse = np.empty((B, H_q, P * Lc), np.float64)
     rc = _load().ora_ring_attention(_ptr(q), _ptr(kc), _ptr(vc), P, B, Lc, H_q, H_kv, D,
                                     float(scale), int(bool(causal)),
                                     _ptr(so) if so is not None else None,
-                                    _ptr(pos) if pos is not None else None, _ptr(out), _ptr(lse),
+                                    _ptr(pos) if pos is not None else None,
+                                    _ptr(lo) if lo is not None else None, _ptr(out), _ptr(lse),
                                     nthreads)
     _check(rc, "ring_attention")
     return out, lse
@@ -148,6 +155,23 @@ def zigzag_positions(P: int, Lc: int) -> np.ndarray:
     pos = np.empty((P * Lc,), np.int64)
     _check(_load().ora_zigzag_positions(P, Lc, _ptr(pos)), "zigzag_positions")
     return pos
+
+
+def packed_lower_bounds(position_ids) -> np.ndarray:
+    """position_ids [B, L] (0, 1, 2, ... within each packed sample) -> the position where
+    each token's sample starts, [B, L] int64."""
+    pid = np.ascontiguousarray(position_ids, dtype=np.int32)
+    B, L = pid.shape
+    lo = np.empty((B, L), np.int64)
+    _check(_load().ora_packed_lower_bounds(_ptr(pid), B, L, _ptr(lo)), "packed_lower_bounds")
+    return lo
+
+
+def ring_attention_packed(q, k_chunks, v_chunks, scale: float, position_ids, nthreads: int = 0):
+    """The causal ring form over packed samples (contiguous shards): query t sees the keys
+    of its own sample up to itself."""
+    return ring_attention(q, k_chunks, v_chunks, scale, True,
+                          lower_bounds=packed_lower_bounds(position_ids), nthreads=nthreads)
 
 
 def ring_attention_zigzag(q, k_chunks, v_chunks, scale: float, causal: bool, nthreads: int = 0):

@@ -35,6 +35,9 @@
 //   * the zigzag layout, only named in [ULYSSES] (introduction), is 2P segments of
 //     Lc/2 tokens with rank i holding segment i then segment 2P-1-i; the causal mask
 //     compares sequence positions, not rank-major indices;
+//   * packed samples ([ACCEL-SP], position_ids instead of an attention mask): samples
+//     are contiguous, position_ids count 0, 1, 2, ... within each, and a query sees
+//     only the keys of its own sample (causal: those not after it);
 //   * Ulysses rank r receives the contiguous head block [r*H/P, (r+1)*H/P),
 //     the global sequence is source-rank-major, and KV replica j of H_out is
 //     source head floor(j * H_in / H_out).
@@ -208,12 +211,17 @@ int ora_attention_rows(const double* q_rows, const int* rb, const long long* rt,
 // mask is pos[key] <= pos[query].  pos == NULL is the contiguous layout of [SP-QA]
 // section 2 (pos[t] = t); any permutation of 0..P*Lc-1 is another assignment of
 // sequence positions to shards (the zigzag layout is one, see ora_zigzag_positions).
+// `lo` (NULL: none) gives, per batch row and rank-major token, the smallest key
+// position its query may see: packed samples ([ACCEL-SP] section "Configuración del
+// backend SP de ALST/Ulysses": several samples combined into one sequence, told apart by
+// position_ids; see ora_packed_lower_bounds).
 //   q  [B][P*Lc][H_q][D]    k, v [P][B][Lc][H_kv][D] (chunk j = rank j's K/V)
+//   lo [B][P*Lc]
 //   out [B][P*Lc][H_q][D]   lse [B][H_q][P*Lc]
 int ora_ring_attention(const double* q, const double* k_chunks, const double* v_chunks, int P,
                        int B, long long Lc, int H_q, int H_kv, int D, double scale, int causal,
-                       const int* step_offset, const long long* pos, double* out, double* lse,
-                       int nthreads) {
+                       const int* step_offset, const long long* pos, const long long* lo,
+                       double* out, double* lse, int nthreads) {
     if (P < 1 || B < 1 || Lc < 1 || H_q < 1 || H_kv < 1 || D < 1 || H_q % H_kv != 0) return 1;
     if (step_offset) {
         std::vector<int> seen(P, 0);
@@ -255,7 +263,11 @@ int ora_ring_attention(const double* q, const double* k_chunks, const double* v_
             const double* vc = v_chunks + j * chunk_elems + ((long long)b * Lc * H_kv + g) * D;
             const long long key0 = (long long)j * Lc;  // rank-major index of the chunk's first key
             const long long qpos = position(t);
-            auto visible = [&](long long c) { return !causal || position(key0 + c) <= qpos; };
+            const long long qlo = lo ? lo[(long long)b * L + t] : 0;
+            auto visible = [&](long long c) {
+                const long long kp = position(key0 + c);
+                return (!causal || kp <= qpos) && kp >= qlo;
+            };
             double lse_part;
             attend_one(qv, kc, vc, (long long)H_kv * D, 0, Lc, D, scale, visible, s,
                        o_part.data(), &lse_part);
@@ -276,6 +288,25 @@ int ora_zigzag_positions(int P, long long Lc, long long* pos) {
     for (int i = 0; i < P; ++i)
         for (long long t = 0; t < Lc; ++t)
             pos[i * Lc + t] = t < h ? i * h + t : (2LL * P - 1 - i) * h + (t - h);
+    return 0;
+}
+
+// Packed samples ([ACCEL-SP] section "Configuración del backend SP de ALST/Ulysses":
+// sequence parallelism there is driven by position_ids, several samples combined into
+// one sequence; the reading taken: samples are contiguous and a sample starts where
+// position_ids is 0, position_ids counting 0, 1, 2, ... within it).  For every token t
+// of every batch row, lo[t] = the position where t's sample starts = t - pid[t]; under
+// the causal mask query t then sees exactly the keys lo[t] .. t of its own sample.
+// Rejects ids that do not follow that rule (pid[t] = 0 or pid[t-1] + 1).
+int ora_packed_lower_bounds(const int* pid, int B, long long L, long long* lo) {
+    if (B < 1 || L < 1) return 1;
+    for (int b = 0; b < B; ++b)
+        for (long long t = 0; t < L; ++t) {
+            const int v = pid[(long long)b * L + t];
+            const bool ok = v == 0 || (t > 0 && v == pid[(long long)b * L + t - 1] + 1);
+            if (!ok) return 1;
+            lo[(long long)b * L + t] = t - v;
+        }
     return 0;
 }
 

@@ -268,6 +268,66 @@ def test_ring_positions_must_be_a_permutation(oracle_mod):
         oracle_mod.zigzag_positions(2, 3)  # odd chunk length
 
 
+# ---------------------------------------------------------------- packed samples
+# "Paralelismo de secuencias en 🤗 accelerate", section "Configuración del backend SP de
+# ALST/Ulysses": sequence parallelism is driven by position_ids and several samples may be
+# combined into one sequence; reading: samples are contiguous, position_ids count
+# 0, 1, 2, ... within each, and attention stays inside a sample.
+
+def _pid_from_lengths(lengths):
+    return np.concatenate([np.arange(n) for n in lengths])
+
+
+def test_packed_lower_bounds_hand_written(oracle_mod):
+    lo = oracle_mod.packed_lower_bounds(np.array([[0, 1, 2, 0, 1, 0, 0, 1]]))
+    assert lo.tolist() == [[0, 0, 0, 3, 3, 5, 6, 6]]
+    with pytest.raises(ValueError):
+        oracle_mod.packed_lower_bounds(np.array([[0, 2, 3]]))  # skips a position
+    with pytest.raises(ValueError):
+        oracle_mod.packed_lower_bounds(np.array([[1, 2, 3]]))  # does not start a sample
+
+
+@pytest.mark.parametrize("P", [1, 3, 4])
+def test_packed_equals_independent_samples_sdpa(oracle_mod, P):
+    """Each packed sample's rows equal float64 library causal attention over that sample
+    alone; two batch rows packed differently."""
+    L = 60
+    lengths = [[7, 1, 20, 32], [60]] if P != 3 else [[13, 13, 34], [1, 1, 58]]
+    pid = np.stack([_pid_from_lengths(x) for x in lengths])
+    q, k, v = rnd((2, L, 4, 8), 70, 2.0), rnd((2, L, 2, 8), 71), rnd((2, L, 2, 8), 72)
+    o, l = oracle_mod.ring_attention_packed(q, _chunks(k, P), _chunks(v, P), 0.4, pid)
+    for b in range(2):
+        s0 = 0
+        for n in lengths[b]:
+            sl = slice(s0, s0 + n)
+            ro, rl = torch_sdpa(q[b:b + 1, sl], k[b:b + 1, sl], v[b:b + 1, sl], 0.4, True)
+            np.testing.assert_allclose(o[b, sl], ro[0], atol=1e-12)
+            np.testing.assert_allclose(l[b, :, sl], rl[0], atol=1e-12)
+            s0 += n
+
+
+def test_packed_single_sample_is_causal_ring(oracle_mod):
+    L, P = 48, 4
+    q, k, v = rnd((1, L, 2, 8), 73), rnd((1, L, 1, 8), 74), rnd((1, L, 1, 8), 75)
+    o0, l0 = oracle_mod.ring_attention(q, _chunks(k, P), _chunks(v, P), 0.5, True)
+    o1, l1 = oracle_mod.ring_attention_packed(q, _chunks(k, P), _chunks(v, P), 0.5,
+                                              np.arange(L)[None])
+    assert np.array_equal(o0, o1) and np.array_equal(l0, l1)
+
+
+def test_packed_one_token_samples_closed_form(oracle_mod):
+    """Every token its own sample: each query sees only its own key, so O = v and
+    LSE = scale * q.k (GQA: query head h reads kv head h // 2)."""
+    L, P = 16, 2
+    q, k, v = rnd((1, L, 4, 8), 76), rnd((1, L, 2, 8), 77), rnd((1, L, 2, 8), 78)
+    o, l = oracle_mod.ring_attention_packed(q, _chunks(k, P), _chunks(v, P), 0.3,
+                                            np.zeros((1, L), np.int64))
+    kv_head = np.arange(4) // 2
+    np.testing.assert_allclose(o[0], v[0][:, kv_head], atol=1e-14)
+    want_l = 0.3 * np.einsum("thd,thd->ht", q[0], k[0][:, kv_head])
+    np.testing.assert_allclose(l[0], want_l, atol=1e-13)
+
+
 def test_attention_rows_sample(oracle_mod):
     q, k, v = rnd((2, 40, 4, 8), 33), rnd((2, 40, 2, 8), 34), rnd((2, 40, 2, 8), 35)
     rb, rt, rh = [0, 1, 1, 0], [0, 39, 17, 5], [3, 0, 2, 1]

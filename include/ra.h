@@ -15,7 +15,9 @@
  *             the GQA rule that KV heads are copied up to the CP-group size.
  *   [ACCEL-SP] "Paralelismo de secuencias en 🤗 accelerate", section "En qué se
  *             diferencia Ulysses SP de FSDP CP": Ulysses needs the head count
- *             divisible by the number of ranks; ring attention does not.
+ *             divisible by the number of ranks; ring attention does not; section
+ *             "Configuración del backend SP de ALST/Ulysses": position_ids and
+ *             packed samples.
  *
  * The P "ranks" of the ring are virtual: P chunk partitions held in the memory
  * of one GPU. Nothing here communicates between devices.
@@ -136,6 +138,32 @@ RA_API ra_status ra_ring_attn_fwd_zigzag(const void* q, const void* const* k_chu
                                          const void* const* v_chunks, int P, int B, int H_q,
                                          int H_kv, int Lc, int D, long long q_bstride,
                                          long long kv_bstride, float scale, int causal,
+                                         ra_dtype in_dtype, ra_dtype out_dtype, void* out,
+                                         float* lse, void* stream);
+
+/*
+ * ra_ring_attn_fwd_packed -- causal ra_ring_attn_fwd over packed samples.
+ * [ACCEL-SP] section "Configuración del backend SP de ALST/Ulysses": sequence
+ * parallelism there is driven by position_ids rather than an attention mask,
+ * and several samples may be combined into one sequence, attention staying
+ * inside each.  The reading taken: the samples of a batch row are contiguous,
+ * position_ids count 0, 1, 2, ... within each sample, and a sample starts where
+ * position_ids is 0.  Query t of batch row b then sees exactly the keys
+ * t - position_ids[b][t] .. t (its own sample, up to itself); the ring
+ * schedule, the merge and the result formula are those of ra_ring_attn_fwd
+ * (contiguous shards, causal).  Tiles and chunks holding no key a row block may
+ * see issue no work, so short samples cost what their own attention costs.
+ * Arguments, layout, ownership and errors: as ra_ring_attn_fwd (without
+ * `causal`, which is implied), plus
+ *   position_ids  device, int32, dense [B][P*Lc], 4-byte aligned; read only.
+ *                 Ids that break the rule above are not detected: each query
+ *                 t then sees the keys max(0, t - id) .. t.
+ *   RA_ERR_INVALID when position_ids is null or misaligned.
+ */
+RA_API ra_status ra_ring_attn_fwd_packed(const void* q, const void* const* k_chunks,
+                                         const void* const* v_chunks, const int* position_ids,
+                                         int P, int B, int H_q, int H_kv, int Lc, int D,
+                                         long long q_bstride, long long kv_bstride, float scale,
                                          ra_dtype in_dtype, ra_dtype out_dtype, void* out,
                                          float* lse, void* stream);
 

@@ -38,13 +38,16 @@ extern "C" {
 static ra_status ring_attn(const void* q, const void* const* k_chunks, const void* const* v_chunks,
                            int P, int B, int H_q, int H_kv, int Lc, int D, long long q_bstride,
                            long long kv_bstride, float scale, int causal, ra_dtype in_dtype,
-                           ra_dtype out_dtype, void* out, float* lse, void* stream, int zigzag) {
+                           ra_dtype out_dtype, void* out, float* lse, void* stream, int zigzag,
+                           const int* position_ids) {
     if (P < 1 || P > RA_MAX_P) return fail(RA_ERR_INVALID, "P must be in [1, RA_MAX_P]");
     if (B < 1 || H_q < 1 || H_kv < 1 || Lc < 1 || D < 1)
         return fail(RA_ERR_INVALID, "B, H_q, H_kv, Lc and D must be >= 1");
     if (H_q % H_kv != 0) return fail(RA_ERR_INVALID, "H_q must be a multiple of H_kv");
     if (zigzag && Lc % 2 != 0)
         return fail(RA_ERR_INVALID, "the zigzag layout needs an even chunk length Lc");
+    if (position_ids && (reinterpret_cast<uintptr_t>(position_ids) & 3u) != 0)
+        return fail(RA_ERR_INVALID, "position_ids must be 4-byte aligned");
     if (causal != 0 && causal != 1) return fail(RA_ERR_INVALID, "causal must be 0 or 1");
     if (!(scale > 0.f) || !std::isfinite(scale))
         return fail(RA_ERR_INVALID, "scale must be finite and > 0");
@@ -88,6 +91,7 @@ static ra_status ring_attn(const void* q, const void* const* k_chunks, const voi
     a.scale = scale;
     a.causal = causal;
     a.zigzag = zigzag;
+    a.pid = position_ids;
     a.out_bf16 = out_dtype == RA_BF16;
     a.out = out;
     a.lse = lse;
@@ -111,7 +115,7 @@ ra_status ra_ring_attn_fwd(const void* q, const void* const* k_chunks, const voi
                            long long kv_bstride, float scale, int causal, ra_dtype in_dtype,
                            ra_dtype out_dtype, void* out, float* lse, void* stream) {
     return ring_attn(q, k_chunks, v_chunks, P, B, H_q, H_kv, Lc, D, q_bstride, kv_bstride, scale,
-                     causal, in_dtype, out_dtype, out, lse, stream, 0);
+                     causal, in_dtype, out_dtype, out, lse, stream, 0, nullptr);
 }
 
 ra_status ra_ring_attn_fwd_zigzag(const void* q, const void* const* k_chunks,
@@ -120,7 +124,17 @@ ra_status ra_ring_attn_fwd_zigzag(const void* q, const void* const* k_chunks,
                                   float scale, int causal, ra_dtype in_dtype, ra_dtype out_dtype,
                                   void* out, float* lse, void* stream) {
     return ring_attn(q, k_chunks, v_chunks, P, B, H_q, H_kv, Lc, D, q_bstride, kv_bstride, scale,
-                     causal, in_dtype, out_dtype, out, lse, stream, 1);
+                     causal, in_dtype, out_dtype, out, lse, stream, 1, nullptr);
+}
+
+ra_status ra_ring_attn_fwd_packed(const void* q, const void* const* k_chunks,
+                                  const void* const* v_chunks, const int* position_ids, int P,
+                                  int B, int H_q, int H_kv, int Lc, int D, long long q_bstride,
+                                  long long kv_bstride, float scale, ra_dtype in_dtype,
+                                  ra_dtype out_dtype, void* out, float* lse, void* stream) {
+    if (!position_ids) return fail(RA_ERR_INVALID, "position_ids must be non-null");
+    return ring_attn(q, k_chunks, v_chunks, P, B, H_q, H_kv, Lc, D, q_bstride, kv_bstride, scale,
+                     1, in_dtype, out_dtype, out, lse, stream, 0, position_ids);
 }
 
 ra_status ra_lse_merge(float* o_a, float* lse_a, const float* o_b, const float* lse_b, int B, int H,

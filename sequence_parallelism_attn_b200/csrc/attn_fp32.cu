@@ -31,6 +31,7 @@ struct Fp32Params {
     float* lse;
     long long q_bstride, kv_bstride;
     int P, B, H_q, H_kv, Lc, L, causal, zigzag;
+    const int* pid;  // packed samples: position_ids [B][L] (nullptr: none)
     float scale;
 };
 
@@ -52,6 +53,18 @@ __global__ void __launch_bounds__(kRows * 32) attn_fwd_fp32(const __grid_constan
     const long long my_pos = active ? shard_pos(p.zigzag, p.P, p.Lc, row / p.Lc, row % p.Lc) : 0;
     long long qmin, qmax;
     row_pos_range(p.zigzag, p.P, p.Lc, r0, last_row, qmin, qmax);
+    // packed samples: row r's sample starts at r - position_ids[r] (clamped to [0, r]);
+    // this warp's row sees no key before its start, and the CTA none before the smallest
+    auto sample_start = [&](int r) {
+        const int st = r - p.pid[(long long)b * p.L + r];
+        return st < 0 ? 0 : (st > r ? r : st);
+    };
+    const long long my_start = (p.pid && active) ? sample_start(row) : 0;
+    long long smin = 0;
+    if (p.pid) {
+        smin = last_row;
+        for (int r = r0; r <= last_row; ++r) smin = min(smin, (long long)sample_start(r));
+    }
 
     for (int i = threadIdx.x; i < kRows * D; i += blockDim.x) {
         const int rr = r0 + i / D;
@@ -68,10 +81,13 @@ __global__ void __launch_bounds__(kRows * 32) attn_fwd_fp32(const __grid_constan
         const int j = ((i0 - s) % p.P + p.P) % p.P;
         // keys of chunk j at a position <= qmax: a prefix of the chunk (all if not causal)
         const int n_keys = p.causal ? (int)shard_prefix(p.zigzag, p.P, p.Lc, j, qmax) : p.Lc;
-        if (n_keys == 0) continue;  // chunk wholly after every query: skipped
+        // packed: keys of the chunk before the smallest sample start are skipped too
+        const long long key0 = (long long)j * p.Lc;
+        const int c_first = smin > key0 ? (int)min(smin - key0, (long long)p.Lc) / kKeys * kKeys : 0;
+        if (n_keys <= c_first) continue;  // nothing in the chunk any row may see: skipped
         const float* kc = p.k[j] + b * p.kv_bstride;
         const float* vc = p.v[j] + b * p.kv_bstride;
-        for (int c0 = 0; c0 < n_keys; c0 += kKeys) {
+        for (int c0 = c_first; c0 < n_keys; c0 += kKeys) {
             __syncthreads();  // previous tile fully consumed (and qs written, first time)
             for (int i = threadIdx.x; i < kKeys * D; i += blockDim.x) {
                 const int c = i / D, d = i % D;
@@ -81,8 +97,9 @@ __global__ void __launch_bounds__(kRows * 32) attn_fwd_fp32(const __grid_constan
                 vs[c][d] = in ? vc[off] : 0.f;
             }
             __syncthreads();
-            const bool vis = active && (c0 + lane < n_keys) &&
-                             (!p.causal || shard_pos(p.zigzag, p.P, p.Lc, j, c0 + lane) <= my_pos);
+            const long long kpos = shard_pos(p.zigzag, p.P, p.Lc, j, c0 + lane);
+            const bool vis = active && (c0 + lane < n_keys) && (!p.causal || kpos <= my_pos) &&
+                             kpos >= my_start;
             float sc = -INFINITY;
             if (vis) {
                 float dot = 0.f;
@@ -142,6 +159,7 @@ cudaError_t launch_attn_fp32(const AttnArgs& a) {
     p.L = a.P * a.Lc;
     p.causal = a.causal;
     p.zigzag = a.zigzag;
+    p.pid = a.pid;
     p.scale = a.scale;
     dim3 grid((p.L + kRows - 1) / kRows, a.B * a.H_q);
     switch (a.D) {

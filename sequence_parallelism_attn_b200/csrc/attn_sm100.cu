@@ -25,8 +25,8 @@
 //   warp 10    TMA producer of the V tiles (NSV-deep ring)
 //   warp 11    idle (it completes the third warpgroup for the register split)
 // Registers: launched at 168 per thread (3 warps per SM sub-partition); the softmax
-// warpgroups raise their budget to 184 and the third warpgroup drops to 136
-// (184 + 184 + 136 = 504 <= 512 per sub-partition; 256*184 + 128*136 = 384*168).
+// warpgroups raise their budget to 192 and the third warpgroup drops to 120
+// (192 + 192 + 120 = 504 <= 512 per sub-partition; 256*192 + 128*120 = 384*168).
 // Tensor memory (512 columns x 128 lanes x 32 bit):
 //   S_A [0,128) S_B [128,256) fp32 scores; P_A/P_B (bf16 probabilities) overwrite the
 //   first 64 columns of S_A/S_B; O_A at 256, O_B at 256+D (fp32 accumulators).
@@ -58,10 +58,11 @@ __device__ unsigned int g_ra_error_word = 0;
 namespace {
 
 constexpr int kThreads = 384;
-constexpr uint32_t kRegsSoftmax = 184, kRegsOther = 136;
+constexpr uint32_t kRegsSoftmax = 192, kRegsOther = 120;
 constexpr int kWarpLoad = 8;
 constexpr int kWarpMma = 9;
 constexpr int kWarpLoadV = 10;
+constexpr int kWarpIdle = 11;  // fills the CTA's schedule in the prologue
 constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 128;  // keys per tile
 constexpr uint32_t kTmemCols = 512;
@@ -79,6 +80,7 @@ struct __align__(64) AttnParams {
     int P, B, H_q, H_kv, Lc, L;
     int causal, zigzag, out_bf16, group, n_row_blocks;
     int position_order;  // visit row blocks by descending sequence position (zigzag, see below)
+    const int* pid;      // packed samples: position_ids [B][L] (nullptr: one sample per row)
     float scale_log2;
     int inject_stall;
     unsigned long long wait_limit_ns;
@@ -100,8 +102,10 @@ struct Cfg {
     // barriers: q_full, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV], s_full[2],
     // p_full[2], o_full[2], drain
     static constexpr int N_BARS = 1 + 2 * NSK + 2 * NSV + 2 + 2 + 2 + 1;
-    static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem base (4 B), abort flag (4 B)
-    static constexpr int SMEM = OFF_MISC + 16 + 1024;      // + slack for 1024-B alignment
+    // tmem base (4 B), abort flag (4 B), the schedule's tile count (4 B)
+    static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
+    static constexpr int OFF_SCHED = OFF_MISC + 16;  // tile ranges: RA_MAX_P starts, RA_MAX_P ends
+    static constexpr int SMEM = OFF_SCHED + 2 * RA_MAX_P * 4 + 1024;  // + 1024-B alignment slack
     static constexpr int BAR_Q = 0;
     __host__ __device__ static constexpr int bar_kf(int s) { return 1 + s; }
     __host__ __device__ static constexpr int bar_ke(int s) { return 1 + NSK + s; }
@@ -116,50 +120,74 @@ struct Cfg {
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
-// The chunk/tile visiting order of one CTA (all roles derive the same sequence).
+// The chunk/tile visiting order of one CTA: chunks in ring order j = (i0 - s) mod P, and
+// of chunk j the tiles [range[j], range[RA_MAX_P + j]) (filled once per CTA into shared
+// memory by make_schedule).
 struct Sched {
-    int P, Lc, ntc, i0, causal, zigzag;
-    long long qmax;  // largest sequence position among the CTA's rows that exist (< L)
-    __device__ int chunk_at(int s) const {
-        int j = (i0 - s) % P;
-        return j < 0 ? j + P : j;
-    }
-    // 128-key tiles of chunk j holding a key at a position <= qmax (all of them if not
-    // causal).  Positions increase along a shard, so those tiles are a prefix of the chunk.
-    __device__ int tiles_in(int j) const {
-        if (!causal) return ntc;
-        const long long nk = shard_prefix(zigzag, P, Lc, j, qmax);
-        const long long t = (nk + kBN - 1) / kBN;
-        return t < ntc ? (int)t : ntc;
-    }
-    __device__ int count() const {
-        int n = 0;
-        for (int s = 0; s < P; ++s) n += tiles_in(chunk_at(s));
-        return n;
-    }
+    const uint32_t* range;
+    int P, i0;
 };
+
+// One warp fills the schedule of a CTA whose rows are r0 .. last_row (rank-major) of batch
+// b: for every chunk j the 128-key tiles holding a key the rows may see.  Causal: keys at
+// positions up to the largest row position (a prefix of the shard, positions increase
+// along it).  Packed samples (position_ids, contiguous layout): keys from the smallest
+// sample start among the rows on (row r's sample starts at r - position_ids[r], clamped
+// to [0, r]).  Returns the number of tiles (in every lane).
+__device__ __forceinline__ int make_schedule(const AttnParams& p, int b, long long r0,
+                                             long long last_row, uint32_t* range) {
+    const int lane = threadIdx.x & 31;
+    const int ntc = (p.Lc + kBN - 1) / kBN;
+    long long qmin, qmax;
+    row_pos_range(p.zigzag, p.P, p.Lc, r0, last_row, qmin, qmax);
+    long long smin = p.pid ? last_row : 0;
+    if (p.pid)
+        for (long long r = r0 + lane; r <= last_row; r += 32) {
+            const long long st = r - (long long)p.pid[(long long)b * p.L + r];
+            smin = min(smin, st < 0 ? 0 : (st > r ? r : st));
+        }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) smin = min(smin, __shfl_xor_sync(0xffffffffu, smin, off));
+    int n = 0;
+    for (int j = lane; j < p.P; j += 32) {
+        long long t_hi = ntc;
+        if (p.causal) {
+            const long long nk = shard_prefix(p.zigzag, p.P, p.Lc, j, qmax);
+            t_hi = min((nk + kBN - 1) / kBN, (long long)ntc);
+        }
+        const long long k0 = (long long)j * p.Lc;
+        long long t_lo = smin > k0 ? min((smin - k0) / kBN, (long long)ntc) : 0;
+        t_lo = min(t_lo, t_hi);
+        range[j] = (uint32_t)t_lo;
+        range[RA_MAX_P + j] = (uint32_t)t_hi;
+        n += (int)(t_hi - t_lo);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) n += __shfl_xor_sync(0xffffffffu, n, off);
+    return n;
+}
 
 // Walks the schedule tile by tile; the chunk index is recomputed only when the step s
 // changes, so a tile costs no integer division.
 struct SchedIter {
-    const Sched* S;
+    Sched S;
     int s, t, nt, j;
-    __device__ void begin(const Sched* sched) {
+    __device__ void load_chunk() {
+        j = (S.i0 - s) % S.P;
+        j = j < 0 ? j + S.P : j;
+        t = (int)S.range[j];
+        nt = (int)S.range[RA_MAX_P + j];
+    }
+    __device__ void begin(const Sched& sched) {
         S = sched;
         s = 0;
-        t = 0;
-        j = S->chunk_at(0);
-        nt = S->tiles_in(j);
+        load_chunk();
         skip_empty();
     }
     __device__ void skip_empty() {
-        while (s < S->P && t >= nt) {
+        while (s < S.P && t >= nt) {
             ++s;
-            t = 0;
-            if (s < S->P) {
-                j = S->chunk_at(s);
-                nt = S->tiles_in(j);
-            }
+            if (s < S.P) load_chunk();
         }
     }
     __device__ void next() {
@@ -257,7 +285,7 @@ __device__ __forceinline__ void producer(const AttnParams& p, uint32_t base, con
         }
     }
     SchedIter it;
-    it.begin(&sched);
+    it.begin(sched);
     for (int jt = 0; jt < n; ++jt, it.next()) {
         const int slot = jt % NS;
         if (jt >= NS && !wait1(bar_empty(slot), ((jt / NS) - 1) & 1, abort_flag, lim, kErrProducer))
@@ -375,15 +403,24 @@ __device__ __forceinline__ void softmax_wg(const AttnParams& p, uint32_t base, u
     const int lane = threadIdx.x & 31;
     const int q_lo = r0 + wg * kBM;
     const long long my_row = (long long)q_lo + wr * 32 + lane;
-    // Sequence positions: this thread's row, and the smallest among the tile's rows (a
-    // key tile needs a mask only if some key comes after it).
-    const long long my_pos =
-        my_row < p.L ? shard_pos(p.zigzag, p.P, p.Lc, (int)(my_row / p.Lc), my_row % p.Lc)
-                     : (long long)p.L;
-    long long tile_qmin = (long long)p.L, tile_qmax = -1;
-    if (q_lo < p.L)
+    // Sequence positions (L <= 2^30, so 32-bit): this thread's row, and the smallest among
+    // the tile's rows (a key tile needs a mask only if some key comes after it).
+    const int my_pos =
+        my_row < p.L ? (int)shard_pos(p.zigzag, p.P, p.Lc, (int)(my_row / p.Lc), my_row % p.Lc)
+                     : p.L;
+    // packed samples: the first key position this row may see (its sample's start)
+    int my_start = 0;
+    if (p.pid && my_row < p.L) {
+        const int r = (int)my_row, st = r - p.pid[(long long)b * p.L + r];
+        my_start = st < 0 ? 0 : (st > r ? r : st);
+    }
+    int tile_qmin = p.L;
+    if (q_lo < p.L) {
+        long long lo_pos, hi_pos;
         row_pos_range(p.zigzag, p.P, p.Lc, q_lo, min((long long)q_lo + kBM - 1, (long long)p.L - 1),
-                      tile_qmin, tile_qmax);
+                      lo_pos, hi_pos);
+        tile_qmin = (int)lo_pos;
+    }
     const uint32_t lane_off = (uint32_t)(wr * 32) << 16;
     const uint32_t tS = tmem + lane_off + (wg ? C::S_COL1 : C::S_COL0);
     const uint32_t tO = tmem + lane_off + (wg ? C::O_COL1 : C::O_COL0);
@@ -395,7 +432,7 @@ __device__ __forceinline__ void softmax_wg(const AttnParams& p, uint32_t base, u
     float m_run = -INFINITY, l_run = 0.f, l_used = 0.f;
     bool ok = true;
     SchedIter it;
-    it.begin(&sched);
+    it.begin(sched);
     for (int jt = 0; jt < n; ++jt, it.next()) {
         if (!wait_warp(bar(C::bar_sf(wg)), jt & 1, abort_flag, lim)) {
             ok = false;
@@ -410,27 +447,34 @@ __device__ __forceinline__ void softmax_wg(const AttnParams& p, uint32_t base, u
         const int kvalid = min(kBN, p.Lc - key0);
         const bool need_mask =
             (kvalid < kBN) ||
-            (p.causal && shard_pos(p.zigzag, p.P, p.Lc, j, key0 + kvalid - 1) > tile_qmin);
+            (p.causal && (int)shard_pos(p.zigzag, p.P, p.Lc, j, key0 + kvalid - 1) > tile_qmin) ||
+            (my_start > (int)shard_pos(p.zigzag, p.P, p.Lc, j, key0));
         if (need_mask) {
-            // Key c of the tile sits at position kpos0 + c; a zigzag tile that straddles
-            // the shard's two segments continues from c = cs at the second segment's start.
-            // Keys c <= lim1 (c < cs) and c <= lim2 (c >= cs) are visible.
-            const long long kpos0 = shard_pos(p.zigzag, p.P, p.Lc, j, key0);
-            const long long lim1 = p.causal ? my_pos - kpos0 : (long long)kBN;
-            int cs = kBN;
-            long long lim2 = lim1;
-            const int hseg = p.Lc / 2;
-            if (p.zigzag && key0 < hseg && key0 + kBN > hseg) {
-                cs = hseg - key0;
-                lim2 = p.causal ? my_pos - shard_pos(1, p.P, p.Lc, j, hseg) + cs : (long long)kBN;
+            // The keys of the tile this row sees form one interval [c_lo, c_hi]: key c sits
+            // at position kpos0 + c, except that a zigzag tile straddling the shard's two
+            // segments continues from c = cs at the second segment's start -- and a row that
+            // sees any key of the second segment sees every key of the first.  c_lo > 0
+            // only for packed samples (keys before the row's sample start).
+            const int kpos0 = (int)shard_pos(p.zigzag, p.P, p.Lc, j, key0);
+            auto clamp_c = [](int x) { return x < -1 ? -1 : (x > kBN ? kBN : x); };
+            int c_hi = kvalid - 1;
+            if (p.causal) {
+                int hi = clamp_c(my_pos - kpos0);
+                const int hseg = p.Lc / 2;
+                if (p.zigzag && key0 < hseg && key0 + kBN > hseg) {
+                    const int cs = hseg - key0;
+                    const int hi2 = clamp_c(my_pos - (int)shard_pos(1, p.P, p.Lc, j, hseg) + cs);
+                    hi = hi2 >= cs ? hi2 : min(hi, cs - 1);
+                }
+                c_hi = min(c_hi, hi);
             }
+            const int c_lo = clamp_c(my_start - kpos0);
 #pragma unroll
             for (int i = 0; i < 64; ++i) {
                 float a, b;
                 f2_unpack(s2[i], a, b);
-                const long long la = 2 * i < cs ? lim1 : lim2, lb = 2 * i + 1 < cs ? lim1 : lim2;
-                if (2 * i >= kvalid || 2 * i > la) a = -INFINITY;
-                if (2 * i + 1 >= kvalid || 2 * i + 1 > lb) b = -INFINITY;
+                if (2 * i < c_lo || 2 * i > c_hi) a = -INFINITY;
+                if (2 * i + 1 < c_lo || 2 * i + 1 > c_hi) b = -INFINITY;
                 s2[i] = f2_pack(a, b);
             }
         }
@@ -575,20 +619,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100(const __grid_const
         r0 = rank * p.Lc + (seg < p.P ? 0 : hseg) + bis * 2 * kBM;
     }
 
-    Sched sched;
-    sched.P = p.P;
-    sched.Lc = p.Lc;
-    sched.ntc = (p.Lc + kBN - 1) / kBN;
-    sched.i0 = r0 / p.Lc;
-    sched.causal = p.causal;
-    sched.zigzag = p.zigzag;
-    {
-        long long qmin;
-        row_pos_range(p.zigzag, p.P, p.Lc, r0, min((long long)r0 + 2 * kBM - 1, (long long)p.L - 1),
-                      qmin, sched.qmax);
-    }
-    const int n = sched.count();
-
     if (threadIdx.x == 0) {
         mbar_init(bar(C::BAR_Q), 1);
         for (int s = 0; s < C::NSK; ++s) {
@@ -612,6 +642,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100(const __grid_const
     if (warp == kWarpLoad && lane == 0) {
         tma_prefetch_desc(&p.tm_q);
     }
+    uint32_t* sched_range = reinterpret_cast<uint32_t*>(smem + C::OFF_SCHED);
+    volatile int* n_slot = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
+    if (warp == kWarpIdle) {
+        const long long last_row = min((long long)r0 + 2 * kBM - 1, (long long)p.L - 1);
+        const int nt = make_schedule(p, b, r0, last_row, sched_range);
+        if (lane == 0) *n_slot = nt;
+    }
     if (warp == kWarpMma) {
         __syncwarp();
         tmem_alloc(base + C::OFF_MISC, kTmemCols);
@@ -621,6 +658,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100(const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+
+    Sched sched;
+    sched.range = sched_range;
+    sched.P = p.P;
+    sched.i0 = r0 / p.Lc;
+    const int n = *n_slot;
 
     if (warp >= 8) {
         regs_decrease<kRegsOther>();
@@ -717,6 +760,7 @@ cudaError_t launch_attn_sm100(const AttnArgs& a, unsigned long long wait_limit_n
     p.L = (int)L;
     p.causal = a.causal;
     p.zigzag = a.zigzag;
+    p.pid = a.pid;
     p.position_order = a.zigzag && a.causal && a.Lc % (4 * kBM) == 0;
     p.out_bf16 = a.out_bf16;
     p.group = a.H_q / a.H_kv;

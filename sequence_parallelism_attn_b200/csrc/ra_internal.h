@@ -32,6 +32,7 @@ struct AttnArgs {
     float scale;
     int causal;
     int zigzag;  // shard layout: 0 contiguous, 1 zigzag (Lc even)
+    const int* pid;  // packed samples: device position_ids [B][P*Lc] (nullptr: none)
     int out_bf16;
     void* out;
     float* lse;

@@ -18,8 +18,8 @@ LIB_PATH = os.path.join(_HERE, "libra_b200.so")
 RA_OK, RA_ERR_INVALID, RA_ERR_UNSUPPORTED, RA_ERR_CUDA, RA_ERR_TIMEOUT = 0, 1, 2, 3, 4
 RA_BF16, RA_FP32 = 0, 1
 RA_MAX_P = 64
-EXPORTED = ("ra_ring_attn_fwd", "ra_ring_attn_fwd_zigzag", "ra_lse_merge", "ra_ulysses_seq2head",
-            "ra_ulysses_head2seq",
+EXPORTED = ("ra_ring_attn_fwd", "ra_ring_attn_fwd_zigzag", "ra_ring_attn_fwd_packed",
+            "ra_lse_merge", "ra_ulysses_seq2head", "ra_ulysses_head2seq",
             "ra_sync_status", "ra_last_error", "ra_set_wait_limit_ns", "ra_debug_inject_stall",
             "ra_version")
 
@@ -46,11 +46,13 @@ def load() -> ctypes.CDLL:
     lib.ra_ring_attn_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i64, i64, f32, i32,
                                      i32, i32, vp, vp, vp]
     lib.ra_ring_attn_fwd_zigzag.argtypes = lib.ra_ring_attn_fwd.argtypes
+    lib.ra_ring_attn_fwd_packed.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i64, i64,
+                                            f32, i32, i32, vp, vp, vp]
     lib.ra_lse_merge.argtypes = [vp, vp, vp, vp, i32, i32, i64, i32, vp]
     lib.ra_ulysses_seq2head.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, vp]
     lib.ra_ulysses_head2seq.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp]
     lib.ra_sync_status.argtypes = [vp]
-    for f in ("ra_ring_attn_fwd", "ra_ring_attn_fwd_zigzag", "ra_lse_merge",
+    for f in ("ra_ring_attn_fwd", "ra_ring_attn_fwd_zigzag", "ra_ring_attn_fwd_packed", "ra_lse_merge",
               "ra_ulysses_seq2head", "ra_ulysses_head2seq", "ra_sync_status"):
         getattr(lib, f).restype = ctypes.c_int
     lib.ra_last_error.restype = ctypes.c_char_p
@@ -104,6 +106,16 @@ def ra_ring_attn_fwd_zigzag(q_ptr, k_ptrs, v_ptrs, P, B, H_q, H_kv, Lc, D, q_bst
     ks, vs = arr(*k_ptrs), arr(*v_ptrs)
     _check(load().ra_ring_attn_fwd_zigzag(q_ptr, ks, vs, P, B, H_q, H_kv, Lc, D, q_bstride,
                                           kv_bstride, scale, int(causal), in_dtype, out_dtype,
+                                          out_ptr, lse_ptr, stream))
+
+
+def ra_ring_attn_fwd_packed(q_ptr, k_ptrs, v_ptrs, pid_ptr, P, B, H_q, H_kv, Lc, D, q_bstride,
+                            kv_bstride, scale, in_dtype, out_dtype, out_ptr, lse_ptr, stream):
+    """The packed-samples C entry point with raw pointers (position_ids: int32 [B][P*Lc])."""
+    arr = ctypes.c_void_p * P
+    ks, vs = arr(*k_ptrs), arr(*v_ptrs)
+    _check(load().ra_ring_attn_fwd_packed(q_ptr, ks, vs, pid_ptr, P, B, H_q, H_kv, Lc, D,
+                                          q_bstride, kv_bstride, scale, in_dtype, out_dtype,
                                           out_ptr, lse_ptr, stream))
 
 
@@ -164,18 +176,31 @@ def ra_debug_inject_stall(on: bool):
 # ------------------------------------------------------------------ tensor-level helper
 def ring_attn_fwd(q: torch.Tensor, k_chunks, v_chunks, causal: bool, scale: float | None = None,
                   out_dtype: torch.dtype = torch.float32, out: torch.Tensor | None = None,
-                  lse: torch.Tensor | None = None, stream=None, layout: str = "contiguous"):
+                  lse: torch.Tensor | None = None, stream=None, layout: str = "contiguous",
+                  position_ids: torch.Tensor | None = None):
     """Ring-chunked attention of q [B, P*Lc, H_q, D] against P K/V chunks.
 
     k_chunks / v_chunks: a tensor [P, B, Lc, H_kv, D] (chunk j = k_chunks[j]) or a list
     of P tensors [B, Lc, H_kv, D], each batch-contiguous with the same batch stride.
     layout: "contiguous" (rank i holds tokens i*Lc .. i*Lc+Lc-1) or "zigzag" (rank i holds
     segments i and 2P-1-i of 2P segments of Lc/2 tokens; see ra_ring_attn_fwd_zigzag).
+    position_ids: int32 [B, P*Lc] on the device (packed samples, causal and contiguous
+    only; see ra_ring_attn_fwd_packed).
     Returns (out [B, P*Lc, H_q, D] in out_dtype, lse [B, H_q, P*Lc] fp32).
     """
     if layout not in ("contiguous", "zigzag"):
         raise ValueError(f"unknown layout {layout!r}")
     entry = ra_ring_attn_fwd_zigzag if layout == "zigzag" else ra_ring_attn_fwd
+    if position_ids is not None:
+        if layout != "contiguous" or not causal:
+            raise ValueError("packed samples need the contiguous layout and causal=True")
+        assert position_ids.dtype == torch.int32 and position_ids.is_cuda
+        assert position_ids.is_contiguous() and position_ids.shape == (q.shape[0], q.shape[1])
+        pid_ptr = position_ids.data_ptr()
+
+        def entry(q_ptr, k_ptrs, v_ptrs, P, B, H_q, H_kv, Lc, D, qs, kvs, sc, causal_, *rest):
+            ra_ring_attn_fwd_packed(q_ptr, k_ptrs, v_ptrs, pid_ptr, P, B, H_q, H_kv, Lc, D, qs,
+                                    kvs, sc, *rest)
     if isinstance(k_chunks, torch.Tensor):
         k_list = [k_chunks[j] for j in range(k_chunks.shape[0])]
         v_list = [v_chunks[j] for j in range(v_chunks.shape[0])]

@@ -153,6 +153,26 @@ def merge_inputs(B: int, H: int, L: int, D: int, seed: int, neg_inf_frac: float 
     return tuple(out)
 
 
+def packed_lengths(L: int, seed: int, min_len: int, max_len: int) -> list[int]:
+    """Seeded lengths of the samples packed into one L-token sequence: log-uniform in
+    [min_len, max_len] (short and long documents alike), the last one cut to fit."""
+    g = _gen(seed)
+    out, total = [], 0
+    lo, hi = math.log(min_len), math.log(max_len)
+    while total < L:
+        n = int(round(math.exp(lo + (hi - lo) * torch.rand((), generator=g).item())))
+        n = max(1, min(n, L - total))
+        out.append(n)
+        total += n
+    return out
+
+
+def position_ids_from_lengths(lengths_per_row: list[list[int]]) -> torch.Tensor:
+    """position_ids [B, L] int32: 0, 1, 2, ... within each packed sample."""
+    rows = [torch.cat([torch.arange(n, dtype=torch.int32) for n in lens]) for lens in lengths_per_row]
+    return torch.stack(rows)
+
+
 def sample_rows(B: int, H_q: int, L: int, n: int, seed: int, Lc: int | None = None,
                 tile: int = 128):
     """Seeded sample of (b, t, h) query rows: n random rows plus every chunk's first and

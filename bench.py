@@ -13,7 +13,8 @@ the steps (max over ranks), in TFLOP/s.  With --gpus N every rank runs its own r
 (weak scaling: the path has no data-path exchange between independent replicas).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload ulysses_e2e|ulysses_32k|long_128k|long_128k_zigzag|llama8b_32k|small_4k]
+                  [--workload ulysses_e2e|ulysses_32k|long_128k|long_128k_zigzag|long_128k_packed|
+                              llama8b_32k|small_4k]
 """
 from __future__ import annotations
 
@@ -55,6 +56,7 @@ def workloads():
         "ulysses_32k": ("ulysses", synth.ULYSSES_32K),
         "long_128k": ("attn", synth.LONG_128K),
         "long_128k_zigzag": ("attn_zigzag", synth.LONG_128K),
+        "long_128k_packed": ("attn_packed", synth.LONG_128K),
         "llama8b_32k": ("attn", synth.LLAMA8B_GQA),
         "small_4k": ("attn", synth.SMALL_BF16),
     }
@@ -202,6 +204,14 @@ class Path:
             self.lse = torch.empty((w.B, w.H_q, w.L), dtype=torch.float32, device=device)
             self.launches_per_step = 1
             self.flops = w.flops()
+            self.pid = None
+            if kind == "attn_packed":
+                # documents of 512..32768 tokens (log-uniform, seeded) packed into each row;
+                # the algorithmic work is each document's own causal attention
+                lens = synth.packed_lengths(w.L, w.seed + 21, 512, 32768)
+                self.pid = synth.position_ids_from_lengths([lens] * w.B).to(device)
+                self.flops = sum(4.0 * w.B * w.H_q * float(n) ** 2 * w.D / 2 for n in lens)
+                self.n_docs = len(lens)
             self.permute_bytes = 0
             self.in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
             self.out_bytes = self.o.numel() * self.o.element_size()
@@ -228,7 +238,7 @@ class Path:
             w = self.w
             rec("attn", 0)
             ra.ring_attn_fwd(self.q, self.k, self.v, w.causal, w.scale, out=self.o, lse=self.lse,
-                             layout=self.layout)
+                             layout=self.layout, position_ids=self.pid)
             rec("attn", 1)
 
     def result(self):
@@ -427,13 +437,17 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": w.name + ("_zigzag" if kind == "attn_zigzag" else ""),
+        "config": {"workload": w.name + {"attn_zigzag": "_zigzag",
+                                         "attn_packed": "_packed"}.get(kind, ""),
                    "global_batch": w_attn.B * world, "seq_len": w_attn.L,
                    "heads_q": w_attn.H_q, "heads_kv": w_attn.H_kv, "head_dim": w_attn.D,
                    "virtual_ranks": w_attn.P, "chunk_len": w_attn.Lc, "causal": w_attn.causal,
                    "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2 (126 MB); no flush between steps"},
     }
+    if kind == "attn_packed":
+        out["config"]["packed_documents"] = path.n_docs
+        out["config"]["document_lengths"] = "512..32768 tokens, log-uniform, seeded"
     sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     traffic = attn_traffic(args.workload)
     out["roofline"] = {"bound": "tensor", "achieved": round(attn_tflops, 2),
@@ -502,7 +516,8 @@ def reference_arm(args, kind, w, w_attn, rank, world):
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
            "data": "synthetic",
-           "config": {"workload": w.name + ("_zigzag" if kind == "attn_zigzag" else ""),
+           "config": {"workload": w.name + {"attn_zigzag": "_zigzag",
+                                            "attn_packed": "_packed"}.get(kind, ""),
                       "seq_len": w_attn.L, "head_dim": w_attn.D,
                       "causal": w_attn.causal, "parallelism": "cpu-oracle"},
            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",

@@ -52,8 +52,8 @@ def _load():
     lib.ora_ring_attention.argtypes = [P, P, P, i32, i32, i64, i32, i32, i32, f64, i32, P, P, P, P, P,
                                        i32]
     lib.ora_lse_merge.argtypes = [P, P, P, P, i32, i32, i64, i32]
-    lib.ora_seq2head.argtypes = [P, P, i32, i32, i64, i32, i32, i32, i32]
-    lib.ora_head2seq.argtypes = [P, P, i32, i32, i64, i32, i32, i32]
+    lib.ora_seq2head.argtypes = [P, P, i32, i32, i32, i64, i32, i32, i32, i32]
+    lib.ora_head2seq.argtypes = [P, P, i32, i32, i32, i64, i32, i32, i32]
     lib.ora_zigzag_positions.argtypes = [i32, i64, P]
     lib.ora_packed_lower_bounds.argtypes = [P, i32, i64, P]
     for f in ("ora_attention", "ora_attention_rows", "ora_ring_attention", "ora_lse_merge",
@@ -192,26 +192,54 @@ def lse_merge(o_a, lse_a, o_b, lse_b):
     return o, l
 
 
-def seq2head(x: np.ndarray, H_out: int) -> np.ndarray:
-    """[P,B,Lc,H_in,D] -> [P,B,P*Lc,H_out/P,D], any dtype, bit-exact."""
+def seq2head(x: np.ndarray, H_out: int, groups: int | None = None) -> np.ndarray:
+    """[P,B,Lc,H_in,D] -> [G,B,P*Lc,H_out/G,D] (G = groups, default P), any dtype, bit-exact."""
     x = np.ascontiguousarray(x)
     P, B, Lc, H_in, D = x.shape
-    if H_out % P or H_out % H_in:
-        raise ValueError("seq2head: H_out must divide by P and by H_in")
-    out = np.empty((P, B, P * Lc, H_out // P, D), x.dtype)
-    _check(_load().ora_seq2head(_ptr(x), _ptr(out), P, B, Lc, H_in, H_out, D, x.itemsize),
+    G = P if groups is None else groups
+    if H_out % G or H_out % H_in:
+        raise ValueError("seq2head: H_out must divide by the group count and by H_in")
+    out = np.empty((G, B, P * Lc, H_out // G, D), x.dtype)
+    _check(_load().ora_seq2head(_ptr(x), _ptr(out), P, G, B, Lc, H_in, H_out, D, x.itemsize),
            "seq2head")
     return out
 
 
-def head2seq(x: np.ndarray) -> np.ndarray:
-    """[P,B,P*Lc,H/P,D] -> [P,B,Lc,H,D], any dtype, bit-exact."""
+def head2seq(x: np.ndarray, P: int | None = None) -> np.ndarray:
+    """[G,B,P*Lc,H/G,D] -> [P,B,Lc,H,D] (P shards, default G), any dtype, bit-exact."""
     x = np.ascontiguousarray(x)
-    P, B, L, Hl, D = x.shape
+    G, B, L, Hl, D = x.shape
+    P = G if P is None else P
     if L % P:
         raise ValueError("head2seq: global length must divide by P")
     Lc = L // P
-    out = np.empty((P, B, Lc, Hl * P, D), x.dtype)
-    _check(_load().ora_head2seq(_ptr(x), _ptr(out), P, B, Lc, Hl * P, D, x.itemsize),
+    out = np.empty((P, B, Lc, Hl * G, D), x.dtype)
+    _check(_load().ora_head2seq(_ptr(x), _ptr(out), P, G, B, Lc, Hl * G, D, x.itemsize),
            "head2seq")
     return out
+
+
+def usp_attention(q, k, v, P_u: int, scale: float, causal: bool, nthreads: int = 0):
+    """The ring x Ulysses hybrid over P sequence shards: q [P,B,Ls,H_q,D], k/v
+    [P,B,Ls,H_kv,D].  The heads are split over P_u Ulysses groups (KV heads copied up to
+    lcm(H_kv, P_u)), each group runs the ring over P/P_u chunks of the whole sequence, and
+    the result comes back sequence-sharded: (out [P,B,Ls,H_q,D], lse [B,H_q,P*Ls])."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    P, B, Ls, H_q, D = q.shape
+    H_kv = k.shape[3]
+    P_r = P // P_u
+    assert P_r * P_u == P and H_q % P_u == 0
+    H_rep = H_kv * P_u // np.gcd(H_kv, P_u)
+    qh = seq2head(q, H_q, groups=P_u)             # [G, B, L, H_q/G, D]
+    kh = seq2head(k, H_rep, groups=P_u)
+    vh = seq2head(v, H_rep, groups=P_u)
+    L = P * Ls
+    Lr = L // P_r
+    G, Hq_l, Hkv_l = P_u, H_q // P_u, H_rep // P_u
+    qa = qh.reshape(G * B, L, Hq_l, D)
+    kc = np.ascontiguousarray(kh.reshape(G * B, P_r, Lr, Hkv_l, D).transpose(1, 0, 2, 3, 4))
+    vc = np.ascontiguousarray(vh.reshape(G * B, P_r, Lr, Hkv_l, D).transpose(1, 0, 2, 3, 4))
+    o, lse = ring_attention(qa, kc, vc, scale, causal, nthreads=nthreads)
+    out = head2seq(o.reshape(G, B, L, Hq_l, D), P=P)
+    lse_full = lse.reshape(G, B, Hq_l, L).transpose(1, 0, 2, 3).reshape(B, H_q, L)
+    return out, lse_full

@@ -325,26 +325,33 @@ int ora_lse_merge(double* o_a, double* lse_a, const double* o_b, const double* l
     return 0;
 }
 
-// Ulysses sequence-sharded -> head-sharded ([ULYSSES]), one element at a time.
-//   in  [P][B][Lc][H_in][D]  ->  out [P][B][P*Lc][H_out/P][D], elements of esize bytes
-//   out[r][b][s*Lc+t][hh][:] = in[s][b][t][((r*Hl + hh) * H_in) / H_out][:],  Hl = H_out/P
-int ora_seq2head(const void* in, void* out, int P, int B, long long Lc, int H_in, int H_out,
-                 int D, int esize) {
-    if (P < 1 || B < 1 || Lc < 1 || H_in < 1 || H_out < 1 || D < 1 || esize < 1) return 1;
-    if (H_out % P != 0 || H_out % H_in != 0) return 1;
-    const int Hl = H_out / P;
+// Ulysses sequence-sharded -> head-sharded ([ULYSSES]: the all-to-all from
+// [local_seqlen, global_heads, head_dim] to [global_seqlen, local_heads, head_dim]),
+// with the head groups counted separately from the shards: G groups of Hl = H_out/G heads,
+// each receiving every one of the P shards' tokens.  G = P is the Ulysses transform
+// itself; G < P is the head split of the ring x Ulysses hybrid (USP), where only P/G ranks
+// share a head group and the ring runs over the rest.  KV heads are copied up to H_out
+// (GQA: replica j is source head floor(j * H_in / H_out)).
+//   in  [P][B][Lc][H_in][D]  ->  out [G][B][P*Lc][Hl][D]
+//   out[g][b][s*Lc+t][hh][:] = in[s][b][t][floor((g*Hl+hh)*H_in/H_out)][:]
+int ora_seq2head(const void* in, void* out, int P, int G, int B, long long Lc, int H_in,
+                 int H_out, int D, int esize) {
+    if (P < 1 || G < 1 || B < 1 || Lc < 1 || H_in < 1 || H_out < 1 || D < 1 || esize < 1)
+        return 1;
+    if (H_out % G != 0 || H_out % H_in != 0) return 1;
+    const int Hl = H_out / G;
     const unsigned char* src = (const unsigned char*)in;
     unsigned char* dst = (unsigned char*)out;
-    for (int r = 0; r < P; ++r)
+    for (int g = 0; g < G; ++g)
         for (int b = 0; b < B; ++b)
             for (int s = 0; s < P; ++s)
                 for (long long t = 0; t < Lc; ++t)
                     for (int hh = 0; hh < Hl; ++hh) {
-                        const int j = r * Hl + hh;                       // replicated head index
+                        const int j = g * Hl + hh;                       // replicated head index
                         const int hs = (int)(((long long)j * H_in) / H_out);  // its source head
                         for (int d = 0; d < D; ++d) {
                             const long long di =
-                                ((((long long)r * B + b) * (P * Lc) + (s * Lc + t)) * Hl + hh) * D + d;
+                                ((((long long)g * B + b) * (P * Lc) + (s * Lc + t)) * Hl + hh) * D + d;
                             const long long si =
                                 ((((long long)s * B + b) * Lc + t) * H_in + hs) * D + d;
                             std::memcpy(dst + di * esize, src + si * esize, (size_t)esize);
@@ -353,24 +360,26 @@ int ora_seq2head(const void* in, void* out, int P, int B, long long Lc, int H_in
     return 0;
 }
 
-// Ulysses head-sharded -> sequence-sharded ([ULYSSES]), the inverse transform.
-//   in  [P][B][P*Lc][H/P][D]  ->  out [P][B][Lc][H][D]
-//   out[s][b][t][r*Hl + hh][:] = in[r][b][s*Lc+t][hh][:],  Hl = H/P
-int ora_head2seq(const void* in, void* out, int P, int B, long long Lc, int H, int D, int esize) {
-    if (P < 1 || B < 1 || Lc < 1 || H < 1 || D < 1 || esize < 1 || H % P != 0) return 1;
-    const int Hl = H / P;
+// Ulysses head-sharded -> sequence-sharded ([ULYSSES]), the inverse transform, for G
+// head groups and P shards.
+//   in  [G][B][P*Lc][H/G][D]  ->  out [P][B][Lc][H][D]
+//   out[s][b][t][g*Hl + hh][:] = in[g][b][s*Lc+t][hh][:],  Hl = H/G
+int ora_head2seq(const void* in, void* out, int P, int G, int B, long long Lc, int H, int D,
+                 int esize) {
+    if (P < 1 || G < 1 || B < 1 || Lc < 1 || H < 1 || D < 1 || esize < 1 || H % G != 0) return 1;
+    const int Hl = H / G;
     const unsigned char* src = (const unsigned char*)in;
     unsigned char* dst = (unsigned char*)out;
     for (int s = 0; s < P; ++s)
         for (int b = 0; b < B; ++b)
             for (long long t = 0; t < Lc; ++t)
-                for (int r = 0; r < P; ++r)
+                for (int g = 0; g < G; ++g)
                     for (int hh = 0; hh < Hl; ++hh)
                         for (int d = 0; d < D; ++d) {
                             const long long di =
-                                ((((long long)s * B + b) * Lc + t) * H + (r * Hl + hh)) * D + d;
+                                ((((long long)s * B + b) * Lc + t) * H + (g * Hl + hh)) * D + d;
                             const long long si =
-                                ((((long long)r * B + b) * (P * Lc) + (s * Lc + t)) * Hl + hh) * D + d;
+                                ((((long long)g * B + b) * (P * Lc) + (s * Lc + t)) * Hl + hh) * D + d;
                             std::memcpy(dst + di * esize, src + si * esize, (size_t)esize);
                         }
     return 0;

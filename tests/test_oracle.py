@@ -459,3 +459,57 @@ def test_seq2head_gqa_replicas_copy_their_source(oracle_mod):
     # with 32 query heads on 8 ranks, rank r's heads 4r..4r+3 use kv head (4r)//(32//4)
     for r in range(P):
         assert (r * H_in) // H_out == (4 * r) // (32 // H_in)
+
+
+# ---------------------------------------------------------------- head groups and the USP hybrid
+# The Ulysses transform with G head groups (G = P is Ulysses itself; G < P is the head split
+# of the ring x Ulysses hybrid, "Paralelismo de secuencias en 🤗 accelerate" naming USP and
+# "Как работает sequence parallelism в контексте LLM?" section 3 the ring over the rest).
+
+def test_seq2head_one_group_concatenates_shards(oracle_mod):
+    """G = 1: the single head group receives every shard's tokens in rank order, all heads."""
+    P, B, Lc, H, D = 3, 2, 4, 5, 2
+    x = np.random.default_rng(80).standard_normal((P, B, Lc, H, D))
+    y = oracle_mod.seq2head(x, H, groups=1)
+    assert y.shape == (1, B, P * Lc, H, D)
+    np.testing.assert_array_equal(y[0], x.transpose(1, 0, 2, 3, 4).reshape(B, P * Lc, H, D))
+
+
+def test_seq2head_groups_hand_written(oracle_mod):
+    # P = 2 shards of 2 tokens, 4 heads, G = 2 groups of 2 heads; value = 100 s + 10 t + h
+    x = np.zeros((2, 1, 2, 4, 1), np.int32)
+    for s in range(2):
+        for t in range(2):
+            for h in range(4):
+                x[s, 0, t, h, 0] = 100 * s + 10 * t + h
+    y = oracle_mod.seq2head(x, 4, groups=2)
+    # group 0: heads 0,1 of tokens (s,t) = (0,0),(0,1),(1,0),(1,1)
+    assert y[0].ravel().tolist() == [0, 1, 10, 11, 100, 101, 110, 111]
+    assert y[1].ravel().tolist() == [2, 3, 12, 13, 102, 103, 112, 113]
+
+
+@pytest.mark.parametrize("P,G", [(4, 2), (6, 3), (6, 2), (3, 1), (4, 4), (2, 4)])
+def test_grouped_round_trip(oracle_mod, P, G):
+    B, Lc, H, D = 2, 3, 8 if G != 3 else 6, 3
+    x = np.random.default_rng(81).integers(0, 1 << 30, (P, B, Lc, H, D)).astype(np.int64)
+    y = oracle_mod.seq2head(x, H, groups=G)
+    assert y.shape == (G, B, P * Lc, H // G, D)
+    np.testing.assert_array_equal(oracle_mod.head2seq(y, P=P), x)
+
+
+@pytest.mark.parametrize("P,P_u", [(4, 2), (6, 3), (4, 4), (4, 1), (8, 2)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_usp_equals_natural_order_sdpa(oracle_mod, P, P_u, causal):
+    """Ring x Ulysses over P shards (P_u head groups, GQA 4:2 with the KV copy) equals the
+    float64 library attention over the whole sequence."""
+    B, Ls, H_kv, D = 2, 5, 2, 8
+    H_q = 6 if P_u == 3 else 4
+    rng = np.random.default_rng(82 + P * 10 + P_u)
+    q = rng.standard_normal((P, B, Ls, H_q, D)) * 2.0
+    k = rng.standard_normal((P, B, Ls, H_kv, D))
+    v = rng.standard_normal((P, B, Ls, H_kv, D))
+    o, l = oracle_mod.usp_attention(q, k, v, P_u, 0.4, causal)
+    seq = lambda x: x.transpose(1, 0, 2, 3, 4).reshape(B, P * Ls, x.shape[3], D)
+    ref_o, ref_l = torch_sdpa(seq(q), seq(k), seq(v), 0.4, causal)
+    np.testing.assert_allclose(seq(o), ref_o, atol=1e-12)
+    np.testing.assert_allclose(l, ref_l, atol=1e-12)

@@ -217,6 +217,28 @@ RA_API ra_status ra_ulysses_head2seq(const void* in, void* out, int P, int B, in
                               int H, int D, ra_dtype dt, void* stream);
 
 /*
+ * ra_ulysses_seq2head_grouped / ra_ulysses_head2seq_grouped -- the two
+ * transforms above with the head groups counted apart from the shards: G
+ * groups of H_out/G heads, each receiving the tokens of all P shards.  G = P is
+ * ra_ulysses_seq2head / ra_ulysses_head2seq.  G < P is the head split of the
+ * ring x Ulysses hybrid (USP; [ACCEL-SP] names it beside Ulysses, and the ring
+ * of [SP-QA] section 3 runs over the rest): with P = P_r * P_u virtual ranks,
+ * the Ulysses all-to-all inside each group of P_u ranks leaves head group g with
+ * the whole sequence, which ra_ring_attn_fwd then treats as P_r ring chunks.
+ *   seq2head: in [P][B][Lc][H_in][D] -> out [G][B][P*Lc][H_out/G][D]
+ *     out[g][b][s*Lc+t][h'][:] = in[s][b][t][floor((g*H_out/G + h')*H_in/H_out)][:]
+ *   head2seq: in [G][B][P*Lc][H/G][D] -> out [P][B][Lc][H][D]
+ *     out[s][b][t][g*H/G + h'][:] = in[g][b][s*Lc+t][h'][:]
+ * Bit-exact.  Errors as the ungrouped forms, with G in place of P in the head
+ * divisibility rules (H_out % G, H % G); RA_ERR_INVALID for G < 1.
+ */
+RA_API ra_status ra_ulysses_seq2head_grouped(const void* in, void* out, int P, int G, int B,
+                                             int Lc, int H_in, int H_out, int D, ra_dtype dt,
+                                             void* stream);
+RA_API ra_status ra_ulysses_head2seq_grouped(const void* in, void* out, int P, int G, int B,
+                                             int Lc, int H, int D, ra_dtype dt, void* stream);
+
+/*
  * ra_sync_status -- synchronise `stream`, then read and clear this device's
  * kernel error word.  Returns RA_ERR_TIMEOUT if a kernel launched since the
  * last call gave up on a bounded wait, RA_ERR_CUDA if the synchronisation

@@ -149,13 +149,14 @@ ra_status ra_lse_merge(float* o_a, float* lse_a, const float* o_b, const float* 
     return RA_OK;
 }
 
-static ra_status check_permute(const void* in, const void* out, int P, int B, int Lc, int H_small,
-                               int H_big, int D, ra_dtype dt) {
-    if (P < 1 || B < 1 || Lc < 1 || H_small < 1 || H_big < 1 || D < 1)
+static ra_status check_permute(const void* in, const void* out, int P, int G, int B, int Lc,
+                               int H_small, int H_big, int D, ra_dtype dt) {
+    if (P < 1 || G < 1 || B < 1 || Lc < 1 || H_small < 1 || H_big < 1 || D < 1)
         return fail(RA_ERR_INVALID, "sizes must be >= 1");
     if (dt != RA_BF16 && dt != RA_FP32) return fail(RA_ERR_INVALID, "bad dtype");
-    if (H_big % P != 0)
-        return fail(RA_ERR_INVALID, "head count must be divisible by the number of ranks P");
+    if (H_big % G != 0)
+        return fail(RA_ERR_INVALID,
+                    "head count must be divisible by the number of head groups (ranks P)");
     if (H_big % H_small != 0)
         return fail(RA_ERR_INVALID, "H_out must be a multiple of H_in");
     if ((D * elem_size(dt)) % 16 != 0)
@@ -169,24 +170,34 @@ static ra_status check_permute(const void* in, const void* out, int P, int B, in
     return RA_OK;
 }
 
-ra_status ra_ulysses_seq2head(const void* in, void* out, int P, int B, int Lc, int H_in, int H_out,
-                              int D, ra_dtype dt, void* stream) {
-    ra_status s = check_permute(in, out, P, B, Lc, H_in, H_out, D, dt);
+ra_status ra_ulysses_seq2head_grouped(const void* in, void* out, int P, int G, int B, int Lc,
+                                      int H_in, int H_out, int D, ra_dtype dt, void* stream) {
+    ra_status s = check_permute(in, out, P, G, B, Lc, H_in, H_out, D, dt);
     if (s != RA_OK) return s;
-    cudaError_t e = ra::launch_seq2head(in, out, P, B, Lc, H_in, H_out, D, elem_size(dt),
+    cudaError_t e = ra::launch_seq2head(in, out, P, G, B, Lc, H_in, H_out, D, elem_size(dt),
                                         (cudaStream_t)stream, g_wait_limit_ns.load());
     if (e != cudaSuccess) return cuda_fail(e, "seq2head launch");
     return RA_OK;
 }
 
-ra_status ra_ulysses_head2seq(const void* in, void* out, int P, int B, int Lc, int H, int D,
-                              ra_dtype dt, void* stream) {
-    ra_status s = check_permute(in, out, P, B, Lc, H, H, D, dt);
+ra_status ra_ulysses_head2seq_grouped(const void* in, void* out, int P, int G, int B, int Lc,
+                                      int H, int D, ra_dtype dt, void* stream) {
+    ra_status s = check_permute(in, out, P, G, B, Lc, H, H, D, dt);
     if (s != RA_OK) return s;
-    cudaError_t e = ra::launch_head2seq(in, out, P, B, Lc, H, D, elem_size(dt),
+    cudaError_t e = ra::launch_head2seq(in, out, P, G, B, Lc, H, D, elem_size(dt),
                                         (cudaStream_t)stream, g_wait_limit_ns.load());
     if (e != cudaSuccess) return cuda_fail(e, "head2seq launch");
     return RA_OK;
+}
+
+ra_status ra_ulysses_seq2head(const void* in, void* out, int P, int B, int Lc, int H_in, int H_out,
+                              int D, ra_dtype dt, void* stream) {
+    return ra_ulysses_seq2head_grouped(in, out, P, P, B, Lc, H_in, H_out, D, dt, stream);
+}
+
+ra_status ra_ulysses_head2seq(const void* in, void* out, int P, int B, int Lc, int H, int D,
+                              ra_dtype dt, void* stream) {
+    return ra_ulysses_head2seq_grouped(in, out, P, P, B, Lc, H, D, dt, stream);
 }
 
 ra_status ra_sync_status(void* stream) {

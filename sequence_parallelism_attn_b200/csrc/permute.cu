@@ -1,6 +1,8 @@
 // permute.cu -- the Ulysses layout transforms ("Метод контекстного параллелизма Ulysses"):
-// sequence-sharded [P][B][Lc][H][D] <-> head-sharded [P][B][P*Lc][H/P][D], with the GQA
-// copy of KV heads up to H_out.  Pure data movement; bit-exact by construction.
+// sequence-sharded [P][B][Lc][H][D] <-> head-sharded [G][B][P*Lc][H/G][D], with the GQA
+// copy of KV heads up to H_out.  G = P is the Ulysses all-to-all; G < P head groups is the
+// head split of the ring x Ulysses hybrid (every group receives all P shards' tokens and
+// the ring runs over them).  Pure data movement; bit-exact by construction.
 //
 // Each thread moves U 16-byte vectors that lie inside one head's D elements, so the
 // per-element index arithmetic is paid once per 16*U bytes; consecutive threads write
@@ -71,7 +73,7 @@ __global__ void __launch_bounds__(256) head2seq_kernel(const int4* __restrict__ 
 // The sequence-sharded side is viewed as a 4-D tensor of 32-bit words
 //   {W = D*elem/4, H, Lc, P*B}              (token t of rank s, batch b at (.., t, s*B + b))
 // and the head-sharded side as a 5-D tensor
-//   {W, Hl, Lc, P, P*B}                      (rank r, batch b, global token s*Lc + t at
+//   {W, Hl, Lc, P, G*B}                      (group r, batch b, global token s*Lc + t at
 //                                             (.., t, s, r*B + b))
 // so a box of T tokens never crosses a chunk boundary: loads past Lc read zeros and stores
 // past Lc are clipped.  One thread per CTA runs a ring of NS shared-memory stages: a tiled
@@ -84,7 +86,7 @@ constexpr int kPermSmem = kPermStages * kPermStageBytes + 128 + 64;
 struct __align__(64) PermTmaParams {
     CUtensorMap src;
     CUtensorMap dst;
-    int P, B, Lc, Hl, H_in, H_out, T, n_tblk, per_head;
+    int P, G, B, Lc, Hl, H_in, H_out, T, n_tblk, per_head;
     int box_bytes;
     long long n_blocks;
     unsigned long long wait_limit_ns;
@@ -117,8 +119,9 @@ __global__ void __launch_bounds__(32) permute_tma_kernel(const __grid_constant__
     const long long n_my =
         p.n_blocks > blockIdx.x ? (p.n_blocks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
-    // block -> coordinates.  seq2head order: (r, b, s, t-block, head); head2seq: (s, b,
-    // t-block, r), so that consecutive blocks write neighbouring destination bytes.
+    // block -> coordinates (r: head group).  seq2head order: (r, b, s, t-block, head);
+    // head2seq: (s, b, t-block, r), so that consecutive blocks write neighbouring
+    // destination bytes.
     auto issue_load = [&](long long i) {
         const long long blk = blockIdx.x + i * gridDim.x;
         const uint32_t stage = base + (uint32_t)(i % kPermStages) * kPermStageBytes;
@@ -142,7 +145,7 @@ __global__ void __launch_bounds__(32) permute_tma_kernel(const __grid_constant__
             tma_load_4d(stage, &p.src, bar, 0, r * p.Hl, tb * p.T, s * p.B + b);
         } else {
             long long x = blk;
-            const int r = (int)(x % p.P); x /= p.P;
+            const int r = (int)(x % p.G); x /= p.G;
             const int tb = (int)(x % p.n_tblk); x /= p.n_tblk;
             const int b = (int)(x % p.B);
             const int s = (int)(x / p.B);
@@ -174,7 +177,7 @@ __global__ void __launch_bounds__(32) permute_tma_kernel(const __grid_constant__
             tma_store_5d(&p.dst, stage, 0, 0, tb * p.T, s, r * p.B + b);
         } else {
             long long x = blk;
-            const int r = (int)(x % p.P); x /= p.P;
+            const int r = (int)(x % p.G); x /= p.G;
             const int tb = (int)(x % p.n_tblk); x /= p.n_tblk;
             const int b = (int)(x % p.B);
             const int s = (int)(x / p.B);
@@ -273,9 +276,10 @@ unsigned grid_for(uint32_t n_groups) {
 
 }  // namespace
 
-cudaError_t launch_seq2head(const void* in, void* out, int P, int B, int Lc, int H_in, int H_out,
-                            int D, int esize, cudaStream_t s, unsigned long long wait_limit_ns) {
-    const int Hl = H_out / P;
+cudaError_t launch_seq2head(const void* in, void* out, int P, int G, int B, int Lc, int H_in,
+                            int H_out, int D, int esize, cudaStream_t s,
+                            unsigned long long wait_limit_ns) {
+    const int Hl = H_out / G;
     if (tma_ok(D, esize) && Hl <= 256 && Hl * (D * esize) <= kPermStageBytes) {
         static thread_local PermTmaParams p;
         const int W = D * esize / 4;
@@ -285,20 +289,20 @@ cudaError_t launch_seq2head(const void* in, void* out, int P, int B, int Lc, int
         const uint64_t sdims[4] = {(uint64_t)W, (uint64_t)H_in, (uint64_t)Lc, (uint64_t)P * B};
         const uint32_t sbox[4] = {(uint32_t)W, (uint32_t)hbox, (uint32_t)p.T, 1};
         const uint64_t ddims[5] = {(uint64_t)W, (uint64_t)Hl, (uint64_t)Lc, (uint64_t)P,
-                                   (uint64_t)P * B};
+                                   (uint64_t)G * B};
         const uint32_t dbox[5] = {(uint32_t)W, (uint32_t)hbox, (uint32_t)p.T, 1, 1};
         if (encode_words(&p.src, in, 4, sdims, sbox) && encode_words(&p.dst, out, 5, ddims, dbox)) {
-            p.P = P; p.B = B; p.Lc = Lc; p.Hl = Hl; p.H_in = H_in; p.H_out = H_out;
+            p.P = P; p.G = G; p.B = B; p.Lc = Lc; p.Hl = Hl; p.H_in = H_in; p.H_out = H_out;
             p.n_tblk = (Lc + p.T - 1) / p.T;
             p.box_bytes = W * 4 * hbox * p.T;
             // per_head: one block per source head (its replicas are stored from one load)
-            p.n_blocks = (long long)(p.per_head ? H_in : P) * B * P * p.n_tblk;
+            p.n_blocks = (long long)(p.per_head ? H_in : G) * B * P * p.n_tblk;
             p.wait_limit_ns = wait_limit_ns;
             return launch_perm_tma<0>(p, s);
         }
     }
-    PermuteGeom geo = make_seq2head_geom(P, B, Lc, H_in, H_out, D, esize);
-    const uint64_t n_vec = (uint64_t)P * B * P * Lc * (uint64_t)(H_out / P) * geo.VD.div;
+    PermuteGeom geo = make_seq2head_geom(P, G, B, Lc, H_in, H_out, D, esize);
+    const uint64_t n_vec = (uint64_t)G * B * P * Lc * (uint64_t)(H_out / G) * geo.VD.div;
     if (geo.VD.div % 4 == 0) {
         const uint32_t n_groups = (uint32_t)(n_vec / 4);
         seq2head_kernel<4><<<grid_for(n_groups), 256, 0, s>>>((const int4*)in, (int4*)out,
@@ -311,29 +315,29 @@ cudaError_t launch_seq2head(const void* in, void* out, int P, int B, int Lc, int
     return cudaGetLastError();
 }
 
-cudaError_t launch_head2seq(const void* in, void* out, int P, int B, int Lc, int H, int D,
+cudaError_t launch_head2seq(const void* in, void* out, int P, int G, int B, int Lc, int H, int D,
                             int esize, cudaStream_t s, unsigned long long wait_limit_ns) {
-    const int Hl = H / P;
+    const int Hl = H / G;
     if (tma_ok(D, esize) && Hl <= 256 && Hl * (D * esize) <= kPermStageBytes) {
         static thread_local PermTmaParams p;
         const int W = D * esize / 4;
         p.per_head = 0;
         p.T = tokens_per_box(W, Hl);
         const uint64_t sdims[5] = {(uint64_t)W, (uint64_t)Hl, (uint64_t)Lc, (uint64_t)P,
-                                   (uint64_t)P * B};
+                                   (uint64_t)G * B};
         const uint32_t sbox[5] = {(uint32_t)W, (uint32_t)Hl, (uint32_t)p.T, 1, 1};
         const uint64_t ddims[4] = {(uint64_t)W, (uint64_t)H, (uint64_t)Lc, (uint64_t)P * B};
         const uint32_t dbox[4] = {(uint32_t)W, (uint32_t)Hl, (uint32_t)p.T, 1};
         if (encode_words(&p.src, in, 5, sdims, sbox) && encode_words(&p.dst, out, 4, ddims, dbox)) {
-            p.P = P; p.B = B; p.Lc = Lc; p.Hl = Hl; p.H_in = H; p.H_out = H;
+            p.P = P; p.G = G; p.B = B; p.Lc = Lc; p.Hl = Hl; p.H_in = H; p.H_out = H;
             p.n_tblk = (Lc + p.T - 1) / p.T;
             p.box_bytes = W * 4 * Hl * p.T;
-            p.n_blocks = (long long)P * B * p.n_tblk * P;
+            p.n_blocks = (long long)P * B * p.n_tblk * G;
             p.wait_limit_ns = wait_limit_ns;
             return launch_perm_tma<1>(p, s);
         }
     }
-    PermuteGeom geo = make_head2seq_geom(P, B, Lc, H, D, esize);
+    PermuteGeom geo = make_head2seq_geom(P, G, B, Lc, H, D, esize);
     const uint64_t n_vec = (uint64_t)P * B * Lc * (uint64_t)H * geo.VD.div;
     if (geo.VD.div % 4 == 0) {
         const uint32_t n_groups = (uint32_t)(n_vec / 4);

@@ -37,11 +37,12 @@ struct PermuteGeom {
     uint32_t H_in;
 };
 
-inline PermuteGeom make_seq2head_geom(int P, int B, int Lc, int H_in, int H_out, int D,
+// G head groups (G = P for the Ulysses transform; fewer for the ring x Ulysses hybrid).
+inline PermuteGeom make_seq2head_geom(int P, int G, int B, int Lc, int H_in, int H_out, int D,
                                       int esize) {
     PermuteGeom g;
     g.VD = make_fastdiv((uint32_t)(D * esize / 16));
-    g.Hl = make_fastdiv((uint32_t)(H_out / P));
+    g.Hl = make_fastdiv((uint32_t)(H_out / G));
     g.H = make_fastdiv((uint32_t)H_out);
     g.PLc = make_fastdiv((uint32_t)P * (uint32_t)Lc);
     g.Lc = make_fastdiv((uint32_t)Lc);
@@ -51,10 +52,10 @@ inline PermuteGeom make_seq2head_geom(int P, int B, int Lc, int H_in, int H_out,
     return g;
 }
 
-inline PermuteGeom make_head2seq_geom(int P, int B, int Lc, int H, int D, int esize) {
+inline PermuteGeom make_head2seq_geom(int P, int G, int B, int Lc, int H, int D, int esize) {
     PermuteGeom g;
     g.VD = make_fastdiv((uint32_t)(D * esize / 16));
-    g.Hl = make_fastdiv((uint32_t)(H / P));
+    g.Hl = make_fastdiv((uint32_t)(H / G));
     g.H = make_fastdiv((uint32_t)H);
     g.PLc = make_fastdiv((uint32_t)P * (uint32_t)Lc);
     g.Lc = make_fastdiv((uint32_t)Lc);
@@ -64,7 +65,7 @@ inline PermuteGeom make_head2seq_geom(int P, int B, int Lc, int H, int D, int es
     return g;
 }
 
-// Output vector `vec` of seq2head, out [P][B][P*Lc][Hl][VD], reads input vector
+// Output vector `vec` of seq2head, out [G][B][P*Lc][Hl][VD] (group r), reads input vector
 //   in [s][b][t][hs][dv] with (r, b, s*Lc+t, hh, dv) = coordinates of vec and
 //   hs = ((r*Hl + hh) * H_in) / H_out  (the GQA copy).
 RA_HD uint64_t seq2head_src_vec(const PermuteGeom& g, uint32_t vec) {
@@ -83,7 +84,7 @@ RA_HD uint64_t seq2head_src_vec(const PermuteGeom& g, uint32_t vec) {
 }
 
 // Output vector `vec` of head2seq, out [P][B][Lc][H][VD] (coordinates s, b, t, hd, dv),
-// reads in [r][b][s*Lc+t][hh][dv] with hd = r*Hl + hh.
+// reads in [r][b][s*Lc+t][hh][dv] (group r of G) with hd = r*Hl + hh.
 RA_HD uint64_t head2seq_src_vec(const PermuteGeom& g, uint32_t vec) {
     const uint32_t seg = fdiv(vec, g.VD);
     const uint32_t dv = vec - seg * g.VD.div;

@@ -98,9 +98,11 @@ cudaError_t launch_attn_sm100(const AttnArgs& a, unsigned long long wait_limit_n
 cudaError_t launch_attn_fp32(const AttnArgs& a);
 cudaError_t launch_lse_merge(float* o_a, float* lse_a, const float* o_b, const float* lse_b, int B,
                              int H, long long L, int D, cudaStream_t s);
-cudaError_t launch_seq2head(const void* in, void* out, int P, int B, int Lc, int H_in, int H_out,
-                            int D, int esize, cudaStream_t s, unsigned long long wait_limit_ns);
-cudaError_t launch_head2seq(const void* in, void* out, int P, int B, int Lc, int H, int D,
+// Ulysses transforms with G head groups (G = P: the Ulysses all-to-all).
+cudaError_t launch_seq2head(const void* in, void* out, int P, int G, int B, int Lc, int H_in,
+                            int H_out, int D, int esize, cudaStream_t s,
+                            unsigned long long wait_limit_ns);
+cudaError_t launch_head2seq(const void* in, void* out, int P, int G, int B, int Lc, int H, int D,
                             int esize, cudaStream_t s, unsigned long long wait_limit_ns);
 // Read and clear the per-device kernel error word (after the caller synchronised).
 cudaError_t read_and_clear_error_word(unsigned int* value);

@@ -20,6 +20,7 @@ RA_BF16, RA_FP32 = 0, 1
 RA_MAX_P = 64
 EXPORTED = ("ra_ring_attn_fwd", "ra_ring_attn_fwd_zigzag", "ra_ring_attn_fwd_packed",
             "ra_lse_merge", "ra_ulysses_seq2head", "ra_ulysses_head2seq",
+            "ra_ulysses_seq2head_grouped", "ra_ulysses_head2seq_grouped",
             "ra_sync_status", "ra_last_error", "ra_set_wait_limit_ns", "ra_debug_inject_stall",
             "ra_version")
 
@@ -51,9 +52,12 @@ def load() -> ctypes.CDLL:
     lib.ra_lse_merge.argtypes = [vp, vp, vp, vp, i32, i32, i64, i32, vp]
     lib.ra_ulysses_seq2head.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, vp]
     lib.ra_ulysses_head2seq.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp]
+    lib.ra_ulysses_seq2head_grouped.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp]
+    lib.ra_ulysses_head2seq_grouped.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, vp]
     lib.ra_sync_status.argtypes = [vp]
     for f in ("ra_ring_attn_fwd", "ra_ring_attn_fwd_zigzag", "ra_ring_attn_fwd_packed", "ra_lse_merge",
-              "ra_ulysses_seq2head", "ra_ulysses_head2seq", "ra_sync_status"):
+              "ra_ulysses_seq2head", "ra_ulysses_head2seq", "ra_ulysses_seq2head_grouped",
+              "ra_ulysses_head2seq_grouped", "ra_sync_status"):
         getattr(lib, f).restype = ctypes.c_int
     lib.ra_last_error.restype = ctypes.c_char_p
     lib.ra_version.restype = ctypes.c_char_p
@@ -131,28 +135,38 @@ def ra_lse_merge(o_a: torch.Tensor, lse_a: torch.Tensor, o_b: torch.Tensor, lse_
 
 
 def ra_ulysses_seq2head(x: torch.Tensor, H_out: int | None = None, out: torch.Tensor | None = None,
-                        stream=None) -> torch.Tensor:
-    """[P,B,Lc,H_in,D] -> [P,B,P*Lc,H_out/P,D] (H_out defaults to H_in)."""
+                        stream=None, groups: int | None = None) -> torch.Tensor:
+    """[P,B,Lc,H_in,D] -> [G,B,P*Lc,H_out/G,D] (H_out defaults to H_in, G = groups to P)."""
     assert x.is_cuda and x.is_contiguous() and x.dim() == 5
     P, B, Lc, H_in, D = x.shape
     H_out = H_in if H_out is None else H_out
+    G = P if groups is None else groups
     if out is None:
-        out = torch.empty((P, B, P * Lc, max(H_out // P, 1), D), dtype=x.dtype, device=x.device)
-    _check(load().ra_ulysses_seq2head(x.data_ptr(), out.data_ptr(), P, B, Lc, H_in, H_out, D,
-                                      _dt(x.dtype), _stream(stream)))
+        out = torch.empty((G, B, P * Lc, max(H_out // G, 1), D), dtype=x.dtype, device=x.device)
+    if G == P:
+        _check(load().ra_ulysses_seq2head(x.data_ptr(), out.data_ptr(), P, B, Lc, H_in, H_out, D,
+                                          _dt(x.dtype), _stream(stream)))
+    else:
+        _check(load().ra_ulysses_seq2head_grouped(x.data_ptr(), out.data_ptr(), P, G, B, Lc, H_in,
+                                                  H_out, D, _dt(x.dtype), _stream(stream)))
     return out
 
 
 def ra_ulysses_head2seq(x: torch.Tensor, out: torch.Tensor | None = None,
-                        stream=None) -> torch.Tensor:
-    """[P,B,P*Lc,H/P,D] -> [P,B,Lc,H,D]."""
+                        stream=None, P: int | None = None) -> torch.Tensor:
+    """[G,B,P*Lc,H/G,D] -> [P,B,Lc,H,D] (P shards, default G)."""
     assert x.is_cuda and x.is_contiguous() and x.dim() == 5
-    P, B, L, Hl, D = x.shape
+    G, B, L, Hl, D = x.shape
+    P = G if P is None else P
     Lc = L // P
     if out is None:
-        out = torch.empty((P, B, Lc, Hl * P, D), dtype=x.dtype, device=x.device)
-    _check(load().ra_ulysses_head2seq(x.data_ptr(), out.data_ptr(), P, B, Lc, Hl * P, D,
-                                      _dt(x.dtype), _stream(stream)))
+        out = torch.empty((P, B, Lc, Hl * G, D), dtype=x.dtype, device=x.device)
+    if G == P:
+        _check(load().ra_ulysses_head2seq(x.data_ptr(), out.data_ptr(), P, B, Lc, Hl * P, D,
+                                          _dt(x.dtype), _stream(stream)))
+    else:
+        _check(load().ra_ulysses_head2seq_grouped(x.data_ptr(), out.data_ptr(), P, G, B, Lc,
+                                                  Hl * G, D, _dt(x.dtype), _stream(stream)))
     return out
 
 

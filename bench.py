@@ -13,7 +13,7 @@ the steps (max over ranks), in TFLOP/s.  With --gpus N every rank runs its own r
 (weak scaling: the path has no data-path exchange between independent replicas).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload ulysses_e2e|ulysses_32k|long_128k|long_128k_zigzag|long_128k_packed|
+                  [--workload ulysses_e2e|ulysses_32k|usp_e2e|long_128k|long_128k_zigzag|long_128k_packed|
                               llama8b_32k|small_4k]
 """
 from __future__ import annotations
@@ -54,6 +54,7 @@ def workloads():
     return {
         "ulysses_e2e": ("ulysses", synth.ULYSSES_128K),
         "ulysses_32k": ("ulysses", synth.ULYSSES_32K),
+        "usp_e2e": ("ulysses", synth.USP_128K),
         "long_128k": ("attn", synth.LONG_128K),
         "long_128k_zigzag": ("attn_zigzag", synth.LONG_128K),
         "long_128k_packed": ("attn_packed", synth.LONG_128K),
@@ -182,8 +183,9 @@ class Path:
             a = w.attn()
             self.a = a
             self.q, self.k, self.v = synth.ulysses_inputs(w, device=device)
-            self.qh = torch.empty((w.P, w.B, a.L, a.H_q, a.D), dtype=w.dtype, device=device)
-            self.kh = torch.empty((w.P, w.B, a.L, a.H_kv, a.D), dtype=w.dtype, device=device)
+            # head-sharded buffers: [G, B, L, heads / G, D] (G = P for Ulysses itself)
+            self.qh = torch.empty((w.G, w.B, a.L, a.H_q, a.D), dtype=w.dtype, device=device)
+            self.kh = torch.empty((w.G, w.B, a.L, a.H_kv, a.D), dtype=w.dtype, device=device)
             self.vh = torch.empty_like(self.kh)
             self.o = torch.empty((a.B, a.L, a.H_q, a.D), dtype=torch.bfloat16, device=device)
             self.lse = torch.empty((a.B, a.H_q, a.L), dtype=torch.float32, device=device)
@@ -223,16 +225,16 @@ class Path:
         if self.kind == "ulysses":
             w, a = self.w, self.a
             rec("permute_in", 0)
-            ra.ra_ulysses_seq2head(self.q, w.H_q, out=self.qh)
-            ra.ra_ulysses_seq2head(self.k, w.H_kv_rep, out=self.kh)
-            ra.ra_ulysses_seq2head(self.v, w.H_kv_rep, out=self.vh)
+            ra.ra_ulysses_seq2head(self.q, w.H_q, out=self.qh, groups=w.G)
+            ra.ra_ulysses_seq2head(self.k, w.H_kv_rep, out=self.kh, groups=w.G)
+            ra.ra_ulysses_seq2head(self.v, w.H_kv_rep, out=self.vh, groups=w.G)
             rec("permute_in", 1)
             rec("attn", 0)
             ra.ring_attn_fwd(self.qa, self.k_chunks, self.v_chunks, True, a.scale,
                              out=self.o, lse=self.lse)
             rec("attn", 1)
             rec("permute_out", 0)
-            ra.ra_ulysses_head2seq(self.o.view(w.P, w.B, a.L, a.H_q, a.D), out=self.o_seq)
+            ra.ra_ulysses_head2seq(self.o.view(w.G, w.B, a.L, a.H_q, a.D), out=self.o_seq, P=w.P)
             rec("permute_out", 1)
         else:
             w = self.w
@@ -445,6 +447,9 @@ def main():
                    "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2 (126 MB); no flush between steps"},
     }
+    if kind == "ulysses":
+        # Ulysses: P head groups; the ring x Ulysses hybrid: fewer, each with a ring
+        out["config"]["head_groups"] = w.G
     if kind == "attn_packed":
         out["config"]["packed_documents"] = path.n_docs
         out["config"]["document_lengths"] = "512..32768 tokens, log-uniform, seeded"

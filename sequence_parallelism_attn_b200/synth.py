@@ -61,18 +61,27 @@ class UlyssesWorkload:
     dtype: torch.dtype
     causal: bool
     seed: int = 0
+    groups: int | None = None  # head groups G (Ulysses: G = P; ring x Ulysses hybrid: G < P)
+
+    @property
+    def G(self) -> int:
+        return self.P if self.groups is None else self.groups
 
     @property
     def H_kv_rep(self) -> int:
-        """KV heads after the GQA copy: the least count that both the ranks and the
+        """KV heads after the GQA copy: the least count that both the head groups and the
         source heads divide (8 for 4 KV heads on 8 ranks)."""
-        return math.lcm(self.H_kv, self.P)
+        return math.lcm(self.H_kv, self.G)
 
     def attn(self) -> AttnWorkload:
-        """The per-rank attention after seq->head: the ranks become the batch."""
-        return AttnWorkload(self.name + "/attn", B=self.P * self.B, H_q=self.H_q // self.P,
-                            H_kv=self.H_kv_rep // self.P, D=self.D, P=self.P, Lc=self.Lc,
-                            dtype=self.dtype, causal=self.causal, seed=self.seed)
+        """The attention after seq->head: the head groups become the batch.  Ulysses itself
+        (no groups given) runs the ring over the P chunks of Lc tokens; the hybrid over the
+        P/G chunks each group's ring ranks hold."""
+        P_r = self.P if self.groups is None else self.P // self.G
+        return AttnWorkload(self.name + "/attn", B=self.G * self.B, H_q=self.H_q // self.G,
+                            H_kv=self.H_kv_rep // self.G, D=self.D, P=P_r,
+                            Lc=self.P * self.Lc // P_r, dtype=self.dtype, causal=self.causal,
+                            seed=self.seed)
 
     def permute_bytes(self) -> int:
         """Bytes a permute step must move: read each input once, write every output once."""
@@ -95,6 +104,8 @@ LONG_128K = AttnWorkload("causal_L131072_H8_D128", B=1, H_q=8, H_kv=8, D=128, P=
                          dtype=torch.bfloat16, causal=True, seed=1004)
 ULYSSES_128K = UlyssesWorkload("ulysses_e2e_L131072", P=8, B=1, Lc=16384, H_q=32, H_kv=4,
                                D=128, dtype=torch.bfloat16, causal=True, seed=1005)
+USP_128K = UlyssesWorkload("usp_e2e_L131072_G4", P=8, B=1, Lc=16384, H_q=32, H_kv=4,
+                           D=128, dtype=torch.bfloat16, causal=True, seed=1005, groups=4)
 ULYSSES_32K = UlyssesWorkload("ulysses_e2e_L32768", P=8, B=1, Lc=4096, H_q=32, H_kv=4,
                               D=128, dtype=torch.bfloat16, causal=True, seed=1006)
 TINY_PERMUTE = UlyssesWorkload("tiny_permute", P=2, B=1, Lc=64, H_q=2, H_kv=2, D=32,

@@ -55,9 +55,12 @@ def _load():
     lib.ora_seq2head.argtypes = [P, P, i32, i32, i32, i64, i32, i32, i32, i32]
     lib.ora_head2seq.argtypes = [P, P, i32, i32, i32, i64, i32, i32, i32]
     lib.ora_zigzag_positions.argtypes = [i32, i64, P]
+    lib.ora_attention_backward.argtypes = [P, P, P, P, i32, i64, i32, i32, i32, f64, i32, P, P,
+                                           P, i32]
     lib.ora_packed_lower_bounds.argtypes = [P, i32, i64, P]
     for f in ("ora_attention", "ora_attention_rows", "ora_ring_attention", "ora_lse_merge",
-              "ora_seq2head", "ora_head2seq", "ora_zigzag_positions", "ora_packed_lower_bounds"):
+              "ora_seq2head", "ora_head2seq", "ora_zigzag_positions", "ora_packed_lower_bounds",
+              "ora_attention_backward"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -88,6 +91,21 @@ def attention(q, k, v, scale: float, causal: bool, nthreads: int = 0):
                                int(bool(causal)), _ptr(out), _ptr(lse), nthreads)
     _check(rc, "attention")
     return out, lse
+
+
+def attention_backward(q, k, v, dout, scale: float, causal: bool, nthreads: int = 0):
+    """Gradients of plain attention.  q/dout [B,L,H_q,D], k/v [B,L,H_kv,D] ->
+    (dq [B,L,H_q,D], dk, dv [B,L,H_kv,D])."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, L, H_q, D = q.shape
+    H_kv = k.shape[2]
+    assert k.shape == (B, L, H_kv, D) and v.shape == k.shape and dout.shape == q.shape
+    dq, dk, dv = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+    rc = _load().ora_attention_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), B, L, H_q, H_kv,
+                                        D, float(scale), int(bool(causal)), _ptr(dq), _ptr(dk),
+                                        _ptr(dv), nthreads)
+    _check(rc, "attention_backward")
+    return dq, dk, dv
 
 
 def attention_rows(q_rows, rb, rt, rh, k, v, H_q: int, scale: float, causal: bool,

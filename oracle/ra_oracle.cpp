@@ -38,6 +38,9 @@
 //   * packed samples ([ACCEL-SP], position_ids instead of an attention mask): samples
 //     are contiguous, position_ids count 0, 1, 2, ... within each, and a query sees
 //     only the keys of its own sample (causal: those not after it);
+//   * the backward pass is the derivative of the definition (the pages train with the
+//     method but print no gradient formula); GQA gradients of a kv head sum over its
+//     query heads;
 //   * Ulysses rank r receives the contiguous head block [r*H/P, (r+1)*H/P),
 //     the global sequence is source-rank-major, and KV replica j of H_out is
 //     source head floor(j * H_in / H_out).
@@ -273,6 +276,92 @@ int ora_ring_attention(const double* q, const double* k_chunks, const double* v_
                        o_part.data(), &lse_part);
             merge_into(o, l, o_part.data(), lse_part, D);
         }
+    });
+    return 0;
+}
+
+// The gradient of plain attention (the backward pass of the method: [SP-QA] trains the
+// model, which needs d/dQ, d/dK, d/dV of O = softmax(scale Q K^T) V; the pages give no
+// formula, so this is the derivative of the definition, written out):
+//   P_ij  = exp(s_ij - lse_i),  s_ij = scale q_i . k_j  (visible j)
+//   dP_ij = dO_i . v_j,          Delta_i = dO_i . O_i = sum_j P_ij dP_ij
+//   dS_ij = P_ij (dP_ij - Delta_i)
+//   dQ_i  = scale sum_j dS_ij k_j
+//   dK_j  = scale sum_{i, h in j's group} dS_ij q_i,   dV_j = sum_{i, h} P_ij dO_i
+// Three passes, each parallel over independent rows: the forward (lse_i, O_i, Delta_i),
+// dQ per query row, dK and dV per (key row, kv head).
+//   q, dout, dq [B][L][H_q][D]    k, v, dk, dv [B][L][H_kv][D]
+int ora_attention_backward(const double* q, const double* k, const double* v,
+                           const double* dout, int B, long long L, int H_q, int H_kv, int D,
+                           double scale, int causal, double* dq, double* dk, double* dv,
+                           int nthreads) {
+    if (B < 1 || L < 1 || H_q < 1 || H_kv < 1 || D < 1 || H_q % H_kv != 0) return 1;
+    const int group = H_q / H_kv;
+    const long long n_rows = (long long)B * H_q * L;
+    std::vector<double> lse(n_rows), delta(n_rows);
+    auto qrow = [&](int b, long long t, int h) { return q + (((long long)b * L + t) * H_q + h) * D; };
+    auto krow = [&](const double* x, int b, long long t, int g) {
+        return x + (((long long)b * L + t) * H_kv + g) * D;
+    };
+    auto dot = [&](const double* a, const double* c) {
+        double r = 0.0;
+        for (int d = 0; d < D; ++d) r += a[d] * c[d];
+        return r;
+    };
+    // pass 1: lse_i and Delta_i = dO_i . O_i
+    parallel_for(n_rows, nthreads, [&](long long row) {
+        thread_local std::vector<double> s, o;
+        const long long t = row % L;
+        const int h = (int)((row / L) % H_q), b = (int)(row / L / H_q), g = h / group;
+        o.assign(D, 0.0);
+        auto visible = [&](long long j) { return !causal || j <= t; };
+        double l;
+        attend_one(qrow(b, t, h), krow(k, b, 0, g), krow(v, b, 0, g), (long long)H_kv * D, 0, L,
+                   D, scale, visible, s, o.data(), &l);
+        lse[row] = l;
+        delta[row] = dot(dout + (((long long)b * L + t) * H_q + h) * D, o.data());
+    });
+    auto P = [&](long long row, const double* qv, const double* kv) {
+        return std::exp(scale * dot(qv, kv) - lse[row]);
+    };
+    // pass 2: dQ
+    parallel_for(n_rows, nthreads, [&](long long row) {
+        const long long t = row % L;
+        const int h = (int)((row / L) % H_q), b = (int)(row / L / H_q), g = h / group;
+        const double* qv = qrow(b, t, h);
+        const double* dov = dout + (((long long)b * L + t) * H_q + h) * D;
+        double* dqv = dq + (((long long)b * L + t) * H_q + h) * D;
+        for (int d = 0; d < D; ++d) dqv[d] = 0.0;
+        const long long jend = causal ? t + 1 : L;
+        for (long long j = 0; j < jend; ++j) {
+            const double p = P(row, qv, krow(k, b, j, g));
+            const double ds = p * (dot(dov, krow(v, b, j, g)) - delta[row]);
+            const double* kj = krow(k, b, j, g);
+            for (int d = 0; d < D; ++d) dqv[d] += scale * ds * kj[d];
+        }
+    });
+    // pass 3: dK, dV per (b, key j, kv head g)
+    const long long n_keys = (long long)B * H_kv * L;
+    parallel_for(n_keys, nthreads, [&](long long kr) {
+        const long long j = kr % L;
+        const int g = (int)((kr / L) % H_kv), b = (int)(kr / L / H_kv);
+        double* dkv = const_cast<double*>(krow(dk, b, j, g));
+        double* dvv = const_cast<double*>(krow(dv, b, j, g));
+        for (int d = 0; d < D; ++d) dkv[d] = dvv[d] = 0.0;
+        const double* kj = krow(k, b, j, g);
+        const double* vj = krow(v, b, j, g);
+        for (int h = g * group; h < (g + 1) * group; ++h)
+            for (long long t = causal ? j : 0; t < L; ++t) {
+                const long long row = ((long long)b * H_q + h) * L + t;
+                const double* qv = qrow(b, t, h);
+                const double* dov = dout + (((long long)b * L + t) * H_q + h) * D;
+                const double p = P(row, qv, kj);
+                const double ds = p * (dot(dov, vj) - delta[row]);
+                for (int d = 0; d < D; ++d) {
+                    dkv[d] += scale * ds * qv[d];
+                    dvv[d] += p * dov[d];
+                }
+            }
     });
     return 0;
 }

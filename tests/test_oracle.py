@@ -513,3 +513,48 @@ def test_usp_equals_natural_order_sdpa(oracle_mod, P, P_u, causal):
     ref_o, ref_l = torch_sdpa(seq(q), seq(k), seq(v), 0.4, causal)
     np.testing.assert_allclose(seq(o), ref_o, atol=1e-12)
     np.testing.assert_allclose(l, ref_l, atol=1e-12)
+
+
+# ---------------------------------------------------------------- backward
+# The gradients of O = softmax(scale Q K^T) V (the pages train with ring attention but give
+# no backward formula; the oracle writes out the derivative of the definition).
+
+def _torch_grads(q, k, v, dout, scale, causal):
+    tq, tk, tv = (torch.from_numpy(x).permute(0, 2, 1, 3).clone().requires_grad_(True)
+                  for x in (q, k, v))
+    out = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, scale=scale,
+                                                           is_causal=causal, enable_gqa=True)
+    out.backward(torch.from_numpy(dout).permute(0, 2, 1, 3))
+    return [t.grad.permute(0, 2, 1, 3).numpy() for t in (tq, tk, tv)]
+
+
+@pytest.mark.parametrize("B,L,H_q,H_kv,D,causal", [(1, 9, 2, 2, 4, True), (2, 17, 4, 2, 8, True),
+                                                   (1, 12, 6, 3, 8, False), (2, 5, 4, 1, 16, True)])
+def test_backward_matches_torch_autograd_fp64(oracle_mod, B, L, H_q, H_kv, D, causal):
+    q, k, v = rnd((B, L, H_q, D), 90, 1.5), rnd((B, L, H_kv, D), 91), rnd((B, L, H_kv, D), 92)
+    dout = rnd((B, L, H_q, D), 93)
+    dq, dk, dv = oracle_mod.attention_backward(q, k, v, dout, 0.37, causal)
+    rq, rk, rv = _torch_grads(q, k, v, dout, 0.37, causal)
+    np.testing.assert_allclose(dq, rq, atol=1e-12)
+    np.testing.assert_allclose(dk, rk, atol=1e-12)
+    np.testing.assert_allclose(dv, rv, atol=1e-12)
+
+
+def test_backward_matches_finite_differences(oracle_mod):
+    """Central differences of sum(O * dO) through the forward oracle (no library)."""
+    B, L, H_q, H_kv, D = 1, 6, 2, 1, 3
+    q, k, v = rnd((B, L, H_q, D), 94), rnd((B, L, H_kv, D), 95), rnd((B, L, H_kv, D), 96)
+    dout = rnd((B, L, H_q, D), 97)
+    dq, dk, dv = oracle_mod.attention_backward(q, k, v, dout, 0.8, True)
+    loss = lambda q_, k_, v_: float(np.sum(oracle_mod.attention(q_, k_, v_, 0.8, True)[0] * dout))
+    eps = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args = {"q": (q, k, v), "k": (q, k, v), "v": (q, k, v)}[name]
+            pa = [xp if a is x else a for a in args]
+            ma = [xm if a is x else a for a in args]
+            fd = (loss(*pa) - loss(*ma)) / (2 * eps)
+            assert abs(fd - g[idx]) < 1e-7, (name, idx, fd, g[idx])

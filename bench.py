@@ -14,6 +14,7 @@ the steps (max over ranks), in TFLOP/s.  With --gpus N every rank runs its own r
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload ulysses_e2e|ulysses_32k|usp_e2e|long_128k|long_128k_zigzag|long_128k_packed|
+                              long_128k_bwd|
                               llama8b_32k|small_4k]
 """
 from __future__ import annotations
@@ -58,6 +59,7 @@ def workloads():
         "long_128k": ("attn", synth.LONG_128K),
         "long_128k_zigzag": ("attn_zigzag", synth.LONG_128K),
         "long_128k_packed": ("attn_packed", synth.LONG_128K),
+        "long_128k_bwd": ("attn_bwd", synth.LONG_128K),
         "llama8b_32k": ("attn", synth.LLAMA8B_GQA),
         "small_4k": ("attn", synth.SMALL_BF16),
     }
@@ -214,6 +216,20 @@ class Path:
                 self.pid = synth.position_ids_from_lengths([lens] * w.B).to(device)
                 self.flops = sum(4.0 * w.B * w.H_q * float(n) ** 2 * w.D / 2 for n in lens)
                 self.n_docs = len(lens)
+            if kind == "attn_bwd":
+                # the backward pass: dout drawn like the inputs; the forward's O and LSE are
+                # produced once, outside the timed steps.  Algorithmic work: five matmuls
+                # (S recomputed, dP, dV, dK, dQ) against the forward's two -> 2.5x.
+                g = torch.Generator(device=device)
+                g.manual_seed(w.seed + 2)
+                self.dout = torch.randn(q.shape, generator=g, device=device).to(torch.bfloat16)
+                ra.ring_attn_fwd(q, k, v, w.causal, w.scale, out=self.o, lse=self.lse)
+                self.dq = torch.empty((w.B, w.L, w.H_q, w.D), dtype=torch.float32, device=device)
+                self.dk = torch.empty(k.shape, dtype=torch.float32, device=device)
+                self.dv = torch.empty_like(self.dk)
+                self.ws = torch.empty((w.B, w.H_q, w.L), dtype=torch.float32, device=device)
+                self.flops = 2.5 * w.flops()
+                self.launches_per_step = 3
             self.permute_bytes = 0
             self.in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
             self.out_bytes = self.o.numel() * self.o.element_size()
@@ -236,6 +252,12 @@ class Path:
             rec("permute_out", 0)
             ra.ra_ulysses_head2seq(self.o.view(w.G, w.B, a.L, a.H_q, a.D), out=self.o_seq, P=w.P)
             rec("permute_out", 1)
+        elif self.kind == "attn_bwd":
+            w = self.w
+            rec("attn", 0)
+            ra.ring_attn_bwd(self.q, self.k, self.v, self.o, self.lse, self.dout, w.causal,
+                             w.scale, dq=self.dq, dk=self.dk, dv=self.dv, workspace=self.ws)
+            rec("attn", 1)
         else:
             w = self.w
             rec("attn", 0)
@@ -439,8 +461,8 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": w.name + {"attn_zigzag": "_zigzag",
-                                         "attn_packed": "_packed"}.get(kind, ""),
+        "config": {"workload": w.name + {"attn_zigzag": "_zigzag", "attn_packed": "_packed",
+                                         "attn_bwd": "_backward"}.get(kind, ""),
                    "global_batch": w_attn.B * world, "seq_len": w_attn.L,
                    "heads_q": w_attn.H_q, "heads_kv": w_attn.H_kv, "head_dim": w_attn.D,
                    "virtual_ranks": w_attn.P, "chunk_len": w_attn.Lc, "causal": w_attn.causal,
@@ -459,7 +481,8 @@ def main():
                        "peak": sustained, "unit": "TFLOP/s",
                        "frac": round(attn_tflops / sustained, 4),
                        "traffic": traffic,
-                       "kernel": "attn_fwd_sm100<128>",
+                       "kernel": ("bwd_delta + bwd_dq_sm100 + bwd_dkdv_sm100, D=128"
+                                  if kind == "attn_bwd" else "attn_fwd_sm100<128>"),
                        "peak_source": f"{peaks_src} bf16_tflops_sustained",
                        "frac_of_burst": round(attn_tflops / peaks.get("bf16_tflops", 1590.0), 4),
                        "frac_of_datasheet": round(attn_tflops / DATASHEET_BF16_TFLOPS, 4)}
@@ -521,8 +544,8 @@ def reference_arm(args, kind, w, w_attn, rank, world):
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
            "data": "synthetic",
-           "config": {"workload": w.name + {"attn_zigzag": "_zigzag",
-                                            "attn_packed": "_packed"}.get(kind, ""),
+           "config": {"workload": w.name + {"attn_zigzag": "_zigzag", "attn_packed": "_packed",
+                                            "attn_bwd": "_backward"}.get(kind, ""),
                       "seq_len": w_attn.L, "head_dim": w_attn.D,
                       "causal": w_attn.causal, "parallelism": "cpu-oracle"},
            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",

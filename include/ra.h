@@ -168,6 +168,44 @@ RA_API ra_status ra_ring_attn_fwd_packed(const void* q, const void* const* k_chu
                                          float* lse, void* stream);
 
 /*
+ * ra_ring_attn_bwd -- the backward pass of ra_ring_attn_fwd (contiguous shards):
+ * the gradients of out with respect to q, k and v given dout = dLoss/dout.
+ * [SP-QA] trains with ring attention (the long-context training the pages
+ * motivate); the pages print no gradient, so this is the derivative of the
+ * forward's definition:
+ *   P_ij  = exp(s_ij - lse_i)            (s as in ra_ring_attn_fwd; lse from it)
+ *   Delta_i = sum_d dout[i][d] * out[i][d]
+ *   dS_ij = P_ij * (dout_i . v_j - Delta_i)
+ *   dq_i = scale * sum_j dS_ij k_j;  dk_j = scale * sum_i dS_ij q_i;  dv_j = sum_i P_ij dout_i
+ * with i over the query rows (of every query head sharing the kv head) that see
+ * key j.  Computed on the tensor cores: a row reduction for Delta, then dq with
+ * the query tile stationary (the chunks in the forward's ring order, causal
+ * tiles skipped), then dk, dv with the key tile stationary.
+ * Arguments
+ *   q, k_chunks, v_chunks, P, B, H_q, H_kv, Lc, D, q_bstride, kv_bstride,
+ *   scale, causal   exactly as given to ra_ring_attn_fwd (bf16, D in {64,128}).
+ *   out        device, bf16, dense [B][P*Lc][H_q][D]: the forward's output.
+ *   lse        device, fp32, dense [B][H_q][P*Lc]: the forward's log-sum-exp.
+ *   dout       device, bf16, dense [B][P*Lc][H_q][D].
+ *   dq         device, fp32, dense [B][P*Lc][H_q][D] (written).
+ *   dk_chunks, dv_chunks  host arrays of P device pointers, chunk j fp32 dense
+ *              [B][Lc][H_kv][D] (written).
+ *   workspace  device, fp32, [B][H_q][P*Lc] scratch owned by the caller (holds
+ *              Delta between the kernels; its contents on return are unspecified).
+ *   stream     cudaStream_t.
+ * Errors: as ra_ring_attn_fwd for the shared arguments; RA_ERR_INVALID for null
+ *   or misaligned out, lse, dout, dq, workspace or gradient chunk pointers;
+ *   RA_ERR_UNSUPPORTED for D outside {64, 128}.
+ */
+RA_API ra_status ra_ring_attn_bwd(const void* q, const void* const* k_chunks,
+                                  const void* const* v_chunks, const void* out,
+                                  const float* lse, const void* dout, int P, int B, int H_q,
+                                  int H_kv, int Lc, int D, long long q_bstride,
+                                  long long kv_bstride, float scale, int causal, float* dq,
+                                  float* const* dk_chunks, float* const* dv_chunks,
+                                  float* workspace, void* stream);
+
+/*
  * ra_lse_merge -- merge two partial attention results over disjoint key sets
  * into one, in place into (o_a, lse_a).  [SP-QA] section 5 (the merge step of
  * the ring loop, read as the exact log-sum-exp combination):

@@ -137,6 +137,66 @@ ra_status ra_ring_attn_fwd_packed(const void* q, const void* const* k_chunks,
                      1, in_dtype, out_dtype, out, lse, stream, 0, position_ids);
 }
 
+ra_status ra_ring_attn_bwd(const void* q, const void* const* k_chunks, const void* const* v_chunks,
+                           const void* out, const float* lse, const void* dout, int P, int B,
+                           int H_q, int H_kv, int Lc, int D, long long q_bstride,
+                           long long kv_bstride, float scale, int causal, float* dq,
+                           float* const* dk_chunks, float* const* dv_chunks, float* workspace,
+                           void* stream) {
+    if (P < 1 || P > RA_MAX_P) return fail(RA_ERR_INVALID, "P must be in [1, RA_MAX_P]");
+    if (B < 1 || H_q < 1 || H_kv < 1 || Lc < 1 || D < 1)
+        return fail(RA_ERR_INVALID, "B, H_q, H_kv, Lc and D must be >= 1");
+    if (H_q % H_kv != 0) return fail(RA_ERR_INVALID, "H_q must be a multiple of H_kv");
+    if (causal != 0 && causal != 1) return fail(RA_ERR_INVALID, "causal must be 0 or 1");
+    if (!(scale > 0.f) || !std::isfinite(scale))
+        return fail(RA_ERR_INVALID, "scale must be finite and > 0");
+    if (D != 64 && D != 128)
+        return fail(RA_ERR_UNSUPPORTED, "the tensor-core backward supports D in {64, 128}");
+    const long long L = (long long)P * Lc;
+    if (L > (1ll << 30)) return fail(RA_ERR_INVALID, "P*Lc must be <= 2^30");
+    if (q_bstride < L * H_q * D) return fail(RA_ERR_INVALID, "q_bstride below the dense size");
+    if (kv_bstride < (long long)Lc * H_kv * D)
+        return fail(RA_ERR_INVALID, "kv_bstride below the dense size");
+    if ((q_bstride * 2) % 16 != 0 || (kv_bstride * 2) % 16 != 0)
+        return fail(RA_ERR_INVALID, "batch strides must be multiples of 16 bytes");
+    if (!aligned16(q) || !aligned16(out) || !aligned16(lse) || !aligned16(dout) ||
+        !aligned16(dq) || !aligned16(workspace))
+        return fail(RA_ERR_INVALID, "q, out, lse, dout, dq and workspace must be non-null and "
+                                    "16-byte aligned");
+    if (!k_chunks || !v_chunks || !dk_chunks || !dv_chunks)
+        return fail(RA_ERR_INVALID, "chunk pointer arrays must be non-null");
+    for (int j = 0; j < P; ++j)
+        if (!aligned16(k_chunks[j]) || !aligned16(v_chunks[j]) || !aligned16(dk_chunks[j]) ||
+            !aligned16(dv_chunks[j]))
+            return fail(RA_ERR_INVALID, "every chunk pointer must be non-null and 16-byte aligned");
+    ra::AttnBwdArgs a;
+    a.q = q;
+    a.k_chunks = k_chunks;
+    a.v_chunks = v_chunks;
+    a.out = out;
+    a.lse = lse;
+    a.dout = dout;
+    a.P = P;
+    a.B = B;
+    a.H_q = H_q;
+    a.H_kv = H_kv;
+    a.Lc = Lc;
+    a.D = D;
+    a.q_bstride = q_bstride;
+    a.kv_bstride = kv_bstride;
+    a.scale = scale;
+    a.causal = causal;
+    a.dq = dq;
+    a.dk_chunks = dk_chunks;
+    a.dv_chunks = dv_chunks;
+    a.workspace = workspace;
+    a.stream = (cudaStream_t)stream;
+    const char* why = "launch failed";
+    cudaError_t e = ra::launch_attn_bwd_sm100(a, g_wait_limit_ns.load(), &why);
+    if (e != cudaSuccess) return cuda_fail(e, why);
+    return RA_OK;
+}
+
 ra_status ra_lse_merge(float* o_a, float* lse_a, const float* o_b, const float* lse_b, int B, int H,
                        long long L, int D, void* stream) {
     if (B < 1 || H < 1 || L < 1 || D < 1) return fail(RA_ERR_INVALID, "sizes must be >= 1");
@@ -203,16 +263,17 @@ ra_status ra_ulysses_head2seq(const void* in, void* out, int P, int B, int Lc, i
 ra_status ra_sync_status(void* stream) {
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
-    unsigned int word = 0, pword = 0;
+    unsigned int word = 0, pword = 0, bword = 0;
     e = ra::read_and_clear_error_word(&word);
     if (e == cudaSuccess) e = ra::read_and_clear_permute_error(&pword);
+    if (e == cudaSuccess) e = ra::read_and_clear_bwd_error(&bword);
     if (e != cudaSuccess) return cuda_fail(e, "reading the kernel error word");
-    word |= pword ? 16u : 0u;
+    word |= (pword ? 16u : 0u) | (bword ? 64u : 0u);
     if (word) {
         char buf[128];
         std::snprintf(buf, sizeof buf,
                       "a kernel gave up on a bounded wait (error bits 0x%x: 1 load, 2 mma, "
-                      "4 softmax, 8 drain, 16 permute)", word);
+                      "4 softmax, 8 drain, 16 permute, 64 backward)", word);
         return fail(RA_ERR_TIMEOUT, buf);
     }
     return RA_OK;

@@ -1,0 +1,749 @@
+// attn_bwd_sm100.cu -- the backward pass of ring-chunked attention on the Blackwell tensor
+// cores (sm_100a): dQ, dK, dV of O = softmax(scale Q K^T) V given dO, with the forward's
+// LSE ("Как работает sequence parallelism в контексте LLM?" trains with ring attention;
+// the gradient is the derivative of the section-5 computation):
+//   P  = exp(scale Q K^T - LSE)        (recomputed from the forward's log-sum-exp)
+//   dP = dO V^T,  Delta = rowsum(dO * O),  dS = P * (dP - Delta)
+//   dQ = scale dS K,   dK = scale dS^T Q,   dV = P^T dO
+// Three kernels: Delta (a row reduction), dQ with the query tile stationary (the chunks
+// visited in the forward's ring order, causal tiles skipped), and dK/dV with the key tile
+// stationary (every query tile of every query head of the kv head's group that can see
+// it).  Each tensor-core kernel keeps its operands for one 128 x 128 tile pair in tensor
+// memory:
+//   dQ kernel   TMEM S [0,128), dP [128,256), dQ [256,256+D); dS (bf16) over S
+//   dK/dV       TMEM S^T [0,128), dP^T [128,256), dV [256,256+D), dK [256+D,256+2D);
+//               P^T (bf16) over S^T, dS^T (bf16) over dP^T
+// Roles (192 threads): warps 0-3 compute P, dS (one TMEM lane = one row each), warp 4
+// loads (TMA), warp 5 issues the MMAs (one thread) and owns tensor memory.  Every wait is
+// bounded: a role that gives up sets the CTA abort flag and this file's error word, every
+// role stops issuing and drains its own work, and the CTA frees its tensor memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <cmath>
+#include <cstdint>
+#include "ra_internal.h"
+#include "attn_sched.cuh"
+#include "sm100_ptx.cuh"
+#include "../../include/ra.h"
+
+namespace ra {
+
+__device__ unsigned int g_bwd_error_word = 0;
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kWarpLoad = 4;
+constexpr int kWarpMma = 5;
+constexpr int kBM = 128;  // query rows per tile
+constexpr int kBN = 128;  // keys per tile
+static_assert(kBN == kSchedTile, "the schedule counts tiles of kBN keys");
+constexpr uint32_t kTmemCols = 512;
+constexpr unsigned kErrLoad = 1u, kErrMma = 2u, kErrCompute = 4u, kErrDrain = 8u;
+
+struct __align__(64) BwdParams {
+    CUtensorMap tm_q;   // [D][H_q][L][B] bf16
+    CUtensorMap tm_do;  // [D][H_q][L][B] bf16
+    CUtensorMap tm_k[RA_MAX_P];
+    CUtensorMap tm_v[RA_MAX_P];
+    const float* lse;    // [B][H_q][L]
+    const float* delta;  // [B][H_q][L]
+    float* dq;           // [B][L][H_q][D]
+    float* dk[RA_MAX_P];  // chunk j: [B][Lc][H_kv][D]
+    float* dv[RA_MAX_P];
+    int P, B, H_q, H_kv, Lc, L, causal, group, n_qblocks, ntc;
+    float scale, scale_log2;
+    unsigned long long wait_limit_ns;
+};
+
+template <int D>
+struct BCfg {
+    static constexpr int TILE = kBM * D * 2;  // bytes of a 128 x D bf16 tile
+    static constexpr int NKB = D / 64;        // 64-column (128-byte) swizzle blocks per tile
+    static constexpr int BLK = kBM * 128;     // bytes of one swizzle block
+    static constexpr int NS = 2;              // ring stages
+    // dQ kernel: Q, dO once; K and V rings.  dK/dV kernel: K, V once; a ring of (Q, dO,
+    // LSE, Delta) stages.
+    static constexpr int OFF_A = 0;                      // Q (dQ) / K (dK/dV)
+    static constexpr int OFF_B = TILE;                   // dO (dQ) / V (dK/dV)
+    static constexpr int OFF_RING = 2 * TILE;            // NS x (two tiles) stages
+    static constexpr int STAGE = 2 * TILE + 2 * kBM * 4; // + LSE and Delta rows (dK/dV)
+    static constexpr int OFF_BAR = OFF_RING + NS * STAGE;
+    // barriers: fixed_full, full[NS], empty[NS], sd_full, ds_full, acc_done, drain
+    static constexpr int N_BARS = 1 + 2 * NS + 4;
+    static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem base, abort flag, n
+    static constexpr int OFF_SCHED = OFF_MISC + 16;
+    static constexpr int SMEM = OFF_SCHED + 2 * RA_MAX_P * 4 + 1024;
+    static constexpr int BAR_FIXED = 0;
+    __host__ __device__ static constexpr int bar_full(int s) { return 1 + s; }
+    __host__ __device__ static constexpr int bar_empty(int s) { return 1 + NS + s; }
+    static constexpr int BAR_SD = 1 + 2 * NS;
+    static constexpr int BAR_DS = 2 + 2 * NS;
+    static constexpr int BAR_ACC = 3 + 2 * NS;
+    static constexpr int BAR_DRAIN = 4 + 2 * NS;
+    static_assert(SMEM <= 232448, "shared memory budget");
+    static_assert(256 + 2 * D <= (int)kTmemCols, "tensor memory budget");
+};
+
+__device__ __forceinline__ void raise_abort(volatile int* abort_flag, unsigned code) {
+    *abort_flag = 1;
+    atomicOr(&g_bwd_error_word, code);
+}
+
+__device__ __forceinline__ bool wait1(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                      unsigned long long limit, unsigned code) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 15u) == 0) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > limit) {
+                raise_abort(abort_flag, code);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                           unsigned long long limit) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 15u) == 0 && global_timer_ns() - t0 > limit) {
+            raise_abort(abort_flag, kErrDrain);
+            return false;
+        }
+    }
+}
+
+// Warp-uniform bounded wait (every lane polls; the give-up decision is lane 0's).
+__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned long long limit, unsigned code) {
+    const unsigned FULL = 0xffffffffu;
+    bool done = mbar_try_wait(bar, parity);
+    if (__all_sync(FULL, done)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (!done) done = mbar_try_wait(bar, parity);
+        if (__all_sync(FULL, done)) return true;
+        if ((it & 15u) == 0) {
+            int stop = 0;
+            if ((threadIdx.x & 31) == 0) {
+                if (*abort_flag) stop = 1;
+                else if (global_timer_ns() - t0 > limit) {
+                    raise_abort(abort_flag, code);
+                    stop = 1;
+                }
+            }
+            if (__shfl_sync(FULL, stop, 0)) return false;
+        }
+    }
+}
+
+// Two 32-column TMEM loads of this thread's lane as 32 fp32 pairs (column 2i low).
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&x)[64]) {
+    uint32_t a[32], b[32];
+    tmem_ld32(taddr, a);
+    tmem_ld32(taddr + 32, b);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        x[i] = __uint_as_float(a[i]);
+        x[32 + i] = __uint_as_float(b[i]);
+    }
+}
+
+// ------------------------------------------------------------------ Delta = rowsum(dO * O)
+// One warp per (b, t, h) row, fp32 accumulation of the bf16 products.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_delta_kernel(const uint16_t* __restrict__ out,
+                                                        const uint16_t* __restrict__ dout,
+                                                        float* __restrict__ delta, int B, int L,
+                                                        int H) {
+    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= (long long)B * L * H) return;
+    const uint16_t* o = out + row * D;
+    const uint16_t* g = dout + row * D;
+    float acc = 0.f;
+#pragma unroll
+    for (int i = lane; i < D; i += 32)
+        acc = fmaf(__uint_as_float((uint32_t)o[i] << 16), __uint_as_float((uint32_t)g[i] << 16), acc);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) {
+        const long long t = (row / H) % L, h = row % H, b = row / H / L;
+        delta[(b * H + h) * L + t] = acc;
+    }
+}
+
+// ------------------------------------------------------------------ dQ (query tile stationary)
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constant__ BwdParams p) {
+    using C = BCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint32_t base = smem_u32(smem_raw);
+    const uint32_t pad = (1024u - (base & 1023u)) & 1023u;
+    base += pad;
+    uint8_t* smem = smem_raw + pad;
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+    volatile int* n_slot = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
+    uint32_t* sched_range = reinterpret_cast<uint32_t*>(smem + C::OFF_SCHED);
+    auto bar = [&](int i) { return base + C::OFF_BAR + 8u * (uint32_t)i; };
+    const unsigned long long lim = p.wait_limit_ns;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // grid: (batch, kv head) outermost, then row blocks heaviest first, then the query
+    // heads of the group (they read the same K/V tiles)
+    const int per_bg = p.n_qblocks * p.group;
+    const int bg = (int)(blockIdx.x / per_bg), rem = (int)(blockIdx.x % per_bg);
+    const int b = bg / p.H_kv, g = bg % p.H_kv;
+    const int h = g * p.group + rem % p.group;
+    const int r0 = (p.n_qblocks - 1 - rem / p.group) * kBM;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(C::BAR_FIXED), 1);
+        for (int s = 0; s < C::NS; ++s) {
+            mbar_init(bar(C::bar_full(s)), 1);
+            mbar_init(bar(C::bar_empty(s)), 1);
+        }
+        mbar_init(bar(C::BAR_SD), 1);
+        mbar_init(bar(C::BAR_DS), 4 * 32);
+        mbar_init(bar(C::BAR_ACC), 1);
+        mbar_init(bar(C::BAR_DRAIN), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == kWarpLoad) {
+        SchedArgs sa;
+        sa.P = p.P; sa.Lc = p.Lc; sa.L = p.L; sa.causal = p.causal; sa.zigzag = 0; sa.pid = nullptr;
+        const long long last_row = min((long long)r0 + kBM - 1, (long long)p.L - 1);
+        const int nt = make_schedule(sa, b, r0, last_row, sched_range);
+        if (lane == 0) *n_slot = nt;
+    }
+    if (warp == kWarpMma) {
+        __syncwarp();
+        tmem_alloc(base + C::OFF_MISC, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    Sched sched;
+    sched.range = sched_range;
+    sched.P = p.P;
+    sched.i0 = r0 / p.Lc;
+    const int n = *n_slot;
+
+    if (warp == kWarpLoad) {
+        if (lane == 0) {
+            // Q and dO once; K and V of each visited tile through an NS-deep ring
+            mbar_arrive_expect_tx(bar(C::BAR_FIXED), 2 * C::TILE);
+            for (int kb = 0; kb < C::NKB; ++kb) {
+                tma_load_4d(base + C::OFF_A + kb * C::BLK, &p.tm_q, bar(C::BAR_FIXED), kb * 64, h, r0, b);
+                tma_load_4d(base + C::OFF_B + kb * C::BLK, &p.tm_do, bar(C::BAR_FIXED), kb * 64, h, r0, b);
+            }
+            int armed[C::NS];
+            for (int s = 0; s < C::NS; ++s) armed[s] = -1;
+            SchedIter it;
+            it.begin(sched);
+            for (int jt = 0; jt < n; ++jt, it.next()) {
+                const int slot = jt % C::NS;
+                if (jt >= C::NS &&
+                    !wait1(bar(C::bar_empty(slot)), ((jt / C::NS) - 1) & 1, abort_flag, lim, kErrLoad))
+                    break;
+                const uint32_t st = base + C::OFF_RING + slot * C::STAGE;
+                mbar_arrive_expect_tx(bar(C::bar_full(slot)), 2 * C::TILE);
+                for (int kb = 0; kb < C::NKB; ++kb) {
+                    tma_load_4d(st + kb * C::BLK, &p.tm_k[it.chunk()], bar(C::bar_full(slot)),
+                                kb * 64, g, it.t * kBN, b);
+                    tma_load_4d(st + C::TILE + kb * C::BLK, &p.tm_v[it.chunk()],
+                                bar(C::bar_full(slot)), kb * 64, g, it.t * kBN, b);
+                }
+                armed[slot] = jt;
+            }
+            wait_drain(bar(C::BAR_FIXED), 0, abort_flag, lim);
+            for (int s = 0; s < C::NS; ++s)
+                if (armed[s] >= 0) wait_drain(bar(C::bar_full(s)), (armed[s] / C::NS) & 1, abort_flag, lim);
+        }
+    } else if (warp == kWarpMma) {
+        if (lane == 0) {
+            constexpr uint32_t IDESC_S = idesc_bf16_f32(kBM, kBN, 0);  // K-major A and B
+            constexpr uint32_t IDESC_O = idesc_bf16_f32(kBM, D, 1);    // B MN-major (D contiguous)
+            const uint64_t dq_ = desc_sw128(base + C::OFF_A, 16, 1024);
+            const uint64_t ddo = desc_sw128(base + C::OFF_B, 16, 1024);
+            bool issued = false;
+            if (wait1(bar(C::BAR_FIXED), 0, abort_flag, lim, kErrMma)) {
+                for (int jt = 0; jt < n; ++jt) {
+                    const int slot = jt % C::NS;
+                    if (!wait1(bar(C::bar_full(slot)), (jt / C::NS) & 1, abort_flag, lim, kErrMma)) break;
+                    tc_fence_after();
+                    const uint32_t st = base + C::OFF_RING + slot * C::STAGE;
+                    const uint64_t dk = desc_sw128(st, 16, 1024);
+                    const uint64_t dv = desc_sw128(st + C::TILE, 16, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = ((kk / 4) * C::BLK + (kk % 4) * 32) >> 4;
+                        mma_ss(tmem + 0, dq_ + off, dk + off, IDESC_S, kk > 0 ? 1u : 0u);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = ((kk / 4) * C::BLK + (kk % 4) * 32) >> 4;
+                        mma_ss(tmem + 128, ddo + off, dv + off, IDESC_S, kk > 0 ? 1u : 0u);
+                    }
+                    tc_commit(bar(C::BAR_SD));
+                    issued = true;
+                    if (!wait1(bar(C::BAR_DS), jt & 1, abort_flag, lim, kErrMma)) break;
+                    tc_fence_after();
+                    // dQ += dS K: dS (bf16 pairs) over S's first 64 columns, K as MN-major B
+                    const uint64_t dkm = desc_sw128(st, C::BLK, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < kBN / 16; ++kk)
+                        mma_ts(tmem + 256, tmem + kk * 8, dkm + (uint64_t)((kk * 2048) >> 4), IDESC_O,
+                               (jt > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(bar(C::bar_empty(slot)));
+                }
+            }
+            if (issued) {
+                tc_commit(bar(C::BAR_ACC));
+                tc_commit(bar(C::BAR_DRAIN));
+                wait_drain(bar(C::BAR_DRAIN), 0, abort_flag, lim);
+            }
+        }
+    } else {
+        // compute warps: P and dS for this thread's row
+        const unsigned FULL = 0xffffffffu;
+        const int wr = warp;
+        const int row_t = wr * 32 + lane;
+        const long long my_row = (long long)r0 + row_t;
+        const bool row_ok = my_row < p.L;
+        const uint32_t lane_off = (uint32_t)(wr * 32) << 16;
+        const long long lrow = ((long long)b * p.H_q + h) * p.L + (row_ok ? my_row : 0);
+        // rows past L see nothing (lse2 = +inf makes every probability 0)
+        const float lse2 = row_ok ? p.lse[lrow] * 1.4426950408889634f : INFINITY;
+        const float dlt = row_ok ? p.delta[lrow] : 0.f;
+        const float sl2 = p.scale_log2;
+        bool ok = true;
+        SchedIter it;
+        it.begin(sched);
+        for (int jt = 0; jt < n; ++jt, it.next()) {
+            if (!wait_warp(bar(C::BAR_SD), jt & 1, abort_flag, lim, kErrCompute)) {
+                ok = false;
+                break;
+            }
+            __syncwarp();
+            tc_fence_after();
+            const long long k0 = (long long)it.chunk() * p.Lc + (long long)it.t * kBN;
+            const int kvalid = min(kBN, p.Lc - it.t * kBN);
+            const long long lim_c = p.causal ? my_row - k0 : (long long)kBN;  // keys c <= lim_c
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                float s[64], dp[64];
+                tmem_ld64(tmem + lane_off + 64 * c, s);
+                tmem_ld64(tmem + lane_off + 128 + 64 * c, dp);
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    float ds2[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int col = 64 * c + 2 * i + e;
+                        const bool vis = col < kvalid && col <= lim_c;
+                        const float pr = vis ? ex2_approx(s[2 * i + e] * sl2 - lse2) : 0.f;
+                        ds2[e] = pr * (dp[2 * i + e] - dlt);
+                    }
+                    pk[i] = pack_bf16x2(ds2[0], ds2[1]);
+                }
+                tmem_st32(tmem + lane_off + 32 * c, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(C::BAR_DS));
+        }
+        (void)FULL;
+        if (ok && n > 0 && wait_warp(bar(C::BAR_ACC), 0, abort_flag, lim, kErrCompute)) {
+            __syncwarp();
+            tc_fence_after();
+#pragma unroll
+            for (int cb = 0; cb < D / 32; ++cb) {
+                uint32_t o[32];
+                tmem_ld32(tmem + lane_off + 256 + cb * 32, o);
+                tmem_wait_ld();
+                if (row_ok) {
+                    float4* dst = reinterpret_cast<float4*>(
+                        p.dq + (((long long)b * p.L + my_row) * p.H_q + h) * D + cb * 32);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        dst[i] = make_float4(__uint_as_float(o[4 * i]) * p.scale,
+                                             __uint_as_float(o[4 * i + 1]) * p.scale,
+                                             __uint_as_float(o[4 * i + 2]) * p.scale,
+                                             __uint_as_float(o[4 * i + 3]) * p.scale);
+                }
+            }
+        } else if (ok && n == 0 && row_ok) {
+            float4* dst = reinterpret_cast<float4*>(p.dq + (((long long)b * p.L + my_row) * p.H_q + h) * D);
+            for (int i = 0; i < D / 4; ++i) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kWarpMma) {
+        __syncwarp();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------ dK, dV (key tile stationary)
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_sm100(const __grid_constant__ BwdParams p) {
+    using C = BCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint32_t base = smem_u32(smem_raw);
+    const uint32_t pad = (1024u - (base & 1023u)) & 1023u;
+    base += pad;
+    uint8_t* smem = smem_raw + pad;
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+    auto bar = [&](int i) { return base + C::OFF_BAR + 8u * (uint32_t)i; };
+    const unsigned long long lim = p.wait_limit_ns;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // grid: (batch, kv head) outermost, then the key tiles (chunk j, tile t) heaviest first
+    // (causal: the first keys are seen by the most query rows)
+    const int n_kt = p.P * p.ntc;
+    const int bg = (int)(blockIdx.x / n_kt), kt = (int)(blockIdx.x % n_kt);
+    const int b = bg / p.H_kv, g = bg % p.H_kv;
+    const int j = kt / p.ntc, t = kt % p.ntc;
+    const long long key0 = (long long)j * p.Lc + (long long)t * kBN;  // sequence position
+    const int kvalid = min(kBN, p.Lc - t * kBN);
+    // query tiles that can see a key of this tile: rows >= key0 when causal
+    const int qt0 = p.causal ? (int)(key0 / kBM) : 0;
+    const int n_qt = p.n_qblocks - qt0;
+    const int n = n_qt * p.group;  // (head, query tile) pairs, head-major
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(C::BAR_FIXED), 1);
+        for (int s = 0; s < C::NS; ++s) {
+            mbar_init(bar(C::bar_full(s)), 1 + 1);  // the load thread's expect_tx + the LSE/Delta rows
+            mbar_init(bar(C::bar_empty(s)), 1);
+        }
+        mbar_init(bar(C::BAR_SD), 1);
+        mbar_init(bar(C::BAR_DS), 4 * 32);
+        mbar_init(bar(C::BAR_ACC), 1);
+        mbar_init(bar(C::BAR_DRAIN), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == kWarpMma) {
+        __syncwarp();
+        tmem_alloc(base + C::OFF_MISC, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == kWarpLoad) {
+        // K and V once; per (head, query tile): Q, dO (TMA) and the 128 LSE / Delta values
+        // (plain loads by the whole warp, rows past L as +inf / 0) into one ring stage
+        if (lane == 0) {
+            mbar_arrive_expect_tx(bar(C::BAR_FIXED), 2 * C::TILE);
+            for (int kb = 0; kb < C::NKB; ++kb) {
+                tma_load_4d(base + C::OFF_A + kb * C::BLK, &p.tm_k[j], bar(C::BAR_FIXED), kb * 64, g, t * kBN, b);
+                tma_load_4d(base + C::OFF_B + kb * C::BLK, &p.tm_v[j], bar(C::BAR_FIXED), kb * 64, g, t * kBN, b);
+            }
+        }
+        int armed[C::NS];
+        for (int s = 0; s < C::NS; ++s) armed[s] = -1;
+        for (int it = 0; it < n; ++it) {
+            const int slot = it % C::NS;
+            const int h = g * p.group + it / n_qt;
+            const int q0 = (qt0 + it % n_qt) * kBM;
+            if (it >= C::NS &&
+                !wait_warp(bar(C::bar_empty(slot)), ((it / C::NS) - 1) & 1, abort_flag, lim, kErrLoad))
+                break;
+            const uint32_t st = base + C::OFF_RING + slot * C::STAGE;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar(C::bar_full(slot)), 2 * C::TILE);
+                for (int kb = 0; kb < C::NKB; ++kb) {
+                    tma_load_4d(st + kb * C::BLK, &p.tm_q, bar(C::bar_full(slot)), kb * 64, h, q0, b);
+                    tma_load_4d(st + C::TILE + kb * C::BLK, &p.tm_do, bar(C::bar_full(slot)), kb * 64, h, q0, b);
+                }
+            }
+            float* rows = reinterpret_cast<float*>(smem + C::OFF_RING + slot * C::STAGE + 2 * C::TILE);
+            const long long lbase = ((long long)b * p.H_q + h) * p.L;
+            for (int r = lane; r < kBM; r += 32) {
+                const long long row = (long long)q0 + r;
+                rows[r] = row < p.L ? p.lse[lbase + row] * 1.4426950408889634f : INFINITY;
+                rows[kBM + r] = row < p.L ? p.delta[lbase + row] : 0.f;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::bar_full(slot)));
+            armed[slot] = it;
+        }
+        if (lane == 0) {
+            wait_drain(bar(C::BAR_FIXED), 0, abort_flag, lim);
+            for (int s = 0; s < C::NS; ++s)
+                if (armed[s] >= 0) wait_drain(bar(C::bar_full(s)), (armed[s] / C::NS) & 1, abort_flag, lim);
+        }
+    } else if (warp == kWarpMma) {
+        if (lane == 0) {
+            constexpr uint32_t IDESC_S = idesc_bf16_f32(kBN, kBM, 0);  // K-major A and B
+            constexpr uint32_t IDESC_O = idesc_bf16_f32(kBN, D, 1);    // B MN-major (D contiguous)
+            const uint64_t dk_ = desc_sw128(base + C::OFF_A, 16, 1024);
+            const uint64_t dv_ = desc_sw128(base + C::OFF_B, 16, 1024);
+            bool issued = false;
+            if (wait1(bar(C::BAR_FIXED), 0, abort_flag, lim, kErrMma)) {
+                for (int it = 0; it < n; ++it) {
+                    const int slot = it % C::NS;
+                    if (!wait1(bar(C::bar_full(slot)), (it / C::NS) & 1, abort_flag, lim, kErrMma)) break;
+                    tc_fence_after();
+                    const uint32_t st = base + C::OFF_RING + slot * C::STAGE;
+                    const uint64_t dq_ = desc_sw128(st, 16, 1024);
+                    const uint64_t ddo = desc_sw128(st + C::TILE, 16, 1024);
+                    // S^T = K Q^T, dP^T = V dO^T (keys are the TMEM lanes)
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = ((kk / 4) * C::BLK + (kk % 4) * 32) >> 4;
+                        mma_ss(tmem + 0, dk_ + off, dq_ + off, IDESC_S, kk > 0 ? 1u : 0u);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = ((kk / 4) * C::BLK + (kk % 4) * 32) >> 4;
+                        mma_ss(tmem + 128, dv_ + off, ddo + off, IDESC_S, kk > 0 ? 1u : 0u);
+                    }
+                    tc_commit(bar(C::BAR_SD));
+                    issued = true;
+                    if (!wait1(bar(C::BAR_DS), it & 1, abort_flag, lim, kErrMma)) break;
+                    tc_fence_after();
+                    // dV += P^T dO and dK += dS^T Q; P^T over S^T, dS^T over dP^T; Q and dO
+                    // as MN-major B (D contiguous, query rows 128 bytes apart)
+                    const uint64_t dom = desc_sw128(st + C::TILE, C::BLK, 1024);
+                    const uint64_t qm = desc_sw128(st, C::BLK, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < kBM / 16; ++kk)
+                        mma_ts(tmem + 256, tmem + kk * 8, dom + (uint64_t)((kk * 2048) >> 4), IDESC_O,
+                               (it > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                    for (int kk = 0; kk < kBM / 16; ++kk)
+                        mma_ts(tmem + 256 + D, tmem + 128 + kk * 8, qm + (uint64_t)((kk * 2048) >> 4),
+                               IDESC_O, (it > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(bar(C::bar_empty(slot)));
+                }
+            }
+            if (issued) {
+                tc_commit(bar(C::BAR_ACC));
+                tc_commit(bar(C::BAR_DRAIN));
+                wait_drain(bar(C::BAR_DRAIN), 0, abort_flag, lim);
+            }
+        }
+    } else {
+        // compute warps: P^T and dS^T for this thread's key against the tile's 128 queries
+        const int wr = warp;
+        const int key_t = wr * 32 + lane;
+        const bool key_ok = key_t < kvalid;
+        const long long my_kpos = key0 + key_t;
+        const uint32_t lane_off = (uint32_t)(wr * 32) << 16;
+        const float sl2 = p.scale_log2;
+        bool ok = true;
+        for (int it = 0; it < n; ++it) {
+            const int slot = it % C::NS;
+            const int q0 = (qt0 + it % n_qt) * kBM;
+            if (!wait_warp(bar(C::BAR_SD), it & 1, abort_flag, lim, kErrCompute)) {
+                ok = false;
+                break;
+            }
+            __syncwarp();
+            tc_fence_after();
+            const float* rows = reinterpret_cast<const float*>(smem + C::OFF_RING + slot * C::STAGE + 2 * C::TILE);
+            // queries c of the tile see this key when q0 + c >= key position (causal)
+            const long long lo_c = p.causal ? my_kpos - q0 : 0;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                float s[64], dp[64];
+                tmem_ld64(tmem + lane_off + 64 * c, s);
+                tmem_ld64(tmem + lane_off + 128 + 64 * c, dp);
+                uint32_t pp[32], pd[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    float pr2[2], ds2[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int col = 64 * c + 2 * i + e;
+                        const bool vis = key_ok && col >= lo_c;
+                        const float pr = vis ? ex2_approx(s[2 * i + e] * sl2 - rows[col]) : 0.f;
+                        pr2[e] = pr;
+                        ds2[e] = pr * (dp[2 * i + e] - rows[kBM + col]);
+                    }
+                    pp[i] = pack_bf16x2(pr2[0], pr2[1]);
+                    pd[i] = pack_bf16x2(ds2[0], ds2[1]);
+                }
+                tmem_st32(tmem + lane_off + 32 * c, pp);
+                tmem_st32(tmem + lane_off + 128 + 32 * c, pd);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(C::BAR_DS));
+        }
+        if (ok && n > 0 && wait_warp(bar(C::BAR_ACC), 0, abort_flag, lim, kErrCompute)) {
+            __syncwarp();
+            tc_fence_after();
+            const long long orow = (((long long)b * p.Lc + t * kBN + key_t) * p.H_kv + g) * D;
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK (times scale)
+                const float mul = which ? p.scale : 1.f;
+                float* outp = which ? p.dk[j] : p.dv[j];
+#pragma unroll
+                for (int cb = 0; cb < D / 32; ++cb) {
+                    uint32_t o[32];
+                    tmem_ld32(tmem + lane_off + 256 + which * D + cb * 32, o);
+                    tmem_wait_ld();
+                    if (key_ok) {
+                        float4* dst = reinterpret_cast<float4*>(outp + orow + cb * 32);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            dst[i] = make_float4(__uint_as_float(o[4 * i]) * mul,
+                                                 __uint_as_float(o[4 * i + 1]) * mul,
+                                                 __uint_as_float(o[4 * i + 2]) * mul,
+                                                 __uint_as_float(o[4 * i + 3]) * mul);
+                    }
+                }
+            }
+        } else if (ok && n == 0 && key_ok) {
+            const long long orow = (((long long)b * p.Lc + t * kBN + key_t) * p.H_kv + g) * D;
+            for (int i = 0; i < D; ++i) p.dk[j][orow + i] = p.dv[j][orow + i] = 0.f;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kWarpMma) {
+        __syncwarp();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 bwd_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// [D][H][rows][B] bf16 tensor, 128-row x 64-column boxes, 128-byte swizzle, zero fill.
+bool bwd_tile_map(CUtensorMap* m, const void* ptr, int D, int H, long long rows, int B,
+                  long long bstride_elems) {
+    auto enc = bwd_encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)bstride_elems * 2};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)kBM, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch_bwd_d(const BwdParams& p, const AttnBwdArgs& a) {
+    using C = BCfg<D>;
+    static int configured_for = -1;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (configured_for != dev) {
+        e = cudaFuncSetAttribute(bwd_dq_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(bwd_dkdv_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (e != cudaSuccess) return e;
+        configured_for = dev;
+    }
+    const long long rows = (long long)a.B * p.L * a.H_q;
+    bwd_delta_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, a.stream>>>(
+        (const uint16_t*)a.out, (const uint16_t*)a.dout, a.workspace, a.B, p.L, a.H_q);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const long long grid_q = (long long)p.n_qblocks * a.B * a.H_q;
+    const long long grid_k = (long long)a.B * a.H_kv * a.P * p.ntc;
+    bwd_dq_sm100<D><<<(unsigned)grid_q, kThreads, C::SMEM, a.stream>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    bwd_dkdv_sm100<D><<<(unsigned)grid_k, kThreads, C::SMEM, a.stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_bwd_sm100(const AttnBwdArgs& a, unsigned long long wait_limit_ns,
+                                  const char** why) {
+    static thread_local BwdParams p;
+    const long long L = (long long)a.P * a.Lc;
+    if (!bwd_tile_map(&p.tm_q, a.q, a.D, a.H_q, L, a.B, a.q_bstride) ||
+        !bwd_tile_map(&p.tm_do, a.dout, a.D, a.H_q, L, a.B, L * a.H_q * a.D)) {
+        *why = "cuTensorMapEncodeTiled failed for q or dout";
+        return cudaErrorInvalidValue;
+    }
+    for (int j = 0; j < a.P; ++j) {
+        if (!bwd_tile_map(&p.tm_k[j], a.k_chunks[j], a.D, a.H_kv, a.Lc, a.B, a.kv_bstride) ||
+            !bwd_tile_map(&p.tm_v[j], a.v_chunks[j], a.D, a.H_kv, a.Lc, a.B, a.kv_bstride)) {
+            *why = "cuTensorMapEncodeTiled failed for a K/V chunk";
+            return cudaErrorInvalidValue;
+        }
+        p.dk[j] = a.dk_chunks[j];
+        p.dv[j] = a.dv_chunks[j];
+    }
+    p.lse = a.lse;
+    p.delta = a.workspace;
+    p.dq = a.dq;
+    p.P = a.P;
+    p.B = a.B;
+    p.H_q = a.H_q;
+    p.H_kv = a.H_kv;
+    p.Lc = a.Lc;
+    p.L = (int)L;
+    p.causal = a.causal;
+    p.group = a.H_q / a.H_kv;
+    p.n_qblocks = (int)((L + kBM - 1) / kBM);
+    p.ntc = (a.Lc + kBN - 1) / kBN;
+    p.scale = a.scale;
+    p.scale_log2 = (float)((double)a.scale * 1.4426950408889634);
+    p.wait_limit_ns = wait_limit_ns;
+    if ((long long)p.n_qblocks * a.B * a.H_q > 0x7fffffffLL) {
+        *why = "problem too large for one launch";
+        return cudaErrorInvalidValue;
+    }
+    if (a.D == 128) return launch_bwd_d<128>(p, a);
+    if (a.D == 64) return launch_bwd_d<64>(p, a);
+    *why = "head dimension not supported by the tensor-core backward";
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t read_and_clear_bwd_error(unsigned int* value) {
+    cudaError_t e = cudaMemcpyFromSymbol(value, g_bwd_error_word, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    if (*value) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_bwd_error_word, &zero, sizeof(unsigned int));
+    }
+    return e;
+}
+
+}  // namespace ra

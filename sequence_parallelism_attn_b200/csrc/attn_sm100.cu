@@ -48,6 +48,7 @@
 #include <cmath>
 #include <cstdint>
 #include "ra_internal.h"
+#include "attn_sched.cuh"
 #include "sm100_ptx.cuh"
 #include "../../include/ra.h"
 
@@ -65,6 +66,7 @@ constexpr int kWarpLoadV = 10;
 constexpr int kWarpIdle = 11;  // fills the CTA's schedule in the prologue
 constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 128;  // keys per tile
+static_assert(kBN == kSchedTile, "the schedule counts tiles of kBN keys");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -118,83 +120,6 @@ struct Cfg {
     static constexpr uint32_t S_COL0 = 0, S_COL1 = 128;
     static constexpr uint32_t O_COL0 = 256, O_COL1 = 256 + D;
     static_assert(SMEM <= 232448, "shared memory budget");
-};
-
-// The chunk/tile visiting order of one CTA: chunks in ring order j = (i0 - s) mod P, and
-// of chunk j the tiles [range[j], range[RA_MAX_P + j]) (filled once per CTA into shared
-// memory by make_schedule).
-struct Sched {
-    const uint32_t* range;
-    int P, i0;
-};
-
-// One warp fills the schedule of a CTA whose rows are r0 .. last_row (rank-major) of batch
-// b: for every chunk j the 128-key tiles holding a key the rows may see.  Causal: keys at
-// positions up to the largest row position (a prefix of the shard, positions increase
-// along it).  Packed samples (position_ids, contiguous layout): keys from the smallest
-// sample start among the rows on (row r's sample starts at r - position_ids[r], clamped
-// to [0, r]).  Returns the number of tiles (in every lane).
-__device__ __forceinline__ int make_schedule(const AttnParams& p, int b, long long r0,
-                                             long long last_row, uint32_t* range) {
-    const int lane = threadIdx.x & 31;
-    const int ntc = (p.Lc + kBN - 1) / kBN;
-    long long qmin, qmax;
-    row_pos_range(p.zigzag, p.P, p.Lc, r0, last_row, qmin, qmax);
-    long long smin = p.pid ? last_row : 0;
-    if (p.pid)
-        for (long long r = r0 + lane; r <= last_row; r += 32) {
-            const long long st = r - (long long)p.pid[(long long)b * p.L + r];
-            smin = min(smin, st < 0 ? 0 : (st > r ? r : st));
-        }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) smin = min(smin, __shfl_xor_sync(0xffffffffu, smin, off));
-    int n = 0;
-    for (int j = lane; j < p.P; j += 32) {
-        long long t_hi = ntc;
-        if (p.causal) {
-            const long long nk = shard_prefix(p.zigzag, p.P, p.Lc, j, qmax);
-            t_hi = min((nk + kBN - 1) / kBN, (long long)ntc);
-        }
-        const long long k0 = (long long)j * p.Lc;
-        long long t_lo = smin > k0 ? min((smin - k0) / kBN, (long long)ntc) : 0;
-        t_lo = min(t_lo, t_hi);
-        range[j] = (uint32_t)t_lo;
-        range[RA_MAX_P + j] = (uint32_t)t_hi;
-        n += (int)(t_hi - t_lo);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) n += __shfl_xor_sync(0xffffffffu, n, off);
-    return n;
-}
-
-// Walks the schedule tile by tile; the chunk index is recomputed only when the step s
-// changes, so a tile costs no integer division.
-struct SchedIter {
-    Sched S;
-    int s, t, nt, j;
-    __device__ void load_chunk() {
-        j = (S.i0 - s) % S.P;
-        j = j < 0 ? j + S.P : j;
-        t = (int)S.range[j];
-        nt = (int)S.range[RA_MAX_P + j];
-    }
-    __device__ void begin(const Sched& sched) {
-        S = sched;
-        s = 0;
-        load_chunk();
-        skip_empty();
-    }
-    __device__ void skip_empty() {
-        while (s < S.P && t >= nt) {
-            ++s;
-            if (s < S.P) load_chunk();
-        }
-    }
-    __device__ void next() {
-        ++t;
-        skip_empty();
-    }
-    __device__ int chunk() const { return j; }
 };
 
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag, unsigned code) {
@@ -646,7 +571,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100(const __grid_const
     volatile int* n_slot = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
     if (warp == kWarpIdle) {
         const long long last_row = min((long long)r0 + 2 * kBM - 1, (long long)p.L - 1);
-        const int nt = make_schedule(p, b, r0, last_row, sched_range);
+        SchedArgs sa;
+        sa.P = p.P;
+        sa.Lc = p.Lc;
+        sa.L = p.L;
+        sa.causal = p.causal;
+        sa.zigzag = p.zigzag;
+        sa.pid = p.pid;
+        const int nt = make_schedule(sa, b, r0, last_row, sched_range);
         if (lane == 0) *n_slot = nt;
     }
     if (warp == kWarpMma) {

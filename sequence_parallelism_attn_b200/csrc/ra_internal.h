@@ -39,6 +39,25 @@ struct AttnArgs {
     cudaStream_t stream;
 };
 
+// The backward pass: gradients of the forward's O given dO, with its LSE.
+struct AttnBwdArgs {
+    const void* q;                // [B][P*Lc][H_q][D] bf16, batch stride q_bstride
+    const void* const* k_chunks;  // host array, P entries, [B][Lc][H_kv][D] bf16
+    const void* const* v_chunks;
+    const void* out;              // [B][P*Lc][H_q][D] bf16, dense (the forward's O)
+    const float* lse;             // [B][H_q][P*Lc]
+    const void* dout;             // [B][P*Lc][H_q][D] bf16, dense
+    int P, B, H_q, H_kv, Lc, D;
+    long long q_bstride, kv_bstride;
+    float scale;
+    int causal;
+    float* dq;                    // [B][P*Lc][H_q][D] fp32, dense
+    float* const* dk_chunks;      // host array, P entries, [B][Lc][H_kv][D] fp32, dense
+    float* const* dv_chunks;
+    float* workspace;             // [B][H_q][P*Lc] fp32 (rowsum(dO * O))
+    cudaStream_t stream;
+};
+
 // ---- sequence positions of the shard layouts ("Как работает sequence parallelism в
 // контексте LLM?", section 2: rank i owns the contiguous tokens i*Lc .. i*Lc+Lc-1; the
 // zigzag layout, named beside the ring in "Метод контекстного параллелизма Ulysses",
@@ -104,6 +123,10 @@ cudaError_t launch_seq2head(const void* in, void* out, int P, int G, int B, int 
                             unsigned long long wait_limit_ns);
 cudaError_t launch_head2seq(const void* in, void* out, int P, int G, int B, int Lc, int H, int D,
                             int esize, cudaStream_t s, unsigned long long wait_limit_ns);
+// Tensor-core backward for bf16 inputs, D in {64, 128}: Delta, dQ, then dK/dV.
+cudaError_t launch_attn_bwd_sm100(const AttnBwdArgs& a, unsigned long long wait_limit_ns,
+                                  const char** why);
+cudaError_t read_and_clear_bwd_error(unsigned int* value);
 // Read and clear the per-device kernel error word (after the caller synchronised).
 cudaError_t read_and_clear_error_word(unsigned int* value);
 cudaError_t read_and_clear_permute_error(unsigned int* value);

@@ -19,6 +19,7 @@ RA_OK, RA_ERR_INVALID, RA_ERR_UNSUPPORTED, RA_ERR_CUDA, RA_ERR_TIMEOUT = 0, 1, 2
 RA_BF16, RA_FP32 = 0, 1
 RA_MAX_P = 64
 EXPORTED = ("ra_ring_attn_fwd", "ra_ring_attn_fwd_zigzag", "ra_ring_attn_fwd_packed",
+            "ra_ring_attn_bwd",
             "ra_lse_merge", "ra_ulysses_seq2head", "ra_ulysses_head2seq",
             "ra_ulysses_seq2head_grouped", "ra_ulysses_head2seq_grouped",
             "ra_sync_status", "ra_last_error", "ra_set_wait_limit_ns", "ra_debug_inject_stall",
@@ -47,6 +48,8 @@ def load() -> ctypes.CDLL:
     lib.ra_ring_attn_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i64, i64, f32, i32,
                                      i32, i32, vp, vp, vp]
     lib.ra_ring_attn_fwd_zigzag.argtypes = lib.ra_ring_attn_fwd.argtypes
+    lib.ra_ring_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i64,
+                                     i64, f32, i32, vp, vp, vp, vp, vp]
     lib.ra_ring_attn_fwd_packed.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i64, i64,
                                             f32, i32, i32, vp, vp, vp]
     lib.ra_lse_merge.argtypes = [vp, vp, vp, vp, i32, i32, i64, i32, vp]
@@ -55,7 +58,8 @@ def load() -> ctypes.CDLL:
     lib.ra_ulysses_seq2head_grouped.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp]
     lib.ra_ulysses_head2seq_grouped.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, vp]
     lib.ra_sync_status.argtypes = [vp]
-    for f in ("ra_ring_attn_fwd", "ra_ring_attn_fwd_zigzag", "ra_ring_attn_fwd_packed", "ra_lse_merge",
+    for f in ("ra_ring_attn_fwd", "ra_ring_attn_fwd_zigzag", "ra_ring_attn_fwd_packed",
+              "ra_ring_attn_bwd", "ra_lse_merge",
               "ra_ulysses_seq2head", "ra_ulysses_head2seq", "ra_ulysses_seq2head_grouped",
               "ra_ulysses_head2seq_grouped", "ra_sync_status"):
         getattr(lib, f).restype = ctypes.c_int
@@ -121,6 +125,49 @@ def ra_ring_attn_fwd_packed(q_ptr, k_ptrs, v_ptrs, pid_ptr, P, B, H_q, H_kv, Lc,
     _check(load().ra_ring_attn_fwd_packed(q_ptr, ks, vs, pid_ptr, P, B, H_q, H_kv, Lc, D,
                                           q_bstride, kv_bstride, scale, in_dtype, out_dtype,
                                           out_ptr, lse_ptr, stream))
+
+
+def ra_ring_attn_bwd(q_ptr, k_ptrs, v_ptrs, out_ptr, lse_ptr, dout_ptr, P, B, H_q, H_kv, Lc, D,
+                     q_bstride, kv_bstride, scale, causal, dq_ptr, dk_ptrs, dv_ptrs, ws_ptr,
+                     stream):
+    """The backward C entry point with raw pointers (chunk pointer lists of length P)."""
+    arr = ctypes.c_void_p * P
+    _check(load().ra_ring_attn_bwd(q_ptr, arr(*k_ptrs), arr(*v_ptrs), out_ptr, lse_ptr, dout_ptr,
+                                   P, B, H_q, H_kv, Lc, D, q_bstride, kv_bstride, scale,
+                                   int(causal), dq_ptr, arr(*dk_ptrs), arr(*dv_ptrs), ws_ptr,
+                                   stream))
+
+
+def ring_attn_bwd(q: torch.Tensor, k_chunks: torch.Tensor, v_chunks: torch.Tensor,
+                  out: torch.Tensor, lse: torch.Tensor, dout: torch.Tensor, causal: bool,
+                  scale: float | None = None, dq: torch.Tensor | None = None,
+                  dk: torch.Tensor | None = None, dv: torch.Tensor | None = None,
+                  workspace: torch.Tensor | None = None, stream=None):
+    """Gradients of ring_attn_fwd: q/out/dout [B, P*Lc, H_q, D] bf16 (dense), k/v chunks
+    [P, B, Lc, H_kv, D] bf16, lse [B, H_q, P*Lc] fp32.  Returns (dq [B, P*Lc, H_q, D],
+    dk, dv [P, B, Lc, H_kv, D]) in fp32; the fp32 workspace [B, H_q, P*Lc] is allocated
+    here when not given (the library itself allocates nothing)."""
+    P, B, Lc, H_kv, D = k_chunks.shape
+    _, L, H_q, _ = q.shape
+    assert L == P * Lc and q.is_contiguous() and out.is_contiguous() and dout.is_contiguous()
+    assert k_chunks.is_contiguous() and v_chunks.is_contiguous()
+    if scale is None:
+        scale = D ** -0.5
+    dev = q.device
+    if dq is None:
+        dq = torch.empty((B, L, H_q, D), dtype=torch.float32, device=dev)
+    if dk is None:
+        dk = torch.empty((P, B, Lc, H_kv, D), dtype=torch.float32, device=dev)
+    if dv is None:
+        dv = torch.empty_like(dk)
+    if workspace is None:
+        workspace = torch.empty((B, H_q, L), dtype=torch.float32, device=dev)
+    ra_ring_attn_bwd(q.data_ptr(), [k_chunks[j].data_ptr() for j in range(P)],
+                     [v_chunks[j].data_ptr() for j in range(P)], out.data_ptr(), lse.data_ptr(),
+                     dout.data_ptr(), P, B, H_q, H_kv, Lc, D, L * H_q * D, Lc * H_kv * D,
+                     float(scale), causal, dq.data_ptr(), [dk[j].data_ptr() for j in range(P)],
+                     [dv[j].data_ptr() for j in range(P)], workspace.data_ptr(), _stream(stream))
+    return dq, dk, dv
 
 
 def ra_lse_merge(o_a: torch.Tensor, lse_a: torch.Tensor, o_b: torch.Tensor, lse_b: torch.Tensor,

@@ -206,6 +206,32 @@ RA_API ra_status ra_ring_attn_bwd(const void* q, const void* const* k_chunks,
                                   float* workspace, void* stream);
 
 /*
+ * ra_ring_attn_bwd_static -- ra_ring_attn_bwd without a workspace argument: the Delta
+ * rows live in a fixed device array inside the library, so a call allocates no device
+ * memory (no cudaMalloc, no cudaFree, no allocating library routine).  The pages have no
+ * counterpart to this entry point; it is a deployment convenience around the backward.
+ * Arguments and results are those of ra_ring_attn_bwd, minus workspace.
+ * Limit: B * H_q * P * Lc <= RA_BWD_STATIC_MAX_ROWS (2^21 rows, an 8 MiB fp32 array per
+ *   device); larger requests return RA_ERR_INVALID before anything is enqueued.
+ * Set-up: the first call on a device resolves the array's address
+ *   (cudaGetSymbolAddress, which may load the library's device code) and the kernels'
+ *   shared-memory attributes; make that first call before any stream capture.
+ * Concurrency: the array is shared by all calls on a device.  Calls that overlap in time
+ *   (on different streams, or from host threads without ordering between them) race on
+ *   it; calls ordered on one stream do not.  Nothing in it needs to start at zero.
+ * Errors: those of ra_ring_attn_bwd; RA_ERR_INVALID when the size limit is exceeded;
+ *   RA_ERR_CUDA if the current device or the array's address cannot be obtained.
+ */
+#define RA_BWD_STATIC_MAX_ROWS (1 << 21)
+RA_API ra_status ra_ring_attn_bwd_static(const void* q, const void* const* k_chunks,
+                                         const void* const* v_chunks, const void* out,
+                                         const float* lse, const void* dout, int P, int B,
+                                         int H_q, int H_kv, int Lc, int D,
+                                         long long q_bstride, long long kv_bstride, float scale,
+                                         int causal, float* dq, float* const* dk_chunks,
+                                         float* const* dv_chunks, void* stream);
+
+/*
  * ra_lse_merge -- merge two partial attention results over disjoint key sets
  * into one, in place into (o_a, lse_a).  [SP-QA] section 5 (the merge step of
  * the ring loop, read as the exact log-sum-exp combination):

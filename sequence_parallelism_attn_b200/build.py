@@ -17,7 +17,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libra_b200.so")
 BUILD_DIR = os.path.join(HERE, "_build")
-SOURCES = ["api.cu", "attn_sm100.cu", "attn_bwd_sm100.cu", "attn_fp32.cu", "lse_merge.cu", "permute.cu"]
+SOURCES = ["api.cu", "attn_sm100.cu", "attn_bwd_sm100.cu", "bwd_static.cu", "attn_fp32.cu", "lse_merge.cu", "permute.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler",
               "-fvisibility=hidden", f"-I{INCLUDE}", f"-I{CSRC}"]

@@ -33,6 +33,10 @@ int elem_size(ra_dtype d) { return d == RA_BF16 ? 2 : (d == RA_FP32 ? 4 : 0); }
 
 }  // namespace
 
+namespace ra {
+int set_last_error(int status, const std::string& msg) { return (int)fail((ra_status)status, msg); }
+}  // namespace ra
+
 extern "C" {
 
 static ra_status ring_attn(const void* q, const void* const* k_chunks, const void* const* v_chunks,

@@ -3,6 +3,7 @@
 #pragma once
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <string>
 
 namespace ra {
 
@@ -127,6 +128,10 @@ cudaError_t launch_head2seq(const void* in, void* out, int P, int G, int B, int 
 cudaError_t launch_attn_bwd_sm100(const AttnBwdArgs& a, unsigned long long wait_limit_ns,
                                   const char** why);
 cudaError_t read_and_clear_bwd_error(unsigned int* value);
+
+// Records msg as the calling thread's ra_last_error() text and returns status (for entry
+// points defined outside api.cu).
+int set_last_error(int status, const std::string& msg);
 // Read and clear the per-device kernel error word (after the caller synchronised).
 cudaError_t read_and_clear_error_word(unsigned int* value);
 cudaError_t read_and_clear_permute_error(unsigned int* value);

@@ -19,7 +19,7 @@ RA_OK, RA_ERR_INVALID, RA_ERR_UNSUPPORTED, RA_ERR_CUDA, RA_ERR_TIMEOUT = 0, 1, 2
 RA_BF16, RA_FP32 = 0, 1
 RA_MAX_P = 64
 EXPORTED = ("ra_ring_attn_fwd", "ra_ring_attn_fwd_zigzag", "ra_ring_attn_fwd_packed",
-            "ra_ring_attn_bwd",
+            "ra_ring_attn_bwd", "ra_ring_attn_bwd_static",
             "ra_lse_merge", "ra_ulysses_seq2head", "ra_ulysses_head2seq",
             "ra_ulysses_seq2head_grouped", "ra_ulysses_head2seq_grouped",
             "ra_sync_status", "ra_last_error", "ra_set_wait_limit_ns", "ra_debug_inject_stall",
@@ -50,6 +50,7 @@ def load() -> ctypes.CDLL:
     lib.ra_ring_attn_fwd_zigzag.argtypes = lib.ra_ring_attn_fwd.argtypes
     lib.ra_ring_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i64,
                                      i64, f32, i32, vp, vp, vp, vp, vp]
+    lib.ra_ring_attn_bwd_static.argtypes = lib.ra_ring_attn_bwd.argtypes[:19] + [vp]
     lib.ra_ring_attn_fwd_packed.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i64, i64,
                                             f32, i32, i32, vp, vp, vp]
     lib.ra_lse_merge.argtypes = [vp, vp, vp, vp, i32, i32, i64, i32, vp]
@@ -59,7 +60,7 @@ def load() -> ctypes.CDLL:
     lib.ra_ulysses_head2seq_grouped.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, vp]
     lib.ra_sync_status.argtypes = [vp]
     for f in ("ra_ring_attn_fwd", "ra_ring_attn_fwd_zigzag", "ra_ring_attn_fwd_packed",
-              "ra_ring_attn_bwd", "ra_lse_merge",
+              "ra_ring_attn_bwd", "ra_ring_attn_bwd_static", "ra_lse_merge",
               "ra_ulysses_seq2head", "ra_ulysses_head2seq", "ra_ulysses_seq2head_grouped",
               "ra_ulysses_head2seq_grouped", "ra_sync_status"):
         getattr(lib, f).restype = ctypes.c_int
@@ -136,6 +137,18 @@ def ra_ring_attn_bwd(q_ptr, k_ptrs, v_ptrs, out_ptr, lse_ptr, dout_ptr, P, B, H_
                                    P, B, H_q, H_kv, Lc, D, q_bstride, kv_bstride, scale,
                                    int(causal), dq_ptr, arr(*dk_ptrs), arr(*dv_ptrs), ws_ptr,
                                    stream))
+
+
+def ra_ring_attn_bwd_static(q_ptr, k_ptrs, v_ptrs, out_ptr, lse_ptr, dout_ptr, P, B, H_q, H_kv,
+                            Lc, D, q_bstride, kv_bstride, scale, causal, dq_ptr, dk_ptrs, dv_ptrs,
+                            stream):
+    """The backward C entry point whose Delta scratch is the library's own fixed device
+    array (no workspace pointer; B*H_q*P*Lc <= RA_BWD_STATIC_MAX_ROWS)."""
+    arr = ctypes.c_void_p * P
+    _check(load().ra_ring_attn_bwd_static(q_ptr, arr(*k_ptrs), arr(*v_ptrs), out_ptr, lse_ptr,
+                                          dout_ptr, P, B, H_q, H_kv, Lc, D, q_bstride,
+                                          kv_bstride, scale, int(causal), dq_ptr, arr(*dk_ptrs),
+                                          arr(*dv_ptrs), stream))
 
 
 def ring_attn_bwd(q: torch.Tensor, k_chunks: torch.Tensor, v_chunks: torch.Tensor,

@@ -1,0 +1,85 @@
+"""ra_ring_attn_bwd_static -- the backward pass with its Delta scratch in the library's fixed
+device array, so that a call allocates no device memory -- against ra_ring_attn_bwd with a
+caller-provided workspace.  Both run the same kernels, so two static calls in a row must
+give the existing entry point's gradients bit for bit; the second call must leave the
+device's free memory unchanged; sizes beyond RA_BWD_STATIC_MAX_ROWS are refused before
+anything is enqueued.  The pages have no counterpart to this entry point."""
+import zlib
+
+import pytest
+import torch
+
+from sequence_parallelism_attn_b200 import synth
+
+MAX_ROWS = 1 << 21  # RA_BWD_STATIC_MAX_ROWS in include/ra.h
+
+
+def _problem(name, B, H_q, H_kv, P, Lc, D=128):
+    w = synth.AttnWorkload(name, B=B, H_q=H_q, H_kv=H_kv, D=D, P=P, Lc=Lc,
+                           dtype=torch.bfloat16, causal=True, q_mult=2.0,
+                           seed=zlib.crc32(name.encode()) % 100000)
+    q, k, v = (t.cuda() for t in synth.attention_inputs(w))
+    g = torch.Generator(device="cuda").manual_seed(w.seed + 1)
+    dout = torch.randn(q.shape, generator=g, device="cuda").to(torch.bfloat16)
+    return w, q, k, v, dout
+
+
+def _static_call(ra, w, q, k, v, o, lse, dout):
+    """One ra_ring_attn_bwd_static call into fresh NaN-filled gradient buffers."""
+    dq = torch.full((w.B, w.L, w.H_q, w.D), float("nan"), device="cuda")
+    dk = torch.full(k.shape, float("nan"), device="cuda")
+    dv = torch.full(k.shape, float("nan"), device="cuda")
+    torch.cuda.synchronize()
+    free_before, _ = torch.cuda.mem_get_info()
+    ra.ra_ring_attn_bwd_static(q.data_ptr(), [k[j].data_ptr() for j in range(w.P)],
+                               [v[j].data_ptr() for j in range(w.P)], o.data_ptr(),
+                               lse.data_ptr(), dout.data_ptr(), w.P, w.B, w.H_q, w.H_kv, w.Lc,
+                               w.D, w.L * w.H_q * w.D, w.Lc * w.H_kv * w.D, w.scale, True,
+                               dq.data_ptr(), [dk[j].data_ptr() for j in range(w.P)],
+                               [dv[j].data_ptr() for j in range(w.P)],
+                               torch.cuda.current_stream().cuda_stream)
+    assert ra.ra_sync_status() == 0, ra.ra_last_error()
+    free_after, _ = torch.cuda.mem_get_info()
+    return (dq, dk, dv), free_before, free_after
+
+
+def _two_calls_match(ra, name, B, H_q, H_kv, P, Lc):
+    w, q, k, v, dout = _problem(name, B, H_q, H_kv, P, Lc)
+    o, lse = ra.ring_attn_fwd(q, k, v, True, w.scale, out_dtype=torch.bfloat16)
+    want = ra.ring_attn_bwd(q, k, v, o, lse, dout, True, w.scale)
+    assert ra.ra_sync_status() == 0, ra.ra_last_error()
+    first, _, _ = _static_call(ra, w, q, k, v, o, lse, dout)
+    second, free_before, free_after = _static_call(ra, w, q, k, v, o, lse, dout)
+    for nm, a, b, c in zip(("dq", "dk", "dv"), want, first, second):
+        assert torch.equal(a, b), f"first static call differs in {nm}"
+        assert torch.equal(a, c), f"second static call differs in {nm}"
+    assert free_after == free_before, (free_before, free_after)
+
+
+@pytest.mark.gpu
+def test_static_two_calls_match_workspace_entry(ra_lib):
+    """Ragged GQA problem: 3 chunks of 200 tokens, H_q = 4 over H_kv = 2, B = 2, causal."""
+    _two_calls_match(ra_lib, "bwd_static_small", 2, 4, 2, 3, 200)
+
+
+@pytest.mark.gpu
+def test_static_at_the_size_limit(ra_lib):
+    """B * H_q * P * Lc exactly RA_BWD_STATIC_MAX_ROWS (2 x 16 heads x 65536 tokens)."""
+    assert 2 * 16 * 8 * 8192 == MAX_ROWS
+    _two_calls_match(ra_lib, "bwd_static_limit", 2, 16, 4, 8, 8192)
+
+
+def test_static_rejects_sizes_beyond_the_limit():
+    """Refused on the host before any CUDA call (runs without a GPU); the pointers are
+    never dereferenced."""
+    from sequence_parallelism_attn_b200 import build, ra
+    build.build()
+    lib = ra.load()
+    fake = 0x10000
+    for B, H_q, P, Lc in ((1, 2, 2, 1 << 20), (2, 16, 8, 8193), (1 << 30, 1 << 30, 64, 1 << 24)):
+        with pytest.raises(ra.RaError) as e:
+            ra.ra_ring_attn_bwd_static(fake, [fake] * P, [fake] * P, fake, fake, fake, P, B, H_q,
+                                       1, Lc, 128, 1 << 40, 1 << 40, 0.1, True, fake,
+                                       [fake] * P, [fake] * P, 0)
+        assert e.value.status == 1  # RA_ERR_INVALID
+        assert "RA_BWD_STATIC_MAX_ROWS" in lib.ra_last_error().decode()

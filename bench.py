@@ -14,7 +14,7 @@ the steps (max over ranks), in TFLOP/s.  With --gpus N every rank runs its own r
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload ulysses_e2e|ulysses_32k|usp_e2e|long_128k|long_128k_zigzag|long_128k_packed|
-                              long_128k_bwd|
+                              long_128k_bwd|llama8b_32k_bwd|
                               llama8b_32k|small_4k]
 """
 from __future__ import annotations
@@ -61,6 +61,7 @@ def workloads():
         "long_128k_packed": ("attn_packed", synth.LONG_128K),
         "long_128k_bwd": ("attn_bwd", synth.LONG_128K),
         "llama8b_32k": ("attn", synth.LLAMA8B_GQA),
+        "llama8b_32k_bwd": ("attn_bwd", synth.LLAMA8B_GQA),
         "small_4k": ("attn", synth.SMALL_BF16),
     }
 

@@ -10,9 +10,15 @@
 // stationary (every query tile of every query head of the kv head's group that can see
 // it).  Each tensor-core kernel keeps its operands for one 128 x 128 tile pair in tensor
 // memory:
-//   dQ kernel   TMEM S [0,128), dP [128,256), dQ [256,256+D); dS (bf16) over S
-//   dK/dV       TMEM S^T [0,128), dP^T [128,256), dV [256,256+D), dK [256+D,256+2D);
-//               P^T (bf16) over S^T, dS^T (bf16) over dP^T
+//   dQ kernel   TMEM S [0,128) or [384,512) by tile parity, dP [128,256), dQ [256,256+D);
+//               dS (bf16) over S
+//   dK/dV       TMEM S^T and dP^T in [0,128) / [128,256), swapping every query tile,
+//               dV [256,256+D), dK [256+D,256+2D); P^T and dS^T (bf16) of each 64-query
+//               half over that half of S^T
+// The compute warps publish P / dS in two 64-column halves (the MMAs over the first half
+// run while the second is formed) and signal when they have read dP, so that the next
+// tile's S (dQ kernel: into the spare region) and dP (dK/dV: S^T into the freed dP^T
+// region) are computed while they work.
 // Roles (192 threads): warps 0-3 compute P, dS (one TMEM lane = one row each), warp 4
 // loads (TMA), warp 5 issues the MMAs (one thread) and owns tensor memory.  Every wait is
 // bounded: a role that gives up sets the CTA abort flag and this file's error word, every
@@ -70,8 +76,9 @@ struct BCfg {
     static constexpr int OFF_RING = 2 * TILE;            // NS x (two tiles) stages
     static constexpr int STAGE = 2 * TILE + 2 * kBM * 4; // + LSE and Delta rows (dK/dV)
     static constexpr int OFF_BAR = OFF_RING + NS * STAGE;
-    // barriers: fixed_full, full[NS], empty[NS], sd_full, ds_full, acc_done, drain
-    static constexpr int N_BARS = 1 + 2 * NS + 4;
+    // barriers: fixed_full, full[NS], empty[NS], sd_full, ds_full[2] (one per 64-column
+    // half of dS / P^T), acc_done, drain, dp_free (the compute warps have read all of dP)
+    static constexpr int N_BARS = 1 + 2 * NS + 6;
     static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem base, abort flag, n
     static constexpr int OFF_SCHED = OFF_MISC + 16;
     static constexpr int SMEM = OFF_SCHED + 2 * RA_MAX_P * 4 + 1024;
@@ -79,11 +86,22 @@ struct BCfg {
     __host__ __device__ static constexpr int bar_full(int s) { return 1 + s; }
     __host__ __device__ static constexpr int bar_empty(int s) { return 1 + NS + s; }
     static constexpr int BAR_SD = 1 + 2 * NS;
-    static constexpr int BAR_DS = 2 + 2 * NS;
-    static constexpr int BAR_ACC = 3 + 2 * NS;
-    static constexpr int BAR_DRAIN = 4 + 2 * NS;
+    __host__ __device__ static constexpr int bar_ds(int half) { return 2 + 2 * NS + half; }
+    static constexpr int BAR_ACC = 4 + 2 * NS;
+    static constexpr int BAR_DRAIN = 5 + 2 * NS;
+    static constexpr int BAR_DPFREE = 6 + 2 * NS;
+    // dQ kernel TMEM: S of even key tiles at column 0, of odd ones at S_ODD (S of the next
+    // tile is computed while this tile's dS is formed), dP at 128, dQ at 256.
+    static constexpr uint32_t S_ODD = 384;
+    __host__ __device__ static constexpr uint32_t s_col(int jt) { return (jt & 1) ? S_ODD : 0u; }
+    // dK/dV kernel TMEM: two 128-column regions at 0 and 128 swap roles every query tile:
+    // S^T(i) in one (P^T and dS^T of each 64-query half are stored over that half of it),
+    // dP^T(i) in the other, which holds S^T(i+1) once dP^T(i) has been read.
+    __host__ __device__ static constexpr uint32_t st_col(int i) { return (i & 1) ? 128u : 0u; }
+    __host__ __device__ static constexpr uint32_t dpt_col(int i) { return (i & 1) ? 0u : 128u; }
     static_assert(SMEM <= 232448, "shared memory budget");
     static_assert(256 + 2 * D <= (int)kTmemCols, "tensor memory budget");
+    static_assert(256 + D <= (int)S_ODD && S_ODD + kBN <= kTmemCols, "dQ kernel columns");
 };
 
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag, unsigned code) {
@@ -213,9 +231,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
             mbar_init(bar(C::bar_empty(s)), 1);
         }
         mbar_init(bar(C::BAR_SD), 1);
-        mbar_init(bar(C::BAR_DS), 4 * 32);
+        mbar_init(bar(C::bar_ds(0)), 4 * 32);
+        mbar_init(bar(C::bar_ds(1)), 4 * 32);
         mbar_init(bar(C::BAR_ACC), 1);
         mbar_init(bar(C::BAR_DRAIN), 1);
+        mbar_init(bar(C::BAR_DPFREE), 4 * 32);
         *abort_flag = 0;
         fence_mbar_init();
         fence_proxy_async_smem();
@@ -279,36 +299,66 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
             constexpr uint32_t IDESC_O = idesc_bf16_f32(kBM, D, 1);    // B MN-major (D contiguous)
             const uint64_t dq_ = desc_sw128(base + C::OFF_A, 16, 1024);
             const uint64_t ddo = desc_sw128(base + C::OFF_B, 16, 1024);
+            auto stage = [&](int jt) { return base + C::OFF_RING + (uint32_t)(jt % C::NS) * C::STAGE; };
+            auto issue_s = [&](int jt) {  // S(jt) = Q K(jt)^T into its column region
+                const uint64_t dk = desc_sw128(stage(jt), 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = ((kk / 4) * C::BLK + (kk % 4) * 32) >> 4;
+                    mma_ss(tmem + C::s_col(jt), dq_ + off, dk + off, IDESC_S, kk > 0 ? 1u : 0u);
+                }
+            };
+            auto issue_dp = [&](int jt) {  // dP(jt) = dO V(jt)^T
+                const uint64_t dv = desc_sw128(stage(jt) + C::TILE, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = ((kk / 4) * C::BLK + (kk % 4) * 32) >> 4;
+                    mma_ss(tmem + 128, ddo + off, dv + off, IDESC_S, kk > 0 ? 1u : 0u);
+                }
+            };
+            auto dq_half = [&](int jt, int half) {  // dQ += dS(jt) K(jt) over 64 keys
+                // dS (bf16 pairs) over S's first 64 columns, K as MN-major B
+                const uint64_t dkm = desc_sw128(stage(jt), C::BLK, 1024);
+#pragma unroll
+                for (int kk = 4 * half; kk < 4 * half + 4; ++kk)
+                    mma_ts(tmem + 256, tmem + C::s_col(jt) + kk * 8,
+                           dkm + (uint64_t)((kk * 2048) >> 4), IDESC_O,
+                           (jt > 0 || kk > 0) ? 1u : 0u);
+            };
+            // Order per key tile jt: S(jt+1) into the other S region; dQ over the first 64
+            // keys once the compute warps publish them; dP(jt+1) once they have read dP(jt);
+            // after the second half is published, one commit for S(jt+1) and dP(jt+1), then
+            // dQ over the second 64 keys.  The compute warps' next tile overlaps that last
+            // part, and dP(jt+1) overlaps their second half.
             bool issued = false;
-            if (wait1(bar(C::BAR_FIXED), 0, abort_flag, lim, kErrMma)) {
+            if (wait1(bar(C::BAR_FIXED), 0, abort_flag, lim, kErrMma) && n > 0 &&
+                wait1(bar(C::bar_full(0)), 0, abort_flag, lim, kErrMma)) {
+                tc_fence_after();
+                issue_s(0);
+                issue_dp(0);
+                tc_commit(bar(C::BAR_SD));
+                issued = true;
                 for (int jt = 0; jt < n; ++jt) {
-                    const int slot = jt % C::NS;
-                    if (!wait1(bar(C::bar_full(slot)), (jt / C::NS) & 1, abort_flag, lim, kErrMma)) break;
-                    tc_fence_after();
-                    const uint32_t st = base + C::OFF_RING + slot * C::STAGE;
-                    const uint64_t dk = desc_sw128(st, 16, 1024);
-                    const uint64_t dv = desc_sw128(st + C::TILE, 16, 1024);
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = ((kk / 4) * C::BLK + (kk % 4) * 32) >> 4;
-                        mma_ss(tmem + 0, dq_ + off, dk + off, IDESC_S, kk > 0 ? 1u : 0u);
+                    const bool more = jt + 1 < n;
+                    const uint32_t ph = jt & 1;
+                    if (more) {
+                        if (!wait1(bar(C::bar_full((jt + 1) % C::NS)), ((jt + 1) / C::NS) & 1,
+                                   abort_flag, lim, kErrMma))
+                            break;
+                        tc_fence_after();
+                        issue_s(jt + 1);
                     }
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = ((kk / 4) * C::BLK + (kk % 4) * 32) >> 4;
-                        mma_ss(tmem + 128, ddo + off, dv + off, IDESC_S, kk > 0 ? 1u : 0u);
-                    }
-                    tc_commit(bar(C::BAR_SD));
-                    issued = true;
-                    if (!wait1(bar(C::BAR_DS), jt & 1, abort_flag, lim, kErrMma)) break;
+                    if (!wait1(bar(C::bar_ds(0)), ph, abort_flag, lim, kErrMma)) break;
                     tc_fence_after();
-                    // dQ += dS K: dS (bf16 pairs) over S's first 64 columns, K as MN-major B
-                    const uint64_t dkm = desc_sw128(st, C::BLK, 1024);
-#pragma unroll
-                    for (int kk = 0; kk < kBN / 16; ++kk)
-                        mma_ts(tmem + 256, tmem + kk * 8, dkm + (uint64_t)((kk * 2048) >> 4), IDESC_O,
-                               (jt > 0 || kk > 0) ? 1u : 0u);
-                    tc_commit(bar(C::bar_empty(slot)));
+                    dq_half(jt, 0);
+                    if (!wait1(bar(C::BAR_DPFREE), ph, abort_flag, lim, kErrMma)) break;
+                    tc_fence_after();
+                    if (more) issue_dp(jt + 1);
+                    if (!wait1(bar(C::bar_ds(1)), ph, abort_flag, lim, kErrMma)) break;
+                    tc_fence_after();
+                    if (more) tc_commit(bar(C::BAR_SD));
+                    dq_half(jt, 1);
+                    tc_commit(bar(C::bar_empty(jt % C::NS)));
                 }
             }
             if (issued) {
@@ -343,11 +393,16 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
             const long long k0 = (long long)it.chunk() * p.Lc + (long long)it.t * kBN;
             const int kvalid = min(kBN, p.Lc - it.t * kBN);
             const long long lim_c = p.causal ? my_row - k0 : (long long)kBN;  // keys c <= lim_c
+            const uint32_t scol = C::s_col(jt);
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 float s[64], dp[64];
-                tmem_ld64(tmem + lane_off + 64 * c, s);
+                tmem_ld64(tmem + lane_off + scol + 64 * c, s);
                 tmem_ld64(tmem + lane_off + 128 + 64 * c, dp);
+                if (c == 1) {  // dP is in registers: its columns may take dP of the next tile
+                    tc_fence_before();
+                    mbar_arrive(bar(C::BAR_DPFREE));
+                }
                 uint32_t pk[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
@@ -361,11 +416,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
                     }
                     pk[i] = pack_bf16x2(ds2[0], ds2[1]);
                 }
-                tmem_st32(tmem + lane_off + 32 * c, pk);
+                // publish this 64-key half: its dQ MMAs overlap the next half's work
+                tmem_st32(tmem + lane_off + scol + 32 * c, pk);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(C::bar_ds(c)));
             }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(bar(C::BAR_DS));
         }
         (void)FULL;
         if (ok && n > 0 && wait_warp(bar(C::BAR_ACC), 0, abort_flag, lim, kErrCompute)) {
@@ -437,9 +493,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_sm100(const __grid_const
             mbar_init(bar(C::bar_empty(s)), 1);
         }
         mbar_init(bar(C::BAR_SD), 1);
-        mbar_init(bar(C::BAR_DS), 4 * 32);
+        mbar_init(bar(C::bar_ds(0)), 4 * 32);
+        mbar_init(bar(C::bar_ds(1)), 4 * 32);
         mbar_init(bar(C::BAR_ACC), 1);
         mbar_init(bar(C::BAR_DRAIN), 1);
+        mbar_init(bar(C::BAR_DPFREE), 4 * 32);
         *abort_flag = 0;
         fence_mbar_init();
         fence_proxy_async_smem();
@@ -503,43 +561,73 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_sm100(const __grid_const
             constexpr uint32_t IDESC_O = idesc_bf16_f32(kBN, D, 1);    // B MN-major (D contiguous)
             const uint64_t dk_ = desc_sw128(base + C::OFF_A, 16, 1024);
             const uint64_t dv_ = desc_sw128(base + C::OFF_B, 16, 1024);
+            auto stage = [&](int i) { return base + C::OFF_RING + (uint32_t)(i % C::NS) * C::STAGE; };
+            auto issue_st = [&](int i) {  // S^T(i) = K Q(i)^T (keys are the TMEM lanes)
+                const uint64_t dq_ = desc_sw128(stage(i), 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = ((kk / 4) * C::BLK + (kk % 4) * 32) >> 4;
+                    mma_ss(tmem + C::st_col(i), dk_ + off, dq_ + off, IDESC_S, kk > 0 ? 1u : 0u);
+                }
+            };
+            auto issue_dpt = [&](int i) {  // dP^T(i) = V dO(i)^T
+                const uint64_t ddo = desc_sw128(stage(i) + C::TILE, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = ((kk / 4) * C::BLK + (kk % 4) * 32) >> 4;
+                    mma_ss(tmem + C::dpt_col(i), dv_ + off, ddo + off, IDESC_S, kk > 0 ? 1u : 0u);
+                }
+            };
+            // dV += P^T dO and dK += dS^T Q over one 64-query half: P^T of the half in columns
+            // [64 half, 64 half + 32) of the S^T region, dS^T in the next 32; Q and dO as
+            // MN-major B (D contiguous, query rows 128 bytes apart)
+            auto dvdk_half = [&](int i, int half) {
+                const uint64_t dom = desc_sw128(stage(i) + C::TILE, C::BLK, 1024);
+                const uint64_t qm = desc_sw128(stage(i), C::BLK, 1024);
+                const uint32_t a0 = tmem + C::st_col(i) + 64 * half;
+#pragma unroll
+                for (int kk = 4 * half; kk < 4 * half + 4; ++kk)
+                    mma_ts(tmem + 256, a0 + (kk % 4) * 8, dom + (uint64_t)((kk * 2048) >> 4),
+                           IDESC_O, (i > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                for (int kk = 4 * half; kk < 4 * half + 4; ++kk)
+                    mma_ts(tmem + 256 + D, a0 + 32 + (kk % 4) * 8, qm + (uint64_t)((kk * 2048) >> 4),
+                           IDESC_O, (i > 0 || kk > 0) ? 1u : 0u);
+            };
+            // Order per query tile i: dV/dK over the first 64 queries once the compute warps
+            // publish them; S^T(i+1) into the dP^T region once they have read dP^T(i) (it
+            // overlaps their second half); dV/dK over the second half; dP^T(i+1) into the
+            // S^T region (after the MMAs that read it) and one commit for S^T(i+1), dP^T(i+1).
             bool issued = false;
-            if (wait1(bar(C::BAR_FIXED), 0, abort_flag, lim, kErrMma)) {
+            if (wait1(bar(C::BAR_FIXED), 0, abort_flag, lim, kErrMma) && n > 0 &&
+                wait1(bar(C::bar_full(0)), 0, abort_flag, lim, kErrMma)) {
+                tc_fence_after();
+                issue_st(0);
+                issue_dpt(0);
+                tc_commit(bar(C::BAR_SD));
+                issued = true;
                 for (int it = 0; it < n; ++it) {
-                    const int slot = it % C::NS;
-                    if (!wait1(bar(C::bar_full(slot)), (it / C::NS) & 1, abort_flag, lim, kErrMma)) break;
+                    const bool more = it + 1 < n;
+                    const uint32_t ph = it & 1;
+                    if (!wait1(bar(C::bar_ds(0)), ph, abort_flag, lim, kErrMma)) break;
                     tc_fence_after();
-                    const uint32_t st = base + C::OFF_RING + slot * C::STAGE;
-                    const uint64_t dq_ = desc_sw128(st, 16, 1024);
-                    const uint64_t ddo = desc_sw128(st + C::TILE, 16, 1024);
-                    // S^T = K Q^T, dP^T = V dO^T (keys are the TMEM lanes)
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = ((kk / 4) * C::BLK + (kk % 4) * 32) >> 4;
-                        mma_ss(tmem + 0, dk_ + off, dq_ + off, IDESC_S, kk > 0 ? 1u : 0u);
+                    dvdk_half(it, 0);
+                    if (!wait1(bar(C::BAR_DPFREE), ph, abort_flag, lim, kErrMma)) break;
+                    if (more) {
+                        if (!wait1(bar(C::bar_full((it + 1) % C::NS)), ((it + 1) / C::NS) & 1,
+                                   abort_flag, lim, kErrMma))
+                            break;
+                        tc_fence_after();
+                        issue_st(it + 1);
                     }
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = ((kk / 4) * C::BLK + (kk % 4) * 32) >> 4;
-                        mma_ss(tmem + 128, dv_ + off, ddo + off, IDESC_S, kk > 0 ? 1u : 0u);
-                    }
-                    tc_commit(bar(C::BAR_SD));
-                    issued = true;
-                    if (!wait1(bar(C::BAR_DS), it & 1, abort_flag, lim, kErrMma)) break;
+                    if (!wait1(bar(C::bar_ds(1)), ph, abort_flag, lim, kErrMma)) break;
                     tc_fence_after();
-                    // dV += P^T dO and dK += dS^T Q; P^T over S^T, dS^T over dP^T; Q and dO
-                    // as MN-major B (D contiguous, query rows 128 bytes apart)
-                    const uint64_t dom = desc_sw128(st + C::TILE, C::BLK, 1024);
-                    const uint64_t qm = desc_sw128(st, C::BLK, 1024);
-#pragma unroll
-                    for (int kk = 0; kk < kBM / 16; ++kk)
-                        mma_ts(tmem + 256, tmem + kk * 8, dom + (uint64_t)((kk * 2048) >> 4), IDESC_O,
-                               (it > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-                    for (int kk = 0; kk < kBM / 16; ++kk)
-                        mma_ts(tmem + 256 + D, tmem + 128 + kk * 8, qm + (uint64_t)((kk * 2048) >> 4),
-                               IDESC_O, (it > 0 || kk > 0) ? 1u : 0u);
-                    tc_commit(bar(C::bar_empty(slot)));
+                    dvdk_half(it, 1);
+                    tc_commit(bar(C::bar_empty(it % C::NS)));
+                    if (more) {
+                        issue_dpt(it + 1);
+                        tc_commit(bar(C::BAR_SD));
+                    }
                 }
             }
             if (issued) {
@@ -569,11 +657,16 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_sm100(const __grid_const
             const float* rows = reinterpret_cast<const float*>(smem + C::OFF_RING + slot * C::STAGE + 2 * C::TILE);
             // queries c of the tile see this key when q0 + c >= key position (causal)
             const long long lo_c = p.causal ? my_kpos - q0 : 0;
+            const uint32_t xs = C::st_col(it), yd = C::dpt_col(it);
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 float s[64], dp[64];
-                tmem_ld64(tmem + lane_off + 64 * c, s);
-                tmem_ld64(tmem + lane_off + 128 + 64 * c, dp);
+                tmem_ld64(tmem + lane_off + xs + 64 * c, s);
+                tmem_ld64(tmem + lane_off + yd + 64 * c, dp);
+                if (c == 1) {  // dP^T is in registers: its region may take S^T of the next tile
+                    tc_fence_before();
+                    mbar_arrive(bar(C::BAR_DPFREE));
+                }
                 uint32_t pp[32], pd[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
@@ -589,12 +682,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_sm100(const __grid_const
                     pp[i] = pack_bf16x2(pr2[0], pr2[1]);
                     pd[i] = pack_bf16x2(ds2[0], ds2[1]);
                 }
-                tmem_st32(tmem + lane_off + 32 * c, pp);
-                tmem_st32(tmem + lane_off + 128 + 32 * c, pd);
+                // publish this 64-query half over the S^T columns just read: its dV/dK MMAs
+                // overlap the next half's work
+                tmem_st32(tmem + lane_off + xs + 64 * c, pp);
+                tmem_st32(tmem + lane_off + xs + 64 * c + 32, pd);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(C::bar_ds(c)));
             }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(bar(C::BAR_DS));
         }
         if (ok && n > 0 && wait_warp(bar(C::BAR_ACC), 0, abort_flag, lim, kErrCompute)) {
             __syncwarp();

@@ -11,7 +11,7 @@
 // it).  Each tensor-core kernel keeps its operands for one 128 x 128 tile pair in tensor
 // memory:
 //   dQ kernel   TMEM S [0,128) or [384,512) by tile parity, dP [128,256), dQ [256,256+D);
-//               dS (bf16) over S
+//               dS (bf16) of each 64-key half over the first 32 columns of that half of S
 //   dK/dV       TMEM S^T and dP^T in [0,128) / [128,256), swapping every query tile,
 //               dV [256,256+D), dK [256+D,256+2D); P^T and dS^T (bf16) of each 64-query
 //               half over that half of S^T
@@ -19,8 +19,9 @@
 // run while the second is formed) and signal when they have read dP, so that the next
 // tile's S (dQ kernel: into the spare region) and dP (dK/dV: S^T into the freed dP^T
 // region) are computed while they work.
-// Roles (192 threads): warps 0-3 compute P, dS (one TMEM lane = one row each), warp 4
-// loads (TMA), warp 5 issues the MMAs (one thread) and owns tensor memory.  Every wait is
+// Roles (320 threads): warps 0-7 compute P, dS (one TMEM lane = one row; warps 0-3 the
+// first 64 columns of a tile, 4-7 the second), warp 8 loads (TMA), warp 9 issues the MMAs
+// (one thread) and owns tensor memory.  Every wait is
 // bounded: a role that gives up sets the CTA abort flag and this file's error word, every
 // role stops issuing and drains its own work, and the CTA frees its tensor memory.
 #include <cuda.h>
@@ -39,9 +40,10 @@ __device__ unsigned int g_bwd_error_word = 0;
 
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kWarpLoad = 4;
-constexpr int kWarpMma = 5;
+constexpr int kThreads = 320;
+constexpr int kComputeWarps = 8;  // two warpgroups: one per 64-column half of every tile
+constexpr int kWarpLoad = 8;
+constexpr int kWarpMma = 9;
 constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 128;  // keys per tile
 static_assert(kBN == kSchedTile, "the schedule counts tiles of kBN keys");
@@ -235,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
         mbar_init(bar(C::bar_ds(1)), 4 * 32);
         mbar_init(bar(C::BAR_ACC), 1);
         mbar_init(bar(C::BAR_DRAIN), 1);
-        mbar_init(bar(C::BAR_DPFREE), 4 * 32);
+        mbar_init(bar(C::BAR_DPFREE), kComputeWarps * 32);
         *abort_flag = 0;
         fence_mbar_init();
         fence_proxy_async_smem();
@@ -317,19 +319,20 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
                 }
             };
             auto dq_half = [&](int jt, int half) {  // dQ += dS(jt) K(jt) over 64 keys
-                // dS (bf16 pairs) over S's first 64 columns, K as MN-major B
+                // dS (bf16 pairs) of the half over the first 32 of its 64 S columns, K as
+                // MN-major B
                 const uint64_t dkm = desc_sw128(stage(jt), C::BLK, 1024);
 #pragma unroll
                 for (int kk = 4 * half; kk < 4 * half + 4; ++kk)
-                    mma_ts(tmem + 256, tmem + C::s_col(jt) + kk * 8,
+                    mma_ts(tmem + 256, tmem + C::s_col(jt) + 64 * half + (kk % 4) * 8,
                            dkm + (uint64_t)((kk * 2048) >> 4), IDESC_O,
                            (jt > 0 || kk > 0) ? 1u : 0u);
             };
-            // Order per key tile jt: S(jt+1) into the other S region; dQ over the first 64
-            // keys once the compute warps publish them; dP(jt+1) once they have read dP(jt);
-            // after the second half is published, one commit for S(jt+1) and dP(jt+1), then
-            // dQ over the second 64 keys.  The compute warps' next tile overlaps that last
-            // part, and dP(jt+1) overlaps their second half.
+            // Order per key tile jt: S(jt+1) into the other S region; dP(jt+1) once the
+            // compute warps have read dP(jt) (both overlap their work on tile jt); dQ over
+            // the first 64 keys once they publish them; after the second half is published,
+            // one commit for S(jt+1) and dP(jt+1), then dQ over the second 64 keys (it
+            // overlaps their next tile).
             bool issued = false;
             if (wait1(bar(C::BAR_FIXED), 0, abort_flag, lim, kErrMma) && n > 0 &&
                 wait1(bar(C::bar_full(0)), 0, abort_flag, lim, kErrMma)) {
@@ -348,12 +351,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
                         tc_fence_after();
                         issue_s(jt + 1);
                     }
-                    if (!wait1(bar(C::bar_ds(0)), ph, abort_flag, lim, kErrMma)) break;
-                    tc_fence_after();
-                    dq_half(jt, 0);
                     if (!wait1(bar(C::BAR_DPFREE), ph, abort_flag, lim, kErrMma)) break;
                     tc_fence_after();
                     if (more) issue_dp(jt + 1);
+                    if (!wait1(bar(C::bar_ds(0)), ph, abort_flag, lim, kErrMma)) break;
+                    tc_fence_after();
+                    dq_half(jt, 0);
                     if (!wait1(bar(C::bar_ds(1)), ph, abort_flag, lim, kErrMma)) break;
                     tc_fence_after();
                     if (more) tc_commit(bar(C::BAR_SD));
@@ -368,13 +371,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
             }
         }
     } else {
-        // compute warps: P and dS for this thread's row
-        const unsigned FULL = 0xffffffffu;
-        const int wr = warp;
-        const int row_t = wr * 32 + lane;
+        // compute warps: P and dS for this thread's row over its warpgroup's 64-key half
+        // (a warp reaches TMEM lanes 32 (warp % 4) .. + 31)
+        const int quarter = warp & 3, c = warp >> 2;
+        const int row_t = quarter * 32 + lane;
         const long long my_row = (long long)r0 + row_t;
         const bool row_ok = my_row < p.L;
-        const uint32_t lane_off = (uint32_t)(wr * 32) << 16;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const long long lrow = ((long long)b * p.H_q + h) * p.L + (row_ok ? my_row : 0);
         // rows past L see nothing (lse2 = +inf makes every probability 0)
         const float lse2 = row_ok ? p.lse[lrow] * 1.4426950408889634f : INFINITY;
@@ -394,15 +397,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
             const int kvalid = min(kBN, p.Lc - it.t * kBN);
             const long long lim_c = p.causal ? my_row - k0 : (long long)kBN;  // keys c <= lim_c
             const uint32_t scol = C::s_col(jt);
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            {
                 float s[64], dp[64];
                 tmem_ld64(tmem + lane_off + scol + 64 * c, s);
                 tmem_ld64(tmem + lane_off + 128 + 64 * c, dp);
-                if (c == 1) {  // dP is in registers: its columns may take dP of the next tile
-                    tc_fence_before();
-                    mbar_arrive(bar(C::BAR_DPFREE));
-                }
+                // dP is in registers: once both halves are, its columns may take dP(jt+1)
+                tc_fence_before();
+                mbar_arrive(bar(C::BAR_DPFREE));
                 uint32_t pk[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
@@ -416,19 +417,18 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
                     }
                     pk[i] = pack_bf16x2(ds2[0], ds2[1]);
                 }
-                // publish this 64-key half: its dQ MMAs overlap the next half's work
-                tmem_st32(tmem + lane_off + scol + 32 * c, pk);
+                // publish this 64-key half over its own S columns (already read)
+                tmem_st32(tmem + lane_off + scol + 64 * c, pk);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(bar(C::bar_ds(c)));
             }
         }
-        (void)FULL;
         if (ok && n > 0 && wait_warp(bar(C::BAR_ACC), 0, abort_flag, lim, kErrCompute)) {
             __syncwarp();
             tc_fence_after();
 #pragma unroll
-            for (int cb = 0; cb < D / 32; ++cb) {
+            for (int cb = c * (D / 64); cb < (c + 1) * (D / 64); ++cb) {  // this half's columns
                 uint32_t o[32];
                 tmem_ld32(tmem + lane_off + 256 + cb * 32, o);
                 tmem_wait_ld();
@@ -444,8 +444,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
                 }
             }
         } else if (ok && n == 0 && row_ok) {
-            float4* dst = reinterpret_cast<float4*>(p.dq + (((long long)b * p.L + my_row) * p.H_q + h) * D);
-            for (int i = 0; i < D / 4; ++i) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            float4* dst = reinterpret_cast<float4*>(
+                p.dq + (((long long)b * p.L + my_row) * p.H_q + h) * D + c * (D / 2));
+            for (int i = 0; i < D / 8; ++i) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
     }
 
@@ -497,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_sm100(const __grid_const
         mbar_init(bar(C::bar_ds(1)), 4 * 32);
         mbar_init(bar(C::BAR_ACC), 1);
         mbar_init(bar(C::BAR_DRAIN), 1);
-        mbar_init(bar(C::BAR_DPFREE), 4 * 32);
+        mbar_init(bar(C::BAR_DPFREE), kComputeWarps * 32);
         *abort_flag = 0;
         fence_mbar_init();
         fence_proxy_async_smem();
@@ -594,10 +595,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_sm100(const __grid_const
                     mma_ts(tmem + 256 + D, a0 + 32 + (kk % 4) * 8, qm + (uint64_t)((kk * 2048) >> 4),
                            IDESC_O, (i > 0 || kk > 0) ? 1u : 0u);
             };
-            // Order per query tile i: dV/dK over the first 64 queries once the compute warps
-            // publish them; S^T(i+1) into the dP^T region once they have read dP^T(i) (it
-            // overlaps their second half); dV/dK over the second half; dP^T(i+1) into the
-            // S^T region (after the MMAs that read it) and one commit for S^T(i+1), dP^T(i+1).
+            // Order per query tile i: S^T(i+1) into the dP^T region once the compute warps
+            // have read dP^T(i) (it overlaps their work on tile i); dV/dK over each 64-query
+            // half as they publish it; dP^T(i+1) into the S^T region (after the MMAs that
+            // read it) and one commit for S^T(i+1), dP^T(i+1).
             bool issued = false;
             if (wait1(bar(C::BAR_FIXED), 0, abort_flag, lim, kErrMma) && n > 0 &&
                 wait1(bar(C::bar_full(0)), 0, abort_flag, lim, kErrMma)) {
@@ -609,9 +610,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_sm100(const __grid_const
                 for (int it = 0; it < n; ++it) {
                     const bool more = it + 1 < n;
                     const uint32_t ph = it & 1;
-                    if (!wait1(bar(C::bar_ds(0)), ph, abort_flag, lim, kErrMma)) break;
-                    tc_fence_after();
-                    dvdk_half(it, 0);
                     if (!wait1(bar(C::BAR_DPFREE), ph, abort_flag, lim, kErrMma)) break;
                     if (more) {
                         if (!wait1(bar(C::bar_full((it + 1) % C::NS)), ((it + 1) / C::NS) & 1,
@@ -620,6 +618,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_sm100(const __grid_const
                         tc_fence_after();
                         issue_st(it + 1);
                     }
+                    if (!wait1(bar(C::bar_ds(0)), ph, abort_flag, lim, kErrMma)) break;
+                    tc_fence_after();
+                    dvdk_half(it, 0);
                     if (!wait1(bar(C::bar_ds(1)), ph, abort_flag, lim, kErrMma)) break;
                     tc_fence_after();
                     dvdk_half(it, 1);
@@ -637,12 +638,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_sm100(const __grid_const
             }
         }
     } else {
-        // compute warps: P^T and dS^T for this thread's key against the tile's 128 queries
-        const int wr = warp;
-        const int key_t = wr * 32 + lane;
+        // compute warps: P^T and dS^T for this thread's key against its warpgroup's 64-query
+        // half of the tile (a warp reaches TMEM lanes 32 (warp % 4) .. + 31)
+        const int quarter = warp & 3, c = warp >> 2;
+        const int key_t = quarter * 32 + lane;
         const bool key_ok = key_t < kvalid;
         const long long my_kpos = key0 + key_t;
-        const uint32_t lane_off = (uint32_t)(wr * 32) << 16;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const float sl2 = p.scale_log2;
         bool ok = true;
         for (int it = 0; it < n; ++it) {
@@ -658,15 +660,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_sm100(const __grid_const
             // queries c of the tile see this key when q0 + c >= key position (causal)
             const long long lo_c = p.causal ? my_kpos - q0 : 0;
             const uint32_t xs = C::st_col(it), yd = C::dpt_col(it);
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            {
                 float s[64], dp[64];
                 tmem_ld64(tmem + lane_off + xs + 64 * c, s);
                 tmem_ld64(tmem + lane_off + yd + 64 * c, dp);
-                if (c == 1) {  // dP^T is in registers: its region may take S^T of the next tile
-                    tc_fence_before();
-                    mbar_arrive(bar(C::BAR_DPFREE));
-                }
+                // dP^T is in registers: once both halves are, its region may take S^T(it+1)
+                tc_fence_before();
+                mbar_arrive(bar(C::BAR_DPFREE));
                 uint32_t pp[32], pd[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
@@ -682,8 +682,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_sm100(const __grid_const
                     pp[i] = pack_bf16x2(pr2[0], pr2[1]);
                     pd[i] = pack_bf16x2(ds2[0], ds2[1]);
                 }
-                // publish this 64-query half over the S^T columns just read: its dV/dK MMAs
-                // overlap the next half's work
+                // publish this 64-query half over the S^T columns just read
                 tmem_st32(tmem + lane_off + xs + 64 * c, pp);
                 tmem_st32(tmem + lane_off + xs + 64 * c + 32, pd);
                 tmem_wait_st();
@@ -695,8 +694,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_sm100(const __grid_const
             __syncwarp();
             tc_fence_after();
             const long long orow = (((long long)b * p.Lc + t * kBN + key_t) * p.H_kv + g) * D;
-#pragma unroll
-            for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK (times scale)
+            {
+                const int which = c;  // warpgroup 0 writes dV, warpgroup 1 dK (times scale)
                 const float mul = which ? p.scale : 1.f;
                 float* outp = which ? p.dk[j] : p.dv[j];
 #pragma unroll
@@ -717,7 +716,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_sm100(const __grid_const
             }
         } else if (ok && n == 0 && key_ok) {
             const long long orow = (((long long)b * p.Lc + t * kBN + key_t) * p.H_kv + g) * D;
-            for (int i = 0; i < D; ++i) p.dk[j][orow + i] = p.dv[j][orow + i] = 0.f;
+            float* outp = c ? p.dk[j] : p.dv[j];
+            for (int i = 0; i < D; ++i) outp[orow + i] = 0.f;
         }
     }
 

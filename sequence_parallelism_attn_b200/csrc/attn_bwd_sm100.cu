@@ -19,9 +19,9 @@
 // run while the second is formed) and signal when they have read dP, so that the next
 // tile's S (dQ kernel: into the spare region) and dP (dK/dV: S^T into the freed dP^T
 // region) are computed while they work.
-// Roles (320 threads): warps 0-7 compute P, dS (one TMEM lane = one row; warps 0-3 the
-// first 64 columns of a tile, 4-7 the second), warp 8 loads (TMA), warp 9 issues the MMAs
-// (one thread) and owns tensor memory.  Every wait is
+// Roles (352 threads): warps 0-7 compute P, dS (one TMEM lane = one row; warps 0-3 the
+// first 64 columns of a tile, 4-7 the second), warp 8 loads (TMA), warps 9 and 10 each
+// issue part of the MMAs from one thread (warp 9 owns tensor memory).  Every wait is
 // bounded: a role that gives up sets the CTA abort flag and this file's error word, every
 // role stops issuing and drains its own work, and the CTA frees its tensor memory.
 #include <cuda.h>
@@ -40,10 +40,11 @@ __device__ unsigned int g_bwd_error_word = 0;
 
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int kComputeWarps = 8;  // two warpgroups: one per 64-column half of every tile
 constexpr int kWarpLoad = 8;
-constexpr int kWarpMma = 9;
+constexpr int kWarpMma = 9;   // MMA-issuing thread A (owns tensor memory)
+constexpr int kWarpMma2 = 10;  // MMA-issuing thread B
 constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 128;  // keys per tile
 static_assert(kBN == kSchedTile, "the schedule counts tiles of kBN keys");
@@ -79,8 +80,9 @@ struct BCfg {
     static constexpr int STAGE = 2 * TILE + 2 * kBM * 4; // + LSE and Delta rows (dK/dV)
     static constexpr int OFF_BAR = OFF_RING + NS * STAGE;
     // barriers: fixed_full, full[NS], empty[NS], sd_full, ds_full[2] (one per 64-column
-    // half of dS / P^T), acc_done, drain, dp_free (the compute warps have read all of dP)
-    static constexpr int N_BARS = 1 + 2 * NS + 6;
+    // half of dS / P^T), acc_done, drain, dp_free (the compute warps have read all of dP),
+    // x_free (dK/dV kernel: the MMAs reading P^T / dS^T of a tile are done)
+    static constexpr int N_BARS = 1 + 2 * NS + 7;
     static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem base, abort flag, n
     static constexpr int OFF_SCHED = OFF_MISC + 16;
     static constexpr int SMEM = OFF_SCHED + 2 * RA_MAX_P * 4 + 1024;
@@ -92,6 +94,7 @@ struct BCfg {
     static constexpr int BAR_ACC = 4 + 2 * NS;
     static constexpr int BAR_DRAIN = 5 + 2 * NS;
     static constexpr int BAR_DPFREE = 6 + 2 * NS;
+    static constexpr int BAR_XFREE = 7 + 2 * NS;
     // dQ kernel TMEM: S of even key tiles at column 0, of odd ones at S_ODD (S of the next
     // tile is computed while this tile's dS is formed), dP at 128, dQ at 256.
     static constexpr uint32_t S_ODD = 384;
@@ -177,6 +180,95 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&x)[64]) {
     }
 }
 
+// 64 fp32 columns of this thread's TMEM lane as 32 register pairs (column 2i in the low
+// half of pair i), loaded and waited for in one block so that every pair is an aligned
+// 64-bit register ready for the packed f32x2 instructions.
+__device__ __forceinline__ void tmem_ld64_pairs(uint32_t taddr, uint64_t (&o)[32]) {
+    asm volatile(
+        "{\n\t.reg .b32 r0, r1, r2, r3, r4, r5, r6, r7, r8, r9, r10, r11, r12, r13, r14, r15, r16, r17, r18, r19, r20, r21, r22, r23, r24, r25, r26, r27, r28, r29, r30, r31, r32, r33, r34, r35, r36, r37, r38, r39, r40, r41, r42, r43, r44, r45, r46, r47, r48, r49, r50, r51, r52, r53, r54, r55, r56, r57, r58, r59, r60, r61, r62, r63;\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {r0, r1, r2, r3, r4, r5, r6, r7, r8, r9, r10, r11, r12, r13, r14, r15, r16, r17, r18, r19, r20, r21, r22, r23, r24, r25, r26, r27, r28, r29, r30, r31}, [%32];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {r32, r33, r34, r35, r36, r37, r38, r39, r40, r41, r42, r43, r44, r45, r46, r47, r48, r49, r50, r51, r52, r53, r54, r55, r56, r57, r58, r59, r60, r61, r62, r63}, [%33];\n\t"
+        "tcgen05.wait::ld.sync.aligned;\n\t"
+        "mov.b64 %0, {r0, r1};\n\t"
+        "mov.b64 %1, {r2, r3};\n\t"
+        "mov.b64 %2, {r4, r5};\n\t"
+        "mov.b64 %3, {r6, r7};\n\t"
+        "mov.b64 %4, {r8, r9};\n\t"
+        "mov.b64 %5, {r10, r11};\n\t"
+        "mov.b64 %6, {r12, r13};\n\t"
+        "mov.b64 %7, {r14, r15};\n\t"
+        "mov.b64 %8, {r16, r17};\n\t"
+        "mov.b64 %9, {r18, r19};\n\t"
+        "mov.b64 %10, {r20, r21};\n\t"
+        "mov.b64 %11, {r22, r23};\n\t"
+        "mov.b64 %12, {r24, r25};\n\t"
+        "mov.b64 %13, {r26, r27};\n\t"
+        "mov.b64 %14, {r28, r29};\n\t"
+        "mov.b64 %15, {r30, r31};\n\t"
+        "mov.b64 %16, {r32, r33};\n\t"
+        "mov.b64 %17, {r34, r35};\n\t"
+        "mov.b64 %18, {r36, r37};\n\t"
+        "mov.b64 %19, {r38, r39};\n\t"
+        "mov.b64 %20, {r40, r41};\n\t"
+        "mov.b64 %21, {r42, r43};\n\t"
+        "mov.b64 %22, {r44, r45};\n\t"
+        "mov.b64 %23, {r46, r47};\n\t"
+        "mov.b64 %24, {r48, r49};\n\t"
+        "mov.b64 %25, {r50, r51};\n\t"
+        "mov.b64 %26, {r52, r53};\n\t"
+        "mov.b64 %27, {r54, r55};\n\t"
+        "mov.b64 %28, {r56, r57};\n\t"
+        "mov.b64 %29, {r58, r59};\n\t"
+        "mov.b64 %30, {r60, r61};\n\t"
+        "mov.b64 %31, {r62, r63};\n\t"
+        "}"
+        : "=l"(o[0]), "=l"(o[1]), "=l"(o[2]), "=l"(o[3]), "=l"(o[4]), "=l"(o[5]), "=l"(o[6]), "=l"(o[7]), "=l"(o[8]), "=l"(o[9]), "=l"(o[10]), "=l"(o[11]), "=l"(o[12]), "=l"(o[13]), "=l"(o[14]), "=l"(o[15]), "=l"(o[16]), "=l"(o[17]), "=l"(o[18]), "=l"(o[19]), "=l"(o[20]), "=l"(o[21]), "=l"(o[22]), "=l"(o[23]), "=l"(o[24]), "=l"(o[25]), "=l"(o[26]), "=l"(o[27]), "=l"(o[28]), "=l"(o[29]), "=l"(o[30]), "=l"(o[31])
+        : "r"(taddr), "r"(taddr + 32)
+        : "memory");
+}
+
+// One column pair of the backward's elementwise step, on packed fp32 pairs:
+//   p  = 2^(s * scale_log2 + neg_lse)     (one packed fma, two MUFU ex2)
+//   ds = p * (dp + neg_delta)             (one packed add, one packed multiply)
+// Returns bf16x2(p) in pp and bf16x2(ds) in pd (lane 0 in the low half).  The roundings are
+// those of the scalar fma, add and multiply.
+__device__ __forceinline__ void p_ds_pair(uint64_t s2, uint64_t dp2, uint64_t sl2x2,
+                                          uint64_t nlse2, uint64_t ndelta2, uint32_t& pp,
+                                          uint32_t& pd) {
+    asm("{\n\t.reg .b32 x0, x1, p0, p1, d0, d1;\n\t.reg .b64 x, p, t, d;\n\t"
+        "fma.rn.f32x2 x, %2, %4, %5;\n\t"
+        "mov.b64 {x0, x1}, x;\n\t"
+        "ex2.approx.ftz.f32 p0, x0;\n\t"
+        "ex2.approx.ftz.f32 p1, x1;\n\t"
+        "cvt.rn.bf16x2.f32 %0, p1, p0;\n\t"
+        "mov.b64 p, {p0, p1};\n\t"
+        "add.rn.f32x2 t, %3, %6;\n\t"
+        "mul.rn.f32x2 d, p, t;\n\t"
+        "mov.b64 {d0, d1}, d;\n\t"
+        "cvt.rn.bf16x2.f32 %1, d1, d0;\n\t}"
+        : "=r"(pp), "=r"(pd)
+        : "l"(s2), "l"(dp2), "l"(sl2x2), "l"(nlse2), "l"(ndelta2));
+}
+
+// The same without bf16(p): the dQ kernel needs only dS.
+__device__ __forceinline__ uint32_t ds_pair(uint64_t s2, uint64_t dp2, uint64_t sl2x2,
+                                            uint64_t nlse2, uint64_t ndelta2) {
+    uint32_t pd;
+    asm("{\n\t.reg .b32 x0, x1, p0, p1, d0, d1;\n\t.reg .b64 x, p, t, d;\n\t"
+        "fma.rn.f32x2 x, %1, %3, %4;\n\t"
+        "mov.b64 {x0, x1}, x;\n\t"
+        "ex2.approx.ftz.f32 p0, x0;\n\t"
+        "ex2.approx.ftz.f32 p1, x1;\n\t"
+        "mov.b64 p, {p0, p1};\n\t"
+        "add.rn.f32x2 t, %2, %5;\n\t"
+        "mul.rn.f32x2 d, p, t;\n\t"
+        "mov.b64 {d0, d1}, d;\n\t"
+        "cvt.rn.bf16x2.f32 %0, d1, d0;\n\t}"
+        : "=r"(pd)
+        : "l"(s2), "l"(dp2), "l"(sl2x2), "l"(nlse2), "l"(ndelta2));
+    return pd;
+}
+
 // ------------------------------------------------------------------ Delta = rowsum(dO * O)
 // One warp per (b, t, h) row, fp32 accumulation of the bf16 products.
 template <int D>
@@ -232,11 +324,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
             mbar_init(bar(C::bar_full(s)), 1);
             mbar_init(bar(C::bar_empty(s)), 1);
         }
-        mbar_init(bar(C::BAR_SD), 1);
+        mbar_init(bar(C::BAR_SD), 2);  // one commit from each MMA thread
         mbar_init(bar(C::bar_ds(0)), 4 * 32);
         mbar_init(bar(C::bar_ds(1)), 4 * 32);
         mbar_init(bar(C::BAR_ACC), 1);
-        mbar_init(bar(C::BAR_DRAIN), 1);
+        mbar_init(bar(C::BAR_DRAIN), 2);
         mbar_init(bar(C::BAR_DPFREE), kComputeWarps * 32);
         *abort_flag = 0;
         fence_mbar_init();
@@ -295,8 +387,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
             for (int s = 0; s < C::NS; ++s)
                 if (armed[s] >= 0) wait_drain(bar(C::bar_full(s)), (armed[s] / C::NS) & 1, abort_flag, lim);
         }
-    } else if (warp == kWarpMma) {
+    } else if (warp == kWarpMma || warp == kWarpMma2) {
         if (lane == 0) {
+            const bool thread_a = warp == kWarpMma;
             constexpr uint32_t IDESC_S = idesc_bf16_f32(kBM, kBN, 0);  // K-major A and B
             constexpr uint32_t IDESC_O = idesc_bf16_f32(kBM, D, 1);    // B MN-major (D contiguous)
             const uint64_t dq_ = desc_sw128(base + C::OFF_A, 16, 1024);
@@ -328,44 +421,55 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
                            dkm + (uint64_t)((kk * 2048) >> 4), IDESC_O,
                            (jt > 0 || kk > 0) ? 1u : 0u);
             };
-            // Order per key tile jt: S(jt+1) into the other S region; dP(jt+1) once the
-            // compute warps have read dP(jt) (both overlap their work on tile jt); dQ over
-            // the first 64 keys once they publish them; after the second half is published,
-            // one commit for S(jt+1) and dP(jt+1), then dQ over the second 64 keys (it
-            // overlaps their next tile).
-            bool issued = false;
+            // Two issuing threads (one thread cannot issue 128-wide MMAs fast enough to keep
+            // the tensor core busy).  A issues S and dQ, B issues dP; no MMA reads the other
+            // thread's output columns, so they share only SD (one commit from each) and the
+            // drain.  A, per key tile jt: S(jt+1) into the other S region; dQ over each
+            // 64-key half as the compute warps publish it; after the second half, its share
+            // of SD(jt+1), then that half's dQ (it overlaps their next tile).  B, per key
+            // tile jt: dP(jt+1) once the compute warps have read dP(jt), and its share of
+            // SD(jt+1): dP(jt+1) overlaps their work on tile jt.
             if (wait1(bar(C::BAR_FIXED), 0, abort_flag, lim, kErrMma) && n > 0 &&
                 wait1(bar(C::bar_full(0)), 0, abort_flag, lim, kErrMma)) {
                 tc_fence_after();
-                issue_s(0);
-                issue_dp(0);
-                tc_commit(bar(C::BAR_SD));
-                issued = true;
-                for (int jt = 0; jt < n; ++jt) {
-                    const bool more = jt + 1 < n;
-                    const uint32_t ph = jt & 1;
-                    if (more) {
+                if (thread_a) {
+                    issue_s(0);
+                    tc_commit(bar(C::BAR_SD));
+                    for (int jt = 0; jt < n; ++jt) {
+                        const bool more = jt + 1 < n;
+                        const uint32_t ph = jt & 1;
+                        if (more) {
+                            if (!wait1(bar(C::bar_full((jt + 1) % C::NS)), ((jt + 1) / C::NS) & 1,
+                                       abort_flag, lim, kErrMma))
+                                break;
+                            tc_fence_after();
+                            issue_s(jt + 1);
+                        }
+                        if (!wait1(bar(C::bar_ds(0)), ph, abort_flag, lim, kErrMma)) break;
+                        tc_fence_after();
+                        dq_half(jt, 0);
+                        if (!wait1(bar(C::bar_ds(1)), ph, abort_flag, lim, kErrMma)) break;
+                        tc_fence_after();
+                        if (more) tc_commit(bar(C::BAR_SD));
+                        dq_half(jt, 1);
+                        tc_commit(bar(C::bar_empty(jt % C::NS)));
+                    }
+                } else {
+                    issue_dp(0);
+                    tc_commit(bar(C::BAR_SD));
+                    for (int jt = 0; jt + 1 < n; ++jt) {
+                        if (!wait1(bar(C::BAR_DPFREE), jt & 1, abort_flag, lim, kErrMma)) break;
                         if (!wait1(bar(C::bar_full((jt + 1) % C::NS)), ((jt + 1) / C::NS) & 1,
                                    abort_flag, lim, kErrMma))
                             break;
                         tc_fence_after();
-                        issue_s(jt + 1);
+                        issue_dp(jt + 1);
+                        tc_commit(bar(C::BAR_SD));
                     }
-                    if (!wait1(bar(C::BAR_DPFREE), ph, abort_flag, lim, kErrMma)) break;
-                    tc_fence_after();
-                    if (more) issue_dp(jt + 1);
-                    if (!wait1(bar(C::bar_ds(0)), ph, abort_flag, lim, kErrMma)) break;
-                    tc_fence_after();
-                    dq_half(jt, 0);
-                    if (!wait1(bar(C::bar_ds(1)), ph, abort_flag, lim, kErrMma)) break;
-                    tc_fence_after();
-                    if (more) tc_commit(bar(C::BAR_SD));
-                    dq_half(jt, 1);
-                    tc_commit(bar(C::bar_empty(jt % C::NS)));
                 }
             }
-            if (issued) {
-                tc_commit(bar(C::BAR_ACC));
+            if (n > 0) {  // a commit with nothing outstanding arrives at once
+                if (thread_a) tc_commit(bar(C::BAR_ACC));
                 tc_commit(bar(C::BAR_DRAIN));
                 wait_drain(bar(C::BAR_DRAIN), 0, abort_flag, lim);
             }
@@ -383,6 +487,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
         const float lse2 = row_ok ? p.lse[lrow] * 1.4426950408889634f : INFINITY;
         const float dlt = row_ok ? p.delta[lrow] : 0.f;
         const float sl2 = p.scale_log2;
+        const uint64_t sl2x2 = f2_pack(sl2, sl2), nlse2 = f2_pack(-lse2, -lse2),
+                       nd2 = f2_pack(-dlt, -dlt);
         bool ok = true;
         SchedIter it;
         it.begin(sched);
@@ -397,14 +503,24 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
             const int kvalid = min(kBN, p.Lc - it.t * kBN);
             const long long lim_c = p.causal ? my_row - k0 : (long long)kBN;  // keys c <= lim_c
             const uint32_t scol = C::s_col(jt);
-            {
-                float s[64], dp[64];
-                tmem_ld64(tmem + lane_off + scol + 64 * c, s);
-                tmem_ld64(tmem + lane_off + 128 + 64 * c, dp);
+            uint32_t pk[32];
+            // warp-uniform: the TMEM loads below are warp-collective
+            if (__all_sync(0xffffffffu, 64 * c + 63 < kvalid && 64 * c + 63 <= lim_c)) {
+                // every key of this half is visible to every row of the warp: packed pairs
+                uint64_t s2[32], d2[32];
+                tmem_ld64_pairs(tmem + lane_off + scol + 64 * c, s2);
+                tmem_ld64_pairs(tmem + lane_off + 128 + 64 * c, d2);
                 // dP is in registers: once both halves are, its columns may take dP(jt+1)
                 tc_fence_before();
                 mbar_arrive(bar(C::BAR_DPFREE));
-                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) pk[i] = ds_pair(s2[i], d2[i], sl2x2, nlse2, nd2);
+            } else {
+                float s[64], dp[64];
+                tmem_ld64(tmem + lane_off + scol + 64 * c, s);
+                tmem_ld64(tmem + lane_off + 128 + 64 * c, dp);
+                tc_fence_before();
+                mbar_arrive(bar(C::BAR_DPFREE));
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     float ds2[2];
@@ -417,12 +533,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
                     }
                     pk[i] = pack_bf16x2(ds2[0], ds2[1]);
                 }
-                // publish this 64-key half over its own S columns (already read)
-                tmem_st32(tmem + lane_off + scol + 64 * c, pk);
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(bar(C::bar_ds(c)));
             }
+            // publish this 64-key half over its own S columns (already read)
+            tmem_st32(tmem + lane_off + scol + 64 * c, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(C::bar_ds(c)));
         }
         if (ok && n > 0 && wait_warp(bar(C::BAR_ACC), 0, abort_flag, lim, kErrCompute)) {
             __syncwarp();
@@ -496,8 +612,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_sm100(const __grid_const
         mbar_init(bar(C::BAR_SD), 1);
         mbar_init(bar(C::bar_ds(0)), 4 * 32);
         mbar_init(bar(C::bar_ds(1)), 4 * 32);
-        mbar_init(bar(C::BAR_ACC), 1);
-        mbar_init(bar(C::BAR_DRAIN), 1);
+        mbar_init(bar(C::BAR_ACC), 2);  // dV from thread A, dK from thread B
+        mbar_init(bar(C::BAR_DRAIN), 2);
+        mbar_init(bar(C::BAR_XFREE), 1);
         mbar_init(bar(C::BAR_DPFREE), kComputeWarps * 32);
         *abort_flag = 0;
         fence_mbar_init();
@@ -514,8 +631,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_sm100(const __grid_const
     const uint32_t tmem = *tmem_slot;
 
     if (warp == kWarpLoad) {
-        // K and V once; per (head, query tile): Q, dO (TMA) and the 128 LSE / Delta values
-        // (plain loads by the whole warp, rows past L as +inf / 0) into one ring stage
+        // K and V once; per (head, query tile): Q, dO (TMA) and the 128 values -LSE log2(e)
+        // and -Delta (plain loads by the whole warp) into one ring stage
         if (lane == 0) {
             mbar_arrive_expect_tx(bar(C::BAR_FIXED), 2 * C::TILE);
             for (int kb = 0; kb < C::NKB; ++kb) {
@@ -544,8 +661,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_sm100(const __grid_const
             const long long lbase = ((long long)b * p.H_q + h) * p.L;
             for (int r = lane; r < kBM; r += 32) {
                 const long long row = (long long)q0 + r;
-                rows[r] = row < p.L ? p.lse[lbase + row] * 1.4426950408889634f : INFINITY;
-                rows[kBM + r] = row < p.L ? p.delta[lbase + row] : 0.f;
+                // negated: the compute warps add them (rows past L give P = 0, dS = 0)
+                rows[r] = row < p.L ? -(p.lse[lbase + row] * 1.4426950408889634f) : -INFINITY;
+                rows[kBM + r] = row < p.L ? -p.delta[lbase + row] : 0.f;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(C::bar_full(slot)));
@@ -556,8 +674,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_sm100(const __grid_const
             for (int s = 0; s < C::NS; ++s)
                 if (armed[s] >= 0) wait_drain(bar(C::bar_full(s)), (armed[s] / C::NS) & 1, abort_flag, lim);
         }
-    } else if (warp == kWarpMma) {
+    } else if (warp == kWarpMma || warp == kWarpMma2) {
         if (lane == 0) {
+            const bool thread_a = warp == kWarpMma;
             constexpr uint32_t IDESC_S = idesc_bf16_f32(kBN, kBM, 0);  // K-major A and B
             constexpr uint32_t IDESC_O = idesc_bf16_f32(kBN, D, 1);    // B MN-major (D contiguous)
             const uint64_t dk_ = desc_sw128(base + C::OFF_A, 16, 1024);
@@ -579,59 +698,73 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_sm100(const __grid_const
                     mma_ss(tmem + C::dpt_col(i), dv_ + off, ddo + off, IDESC_S, kk > 0 ? 1u : 0u);
                 }
             };
-            // dV += P^T dO and dK += dS^T Q over one 64-query half: P^T of the half in columns
-            // [64 half, 64 half + 32) of the S^T region, dS^T in the next 32; Q and dO as
-            // MN-major B (D contiguous, query rows 128 bytes apart)
-            auto dvdk_half = [&](int i, int half) {
-                const uint64_t dom = desc_sw128(stage(i) + C::TILE, C::BLK, 1024);
-                const uint64_t qm = desc_sw128(stage(i), C::BLK, 1024);
-                const uint32_t a0 = tmem + C::st_col(i) + 64 * half;
+            // dV += P^T dO (acc 0) or dK += dS^T Q (acc 1) over one 64-query half: P^T of the
+            // half in columns [64 half, 64 half + 32) of the S^T region, dS^T in the next 32;
+            // Q and dO as MN-major B (D contiguous, query rows 128 bytes apart)
+            auto acc_half = [&](int i, int half, int acc) {
+                const uint64_t bm = desc_sw128(stage(i) + (acc ? 0u : (uint32_t)C::TILE), C::BLK, 1024);
+                const uint32_t a0 = tmem + C::st_col(i) + 64 * half + 32 * acc;
 #pragma unroll
                 for (int kk = 4 * half; kk < 4 * half + 4; ++kk)
-                    mma_ts(tmem + 256, a0 + (kk % 4) * 8, dom + (uint64_t)((kk * 2048) >> 4),
-                           IDESC_O, (i > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-                for (int kk = 4 * half; kk < 4 * half + 4; ++kk)
-                    mma_ts(tmem + 256 + D, a0 + 32 + (kk % 4) * 8, qm + (uint64_t)((kk * 2048) >> 4),
+                    mma_ts(tmem + 256 + acc * D, a0 + (kk % 4) * 8, bm + (uint64_t)((kk * 2048) >> 4),
                            IDESC_O, (i > 0 || kk > 0) ? 1u : 0u);
             };
-            // Order per query tile i: S^T(i+1) into the dP^T region once the compute warps
-            // have read dP^T(i) (it overlaps their work on tile i); dV/dK over each 64-query
-            // half as they publish it; dP^T(i+1) into the S^T region (after the MMAs that
-            // read it) and one commit for S^T(i+1), dP^T(i+1).
-            bool issued = false;
+            // Two issuing threads.  A issues dP^T and dV, B issues S^T and dK.  dP^T(i+1)
+            // overwrites the region that dK(i) reads, so A first waits for B's x_free commit
+            // (after dK(i)); that commit also covers S^T(i+1), so A's commit of SD(i+1)
+            // alone tells the compute warps that the next tile's S^T and dP^T are ready.
+            // B, per query tile i: S^T(i+1) into the dP^T region once the compute warps have
+            // read dP^T(i) (it overlaps their work on tile i); dK over each half as they
+            // publish it; x_free.  A: dV over each half; then dP^T(i+1) into the S^T region
+            // and SD(i+1).
             if (wait1(bar(C::BAR_FIXED), 0, abort_flag, lim, kErrMma) && n > 0 &&
                 wait1(bar(C::bar_full(0)), 0, abort_flag, lim, kErrMma)) {
                 tc_fence_after();
-                issue_st(0);
-                issue_dpt(0);
-                tc_commit(bar(C::BAR_SD));
-                issued = true;
-                for (int it = 0; it < n; ++it) {
-                    const bool more = it + 1 < n;
-                    const uint32_t ph = it & 1;
-                    if (!wait1(bar(C::BAR_DPFREE), ph, abort_flag, lim, kErrMma)) break;
-                    if (more) {
-                        if (!wait1(bar(C::bar_full((it + 1) % C::NS)), ((it + 1) / C::NS) & 1,
-                                   abort_flag, lim, kErrMma))
-                            break;
+                if (thread_a) {
+                    issue_st(0);  // tile 0's S^T as well, so that SD has one committer
+                    issue_dpt(0);
+                    tc_commit(bar(C::BAR_SD));
+                    for (int it = 0; it < n; ++it) {
+                        const bool more = it + 1 < n;
+                        const uint32_t ph = it & 1;
+                        if (!wait1(bar(C::bar_ds(0)), ph, abort_flag, lim, kErrMma)) break;
                         tc_fence_after();
-                        issue_st(it + 1);
+                        acc_half(it, 0, 0);
+                        if (!wait1(bar(C::bar_ds(1)), ph, abort_flag, lim, kErrMma)) break;
+                        tc_fence_after();
+                        acc_half(it, 1, 0);
+                        if (more) {
+                            if (!wait1(bar(C::BAR_XFREE), ph, abort_flag, lim, kErrMma)) break;
+                            tc_fence_after();
+                        }
+                        tc_commit(bar(C::bar_empty(it % C::NS)));
+                        if (more) {
+                            issue_dpt(it + 1);
+                            tc_commit(bar(C::BAR_SD));
+                        }
                     }
-                    if (!wait1(bar(C::bar_ds(0)), ph, abort_flag, lim, kErrMma)) break;
-                    tc_fence_after();
-                    dvdk_half(it, 0);
-                    if (!wait1(bar(C::bar_ds(1)), ph, abort_flag, lim, kErrMma)) break;
-                    tc_fence_after();
-                    dvdk_half(it, 1);
-                    tc_commit(bar(C::bar_empty(it % C::NS)));
-                    if (more) {
-                        issue_dpt(it + 1);
-                        tc_commit(bar(C::BAR_SD));
+                } else {
+                    for (int it = 0; it < n; ++it) {
+                        const uint32_t ph = it & 1;
+                        if (it + 1 < n) {
+                            if (!wait1(bar(C::BAR_DPFREE), ph, abort_flag, lim, kErrMma)) break;
+                            if (!wait1(bar(C::bar_full((it + 1) % C::NS)), ((it + 1) / C::NS) & 1,
+                                       abort_flag, lim, kErrMma))
+                                break;
+                            tc_fence_after();
+                            issue_st(it + 1);
+                        }
+                        if (!wait1(bar(C::bar_ds(0)), ph, abort_flag, lim, kErrMma)) break;
+                        tc_fence_after();
+                        acc_half(it, 0, 1);
+                        if (!wait1(bar(C::bar_ds(1)), ph, abort_flag, lim, kErrMma)) break;
+                        tc_fence_after();
+                        acc_half(it, 1, 1);
+                        tc_commit(bar(C::BAR_XFREE));
                     }
                 }
             }
-            if (issued) {
+            if (n > 0) {  // a commit with nothing outstanding arrives at once
                 tc_commit(bar(C::BAR_ACC));
                 tc_commit(bar(C::BAR_DRAIN));
                 wait_drain(bar(C::BAR_DRAIN), 0, abort_flag, lim);
@@ -646,6 +779,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_sm100(const __grid_const
         const long long my_kpos = key0 + key_t;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const float sl2 = p.scale_log2;
+        const uint64_t sl2x2 = f2_pack(sl2, sl2);
         bool ok = true;
         for (int it = 0; it < n; ++it) {
             const int slot = it % C::NS;
@@ -660,14 +794,31 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_sm100(const __grid_const
             // queries c of the tile see this key when q0 + c >= key position (causal)
             const long long lo_c = p.causal ? my_kpos - q0 : 0;
             const uint32_t xs = C::st_col(it), yd = C::dpt_col(it);
-            {
-                float s[64], dp[64];
-                tmem_ld64(tmem + lane_off + xs + 64 * c, s);
-                tmem_ld64(tmem + lane_off + yd + 64 * c, dp);
+            uint32_t pp[32], pd[32];
+            // warp-uniform: the TMEM loads below are warp-collective
+            if (__all_sync(0xffffffffu, key_ok && lo_c <= 64 * c)) {
+                // every query of this half sees every key of the warp: packed pairs
+                uint64_t s2[32], d2[32];
+                tmem_ld64_pairs(tmem + lane_off + xs + 64 * c, s2);
+                tmem_ld64_pairs(tmem + lane_off + yd + 64 * c, d2);
                 // dP^T is in registers: once both halves are, its region may take S^T(it+1)
                 tc_fence_before();
                 mbar_arrive(bar(C::BAR_DPFREE));
-                uint32_t pp[32], pd[32];
+                const ulonglong2* nl = reinterpret_cast<const ulonglong2*>(rows + 64 * c);
+                const ulonglong2* nd = reinterpret_cast<const ulonglong2*>(rows + kBM + 64 * c);
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const ulonglong2 a = nl[k], d = nd[k];
+                    p_ds_pair(s2[2 * k], d2[2 * k], sl2x2, a.x, d.x, pp[2 * k], pd[2 * k]);
+                    p_ds_pair(s2[2 * k + 1], d2[2 * k + 1], sl2x2, a.y, d.y, pp[2 * k + 1],
+                              pd[2 * k + 1]);
+                }
+            } else {
+                float s[64], dp[64];
+                tmem_ld64(tmem + lane_off + xs + 64 * c, s);
+                tmem_ld64(tmem + lane_off + yd + 64 * c, dp);
+                tc_fence_before();
+                mbar_arrive(bar(C::BAR_DPFREE));
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     float pr2[2], ds2[2];
@@ -675,20 +826,20 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_sm100(const __grid_const
                     for (int e = 0; e < 2; ++e) {
                         const int col = 64 * c + 2 * i + e;
                         const bool vis = key_ok && col >= lo_c;
-                        const float pr = vis ? ex2_approx(s[2 * i + e] * sl2 - rows[col]) : 0.f;
+                        const float pr = vis ? ex2_approx(s[2 * i + e] * sl2 + rows[col]) : 0.f;
                         pr2[e] = pr;
-                        ds2[e] = pr * (dp[2 * i + e] - rows[kBM + col]);
+                        ds2[e] = pr * (dp[2 * i + e] + rows[kBM + col]);
                     }
                     pp[i] = pack_bf16x2(pr2[0], pr2[1]);
                     pd[i] = pack_bf16x2(ds2[0], ds2[1]);
                 }
-                // publish this 64-query half over the S^T columns just read
-                tmem_st32(tmem + lane_off + xs + 64 * c, pp);
-                tmem_st32(tmem + lane_off + xs + 64 * c + 32, pd);
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(bar(C::bar_ds(c)));
             }
+            // publish this 64-query half over the S^T columns just read
+            tmem_st32(tmem + lane_off + xs + 64 * c, pp);
+            tmem_st32(tmem + lane_off + xs + 64 * c + 32, pd);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(C::bar_ds(c)));
         }
         if (ok && n > 0 && wait_warp(bar(C::BAR_ACC), 0, abort_flag, lim, kErrCompute)) {
             __syncwarp();

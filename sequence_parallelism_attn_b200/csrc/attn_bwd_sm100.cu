@@ -40,7 +40,14 @@ __device__ unsigned int g_bwd_error_word = 0;
 
 namespace {
 
-constexpr int kThreads = 352;
+constexpr int kThreads = 352;    // dQ kernel
+constexpr int kThreadsKV = 384;  // dK/dV kernel: warp 11 only fills the third warpgroup
+// dK/dV register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64512), the
+// compute warpgroups rise to 200 and the third (load, MMA) falls to 104:
+// 2 x 128 x 200 + 128 x 104 = 64512, and per sub-partition 200 + 200 + 104 = 3 x 168.
+constexpr uint32_t kRegsKVLaunch = 168, kRegsKVCompute = 200, kRegsKVOther = 104;
+static_assert(2 * 128 * kRegsKVCompute + 128 * kRegsKVOther == kThreadsKV * kRegsKVLaunch,
+              "register split must use exactly the launch allocation");
 constexpr int kComputeWarps = 8;  // two warpgroups: one per 64-column half of every tile
 constexpr int kWarpLoad = 8;
 constexpr int kWarpMma = 9;   // MMA-issuing thread A (owns tensor memory)
@@ -577,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
 
 // ------------------------------------------------------------------ dK, dV (key tile stationary)
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_sm100(const __grid_constant__ BwdParams p) {
+__global__ void __launch_bounds__(kThreadsKV, 1) bwd_dkdv_sm100(const __grid_constant__ BwdParams p) {
     using C = BCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint32_t base = smem_u32(smem_raw);
@@ -630,7 +637,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_sm100(const __grid_const
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == kWarpLoad) {
+    if (warp >= kComputeWarps) {
+      regs_decrease<kRegsKVOther>();  // the whole third warpgroup, before its roles diverge
+      if (warp == kWarpLoad) {
         // K and V once; per (head, query tile): Q, dO (TMA) and the 128 values -LSE log2(e)
         // and -Delta (plain loads by the whole warp) into one ring stage
         if (lane == 0) {
@@ -770,7 +779,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_sm100(const __grid_const
                 wait_drain(bar(C::BAR_DRAIN), 0, abort_flag, lim);
             }
         }
+      }  // warp 11: no role
     } else {
+        regs_increase<kRegsKVCompute>();
         // compute warps: P^T and dS^T for this thread's key against its warpgroup's 64-query
         // half of the tile (a warp reaches TMEM lanes 32 (warp % 4) .. + 31)
         const int quarter = warp & 3, c = warp >> 2;
@@ -909,13 +920,22 @@ bool bwd_tile_map(CUtensorMap* m, const void* ptr, int D, int H, long long rows,
 }
 
 template <int D>
-cudaError_t launch_bwd_d(const BwdParams& p, const AttnBwdArgs& a) {
+cudaError_t launch_bwd_d(const BwdParams& p, const AttnBwdArgs& a, const char** why) {
     using C = BCfg<D>;
     static int configured_for = -1;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (configured_for != dev) {
+        // the dK/dV kernel's register split assumes its launch allocation: a raise beyond it
+        // would never complete
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, bwd_dkdv_sm100<D>);
+        if (e != cudaSuccess) return e;
+        if (fa.numRegs != (int)kRegsKVLaunch) {
+            *why = "dK/dV kernel compiled with a register count its register split does not assume";
+            return cudaErrorInvalidKernelImage;
+        }
         e = cudaFuncSetAttribute(bwd_dq_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(bwd_dkdv_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -932,7 +952,7 @@ cudaError_t launch_bwd_d(const BwdParams& p, const AttnBwdArgs& a) {
     bwd_dq_sm100<D><<<(unsigned)grid_q, kThreads, C::SMEM, a.stream>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    bwd_dkdv_sm100<D><<<(unsigned)grid_k, kThreads, C::SMEM, a.stream>>>(p);
+    bwd_dkdv_sm100<D><<<(unsigned)grid_k, kThreadsKV, C::SMEM, a.stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -976,8 +996,8 @@ cudaError_t launch_attn_bwd_sm100(const AttnBwdArgs& a, unsigned long long wait_
         *why = "problem too large for one launch";
         return cudaErrorInvalidValue;
     }
-    if (a.D == 128) return launch_bwd_d<128>(p, a);
-    if (a.D == 64) return launch_bwd_d<64>(p, a);
+    if (a.D == 128) return launch_bwd_d<128>(p, a, why);
+    if (a.D == 64) return launch_bwd_d<64>(p, a, why);
     *why = "head dimension not supported by the tensor-core backward";
     return cudaErrorInvalidValue;
 }

@@ -59,7 +59,13 @@ __device__ unsigned int g_ra_error_word = 0;
 namespace {
 
 constexpr int kThreads = 384;
-constexpr uint32_t kRegsSoftmax = 192, kRegsOther = 120;
+// setmaxnreg split of the launch allocation (168 per thread): the softmax warpgroups rise
+// to 192, the third falls to 120 (2 x 128 x 192 + 128 x 120 = 384 x 168).  The host checks
+// the compiled register count before the first launch: a raise beyond what the block was
+// launched with would never complete.
+constexpr uint32_t kRegsLaunch = 168, kRegsSoftmax = 192, kRegsOther = 120;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther == kThreads * kRegsLaunch,
+              "register split must use exactly the launch allocation");
 constexpr int kWarpLoad = 8;
 constexpr int kWarpMma = 9;
 constexpr int kWarpLoadV = 10;
@@ -649,13 +655,20 @@ bool encode_tile_map(CUtensorMap* m, const void* ptr, int D, int H, long long ro
 }
 
 template <int D>
-cudaError_t launch_d(const AttnParams& p, int grid, cudaStream_t stream) {
+cudaError_t launch_d(const AttnParams& p, int grid, cudaStream_t stream, const char** why) {
     using C = Cfg<D>;
     static int configured_for = -1;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (configured_for != dev) {
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, attn_fwd_sm100<D>);
+        if (e != cudaSuccess) return e;
+        if (fa.numRegs != (int)kRegsLaunch) {
+            *why = "attention kernel compiled with a register count its register split does not assume";
+            return cudaErrorInvalidKernelImage;
+        }
         e = cudaFuncSetAttribute(attn_fwd_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::SMEM);
         if (e != cudaSuccess) return e;
@@ -705,8 +718,8 @@ cudaError_t launch_attn_sm100(const AttnArgs& a, unsigned long long wait_limit_n
         *why = "problem too large for one launch";
         return cudaErrorInvalidValue;
     }
-    if (a.D == 128) return launch_d<128>(p, (int)grid, a.stream);
-    if (a.D == 64) return launch_d<64>(p, (int)grid, a.stream);
+    if (a.D == 128) return launch_d<128>(p, (int)grid, a.stream, why);
+    if (a.D == 64) return launch_d<64>(p, (int)grid, a.stream, why);
     *why = "head dimension not supported by the tensor-core path";
     return cudaErrorInvalidValue;
 }

@@ -59,6 +59,9 @@ __device__ unsigned int g_ra_error_word = 0;
 namespace {
 
 constexpr int kThreads = 384;
+// Shard layouts, compiled as separate kernels so that the contiguous layout's per-tile
+// softmax keeps plain index arithmetic: positions and sample starts only where they vary.
+constexpr int kLayoutContiguous = 0, kLayoutZigzag = 1, kLayoutPacked = 2;
 // setmaxnreg split of the launch allocation (168 per thread): the softmax warpgroups rise
 // to 192, the third falls to 120 (2 x 128 x 192 + 128 x 120 = 384 x 168).  The host checks
 // the compiled register count before the first launch: a raise beyond what the block was
@@ -322,7 +325,7 @@ __device__ __forceinline__ void mma_issuer(const AttnParams& p, uint32_t base, u
     }
 }
 
-template <int D>
+template <int D, int LAYOUT>
 __device__ __forceinline__ void softmax_wg(const AttnParams& p, uint32_t base, uint32_t tmem,
                                            const Sched& sched, int n, int wg, int b, int h,
                                            int r0, volatile int* abort_flag) {
@@ -336,19 +339,21 @@ __device__ __forceinline__ void softmax_wg(const AttnParams& p, uint32_t base, u
     const long long my_row = (long long)q_lo + wr * 32 + lane;
     // Sequence positions (L <= 2^30, so 32-bit): this thread's row, and the smallest among
     // the tile's rows (a key tile needs a mask only if some key comes after it).
+    constexpr int ZZ = LAYOUT == kLayoutZigzag ? 1 : 0;
+    constexpr bool PACKED = LAYOUT == kLayoutPacked;
     const int my_pos =
-        my_row < p.L ? (int)shard_pos(p.zigzag, p.P, p.Lc, (int)(my_row / p.Lc), my_row % p.Lc)
+        my_row < p.L ? (int)shard_pos(ZZ, p.P, p.Lc, (int)(my_row / p.Lc), my_row % p.Lc)
                      : p.L;
     // packed samples: the first key position this row may see (its sample's start)
     int my_start = 0;
-    if (p.pid && my_row < p.L) {
+    if (PACKED && my_row < p.L) {
         const int r = (int)my_row, st = r - p.pid[(long long)b * p.L + r];
         my_start = st < 0 ? 0 : (st > r ? r : st);
     }
     int tile_qmin = p.L;
     if (q_lo < p.L) {
         long long lo_pos, hi_pos;
-        row_pos_range(p.zigzag, p.P, p.Lc, q_lo, min((long long)q_lo + kBM - 1, (long long)p.L - 1),
+        row_pos_range(ZZ, p.P, p.Lc, q_lo, min((long long)q_lo + kBM - 1, (long long)p.L - 1),
                       lo_pos, hi_pos);
         tile_qmin = (int)lo_pos;
     }
@@ -378,28 +383,28 @@ __device__ __forceinline__ void softmax_wg(const AttnParams& p, uint32_t base, u
         const int kvalid = min(kBN, p.Lc - key0);
         const bool need_mask =
             (kvalid < kBN) ||
-            (p.causal && (int)shard_pos(p.zigzag, p.P, p.Lc, j, key0 + kvalid - 1) > tile_qmin) ||
-            (my_start > (int)shard_pos(p.zigzag, p.P, p.Lc, j, key0));
+            (p.causal && (int)shard_pos(ZZ, p.P, p.Lc, j, key0 + kvalid - 1) > tile_qmin) ||
+            (PACKED && my_start > (int)shard_pos(ZZ, p.P, p.Lc, j, key0));
         if (need_mask) {
             // The keys of the tile this row sees form one interval [c_lo, c_hi]: key c sits
             // at position kpos0 + c, except that a zigzag tile straddling the shard's two
             // segments continues from c = cs at the second segment's start -- and a row that
             // sees any key of the second segment sees every key of the first.  c_lo > 0
             // only for packed samples (keys before the row's sample start).
-            const int kpos0 = (int)shard_pos(p.zigzag, p.P, p.Lc, j, key0);
+            const int kpos0 = (int)shard_pos(ZZ, p.P, p.Lc, j, key0);
             auto clamp_c = [](int x) { return x < -1 ? -1 : (x > kBN ? kBN : x); };
             int c_hi = kvalid - 1;
             if (p.causal) {
                 int hi = clamp_c(my_pos - kpos0);
                 const int hseg = p.Lc / 2;
-                if (p.zigzag && key0 < hseg && key0 + kBN > hseg) {
+                if (ZZ && key0 < hseg && key0 + kBN > hseg) {
                     const int cs = hseg - key0;
                     const int hi2 = clamp_c(my_pos - (int)shard_pos(1, p.P, p.Lc, j, hseg) + cs);
                     hi = hi2 >= cs ? hi2 : min(hi, cs - 1);
                 }
                 c_hi = min(c_hi, hi);
             }
-            const int c_lo = clamp_c(my_start - kpos0);
+            const int c_lo = PACKED ? clamp_c(my_start - kpos0) : -1;
 #pragma unroll
             for (int i = 0; i < 64; ++i) {
                 float a, b;
@@ -513,7 +518,7 @@ __device__ __forceinline__ void softmax_wg(const AttnParams& p, uint32_t base, u
             (m_run + lg2_approx(l_run)) * 0.69314718055994530942f;
 }
 
-template <int D>
+template <int D, int LAYOUT>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100(const __grid_constant__ AttnParams p) {
     using C = Cfg<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -614,7 +619,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100(const __grid_const
         }
     } else {
         regs_increase<kRegsSoftmax>();
-        softmax_wg<D>(p, base, tmem, sched, n, warp >> 2, b, h, r0, abort_flag);
+        softmax_wg<D, LAYOUT>(p, base, tmem, sched, n, warp >> 2, b, h, r0, abort_flag);
     }
 
     tc_fence_before();
@@ -661,20 +666,25 @@ cudaError_t launch_d(const AttnParams& p, int grid, cudaStream_t stream, const c
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    decltype(&attn_fwd_sm100<D, kLayoutContiguous>) kernels[3] = {
+        attn_fwd_sm100<D, kLayoutContiguous>, attn_fwd_sm100<D, kLayoutZigzag>,
+        attn_fwd_sm100<D, kLayoutPacked>};
     if (configured_for != dev) {
-        cudaFuncAttributes fa;
-        e = cudaFuncGetAttributes(&fa, attn_fwd_sm100<D>);
-        if (e != cudaSuccess) return e;
-        if (fa.numRegs != (int)kRegsLaunch) {
-            *why = "attention kernel compiled with a register count its register split does not assume";
-            return cudaErrorInvalidKernelImage;
+        for (auto k : kernels) {
+            cudaFuncAttributes fa;
+            e = cudaFuncGetAttributes(&fa, k);
+            if (e != cudaSuccess) return e;
+            if (fa.numRegs != (int)kRegsLaunch) {
+                *why = "attention kernel compiled with a register count its register split does not assume";
+                return cudaErrorInvalidKernelImage;
+            }
+            e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+            if (e != cudaSuccess) return e;
         }
-        e = cudaFuncSetAttribute(attn_fwd_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::SMEM);
-        if (e != cudaSuccess) return e;
         configured_for = dev;
     }
-    attn_fwd_sm100<D><<<grid, kThreads, C::SMEM, stream>>>(p);
+    const int layout = p.pid ? kLayoutPacked : (p.zigzag ? kLayoutZigzag : kLayoutContiguous);
+    kernels[layout]<<<grid, kThreads, C::SMEM, stream>>>(p);
     return cudaGetLastError();
 }
 

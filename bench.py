@@ -14,7 +14,8 @@ the steps (max over ranks), in TFLOP/s.  With --gpus N every rank runs its own r
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload ulysses_e2e|ulysses_32k|usp_e2e|long_128k|long_128k_zigzag|long_128k_packed|
-                              long_128k_bwd|llama8b_32k_bwd|
+                              long_128k_bwd|long_128k_bwd_zigzag|long_128k_bwd_packed|
+                              llama8b_32k_bwd|
                               llama8b_32k|small_4k]
 """
 from __future__ import annotations
@@ -37,6 +38,9 @@ METRIC = "ring-chunked attention TFLOP/s & % BF16 tensor peak (1 B200); permute 
 UNIT = "TFLOP/s"
 DATASHEET_BF16_TFLOPS = 2250.0
 DATASHEET_HBM_GBS = 8000.0
+# workload name suffix of each path kind
+SUFFIX = {"attn_zigzag": "_zigzag", "attn_packed": "_packed", "attn_bwd": "_backward",
+          "attn_bwd_zigzag": "_zigzag_backward", "attn_bwd_packed": "_packed_backward"}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -60,6 +64,8 @@ def workloads():
         "long_128k_zigzag": ("attn_zigzag", synth.LONG_128K),
         "long_128k_packed": ("attn_packed", synth.LONG_128K),
         "long_128k_bwd": ("attn_bwd", synth.LONG_128K),
+        "long_128k_bwd_zigzag": ("attn_bwd_zigzag", synth.LONG_128K),
+        "long_128k_bwd_packed": ("attn_bwd_packed", synth.LONG_128K),
         "llama8b_32k": ("attn", synth.LLAMA8B_GQA),
         "llama8b_32k_bwd": ("attn_bwd", synth.LLAMA8B_GQA),
         "small_4k": ("attn", synth.SMALL_BF16),
@@ -181,7 +187,7 @@ class Path:
         self.ra, self.kind, self.w, self.dev = ra, kind, w, device
         # shard layout of the plain attention workloads (zigzag: rank i holds segments i and
         # 2P-1-i of 2P segments of Lc/2 tokens)
-        self.layout = "zigzag" if kind == "attn_zigzag" else "contiguous"
+        self.layout = "zigzag" if kind in ("attn_zigzag", "attn_bwd_zigzag") else "contiguous"
         if kind == "ulysses":
             a = w.attn()
             self.a = a
@@ -210,26 +216,27 @@ class Path:
             self.launches_per_step = 1
             self.flops = w.flops()
             self.pid = None
-            if kind == "attn_packed":
+            if kind in ("attn_packed", "attn_bwd_packed"):
                 # documents of 512..32768 tokens (log-uniform, seeded) packed into each row;
                 # the algorithmic work is each document's own causal attention
                 lens = synth.packed_lengths(w.L, w.seed + 21, 512, 32768)
                 self.pid = synth.position_ids_from_lengths([lens] * w.B).to(device)
                 self.flops = sum(4.0 * w.B * w.H_q * float(n) ** 2 * w.D / 2 for n in lens)
                 self.n_docs = len(lens)
-            if kind == "attn_bwd":
+            if kind.startswith("attn_bwd"):
                 # the backward pass: dout drawn like the inputs; the forward's O and LSE are
                 # produced once, outside the timed steps.  Algorithmic work: five matmuls
                 # (S recomputed, dP, dV, dK, dQ) against the forward's two -> 2.5x.
                 g = torch.Generator(device=device)
                 g.manual_seed(w.seed + 2)
                 self.dout = torch.randn(q.shape, generator=g, device=device).to(torch.bfloat16)
-                ra.ring_attn_fwd(q, k, v, w.causal, w.scale, out=self.o, lse=self.lse)
+                ra.ring_attn_fwd(q, k, v, w.causal, w.scale, out=self.o, lse=self.lse,
+                                 layout=self.layout, position_ids=self.pid)
                 self.dq = torch.empty((w.B, w.L, w.H_q, w.D), dtype=torch.float32, device=device)
                 self.dk = torch.empty(k.shape, dtype=torch.float32, device=device)
                 self.dv = torch.empty_like(self.dk)
                 self.ws = torch.empty((w.B, w.H_q, w.L), dtype=torch.float32, device=device)
-                self.flops = 2.5 * w.flops()
+                self.flops = 2.5 * self.flops
                 self.launches_per_step = 3
             self.permute_bytes = 0
             self.in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
@@ -253,11 +260,12 @@ class Path:
             rec("permute_out", 0)
             ra.ra_ulysses_head2seq(self.o.view(w.G, w.B, a.L, a.H_q, a.D), out=self.o_seq, P=w.P)
             rec("permute_out", 1)
-        elif self.kind == "attn_bwd":
+        elif self.kind.startswith("attn_bwd"):
             w = self.w
             rec("attn", 0)
             ra.ring_attn_bwd(self.q, self.k, self.v, self.o, self.lse, self.dout, w.causal,
-                             w.scale, dq=self.dq, dk=self.dk, dv=self.dv, workspace=self.ws)
+                             w.scale, dq=self.dq, dk=self.dk, dv=self.dv, workspace=self.ws,
+                             layout=self.layout, position_ids=self.pid)
             rec("attn", 1)
         else:
             w = self.w
@@ -462,8 +470,7 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": w.name + {"attn_zigzag": "_zigzag", "attn_packed": "_packed",
-                                         "attn_bwd": "_backward"}.get(kind, ""),
+        "config": {"workload": w.name + SUFFIX.get(kind, ""),
                    "global_batch": w_attn.B * world, "seq_len": w_attn.L,
                    "heads_q": w_attn.H_q, "heads_kv": w_attn.H_kv, "head_dim": w_attn.D,
                    "virtual_ranks": w_attn.P, "chunk_len": w_attn.Lc, "causal": w_attn.causal,
@@ -473,7 +480,7 @@ def main():
     if kind == "ulysses":
         # Ulysses: P head groups; the ring x Ulysses hybrid: fewer, each with a ring
         out["config"]["head_groups"] = w.G
-    if kind == "attn_packed":
+    if kind in ("attn_packed", "attn_bwd_packed"):
         out["config"]["packed_documents"] = path.n_docs
         out["config"]["document_lengths"] = "512..32768 tokens, log-uniform, seeded"
     sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
@@ -483,7 +490,7 @@ def main():
                        "frac": round(attn_tflops / sustained, 4),
                        "traffic": traffic,
                        "kernel": ("bwd_delta + bwd_dq_sm100 + bwd_dkdv_sm100, D=128"
-                                  if kind == "attn_bwd" else "attn_fwd_sm100<128>"),
+                                  if kind.startswith("attn_bwd") else "attn_fwd_sm100<128>"),
                        "peak_source": f"{peaks_src} bf16_tflops_sustained",
                        "frac_of_burst": round(attn_tflops / peaks.get("bf16_tflops", 1590.0), 4),
                        "frac_of_datasheet": round(attn_tflops / DATASHEET_BF16_TFLOPS, 4)}
@@ -545,8 +552,7 @@ def reference_arm(args, kind, w, w_attn, rank, world):
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
            "data": "synthetic",
-           "config": {"workload": w.name + {"attn_zigzag": "_zigzag", "attn_packed": "_packed",
-                                            "attn_bwd": "_backward"}.get(kind, ""),
+           "config": {"workload": w.name + SUFFIX.get(kind, ""),
                       "seq_len": w_attn.L, "head_dim": w_attn.D,
                       "causal": w_attn.causal, "parallelism": "cpu-oracle"},
            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",

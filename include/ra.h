@@ -206,6 +206,39 @@ RA_API ra_status ra_ring_attn_bwd(const void* q, const void* const* k_chunks,
                                   float* workspace, void* stream);
 
 /*
+ * ra_ring_attn_bwd_zigzag -- ra_ring_attn_bwd for shards in the zigzag layout: the
+ * gradients of ra_ring_attn_fwd_zigzag.  The same definition with every token at its
+ * sequence position (the layout of ra_ring_attn_fwd_zigzag); dq, dk_chunks and
+ * dv_chunks are in the same shard layout as q, k_chunks and v_chunks.
+ * Arguments as ra_ring_attn_bwd.  Errors: as ra_ring_attn_bwd; RA_ERR_INVALID when Lc
+ * is odd.
+ */
+RA_API ra_status ra_ring_attn_bwd_zigzag(const void* q, const void* const* k_chunks,
+                                         const void* const* v_chunks, const void* out,
+                                         const float* lse, const void* dout, int P, int B,
+                                         int H_q, int H_kv, int Lc, int D, long long q_bstride,
+                                         long long kv_bstride, float scale, int causal,
+                                         float* dq, float* const* dk_chunks,
+                                         float* const* dv_chunks, float* workspace, void* stream);
+
+/*
+ * ra_ring_attn_bwd_packed -- ra_ring_attn_bwd over packed samples: the gradients of
+ * ra_ring_attn_fwd_packed (causal; query t of batch row b sees the keys
+ * t - position_ids[b][t] .. t).  Every gradient is the sum over the pairs that the forward
+ * attended, so each sample's gradients are those of its own causal attention.
+ * position_ids: device, int32, [B][P*Lc] (the forward's).  Other arguments as
+ * ra_ring_attn_bwd (causal is implied).  Errors: as ra_ring_attn_bwd; RA_ERR_INVALID when
+ * position_ids is null or misaligned.
+ */
+RA_API ra_status ra_ring_attn_bwd_packed(const void* q, const void* const* k_chunks,
+                                         const void* const* v_chunks, const int* position_ids,
+                                         const void* out, const float* lse, const void* dout,
+                                         int P, int B, int H_q, int H_kv, int Lc, int D,
+                                         long long q_bstride, long long kv_bstride, float scale,
+                                         float* dq, float* const* dk_chunks,
+                                         float* const* dv_chunks, float* workspace, void* stream);
+
+/*
  * ra_ring_attn_bwd_static -- ra_ring_attn_bwd without a workspace argument: the Delta
  * rows live in a fixed device array inside the library, so a call allocates no device
  * memory (no cudaMalloc, no cudaFree, no allocating library routine).  The pages have no

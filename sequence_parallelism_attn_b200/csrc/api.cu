@@ -141,13 +141,18 @@ ra_status ra_ring_attn_fwd_packed(const void* q, const void* const* k_chunks,
                      1, in_dtype, out_dtype, out, lse, stream, 0, position_ids);
 }
 
-ra_status ra_ring_attn_bwd(const void* q, const void* const* k_chunks, const void* const* v_chunks,
-                           const void* out, const float* lse, const void* dout, int P, int B,
-                           int H_q, int H_kv, int Lc, int D, long long q_bstride,
-                           long long kv_bstride, float scale, int causal, float* dq,
-                           float* const* dk_chunks, float* const* dv_chunks, float* workspace,
-                           void* stream) {
+static ra_status ring_attn_bwd(const void* q, const void* const* k_chunks,
+                               const void* const* v_chunks, const void* out, const float* lse,
+                               const void* dout, int P, int B, int H_q, int H_kv, int Lc, int D,
+                               long long q_bstride, long long kv_bstride, float scale, int causal,
+                               float* dq, float* const* dk_chunks, float* const* dv_chunks,
+                               float* workspace, void* stream, int zigzag,
+                               const int* position_ids) {
     if (P < 1 || P > RA_MAX_P) return fail(RA_ERR_INVALID, "P must be in [1, RA_MAX_P]");
+    if (zigzag && Lc % 2 != 0)
+        return fail(RA_ERR_INVALID, "the zigzag layout needs an even chunk length Lc");
+    if (position_ids && (reinterpret_cast<uintptr_t>(position_ids) & 3u) != 0)
+        return fail(RA_ERR_INVALID, "position_ids must be 4-byte aligned");
     if (B < 1 || H_q < 1 || H_kv < 1 || Lc < 1 || D < 1)
         return fail(RA_ERR_INVALID, "B, H_q, H_kv, Lc and D must be >= 1");
     if (H_q % H_kv != 0) return fail(RA_ERR_INVALID, "H_q must be a multiple of H_kv");
@@ -194,11 +199,48 @@ ra_status ra_ring_attn_bwd(const void* q, const void* const* k_chunks, const voi
     a.dk_chunks = dk_chunks;
     a.dv_chunks = dv_chunks;
     a.workspace = workspace;
+    a.zigzag = zigzag;
+    a.pid = position_ids;
     a.stream = (cudaStream_t)stream;
     const char* why = "launch failed";
     cudaError_t e = ra::launch_attn_bwd_sm100(a, g_wait_limit_ns.load(), &why);
     if (e != cudaSuccess) return cuda_fail(e, why);
     return RA_OK;
+}
+
+ra_status ra_ring_attn_bwd(const void* q, const void* const* k_chunks, const void* const* v_chunks,
+                           const void* out, const float* lse, const void* dout, int P, int B,
+                           int H_q, int H_kv, int Lc, int D, long long q_bstride,
+                           long long kv_bstride, float scale, int causal, float* dq,
+                           float* const* dk_chunks, float* const* dv_chunks, float* workspace,
+                           void* stream) {
+    return ring_attn_bwd(q, k_chunks, v_chunks, out, lse, dout, P, B, H_q, H_kv, Lc, D, q_bstride,
+                         kv_bstride, scale, causal, dq, dk_chunks, dv_chunks, workspace, stream, 0,
+                         nullptr);
+}
+
+ra_status ra_ring_attn_bwd_zigzag(const void* q, const void* const* k_chunks,
+                                  const void* const* v_chunks, const void* out, const float* lse,
+                                  const void* dout, int P, int B, int H_q, int H_kv, int Lc, int D,
+                                  long long q_bstride, long long kv_bstride, float scale,
+                                  int causal, float* dq, float* const* dk_chunks,
+                                  float* const* dv_chunks, float* workspace, void* stream) {
+    return ring_attn_bwd(q, k_chunks, v_chunks, out, lse, dout, P, B, H_q, H_kv, Lc, D, q_bstride,
+                         kv_bstride, scale, causal, dq, dk_chunks, dv_chunks, workspace, stream, 1,
+                         nullptr);
+}
+
+ra_status ra_ring_attn_bwd_packed(const void* q, const void* const* k_chunks,
+                                  const void* const* v_chunks, const int* position_ids,
+                                  const void* out, const float* lse, const void* dout, int P, int B,
+                                  int H_q, int H_kv, int Lc, int D, long long q_bstride,
+                                  long long kv_bstride, float scale, float* dq,
+                                  float* const* dk_chunks, float* const* dv_chunks,
+                                  float* workspace, void* stream) {
+    if (!position_ids) return fail(RA_ERR_INVALID, "position_ids must be non-null");
+    return ring_attn_bwd(q, k_chunks, v_chunks, out, lse, dout, P, B, H_q, H_kv, Lc, D, q_bstride,
+                         kv_bstride, scale, 1, dq, dk_chunks, dv_chunks, workspace, stream, 0,
+                         position_ids);
 }
 
 ra_status ra_lse_merge(float* o_a, float* lse_a, const float* o_b, const float* lse_b, int B, int H,

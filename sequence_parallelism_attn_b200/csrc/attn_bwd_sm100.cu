@@ -27,6 +27,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
+#include <climits>
 #include <cmath>
 #include <cstdint>
 #include "ra_internal.h"
@@ -69,9 +70,15 @@ struct __align__(64) BwdParams {
     float* dk[RA_MAX_P];  // chunk j: [B][Lc][H_kv][D]
     float* dv[RA_MAX_P];
     int P, B, H_q, H_kv, Lc, L, causal, group, n_qblocks, ntc;
+    int zigzag;       // shards in the zigzag layout
+    const int* pid;   // packed samples: position_ids [B][L] (else null)
     float scale, scale_log2;
     unsigned long long wait_limit_ns;
 };
+
+// Shard layouts, compiled as separate kernels (the contiguous one keeps plain index
+// arithmetic per tile).
+constexpr int kLayoutContiguous = 0, kLayoutZigzag = 1, kLayoutPacked = 2;
 
 template <int D>
 struct BCfg {
@@ -84,7 +91,11 @@ struct BCfg {
     static constexpr int OFF_A = 0;                      // Q (dQ) / K (dK/dV)
     static constexpr int OFF_B = TILE;                   // dO (dQ) / V (dK/dV)
     static constexpr int OFF_RING = 2 * TILE;            // NS x (two tiles) stages
-    static constexpr int STAGE = 2 * TILE + 2 * kBM * 4; // + LSE and Delta rows (dK/dV)
+    // + per query row of the stage (dK/dV kernel): -LSE log2(e), -Delta (fp32), sequence
+    // position and sample start (int32), and per 64-row half the smallest position and the
+    // largest start; padded to keep every stage 1024-byte aligned
+    static constexpr int ROWS_BYTES = 4 * kBM * 4 + 4 * 4;
+    static constexpr int STAGE = 2 * TILE + ((ROWS_BYTES + 1023) / 1024) * 1024;
     static constexpr int OFF_BAR = OFF_RING + NS * STAGE;
     // barriers: fixed_full, full[NS], empty[NS], sd_full, ds_full[2] (one per 64-column
     // half of dS / P^T), acc_done, drain, dp_free (the compute warps have read all of dP),
@@ -92,7 +103,9 @@ struct BCfg {
     static constexpr int N_BARS = 1 + 2 * NS + 7;
     static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem base, abort flag, n
     static constexpr int OFF_SCHED = OFF_MISC + 16;
-    static constexpr int SMEM = OFF_SCHED + 2 * RA_MAX_P * 4 + 1024;
+    // dK/dV kernel, zigzag / packed: ascending query-tile ranges [lo, hi), at most 2 per rank
+    static constexpr int OFF_QR = OFF_SCHED + 2 * RA_MAX_P * 4;
+    static constexpr int SMEM = OFF_QR + 2 * RA_MAX_P * 8 + 1024;
     static constexpr int BAR_FIXED = 0;
     __host__ __device__ static constexpr int bar_full(int s) { return 1 + s; }
     __host__ __device__ static constexpr int bar_empty(int s) { return 1 + NS + s; }
@@ -112,6 +125,7 @@ struct BCfg {
     __host__ __device__ static constexpr uint32_t st_col(int i) { return (i & 1) ? 128u : 0u; }
     __host__ __device__ static constexpr uint32_t dpt_col(int i) { return (i & 1) ? 0u : 128u; }
     static_assert(SMEM <= 232448, "shared memory budget");
+    static_assert(STAGE % 1024 == 0, "TMA destinations of every stage stay 1024-byte aligned");
     static_assert(256 + 2 * D <= (int)kTmemCols, "tensor memory budget");
     static_assert(256 + D <= (int)S_ODD && S_ODD + kBN <= kTmemCols, "dQ kernel columns");
 };
@@ -276,6 +290,88 @@ __device__ __forceinline__ uint32_t ds_pair(uint64_t s2, uint64_t dp2, uint64_t 
     return pd;
 }
 
+// ------------------------------------------------------------------ layout helpers
+// Sample start of row r of batch row b (packed samples: r - position_ids[b][r], clamped to
+// [0, r] as in the forward).
+__device__ __forceinline__ int sample_start(const BwdParams& p, int b, int r) {
+    const int st = r - p.pid[(long long)b * p.L + r];
+    return st < 0 ? 0 : (st > r ? r : st);
+}
+
+// The keys of tile (chunk j, local keys key0 .. key0 + kvalid - 1) that a query at sequence
+// position my_pos with sample start my_start sees form one interval [c_lo, c_hi] of tile
+// columns (empty when c_lo > c_hi).  Key c sits at position kpos0 + c, except that a zigzag
+// tile straddling the shard's two segments continues from c = cs at the second segment's
+// start, and a query that sees a key of the second segment sees all of the first.
+template <int LAYOUT>
+__device__ __forceinline__ void key_interval(const BwdParams& p, int j, int key0, int kvalid,
+                                             int my_pos, int my_start, int& c_lo, int& c_hi) {
+    constexpr int ZZ = LAYOUT == kLayoutZigzag ? 1 : 0;
+    const int kpos0 = (int)shard_pos(ZZ, p.P, p.Lc, j, key0);
+    auto clamp_c = [](int x) { return x < -1 ? -1 : (x > kBN ? kBN : x); };
+    c_hi = kvalid - 1;
+    if (p.causal) {
+        int hi = clamp_c(my_pos - kpos0);
+        const int hseg = p.Lc / 2;
+        if (ZZ && key0 < hseg && key0 + kBN > hseg) {
+            const int cs = hseg - key0;
+            const int hi2 = clamp_c(my_pos - (int)shard_pos(1, p.P, p.Lc, j, hseg) + cs);
+            hi = hi2 >= cs ? hi2 : min(hi, cs - 1);
+        }
+        c_hi = min(c_hi, hi);
+    }
+    c_lo = LAYOUT == kLayoutPacked ? clamp_c(my_start - kpos0) : -1;
+}
+
+// dK/dV kernel: the query tiles whose rows may see a key of the tile (chunk j, local keys
+// key0 .. key0 + kvalid - 1), as ascending disjoint ranges [lo, hi) of tile indices written
+// to qr (at most 2 P).  Returns the number of ranges and sets *n_tiles.  Zigzag, causal:
+// rows at a position >= the tile's first key position, which in every half-shard is a
+// suffix; packed (causal): rows from the tile's first key to the last row whose sample
+// starts at or before the tile's last key (sample starts do not decrease along a row).
+template <int LAYOUT>
+__device__ int build_q_ranges(const BwdParams& p, int b, int j, int key0, int kvalid, int2* qr,
+                              int* n_tiles) {
+    int nr = 0;
+    auto add_rows = [&](long long row_lo, long long row_hi) {  // rows [row_lo, row_hi)
+        if (row_lo >= row_hi) return;
+        const int lo = (int)(row_lo / kBM), hi = (int)((row_hi - 1) / kBM) + 1;
+        if (nr > 0 && lo <= qr[nr - 1].y) {
+            qr[nr - 1].y = max(qr[nr - 1].y, hi);
+        } else {
+            qr[nr].x = lo;
+            qr[nr].y = hi;
+            ++nr;
+        }
+    };
+    if (!p.causal) {
+        add_rows(0, p.L);
+    } else if (LAYOUT == kLayoutZigzag) {
+        const long long h = p.Lc / 2;
+        const long long kmin = shard_pos(1, p.P, p.Lc, j, key0);
+        for (int r = 0; r < p.P; ++r) {
+            const long long base = (long long)r * p.Lc;
+            const long long u1 = max(0LL, kmin - (long long)r * h);  // first half: r h + u
+            if (u1 < h) add_rows(base + u1, base + h);
+            const long long u2 = h + max(0LL, kmin - (2LL * p.P - 1 - r) * h);
+            if (u2 < p.Lc) add_rows(base + u2, base + p.Lc);
+        }
+    } else {
+        const int k0 = j * p.Lc + key0, k_last = k0 + kvalid - 1;
+        int lo = k0 / kBM, hi = p.n_qblocks - 1;  // the last tile whose first row's sample
+        while (lo < hi) {                         // starts at or before k_last
+            const int mid = (lo + hi + 1) / 2;
+            if (sample_start(p, b, mid * kBM) <= k_last) lo = mid;
+            else hi = mid - 1;
+        }
+        add_rows((long long)(k0 / kBM) * kBM, (long long)(lo + 1) * kBM);
+    }
+    int n = 0;
+    for (int i = 0; i < nr; ++i) n += qr[i].y - qr[i].x;
+    *n_tiles = n;
+    return nr;
+}
+
 // ------------------------------------------------------------------ Delta = rowsum(dO * O)
 // One warp per (b, t, h) row, fp32 accumulation of the bf16 products.
 template <int D>
@@ -301,7 +397,7 @@ __global__ void __launch_bounds__(256) bwd_delta_kernel(const uint16_t* __restri
 }
 
 // ------------------------------------------------------------------ dQ (query tile stationary)
-template <int D>
+template <int D, int LAYOUT>
 __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constant__ BwdParams p) {
     using C = BCfg<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -343,7 +439,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
     }
     if (warp == kWarpLoad) {
         SchedArgs sa;
-        sa.P = p.P; sa.Lc = p.Lc; sa.L = p.L; sa.causal = p.causal; sa.zigzag = 0; sa.pid = nullptr;
+        sa.P = p.P; sa.Lc = p.Lc; sa.L = p.L; sa.causal = p.causal;
+        sa.zigzag = LAYOUT == kLayoutZigzag ? 1 : 0;
+        sa.pid = LAYOUT == kLayoutPacked ? p.pid : nullptr;
         const long long last_row = min((long long)r0 + kBM - 1, (long long)p.L - 1);
         const int nt = make_schedule(sa, b, r0, last_row, sched_range);
         if (lane == 0) *n_slot = nt;
@@ -496,6 +594,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
         const float sl2 = p.scale_log2;
         const uint64_t sl2x2 = f2_pack(sl2, sl2), nlse2 = f2_pack(-lse2, -lse2),
                        nd2 = f2_pack(-dlt, -dlt);
+        // zigzag / packed: this row's sequence position and sample start (L <= 2^30)
+        constexpr int ZZ = LAYOUT == kLayoutZigzag ? 1 : 0;
+        const int my_pos = row_ok ? (int)shard_pos(ZZ, p.P, p.Lc, (int)(my_row / p.Lc), my_row % p.Lc)
+                                  : p.L;
+        const int my_start = (LAYOUT == kLayoutPacked && row_ok) ? sample_start(p, b, (int)my_row) : 0;
         bool ok = true;
         SchedIter it;
         it.begin(sched);
@@ -506,13 +609,20 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
             }
             __syncwarp();
             tc_fence_after();
-            const long long k0 = (long long)it.chunk() * p.Lc + (long long)it.t * kBN;
             const int kvalid = min(kBN, p.Lc - it.t * kBN);
-            const long long lim_c = p.causal ? my_row - k0 : (long long)kBN;  // keys c <= lim_c
+            // this row sees the tile's keys c with c_lo <= c <= c_hi
+            int c_lo = -1, c_hi;
+            if (LAYOUT == kLayoutContiguous) {
+                const long long k0 = (long long)it.chunk() * p.Lc + (long long)it.t * kBN;
+                const long long lim = p.causal ? my_row - k0 : (long long)kBN;
+                c_hi = (int)min((long long)(kvalid - 1), lim < -1 ? -1LL : lim);
+            } else {
+                key_interval<LAYOUT>(p, it.chunk(), it.t * kBN, kvalid, my_pos, my_start, c_lo, c_hi);
+            }
             const uint32_t scol = C::s_col(jt);
             uint32_t pk[32];
             // warp-uniform: the TMEM loads below are warp-collective
-            if (__all_sync(0xffffffffu, 64 * c + 63 < kvalid && 64 * c + 63 <= lim_c)) {
+            if (__all_sync(0xffffffffu, 64 * c >= c_lo && 64 * c + 63 <= c_hi)) {
                 // every key of this half is visible to every row of the warp: packed pairs
                 uint64_t s2[32], d2[32];
                 tmem_ld64_pairs(tmem + lane_off + scol + 64 * c, s2);
@@ -534,7 +644,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         const int col = 64 * c + 2 * i + e;
-                        const bool vis = col < kvalid && col <= lim_c;
+                        const bool vis = col >= c_lo && col <= c_hi;
                         const float pr = vis ? ex2_approx(s[2 * i + e] * sl2 - lse2) : 0.f;
                         ds2[e] = pr * (dp[2 * i + e] - dlt);
                     }
@@ -583,7 +693,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
 }
 
 // ------------------------------------------------------------------ dK, dV (key tile stationary)
-template <int D>
+template <int D, int LAYOUT>
 __global__ void __launch_bounds__(kThreadsKV, 1) bwd_dkdv_sm100(const __grid_constant__ BwdParams p) {
     using C = BCfg<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -593,9 +703,13 @@ __global__ void __launch_bounds__(kThreadsKV, 1) bwd_dkdv_sm100(const __grid_con
     uint8_t* smem = smem_raw + pad;
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+    volatile int* n_slot = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
+    volatile int* nr_slot = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 12);
+    int2* qr = reinterpret_cast<int2*>(smem + C::OFF_QR);
     auto bar = [&](int i) { return base + C::OFF_BAR + 8u * (uint32_t)i; };
     const unsigned long long lim = p.wait_limit_ns;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr bool CONTIG = LAYOUT == kLayoutContiguous;
 
     // grid: (batch, kv head) outermost, then the key tiles (chunk j, tile t) heaviest first
     // (causal: the first keys are seen by the most query rows)
@@ -603,12 +717,12 @@ __global__ void __launch_bounds__(kThreadsKV, 1) bwd_dkdv_sm100(const __grid_con
     const int bg = (int)(blockIdx.x / n_kt), kt = (int)(blockIdx.x % n_kt);
     const int b = bg / p.H_kv, g = bg % p.H_kv;
     const int j = kt / p.ntc, t = kt % p.ntc;
-    const long long key0 = (long long)j * p.Lc + (long long)t * kBN;  // sequence position
+    const long long key0 = (long long)j * p.Lc + (long long)t * kBN;  // contiguous position
     const int kvalid = min(kBN, p.Lc - t * kBN);
-    // query tiles that can see a key of this tile: rows >= key0 when causal
+    // contiguous layout: the query tiles that can see a key of this tile are those holding
+    // rows >= key0 when causal (zigzag / packed: the ranges built below)
     const int qt0 = p.causal ? (int)(key0 / kBM) : 0;
     const int n_qt = p.n_qblocks - qt0;
-    const int n = n_qt * p.group;  // (head, query tile) pairs, head-major
 
     if (threadIdx.x == 0) {
         mbar_init(bar(C::BAR_FIXED), 1);
@@ -627,6 +741,11 @@ __global__ void __launch_bounds__(kThreadsKV, 1) bwd_dkdv_sm100(const __grid_con
         fence_mbar_init();
         fence_proxy_async_smem();
     }
+    if (!CONTIG && warp == kWarpLoad && lane == 0) {
+        int nt = 0;
+        *nr_slot = build_q_ranges<LAYOUT>(p, b, j, t * kBN, kvalid, qr, &nt);
+        *n_slot = nt * p.group;
+    }
     if (warp == kWarpMma) {
         __syncwarp();
         tmem_alloc(base + C::OFF_MISC, kTmemCols);
@@ -636,6 +755,7 @@ __global__ void __launch_bounds__(kThreadsKV, 1) bwd_dkdv_sm100(const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    const int n = CONTIG ? n_qt * p.group : *n_slot;  // (head, query tile) pairs, head-major
 
     if (warp >= kComputeWarps) {
       regs_decrease<kRegsKVOther>();  // the whole third warpgroup, before its roles diverge
@@ -651,13 +771,12 @@ __global__ void __launch_bounds__(kThreadsKV, 1) bwd_dkdv_sm100(const __grid_con
         }
         int armed[C::NS];
         for (int s = 0; s < C::NS; ++s) armed[s] = -1;
-        for (int it = 0; it < n; ++it) {
+        // item it = (query head h, query tile starting at row q0) into stage it % NS
+        auto produce = [&](int it, int h, int q0) -> bool {
             const int slot = it % C::NS;
-            const int h = g * p.group + it / n_qt;
-            const int q0 = (qt0 + it % n_qt) * kBM;
             if (it >= C::NS &&
                 !wait_warp(bar(C::bar_empty(slot)), ((it / C::NS) - 1) & 1, abort_flag, lim, kErrLoad))
-                break;
+                return false;
             const uint32_t st = base + C::OFF_RING + slot * C::STAGE;
             if (lane == 0) {
                 mbar_arrive_expect_tx(bar(C::bar_full(slot)), 2 * C::TILE);
@@ -668,15 +787,56 @@ __global__ void __launch_bounds__(kThreadsKV, 1) bwd_dkdv_sm100(const __grid_con
             }
             float* rows = reinterpret_cast<float*>(smem + C::OFF_RING + slot * C::STAGE + 2 * C::TILE);
             const long long lbase = ((long long)b * p.H_q + h) * p.L;
+            int pmin0 = INT_MAX, pmin1 = INT_MAX, smax0 = 0, smax1 = 0;
             for (int r = lane; r < kBM; r += 32) {
                 const long long row = (long long)q0 + r;
                 // negated: the compute warps add them (rows past L give P = 0, dS = 0)
                 rows[r] = row < p.L ? -(p.lse[lbase + row] * 1.4426950408889634f) : -INFINITY;
                 rows[kBM + r] = row < p.L ? -p.delta[lbase + row] : 0.f;
+                if (!CONTIG) {
+                    // the row's sequence position and sample start: it sees the keys at
+                    // positions start .. pos (every key when not causal)
+                    int pos = INT_MAX, start = 0;
+                    if (row < p.L && p.causal) {
+                        pos = (int)shard_pos(LAYOUT == kLayoutZigzag ? 1 : 0, p.P, p.Lc,
+                                             (int)(row / p.Lc), row % p.Lc);
+                        if (LAYOUT == kLayoutPacked) start = sample_start(p, b, (int)row);
+                    }
+                    reinterpret_cast<int*>(rows)[2 * kBM + r] = pos;
+                    reinterpret_cast<int*>(rows)[3 * kBM + r] = start;
+                    if (r < kBM / 2) { pmin0 = min(pmin0, pos); smax0 = max(smax0, start); }
+                    else { pmin1 = min(pmin1, pos); smax1 = max(smax1, start); }
+                }
+            }
+            if (!CONTIG) {
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    pmin0 = min(pmin0, __shfl_xor_sync(0xffffffffu, pmin0, off));
+                    pmin1 = min(pmin1, __shfl_xor_sync(0xffffffffu, pmin1, off));
+                    smax0 = max(smax0, __shfl_xor_sync(0xffffffffu, smax0, off));
+                    smax1 = max(smax1, __shfl_xor_sync(0xffffffffu, smax1, off));
+                }
+                if (lane == 0) {
+                    int* sum = reinterpret_cast<int*>(rows) + 4 * kBM;
+                    sum[0] = pmin0; sum[1] = pmin1; sum[2] = smax0; sum[3] = smax1;
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(C::bar_full(slot)));
             armed[slot] = it;
+            return true;
+        };
+        if (CONTIG) {
+            for (int it = 0; it < n; ++it)
+                if (!produce(it, g * p.group + it / n_qt, (qt0 + it % n_qt) * kBM)) break;
+        } else {
+            const int nr = *nr_slot;
+            int it = 0;
+            bool go = true;
+            for (int hh = 0; go && hh < p.group; ++hh)
+                for (int ri = 0; go && ri < nr; ++ri)
+                    for (int qt = qr[ri].x; go && qt < qr[ri].y; ++qt, ++it)
+                        go = produce(it, g * p.group + hh, qt * kBM);
         }
         if (lane == 0) {
             wait_drain(bar(C::BAR_FIXED), 0, abort_flag, lim);
@@ -787,7 +947,10 @@ __global__ void __launch_bounds__(kThreadsKV, 1) bwd_dkdv_sm100(const __grid_con
         const int quarter = warp & 3, c = warp >> 2;
         const int key_t = quarter * 32 + lane;
         const bool key_ok = key_t < kvalid;
-        const long long my_kpos = key0 + key_t;
+        // the key's sequence position (contiguous: key0 + key_t)
+        const int my_kpos = key_ok ? (int)shard_pos(LAYOUT == kLayoutZigzag ? 1 : 0, p.P, p.Lc, j,
+                                                    t * kBN + key_t)
+                                   : INT_MAX;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const float sl2 = p.scale_log2;
         const uint64_t sl2x2 = f2_pack(sl2, sl2);
@@ -802,12 +965,19 @@ __global__ void __launch_bounds__(kThreadsKV, 1) bwd_dkdv_sm100(const __grid_con
             __syncwarp();
             tc_fence_after();
             const float* rows = reinterpret_cast<const float*>(smem + C::OFF_RING + slot * C::STAGE + 2 * C::TILE);
-            // queries c of the tile see this key when q0 + c >= key position (causal)
-            const long long lo_c = p.causal ? my_kpos - q0 : 0;
+            // contiguous: queries c of the tile see this key when q0 + c >= its position
+            // (causal); zigzag / packed: when start[c] <= its position <= pos[c], with the
+            // per-row positions and starts, and their per-half bounds, in the stage
+            const long long lo_c = p.causal ? (long long)my_kpos - q0 : 0;
+            const int* posv = reinterpret_cast<const int*>(rows) + 2 * kBM;
+            const int* startv = reinterpret_cast<const int*>(rows) + 3 * kBM;
+            const bool half_visible =
+                CONTIG ? lo_c <= 64 * c
+                       : (my_kpos <= posv[2 * kBM + c] && my_kpos >= posv[2 * kBM + 2 + c]);
             const uint32_t xs = C::st_col(it), yd = C::dpt_col(it);
             uint32_t pp[32], pd[32];
             // warp-uniform: the TMEM loads below are warp-collective
-            if (__all_sync(0xffffffffu, key_ok && lo_c <= 64 * c)) {
+            if (__all_sync(0xffffffffu, key_ok && half_visible)) {
                 // every query of this half sees every key of the warp: packed pairs
                 uint64_t s2[32], d2[32];
                 tmem_ld64_pairs(tmem + lane_off + xs + 64 * c, s2);
@@ -836,7 +1006,9 @@ __global__ void __launch_bounds__(kThreadsKV, 1) bwd_dkdv_sm100(const __grid_con
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         const int col = 64 * c + 2 * i + e;
-                        const bool vis = key_ok && col >= lo_c;
+                        const bool vis =
+                            key_ok && (CONTIG ? col >= lo_c
+                                              : (my_kpos <= posv[col] && my_kpos >= startv[col]));
                         const float pr = vis ? ex2_approx(s[2 * i + e] * sl2 + rows[col]) : 0.f;
                         pr2[e] = pr;
                         ds2[e] = pr * (dp[2 * i + e] + rows[kBM + col]);
@@ -926,22 +1098,31 @@ cudaError_t launch_bwd_d(const BwdParams& p, const AttnBwdArgs& a, const char** 
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    decltype(&bwd_dq_sm100<D, kLayoutContiguous>) dq_k[3] = {
+        bwd_dq_sm100<D, kLayoutContiguous>, bwd_dq_sm100<D, kLayoutZigzag>,
+        bwd_dq_sm100<D, kLayoutPacked>};
+    decltype(&bwd_dkdv_sm100<D, kLayoutContiguous>) kv_k[3] = {
+        bwd_dkdv_sm100<D, kLayoutContiguous>, bwd_dkdv_sm100<D, kLayoutZigzag>,
+        bwd_dkdv_sm100<D, kLayoutPacked>};
     if (configured_for != dev) {
-        // the dK/dV kernel's register split assumes its launch allocation: a raise beyond it
-        // would never complete
-        cudaFuncAttributes fa;
-        e = cudaFuncGetAttributes(&fa, bwd_dkdv_sm100<D>);
-        if (e != cudaSuccess) return e;
-        if (fa.numRegs != (int)kRegsKVLaunch) {
-            *why = "dK/dV kernel compiled with a register count its register split does not assume";
-            return cudaErrorInvalidKernelImage;
+        for (int l = 0; l < 3; ++l) {
+            // the dK/dV kernel's register split assumes its launch allocation: a raise
+            // beyond it would never complete
+            cudaFuncAttributes fa;
+            e = cudaFuncGetAttributes(&fa, kv_k[l]);
+            if (e != cudaSuccess) return e;
+            if (fa.numRegs != (int)kRegsKVLaunch) {
+                *why = "dK/dV kernel compiled with a register count its register split does not assume";
+                return cudaErrorInvalidKernelImage;
+            }
+            e = cudaFuncSetAttribute(dq_k[l], cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(kv_k[l], cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+            if (e != cudaSuccess) return e;
         }
-        e = cudaFuncSetAttribute(bwd_dq_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(bwd_dkdv_sm100<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-        if (e != cudaSuccess) return e;
         configured_for = dev;
     }
+    const int layout = p.pid ? kLayoutPacked : (p.zigzag ? kLayoutZigzag : kLayoutContiguous);
     const long long rows = (long long)a.B * p.L * a.H_q;
     bwd_delta_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, a.stream>>>(
         (const uint16_t*)a.out, (const uint16_t*)a.dout, a.workspace, a.B, p.L, a.H_q);
@@ -949,10 +1130,10 @@ cudaError_t launch_bwd_d(const BwdParams& p, const AttnBwdArgs& a, const char** 
     if (e != cudaSuccess) return e;
     const long long grid_q = (long long)p.n_qblocks * a.B * a.H_q;
     const long long grid_k = (long long)a.B * a.H_kv * a.P * p.ntc;
-    bwd_dq_sm100<D><<<(unsigned)grid_q, kThreads, C::SMEM, a.stream>>>(p);
+    dq_k[layout]<<<(unsigned)grid_q, kThreads, C::SMEM, a.stream>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    bwd_dkdv_sm100<D><<<(unsigned)grid_k, kThreadsKV, C::SMEM, a.stream>>>(p);
+    kv_k[layout]<<<(unsigned)grid_k, kThreadsKV, C::SMEM, a.stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -986,6 +1167,8 @@ cudaError_t launch_attn_bwd_sm100(const AttnBwdArgs& a, unsigned long long wait_
     p.Lc = a.Lc;
     p.L = (int)L;
     p.causal = a.causal;
+    p.zigzag = a.zigzag;
+    p.pid = a.pid;
     p.group = a.H_q / a.H_kv;
     p.n_qblocks = (int)((L + kBM - 1) / kBM);
     p.ntc = (a.Lc + kBN - 1) / kBN;

@@ -56,6 +56,8 @@ struct AttnBwdArgs {
     float* const* dk_chunks;      // host array, P entries, [B][Lc][H_kv][D] fp32, dense
     float* const* dv_chunks;
     float* workspace;             // [B][H_q][P*Lc] fp32 (rowsum(dO * O))
+    int zigzag = 0;               // shards in the zigzag layout
+    const int* pid = nullptr;     // packed samples: position_ids [B][P*Lc] (causal), else null
     cudaStream_t stream;
 };
 

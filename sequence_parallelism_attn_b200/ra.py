@@ -19,7 +19,8 @@ RA_OK, RA_ERR_INVALID, RA_ERR_UNSUPPORTED, RA_ERR_CUDA, RA_ERR_TIMEOUT = 0, 1, 2
 RA_BF16, RA_FP32 = 0, 1
 RA_MAX_P = 64
 EXPORTED = ("ra_ring_attn_fwd", "ra_ring_attn_fwd_zigzag", "ra_ring_attn_fwd_packed",
-            "ra_ring_attn_bwd", "ra_ring_attn_bwd_static",
+            "ra_ring_attn_bwd", "ra_ring_attn_bwd_zigzag", "ra_ring_attn_bwd_packed",
+            "ra_ring_attn_bwd_static",
             "ra_lse_merge", "ra_ulysses_seq2head", "ra_ulysses_head2seq",
             "ra_ulysses_seq2head_grouped", "ra_ulysses_head2seq_grouped",
             "ra_sync_status", "ra_last_error", "ra_set_wait_limit_ns", "ra_debug_inject_stall",
@@ -51,6 +52,9 @@ def load() -> ctypes.CDLL:
     lib.ra_ring_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i64,
                                      i64, f32, i32, vp, vp, vp, vp, vp]
     lib.ra_ring_attn_bwd_static.argtypes = lib.ra_ring_attn_bwd.argtypes[:19] + [vp]
+    lib.ra_ring_attn_bwd_zigzag.argtypes = lib.ra_ring_attn_bwd.argtypes
+    lib.ra_ring_attn_bwd_packed.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                            i32, i64, i64, f32, vp, vp, vp, vp, vp]
     lib.ra_ring_attn_fwd_packed.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i64, i64,
                                             f32, i32, i32, vp, vp, vp]
     lib.ra_lse_merge.argtypes = [vp, vp, vp, vp, i32, i32, i64, i32, vp]
@@ -60,7 +64,8 @@ def load() -> ctypes.CDLL:
     lib.ra_ulysses_head2seq_grouped.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, vp]
     lib.ra_sync_status.argtypes = [vp]
     for f in ("ra_ring_attn_fwd", "ra_ring_attn_fwd_zigzag", "ra_ring_attn_fwd_packed",
-              "ra_ring_attn_bwd", "ra_ring_attn_bwd_static", "ra_lse_merge",
+              "ra_ring_attn_bwd", "ra_ring_attn_bwd_zigzag", "ra_ring_attn_bwd_packed",
+              "ra_ring_attn_bwd_static", "ra_lse_merge",
               "ra_ulysses_seq2head", "ra_ulysses_head2seq", "ra_ulysses_seq2head_grouped",
               "ra_ulysses_head2seq_grouped", "ra_sync_status"):
         getattr(lib, f).restype = ctypes.c_int
@@ -139,6 +144,28 @@ def ra_ring_attn_bwd(q_ptr, k_ptrs, v_ptrs, out_ptr, lse_ptr, dout_ptr, P, B, H_
                                    stream))
 
 
+def ra_ring_attn_bwd_zigzag(q_ptr, k_ptrs, v_ptrs, out_ptr, lse_ptr, dout_ptr, P, B, H_q, H_kv, Lc,
+                            D, q_bstride, kv_bstride, scale, causal, dq_ptr, dk_ptrs, dv_ptrs,
+                            ws_ptr, stream):
+    """The backward C entry point for zigzag shards (raw pointers)."""
+    arr = ctypes.c_void_p * P
+    _check(load().ra_ring_attn_bwd_zigzag(q_ptr, arr(*k_ptrs), arr(*v_ptrs), out_ptr, lse_ptr,
+                                          dout_ptr, P, B, H_q, H_kv, Lc, D, q_bstride, kv_bstride,
+                                          scale, int(causal), dq_ptr, arr(*dk_ptrs),
+                                          arr(*dv_ptrs), ws_ptr, stream))
+
+
+def ra_ring_attn_bwd_packed(q_ptr, k_ptrs, v_ptrs, pid_ptr, out_ptr, lse_ptr, dout_ptr, P, B, H_q,
+                            H_kv, Lc, D, q_bstride, kv_bstride, scale, dq_ptr, dk_ptrs, dv_ptrs,
+                            ws_ptr, stream):
+    """The backward C entry point for packed samples (raw pointers; causal)."""
+    arr = ctypes.c_void_p * P
+    _check(load().ra_ring_attn_bwd_packed(q_ptr, arr(*k_ptrs), arr(*v_ptrs), pid_ptr, out_ptr,
+                                          lse_ptr, dout_ptr, P, B, H_q, H_kv, Lc, D, q_bstride,
+                                          kv_bstride, scale, dq_ptr, arr(*dk_ptrs),
+                                          arr(*dv_ptrs), ws_ptr, stream))
+
+
 def ra_ring_attn_bwd_static(q_ptr, k_ptrs, v_ptrs, out_ptr, lse_ptr, dout_ptr, P, B, H_q, H_kv,
                             Lc, D, q_bstride, kv_bstride, scale, causal, dq_ptr, dk_ptrs, dv_ptrs,
                             stream):
@@ -155,11 +182,17 @@ def ring_attn_bwd(q: torch.Tensor, k_chunks: torch.Tensor, v_chunks: torch.Tenso
                   out: torch.Tensor, lse: torch.Tensor, dout: torch.Tensor, causal: bool,
                   scale: float | None = None, dq: torch.Tensor | None = None,
                   dk: torch.Tensor | None = None, dv: torch.Tensor | None = None,
-                  workspace: torch.Tensor | None = None, stream=None):
+                  workspace: torch.Tensor | None = None, stream=None,
+                  layout: str = "contiguous", position_ids: torch.Tensor | None = None):
     """Gradients of ring_attn_fwd: q/out/dout [B, P*Lc, H_q, D] bf16 (dense), k/v chunks
     [P, B, Lc, H_kv, D] bf16, lse [B, H_q, P*Lc] fp32.  Returns (dq [B, P*Lc, H_q, D],
     dk, dv [P, B, Lc, H_kv, D]) in fp32; the fp32 workspace [B, H_q, P*Lc] is allocated
-    here when not given (the library itself allocates nothing)."""
+    here when not given (the library itself allocates nothing).  layout and position_ids
+    as for ring_attn_fwd (the forward's)."""
+    if layout not in ("contiguous", "zigzag"):
+        raise ValueError(f"unknown layout {layout!r}")
+    if position_ids is not None and (layout != "contiguous" or not causal):
+        raise ValueError("packed samples need the contiguous layout and causal=True")
     P, B, Lc, H_kv, D = k_chunks.shape
     _, L, H_q, _ = q.shape
     assert L == P * Lc and q.is_contiguous() and out.is_contiguous() and dout.is_contiguous()
@@ -175,11 +208,20 @@ def ring_attn_bwd(q: torch.Tensor, k_chunks: torch.Tensor, v_chunks: torch.Tenso
         dv = torch.empty_like(dk)
     if workspace is None:
         workspace = torch.empty((B, H_q, L), dtype=torch.float32, device=dev)
-    ra_ring_attn_bwd(q.data_ptr(), [k_chunks[j].data_ptr() for j in range(P)],
-                     [v_chunks[j].data_ptr() for j in range(P)], out.data_ptr(), lse.data_ptr(),
-                     dout.data_ptr(), P, B, H_q, H_kv, Lc, D, L * H_q * D, Lc * H_kv * D,
-                     float(scale), causal, dq.data_ptr(), [dk[j].data_ptr() for j in range(P)],
-                     [dv[j].data_ptr() for j in range(P)], workspace.data_ptr(), _stream(stream))
+    kp, vp_ = [k_chunks[j].data_ptr() for j in range(P)], [v_chunks[j].data_ptr() for j in range(P)]
+    dkp, dvp = [dk[j].data_ptr() for j in range(P)], [dv[j].data_ptr() for j in range(P)]
+    if position_ids is not None:
+        assert position_ids.dtype == torch.int32 and position_ids.is_cuda
+        assert position_ids.is_contiguous() and position_ids.shape == (B, L)
+        ra_ring_attn_bwd_packed(q.data_ptr(), kp, vp_, position_ids.data_ptr(), out.data_ptr(),
+                                lse.data_ptr(), dout.data_ptr(), P, B, H_q, H_kv, Lc, D,
+                                L * H_q * D, Lc * H_kv * D, float(scale), dq.data_ptr(), dkp, dvp,
+                                workspace.data_ptr(), _stream(stream))
+    else:
+        entry = ra_ring_attn_bwd_zigzag if layout == "zigzag" else ra_ring_attn_bwd
+        entry(q.data_ptr(), kp, vp_, out.data_ptr(), lse.data_ptr(), dout.data_ptr(), P, B, H_q,
+              H_kv, Lc, D, L * H_q * D, Lc * H_kv * D, float(scale), causal, dq.data_ptr(), dkp,
+              dvp, workspace.data_ptr(), _stream(stream))
     return dq, dk, dv
 
 

@@ -71,6 +71,7 @@ struct __align__(64) BwdParams {
     float* dv[RA_MAX_P];
     int P, B, H_q, H_kv, Lc, L, causal, group, n_qblocks, ntc;
     int zigzag;       // shards in the zigzag layout
+    int position_order;  // zigzag, causal, Lc/2 a multiple of 128: grids by sequence position
     const int* pid;   // packed samples: position_ids [B][L] (else null)
     float scale, scale_log2;
     unsigned long long wait_limit_ns;
@@ -419,7 +420,16 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
     const int bg = (int)(blockIdx.x / per_bg), rem = (int)(blockIdx.x % per_bg);
     const int b = bg / p.H_kv, g = bg % p.H_kv;
     const int h = g * p.group + rem % p.group;
-    const int r0 = (p.n_qblocks - 1 - rem / p.group) * kBM;
+    int r0 = (p.n_qblocks - 1 - rem / p.group) * kBM;
+    if (LAYOUT == kLayoutZigzag && p.position_order) {
+        // the k-th block visited is the one at the k-th latest position: segments 2P-1 down
+        // to 0 (segment s >= P is the second half of rank 2P-1-s, s < P the first of rank s)
+        const int kvis = rem / p.group, hseg = p.Lc / 2, seg_blocks = hseg / kBM;
+        const int seg = 2 * p.P - 1 - kvis / seg_blocks;
+        const int bis = seg_blocks - 1 - kvis % seg_blocks;
+        const int rank = seg < p.P ? seg : 2 * p.P - 1 - seg;
+        r0 = rank * p.Lc + (seg < p.P ? 0 : hseg) + bis * kBM;
+    }
 
     if (threadIdx.x == 0) {
         mbar_init(bar(C::BAR_FIXED), 1);
@@ -716,7 +726,14 @@ __global__ void __launch_bounds__(kThreadsKV, 1) bwd_dkdv_sm100(const __grid_con
     const int n_kt = p.P * p.ntc;
     const int bg = (int)(blockIdx.x / n_kt), kt = (int)(blockIdx.x % n_kt);
     const int b = bg / p.H_kv, g = bg % p.H_kv;
-    const int j = kt / p.ntc, t = kt % p.ntc;
+    int j = kt / p.ntc, t = kt % p.ntc;
+    if (LAYOUT == kLayoutZigzag && p.position_order) {
+        // key tiles by ascending sequence position (the earliest keys are seen by the most
+        // queries): segment s < P is the first half of rank s, s >= P the second of 2P-1-s
+        const int seg_tiles = (p.Lc / 2) / kBN, seg = kt / seg_tiles;
+        j = seg < p.P ? seg : 2 * p.P - 1 - seg;
+        t = (seg < p.P ? 0 : seg_tiles) + kt % seg_tiles;
+    }
     const long long key0 = (long long)j * p.Lc + (long long)t * kBN;  // contiguous position
     const int kvalid = min(kBN, p.Lc - t * kBN);
     // contiguous layout: the query tiles that can see a key of this tile are those holding
@@ -798,8 +815,9 @@ __global__ void __launch_bounds__(kThreadsKV, 1) bwd_dkdv_sm100(const __grid_con
                     // positions start .. pos (every key when not causal)
                     int pos = INT_MAX, start = 0;
                     if (row < p.L && p.causal) {
+                        const int ri = (int)row;  // L <= 2^30
                         pos = (int)shard_pos(LAYOUT == kLayoutZigzag ? 1 : 0, p.P, p.Lc,
-                                             (int)(row / p.Lc), row % p.Lc);
+                                             ri / p.Lc, ri % p.Lc);
                         if (LAYOUT == kLayoutPacked) start = sample_start(p, b, (int)row);
                     }
                     reinterpret_cast<int*>(rows)[2 * kBM + r] = pos;
@@ -1168,6 +1186,7 @@ cudaError_t launch_attn_bwd_sm100(const AttnBwdArgs& a, unsigned long long wait_
     p.L = (int)L;
     p.causal = a.causal;
     p.zigzag = a.zigzag;
+    p.position_order = a.zigzag && a.causal && (a.Lc / 2) % kBM == 0;
     p.pid = a.pid;
     p.group = a.H_q / a.H_kv;
     p.n_qblocks = (int)((L + kBM - 1) / kBM);

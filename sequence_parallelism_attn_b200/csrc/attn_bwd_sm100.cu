@@ -292,11 +292,9 @@ __device__ __forceinline__ uint32_t ds_pair(uint64_t s2, uint64_t dp2, uint64_t 
 }
 
 // ------------------------------------------------------------------ layout helpers
-// Sample start of row r of batch row b (packed samples: r - position_ids[b][r], clamped to
-// [0, r] as in the forward).
+// Sample start of row r of batch row b (packed samples).
 __device__ __forceinline__ int sample_start(const BwdParams& p, int b, int r) {
-    const int st = r - p.pid[(long long)b * p.L + r];
-    return st < 0 ? 0 : (st > r ? r : st);
+    return ra::sample_start(p.pid + (long long)b * p.L, r);
 }
 
 // The keys of tile (chunk j, local keys key0 .. key0 + kvalid - 1) that a query at sequence
@@ -322,55 +320,6 @@ __device__ __forceinline__ void key_interval(const BwdParams& p, int j, int key0
         c_hi = min(c_hi, hi);
     }
     c_lo = LAYOUT == kLayoutPacked ? clamp_c(my_start - kpos0) : -1;
-}
-
-// dK/dV kernel: the query tiles whose rows may see a key of the tile (chunk j, local keys
-// key0 .. key0 + kvalid - 1), as ascending disjoint ranges [lo, hi) of tile indices written
-// to qr (at most 2 P).  Returns the number of ranges and sets *n_tiles.  Zigzag, causal:
-// rows at a position >= the tile's first key position, which in every half-shard is a
-// suffix; packed (causal): rows from the tile's first key to the last row whose sample
-// starts at or before the tile's last key (sample starts do not decrease along a row).
-template <int LAYOUT>
-__device__ int build_q_ranges(const BwdParams& p, int b, int j, int key0, int kvalid, int2* qr,
-                              int* n_tiles) {
-    int nr = 0;
-    auto add_rows = [&](long long row_lo, long long row_hi) {  // rows [row_lo, row_hi)
-        if (row_lo >= row_hi) return;
-        const int lo = (int)(row_lo / kBM), hi = (int)((row_hi - 1) / kBM) + 1;
-        if (nr > 0 && lo <= qr[nr - 1].y) {
-            qr[nr - 1].y = max(qr[nr - 1].y, hi);
-        } else {
-            qr[nr].x = lo;
-            qr[nr].y = hi;
-            ++nr;
-        }
-    };
-    if (!p.causal) {
-        add_rows(0, p.L);
-    } else if (LAYOUT == kLayoutZigzag) {
-        const long long h = p.Lc / 2;
-        const long long kmin = shard_pos(1, p.P, p.Lc, j, key0);
-        for (int r = 0; r < p.P; ++r) {
-            const long long base = (long long)r * p.Lc;
-            const long long u1 = max(0LL, kmin - (long long)r * h);  // first half: r h + u
-            if (u1 < h) add_rows(base + u1, base + h);
-            const long long u2 = h + max(0LL, kmin - (2LL * p.P - 1 - r) * h);
-            if (u2 < p.Lc) add_rows(base + u2, base + p.Lc);
-        }
-    } else {
-        const int k0 = j * p.Lc + key0, k_last = k0 + kvalid - 1;
-        int lo = k0 / kBM, hi = p.n_qblocks - 1;  // the last tile whose first row's sample
-        while (lo < hi) {                         // starts at or before k_last
-            const int mid = (lo + hi + 1) / 2;
-            if (sample_start(p, b, mid * kBM) <= k_last) lo = mid;
-            else hi = mid - 1;
-        }
-        add_rows((long long)(k0 / kBM) * kBM, (long long)(lo + 1) * kBM);
-    }
-    int n = 0;
-    for (int i = 0; i < nr; ++i) n += qr[i].y - qr[i].x;
-    *n_tiles = n;
-    return nr;
 }
 
 // ------------------------------------------------------------------ Delta = rowsum(dO * O)
@@ -715,7 +664,8 @@ __global__ void __launch_bounds__(kThreadsKV, 1) bwd_dkdv_sm100(const __grid_con
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
     volatile int* n_slot = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
     volatile int* nr_slot = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 12);
-    int2* qr = reinterpret_cast<int2*>(smem + C::OFF_QR);
+    int* qr_lo = reinterpret_cast<int*>(smem + C::OFF_QR);
+    int* qr_hi = qr_lo + 2 * RA_MAX_P;
     auto bar = [&](int i) { return base + C::OFF_BAR + 8u * (uint32_t)i; };
     const unsigned long long lim = p.wait_limit_ns;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -759,8 +709,11 @@ __global__ void __launch_bounds__(kThreadsKV, 1) bwd_dkdv_sm100(const __grid_con
         fence_proxy_async_smem();
     }
     if (!CONTIG && warp == kWarpLoad && lane == 0) {
+        // query-tile ranges [qr_lo, qr_hi) that can see this key tile (ra_internal.h)
         int nt = 0;
-        *nr_slot = build_q_ranges<LAYOUT>(p, b, j, t * kBN, kvalid, qr, &nt);
+        *nr_slot = key_tile_q_ranges(LAYOUT, p.P, p.Lc, p.causal, kBM,
+                                     p.pid ? p.pid + (long long)b * p.L : nullptr, j, t * kBN,
+                                     kvalid, qr_lo, qr_hi, &nt);
         *n_slot = nt * p.group;
     }
     if (warp == kWarpMma) {
@@ -853,7 +806,7 @@ __global__ void __launch_bounds__(kThreadsKV, 1) bwd_dkdv_sm100(const __grid_con
             bool go = true;
             for (int hh = 0; go && hh < p.group; ++hh)
                 for (int ri = 0; go && ri < nr; ++ri)
-                    for (int qt = qr[ri].x; go && qt < qr[ri].y; ++qt, ++it)
+                    for (int qt = qr_lo[ri]; go && qt < qr_hi[ri]; ++qt, ++it)
                         go = produce(it, g * p.group + hh, qt * kBM);
         }
         if (lane == 0) {

@@ -113,6 +113,69 @@ __host__ __device__ inline void row_pos_range(int zigzag, int P, int Lc, long lo
     }
 }
 
+// Sample start of row r of one batch row of packed samples ("Paralelismo de secuencias en
+// 🤗 accelerate", section "Configuración del backend SP de ALST/Ulysses"): r minus its
+// position_ids entry, clamped to [0, r].
+__host__ __device__ inline int sample_start(const int* pid_row, int r) {
+    const int st = r - pid_row[r];
+    return st < 0 ? 0 : (st > r ? r : st);
+}
+
+// The query tiles (of `tile` rows, rank-major) whose rows may see a key of the key tile
+// (chunk j, local keys key0 .. key0 + kvalid - 1), as ascending disjoint ranges
+// [qr_lo[i], qr_hi[i]) of tile indices (at most 2 P).  Returns the number of ranges and
+// sets *n_tiles to the tiles they hold.  layout: 1 zigzag, 2 packed (pid_row: the batch
+// row's position_ids).  Not causal: every tile.  Zigzag, causal: rows at a position >= the
+// key tile's first position, a suffix of every half-shard.  Packed (causal): rows from the
+// tile's first key to the last row whose sample starts at or before its last key (sample
+// starts do not decrease along a row, so a binary search over tiles finds it).
+__host__ __device__ inline int key_tile_q_ranges(int layout, int P, int Lc, int causal, int tile,
+                                                 const int* pid_row, int j, int key0, int kvalid,
+                                                 int* qr_lo, int* qr_hi, int* n_tiles) {
+    const long long L = (long long)P * Lc;
+    const int n_qt = (int)((L + tile - 1) / tile);
+    int nr = 0;
+    auto add_rows = [&](long long row_lo, long long row_hi) {  // rows [row_lo, row_hi)
+        if (row_lo >= row_hi) return;
+        const int lo = (int)(row_lo / tile), hi = (int)((row_hi - 1) / tile) + 1;
+        if (nr > 0 && lo <= qr_hi[nr - 1]) {
+            qr_hi[nr - 1] = qr_hi[nr - 1] > hi ? qr_hi[nr - 1] : hi;
+        } else {
+            qr_lo[nr] = lo;
+            qr_hi[nr] = hi;
+            ++nr;
+        }
+    };
+    if (!causal) {
+        add_rows(0, L);
+    } else if (layout == 1) {
+        const long long h = Lc / 2;
+        const long long kmin = shard_pos(1, P, Lc, j, key0);
+        for (int r = 0; r < P; ++r) {
+            const long long base = (long long)r * Lc;
+            const long long d1 = kmin - (long long)r * h;  // first half: positions r h + u
+            const long long u1 = d1 > 0 ? d1 : 0;
+            if (u1 < h) add_rows(base + u1, base + h);
+            const long long d2 = kmin - (2LL * P - 1 - r) * h;
+            const long long u2 = h + (d2 > 0 ? d2 : 0);
+            if (u2 < Lc) add_rows(base + u2, base + Lc);
+        }
+    } else {
+        const int k0 = j * Lc + key0, k_last = k0 + kvalid - 1;
+        int lo = k0 / tile, hi = n_qt - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) / 2;
+            if (sample_start(pid_row, mid * tile) <= k_last) lo = mid;
+            else hi = mid - 1;
+        }
+        add_rows((long long)(k0 / tile) * tile, (long long)(lo + 1) * tile);
+    }
+    int n = 0;
+    for (int i = 0; i < nr; ++i) n += qr_hi[i] - qr_lo[i];
+    *n_tiles = n;
+    return nr;
+}
+
 // Tensor-core (tcgen05) attention for bf16 inputs, D in {64, 128}.
 cudaError_t launch_attn_sm100(const AttnArgs& a, unsigned long long wait_limit_ns,
                               int inject_stall, const char** why);

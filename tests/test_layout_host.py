@@ -1,5 +1,6 @@
 """Host logic of the CUDA library on the CPU: the shard-layout position helpers that the
-attention kernels use for causal scheduling and masking (contiguous and zigzag layouts),
+attention kernels use for causal scheduling and masking (contiguous and zigzag layouts) and
+the query-tile ranges of the backward's key-tile kernel (zigzag and packed samples),
 compiled from the library's own header and checked against brute force."""
 import os
 import subprocess

@@ -58,7 +58,7 @@ extern "C" {
 typedef enum {
     RA_OK = 0,
     RA_ERR_INVALID = 1,      /* bad argument: null/misaligned pointer, bad size or divisibility */
-    RA_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement (e.g. D not in {32,64,128}) */
+    RA_ERR_UNSUPPORTED = 2,  /* valid request the library does not implement (e.g. D not in {32,64,128}) */
     RA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed; see ra_last_error() */
     RA_ERR_TIMEOUT = 4       /* a kernel gave up on a bounded internal wait; outputs are undefined */
 } ra_status;

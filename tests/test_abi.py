@@ -108,3 +108,53 @@ def test_wait_limit_roundtrip(lib):
     old = lib.ra_set_wait_limit_ns(12345)
     assert lib.ra_set_wait_limit_ns(0) == 12345
     assert lib.ra_set_wait_limit_ns(old) == 4000000000
+
+
+def _bwd(lib, entry="ra_ring_attn_bwd", **kw):
+    """One backward call with fake pointers (every case below fails validation first)."""
+    a = dict(q=FAKE, k=[FAKE], v=[FAKE], pid=FAKE, out=FAKE, lse=FAKE, dout=FAKE, P=1, B=1,
+             H_q=2, H_kv=1, Lc=128, D=128, scale=0.1, causal=1, dq=FAKE, dk=[FAKE], dv=[FAKE],
+             ws=FAKE)
+    a.update(kw)
+    P = a["P"]
+    arr = ctypes.c_void_p * max(P, 1)
+    rep = lambda x: arr(*(x * max(P, 1))[:max(P, 1)])
+    L = max(P, 1) * a["Lc"]
+    qb, kvb = L * a["H_q"] * a["D"], a["Lc"] * a["H_kv"] * a["D"]
+    if entry == "ra_ring_attn_bwd_packed":
+        return lib.ra_ring_attn_bwd_packed(a["q"], rep(a["k"]), rep(a["v"]), a["pid"], a["out"],
+                                           a["lse"], a["dout"], P, a["B"], a["H_q"], a["H_kv"],
+                                           a["Lc"], a["D"], qb, kvb, a["scale"], a["dq"],
+                                           rep(a["dk"]), rep(a["dv"]), a["ws"], None)
+    return getattr(lib, entry)(a["q"], rep(a["k"]), rep(a["v"]), a["out"], a["lse"], a["dout"],
+                               P, a["B"], a["H_q"], a["H_kv"], a["Lc"], a["D"], qb, kvb,
+                               a["scale"], a["causal"], a["dq"], rep(a["dk"]), rep(a["dv"]),
+                               a["ws"], None)
+
+
+@pytest.mark.parametrize("entry", ["ra_ring_attn_bwd", "ra_ring_attn_bwd_zigzag",
+                                   "ra_ring_attn_bwd_packed"])
+@pytest.mark.parametrize("kw,status", [
+    (dict(P=0), 1), (dict(P=65), 1), (dict(H_q=3, H_kv=2), 1), (dict(scale=0.0), 1),
+    (dict(D=32), 2), (dict(D=96), 2), (dict(q=FAKE + 8), 1), (dict(out=0), 1),
+    (dict(lse=FAKE + 4), 1), (dict(dout=0), 1), (dict(dq=FAKE + 2), 1), (dict(ws=0), 1),
+    (dict(k=[0]), 1), (dict(dk=[FAKE + 4]), 1), (dict(dv=[0]), 1),
+])
+def test_backward_argument_validation(lib, entry, kw, status):
+    """The backward entry points refuse bad arguments on the host, before any CUDA call."""
+    assert _bwd(lib, entry, **kw) == status
+    assert lib.ra_last_error()
+
+
+def test_backward_layout_argument_validation(lib):
+    # zigzag needs an even chunk length
+    assert _bwd(lib, "ra_ring_attn_bwd_zigzag", Lc=129) == 1
+    assert b"even" in lib.ra_last_error()
+    # packed samples need non-null, 4-byte aligned position_ids
+    assert _bwd(lib, "ra_ring_attn_bwd_packed", pid=0) == 1
+    assert b"position_ids" in lib.ra_last_error()
+    assert _bwd(lib, "ra_ring_attn_bwd_packed", pid=FAKE + 2) == 1
+    assert b"aligned" in lib.ra_last_error()
+    # causal must be 0 or 1 where it is an argument
+    assert _bwd(lib, "ra_ring_attn_bwd", causal=2) == 1
+    assert _bwd(lib, "ra_ring_attn_bwd_zigzag", causal=-1) == 1

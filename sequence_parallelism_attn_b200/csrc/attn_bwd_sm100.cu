@@ -8,8 +8,9 @@
 // Three kernels: Delta (a row reduction), dQ with the query tile stationary (the chunks
 // visited in the forward's ring order, causal tiles skipped), and dK/dV with the key tile
 // stationary (every query tile of every query head of the kv head's group that can see
-// it).  Each tensor-core kernel keeps its operands for one 128 x 128 tile pair in tensor
-// memory:
+// it).  Both tensor-core kernels are compiled per shard layout (contiguous, zigzag,
+// packed samples), like the forward.  Each keeps its operands for one 128 x 128 tile
+// pair in tensor memory:
 //   dQ kernel   TMEM S [0,128) or [384,512) by tile parity, dP [128,256), dQ [256,256+D);
 //               dS (bf16) of each 64-key half over the first 32 columns of that half of S
 //   dK/dV       TMEM S^T and dP^T in [0,128) / [128,256), swapping every query tile,
@@ -19,9 +20,11 @@
 // run while the second is formed) and signal when they have read dP, so that the next
 // tile's S (dQ kernel: into the spare region) and dP (dK/dV: S^T into the freed dP^T
 // region) are computed while they work.
-// Roles (352 threads): warps 0-7 compute P, dS (one TMEM lane = one row; warps 0-3 the
-// first 64 columns of a tile, 4-7 the second), warp 8 loads (TMA), warps 9 and 10 each
-// issue part of the MMAs from one thread (warp 9 owns tensor memory).  Every wait is
+// Roles (dQ kernel 352 threads, dK/dV 384 with an idle warp 11 and a setmaxnreg split):
+// warps 0-7 compute P, dS (one TMEM lane = one row; warps 0-3 the first 64 columns of a
+// tile, 4-7 the second), warp 8 loads (TMA, and in dK/dV the per-row LSE, Delta,
+// positions and sample starts), warps 9 and 10 each issue part of the MMAs from one
+// thread (warp 9 owns tensor memory).  Every wait is
 // bounded: a role that gives up sets the CTA abort flag and this file's error word, every
 // role stops issuing and drains its own work, and the CTA frees its tensor memory.
 #include <cuda.h>
@@ -694,7 +697,7 @@ __global__ void __launch_bounds__(kThreadsKV, 1) bwd_dkdv_sm100(const __grid_con
     if (threadIdx.x == 0) {
         mbar_init(bar(C::BAR_FIXED), 1);
         for (int s = 0; s < C::NS; ++s) {
-            mbar_init(bar(C::bar_full(s)), 1 + 1);  // the load thread's expect_tx + the LSE/Delta rows
+            mbar_init(bar(C::bar_full(s)), 1 + 1);  // the load thread's expect_tx + the per-row values
             mbar_init(bar(C::bar_empty(s)), 1);
         }
         mbar_init(bar(C::BAR_SD), 1);

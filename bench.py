@@ -412,6 +412,37 @@ def run_oracle_sample(w_attn, target_s=15.0, max_rows=4096):
         n = min(max_rows, max(n * 2, int(n * target_s / max(dt, 1e-3))))
 
 
+def oracle_bwd_sample(w_attn, Ls, seed=4243):
+    """A bounded sample of a backward workload for the oracle: one head's sequence of Ls
+    tokens (same distribution, causal as the workload) with dO; algorithmic FLOPs as for
+    the GPU line (2.5x the forward's)."""
+    import torch
+    g = torch.Generator().manual_seed(seed)
+    D = w_attn.D
+    draw = lambda mult=1.0: (torch.randn(1, Ls, 1, D, generator=g) * mult).to(
+        w_attn.dtype).double().numpy()
+    q, k, v, dout = draw(w_attn.q_mult), draw(), draw(), draw()
+    flops = 2.5 * 4.0 * float(Ls) * Ls * D / (2 if w_attn.causal else 1)
+    return q, k, v, dout, flops
+
+
+def run_oracle_bwd_sample(w_attn, target_s=15.0):
+    """Time the oracle's gradients as they stand on a bounded sample; returns
+    (TFLOP/s, Ls, seconds, cores)."""
+    import oracle
+    oracle.build()
+    cores = os.cpu_count() or 1
+    Ls = 256
+    while True:
+        q, k, v, dout, flops = oracle_bwd_sample(w_attn, Ls)
+        t0 = time.perf_counter()
+        oracle.attention_backward(q, k, v, dout, w_attn.scale, w_attn.causal)
+        dt = time.perf_counter() - t0
+        if dt >= target_s * 0.5 or Ls >= w_attn.L:
+            return flops / dt / 1e12, Ls, dt, cores
+        Ls = min(w_attn.L, Ls * 2)  # the cost grows about 4x per doubling
+
+
 # ------------------------------------------------------------------ main
 def main():
     faulthandler.enable()
@@ -515,11 +546,16 @@ def main():
                       "pipelined": "step i+1 inputs up and step i output down on two copy "
                                    "streams, overlapping compute; all copies timed"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tf, n, dt, cores = run_oracle_sample(w_attn)
+        if kind.startswith("attn_bwd"):
+            tf, n, dt, cores = run_oracle_bwd_sample(w_attn)
+            sample = (f"gradients of one head's {n}-token sequence (D={w_attn.D}, "
+                      f"{'causal' if w_attn.causal else 'non-causal'}), fp64 oracle, {dt:.1f} s")
+        else:
+            tf, n, dt, cores = run_oracle_sample(w_attn)
+            sample = (f"{n} query rows x all visible keys of one {w_attn.L}-token sequence "
+                      f"(D={w_attn.D}), fp64 oracle, {dt:.1f} s")
         out["cpu_baseline"] = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle",
-                               "sample": f"{n} query rows x all visible keys of one "
-                                         f"{w_attn.L}-token sequence (D={w_attn.D}), fp64 "
-                                         f"oracle, {dt:.1f} s"}
+                               "sample": sample}
     if rank == 0:
         print(json.dumps(out), flush=True)
     if dist is not None:
@@ -536,15 +572,26 @@ def reference_arm(args, kind, w, w_attn, rank, world):
     cores = os.cpu_count() or 1
     # size one step's sample so that warmup + steps end within a few minutes
     per_step_s = args.ref_step_seconds or max(2.0, min(20.0, 150.0 / (args.steps + args.warmup)))
-    tf, n, dt, _ = run_oracle_sample(w_attn, target_s=per_step_s)
-    import numpy as np
-    q, rb, rt, rh, k, v, flops = oracle_sample(w_attn, n)
+    bwd = kind.startswith("attn_bwd")
+    if bwd:
+        _, n, _, _ = run_oracle_bwd_sample(w_attn, target_s=per_step_s)
+        bq, bk, bv, bdo, flops = oracle_bwd_sample(w_attn, n)
+        one_step = lambda: oracle.attention_backward(bq, bk, bv, bdo, w_attn.scale, w_attn.causal)
+        sample = (f"gradients of one head's {n}-token sequence per step (D={w_attn.D}), "
+                  f"fp64 oracle")
+    else:
+        _, n, _, _ = run_oracle_sample(w_attn, target_s=per_step_s)
+        q, rb, rt, rh, k, v, flops = oracle_sample(w_attn, n)
+        one_step = lambda: oracle.attention_rows(q, rb, rt, rh, k, v, 1, w_attn.scale,
+                                                 w_attn.causal)
+        sample = (f"{n} query rows x all visible keys of one {w_attn.L}-token sequence per "
+                  f"step, fp64 oracle")
     for _ in range(args.warmup):
         pass  # the oracle has no warm state; the calibration run above served as warm-up
     times = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        oracle.attention_rows(q, rb, rt, rh, k, v, 1, w_attn.scale, w_attn.causal)
+        one_step()
         times.append(time.perf_counter() - t0)
     sec = sum(times) / len(times)
     value = flops / sec / 1e12
@@ -556,8 +603,7 @@ def reference_arm(args, kind, w, w_attn, rank, world):
                       "seq_len": w_attn.L, "head_dim": w_attn.D,
                       "causal": w_attn.causal, "parallelism": "cpu-oracle"},
            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                            "sample": f"{n} query rows x all visible keys of one {w_attn.L}-token "
-                                      f"sequence per step, fp64 oracle"},
+                            "sample": sample},
            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 

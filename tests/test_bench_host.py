@@ -105,3 +105,17 @@ def test_reference_arm_json_line_cpu():
         assert key in line
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_reference_arm_backward_times_the_oracle_gradients():
+    """For a backward workload the reference arm times the oracle's gradients (a one-head
+    causal sample) under the workload's backward name."""
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "3", "--workload", "llama8b_32k_bwd",
+                        "--ref-step-seconds", "1"],
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["config"]["workload"].endswith("_backward")
+    assert "gradients" in line["cpu_baseline"]["sample"]

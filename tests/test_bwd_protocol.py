@@ -1,0 +1,337 @@
+"""A model of the synchronisation protocol of the two tensor-core backward kernels
+(bwd_dq_sm100 and bwd_dkdv_sm100 in sequence_parallelism_attn_b200/csrc/attn_bwd_sm100.cu),
+run under random latencies on the CPU.
+
+Each role of a CTA -- the loader, the two MMA-issuing threads, the two compute warpgroups --
+is a generator that performs, in the kernel's order, its mbarrier waits and arrivals, its
+MMA issues and commits, its TMA loads and its tensor-memory loads and stores.  The model
+executes:
+  * mbarriers with the hardware's parity rule (a wait for phase k succeeds while the phase
+    count differs from k in its low bit), arrival counts and TMA transaction counts;
+  * MMAs per issuing thread in issue order (tcgen05 operations of one thread complete in
+    order), interleaved at random across threads, and a commit arriving once everything
+    its thread issued before it has completed;
+  * TMA loads completing at random times.
+Every read of a tensor-memory region half or a shared-memory stage names the data it must
+see (which tile's S, dP, P/dS, or which tile's Q/dO, K/V); the model flags a read that sees
+anything else, a barrier that completes a phase twice before one of its waiters has seen
+the first (the parity hazard), and a schedule in which no role can proceed.  Mutated
+protocols (one wait removed) must be flagged, which shows the checks can fail."""
+import random
+
+import pytest
+
+
+class Violation(Exception):
+    pass
+
+
+class Barrier:
+    def __init__(self, name, count):
+        self.name, self.count = name, count
+        self.pending, self.tx, self.phase = count, 0, 0
+
+    def _maybe_complete(self):
+        if self.pending == 0 and self.tx == 0:
+            self.phase += 1
+            self.pending = self.count
+
+    def arrive(self, tx=0):
+        self.tx += tx
+        self.pending -= 1
+        if self.pending < 0:
+            raise Violation(f"{self.name}: more arrivals than its count")
+        self._maybe_complete()
+
+    def tx_done(self):
+        self.tx -= 1
+        self._maybe_complete()
+
+    def ready(self, k):
+        """A wait for the completion of phase k (parity k & 1)."""
+        if self.phase >= k + 2:
+            raise Violation(f"{self.name}: phase {k} overrun (count {self.phase})")
+        return (self.phase & 1) != (k & 1)
+
+
+class Sim:
+    def __init__(self, seed):
+        self.rng = random.Random(seed)
+        self.bars, self.mem, self.queues, self.tma = {}, {}, {}, []
+
+    def bar(self, name, count):
+        self.bars[name] = Barrier(name, count)
+
+    # data ------------------------------------------------------------------------------
+    def write(self, region, label):
+        self.mem[region] = label
+
+    def read(self, region, want, who):
+        got = self.mem.get(region)
+        if got != want:
+            raise Violation(f"{who} read {region}: saw {got}, expected {want}")
+
+    # asynchronous work ---------------------------------------------------------------------
+    def mma(self, thread, reads, writes, who):
+        """An MMA group: checks its reads and performs its writes when it executes."""
+        self.queues.setdefault(thread, []).append(("mma", reads, writes, who))
+
+    def commit(self, thread, barrier):
+        self.queues.setdefault(thread, []).append(("commit", barrier))
+
+    def tma_load(self, barrier, region, label):
+        self.tma.append((barrier, region, label))
+
+    def _step_async(self):
+        choices = [q for q in self.queues.values() if q]
+        if self.tma:
+            choices.append(self.tma)
+        if not choices:
+            return False
+        q = self.rng.choice(choices)
+        if q is self.tma:
+            barrier, region, label = self.tma.pop(self.rng.randrange(len(self.tma)))
+            self.write(region, label)
+            self.bars[barrier].tx_done()
+        else:
+            op = q.pop(0)
+            if op[0] == "mma":
+                _, reads, writes, who = op
+                for region, want in reads:
+                    self.read(region, want, who)
+                for region, label in writes:
+                    self.write(region, label)
+            else:
+                self.bars[op[1]].arrive()
+        return True
+
+    def run(self, roles):
+        """roles: generators yielding ("wait", barrier, phase) or None (a plain step)."""
+        state = {name: None for name in roles}  # pending wait of each role
+        live = dict(roles)
+        idle = 0
+        while live or any(self.queues.values()) or self.tma:
+            runnable = [n for n in live if state[n] is None or
+                        self.bars[state[n][0]].ready(state[n][1])]
+            options = runnable + (["async"] if (any(self.queues.values()) or self.tma) else [])
+            if not options:
+                waits = {n: state[n] for n in live}
+                raise Violation(f"deadlock: {waits}")
+            pick = self.rng.choice(options)
+            if pick == "async":
+                self._step_async()
+                continue
+            try:
+                req = next(live[pick])
+                state[pick] = (req[1], req[2]) if req is not None and req[0] == "wait" else None
+            except StopIteration:
+                del live[pick]
+                state.pop(pick)
+            idle += 1
+            if idle > 10_000_000:
+                raise Violation("no termination")
+
+
+# ------------------------------------------------------------------ the dK/dV kernel
+def dkdv_roles(sim, n, mutation=None):
+    NS = 2
+    st_col = lambda i: "R1" if i & 1 else "R0"   # S^T region of query tile i
+    dpt_col = lambda i: "R0" if i & 1 else "R1"  # dP^T region of query tile i
+    for name, count in (("fixed", 1), ("sd", 1), ("ds0", 1), ("ds1", 1), ("acc", 2),
+                        ("drain", 2), ("xfree", 1), ("dpfree", 2)):
+        sim.bar(name, count)
+    for s in range(NS):
+        sim.bar(f"full{s}", 2)
+        sim.bar(f"empty{s}", 1)
+
+    def loader():
+        sim.bars["fixed"].arrive(tx=1)
+        sim.tma_load("fixed", "KV", "KV")
+        yield None
+        for it in range(n):
+            slot = it % NS
+            if it >= NS:
+                yield ("wait", f"empty{slot}", it // NS - 1)
+            sim.bars[f"full{slot}"].arrive(tx=1)       # expect_tx, then Q and dO
+            sim.tma_load(f"full{slot}", f"stage{slot}", ("QdO", it))
+            sim.write(f"rows{slot}", ("rows", it))      # LSE, Delta, positions: plain stores
+            yield None
+            sim.bars[f"full{slot}"].arrive()
+
+    def stage_reads(i):
+        return [(f"stage{i % NS}", ("QdO", i))]
+
+    def half_regions(region):
+        return [region + "h0", region + "h1"]
+
+    def mma_a():  # dP^T and dV
+        yield ("wait", "fixed", 0)
+        yield ("wait", "full0", 0)
+        sim.mma("A", [("KV", "KV")] + stage_reads(0),
+                [(r, ("S", 0)) for r in half_regions(st_col(0))], "S^T(0)")
+        sim.mma("A", [("KV", "KV")] + stage_reads(0),
+                [(r, ("dP", 0)) for r in half_regions(dpt_col(0))], "dP^T(0)")
+        sim.commit("A", "sd")
+        for it in range(n):
+            more = it + 1 < n
+            yield ("wait", "ds0", it)
+            sim.mma("A", [(st_col(it) + "h0", ("PdS", it))] + stage_reads(it), [], f"dV h0({it})")
+            yield ("wait", "ds1", it)
+            sim.mma("A", [(st_col(it) + "h1", ("PdS", it))] + stage_reads(it), [], f"dV h1({it})")
+            if more and mutation != "no_xfree_wait":
+                yield ("wait", "xfree", it)
+            sim.commit("A", f"empty{it % NS}")
+            if more:
+                sim.mma("A", [("KV", "KV")] + stage_reads(it + 1),
+                        [(r, ("dP", it + 1)) for r in half_regions(dpt_col(it + 1))],
+                        f"dP^T({it + 1})")
+                sim.commit("A", "sd")
+        sim.commit("A", "acc")
+        sim.commit("A", "drain")
+        yield ("wait", "drain", 0)
+
+    def mma_b():  # S^T and dK
+        yield ("wait", "fixed", 0)
+        yield ("wait", "full0", 0)
+        for it in range(n):
+            if it + 1 < n:
+                if mutation != "no_dpfree_wait":
+                    yield ("wait", "dpfree", it)
+                yield ("wait", f"full{(it + 1) % NS}", (it + 1) // NS)
+                sim.mma("B", [("KV", "KV")] + stage_reads(it + 1),
+                        [(r, ("S", it + 1)) for r in half_regions(st_col(it + 1))],
+                        f"S^T({it + 1})")
+            yield ("wait", "ds0", it)
+            sim.mma("B", [(st_col(it) + "h0", ("PdS", it))] + stage_reads(it), [], f"dK h0({it})")
+            yield ("wait", "ds1", it)
+            sim.mma("B", [(st_col(it) + "h1", ("PdS", it))] + stage_reads(it), [], f"dK h1({it})")
+            sim.commit("B", "xfree")
+        sim.commit("B", "acc")
+        sim.commit("B", "drain")
+        yield ("wait", "drain", 0)
+
+    def compute(c):
+        for it in range(n):
+            yield ("wait", "sd", it)
+            sim.read(f"{st_col(it)}h{c}", ("S", it), f"WG{c} S({it})")
+            sim.read(f"{dpt_col(it)}h{c}", ("dP", it), f"WG{c} dP({it})")
+            yield None
+            sim.bars["dpfree"].arrive()
+            sim.read(f"rows{it % NS}", ("rows", it), f"WG{c} rows({it})")
+            yield None
+            if mutation == "store_before_read" and c == 1:
+                sim.write(f"{st_col(it)}h0", ("PdS", it))  # a half it does not own
+            sim.write(f"{st_col(it)}h{c}", ("PdS", it))
+            yield None
+            sim.bars[f"ds{c}"].arrive()
+        if n > 0:
+            yield ("wait", "acc", 0)
+
+    return {"load": loader(), "A": mma_a(), "B": mma_b(), "WG0": compute(0), "WG1": compute(1)}
+
+
+# ------------------------------------------------------------------ the dQ kernel
+def dq_roles(sim, n, mutation=None):
+    NS = 2
+    s_col = lambda j: "S1" if j & 1 else "S0"
+    for name, count in (("fixed", 1), ("sd", 2), ("ds0", 1), ("ds1", 1), ("acc", 1),
+                        ("drain", 2), ("dpfree", 2)):
+        sim.bar(name, count)
+    for s in range(NS):
+        sim.bar(f"full{s}", 1)
+        sim.bar(f"empty{s}", 1)
+
+    def loader():
+        sim.bars["fixed"].arrive(tx=1)
+        sim.tma_load("fixed", "QdO", "QdO")
+        yield None
+        for jt in range(n):
+            slot = jt % NS
+            if jt >= NS:
+                yield ("wait", f"empty{slot}", jt // NS - 1)
+            sim.bars[f"full{slot}"].arrive(tx=1)
+            sim.tma_load(f"full{slot}", f"stage{slot}", ("KV", jt))
+            yield None
+
+    kv = lambda j: [(f"stage{j % NS}", ("KV", j)), ("QdO", "QdO")]
+
+    def mma_a():  # S and dQ
+        yield ("wait", "fixed", 0)
+        yield ("wait", "full0", 0)
+        sim.mma("A", kv(0), [(s_col(0) + "h0", ("S", 0)), (s_col(0) + "h1", ("S", 0))], "S(0)")
+        sim.commit("A", "sd")
+        for jt in range(n):
+            more = jt + 1 < n
+            if more:
+                yield ("wait", f"full{(jt + 1) % NS}", (jt + 1) // NS)
+                sim.mma("A", kv(jt + 1), [(s_col(jt + 1) + "h0", ("S", jt + 1)),
+                                          (s_col(jt + 1) + "h1", ("S", jt + 1))], f"S({jt + 1})")
+            yield ("wait", "ds0", jt)
+            sim.mma("A", [(s_col(jt) + "h0", ("dS", jt))] + kv(jt), [], f"dQ h0({jt})")
+            if mutation != "no_ds1_wait":
+                yield ("wait", "ds1", jt)
+            if more:
+                sim.commit("A", "sd")
+            sim.mma("A", [(s_col(jt) + "h1", ("dS", jt))] + kv(jt), [], f"dQ h1({jt})")
+            sim.commit("A", f"empty{jt % NS}")
+        sim.commit("A", "acc")
+        sim.commit("A", "drain")
+        yield ("wait", "drain", 0)
+
+    def mma_b():  # dP
+        yield ("wait", "fixed", 0)
+        yield ("wait", "full0", 0)
+        sim.mma("B", kv(0), [("dPh0", ("dP", 0)), ("dPh1", ("dP", 0))], "dP(0)")
+        sim.commit("B", "sd")
+        for jt in range(n - 1):
+            if mutation != "no_dpfree_wait":
+                yield ("wait", "dpfree", jt)
+            yield ("wait", f"full{(jt + 1) % NS}", (jt + 1) // NS)
+            sim.mma("B", kv(jt + 1), [("dPh0", ("dP", jt + 1)), ("dPh1", ("dP", jt + 1))],
+                    f"dP({jt + 1})")
+            sim.commit("B", "sd")
+        sim.commit("B", "drain")
+        yield ("wait", "drain", 0)
+
+    def compute(c):
+        for jt in range(n):
+            yield ("wait", "sd", jt)
+            sim.read(f"{s_col(jt)}h{c}", ("S", jt), f"WG{c} S({jt})")
+            sim.read(f"dPh{c}", ("dP", jt), f"WG{c} dP({jt})")
+            yield None
+            sim.bars["dpfree"].arrive()
+            yield None
+            sim.write(f"{s_col(jt)}h{c}", ("dS", jt))
+            yield None
+            sim.bars[f"ds{c}"].arrive()
+        if n > 0:
+            yield ("wait", "acc", 0)
+
+    return {"load": loader(), "A": mma_a(), "B": mma_b(), "WG0": compute(0), "WG1": compute(1)}
+
+
+KERNELS = {"dkdv": dkdv_roles, "dq": dq_roles}
+
+
+@pytest.mark.parametrize("kernel", ["dkdv", "dq"])
+@pytest.mark.parametrize("n", [1, 2, 3, 4, 7])
+def test_protocol_holds_under_random_latencies(kernel, n):
+    for seed in range(300):
+        sim = Sim(seed * 1000 + n)
+        sim.run(KERNELS[kernel](sim, n))
+
+
+@pytest.mark.parametrize("kernel,mutation", [("dkdv", "no_xfree_wait"),
+                                             ("dkdv", "no_dpfree_wait"),
+                                             ("dkdv", "store_before_read"),
+                                             ("dq", "no_dpfree_wait"),
+                                             ("dq", "no_ds1_wait")])
+def test_mutated_protocols_are_caught(kernel, mutation):
+    caught = 0
+    for seed in range(300):
+        sim = Sim(seed)
+        try:
+            sim.run(KERNELS[kernel](sim, 4, mutation))
+        except Violation:
+            caught += 1
+    assert caught > 0, f"{kernel} with {mutation} was never flagged"

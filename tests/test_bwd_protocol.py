@@ -17,119 +17,9 @@ see (which tile's S, dP, P/dS, or which tile's Q/dO, K/V); the model flags a rea
 anything else, a barrier that completes a phase twice before one of its waiters has seen
 the first (the parity hazard), and a schedule in which no role can proceed.  Mutated
 protocols (one wait removed) must be flagged, which shows the checks can fail."""
-import random
-
 import pytest
 
-
-class Violation(Exception):
-    pass
-
-
-class Barrier:
-    def __init__(self, name, count):
-        self.name, self.count = name, count
-        self.pending, self.tx, self.phase = count, 0, 0
-
-    def _maybe_complete(self):
-        if self.pending == 0 and self.tx == 0:
-            self.phase += 1
-            self.pending = self.count
-
-    def arrive(self, tx=0):
-        self.tx += tx
-        self.pending -= 1
-        if self.pending < 0:
-            raise Violation(f"{self.name}: more arrivals than its count")
-        self._maybe_complete()
-
-    def tx_done(self):
-        self.tx -= 1
-        self._maybe_complete()
-
-    def ready(self, k):
-        """A wait for the completion of phase k (parity k & 1)."""
-        if self.phase >= k + 2:
-            raise Violation(f"{self.name}: phase {k} overrun (count {self.phase})")
-        return (self.phase & 1) != (k & 1)
-
-
-class Sim:
-    def __init__(self, seed):
-        self.rng = random.Random(seed)
-        self.bars, self.mem, self.queues, self.tma = {}, {}, {}, []
-
-    def bar(self, name, count):
-        self.bars[name] = Barrier(name, count)
-
-    # data ------------------------------------------------------------------------------
-    def write(self, region, label):
-        self.mem[region] = label
-
-    def read(self, region, want, who):
-        got = self.mem.get(region)
-        if got != want:
-            raise Violation(f"{who} read {region}: saw {got}, expected {want}")
-
-    # asynchronous work ---------------------------------------------------------------------
-    def mma(self, thread, reads, writes, who):
-        """An MMA group: checks its reads and performs its writes when it executes."""
-        self.queues.setdefault(thread, []).append(("mma", reads, writes, who))
-
-    def commit(self, thread, barrier):
-        self.queues.setdefault(thread, []).append(("commit", barrier))
-
-    def tma_load(self, barrier, region, label):
-        self.tma.append((barrier, region, label))
-
-    def _step_async(self):
-        choices = [q for q in self.queues.values() if q]
-        if self.tma:
-            choices.append(self.tma)
-        if not choices:
-            return False
-        q = self.rng.choice(choices)
-        if q is self.tma:
-            barrier, region, label = self.tma.pop(self.rng.randrange(len(self.tma)))
-            self.write(region, label)
-            self.bars[barrier].tx_done()
-        else:
-            op = q.pop(0)
-            if op[0] == "mma":
-                _, reads, writes, who = op
-                for region, want in reads:
-                    self.read(region, want, who)
-                for region, label in writes:
-                    self.write(region, label)
-            else:
-                self.bars[op[1]].arrive()
-        return True
-
-    def run(self, roles):
-        """roles: generators yielding ("wait", barrier, phase) or None (a plain step)."""
-        state = {name: None for name in roles}  # pending wait of each role
-        live = dict(roles)
-        idle = 0
-        while live or any(self.queues.values()) or self.tma:
-            runnable = [n for n in live if state[n] is None or
-                        self.bars[state[n][0]].ready(state[n][1])]
-            options = runnable + (["async"] if (any(self.queues.values()) or self.tma) else [])
-            if not options:
-                waits = {n: state[n] for n in live}
-                raise Violation(f"deadlock: {waits}")
-            pick = self.rng.choice(options)
-            if pick == "async":
-                self._step_async()
-                continue
-            try:
-                req = next(live[pick])
-                state[pick] = (req[1], req[2]) if req is not None and req[0] == "wait" else None
-            except StopIteration:
-                del live[pick]
-                state.pop(pick)
-            idle += 1
-            if idle > 10_000_000:
-                raise Violation("no termination")
+from _protocol_sim import Sim, Violation
 
 
 # ------------------------------------------------------------------ the dK/dV kernel

@@ -1,0 +1,139 @@
+"""A model of the synchronisation protocol of the tensor-core attention kernel
+(attn_fwd_sm100 in sequence_parallelism_attn_b200/csrc/attn_sm100.cu), run under random
+latencies on the CPU with the simulator of tests/_protocol_sim.py.
+
+Roles, in the kernel's order: the K producer (which also loads the two Q tiles) with a ring
+of NSK stages, the V producer with NSV stages, the MMA thread (S_A(0), S_B(0); then per key
+tile j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), with commits to sf[w], ke[], ve[] and of[w]),
+and the two softmax warpgroups (wait sf[w]; read S; write P over S; sometimes rescale O;
+signal pf[w]; at the end wait of[w] and read O).  Checked: no deadlock, no mbarrier phase
+overrun, and every read of S / P, O, a K or V stage and Q sees the data it must -- in
+particular that a rescale of O falls after PV(j-1) has completed and before PV(j) reads it.
+Mutated protocols (one wait removed, or a commit moved) must be flagged."""
+import pytest
+
+from _protocol_sim import Sim, Violation
+
+
+def fwd_roles(sim, n, NSK, NSV, mutation=None):
+    for name, count in (("q", 1), ("sf0", 1), ("sf1", 1), ("pf0", 1), ("pf1", 1),
+                        ("of0", 1), ("of1", 1), ("drain", 1)):
+        sim.bar(name, count)
+    for s in range(NSK):
+        sim.bar(f"kf{s}", 1)
+        sim.bar(f"ke{s}", 1)
+    for s in range(NSV):
+        sim.bar(f"vf{s}", 1)
+        sim.bar(f"ve{s}", 1)
+    S = {0: "SA", 1: "SB"}
+    O = {0: "OA", 1: "OB"}
+
+    def producer(is_k):
+        ns, full, empty, tag = (NSK, "kf", "ke", "K") if is_k else (NSV, "vf", "ve", "V")
+        if is_k:
+            sim.bars["q"].arrive(tx=1)
+            sim.tma_load("q", "Q", "Q")
+        armed = {}
+        for jt in range(n):
+            slot = jt % ns
+            if jt >= ns:
+                yield ("wait", f"{empty}{slot}", jt // ns - 1)
+            sim.bars[f"{full}{slot}"].arrive(tx=1)
+            sim.tma_load(f"{full}{slot}", f"{tag}{slot}", (tag, jt))
+            armed[slot] = jt
+            yield None
+        if is_k:
+            yield ("wait", "q", 0)
+        for slot, jt in armed.items():  # drain: every copy landed
+            yield ("wait", f"{full}{slot}", jt // ns)
+
+    def s_mma(w, j):
+        return (("Q", "Q"), (f"K{j % NSK}", ("K", j))), ((S[w], ("S", j)),), f"S_{'AB'[w]}({j})"
+
+    def pv_mma(w, j):
+        reads = [(S[w], ("P", j)), (f"V{j % NSV}", ("V", j))]
+        if j > 0:
+            reads.append((O[w], ("O", j - 1)))
+        return reads, [(O[w], ("O", j))], f"PV_{'AB'[w]}({j})"
+
+    def mma():
+        yield ("wait", "q", 0)
+        yield ("wait", "kf0", 0)
+        sim.mma("M", *s_mma(0, 0))
+        sim.commit("M", "sf0")
+        sim.mma("M", *s_mma(1, 0))
+        sim.commit("M", "sf1")
+        sim.commit("M", "ke0")
+        for jt in range(n):
+            slot_v, slot_k, more = jt % NSV, (jt + 1) % NSK, jt + 1 < n
+            yield ("wait", f"vf{slot_v}", jt // NSV)
+            if more:
+                yield ("wait", f"kf{slot_k}", (jt + 1) // NSK)
+            yield ("wait", "pf0", jt)
+            if mutation == "s_before_pv" and more:  # S_A(j+1) over P_A(j) before PV_A(j)
+                sim.mma("M", *s_mma(0, jt + 1))
+                sim.commit("M", "sf0")
+            sim.mma("M", *pv_mma(0, jt))
+            if mutation == "ve_commit_early":  # V(j) released before PV_B(j) reads it
+                sim.commit("M", f"ve{slot_v}")
+            if more and mutation != "s_before_pv":
+                sim.mma("M", *s_mma(0, jt + 1))
+                sim.commit("M", "sf0")
+            elif not more:
+                sim.commit("M", "of0")
+            if mutation != "no_pf1_wait":
+                yield ("wait", "pf1", jt)
+            sim.mma("M", *pv_mma(1, jt))
+            if mutation != "ve_commit_early":
+                sim.commit("M", f"ve{slot_v}")
+            if more:
+                sim.mma("M", *s_mma(1, jt + 1))
+                sim.commit("M", "sf1")
+                sim.commit("M", f"ke{slot_k}")
+            else:
+                sim.commit("M", "of1")
+        sim.commit("M", "drain")
+        yield ("wait", "drain", 0)
+
+    def softmax(w, rescale_pattern):
+        for jt in range(n):
+            yield ("wait", f"sf{w}", jt)
+            sim.read(S[w], ("S", jt), f"softmax{w} S({jt})")
+            yield None
+            sim.write(S[w], ("P", jt))
+            if jt > 0 and rescale_pattern[jt]:
+                # O holds the sum through tile jt-1; it is scaled in place
+                sim.read(O[w], ("O", jt - 1), f"softmax{w} rescale O({jt})")
+                yield None
+                sim.write(O[w], ("O", jt - 1))
+            yield None
+            sim.bars[f"pf{w}"].arrive()
+        if n > 0:
+            yield ("wait", f"of{w}", 0)
+            sim.read(O[w], ("O", n - 1), f"softmax{w} epilogue O")
+
+    roles = {"prodK": producer(True), "prodV": producer(False), "mma": mma()}
+    for w in (0, 1):
+        pattern = [sim.rng.random() < 0.5 for _ in range(n)]
+        roles[f"sm{w}"] = softmax(w, pattern)
+    return roles
+
+
+@pytest.mark.parametrize("NSK,NSV", [(3, 2), (4, 4)])  # D = 128 and D = 64 rings
+@pytest.mark.parametrize("n", [1, 2, 3, 5, 9])
+def test_forward_protocol_holds_under_random_latencies(NSK, NSV, n):
+    for seed in range(300):
+        sim = Sim(seed * 7919 + n * 31 + NSK)
+        sim.run(fwd_roles(sim, n, NSK, NSV))
+
+
+@pytest.mark.parametrize("mutation", ["no_pf1_wait", "ve_commit_early", "s_before_pv"])
+def test_forward_mutated_protocols_are_caught(mutation):
+    caught = 0
+    for seed in range(300):
+        sim = Sim(seed)
+        try:
+            sim.run(fwd_roles(sim, 6, 3, 2, mutation))
+        except Violation:
+            caught += 1
+    assert caught > 0, f"{mutation} was never flagged"

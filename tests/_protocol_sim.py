@@ -3,7 +3,9 @@ with the hardware's parity rule, arrival counts and TMA transaction counts; MMAs
 issue order per issuing thread and interleaved at random across threads; commits that
 arrive once everything their thread issued before them has completed; TMA loads completing
 at random times; and reads of named memory regions checked against the data they must see.
-Roles are generators that yield ("wait", barrier, phase) or None (a plain step)."""
+Roles are generators that yield ("wait", barrier, phase), ("until", predicate) or None (a
+plain step).  Bulk store groups (TMA stores committed as a group) read their sources when
+they execute, in any order."""
 import random
 
 
@@ -43,6 +45,7 @@ class Sim:
     def __init__(self, seed):
         self.rng = random.Random(seed)
         self.bars, self.mem, self.queues, self.tma = {}, {}, {}, []
+        self.bulk, self.bulk_seq = [], 0  # bulk store groups: (seq, reads, who)
 
     def bar(self, name, count):
         self.bars[name] = Barrier(name, count)
@@ -67,14 +70,30 @@ class Sim:
     def tma_load(self, barrier, region, label):
         self.tma.append((barrier, region, label))
 
+    def bulk_group(self, reads, who):
+        """A committed group of bulk (TMA) stores: it reads its source regions when it
+        executes; groups execute in any order."""
+        self.bulk_seq += 1
+        self.bulk.append((self.bulk_seq, reads, who))
+
+    def bulk_read_done_but(self, k):
+        """cp.async.bulk.wait_group.read k: every group but the k most recent has read."""
+        return all(seq > self.bulk_seq - k for seq, _, _ in self.bulk)
+
     def _step_async(self):
         choices = [q for q in self.queues.values() if q]
         if self.tma:
             choices.append(self.tma)
+        if self.bulk:
+            choices.append(self.bulk)
         if not choices:
             return False
         q = self.rng.choice(choices)
-        if q is self.tma:
+        if q is self.bulk:
+            _, reads, who = self.bulk.pop(self.rng.randrange(len(self.bulk)))
+            for region, want in reads:
+                self.read(region, want, who)
+        elif q is self.tma:
             barrier, region, label = self.tma.pop(self.rng.randrange(len(self.tma)))
             self.write(region, label)
             self.bars[barrier].tx_done()
@@ -91,14 +110,23 @@ class Sim:
         return True
 
     def run(self, roles):
-        """roles: generators yielding ("wait", barrier, phase) or None (a plain step)."""
+        """roles: generators yielding ("wait", barrier, phase), ("until", predicate) or None
+        (a plain step)."""
         state = {name: None for name in roles}  # pending wait of each role
         live = dict(roles)
         idle = 0
-        while live or any(self.queues.values()) or self.tma:
-            runnable = [n for n in live if state[n] is None or
-                        self.bars[state[n][0]].ready(state[n][1])]
-            options = runnable + (["async"] if (any(self.queues.values()) or self.tma) else [])
+
+        def ready(w):
+            if w is None:
+                return True
+            if w[0] == "until":
+                return w[1]()
+            return self.bars[w[0]].ready(w[1])
+
+        while live or any(self.queues.values()) or self.tma or self.bulk:
+            runnable = [n for n in live if ready(state[n])]
+            pending = any(self.queues.values()) or self.tma or self.bulk
+            options = runnable + (["async"] if pending else [])
             if not options:
                 waits = {n: state[n] for n in live}
                 raise Violation(f"deadlock: {waits}")
@@ -108,7 +136,12 @@ class Sim:
                 continue
             try:
                 req = next(live[pick])
-                state[pick] = (req[1], req[2]) if req is not None and req[0] == "wait" else None
+                if req is None:
+                    state[pick] = None
+                elif req[0] == "wait":
+                    state[pick] = (req[1], req[2])
+                else:
+                    state[pick] = ("until", req[1])
             except StopIteration:
                 del live[pick]
                 state.pop(pick)

@@ -69,8 +69,10 @@ def test_plain_matches_torch_sdpa_fp64(oracle_mod, B, L, H_q, H_kv, D, causal):
     scale = 1.0 / math.sqrt(D)
     out, lse = oracle_mod.attention(q, k, v, scale, causal)
     ref_o, ref_l = torch_sdpa(q, k, v, scale, causal)
-    np.testing.assert_allclose(out, ref_o, rtol=0, atol=1e-12)
-    np.testing.assert_allclose(lse, ref_l, rtol=0, atol=1e-12)
+    # both sides are fp64 with different summation orders (the library blocks the keys by
+    # its own rule): up to 129 terms of log-sum-exps near 20 differ by a few 1e-13
+    np.testing.assert_allclose(out, ref_o, rtol=0, atol=1e-11)
+    np.testing.assert_allclose(lse, ref_l, rtol=0, atol=1e-11)
 
 
 # ---------------------------------------------------------------- closed forms

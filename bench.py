@@ -536,7 +536,12 @@ def main():
                           "frac_of_datasheet_hbm": round(perm_gbs / DATASHEET_HBM_GBS, 4)}
     out["gpu_launches"] = path.launches_per_step * args.steps
     out["clocks"] = clk.summary()
-    if not args.no_e2e:
+    if not args.no_e2e and kind.startswith("attn_bwd"):
+        # the leg streams the forward's inputs and output; a backward step's inputs (q, k,
+        # v, O, LSE, dO) and results (dq, dk, dv) are not what it moves, so no number
+        out["e2e"] = None
+        out["e2e_note"] = "not measured for backward workloads"
+    elif not args.no_e2e:
         path2 = Path(kind, w, device)  # second buffer set for the pipelined end-to-end leg
         e2e_ms = e2e_region([path, path2], max(3, min(args.steps, 6)), torch, dist, device)
         del path2

@@ -158,3 +158,16 @@ def test_backward_layout_argument_validation(lib):
     # causal must be 0 or 1 where it is an argument
     assert _bwd(lib, "ra_ring_attn_bwd", causal=2) == 1
     assert _bwd(lib, "ra_ring_attn_bwd_zigzag", causal=-1) == 1
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/ra.h is a C ABI: it compiles as pedantic C99 with no C++ or torch types."""
+    import subprocess
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "ra.h"\n'
+                   "int main(void) { ra_status s = RA_OK; ra_dtype d = RA_BF16; (void)s; (void)d;\n"
+                   "  return RA_BWD_STATIC_MAX_ROWS > 0 && RA_MAX_P > 0 ? 0 : 1; }\n")
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                        "-I", os.path.join(ROOT, "include"), "-c", str(src), "-o",
+                        str(tmp_path / "use_header.o")], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr

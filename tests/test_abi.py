@@ -171,3 +171,22 @@ def test_header_is_plain_c(tmp_path):
                         "-I", os.path.join(ROOT, "include"), "-c", str(src), "-o",
                         str(tmp_path / "use_header.o")], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_tensor_helpers_reject_bad_layouts(lib):
+    """ring_attn_fwd / ring_attn_bwd refuse an unknown layout, and packed samples outside
+    the causal contiguous layout, before touching a device."""
+    import torch
+    from sequence_parallelism_attn_b200 import ra
+    q = torch.zeros(1, 8, 2, 64, dtype=torch.bfloat16)
+    k = torch.zeros(2, 1, 4, 1, 64, dtype=torch.bfloat16)
+    lse = torch.zeros(1, 2, 8)
+    pid = torch.zeros(1, 8, dtype=torch.int32)
+    for call in (lambda: ra.ring_attn_bwd(q, k, k, q, lse, q, True, layout="diagonal"),
+                 lambda: ra.ring_attn_bwd(q, k, k, q, lse, q, True, layout="zigzag",
+                                          position_ids=pid),
+                 lambda: ra.ring_attn_bwd(q, k, k, q, lse, q, False, position_ids=pid),
+                 lambda: ra.ring_attn_fwd(q, k, k, True, layout="diagonal"),
+                 lambda: ra.ring_attn_fwd(q, k, k, False, position_ids=pid)):
+        with pytest.raises(ValueError):
+            call()

@@ -42,8 +42,11 @@ class Barrier:
 
 
 class Sim:
-    def __init__(self, seed):
+    def __init__(self, seed, abort_after=None):
         self.rng = random.Random(seed)
+        # abort injection: after this many scheduler steps a role's bounded wait gives up;
+        # from then on every abortable wait returns False (the CTA abort flag)
+        self.abort_after, self.aborted, self.steps = abort_after, False, 0
         self.bars, self.mem, self.queues, self.tma = {}, {}, {}, []
         self.bulk, self.bulk_seq = [], 0  # bulk store groups: (seq, reads, who)
 
@@ -55,6 +58,8 @@ class Sim:
         self.mem[region] = label
 
     def read(self, region, want, who):
+        if self.aborted:
+            return  # after an abort the outputs are undefined; only teardown is checked
         got = self.mem.get(region)
         if got != want:
             raise Violation(f"{who} read {region}: saw {got}, expected {want}")
@@ -110,8 +115,12 @@ class Sim:
         return True
 
     def run(self, roles):
-        """roles: generators yielding ("wait", barrier, phase), ("until", predicate) or None
-        (a plain step)."""
+        """roles: generators yielding ("wait", barrier, phase) (a bounded wait: the value sent
+        back is False once the CTA has aborted), ("drain", barrier, phase) (a wait for the
+        role's own asynchronous work, which must complete), ("until", predicate) or None
+        (a plain step).  When the last role returns -- the kernel's final block barrier,
+        after which tensor memory is freed -- no MMA, TMA load or bulk store may be in
+        flight."""
         state = {name: None for name in roles}  # pending wait of each role
         live = dict(roles)
         idle = 0
@@ -121,9 +130,15 @@ class Sim:
                 return True
             if w[0] == "until":
                 return w[1]()
-            return self.bars[w[0]].ready(w[1])
+            if w[0] == "wait" and self.aborted:
+                return True
+            return self.bars[w[1]].ready(w[2])
 
+        sent = {name: None for name in roles}
         while live or any(self.queues.values()) or self.tma or self.bulk:
+            self.steps += 1
+            if self.abort_after is not None and self.steps >= self.abort_after:
+                self.aborted = True
             runnable = [n for n in live if ready(state[n])]
             pending = any(self.queues.values()) or self.tma or self.bulk
             options = runnable + (["async"] if pending else [])
@@ -134,17 +149,25 @@ class Sim:
             if pick == "async":
                 self._step_async()
                 continue
+            w = state[pick]
+            if w is not None and w[0] in ("wait", "drain") and w[0] == "wait":
+                value = not (self.aborted and not self.bars[w[1]].ready(w[2]))
+            else:
+                value = True
             try:
-                req = next(live[pick])
+                req = live[pick].send(value if sent[pick] is not None else None)
+                sent[pick] = True
                 if req is None:
                     state[pick] = None
-                elif req[0] == "wait":
-                    state[pick] = (req[1], req[2])
+                elif req[0] in ("wait", "drain"):
+                    state[pick] = (req[0], req[1], req[2])
                 else:
                     state[pick] = ("until", req[1])
             except StopIteration:
                 del live[pick]
                 state.pop(pick)
+                if not live and (any(self.queues.values()) or self.tma or self.bulk):
+                    raise Violation("the CTA finished with asynchronous work in flight")
             idle += 1
             if idle > 10_000_000:
                 raise Violation("no termination")

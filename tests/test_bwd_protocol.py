@@ -38,15 +38,21 @@ def dkdv_roles(sim, n, mutation=None):
         sim.bars["fixed"].arrive(tx=1)
         sim.tma_load("fixed", "KV", "KV")
         yield None
+        armed = {}
         for it in range(n):
             slot = it % NS
-            if it >= NS:
-                yield ("wait", f"empty{slot}", it // NS - 1)
+            if it >= NS and not (yield ("wait", f"empty{slot}", it // NS - 1)):
+                break
             sim.bars[f"full{slot}"].arrive(tx=1)       # expect_tx, then Q and dO
             sim.tma_load(f"full{slot}", f"stage{slot}", ("QdO", it))
             sim.write(f"rows{slot}", ("rows", it))      # LSE, Delta, positions: plain stores
             yield None
             sim.bars[f"full{slot}"].arrive()
+            armed[slot] = it
+        if mutation != "no_load_drain":
+            yield ("drain", "fixed", 0)                 # every copy it started has landed
+            for slot, it in armed.items():
+                yield ("drain", f"full{slot}", it // NS)
 
     def stage_reads(i):
         return [(f"stage{i % NS}", ("QdO", i))]
@@ -55,54 +61,66 @@ def dkdv_roles(sim, n, mutation=None):
         return [region + "h0", region + "h1"]
 
     def mma_a():  # dP^T and dV
-        yield ("wait", "fixed", 0)
-        yield ("wait", "full0", 0)
-        sim.mma("A", [("KV", "KV")] + stage_reads(0),
-                [(r, ("S", 0)) for r in half_regions(st_col(0))], "S^T(0)")
-        sim.mma("A", [("KV", "KV")] + stage_reads(0),
-                [(r, ("dP", 0)) for r in half_regions(dpt_col(0))], "dP^T(0)")
-        sim.commit("A", "sd")
-        for it in range(n):
-            more = it + 1 < n
-            yield ("wait", "ds0", it)
-            sim.mma("A", [(st_col(it) + "h0", ("PdS", it))] + stage_reads(it), [], f"dV h0({it})")
-            yield ("wait", "ds1", it)
-            sim.mma("A", [(st_col(it) + "h1", ("PdS", it))] + stage_reads(it), [], f"dV h1({it})")
-            if more and mutation != "no_xfree_wait":
-                yield ("wait", "xfree", it)
-            sim.commit("A", f"empty{it % NS}")
-            if more:
-                sim.mma("A", [("KV", "KV")] + stage_reads(it + 1),
-                        [(r, ("dP", it + 1)) for r in half_regions(dpt_col(it + 1))],
-                        f"dP^T({it + 1})")
-                sim.commit("A", "sd")
-        sim.commit("A", "acc")
+        if (yield ("wait", "fixed", 0)) and (yield ("wait", "full0", 0)):
+            sim.mma("A", [("KV", "KV")] + stage_reads(0),
+                    [(r, ("S", 0)) for r in half_regions(st_col(0))], "S^T(0)")
+            sim.mma("A", [("KV", "KV")] + stage_reads(0),
+                    [(r, ("dP", 0)) for r in half_regions(dpt_col(0))], "dP^T(0)")
+            sim.commit("A", "sd")
+            for it in range(n):
+                more = it + 1 < n
+                if not (yield ("wait", "ds0", it)):
+                    break
+                sim.mma("A", [(st_col(it) + "h0", ("PdS", it))] + stage_reads(it), [],
+                        f"dV h0({it})")
+                if not (yield ("wait", "ds1", it)):
+                    break
+                sim.mma("A", [(st_col(it) + "h1", ("PdS", it))] + stage_reads(it), [],
+                        f"dV h1({it})")
+                if more and mutation != "no_xfree_wait" and not (yield ("wait", "xfree", it)):
+                    break
+                sim.commit("A", f"empty{it % NS}")
+                if more:
+                    sim.mma("A", [("KV", "KV")] + stage_reads(it + 1),
+                            [(r, ("dP", it + 1)) for r in half_regions(dpt_col(it + 1))],
+                            f"dP^T({it + 1})")
+                    sim.commit("A", "sd")
+        sim.commit("A", "acc")  # unconditional (n > 0): a commit with nothing pending arrives
         sim.commit("A", "drain")
-        yield ("wait", "drain", 0)
+        if mutation != "no_mma_drain":
+            yield ("drain", "drain", 0)
 
     def mma_b():  # S^T and dK
-        yield ("wait", "fixed", 0)
-        yield ("wait", "full0", 0)
-        for it in range(n):
-            if it + 1 < n:
-                if mutation != "no_dpfree_wait":
-                    yield ("wait", "dpfree", it)
-                yield ("wait", f"full{(it + 1) % NS}", (it + 1) // NS)
-                sim.mma("B", [("KV", "KV")] + stage_reads(it + 1),
-                        [(r, ("S", it + 1)) for r in half_regions(st_col(it + 1))],
-                        f"S^T({it + 1})")
-            yield ("wait", "ds0", it)
-            sim.mma("B", [(st_col(it) + "h0", ("PdS", it))] + stage_reads(it), [], f"dK h0({it})")
-            yield ("wait", "ds1", it)
-            sim.mma("B", [(st_col(it) + "h1", ("PdS", it))] + stage_reads(it), [], f"dK h1({it})")
-            sim.commit("B", "xfree")
+        if (yield ("wait", "fixed", 0)) and (yield ("wait", "full0", 0)):
+            for it in range(n):
+                if it + 1 < n:
+                    if mutation != "no_dpfree_wait" and not (yield ("wait", "dpfree", it)):
+                        break
+                    if not (yield ("wait", f"full{(it + 1) % NS}", (it + 1) // NS)):
+                        break
+                    sim.mma("B", [("KV", "KV")] + stage_reads(it + 1),
+                            [(r, ("S", it + 1)) for r in half_regions(st_col(it + 1))],
+                            f"S^T({it + 1})")
+                if not (yield ("wait", "ds0", it)):
+                    break
+                sim.mma("B", [(st_col(it) + "h0", ("PdS", it))] + stage_reads(it), [],
+                        f"dK h0({it})")
+                if not (yield ("wait", "ds1", it)):
+                    break
+                sim.mma("B", [(st_col(it) + "h1", ("PdS", it))] + stage_reads(it), [],
+                        f"dK h1({it})")
+                sim.commit("B", "xfree")
         sim.commit("B", "acc")
         sim.commit("B", "drain")
-        yield ("wait", "drain", 0)
+        if mutation != "no_mma_drain":
+            yield ("drain", "drain", 0)
 
     def compute(c):
+        ok = True
         for it in range(n):
-            yield ("wait", "sd", it)
+            if not (yield ("wait", "sd", it)):
+                ok = False
+                break
             sim.read(f"{st_col(it)}h{c}", ("S", it), f"WG{c} S({it})")
             sim.read(f"{dpt_col(it)}h{c}", ("dP", it), f"WG{c} dP({it})")
             yield None
@@ -114,7 +132,7 @@ def dkdv_roles(sim, n, mutation=None):
             sim.write(f"{st_col(it)}h{c}", ("PdS", it))
             yield None
             sim.bars[f"ds{c}"].arrive()
-        if n > 0:
+        if ok and n > 0:
             yield ("wait", "acc", 0)
 
     return {"load": loader(), "A": mma_a(), "B": mma_b(), "WG0": compute(0), "WG1": compute(1)}
@@ -135,57 +153,68 @@ def dq_roles(sim, n, mutation=None):
         sim.bars["fixed"].arrive(tx=1)
         sim.tma_load("fixed", "QdO", "QdO")
         yield None
+        armed = {}
         for jt in range(n):
             slot = jt % NS
-            if jt >= NS:
-                yield ("wait", f"empty{slot}", jt // NS - 1)
+            if jt >= NS and not (yield ("wait", f"empty{slot}", jt // NS - 1)):
+                break
             sim.bars[f"full{slot}"].arrive(tx=1)
             sim.tma_load(f"full{slot}", f"stage{slot}", ("KV", jt))
+            armed[slot] = jt
             yield None
+        yield ("drain", "fixed", 0)
+        for slot, jt in armed.items():
+            yield ("drain", f"full{slot}", jt // NS)
 
     kv = lambda j: [(f"stage{j % NS}", ("KV", j)), ("QdO", "QdO")]
 
     def mma_a():  # S and dQ
-        yield ("wait", "fixed", 0)
-        yield ("wait", "full0", 0)
-        sim.mma("A", kv(0), [(s_col(0) + "h0", ("S", 0)), (s_col(0) + "h1", ("S", 0))], "S(0)")
-        sim.commit("A", "sd")
-        for jt in range(n):
-            more = jt + 1 < n
-            if more:
-                yield ("wait", f"full{(jt + 1) % NS}", (jt + 1) // NS)
-                sim.mma("A", kv(jt + 1), [(s_col(jt + 1) + "h0", ("S", jt + 1)),
-                                          (s_col(jt + 1) + "h1", ("S", jt + 1))], f"S({jt + 1})")
-            yield ("wait", "ds0", jt)
-            sim.mma("A", [(s_col(jt) + "h0", ("dS", jt))] + kv(jt), [], f"dQ h0({jt})")
-            if mutation != "no_ds1_wait":
-                yield ("wait", "ds1", jt)
-            if more:
-                sim.commit("A", "sd")
-            sim.mma("A", [(s_col(jt) + "h1", ("dS", jt))] + kv(jt), [], f"dQ h1({jt})")
-            sim.commit("A", f"empty{jt % NS}")
+        if (yield ("wait", "fixed", 0)) and (yield ("wait", "full0", 0)):
+            sim.mma("A", kv(0), [(s_col(0) + "h0", ("S", 0)), (s_col(0) + "h1", ("S", 0))],
+                    "S(0)")
+            sim.commit("A", "sd")
+            for jt in range(n):
+                more = jt + 1 < n
+                if more:
+                    if not (yield ("wait", f"full{(jt + 1) % NS}", (jt + 1) // NS)):
+                        break
+                    sim.mma("A", kv(jt + 1), [(s_col(jt + 1) + "h0", ("S", jt + 1)),
+                                              (s_col(jt + 1) + "h1", ("S", jt + 1))],
+                            f"S({jt + 1})")
+                if not (yield ("wait", "ds0", jt)):
+                    break
+                sim.mma("A", [(s_col(jt) + "h0", ("dS", jt))] + kv(jt), [], f"dQ h0({jt})")
+                if mutation != "no_ds1_wait" and not (yield ("wait", "ds1", jt)):
+                    break
+                if more:
+                    sim.commit("A", "sd")
+                sim.mma("A", [(s_col(jt) + "h1", ("dS", jt))] + kv(jt), [], f"dQ h1({jt})")
+                sim.commit("A", f"empty{jt % NS}")
         sim.commit("A", "acc")
         sim.commit("A", "drain")
-        yield ("wait", "drain", 0)
+        yield ("drain", "drain", 0)
 
     def mma_b():  # dP
-        yield ("wait", "fixed", 0)
-        yield ("wait", "full0", 0)
-        sim.mma("B", kv(0), [("dPh0", ("dP", 0)), ("dPh1", ("dP", 0))], "dP(0)")
-        sim.commit("B", "sd")
-        for jt in range(n - 1):
-            if mutation != "no_dpfree_wait":
-                yield ("wait", "dpfree", jt)
-            yield ("wait", f"full{(jt + 1) % NS}", (jt + 1) // NS)
-            sim.mma("B", kv(jt + 1), [("dPh0", ("dP", jt + 1)), ("dPh1", ("dP", jt + 1))],
-                    f"dP({jt + 1})")
+        if (yield ("wait", "fixed", 0)) and (yield ("wait", "full0", 0)):
+            sim.mma("B", kv(0), [("dPh0", ("dP", 0)), ("dPh1", ("dP", 0))], "dP(0)")
             sim.commit("B", "sd")
+            for jt in range(n - 1):
+                if mutation != "no_dpfree_wait" and not (yield ("wait", "dpfree", jt)):
+                    break
+                if not (yield ("wait", f"full{(jt + 1) % NS}", (jt + 1) // NS)):
+                    break
+                sim.mma("B", kv(jt + 1), [("dPh0", ("dP", jt + 1)), ("dPh1", ("dP", jt + 1))],
+                        f"dP({jt + 1})")
+                sim.commit("B", "sd")
         sim.commit("B", "drain")
-        yield ("wait", "drain", 0)
+        yield ("drain", "drain", 0)
 
     def compute(c):
+        ok = True
         for jt in range(n):
-            yield ("wait", "sd", jt)
+            if not (yield ("wait", "sd", jt)):
+                ok = False
+                break
             sim.read(f"{s_col(jt)}h{c}", ("S", jt), f"WG{c} S({jt})")
             sim.read(f"dPh{c}", ("dP", jt), f"WG{c} dP({jt})")
             yield None
@@ -194,7 +223,7 @@ def dq_roles(sim, n, mutation=None):
             sim.write(f"{s_col(jt)}h{c}", ("dS", jt))
             yield None
             sim.bars[f"ds{c}"].arrive()
-        if n > 0:
+        if ok and n > 0:
             yield ("wait", "acc", 0)
 
     return {"load": loader(), "A": mma_a(), "B": mma_b(), "WG0": compute(0), "WG1": compute(1)}
@@ -225,3 +254,28 @@ def test_mutated_protocols_are_caught(kernel, mutation):
         except Violation:
             caught += 1
     assert caught > 0, f"{kernel} with {mutation} was never flagged"
+
+
+@pytest.mark.parametrize("kernel", ["dkdv", "dq"])
+@pytest.mark.parametrize("n", [1, 3, 6])
+def test_abort_at_any_point_tears_down_cleanly(kernel, n):
+    """A bounded wait that gives up at any step: every role stops, drains only its own
+    work, and the CTA ends with no MMA or TMA load in flight (tensor memory and shared
+    memory may then be released), without deadlock."""
+    for seed in range(400):
+        sim = Sim(seed, abort_after=1 + seed % (40 * n))
+        sim.run(KERNELS[kernel](sim, n))
+
+
+@pytest.mark.parametrize("mutation", ["no_mma_drain", "no_load_drain"])
+def test_teardown_without_a_drain_is_caught(mutation):
+    """Both MMA threads skipping their drain wait (either one alone is covered by the
+    other's, since the drain barrier counts both commits), or the loader skipping its own."""
+    caught = 0
+    for seed in range(400):
+        sim = Sim(seed, abort_after=1 + seed % 200)
+        try:
+            sim.run(dkdv_roles(sim, 5, mutation))
+        except Violation:
+            caught += 1
+    assert caught > 0, f"{mutation} was never flagged"

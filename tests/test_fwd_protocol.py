@@ -36,16 +36,16 @@ def fwd_roles(sim, n, NSK, NSV, mutation=None):
         armed = {}
         for jt in range(n):
             slot = jt % ns
-            if jt >= ns:
-                yield ("wait", f"{empty}{slot}", jt // ns - 1)
+            if jt >= ns and not (yield ("wait", f"{empty}{slot}", jt // ns - 1)):
+                break
             sim.bars[f"{full}{slot}"].arrive(tx=1)
             sim.tma_load(f"{full}{slot}", f"{tag}{slot}", (tag, jt))
             armed[slot] = jt
             yield None
         if is_k:
-            yield ("wait", "q", 0)
-        for slot, jt in armed.items():  # drain: every copy landed
-            yield ("wait", f"{full}{slot}", jt // ns)
+            yield ("drain", "q", 0)
+        for slot, jt in armed.items():  # drain: every copy this thread started has landed
+            yield ("drain", f"{full}{slot}", jt // ns)
 
     def s_mma(w, j):
         return (("Q", "Q"), (f"K{j % NSK}", ("K", j))), ((S[w], ("S", j)),), f"S_{'AB'[w]}({j})"
@@ -57,47 +57,55 @@ def fwd_roles(sim, n, NSK, NSV, mutation=None):
         return reads, [(O[w], ("O", j))], f"PV_{'AB'[w]}({j})"
 
     def mma():
-        yield ("wait", "q", 0)
-        yield ("wait", "kf0", 0)
-        sim.mma("M", *s_mma(0, 0))
-        sim.commit("M", "sf0")
-        sim.mma("M", *s_mma(1, 0))
-        sim.commit("M", "sf1")
-        sim.commit("M", "ke0")
-        for jt in range(n):
-            slot_v, slot_k, more = jt % NSV, (jt + 1) % NSK, jt + 1 < n
-            yield ("wait", f"vf{slot_v}", jt // NSV)
-            if more:
-                yield ("wait", f"kf{slot_k}", (jt + 1) // NSK)
-            yield ("wait", "pf0", jt)
-            if mutation == "s_before_pv" and more:  # S_A(j+1) over P_A(j) before PV_A(j)
-                sim.mma("M", *s_mma(0, jt + 1))
-                sim.commit("M", "sf0")
-            sim.mma("M", *pv_mma(0, jt))
-            if mutation == "ve_commit_early":  # V(j) released before PV_B(j) reads it
-                sim.commit("M", f"ve{slot_v}")
-            if more and mutation != "s_before_pv":
-                sim.mma("M", *s_mma(0, jt + 1))
-                sim.commit("M", "sf0")
-            elif not more:
-                sim.commit("M", "of0")
-            if mutation != "no_pf1_wait":
-                yield ("wait", "pf1", jt)
-            sim.mma("M", *pv_mma(1, jt))
-            if mutation != "ve_commit_early":
-                sim.commit("M", f"ve{slot_v}")
-            if more:
-                sim.mma("M", *s_mma(1, jt + 1))
-                sim.commit("M", "sf1")
-                sim.commit("M", f"ke{slot_k}")
-            else:
-                sim.commit("M", "of1")
-        sim.commit("M", "drain")
-        yield ("wait", "drain", 0)
+        issued = False
+        if (yield ("wait", "q", 0)) and (yield ("wait", "kf0", 0)):
+            sim.mma("M", *s_mma(0, 0))
+            sim.commit("M", "sf0")
+            sim.mma("M", *s_mma(1, 0))
+            sim.commit("M", "sf1")
+            sim.commit("M", "ke0")
+            issued = True
+            for jt in range(n):
+                slot_v, slot_k, more = jt % NSV, (jt + 1) % NSK, jt + 1 < n
+                if not (yield ("wait", f"vf{slot_v}", jt // NSV)):
+                    break
+                if more and not (yield ("wait", f"kf{slot_k}", (jt + 1) // NSK)):
+                    break
+                if not (yield ("wait", "pf0", jt)):
+                    break
+                if mutation == "s_before_pv" and more:  # S_A(j+1) over P_A(j) before PV_A(j)
+                    sim.mma("M", *s_mma(0, jt + 1))
+                    sim.commit("M", "sf0")
+                sim.mma("M", *pv_mma(0, jt))
+                if mutation == "ve_commit_early":  # V(j) released before PV_B(j) reads it
+                    sim.commit("M", f"ve{slot_v}")
+                if more and mutation != "s_before_pv":
+                    sim.mma("M", *s_mma(0, jt + 1))
+                    sim.commit("M", "sf0")
+                elif not more:
+                    sim.commit("M", "of0")
+                if mutation != "no_pf1_wait" and not (yield ("wait", "pf1", jt)):
+                    break
+                sim.mma("M", *pv_mma(1, jt))
+                if mutation != "ve_commit_early":
+                    sim.commit("M", f"ve{slot_v}")
+                if more:
+                    sim.mma("M", *s_mma(1, jt + 1))
+                    sim.commit("M", "sf1")
+                    sim.commit("M", f"ke{slot_k}")
+                else:
+                    sim.commit("M", "of1")
+        if issued:  # every MMA this thread issued completes before tensor memory is freed
+            sim.commit("M", "drain")
+            if mutation != "no_mma_drain":
+                yield ("drain", "drain", 0)
 
     def softmax(w, rescale_pattern):
+        ok = True
         for jt in range(n):
-            yield ("wait", f"sf{w}", jt)
+            if not (yield ("wait", f"sf{w}", jt)):
+                ok = False
+                break
             sim.read(S[w], ("S", jt), f"softmax{w} S({jt})")
             yield None
             sim.write(S[w], ("P", jt))
@@ -108,8 +116,7 @@ def fwd_roles(sim, n, NSK, NSV, mutation=None):
                 sim.write(O[w], ("O", jt - 1))
             yield None
             sim.bars[f"pf{w}"].arrive()
-        if n > 0:
-            yield ("wait", f"of{w}", 0)
+        if ok and n > 0 and (yield ("wait", f"of{w}", 0)):
             sim.read(O[w], ("O", n - 1), f"softmax{w} epilogue O")
 
     roles = {"prodK": producer(True), "prodV": producer(False), "mma": mma()}
@@ -137,3 +144,21 @@ def test_forward_mutated_protocols_are_caught(mutation):
         except Violation:
             caught += 1
     assert caught > 0, f"{mutation} was never flagged"
+
+
+@pytest.mark.parametrize("n", [1, 3, 6])
+def test_forward_abort_at_any_point_tears_down_cleanly(n):
+    """A bounded wait that gives up at any step: every role stops, drains only its own
+    work, and the CTA ends with no MMA or TMA load in flight, without deadlock; without the
+    MMA thread's drain it may not."""
+    for seed in range(400):
+        sim = Sim(seed, abort_after=1 + seed % (30 * n))
+        sim.run(fwd_roles(sim, n, 3, 2))
+    caught = 0
+    for seed in range(400):
+        sim = Sim(seed, abort_after=1 + seed % (30 * n))
+        try:
+            sim.run(fwd_roles(sim, n, 3, 2, "no_mma_drain"))
+        except Violation:
+            caught += 1
+    assert caught > 0

@@ -28,8 +28,10 @@ def permute_role(sim, n_blocks, NS, rep, mutation=None):
         while issued < NS - 1 and issued < n_blocks:
             issue_load(issued)
             issued += 1
-        for n in range(n_blocks):
-            yield ("wait", f"b{n % NS}", n // NS)
+        n = 0
+        while n < n_blocks:
+            if not (yield ("wait", f"b{n % NS}", n // NS)):
+                break  # the bounded wait gave up
             sim.bulk_group([(f"stage{n % NS}", ("blk", n))] * rep, f"stores of block {n}")
             if issued < n_blocks:
                 if mutation == "no_read_wait":
@@ -39,8 +41,12 @@ def permute_role(sim, n_blocks, NS, rep, mutation=None):
                     yield ("until", lambda k=k: sim.bulk_read_done_but(k))
                 issue_load(issued)
                 issued += 1
+            n += 1
             yield None
         yield ("until", lambda: sim.bulk_read_done_but(0))  # bulk_wait_all
+        if mutation != "no_load_drain":
+            for i in range(n, issued):  # loads issued but never consumed land before exit
+                yield ("drain", f"b{i % NS}", i // NS)
 
     return {"thread": thread()}
 
@@ -63,3 +69,20 @@ def test_permute_ring_mutations_are_caught(mutation):
         except Violation:
             caught += 1
     assert caught > 0, f"{mutation} was never flagged"
+
+
+@pytest.mark.parametrize("n_blocks", [2, 5, 9])
+def test_permute_ring_abort_tears_down_cleanly(n_blocks):
+    """A wait that gives up at any step: the thread waits for its stores and the loads it
+    issued, so the CTA ends with nothing in flight; without the load drain it may not."""
+    for seed in range(400):
+        sim = Sim(seed, abort_after=1 + seed % (12 * n_blocks))
+        sim.run(permute_role(sim, n_blocks, 3, 2))
+    caught = 0
+    for seed in range(400):
+        sim = Sim(seed, abort_after=1 + seed % (12 * n_blocks))
+        try:
+            sim.run(permute_role(sim, n_blocks, 3, 2, "no_load_drain"))
+        except Violation:
+            caught += 1
+    assert caught > 0

@@ -190,3 +190,46 @@ def test_tensor_helpers_reject_bad_layouts(lib):
                  lambda: ra.ring_attn_fwd(q, k, k, False, position_ids=pid)):
         with pytest.raises(ValueError):
             call()
+
+
+def _c_params():
+    """name -> list of parameter kinds parsed from the RA_API declarations of ra.h."""
+    text = open(os.path.join(ROOT, "include", "ra.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    out = {}
+    for m in re.finditer(r"RA_API\s+[\w\s\*]+?\b(ra_\w+)\s*\(([^)]*)\)\s*;", text):
+        params = [p.strip() for p in m.group(2).split(",") if p.strip() and p.strip() != "void"]
+        kinds = []
+        for p in params:
+            p = " ".join(p.split())
+            if "*" in p:
+                kinds.append("ptr")
+            elif p.startswith("unsigned long long"):
+                kinds.append("u64")
+            elif p.startswith("long long"):
+                kinds.append("i64")
+            elif p.startswith("float"):
+                kinds.append("f32")
+            elif p.startswith("int") or p.startswith("ra_dtype"):
+                kinds.append("i32")
+            else:
+                raise AssertionError(f"unmapped parameter {p!r} of {m.group(1)}")
+        out[m.group(1)] = kinds
+    return out
+
+
+def test_binding_argtypes_match_the_header(lib):
+    """Every entry point's ctypes argtypes agree with its C parameter list in ra.h."""
+    kind = {ctypes.c_void_p: "ptr", ctypes.c_int: "i32", ctypes.c_longlong: "i64",
+            ctypes.c_float: "f32", ctypes.c_ulonglong: "u64"}
+    params = _c_params()
+    assert set(params) == set(declared_symbols())
+    checked = 0
+    for name, want in params.items():
+        argtypes = getattr(lib, name).argtypes
+        if argtypes is None:
+            assert want == [], f"{name} takes arguments but has no argtypes"
+            continue
+        assert [kind[t] for t in argtypes] == want, name
+        checked += 1
+    assert checked >= 12

@@ -25,20 +25,35 @@ def rnd(shape, seed, scale=1.0):
     return np.random.default_rng(seed).standard_normal(shape) * scale
 
 
+def exact_lse(q, k, scale, causal):
+    """The log-sum-exp of every query row by its definition with exactly rounded sums
+    (math.fsum for the dot products and for the sum of exponentials)."""
+    B, L, H_q, D = q.shape
+    rep = H_q // k.shape[2]
+    out = np.empty((B, H_q, L))
+    for b in range(B):
+        for h in range(H_q):
+            kh = k[b, :, h // rep]
+            for t in range(L):
+                n = t + 1 if causal else L
+                s = [scale * math.fsum(q[b, t, h] * kh[j]) for j in range(n)]
+                m = max(s)
+                out[b, h, t] = m + math.log(math.fsum(math.exp(x - m) for x in s))
+    return out
+
+
 def torch_sdpa(q, k, v, scale, causal):
-    """float64 library attention; q [B,L,H_q,D], k/v [B,L,H_kv,D] -> out, lse."""
+    """float64 library attention (torch SDPA) for the output; the LSE, which the library
+    does not return, by its definition with exactly rounded sums.  (torch's own float64
+    matmul + logsumexp on the CPU was seen, in about one process in twenty, to take a path
+    about 1e-10 off the exact value, so it serves as no reference.)
+    q [B,L,H_q,D], k/v [B,L,H_kv,D] -> out, lse."""
     tq = torch.from_numpy(q).permute(0, 2, 1, 3)
     tk = torch.from_numpy(k).permute(0, 2, 1, 3)
     tv = torch.from_numpy(v).permute(0, 2, 1, 3)
     out = torch.nn.functional.scaled_dot_product_attention(
         tq, tk, tv, scale=scale, is_causal=causal, enable_gqa=True)
-    rep = q.shape[2] // k.shape[2]
-    s = torch.matmul(tq, tk.repeat_interleave(rep, dim=1).transpose(-1, -2)) * scale
-    if causal:
-        L = q.shape[1]
-        s = s.masked_fill(torch.ones(L, L, dtype=torch.bool).triu(1), float("-inf"))
-    lse = torch.logsumexp(s, dim=-1)
-    return out.permute(0, 2, 1, 3).numpy(), lse.numpy()
+    return out.permute(0, 2, 1, 3).numpy(), exact_lse(q, k, scale, causal)
 
 
 # ---------------------------------------------------------------- worked example
@@ -69,10 +84,8 @@ def test_plain_matches_torch_sdpa_fp64(oracle_mod, B, L, H_q, H_kv, D, causal):
     scale = 1.0 / math.sqrt(D)
     out, lse = oracle_mod.attention(q, k, v, scale, causal)
     ref_o, ref_l = torch_sdpa(q, k, v, scale, causal)
-    # both sides are fp64 with different summation orders (the library blocks the keys by
-    # its own rule): up to 129 terms of log-sum-exps near 20 differ by a few 1e-13
-    np.testing.assert_allclose(out, ref_o, rtol=0, atol=1e-11)
-    np.testing.assert_allclose(lse, ref_l, rtol=0, atol=1e-11)
+    np.testing.assert_allclose(out, ref_o, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, ref_l, rtol=0, atol=1e-12)
 
 
 # ---------------------------------------------------------------- closed forms

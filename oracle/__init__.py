@@ -58,9 +58,11 @@ def _load():
     lib.ora_attention_backward.argtypes = [P, P, P, P, i32, i64, i32, i32, i32, f64, i32, P, P,
                                            P, i32]
     lib.ora_packed_lower_bounds.argtypes = [P, i32, i64, P]
+    lib.ora_attention_backward_rows.argtypes = [P, P, P, P, i32, i64, i32, i32, i32, f64, i32, P,
+                                                P, i64, P, P, P, i64, P, P, P, P, P, P, i32]
     for f in ("ora_attention", "ora_attention_rows", "ora_ring_attention", "ora_lse_merge",
               "ora_seq2head", "ora_head2seq", "ora_zigzag_positions", "ora_packed_lower_bounds",
-              "ora_attention_backward"):
+              "ora_attention_backward", "ora_attention_backward_rows"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -105,6 +107,39 @@ def attention_backward(q, k, v, dout, scale: float, causal: bool, nthreads: int 
                                         D, float(scale), int(bool(causal)), _ptr(dq), _ptr(dk),
                                         _ptr(dv), nthreads)
     _check(rc, "attention_backward")
+    return dq, dk, dv
+
+
+def attention_backward_rows(q, k, v, dout, scale: float, causal: bool, q_rows, k_rows,
+                            positions=None, lower_bounds=None, nthreads: int = 0):
+    """Gradients of plain attention on sampled rows: dQ of the query rows q_rows = (b, t, h)
+    and dK, dV of the key rows k_rows = (b, t, kv head).  q/dout [B,L,H_q,D], k/v
+    [B,L,H_kv,D] in storage order; positions [L] (sequence position of each stored token,
+    default t) and lower_bounds [B,L] (smallest key position a query may see) as for
+    ring_attention.  Returns (dq [nq,D], dk [nk,D], dv [nk,D])."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, L, H_q, D = q.shape
+    H_kv = k.shape[2]
+    assert k.shape == (B, L, H_kv, D) and v.shape == k.shape and dout.shape == q.shape
+    qb, qt, qh = (np.ascontiguousarray(x, dtype=dt) for x, dt in
+                  zip(q_rows, (np.int32, np.int64, np.int32)))
+    kb, kt, kg = (np.ascontiguousarray(x, dtype=dt) for x, dt in
+                  zip(k_rows, (np.int32, np.int64, np.int32)))
+    assert qb.shape == qt.shape == qh.shape and kb.shape == kt.shape == kg.shape
+    pos = None if positions is None else np.ascontiguousarray(positions, dtype=np.int64)
+    lo = None if lower_bounds is None else np.ascontiguousarray(lower_bounds, dtype=np.int64)
+    assert pos is None or pos.shape == (L,)
+    assert lo is None or lo.shape == (B, L)
+    nq, nk = qb.shape[0], kb.shape[0]
+    dq = np.empty((nq, D), np.float64)
+    dk = np.empty((nk, D), np.float64)
+    dv = np.empty((nk, D), np.float64)
+    rc = _load().ora_attention_backward_rows(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(dout), B, L, H_q, H_kv, D, float(scale),
+        int(bool(causal)), _ptr(pos) if pos is not None else None,
+        _ptr(lo) if lo is not None else None, nq, _ptr(qb), _ptr(qt), _ptr(qh), nk, _ptr(kb),
+        _ptr(kt), _ptr(kg), _ptr(dq), _ptr(dk), _ptr(dv), nthreads)
+    _check(rc, "attention_backward_rows")
     return dq, dk, dv
 
 

@@ -366,6 +366,131 @@ int ora_attention_backward(const double* q, const double* k, const double* v,
     return 0;
 }
 
+// The same gradients for a sample of rows, at sizes where every row is too slow: dQ of
+// the query rows (qb, qt, qh) and dK, dV of the key rows (kb, kt, kg).  Tokens are given
+// in storage order; `pos` (NULL: pos[t] = t) gives the sequence position of each stored
+// token and `lo` (NULL: none) the smallest key position each query of each batch row may
+// see, as in ora_ring_attention, so one function serves the contiguous and zigzag shard
+// layouts and packed samples.  Visibility of key j to query t (same batch row b):
+//   (!causal || pos[j] <= pos[t]) && pos[j] >= lo[b][t].
+// The formulas are those of ora_attention_backward.  A key row's dK, dV sum over every
+// query row of its kv group that sees it, which needs lse and Delta of all those rows:
+// pass 1 computes them for every row of each (b, h) with a sampled key row of its group,
+// and for the sampled query rows.  A row that sees no key has P = 0 everywhere.
+//   q, dout [B][L][H_q][D]   k, v [B][L][H_kv][D]   lo [B][L]   pos [L]
+//   dq_rows [nq][D]   dk_rows, dv_rows [nk][D]
+int ora_attention_backward_rows(const double* q, const double* k, const double* v,
+                                const double* dout, int B, long long L, int H_q, int H_kv, int D,
+                                double scale, int causal, const long long* pos,
+                                const long long* lo, long long nq, const int* qb,
+                                const long long* qt, const int* qh, long long nk, const int* kb,
+                                const long long* kt, const int* kg, double* dq_rows,
+                                double* dk_rows, double* dv_rows, int nthreads) {
+    if (B < 1 || L < 1 || H_q < 1 || H_kv < 1 || D < 1 || H_q % H_kv != 0 || nq < 0 || nk < 0)
+        return 1;
+    for (long long i = 0; i < nq; ++i)
+        if (qb[i] < 0 || qb[i] >= B || qt[i] < 0 || qt[i] >= L || qh[i] < 0 || qh[i] >= H_q)
+            return 1;
+    for (long long i = 0; i < nk; ++i)
+        if (kb[i] < 0 || kb[i] >= B || kt[i] < 0 || kt[i] >= L || kg[i] < 0 || kg[i] >= H_kv)
+            return 1;
+    if (pos) {
+        std::vector<char> seen(L, 0);
+        for (long long t = 0; t < L; ++t) {
+            if (pos[t] < 0 || pos[t] >= L || seen[pos[t]]) return 1;
+            seen[pos[t]] = 1;
+        }
+    }
+    const int group = H_q / H_kv;
+    auto position = [&](long long t) { return pos ? pos[t] : t; };
+    auto visible = [&](int b, long long t, long long j) {
+        const long long kp = position(j);
+        return (!causal || kp <= position(t)) && kp >= (lo ? lo[(long long)b * L + t] : 0);
+    };
+    auto qrow = [&](const double* x, int b, long long t, int h) {
+        return x + (((long long)b * L + t) * H_q + h) * D;
+    };
+    auto krow = [&](const double* x, int b, long long t, int g) {
+        return x + (((long long)b * L + t) * H_kv + g) * D;
+    };
+    auto dot = [&](const double* a, const double* c) {
+        double r = 0.0;
+        for (int d = 0; d < D; ++d) r += a[d] * c[d];
+        return r;
+    };
+    // pass 1: which rows need lse and Delta, then compute them (lse_i and O_i by the
+    // definition, Delta_i = dO_i . O_i)
+    const long long n_rows = (long long)B * H_q * L;  // row index ((b * H_q + h) * L + t)
+    std::vector<char> need(n_rows, 0);
+    std::vector<char> whole_seq((size_t)B * H_q, 0);
+    for (long long i = 0; i < nk; ++i)
+        for (int h = kg[i] * group; h < (kg[i] + 1) * group; ++h)
+            whole_seq[(size_t)kb[i] * H_q + h] = 1;
+    for (long long r = 0; r < n_rows; ++r)
+        if (whole_seq[(size_t)(r / L)]) need[r] = 1;
+    for (long long i = 0; i < nq; ++i) need[((long long)qb[i] * H_q + qh[i]) * L + qt[i]] = 1;
+    std::vector<long long> rows;
+    for (long long r = 0; r < n_rows; ++r)
+        if (need[r]) rows.push_back(r);
+    std::vector<double> lse(n_rows, NEG_INF), delta(n_rows, 0.0);
+    parallel_for((long long)rows.size(), nthreads, [&](long long ri) {
+        thread_local std::vector<double> s, o;
+        const long long row = rows[(size_t)ri];
+        const long long t = row % L;
+        const int h = (int)((row / L) % H_q), b = (int)(row / L / H_q), g = h / group;
+        o.assign(D, 0.0);
+        double l;
+        attend_one(qrow(q, b, t, h), krow(k, b, 0, g), krow(v, b, 0, g), (long long)H_kv * D, 0,
+                   L, D, scale, [&](long long j) { return visible(b, t, j); }, s, o.data(), &l);
+        lse[row] = l;
+        delta[row] = dot(qrow(dout, b, t, h), o.data());
+    });
+    // P_ij and dS_ij of one (query row, key) pair
+    auto p_ds = [&](long long row, int b, long long t, int h, long long j, double* p,
+                    double* ds) {
+        const int g = h / group;
+        *p = std::exp(scale * dot(qrow(q, b, t, h), krow(k, b, j, g)) - lse[row]);
+        *ds = *p * (dot(qrow(dout, b, t, h), krow(v, b, j, g)) - delta[row]);
+    };
+    // pass 2: dQ of the sampled query rows
+    parallel_for(nq, nthreads, [&](long long i) {
+        const int b = qb[i], h = qh[i], g = h / group;
+        const long long t = qt[i], row = ((long long)b * H_q + h) * L + t;
+        double* dqv = dq_rows + i * D;
+        for (int d = 0; d < D; ++d) dqv[d] = 0.0;
+        for (long long j = 0; j < L; ++j) {
+            if (!visible(b, t, j)) continue;
+            double p, ds;
+            p_ds(row, b, t, h, j, &p, &ds);
+            const double* kj = krow(k, b, j, g);
+            for (int d = 0; d < D; ++d) dqv[d] += scale * ds * kj[d];
+        }
+    });
+    // pass 3: dK, dV of the sampled key rows, over every query head of the group and every
+    // query row that sees the key
+    parallel_for(nk, nthreads, [&](long long i) {
+        const int b = kb[i], g = kg[i];
+        const long long j = kt[i];
+        double* dkv = dk_rows + i * D;
+        double* dvv = dv_rows + i * D;
+        for (int d = 0; d < D; ++d) dkv[d] = dvv[d] = 0.0;
+        for (int h = g * group; h < (g + 1) * group; ++h)
+            for (long long t = 0; t < L; ++t) {
+                if (!visible(b, t, j)) continue;
+                const long long row = ((long long)b * H_q + h) * L + t;
+                double p, ds;
+                p_ds(row, b, t, h, j, &p, &ds);
+                const double* qv = qrow(q, b, t, h);
+                const double* dov = qrow(dout, b, t, h);
+                for (int d = 0; d < D; ++d) {
+                    dkv[d] += scale * ds * qv[d];
+                    dvv[d] += p * dov[d];
+                }
+            }
+    });
+    return 0;
+}
+
 // The zigzag layout (named beside the plain ring in [ULYSSES], introduction; the layout
 // is a reading): the sequence of P*Lc tokens (Lc even) is cut into 2P segments of
 // h = Lc/2 tokens and rank i holds segment i followed by segment 2P-1-i, so that under a

@@ -25,21 +25,34 @@ def rnd(shape, seed, scale=1.0):
     return np.random.default_rng(seed).standard_normal(shape) * scale
 
 
-def exact_lse(q, k, scale, causal):
-    """The log-sum-exp of every query row by its definition with exactly rounded sums
-    (math.fsum for the dot products and for the sum of exponentials)."""
-    B, L, H_q, D = q.shape
+def exact_attention(q, k, v, scale, causal):
+    """Attention of every query row by its definition with exactly rounded sums (math.fsum
+    for the dot products, for the sum of exponentials and for each output element's
+    weighted sum of V): O [B,L,H_q,D] and LSE [B,H_q,L] to within a few ulps of the
+    real values."""
+    B, L, H_q, _ = q.shape
+    D = v.shape[3]
     rep = H_q // k.shape[2]
-    out = np.empty((B, H_q, L))
+    out = np.empty((B, L, H_q, D))
+    lse = np.empty((B, H_q, L))
     for b in range(B):
         for h in range(H_q):
-            kh = k[b, :, h // rep]
+            kh, vh = k[b, :, h // rep], v[b, :, h // rep]
             for t in range(L):
                 n = t + 1 if causal else L
                 s = [scale * math.fsum(q[b, t, h] * kh[j]) for j in range(n)]
                 m = max(s)
-                out[b, h, t] = m + math.log(math.fsum(math.exp(x - m) for x in s))
-    return out
+                l = m + math.log(math.fsum(math.exp(x - m) for x in s))
+                w = [math.exp(x - l) for x in s]
+                lse[b, h, t] = l
+                for d in range(D):
+                    out[b, t, h, d] = math.fsum(w[j] * vh[j, d] for j in range(n))
+    return out, lse
+
+
+def exact_lse(q, k, scale, causal):
+    """The log-sum-exp of every query row by its definition with exactly rounded sums."""
+    return exact_attention(q, k, np.zeros(k.shape[:3] + (1,)), scale, causal)[1]
 
 
 def torch_sdpa(q, k, v, scale, causal):
@@ -78,14 +91,21 @@ def test_golden_three_keys(oracle_mod):
     (1, 37, 2, 2, 8, False), (2, 64, 4, 2, 16, True), (1, 50, 6, 3, 32, True),
     (1, 129, 8, 1, 4, False), (1, 33, 4, 4, 64, True)])
 def test_plain_matches_torch_sdpa_fp64(oracle_mod, B, L, H_q, H_kv, D, causal):
+    """O and LSE against the definition with exactly rounded sums at 1e-12, and O against
+    the float64 library routine as a second, independent implementation.  The library
+    comparison is held to 1e-9: torch's float64 CPU path was once seen 6.8e-10 off the
+    exact value, a fault of the library, not of the oracle, which the exact reference
+    bounds at 1e-12."""
     q = rnd((B, L, H_q, D), 1, 2.0)
     k = rnd((B, L, H_kv, D), 2)
     v = rnd((B, L, H_kv, D), 3)
     scale = 1.0 / math.sqrt(D)
     out, lse = oracle_mod.attention(q, k, v, scale, causal)
-    ref_o, ref_l = torch_sdpa(q, k, v, scale, causal)
-    np.testing.assert_allclose(out, ref_o, rtol=0, atol=1e-12)
-    np.testing.assert_allclose(lse, ref_l, rtol=0, atol=1e-12)
+    ex_o, ex_l = exact_attention(q, k, v, scale, causal)
+    np.testing.assert_allclose(out, ex_o, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, ex_l, rtol=0, atol=1e-12)
+    ref_o, _ = torch_sdpa(q, k, v, scale, causal)
+    np.testing.assert_allclose(out, ref_o, rtol=0, atol=1e-9)
 
 
 # ---------------------------------------------------------------- closed forms
@@ -573,3 +593,100 @@ def test_backward_matches_finite_differences(oracle_mod):
             ma = [xm if a is x else a for a in args]
             fd = (loss(*pa) - loss(*ma)) / (2 * eps)
             assert abs(fd - g[idx]) < 1e-7, (name, idx, fd, g[idx])
+
+
+# ---------------------------------------------------------------- backward on sampled rows
+def _torch_grads_masked(q, k, v, dout, scale, visible):
+    """float64 library gradients of attention under an explicit boolean mask
+    visible [B, L_query, L_key] (True = attended)."""
+    tq, tk, tv = (torch.from_numpy(x).permute(0, 2, 1, 3).clone().requires_grad_(True)
+                  for x in (q, k, v))
+    mask = torch.from_numpy(visible)[:, None]
+    out = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask,
+                                                           scale=scale, enable_gqa=True)
+    out.backward(torch.from_numpy(dout).permute(0, 2, 1, 3))
+    return [t.grad.permute(0, 2, 1, 3).numpy() for t in (tq, tk, tv)]
+
+
+def _visible(B, L, causal, pos, lo):
+    p = np.arange(L) if pos is None else np.asarray(pos)
+    low = np.zeros((B, L), np.int64) if lo is None else np.asarray(lo)
+    vis = np.ones((B, L, L), bool)
+    if causal:
+        vis &= p[None, None, :] <= p[None, :, None]
+    vis &= p[None, None, :] >= low[:, :, None]
+    return vis
+
+
+def _sample(B, L, H, n, seed):
+    g = np.random.default_rng(seed)
+    return (g.integers(0, B, n), g.integers(0, L, n), g.integers(0, H, n))
+
+
+@pytest.mark.parametrize("layout", ["contiguous", "noncausal", "zigzag", "permuted", "packed"])
+def test_backward_rows_match_torch_autograd_masked(oracle_mod, layout):
+    """dQ, dK, dV of sampled rows against float64 library autograd under the explicit mask
+    that the positions and lower bounds define: contiguous causal and non-causal, the
+    zigzag layout (P = 3, Lc = 10), an arbitrary permutation of positions, and packed
+    samples (GQA 4:2, B = 2)."""
+    B, P, Lc, H_q, H_kv, D = 2, 3, 10, 4, 2, 8
+    L = P * Lc
+    q, k, v = rnd((B, L, H_q, D), 120, 1.5), rnd((B, L, H_kv, D), 121), rnd((B, L, H_kv, D), 122)
+    dout = rnd((B, L, H_q, D), 123)
+    causal, pos, lo = layout != "noncausal", None, None
+    if layout == "zigzag":
+        pos = oracle_mod.zigzag_positions(P, Lc)
+    elif layout == "permuted":
+        pos = np.random.default_rng(5).permutation(L)
+    elif layout == "packed":
+        pid = np.stack([_pid_from_lengths([1, 9, 4, 16]), _pid_from_lengths([30])])
+        lo = oracle_mod.packed_lower_bounds(pid)
+    rq, rk, rv = _torch_grads_masked(q, k, v, dout, 0.45, _visible(B, L, causal, pos, lo))
+    qr, kr = _sample(B, L, H_q, 40, 7), _sample(B, L, H_kv, 30, 8)
+    dq, dk, dv = oracle_mod.attention_backward_rows(q, k, v, dout, 0.45, causal, qr, kr,
+                                                    positions=pos, lower_bounds=lo)
+    np.testing.assert_allclose(dq, rq[qr[0], qr[1], qr[2]], atol=1e-12)
+    np.testing.assert_allclose(dk, rk[kr[0], kr[1], kr[2]], atol=1e-12)
+    np.testing.assert_allclose(dv, rv[kr[0], kr[1], kr[2]], atol=1e-12)
+
+
+def test_backward_rows_equal_every_row_backward(oracle_mod):
+    """Every row sampled: the same numbers as the full backward (same formulas, same order
+    of summation), causal GQA."""
+    B, L, H_q, H_kv, D = 1, 23, 4, 1, 8
+    q, k, v = rnd((B, L, H_q, D), 124), rnd((B, L, H_kv, D), 125), rnd((B, L, H_kv, D), 126)
+    dout = rnd((B, L, H_q, D), 127)
+    full = oracle_mod.attention_backward(q, k, v, dout, 0.3, True)
+    qr = [a.ravel() for a in np.meshgrid(np.arange(B), np.arange(L), np.arange(H_q), indexing="ij")]
+    kr = [a.ravel() for a in np.meshgrid(np.arange(B), np.arange(L), np.arange(H_kv), indexing="ij")]
+    dq, dk, dv = oracle_mod.attention_backward_rows(q, k, v, dout, 0.3, True, qr, kr)
+    np.testing.assert_allclose(dq, full[0][qr[0], qr[1], qr[2]], atol=1e-13)
+    np.testing.assert_allclose(dk, full[1][kr[0], kr[1], kr[2]], atol=1e-13)
+    np.testing.assert_allclose(dv, full[2][kr[0], kr[1], kr[2]], atol=1e-13)
+
+
+def test_backward_rows_closed_forms(oracle_mod):
+    """One-token packed samples: each query sees only its own key, P = 1, so dQ = dK = 0 and
+    dV of key t is the sum of dO over the query heads of its group."""
+    B, L, H_q, H_kv, D = 1, 12, 4, 2, 8
+    q, k, v = rnd((B, L, H_q, D), 128), rnd((B, L, H_kv, D), 129), rnd((B, L, H_kv, D), 130)
+    dout = rnd((B, L, H_q, D), 131)
+    lo = np.arange(L)[None].astype(np.int64)
+    qr, kr = _sample(B, L, H_q, 10, 9), _sample(B, L, H_kv, 10, 10)
+    dq, dk, dv = oracle_mod.attention_backward_rows(q, k, v, dout, 0.7, True, qr, kr,
+                                                    lower_bounds=lo)
+    np.testing.assert_allclose(dq, 0.0, atol=1e-14)
+    np.testing.assert_allclose(dk, 0.0, atol=1e-14)
+    want = dout[kr[0], kr[1], 2 * kr[2]] + dout[kr[0], kr[1], 2 * kr[2] + 1]
+    np.testing.assert_allclose(dv, want, atol=1e-14)
+
+
+def test_backward_rows_invalid_arguments(oracle_mod):
+    z = np.zeros((1, 4, 2, 8))
+    with pytest.raises(ValueError):
+        oracle_mod.attention_backward_rows(z, z, z, z, 1.0, True, ([0], [4], [0]), ([], [], []))
+    with pytest.raises(ValueError):
+        oracle_mod.attention_backward_rows(z, z, z, z, 1.0, True, ([], [], []), ([0], [0], [2]))
+    with pytest.raises(ValueError):
+        oracle_mod.attention_backward_rows(z, z, z, z, 1.0, True, ([0], [0], [0]), ([], [], []),
+                                           positions=[0, 1, 1, 3])

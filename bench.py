@@ -16,7 +16,11 @@ the steps (max over ranks), in TFLOP/s.  With --gpus N every rank runs its own r
                   [--workload ulysses_e2e|ulysses_32k|usp_e2e|long_128k|long_128k_zigzag|long_128k_packed|
                               long_128k_bwd|long_128k_bwd_zigzag|long_128k_bwd_packed|
                               llama8b_32k_bwd|
-                              llama8b_32k|small_4k]
+                              llama8b_32k|small_4k|merge_128k]
+
+merge_128k times the log-sum-exp merge alone (ra_lse_merge, B=1, H=8, L=131072, D=128,
+fp32): one step = one merge of two partials, reported in GB/s of 3*D*4 + 12 bytes per row
+against the measured HBM copy rate.
 """
 from __future__ import annotations
 
@@ -69,6 +73,7 @@ def workloads():
         "llama8b_32k": ("attn", synth.LLAMA8B_GQA),
         "llama8b_32k_bwd": ("attn_bwd", synth.LLAMA8B_GQA),
         "small_4k": ("attn", synth.SMALL_BF16),
+        "merge_128k": ("merge", synth.MERGE_128K),
     }
 
 
@@ -188,7 +193,24 @@ class Path:
         # shard layout of the plain attention workloads (zigzag: rank i holds segments i and
         # 2P-1-i of 2P segments of Lc/2 tokens)
         self.layout = "zigzag" if kind in ("attn_zigzag", "attn_bwd_zigzag") else "contiguous"
-        if kind == "ulysses":
+        if kind == "merge":
+            self.a = w
+            # two partials with LSE ~ 4 N(0,1), drawn on the device; each step merges b into
+            # a in place (a valid merge every time: the LSEs only grow)
+            g = torch.Generator(device=device)
+            g.manual_seed(w.seed)
+            shape_o, shape_l = (w.B, w.L, w.H, w.D), (w.B, w.H, w.L)
+            self.oa = torch.randn(shape_o, generator=g, device=device)
+            self.la = 4.0 * torch.randn(shape_l, generator=g, device=device)
+            self.ob = torch.randn(shape_o, generator=g, device=device)
+            self.lb = 4.0 * torch.randn(shape_l, generator=g, device=device)
+            self.launches_per_step = 1
+            self.bytes = w.bytes()
+            self.flops = 0.0
+            self.permute_bytes = 0
+            self.in_bytes = sum(t.numel() * 4 for t in (self.oa, self.la, self.ob, self.lb))
+            self.out_bytes = (self.oa.numel() + self.la.numel()) * 4
+        elif kind == "ulysses":
             a = w.attn()
             self.a = a
             self.q, self.k, self.v = synth.ulysses_inputs(w, device=device)
@@ -246,7 +268,11 @@ class Path:
         """One pass of the path.  ev: optional dict of CUDA event pairs per stage."""
         ra = self.ra
         rec = (lambda name, i: ev[name][i].record()) if ev is not None else (lambda *_: None)
-        if self.kind == "ulysses":
+        if self.kind == "merge":
+            rec("attn", 0)
+            ra.ra_lse_merge(self.oa, self.la, self.ob, self.lb)
+            rec("attn", 1)
+        elif self.kind == "ulysses":
             w, a = self.w, self.a
             rec("permute_in", 0)
             ra.ra_ulysses_seq2head(self.q, w.H_q, out=self.qh, groups=w.G)
@@ -275,7 +301,15 @@ class Path:
             rec("attn", 1)
 
     def result(self):
+        if self.kind == "merge":
+            return self.oa
         return self.o_seq if self.kind == "ulysses" else self.o
+
+    def inputs(self):
+        """The step's input tensors (what the end-to-end leg uploads every step)."""
+        if self.kind == "merge":
+            return (self.oa, self.la, self.ob, self.lb)
+        return (self.q, self.k, self.v)
 
 
 def time_region(path, steps, torch, dist, ev_stages):
@@ -318,7 +352,7 @@ def e2e_region(paths, steps, torch, dist, device):
     comp = torch.cuda.current_stream()
     up = torch.cuda.Stream(device=device)
     down = torch.cuda.Stream(device=device)
-    host_in = [t.cpu().pin_memory() for t in (paths[0].q, paths[0].k, paths[0].v)]
+    host_in = [t.cpu().pin_memory() for t in paths[0].inputs()]
     res = paths[0].result()
     host_out = [torch.empty(res.shape, dtype=res.dtype, pin_memory=True) for _ in range(2)]
     ev = lambda: [torch.cuda.Event() for _ in range(2)]
@@ -331,7 +365,7 @@ def e2e_region(paths, steps, torch, dist, device):
         with torch.cuda.stream(up):
             if i >= 2:
                 up.wait_event(comp_done[s])  # step i-2 has finished reading set s
-            for h, d in zip(host_in, (paths[s].q, paths[s].k, paths[s].v)):
+            for h, d in zip(host_in, paths[s].inputs()):
                 d.copy_(h, non_blocking=True)
             up_done[s].record(up)
 
@@ -464,6 +498,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     kind, w = workloads()[args.workload]
     w_attn = w.attn() if kind == "ulysses" else w
+    if kind == "merge":
+        return merge_main(args, w)
 
     if args.impl == "reference":
         return reference_arm(args, kind, w, w_attn, rank, world)
@@ -543,11 +579,12 @@ def main():
         out["e2e_note"] = "not measured for backward workloads"
     elif not args.no_e2e:
         path2 = Path(kind, w, device)  # second buffer set for the pipelined end-to-end leg
-        e2e_ms = e2e_region([path, path2], max(3, min(args.steps, 6)), torch, dist, device)
+        e2e_ms = e2e_region([path, path2], args.steps, torch, dist, device)
         del path2
         out["e2e"] = {"value": round(path.flops * world / (e2e_ms * 1e-3) / 1e12, 2),
                       "unit": UNIT, "h2d_bytes_per_step": path.in_bytes,
                       "d2h_bytes_per_step": path.out_bytes, "ms_per_step": round(e2e_ms, 3),
+                      "steps": args.steps,
                       "pipelined": "step i+1 inputs up and step i output down on two copy "
                                    "streams, overlapping compute; all copies timed"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -561,6 +598,123 @@ def main():
                       f"(D={w_attn.D}), fp64 oracle, {dt:.1f} s")
         out["cpu_baseline"] = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle",
                                "sample": sample}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def merge_sample(w, n_rows, seed=4244):
+    """A bounded sample of the merge workload for the oracle: n rows of two partials drawn
+    like the GPU inputs (O ~ N(0,1), LSE ~ 4 N(0,1))."""
+    import torch
+    g = torch.Generator().manual_seed(seed)
+    oa = torch.randn(1, n_rows, 1, w.D, generator=g).double().numpy()
+    ob = torch.randn(1, n_rows, 1, w.D, generator=g).double().numpy()
+    la = (4.0 * torch.randn(1, 1, n_rows, generator=g)).double().numpy()
+    lb = (4.0 * torch.randn(1, 1, n_rows, generator=g)).double().numpy()
+    return oa, la, ob, lb, n_rows * (3 * w.D * 4 + 12)
+
+
+def run_oracle_merge(w, target_s=10.0):
+    """Time the oracle's merge as it stands on a bounded sample of rows; returns
+    (GB/s, rows, seconds, cores)."""
+    import oracle
+    oracle.build()
+    n = 1 << 14
+    while True:
+        oa, la, ob, lb, nbytes = merge_sample(w, n)
+        t0 = time.perf_counter()
+        oracle.lse_merge(oa, la, ob, lb)
+        dt = time.perf_counter() - t0
+        if dt >= target_s * 0.5 or n >= w.B * w.H * w.L:
+            return nbytes / dt / 1e9, n, dt, 1
+        n = min(w.B * w.H * w.L, n * 4)
+
+
+def merge_main(args, w):
+    """The merge workload: ra_lse_merge alone, GB/s against the HBM copy rate."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    config = {"workload": w.name, "rows": w.B * w.H * w.L, "heads": w.H, "seq_len": w.L,
+              "head_dim": w.D, "bytes_per_row": 3 * w.D * 4 + 12,
+              "l2": "inputs larger than L2 (126 MB); no flush between steps"}
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        per_step = args.ref_step_seconds or max(1.0, min(10.0, 120.0 / (args.steps + args.warmup)))
+        _, n, _, cores = run_oracle_merge(w, target_s=per_step)
+        oa, la, ob, lb, nbytes = merge_sample(w, n)
+        import oracle
+        times = []
+        for _ in range(args.steps):
+            t0 = time.perf_counter()
+            oracle.lse_merge(oa, la, ob, lb)
+            times.append(time.perf_counter() - t0)
+        sec = sum(times) / len(times)
+        value = nbytes / sec / 1e9
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": dict(config, parallelism="cpu-oracle"),
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{n} rows per step, fp64 oracle merge"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}), flush=True)
+        return
+    import torch
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    peaks, peaks_src = load_peaks()
+    path = Path("merge", w, device)
+    for _ in range(args.warmup):
+        path.step()
+    torch.cuda.synchronize()
+    for attempt in range(2):
+        with ClockSampler(local_rank) as clk:
+            total_ms, stage_ms = time_region(path, args.steps, torch, dist, ["attn"])
+        if not clk.rejected():
+            break
+    st = path.ra.ra_sync_status()
+    if st != 0:
+        raise RuntimeError(f"kernel status {st}: {path.ra.ra_last_error()}")
+    ms_step = max_over_ranks(total_ms / args.steps, dist, torch, device)
+    k_ms = max_over_ranks(statistics.mean(stage_ms["attn"]), dist, torch, device)
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    value = path.bytes * world / (ms_step * 1e-3) / 1e9
+    achieved = path.bytes / (k_ms * 1e-3) / 1e9
+    out = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+           "data": "synthetic", "config": dict(config, parallelism=f"replicas{world}"),
+           "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
+                        "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": None,
+                        "kernel": "lse_merge_kernel", "peak_source": f"{peaks_src} hbm_gbs",
+                        "frac_of_datasheet": round(achieved / DATASHEET_HBM_GBS, 4)},
+           "gpu_launches": path.launches_per_step * args.steps, "clocks": clk.summary()}
+    if not args.no_e2e:
+        path2 = Path("merge", w, device)
+        e2e_ms = e2e_region([path, path2], args.steps, torch, dist, device)
+        del path2
+        out["e2e"] = {"value": round(path.bytes * world / (e2e_ms * 1e-3) / 1e9, 1),
+                      "unit": "GB/s", "h2d_bytes_per_step": path.in_bytes,
+                      "d2h_bytes_per_step": path.out_bytes, "ms_per_step": round(e2e_ms, 3),
+                      "steps": args.steps}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, n, dt, cores = run_oracle_merge(w)
+        out["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                               "sample": f"{n} rows of two partials (D={w.D}), fp64 oracle "
+                                         f"merge, {dt:.1f} s"}
     if rank == 0:
         print(json.dumps(out), flush=True)
     if dist is not None:

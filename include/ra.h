@@ -246,14 +246,17 @@ RA_API ra_status ra_ring_attn_bwd_packed(const void* q, const void* const* k_chu
  * Arguments and results are those of ra_ring_attn_bwd, minus workspace.
  * Limit: B * H_q * P * Lc <= RA_BWD_STATIC_MAX_ROWS (2^21 rows, an 8 MiB fp32 array per
  *   device); larger requests return RA_ERR_INVALID before anything is enqueued.
- * Set-up: the first call on a device resolves the array's address
- *   (cudaGetSymbolAddress, which may load the library's device code) and the kernels'
- *   shared-memory attributes; make that first call before any stream capture.
+ * Set-up: every call looks the array's address up in the context current at the call
+ *   (cudaGetSymbolAddress; nothing is cached, so after cudaDeviceReset or any other
+ *   teardown and re-creation of the context the next call finds the array in the new
+ *   context).  The first call in a context may load the library's device code and sets
+ *   the kernels' shared-memory attributes; make that first call before any stream
+ *   capture.
  * Concurrency: the array is shared by all calls on a device.  Calls that overlap in time
  *   (on different streams, or from host threads without ordering between them) race on
  *   it; calls ordered on one stream do not.  Nothing in it needs to start at zero.
  * Errors: those of ra_ring_attn_bwd; RA_ERR_INVALID when the size limit is exceeded;
- *   RA_ERR_CUDA if the current device or the array's address cannot be obtained.
+ *   RA_ERR_CUDA if the array's address cannot be obtained in the current context.
  */
 #define RA_BWD_STATIC_MAX_ROWS (1 << 21)
 RA_API ra_status ra_ring_attn_bwd_static(const void* q, const void* const* k_chunks,

@@ -1,15 +1,16 @@
 // bwd_static.cu -- ra_ring_attn_bwd_static: the backward pass with its Delta scratch in a
 // fixed file-scope device array instead of a caller-provided workspace, so that a call makes
-// no device allocation of any kind.  The array's address is resolved once per device with
-// cudaGetSymbolAddress; every later call only reads the cached pointer and forwards to
-// ra_ring_attn_bwd, whose validation and kernels are used unchanged.
+// no device allocation of any kind.  Every call looks the array's address up in the current
+// context with cudaGetSymbolAddress (a host-side lookup once the module is loaded; nothing
+// is cached, so a context torn down and made again -- cudaDeviceReset -- gives the new
+// module's address, never a stale one) and forwards to ra_ring_attn_bwd, whose validation
+// and kernels are used unchanged.
 //
 // Nothing in the scratch has to start at zero: the Delta kernel writes every row that the
 // dQ and dK/dV kernels read, earlier on the same stream.  The one array is shared by every
 // call on a device, so calls that overlap in time (different streams, or different host
 // threads without ordering) race on it.
 #include <cuda_runtime.h>
-#include <mutex>
 #include <string>
 #include "ra_internal.h"
 #include "../../include/ra.h"
@@ -17,12 +18,8 @@
 namespace {
 
 constexpr long long kMaxRows = RA_BWD_STATIC_MAX_ROWS;
-constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) float g_bwd_scratch[RA_BWD_STATIC_MAX_ROWS];
-
-std::mutex g_mu;
-float* g_addr[kMaxDevices] = {};
 
 // B * H_q * P * Lc, or -1 once the running product passes kMaxRows (each factor is >= 1
 // and < 2^31, so no intermediate product exceeds 2^52).
@@ -50,28 +47,14 @@ extern "C" ra_status ra_ring_attn_bwd_static(
             "B*H_q*P*Lc exceeds the static backward scratch (RA_BWD_STATIC_MAX_ROWS = " +
                 std::to_string(kMaxRows) + " rows, " + std::to_string(kMaxRows * 4 >> 20) +
                 " MiB); use ra_ring_attn_bwd with a caller-provided workspace");
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess)
+    // the address in the context that is current now, looked up on every call
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_bwd_scratch);
+    if (e != cudaSuccess || !p)
         return (ra_status)ra::set_last_error(
-            RA_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorName(e));
-    if (dev < 0 || dev >= kMaxDevices)
-        return (ra_status)ra::set_last_error(RA_ERR_UNSUPPORTED,
-                                             "device ordinal beyond the static scratch table");
-    float* scratch;
-    {
-        std::lock_guard<std::mutex> lock(g_mu);
-        if (!g_addr[dev]) {
-            void* p = nullptr;
-            e = cudaGetSymbolAddress(&p, g_bwd_scratch);
-            if (e != cudaSuccess || !p)
-                return (ra_status)ra::set_last_error(
-                    RA_ERR_CUDA, std::string("cudaGetSymbolAddress of the backward scratch: ") +
-                                     cudaGetErrorName(e));
-            g_addr[dev] = static_cast<float*>(p);
-        }
-        scratch = g_addr[dev];
-    }
+            RA_ERR_CUDA, std::string("cudaGetSymbolAddress of the backward scratch: ") +
+                             cudaGetErrorName(e));
+    float* scratch = static_cast<float*>(p);
     return ra_ring_attn_bwd(q, k_chunks, v_chunks, out, lse, dout, P, B, H_q, H_kv, Lc, D,
                             q_bstride, kv_bstride, scale, causal, dq, dk_chunks, dv_chunks,
                             scratch, stream);

@@ -93,6 +93,21 @@ class UlyssesWorkload:
         return (q + kv + o) * es
 
 
+@dataclass(frozen=True)
+class MergeWorkload:
+    """Two partial attention results (O [B,L,H,D], LSE [B,H,L], fp32) merged into one."""
+    name: str
+    B: int
+    H: int
+    L: int
+    D: int
+    seed: int = 0
+
+    def bytes(self) -> int:
+        """Bytes a merge must move: read O_a, O_b and both LSEs, write O_a and LSE_a."""
+        return self.B * self.H * self.L * (3 * self.D * 4 + 12)
+
+
 # The workloads, named by what they are.
 TINY_FP32 = AttnWorkload("tiny_fp32_L128", B=1, H_q=2, H_kv=2, D=32, P=2, Lc=64,
                          dtype=torch.float32, causal=False, seed=1001)
@@ -202,3 +217,4 @@ def sample_rows(B: int, H_q: int, L: int, n: int, seed: int, Lc: int | None = No
     eh = torch.randint(0, H_q, (len(extra_t),), generator=g)
     return (torch.cat([b, eb]).tolist(), torch.cat([t, extra_t]).tolist(),
             torch.cat([h, eh]).tolist())
+MERGE_128K = MergeWorkload("lse_merge_L131072_H8_D128", B=1, H=8, L=131072, D=128, seed=1007)

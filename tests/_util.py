@@ -40,3 +40,27 @@ def rows_oracle(oracle_mod, q, k_seq, v_seq, rows, scale, causal):
     qn = f64(q[torch.tensor(rb), torch.tensor(rt), torch.tensor(rh)])
     return oracle_mod.attention_rows(qn, rb, rt, rh, f64(k_seq), f64(v_seq), q.shape[2], scale,
                                      causal)
+
+
+# Backward bar: per gradient tensor, max|error| <= GRAD_REL * max|reference| + GRAD_ABS (the
+# gradients are sums of products of bf16-rounded operands accumulated in fp32; the floor
+# covers gradients that vanish analytically).
+GRAD_REL = 1e-2
+GRAD_ABS = 1e-4
+
+
+def check_grad(name: str, nm: str, got: np.ndarray, ref: np.ndarray) -> float:
+    """Assert the backward bar for one gradient tensor (or sampled rows of it) and print,
+    beside it, the worst elementwise relative error over the elements whose reference is
+    above 1e-2 of the largest, so that errors on small gradient elements are visible.
+    Returns that relative error."""
+    assert np.all(np.isfinite(got)), (name, nm)
+    err = np.abs(got - ref)
+    mx = float(np.abs(ref).max()) if ref.size else 0.0
+    e = float(err.max()) if err.size else 0.0
+    big = np.abs(ref) > 1e-2 * mx
+    rel = float((err[big] / np.abs(ref[big])).max()) if big.any() else 0.0
+    print(f"[parity] bwd {name} {nm}: max|err|={e:.3e} max|ref|={mx:.3e} "
+          f"ratio={e / max(mx, 1e-30):.2e} worst rel (|ref| > 1e-2 max)={rel:.2e}")
+    assert e <= GRAD_REL * mx + GRAD_ABS, (name, nm, e, mx)
+    return rel

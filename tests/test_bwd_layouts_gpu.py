@@ -21,13 +21,9 @@ import pytest
 import torch
 
 from sequence_parallelism_attn_b200 import synth
-from _util import chunks_to_seq, f64
+from _util import check_grad, chunks_to_seq, f64
 
 pytestmark = pytest.mark.gpu
-
-REL = 1e-2
-ABS_FLOOR = 1e-4
-
 
 @pytest.fixture(scope="module", autouse=True)
 def _short_waits(ra_lib):
@@ -48,12 +44,7 @@ def problem(name, B, H_q, H_kv, D, P, Lc, causal, q_mult=1.0):
 
 def compare(name, got, want):
     for nm, a, b in zip(("dq", "dk", "dv"), got, want):
-        a = f64(a) if isinstance(a, torch.Tensor) else a
-        assert np.all(np.isfinite(a)), nm
-        err, mx = float(np.abs(a - b).max()), float(np.abs(b).max())
-        print(f"[parity] bwd {name} {nm}: max|err|={err:.3e} max|ref|={mx:.3e} "
-              f"ratio={err / max(mx, 1e-30):.2e}")
-        assert err <= REL * mx + ABS_FLOOR, (name, nm, err, mx)
+        check_grad(name, nm, f64(a) if isinstance(a, torch.Tensor) else a, b)
 
 
 def gpu_grads(ra_lib, w, q, k, v, dout, **layout):

@@ -105,17 +105,24 @@ def test_usp_128k_sampled(ra_lib, oracle_mod):
     sequence-sharded output against plain attention over the whole sequence."""
     w = synth.ULYSSES_128K
     q, k, v = synth.ulysses_inputs(w)
-    out, _ = usp_forward(ra_lib, q.cuda(), k.cuda(), v.cuda(), 4, w.attn().scale, True)
+    G = 4
+    out, lse = usp_forward(ra_lib, q.cuda(), k.cuda(), v.cuda(), G, w.attn().scale, True)
     seq = lambda x: x.permute(1, 0, 2, 3, 4).reshape(w.B, w.P * w.Lc, x.shape[3], w.D)
     rb, rt, rh = synth.sample_rows(w.B, w.H_q, w.P * w.Lc, 1024, seed=w.seed + 3, Lc=w.Lc)
     rt = np.asarray(rt, np.int64)
     qs = seq(q)
     qn = f64(qs[torch.tensor(rb), torch.from_numpy(rt), torch.tensor(rh)])
-    want_o, _ = oracle_mod.attention_rows(qn, rb, rt, rh, f64(seq(k)), f64(seq(v)), w.H_q,
-                                          w.attn().scale, True)
+    want_o, want_l = oracle_mod.attention_rows(qn, rb, rt, rh, f64(seq(k)), f64(seq(v)),
+                                               w.H_q, w.attn().scale, True)
     o_seq = seq(out.cpu())
     got_o = f64(o_seq[torch.tensor(rb), torch.from_numpy(rt), torch.tensor(rh)])
-    eo = max_abs(got_o, want_o)
-    print(f"[parity] usp 128k (4 groups x 2 ring chunks, {len(rt)} rows): max|dO|={eo:.3e}")
-    assert eo <= 1e-2
-    assert torch.isfinite(out).all()
+    # LSE rows of head group g = h // (H_q / G) sit at [g * B + b, h % (H_q / G), t]
+    Hg = w.H_q // G
+    rbn, rhn = np.asarray(rb), np.asarray(rh)
+    got_l = f64(lse[torch.from_numpy((rhn // Hg) * w.B + rbn), torch.from_numpy(rhn % Hg),
+                    torch.from_numpy(rt)])
+    eo, el = max_abs(got_o, want_o), max_abs(got_l, want_l)
+    print(f"[parity] usp 128k (4 groups x 2 ring chunks, {len(rt)} rows): max|dO|={eo:.3e} "
+          f"max|dLSE|={el:.3e}")
+    assert eo <= 1e-2 and el <= 1e-3, (eo, el)
+    assert torch.isfinite(out).all() and torch.isfinite(lse).all()

@@ -2,8 +2,8 @@
 device array, so that a call allocates no device memory -- against ra_ring_attn_bwd with a
 caller-provided workspace.  Both run the same kernels, so two static calls in a row must
 give the existing entry point's gradients bit for bit; the second call must leave the
-device's free memory unchanged; sizes beyond RA_BWD_STATIC_MAX_ROWS are refused before
-anything is enqueued.  The pages have no counterpart to this entry point."""
+device's free memory and torch's allocated and reserved memory unchanged; sizes beyond
+RA_BWD_STATIC_MAX_ROWS are refused before anything is enqueued.  The pages have no counterpart to this entry point."""
 import zlib
 
 import pytest
@@ -29,18 +29,37 @@ def _static_call(ra, w, q, k, v, o, lse, dout):
     dq = torch.full((w.B, w.L, w.H_q, w.D), float("nan"), device="cuda")
     dk = torch.full(k.shape, float("nan"), device="cuda")
     dv = torch.full(k.shape, float("nan"), device="cuda")
+    call = lambda: ra.ra_ring_attn_bwd_static(
+        q.data_ptr(), [k[j].data_ptr() for j in range(w.P)],
+        [v[j].data_ptr() for j in range(w.P)], o.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+        w.P, w.B, w.H_q, w.H_kv, w.Lc, w.D, w.L * w.H_q * w.D, w.Lc * w.H_kv * w.D, w.scale,
+        True, dq.data_ptr(), [dk[j].data_ptr() for j in range(w.P)],
+        [dv[j].data_ptr() for j in range(w.P)], torch.cuda.current_stream().cuda_stream)
+    return (dq, dk, dv), _memory_around(ra, call)
+
+
+def _memory_around(ra, call):
+    """Run one static call; return (device free memory, torch allocated, torch reserved)
+    before and after it."""
     torch.cuda.synchronize()
-    free_before, _ = torch.cuda.mem_get_info()
-    ra.ra_ring_attn_bwd_static(q.data_ptr(), [k[j].data_ptr() for j in range(w.P)],
-                               [v[j].data_ptr() for j in range(w.P)], o.data_ptr(),
-                               lse.data_ptr(), dout.data_ptr(), w.P, w.B, w.H_q, w.H_kv, w.Lc,
-                               w.D, w.L * w.H_q * w.D, w.Lc * w.H_kv * w.D, w.scale, True,
-                               dq.data_ptr(), [dk[j].data_ptr() for j in range(w.P)],
-                               [dv[j].data_ptr() for j in range(w.P)],
-                               torch.cuda.current_stream().cuda_stream)
+    before = (torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated(),
+              torch.cuda.memory_reserved())
+    call()
     assert ra.ra_sync_status() == 0, ra.ra_last_error()
-    free_after, _ = torch.cuda.mem_get_info()
-    return (dq, dk, dv), free_before, free_after
+    after = (torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated(),
+             torch.cuda.memory_reserved())
+    return before, after
+
+
+def _assert_no_allocation(ra, w, q, k, v, o, lse, dout, mem):
+    """The call changed neither torch's allocated nor its reserved memory, nor the device's
+    free memory.  Free memory counts every process on the device, so on a difference the
+    measurement is taken once more before it counts against the library."""
+    before, after = mem
+    assert before[1:] == after[1:], (before, after)
+    if before[0] != after[0]:
+        _, (before, after) = _static_call(ra, w, q, k, v, o, lse, dout)
+    assert before == after, (before, after)
 
 
 def _two_calls_match(ra, name, B, H_q, H_kv, P, Lc):
@@ -48,12 +67,12 @@ def _two_calls_match(ra, name, B, H_q, H_kv, P, Lc):
     o, lse = ra.ring_attn_fwd(q, k, v, True, w.scale, out_dtype=torch.bfloat16)
     want = ra.ring_attn_bwd(q, k, v, o, lse, dout, True, w.scale)
     assert ra.ra_sync_status() == 0, ra.ra_last_error()
-    first, _, _ = _static_call(ra, w, q, k, v, o, lse, dout)
-    second, free_before, free_after = _static_call(ra, w, q, k, v, o, lse, dout)
+    first, _ = _static_call(ra, w, q, k, v, o, lse, dout)
+    second, mem = _static_call(ra, w, q, k, v, o, lse, dout)
     for nm, a, b, c in zip(("dq", "dk", "dv"), want, first, second):
         assert torch.equal(a, b), f"first static call differs in {nm}"
         assert torch.equal(a, c), f"second static call differs in {nm}"
-    assert free_after == free_before, (free_before, free_after)
+    _assert_no_allocation(ra, w, q, k, v, o, lse, dout, mem)
 
 
 @pytest.mark.gpu
@@ -67,6 +86,21 @@ def test_static_at_the_size_limit(ra_lib):
     """B * H_q * P * Lc exactly RA_BWD_STATIC_MAX_ROWS (2 x 16 heads x 65536 tokens)."""
     assert 2 * 16 * 8 * 8192 == MAX_ROWS
     _two_calls_match(ra_lib, "bwd_static_limit", 2, 16, 4, 8, 8192)
+
+
+@pytest.mark.gpu
+def test_static_padded_batch_strides(ra_lib):
+    """q and the K/V chunks as slices of larger NaN-filled buffers (batch strides above the
+    dense size, B = 2): the static entry gives the dense workspace call's gradients bit for
+    bit."""
+    from test_bwd_gpu import padded_call
+    w, q, k, v, dout = _problem("bwd_static_padded", 2, 4, 2, 3, 200)
+    o, lse = ra_lib.ring_attn_fwd(q, k, v, True, w.scale, out_dtype=torch.bfloat16)
+    want = ra_lib.ring_attn_bwd(q, k, v, o, lse, dout, True, w.scale)
+    got = padded_call(ra_lib, ra_lib.ra_ring_attn_bwd_static, w, q, k, v, o, lse, dout,
+                      ws=False)
+    for nm, a, b in zip(("dq", "dk", "dv"), want, got):
+        assert torch.equal(a, b), nm
 
 
 def test_static_rejects_sizes_beyond_the_limit():

@@ -312,6 +312,67 @@ class Path:
         return (self.q, self.k, self.v)
 
 
+class DistUlyssesPath:
+    """The Ulysses step across N GPUs, one process each, with real exchanges: this rank's
+    sequence shard of Q, K, V (L/N tokens, every head) -> seq->head all-to-all (pack
+    kernel, NCCL all-to-all, unpack) -> causal attention of its H_q/N query heads over the
+    whole sequence (the attention kernel over the workload's chunk count) -> head->seq
+    all-to-all of O.  The total problem is the one-GPU workload's (strong scaling)."""
+
+    def __init__(self, w, device, rank, world):
+        import torch
+        from sequence_parallelism_attn_b200 import dist as rd, ra
+        self.ra, self.rd, self.kind, self.w, self.dev = ra, rd, "ulysses_dist", w, device
+        L = w.P * w.Lc
+        if w.H_q % world or L % world or w.G != w.P:
+            raise ValueError(f"{w.name} does not split over {world} ranks")
+        self.world, self.Ls, self.L = world, L // world, L
+        self.H_kv_rep = math.lcm(w.H_kv, world)
+        g = torch.Generator(device=device)
+        g.manual_seed(w.seed + 7919 * rank)
+        draw = lambda h: torch.randn((w.B, self.Ls, h, w.D), generator=g,
+                                     device=device).to(w.dtype)
+        self.q, self.k, self.v = draw(w.H_q), draw(w.H_kv), draw(w.H_kv)
+        self.Hq_l, self.Hkv_l = w.H_q // world, self.H_kv_rep // world
+        self.chunks = w.P  # the attention walks the same chunk count as on one GPU
+        self.o = torch.empty((w.B, L, self.Hq_l, w.D), dtype=torch.bfloat16, device=device)
+        self.lse = torch.empty((w.B, self.Hq_l, L), dtype=torch.float32, device=device)
+        self.o_seq = torch.empty((w.B, self.Ls, w.H_q, w.D), dtype=w.dtype, device=device)
+        self.scale = w.D ** -0.5
+        self.flops = 4.0 * w.B * self.Hq_l * float(L) ** 2 * w.D / 2
+        self.launches_per_step = 3 + 1 + (1 if w.B == 1 else 2) + (3 if w.B > 1 else 0)
+        es = torch.tensor([], dtype=w.dtype).element_size()
+        part = (world - 1) / world
+        self.bytes_sent = int(es * w.B * self.Ls * w.D * part *
+                              (2 * w.H_q + 2 * self.H_kv_rep))
+        self.permute_bytes = 0
+        self.in_bytes = sum(t.numel() * t.element_size() for t in (self.q, self.k, self.v))
+        self.out_bytes = self.q.numel() * self.q.element_size()
+
+    def step(self, ev=None):
+        rd, w = self.rd, self.w
+        rec = (lambda name, i: ev[name][i].record()) if ev is not None else (lambda *_: None)
+        rec("permute_in", 0)
+        qh = rd.ulysses_seq2head_dist(self.q, w.H_q)
+        kh = rd.ulysses_seq2head_dist(self.k, self.H_kv_rep)
+        vh = rd.ulysses_seq2head_dist(self.v, self.H_kv_rep)
+        rec("permute_in", 1)
+        rec("attn", 0)
+        C, Lc = self.chunks, self.L // self.chunks
+        kv = lambda x: [x.view(w.B, C, Lc, self.Hkv_l, w.D)[:, j] for j in range(C)]
+        self.ra.ring_attn_fwd(qh, kv(kh), kv(vh), True, self.scale, out=self.o, lse=self.lse)
+        rec("attn", 1)
+        rec("permute_out", 0)
+        self.o_seq = rd.ulysses_head2seq_dist(self.o)
+        rec("permute_out", 1)
+
+    def result(self):
+        return self.o_seq
+
+    def inputs(self):
+        return (self.q, self.k, self.v)
+
+
 def time_region(path, steps, torch, dist, ev_stages):
     """Time exactly `steps` steps between barrier+synchronize; returns (ms_total, stage_ms)."""
     events = {k: [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
@@ -515,7 +576,11 @@ def main():
                                 device_id=device)
     peaks, peaks_src = load_peaks()
 
-    path = Path(kind, w, device)
+    if world > 1 and kind == "ulysses":
+        # N GPUs: the Ulysses layer with real all-to-alls between the ranks
+        path = DistUlyssesPath(w, device, rank, world)
+    else:
+        path = Path(kind, w, device)
     for _ in range(args.warmup):
         path.step()
     torch.cuda.synchronize()
@@ -532,18 +597,26 @@ def main():
     attn_ms = max_over_ranks(statistics.mean(stage_ms["attn"]), dist, torch, device)
     value = path.flops * world / (ms_step * 1e-3) / 1e12
     attn_tflops = path.flops / (attn_ms * 1e-3) / 1e12
+    dist_ulysses = path.kind == "ulysses_dist"
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic",
+        "higher_is_better": True, "scaling": "strong" if dist_ulysses else "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name + SUFFIX.get(kind, ""),
-                   "global_batch": w_attn.B * world, "seq_len": w_attn.L,
+                   "global_batch": w_attn.B * (1 if dist_ulysses else world),
+                   "seq_len": w_attn.L,
                    "heads_q": w_attn.H_q, "heads_kv": w_attn.H_kv, "head_dim": w_attn.D,
                    "virtual_ranks": w_attn.P, "chunk_len": w_attn.Lc, "causal": w_attn.causal,
-                   "parallelism": f"replicas{world}",
+                   "parallelism": f"ulysses{world}" if dist_ulysses else f"replicas{world}",
                    "l2": "inputs larger than L2 (126 MB); no flush between steps"},
     }
+    if dist_ulysses:
+        out["config"].update({"global_batch": w.B, "seq_len": path.L, "heads_q": w.H_q,
+                              "heads_kv": w.H_kv, "tokens_per_rank": path.Ls,
+                              "heads_q_per_rank": path.Hq_l, "heads_kv_per_rank": path.Hkv_l,
+                              "exchange": "NCCL all-to-all between the ranks, pack/unpack "
+                                          "kernels around it"})
     if kind == "ulysses":
         # Ulysses: P head groups; the ring x Ulysses hybrid: fewer, each with a ring
         out["config"]["head_groups"] = w.G
@@ -551,7 +624,9 @@ def main():
         out["config"]["packed_documents"] = path.n_docs
         out["config"]["document_lengths"] = "512..32768 tokens, log-uniform, seeded"
     sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-    traffic = attn_traffic(args.workload)
+    # DRAM bytes from the committed capture of the one-GPU launch (another launch shape
+    # when the heads are split over several GPUs)
+    traffic = None if dist_ulysses else attn_traffic(args.workload)
     out["roofline"] = {"bound": "tensor", "achieved": round(attn_tflops, 2),
                        "peak": sustained, "unit": "TFLOP/s",
                        "frac": round(attn_tflops / sustained, 4),
@@ -561,7 +636,14 @@ def main():
                        "peak_source": f"{peaks_src} bf16_tflops_sustained",
                        "frac_of_burst": round(attn_tflops / peaks.get("bf16_tflops", 1590.0), 4),
                        "frac_of_datasheet": round(attn_tflops / DATASHEET_BF16_TFLOPS, 4)}
-    if kind == "ulysses":
+    if dist_ulysses:
+        ex_ms = max_over_ranks(statistics.mean(
+            a + b for a, b in zip(stage_ms["permute_in"], stage_ms["permute_out"])),
+            dist, torch, device)
+        out["exchange"] = {"ms_per_step": round(ex_ms, 4),
+                           "bytes_sent_per_rank": path.bytes_sent,
+                           "gbs_per_rank": round(path.bytes_sent / (ex_ms * 1e-3) / 1e9, 1)}
+    elif kind == "ulysses":
         perm_ms = max_over_ranks(statistics.mean(
             a + b for a, b in zip(stage_ms["permute_in"], stage_ms["permute_out"])),
             dist, torch, device)
@@ -578,7 +660,8 @@ def main():
         out["e2e"] = None
         out["e2e_note"] = "not measured for backward workloads"
     elif not args.no_e2e:
-        path2 = Path(kind, w, device)  # second buffer set for the pipelined end-to-end leg
+        # second buffer set for the pipelined end-to-end leg
+        path2 = DistUlyssesPath(w, device, rank, world) if dist_ulysses else Path(kind, w, device)
         e2e_ms = e2e_region([path, path2], args.steps, torch, dist, device)
         del path2
         out["e2e"] = {"value": round(path.flops * world / (e2e_ms * 1e-3) / 1e12, 2),

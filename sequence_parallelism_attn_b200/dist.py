@@ -1,0 +1,212 @@
+"""The data plane across GPUs: the ring's K/V exchange and the Ulysses all-to-alls over
+torch.distributed (NCCL between GPUs, one process per GPU), with the library's kernels
+for every computation.
+
+Ring ("Как работает sequence parallelism в контексте LLM?", sections 3 and 5): rank i
+keeps its query chunk; at step s = 0 .. P-1 it holds K/V chunk j = (i - s) mod P and
+attends its queries to it while that chunk travels on to rank i + 1 and the next one
+arrives from rank i - 1 into a second buffer (P - 1 exchanges, each overlapped with one
+step's attention).  Each step's partial (O, LSE) is merged into the running result by
+ra_lse_merge.  Under the causal mask (global positions in rank order) chunk j < i is
+wholly visible, j == i is the diagonal, and j > i is skipped: no launch, although the
+chunk still travels on.
+
+Ulysses ("Метод контекстного параллелизма Ulysses"): seq->head is pack -> all-to-all ->
+unpack.  The pack is the library's grouped transform of this rank's tokens into P
+destination blocks of H_out / P heads (with the GQA copy), so each peer's slice is one
+contiguous block; the all-to-all swaps block r of every rank into rank r; the unpack puts
+the P received token blocks in source-rank order (a view when B = 1).  head->seq is the
+inverse.  No kernel reads another GPU's memory: every remote block lands in this GPU's
+own buffers through NCCL before a kernel touches it.
+
+Every rank takes the same collective steps in the same order.  A peer that leaves between
+steps ends the next exchange with an error (the process group's timeout bounds the wait),
+raised here as ExchangeError naming the step and the peers.
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+
+class ExchangeError(RuntimeError):
+    """An exchange with a peer failed (a peer left, or the process group timed out)."""
+
+
+def chunk_pair(i: int, j: int, causal: bool) -> str:
+    """How query chunk i sees K/V chunk j: "full", "diagonal" (causal inside the chunk) or
+    "skip" (every key after every query).  Non-causal: always "full"."""
+    if not causal:
+        return "full"
+    if j < i:
+        return "full"
+    return "diagonal" if j == i else "skip"
+
+
+def ring_schedule(rank: int, world: int) -> list[int]:
+    """The K/V chunk rank `rank` holds at each step: (rank - s) mod world, s = 0 .. world-1."""
+    return [(rank - s) % world for s in range(world)]
+
+
+class DeviceOps:
+    """The computations of the distributed path, each one library call."""
+
+    @staticmethod
+    def attend(q, k, v, causal_diagonal, scale, out, lse):
+        from . import ra
+        ra.ring_attn_fwd(q, [k], [v], causal_diagonal, scale, out=out, lse=lse)
+
+    @staticmethod
+    def merge(o_a, lse_a, o_b, lse_b):
+        from . import ra
+        ra.ra_lse_merge(o_a, lse_a, o_b, lse_b)
+
+    @staticmethod
+    def seq2head_pack(x, H_out, P):
+        """[B, Lc, H_in, D] -> [P, B, Lc, H_out / P, D]: block r = the heads of rank r."""
+        from . import ra
+        return ra.ra_ulysses_seq2head(x.unsqueeze(0), H_out, groups=P)
+
+    @staticmethod
+    def seq2head_unpack(recv):
+        """[P, B, Lc, Hl, D] (block s from rank s) -> [B, P * Lc, Hl, D]."""
+        from . import ra
+        P, B, Lc, Hl, D = recv.shape
+        if B == 1:
+            return recv.view(1, P * Lc, Hl, D)
+        return ra.ra_ulysses_seq2head(recv, Hl, groups=1).view(B, P * Lc, Hl, D)
+
+    @staticmethod
+    def head2seq_pack(y, P):
+        """[B, P * Lc, Hl, D] -> [P, B, Lc, Hl, D]: block s = the tokens of rank s."""
+        from . import ra
+        B, L, Hl, D = y.shape
+        if B == 1:
+            return y.view(P, 1, L // P, Hl, D)
+        return ra.ra_ulysses_head2seq(y.unsqueeze(0), P=P)
+
+    @staticmethod
+    def head2seq_unpack(recv):
+        """[P, B, Lc, Hl, D] (block r = rank r's heads) -> [B, Lc, P * Hl, D]."""
+        from . import ra
+        P, B, Lc, Hl, D = recv.shape
+        return ra.ra_ulysses_head2seq(recv, P=1).view(B, Lc, P * Hl, D)
+
+
+def _group_info(group):
+    return dist.get_rank(group), dist.get_world_size(group)
+
+
+def _peer(group, r):
+    """Global rank of group rank r (P2P ops address global ranks)."""
+    return r if group is None else dist.get_global_rank(group, r)
+
+
+def _wait(works, what):
+    try:
+        for w in works:
+            w.wait()
+    except Exception as e:  # a peer left or the process group timed out
+        raise ExchangeError(f"{what}: {e}") from e
+
+
+class RingAccumulator:
+    """Rank i's running attention result over the K/V chunks it visits: the first visited
+    chunk writes (O, LSE) directly, every later one is attended into a partial and merged
+    in (ra_lse_merge); chunks wholly after the queries (causal) are skipped."""
+
+    def __init__(self, q, rank: int, causal: bool, scale: float | None = None, out=None,
+                 lse=None, ops=DeviceOps):
+        B, Lc, H_q, D = q.shape
+        self.q, self.rank, self.causal, self.ops = q, rank, causal, ops
+        self.scale = D ** -0.5 if scale is None else scale
+        dev = q.device
+        self.out = torch.empty((B, Lc, H_q, D), dtype=torch.float32, device=dev) \
+            if out is None else out
+        self.lse = torch.empty((B, H_q, Lc), dtype=torch.float32, device=dev) \
+            if lse is None else lse
+        self.part = None
+        self.visited = 0
+
+    def visit(self, j: int, k, v):
+        kind = chunk_pair(self.rank, j, self.causal)
+        if kind == "skip":
+            return
+        diag = kind == "diagonal"
+        if self.visited == 0:
+            self.ops.attend(self.q, k, v, diag, self.scale, self.out, self.lse)
+        else:
+            if self.part is None:
+                self.part = (torch.empty_like(self.out), torch.empty_like(self.lse))
+            self.ops.attend(self.q, k, v, diag, self.scale, *self.part)
+            self.ops.merge(self.out, self.lse, *self.part)
+        self.visited += 1
+
+
+def ring_attn_fwd_dist(q, k, v, causal: bool, scale: float | None = None, group=None,
+                       out=None, lse=None, ops=DeviceOps):
+    """Ring attention across the ranks of `group`: q [B, Lc, H_q, D] is this rank's query
+    chunk, k/v [B, Lc, H_kv, D] its K/V chunk (contiguous), rank i holding tokens
+    i*Lc .. i*Lc+Lc-1 of the sequence.  Returns this rank's (out [B, Lc, H_q, D] fp32,
+    lse [B, H_q, Lc] fp32), equal to attention of its queries over the whole sequence.
+    The chunk received during step s is sent on during step s + 1; two receive buffers
+    alternate, and a buffer is received into only after the step that read it has been
+    enqueued (NCCL's stream waits for it) and its own send has completed."""
+    rank, world = _group_info(group)
+    acc = RingAccumulator(q, rank, causal, scale, out, lse, ops)
+    bufs = [(torch.empty_like(k), torch.empty_like(v)) for _ in range(2)] if world > 1 else []
+    held = (k, v)
+    nxt_rank, prv_rank = _peer(group, (rank + 1) % world), _peer(group, (rank - 1) % world)
+    for s, j in enumerate(ring_schedule(rank, world)):
+        works = []
+        if s < world - 1:
+            nxt = bufs[s % 2]
+            p2p = [dist.P2POp(dist.isend, held[0], nxt_rank, group),
+                   dist.P2POp(dist.isend, held[1], nxt_rank, group),
+                   dist.P2POp(dist.irecv, nxt[0], prv_rank, group),
+                   dist.P2POp(dist.irecv, nxt[1], prv_rank, group)]
+            try:
+                works = dist.batch_isend_irecv(p2p)
+            except Exception as e:
+                raise ExchangeError(f"ring step {s}: posting the exchange with ranks "
+                                    f"{(rank + 1) % world} / {(rank - 1) % world}: {e}") from e
+        acc.visit(j, held[0], held[1])
+        if works:
+            _wait(works, f"ring step {s}: chunk from rank {(rank - 1) % world}")
+            held = nxt
+    return acc.out, acc.lse
+
+
+def _all_to_all(send, group, what):
+    recv = torch.empty_like(send)
+    try:
+        dist.all_to_all_single(recv, send, group=group)
+    except Exception as e:
+        raise ExchangeError(f"{what}: {e}") from e
+    return recv
+
+
+def ulysses_seq2head_dist(x, H_out: int | None = None, group=None, ops=DeviceOps):
+    """Ulysses seq->head across the ranks of `group`: x [B, Lc, H_in, D] is this rank's
+    sequence shard with every head; returns [B, P*Lc, H_out/P, D], this rank's head block
+    (heads [r*H_out/P, (r+1)*H_out/P) after the GQA copy to H_out heads) over the whole
+    sequence, tokens in source-rank order."""
+    rank, world = _group_info(group)
+    H_out = x.shape[2] if H_out is None else H_out
+    if H_out % world or H_out % x.shape[2]:
+        raise ValueError(f"{H_out} heads do not split over {world} ranks / copy {x.shape[2]}")
+    send = ops.seq2head_pack(x, H_out, world)
+    recv = _all_to_all(send, group, f"seq2head all-to-all on rank {rank}")
+    return ops.seq2head_unpack(recv)
+
+
+def ulysses_head2seq_dist(y, group=None, ops=DeviceOps):
+    """Ulysses head->seq across the ranks of `group`: y [B, P*Lc, Hl, D] is this rank's
+    head block over the whole sequence; returns [B, Lc, P*Hl, D], this rank's sequence
+    shard with every head."""
+    rank, world = _group_info(group)
+    if y.shape[1] % world:
+        raise ValueError(f"sequence of {y.shape[1]} tokens does not split over {world} ranks")
+    send = ops.head2seq_pack(y, world)
+    recv = _all_to_all(send, group, f"head2seq all-to-all on rank {rank}")
+    return ops.head2seq_unpack(recv)

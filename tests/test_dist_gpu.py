@@ -1,0 +1,111 @@
+"""The multi-GPU data plane's computations on one GPU: the ring's per-step attention and
+merge (RingAccumulator with the library's kernels) for P virtual ranks visiting the chunks
+in ring order, against the oracle's attention over the whole sequence; the Ulysses pack and
+unpack kernels around an all-to-all emulated on the device, bit for bit against the
+oracle's seq->head / head->seq; and the distributed functions themselves through a
+one-rank NCCL process group.  The exchanges between ranks are tested on CPU ranks
+(tests/test_dist_host.py).
+
+Sources: "Как работает sequence parallelism в контексте LLM?" sections 3 and 5; "Метод
+контекстного параллелизма Ulysses"."""
+import socket
+
+import numpy as np
+import pytest
+import torch
+
+from sequence_parallelism_attn_b200 import dist as rd
+from _util import TOL, f64, max_abs
+
+pytestmark = pytest.mark.gpu
+
+
+def _bits(t):
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy()
+    return t.view(torch.int32).numpy()
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("P", [1, 4])
+def test_ring_steps_equal_whole_sequence(ra_lib, oracle_mod, P, causal):
+    """Every virtual rank's accumulator over its ring steps (attention launches per held
+    chunk, merges by ra_lse_merge) equals attention of its queries over the whole sequence,
+    every row (B = 2, ragged chunks of 200 tokens, GQA 4:2, bf16)."""
+    B, Lc, H_q, H_kv, D = 2, 200, 4, 2, 128
+    g = torch.Generator().manual_seed(300 + P)
+    L = P * Lc
+    q = (torch.randn(B, L, H_q, D, generator=g) * 2).to(torch.bfloat16)
+    k = torch.randn(B, L, H_kv, D, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, L, H_kv, D, generator=g).to(torch.bfloat16)
+    scale = D ** -0.5
+    want_o, want_l = oracle_mod.attention(f64(q), f64(k), f64(v), scale, causal)
+    shard = lambda x, i: x[:, i * Lc:(i + 1) * Lc].contiguous().cuda()
+    for i in range(P):
+        acc = rd.RingAccumulator(shard(q, i), i, causal, scale)
+        for j in rd.ring_schedule(i, P):
+            acc.visit(j, shard(k, j), shard(v, j))
+        assert ra_lib.ra_sync_status() == 0, ra_lib.ra_last_error()
+        sl = slice(i * Lc, (i + 1) * Lc)
+        eo = max_abs(f64(acc.out), want_o[:, sl])
+        el = max_abs(f64(acc.lse), want_l[:, :, sl])
+        print(f"[parity] ring steps P={P} causal={causal} rank {i}: max|dO|={eo:.3e} "
+              f"max|dLSE|={el:.3e}")
+        assert eo <= TOL[torch.bfloat16][0] and el <= TOL[torch.bfloat16][1]
+
+
+@pytest.mark.parametrize("B,dtype", [(1, torch.bfloat16), (2, torch.bfloat16),
+                                     (2, torch.float32)])
+def test_ulysses_pack_unpack_bit_exact(ra_lib, oracle_mod, B, dtype):
+    """pack on every virtual rank, the all-to-all emulated on the device (block r of rank s
+    to rank r), unpack: each rank's result is its block of the oracle's seq->head, with the
+    GQA copy of 2 KV heads to 4; and head->seq likewise."""
+    P, Lc, H_kv, H_q, D = 4, 96, 2, 8, 128
+    g = torch.Generator().manual_seed(400 + B)
+    x = torch.randn(P, B, Lc, H_kv, D, generator=g).to(dtype)
+    H_out = int(np.lcm(H_kv, P))
+    sends = [rd.DeviceOps.seq2head_pack(x[s].cuda(), H_out, P) for s in range(P)]
+    want = oracle_mod.seq2head(_bits(x), H_out)
+    for r in range(P):
+        recv = torch.stack([sends[s][r] for s in range(P)])
+        y = rd.DeviceOps.seq2head_unpack(recv)
+        assert y.shape == (B, P * Lc, H_out // P, D)
+        assert np.array_equal(_bits(y), want[r])
+    h = torch.randn(P, B, P * Lc, H_q // P, D, generator=g).to(dtype)
+    sends = [rd.DeviceOps.head2seq_pack(h[r].cuda(), P) for r in range(P)]
+    want = oracle_mod.head2seq(_bits(h))
+    for s in range(P):
+        recv = torch.stack([sends[r][s] for r in range(P)])
+        z = rd.DeviceOps.head2seq_unpack(recv)
+        assert z.shape == (B, Lc, H_q, D)
+        assert np.array_equal(_bits(z), want[s])
+    assert ra_lib.ra_sync_status() == 0
+
+
+def test_distributed_functions_on_one_rank(ra_lib, oracle_mod):
+    """ring_attn_fwd_dist and the Ulysses functions through a one-rank NCCL process group
+    (the all-to-all moves one block to itself; the ring has one step)."""
+    import torch.distributed as dist
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0,
+                            world_size=1, device_id=torch.device("cuda", 0))
+    try:
+        B, Lc, H_q, H_kv, D = 1, 300, 4, 2, 128
+        g = torch.Generator().manual_seed(501)
+        q = torch.randn(B, Lc, H_q, D, generator=g).to(torch.bfloat16)
+        k = torch.randn(B, Lc, H_kv, D, generator=g).to(torch.bfloat16)
+        v = torch.randn(B, Lc, H_kv, D, generator=g).to(torch.bfloat16)
+        o, l = rd.ring_attn_fwd_dist(q.cuda(), k.cuda(), v.cuda(), True, D ** -0.5)
+        want_o, want_l = oracle_mod.attention(f64(q), f64(k), f64(v), D ** -0.5, True)
+        assert max_abs(f64(o), want_o) <= 1e-2 and max_abs(f64(l), want_l) <= 1e-3
+        y = rd.ulysses_seq2head_dist(k.cuda(), 2)
+        assert np.array_equal(_bits(y), oracle_mod.seq2head(_bits(k)[None], 2)[0])
+        z = rd.ulysses_head2seq_dist(y)
+        assert np.array_equal(_bits(z), _bits(k))
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()

@@ -1,0 +1,253 @@
+"""The multi-GPU data plane's exchange logic on CPU ranks (gloo, world sizes 2 and 4): the
+ring schedule and its double-buffered K/V exchange, ring attention across ranks equal to
+attention over the whole sequence, the Ulysses pack -> all-to-all -> unpack equal to the
+oracle's seq->head / head->seq bit for bit, and a rank that leaves between steps reported
+as an error rather than a hang.
+
+The computations are the oracle's here (no GPU on these ranks); on the GPU the same
+functions call the library's kernels (DeviceOps), whose pack / unpack and per-step
+attention + merge are checked against the oracle in tests/test_dist_gpu.py.
+
+Sources: "Как работает sequence parallelism в контексте LLM?" section 3 (rank i holds
+chunk (i - s) mod P at step s; P - 1 exchanges) and section 5 (merge of the partials);
+"Метод контекстного параллелизма Ulysses" (the all-to-all before and after attention)."""
+import os
+import queue
+import socket
+import time
+import traceback
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, fn, args, q):
+    import datetime
+    import sys
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    try:
+        dist.init_process_group("gloo", rank=rank, world_size=world,
+                                timeout=datetime.timedelta(seconds=20))
+        res = fn(rank, world, *args)
+        q.put((rank, "ok", res))
+        dist.destroy_process_group()
+    except BaseException as e:  # reported to the parent, which fails the test
+        q.put((rank, "error", f"{type(e).__name__}: {e}\n{traceback.format_exc()}"))
+
+
+def run_ranks(world, fn, *args, timeout=120):
+    """Run fn(rank, world, *args) on `world` gloo ranks (spawned processes); returns
+    {rank: (status, result)}."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, fn, args, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = {}
+    deadline = time.monotonic() + timeout
+    try:
+        # a rank that exits without reporting (a rank that leaves) sends nothing: collect
+        # until every rank has reported or exited
+        while len(out) < world and time.monotonic() < deadline:
+            try:
+                rank, status, res = q.get(timeout=1.0)
+                out[rank] = (status, res)
+            except queue.Empty:
+                if all(not p.is_alive() for p in procs) and q.empty():
+                    break
+    finally:
+        for p in procs:
+            p.join(timeout=30)
+            if p.is_alive():
+                p.kill()
+    return out
+
+
+class OracleOps:
+    """The oracle's arithmetic behind the data plane's compute hooks (CPU ranks only)."""
+
+    @staticmethod
+    def attend(q, k, v, causal_diagonal, scale, out, lse):
+        import oracle
+        o, l = oracle.attention(q.numpy(), k.numpy(), v.numpy(), scale, causal_diagonal)
+        out.copy_(torch.from_numpy(o))
+        lse.copy_(torch.from_numpy(l))
+
+    @staticmethod
+    def merge(o_a, lse_a, o_b, lse_b):
+        import oracle
+        o, l = oracle.lse_merge(o_a.numpy(), lse_a.numpy(), o_b.numpy(), lse_b.numpy())
+        o_a.copy_(torch.from_numpy(o))
+        lse_a.copy_(torch.from_numpy(l))
+
+    @staticmethod
+    def seq2head_pack(x, H_out, P):
+        import oracle
+        return torch.from_numpy(oracle.seq2head(x.numpy()[None], H_out, groups=P))
+
+    @staticmethod
+    def seq2head_unpack(recv):
+        import oracle
+        P, B, Lc, Hl, D = recv.shape
+        return torch.from_numpy(oracle.seq2head(recv.numpy(), Hl, groups=1)).view(
+            B, P * Lc, Hl, D)
+
+    @staticmethod
+    def head2seq_pack(y, P):
+        import oracle
+        return torch.from_numpy(oracle.head2seq(y.numpy()[None], P=P))
+
+    @staticmethod
+    def head2seq_unpack(recv):
+        import oracle
+        P, B, Lc, Hl, D = recv.shape
+        return torch.from_numpy(oracle.head2seq(recv.numpy(), P=1)).view(B, Lc, P * Hl, D)
+
+
+class RecordingOps(OracleOps):
+    """Records the first element of every chunk a rank attends to (each rank's K/V is
+    filled with its own rank index)."""
+    seen = []
+
+    @staticmethod
+    def attend(q, k, v, causal_diagonal, scale, out, lse):
+        RecordingOps.seen.append((int(k.flatten()[0].item()), int(v.flatten()[0].item()),
+                                  bool(causal_diagonal)))
+        out.zero_()
+        lse.fill_(0.0)
+
+    @staticmethod
+    def merge(o_a, lse_a, o_b, lse_b):
+        pass
+
+
+# ------------------------------------------------------------------ ring
+def _ring_holds(rank, world, causal):
+    from sequence_parallelism_attn_b200 import dist as rd
+    q = torch.zeros(1, 4, 2, 8, dtype=torch.float64)
+    k = torch.full((1, 4, 1, 8), float(rank), dtype=torch.float64)
+    v = torch.full((1, 4, 1, 8), float(100 + rank), dtype=torch.float64)
+    RecordingOps.seen = []
+    rd.ring_attn_fwd_dist(q, k, v, causal, 0.5, out=torch.empty(1, 4, 2, 8, dtype=torch.float64),
+                          lse=torch.empty(1, 2, 4, dtype=torch.float64), ops=RecordingOps)
+    return RecordingOps.seen
+
+
+@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("causal", [False, True])
+def test_ring_rank_holds_chunk_i_minus_s(world, causal):
+    """Step s of rank i attends to the chunk that rank (i - s) mod P started with; causal:
+    chunks after the rank's own are skipped, its own is the diagonal."""
+    res = run_ranks(world, _ring_holds, causal)
+    for rank in range(world):
+        status, seen = res[rank]
+        assert status == "ok", seen
+        want = [(j, 100 + j, causal and j == rank) for j in
+                [(rank - s) % world for s in range(world)] if not (causal and j > rank)]
+        assert seen == want, (rank, seen, want)
+
+
+def _ring_attention(rank, world, causal, B, Lc, H_q, H_kv, D):
+    from sequence_parallelism_attn_b200 import dist as rd
+    g = np.random.default_rng(11)
+    L = world * Lc
+    q = g.standard_normal((B, L, H_q, D)) * 2.0
+    k = g.standard_normal((B, L, H_kv, D))
+    v = g.standard_normal((B, L, H_kv, D))
+    sl = slice(rank * Lc, (rank + 1) * Lc)
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x[:, sl]))
+    out = torch.empty(B, Lc, H_q, D, dtype=torch.float64)
+    lse = torch.empty(B, H_q, Lc, dtype=torch.float64)
+    rd.ring_attn_fwd_dist(t(q), t(k), t(v), causal, 0.3, out=out, lse=lse, ops=OracleOps)
+    import oracle
+    want_o, want_l = oracle.attention(q, k, v, 0.3, causal)
+    return (float(np.abs(out.numpy() - want_o[:, sl]).max()),
+            float(np.abs(lse.numpy() - want_l[:, :, sl]).max()))
+
+
+@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("causal", [False, True])
+def test_ring_attention_equals_whole_sequence(world, causal):
+    """Each rank's merged result over the exchanged chunks equals attention of its queries
+    over the whole sequence (GQA 4:2, B = 2)."""
+    res = run_ranks(world, _ring_attention, causal, 2, 6, 4, 2, 8)
+    for rank in range(world):
+        status, errs = res[rank]
+        assert status == "ok", errs
+        assert errs[0] <= 1e-12 and errs[1] <= 1e-12, (rank, errs)
+
+
+# ------------------------------------------------------------------ Ulysses
+def _ulysses(rank, world, B, Lc, H_q, H_kv, D):
+    from sequence_parallelism_attn_b200 import dist as rd
+    import oracle
+    g = np.random.default_rng(5)
+    x = g.standard_normal((world, B, Lc, H_kv, D)).astype(np.float32)  # every rank's shard
+    H_out = int(np.lcm(H_kv, world))
+    y = rd.ulysses_seq2head_dist(torch.from_numpy(x[rank]), H_out, ops=OracleOps)
+    want = oracle.seq2head(x, H_out)[rank]                             # [B, P*Lc, Hl, D]
+    ok_fwd = y.numpy().tobytes() == want.tobytes() and y.shape == want.shape
+    h = g.standard_normal((world, B, world * Lc, H_q // world, D)).astype(np.float32)
+    z = rd.ulysses_head2seq_dist(torch.from_numpy(h[rank]), ops=OracleOps)
+    want_z = oracle.head2seq(h)[rank]                                   # [B, Lc, H_q, D]
+    ok_back = z.numpy().tobytes() == want_z.tobytes() and z.shape == want_z.shape
+    return ok_fwd, ok_back
+
+
+@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("B", [1, 2])
+def test_ulysses_pack_all_to_all_unpack_bit_exact(world, B):
+    """pack -> all-to-all -> unpack on every rank equals that rank's block of the oracle's
+    seq->head over all shards (with the GQA copy of 2 KV heads), and head->seq likewise."""
+    res = run_ranks(world, _ulysses, B, 5, 8, 2, 4)
+    for rank in range(world):
+        status, ok = res[rank]
+        assert status == "ok", ok
+        assert ok == (True, True), (rank, ok)
+
+
+# ------------------------------------------------------------------ a rank that leaves
+def _leaver(rank, world, leave_rank):
+    from sequence_parallelism_attn_b200 import dist as rd
+    if rank == leave_rank:
+        os._exit(0)  # leaves between steps: never posts its exchange
+    q = torch.zeros(1, 4, 2, 8, dtype=torch.float64)
+    k = torch.zeros(1, 4, 1, 8, dtype=torch.float64)
+    try:
+        rd.ring_attn_fwd_dist(q, k, k.clone(), True, 0.5,
+                              out=torch.empty(1, 4, 2, 8, dtype=torch.float64),
+                              lse=torch.empty(1, 2, 4, dtype=torch.float64), ops=RecordingOps)
+    except rd.ExchangeError as e:
+        return "ExchangeError: " + str(e)[:200]
+    return "completed"
+
+
+def test_rank_leaving_is_reported_not_hung():
+    """Rank 2 of 3 exits before the ring's first exchange: its ring neighbours get an
+    ExchangeError within the process group's timeout instead of waiting for good."""
+    res = run_ranks(3, _leaver, 2, timeout=90)
+    assert 2 not in res
+    # rank 0 receives from rank 2: its exchange must fail
+    status, msg = res[0]
+    assert status == "ok" and msg.startswith("ExchangeError"), msg
+    # rank 1 sends to rank 2 and receives from rank 0; it ends with an error too (its
+    # neighbour rank 0 gave up), never by waiting for good
+    status, msg = res[1]
+    assert status == "ok" and msg.startswith("ExchangeError"), msg

@@ -28,14 +28,18 @@
 // warpgroups raise their budget to 192 and the third warpgroup drops to 120
 // (192 + 192 + 120 = 504 <= 512 per sub-partition; 256*192 + 128*120 = 384*168).
 // Tensor memory (512 columns x 128 lanes x 32 bit):
-//   S_A [0,128) S_B [128,256) fp32 scores; P_A/P_B (bf16 probabilities) overwrite the
-//   first 64 columns of S_A/S_B; O_A at 256, O_B at 256+D (fp32 accumulators).
+//   S [0,128): one fp32 score buffer shared by the two query tiles; P_A [128,192) and
+//   P_B [192,256): bf16 probabilities (two per column); O_A at 256, O_B at 256+D (fp32).
 // Per KV tile j the MMA thread issues, in this order,
-//   PV_A(j) = P_A V(j);  S_A(j+1) = Q_A K(j+1)^T;  PV_B(j);  S_B(j+1)
-// so the tensor core works on one query tile while the softmax warps of the other
-// tile turn its scores into probabilities.  tcgen05.commit after S_A(j+1) signals both
-// "S_A(j+1) ready" and "PV_A(j) done", which is what the softmax needs before it may
-// rescale O_A.  The O rescale is skipped unless the row max grew by more than 2^8
+//   S_A(j+1) = Q_A K(j+1)^T  once softmax B has read S_B(j) out of S,
+//   PV_A(j)  = P_A V(j)      once softmax A has written P_A(j),
+//   S_B(j+1)                 once softmax A has read S_A(j+1),
+//   PV_B(j)                  once softmax B has written P_B(j),
+// so a tile's next scores are computed while its softmax still works on the current ones:
+// a softmax warpgroup finds S(j+1) ready when it finishes P(j), and the tensor core is
+// never waiting on a chain of PV(j) then S(j+1).  A softmax warpgroup reads S, signals that
+// S is free, and waits for PV(j-1) (its commit) only before it overwrites P(j-1) with P(j)
+// -- and before it rescales O, which it does only when the row max grew by more than 2^8
 // (exact: the final normalisation uses the same stale max as the probabilities).
 //
 // Every wait is bounded (a time limit on %globaltimer): a role that gives up sets a CTA
@@ -111,8 +115,8 @@ struct Cfg {
     static constexpr int OFF_V = OFF_K + NSK * TILE;
     static constexpr int OFF_BAR = OFF_V + NSV * TILE;
     // barriers: q_full, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV], s_full[2],
-    // p_full[2], o_full[2], drain
-    static constexpr int N_BARS = 1 + 2 * NSK + 2 * NSV + 2 + 2 + 2 + 1;
+    // p_full[2], o_full[2], drain, s_free[2] (softmax w has read S), pv_done[2]
+    static constexpr int N_BARS = 1 + 2 * NSK + 2 * NSV + 2 + 2 + 2 + 1 + 2 + 2;
     // tmem base (4 B), abort flag (4 B), the schedule's tile count (4 B)
     static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
     static constexpr int OFF_SCHED = OFF_MISC + 16;  // tile ranges: RA_MAX_P starts, RA_MAX_P ends
@@ -126,8 +130,12 @@ struct Cfg {
     __host__ __device__ static constexpr int bar_pf(int w) { return 3 + 2 * NSK + 2 * NSV + w; }
     __host__ __device__ static constexpr int bar_of(int w) { return 5 + 2 * NSK + 2 * NSV + w; }
     static constexpr int BAR_DRAIN = 7 + 2 * NSK + 2 * NSV;
-    static constexpr uint32_t S_COL0 = 0, S_COL1 = 128;
+    __host__ __device__ static constexpr int bar_sfree(int w) { return 8 + 2 * NSK + 2 * NSV + w; }
+    __host__ __device__ static constexpr int bar_pvd(int w) { return 10 + 2 * NSK + 2 * NSV + w; }
+    static constexpr uint32_t S_COL = 0;
+    static constexpr uint32_t P_COL0 = 128, P_COL1 = 192;
     static constexpr uint32_t O_COL0 = 256, O_COL1 = 256 + D;
+    static_assert(O_COL1 + D <= kTmemCols, "tensor memory budget");
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -248,7 +256,7 @@ __device__ __forceinline__ void mma_issuer(const AttnParams& p, uint32_t base, u
     const unsigned long long lim = p.wait_limit_ns;
     constexpr uint32_t IDESC_S = idesc_bf16_f32(kBM, kBN, 0);  // K-major Q and K
     constexpr uint32_t IDESC_O = idesc_bf16_f32(kBM, D, 1);    // V is MN-major (D contiguous)
-    const uint32_t s_col[2] = {C::S_COL0, C::S_COL1};
+    const uint32_t p_col[2] = {C::P_COL0, C::P_COL1};
     const uint32_t o_col[2] = {C::O_COL0, C::O_COL1};
 
     // Descriptors are built once per operand tile; a K step only moves the start address,
@@ -258,13 +266,13 @@ __device__ __forceinline__ void mma_issuer(const AttnParams& p, uint32_t base, u
                             desc_sw128(base + C::OFF_Q + C::TILE, 16, 1024)};
     const uint64_t dk0 = desc_sw128(base + C::OFF_K, 16, 1024);
     const uint64_t dv0 = desc_sw128(base + C::OFF_V, C::BLK, 1024);
-    // S_w = Q_w K^T over D in steps of 16: step kk lives in swizzle block kk/4 at byte 32*(kk%4).
+    // S = Q_w K^T over D in steps of 16: step kk lives in swizzle block kk/4 at byte 32*(kk%4).
     auto issue_s = [&](int w, int slot) {
         const uint64_t dk = dk0 + (uint64_t)((slot * C::TILE) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = ((kk / 4) * C::BLK + (kk % 4) * 32) >> 4;
-            mma_ss(tmem + s_col[w], dq[w] + off, dk + off, IDESC_S, kk > 0 ? 1u : 0u);
+            mma_ss(tmem + C::S_COL, dq[w] + off, dk + off, IDESC_S, kk > 0 ? 1u : 0u);
         }
     };
     // O_w (+)= P_w V over 128 keys in steps of 16: P from TMEM (8 columns of bf16 pairs per
@@ -273,7 +281,7 @@ __device__ __forceinline__ void mma_issuer(const AttnParams& p, uint32_t base, u
         const uint64_t dv = dv0 + (uint64_t)((slot * C::TILE) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-            mma_ts(tmem + o_col[w], tmem + s_col[w] + kk * 8, dv + (uint64_t)((kk * 2048) >> 4),
+            mma_ts(tmem + o_col[w], tmem + p_col[w] + kk * 8, dv + (uint64_t)((kk * 2048) >> 4),
                    IDESC_O, (acc || kk > 0) ? 1u : 0u);
     };
 
@@ -283,39 +291,47 @@ __device__ __forceinline__ void mma_issuer(const AttnParams& p, uint32_t base, u
         tc_fence_after();
         issue_s(0, 0);
         tc_commit(bar(C::bar_sf(0)));
-        issue_s(1, 0);
-        tc_commit(bar(C::bar_sf(1)));
-        tc_commit(bar(C::bar_ke(0)));
         issued = true;
-        for (int jt = 0; jt < n; ++jt) {
-            const int slot_v = jt % C::NSV;
-            const int slot_k = (jt + 1) % C::NSK;
-            const bool more = jt + 1 < n;
-            // V(j) and K(j+1) are awaited before P_A(j): the loads have long landed by then,
-            // so the waits cost nothing on the path from P_A(j) to S_A(j+1).
-            if (!wait1(bar(C::bar_vf(slot_v)), (jt / C::NSV) & 1, abort_flag, lim, kErrMma)) break;
-            if (more && !wait1(bar(C::bar_kf(slot_k)), ((jt + 1) / C::NSK) & 1, abort_flag, lim,
+        // S_B(0) goes into S once softmax A has read S_A(0) out of it
+        if (wait1(bar(C::bar_sfree(0)), 0, abort_flag, lim, kErrMma)) {
+            tc_fence_after();
+            issue_s(1, 0);
+            tc_commit(bar(C::bar_sf(1)));
+            tc_commit(bar(C::bar_ke(0)));
+            for (int jt = 0; jt < n; ++jt) {
+                const int slot_v = jt % C::NSV;
+                const int slot_k = (jt + 1) % C::NSK;
+                const bool more = jt + 1 < n;
+                if (more) {  // S_A(j+1): softmax B has read S_B(j), K(j+1) has landed
+                    if (!wait1(bar(C::bar_sfree(1)), jt & 1, abort_flag, lim, kErrMma)) break;
+                    if (!wait1(bar(C::bar_kf(slot_k)), ((jt + 1) / C::NSK) & 1, abort_flag, lim,
                                kErrMma))
-                break;
-            if (!wait1(bar(C::bar_pf(0)), jt & 1, abort_flag, lim, kErrMma)) break;
-            tc_fence_after();
-            issue_pv(0, slot_v, jt > 0);
-            if (more) {
-                issue_s(0, slot_k);
-                tc_commit(bar(C::bar_sf(0)));
-            } else {
-                tc_commit(bar(C::bar_of(0)));
-            }
-            if (!wait1(bar(C::bar_pf(1)), jt & 1, abort_flag, lim, kErrMma)) break;
-            tc_fence_after();
-            issue_pv(1, slot_v, jt > 0);
-            tc_commit(bar(C::bar_ve(slot_v)));
-            if (more) {
-                issue_s(1, slot_k);
-                tc_commit(bar(C::bar_sf(1)));
-                tc_commit(bar(C::bar_ke(slot_k)));
-            } else {
-                tc_commit(bar(C::bar_of(1)));
+                        break;
+                    tc_fence_after();
+                    issue_s(0, slot_k);
+                    tc_commit(bar(C::bar_sf(0)));
+                }
+                if (!wait1(bar(C::bar_vf(slot_v)), (jt / C::NSV) & 1, abort_flag, lim, kErrMma))
+                    break;
+                if (!wait1(bar(C::bar_pf(0)), jt & 1, abort_flag, lim, kErrMma)) break;
+                tc_fence_after();
+                issue_pv(0, slot_v, jt > 0);
+                tc_commit(bar(C::bar_pvd(0)));
+                if (!more) tc_commit(bar(C::bar_of(0)));
+                if (more) {  // S_B(j+1): softmax A has read S_A(j+1)
+                    if (!wait1(bar(C::bar_sfree(0)), (jt + 1) & 1, abort_flag, lim, kErrMma))
+                        break;
+                    tc_fence_after();
+                    issue_s(1, slot_k);
+                    tc_commit(bar(C::bar_sf(1)));
+                    tc_commit(bar(C::bar_ke(slot_k)));
+                }
+                if (!wait1(bar(C::bar_pf(1)), jt & 1, abort_flag, lim, kErrMma)) break;
+                tc_fence_after();
+                issue_pv(1, slot_v, jt > 0);
+                tc_commit(bar(C::bar_pvd(1)));
+                tc_commit(bar(C::bar_ve(slot_v)));
+                if (!more) tc_commit(bar(C::bar_of(1)));
             }
         }
     }
@@ -358,7 +374,8 @@ __device__ __forceinline__ void softmax_wg(const AttnParams& p, uint32_t base, u
         tile_qmin = (int)lo_pos;
     }
     const uint32_t lane_off = (uint32_t)(wr * 32) << 16;
-    const uint32_t tS = tmem + lane_off + (wg ? C::S_COL1 : C::S_COL0);
+    const uint32_t tS = tmem + lane_off + C::S_COL;
+    const uint32_t tP = tmem + lane_off + (wg ? C::P_COL1 : C::P_COL0);
     const uint32_t tO = tmem + lane_off + (wg ? C::O_COL1 : C::O_COL0);
     const float sl2 = p.scale_log2;
 
@@ -378,6 +395,9 @@ __device__ __forceinline__ void softmax_wg(const AttnParams& p, uint32_t base, u
         tc_fence_after();
         uint64_t s2[64];  // the row's 128 scores as pairs (2i, 2i+1)
         tmem_ld128_pairs(tS, s2);
+        // the scores are in registers: S may take the other tile's next scores
+        tc_fence_before();
+        mbar_arrive(bar(C::bar_sfree(wg)));
 
         const int j = it.chunk(), key0 = it.t * kBN;  // chunk and first local key of the tile
         const int kvalid = min(kBN, p.Lc - key0);
@@ -442,8 +462,8 @@ __device__ __forceinline__ void softmax_wg(const AttnParams& p, uint32_t base, u
             resc = true;
         }
         const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
-        // P = 2^(s*scale*log2e - m) in bf16 pairs, written over the first 64 columns of S
-        // (all of S is already in registers), one 64-key half at a time.
+        // P = 2^(s*scale*log2e - m) in bf16 pairs into this tile's P columns, one 64-key
+        // half at a time.  P(j-1) there is overwritten only once PV(j-1) has read it.
         const uint64_t sl2x2 = f2_pack(sl2, sl2), negm_x2 = f2_pack(neg_m, neg_m);
         uint64_t sum_a = 0, sum_b = 0, used_a = 0, used_b = 0;  // (0.f, 0.f) pairs
 #pragma unroll
@@ -456,15 +476,24 @@ __device__ __forceinline__ void softmax_wg(const AttnParams& p, uint32_t base, u
                 else
                     pk[c2] = softmax_pair(s2[half * 32 + c2], sl2x2, negm_x2, sum_a, used_a);
             }
-            tmem_st32(tS + half * 32, pk);
+            if (half == 0 && jt > 0) {
+                if (!wait_warp(bar(C::bar_pvd(wg)), (jt - 1) & 1, abort_flag, lim)) {
+                    ok = false;
+                    break;
+                }
+                __syncwarp();
+                tc_fence_after();
+            }
+            tmem_st32(tP + half * 32, pk);
         }
+        if (!ok) break;
         float s0, s1, u0, u1;
         f2_unpack(f2_add(sum_a, sum_b), s0, s1);
         f2_unpack(f2_add(used_a, used_b), u0, u1);
         l_run = l_run * alpha + (s0 + s1);
         l_used = l_used * alpha + (u0 + u1);
         if (__any_sync(FULL, resc)) {
-            // PV of the previous tile is complete: its commit preceded this tile's S commit.
+            // PV of the previous tile is complete: its commit (pv_done) was awaited above.
 #pragma unroll
             for (int cb = 0; cb < D / 32; ++cb) {
                 uint32_t o[32];
@@ -569,6 +598,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_sm100(const __grid_const
             mbar_init(bar(C::bar_sf(w)), 1);
             mbar_init(bar(C::bar_pf(w)), 4 * 32);
             mbar_init(bar(C::bar_of(w)), 1);
+            mbar_init(bar(C::bar_sfree(w)), 4 * 32);
+            mbar_init(bar(C::bar_pvd(w)), 1);
         }
         mbar_init(bar(C::BAR_DRAIN), 1);
         *abort_flag = 0;

@@ -363,7 +363,8 @@ class DistUlyssesPath:
         self.ra.ring_attn_fwd(qh, kv(kh), kv(vh), True, self.scale, out=self.o, lse=self.lse)
         rec("attn", 1)
         rec("permute_out", 0)
-        self.o_seq = rd.ulysses_head2seq_dist(self.o)
+        # into the same buffer every step: the end-to-end leg reads it on another stream
+        rd.ulysses_head2seq_dist(self.o, out=self.o_seq)
         rec("permute_out", 1)
 
     def result(self):

@@ -86,11 +86,13 @@ class DeviceOps:
         return ra.ra_ulysses_head2seq(y.unsqueeze(0), P=P)
 
     @staticmethod
-    def head2seq_unpack(recv):
-        """[P, B, Lc, Hl, D] (block r = rank r's heads) -> [B, Lc, P * Hl, D]."""
+    def head2seq_unpack(recv, out=None):
+        """[P, B, Lc, Hl, D] (block r = rank r's heads) -> [B, Lc, P * Hl, D] (into `out`
+        when given)."""
         from . import ra
         P, B, Lc, Hl, D = recv.shape
-        return ra.ra_ulysses_head2seq(recv, P=1).view(B, Lc, P * Hl, D)
+        dst = None if out is None else out.view(1, B, Lc, P * Hl, D)
+        return ra.ra_ulysses_head2seq(recv, out=dst, P=1).view(B, Lc, P * Hl, D)
 
 
 def _group_info(group):
@@ -200,13 +202,13 @@ def ulysses_seq2head_dist(x, H_out: int | None = None, group=None, ops=DeviceOps
     return ops.seq2head_unpack(recv)
 
 
-def ulysses_head2seq_dist(y, group=None, ops=DeviceOps):
+def ulysses_head2seq_dist(y, group=None, ops=DeviceOps, out=None):
     """Ulysses head->seq across the ranks of `group`: y [B, P*Lc, Hl, D] is this rank's
     head block over the whole sequence; returns [B, Lc, P*Hl, D], this rank's sequence
-    shard with every head."""
+    shard with every head (written into `out`, contiguous, when given)."""
     rank, world = _group_info(group)
     if y.shape[1] % world:
         raise ValueError(f"sequence of {y.shape[1]} tokens does not split over {world} ranks")
     send = ops.head2seq_pack(y, world)
     recv = _all_to_all(send, group, f"head2seq all-to-all on rank {rank}")
-    return ops.head2seq_unpack(recv)
+    return ops.head2seq_unpack(recv) if out is None else ops.head2seq_unpack(recv, out=out)

@@ -106,6 +106,9 @@ def test_distributed_functions_on_one_rank(ra_lib, oracle_mod):
         assert np.array_equal(_bits(y), oracle_mod.seq2head(_bits(k)[None], 2)[0])
         z = rd.ulysses_head2seq_dist(y)
         assert np.array_equal(_bits(z), _bits(k))
+        z2 = torch.full_like(z, float("nan"))
+        rd.ulysses_head2seq_dist(y, out=z2)  # into a caller's buffer
+        assert np.array_equal(_bits(z2), _bits(k))
         torch.cuda.synchronize()
     finally:
         dist.destroy_process_group()

@@ -50,3 +50,27 @@ def test_merge_of_two_chunk_partials_equals_whole(ra_lib, oracle_mod):
     want_o, want_l = oracle_mod.attention(f64(q), f64(kk), f64(vv), w.scale, False)
     assert max_abs(f64(oa), want_o) <= 1e-2
     assert max_abs(f64(la), want_l) <= 1e-3
+
+
+def test_merge_full_size_sampled(ra_lib, oracle_mod):
+    """The benchmarked merge (B = 1, H = 8, L = 131072, D = 128, fp32; 10% empty partials):
+    4096 seeded rows, plus the first and last row, against the oracle's merge of those
+    rows; every output finite where a partial is."""
+    B, H, L, D = 1, 8, 131072, 128
+    oa, la, ob, lb = synth.merge_inputs(B, H, L, D, seed=1007, neg_inf_frac=0.1)
+    goa, gla = oa.cuda(), la.cuda()
+    ra_lib.ra_lse_merge(goa, gla, ob.cuda(), lb.cuda())
+    torch.cuda.synchronize()
+    g = torch.Generator().manual_seed(8)
+    t = torch.cat([torch.randint(0, L, (4096,), generator=g), torch.tensor([0, L - 1])])
+    h = torch.cat([torch.randint(0, H, (4096,), generator=g), torch.tensor([0, H - 1])])
+    pick_o = lambda x: x[0, t, h].unsqueeze(0).unsqueeze(2)   # [1, n, 1, D]
+    pick_l = lambda x: x[0, h, t].view(1, 1, -1)               # [1, 1, n]
+    want_o, want_l = oracle_mod.lse_merge(f64(pick_o(oa)), f64(pick_l(la)), f64(pick_o(ob)),
+                                          f64(pick_l(lb)))
+    got_o, got_l = f64(pick_o(goa.cpu())), f64(pick_l(gla.cpu()))
+    both_empty = np.isneginf(want_l)
+    assert np.array_equal(np.isneginf(got_l), both_empty)
+    assert max_abs(got_l[~both_empty], want_l[~both_empty]) <= 1e-5
+    assert max_abs(got_o, want_o) <= 1e-5
+    assert torch.isfinite(goa).all()

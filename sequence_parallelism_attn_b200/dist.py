@@ -123,10 +123,10 @@ class RingAccumulator:
         self.q, self.rank, self.causal, self.ops = q, rank, causal, ops
         self.scale = D ** -0.5 if scale is None else scale
         dev = q.device
-        self.out = torch.empty((B, Lc, H_q, D), dtype=torch.float32, device=dev) \
-            if out is None else out
-        self.lse = torch.empty((B, H_q, Lc), dtype=torch.float32, device=dev) \
-            if lse is None else lse
+        # fp32 results (float64 ones for float64 inputs, which only host-side checks use)
+        rdt = torch.float64 if q.dtype == torch.float64 else torch.float32
+        self.out = torch.empty((B, Lc, H_q, D), dtype=rdt, device=dev) if out is None else out
+        self.lse = torch.empty((B, H_q, Lc), dtype=rdt, device=dev) if lse is None else lse
         self.part = None
         self.visited = 0
 
@@ -212,3 +212,25 @@ def ulysses_head2seq_dist(y, group=None, ops=DeviceOps, out=None):
     send = ops.head2seq_pack(y, world)
     recv = _all_to_all(send, group, f"head2seq all-to-all on rank {rank}")
     return ops.head2seq_unpack(recv) if out is None else ops.head2seq_unpack(recv, out=out)
+
+
+def usp_attn_fwd_dist(q, k, v, causal: bool, scale: float | None = None, ulysses_group=None,
+                      ring_group=None, ops=DeviceOps):
+    """The ring x Ulysses hybrid (USP) across GPUs: the ranks form P_r ring groups of P_u
+    Ulysses ranks.  q [B, Ls, H_q, D], k/v [B, Ls, H_kv, D] are this rank's sequence shard
+    (every head); the P_u ranks of `ulysses_group` hold consecutive shards and share a head
+    split, and `ring_group` holds the P_r ranks at this rank's place in every Ulysses group,
+    in sequence order.  seq->head inside the Ulysses group gives this rank H/P_u heads over
+    its group's P_u*Ls tokens (KV heads copied up to lcm(H_kv, P_u)); the ring runs across
+    the ring group over P_r chunks of P_u*Ls tokens; head->seq brings the output back.
+    Returns (out [B, Ls, H_q, D] fp32, lse [B, H_q/P_u, P_u*Ls] of this rank's head block
+    over its Ulysses group's tokens)."""
+    import math
+    P_u = dist.get_world_size(ulysses_group)
+    H_q, H_kv = q.shape[2], k.shape[2]
+    H_rep = H_kv * P_u // math.gcd(H_kv, P_u)
+    qh = ulysses_seq2head_dist(q, H_q, group=ulysses_group, ops=ops)
+    kh = ulysses_seq2head_dist(k, H_rep, group=ulysses_group, ops=ops)
+    vh = ulysses_seq2head_dist(v, H_rep, group=ulysses_group, ops=ops)
+    o, lse = ring_attn_fwd_dist(qh, kh, vh, causal, scale, group=ring_group, ops=ops)
+    return ulysses_head2seq_dist(o, group=ulysses_group, ops=ops), lse

@@ -84,8 +84,9 @@ def test_ulysses_pack_unpack_bit_exact(ra_lib, oracle_mod, B, dtype):
 
 
 def test_distributed_functions_on_one_rank(ra_lib, oracle_mod):
-    """ring_attn_fwd_dist and the Ulysses functions through a one-rank NCCL process group
-    (the all-to-all moves one block to itself; the ring has one step)."""
+    """ring_attn_fwd_dist, the Ulysses functions and their composition (USP) through a
+    one-rank NCCL process group (the all-to-all moves one block to itself; the ring has one
+    step)."""
     import torch.distributed as dist
     s = socket.socket()
     s.bind(("127.0.0.1", 0))
@@ -109,6 +110,8 @@ def test_distributed_functions_on_one_rank(ra_lib, oracle_mod):
         z2 = torch.full_like(z, float("nan"))
         rd.ulysses_head2seq_dist(y, out=z2)  # into a caller's buffer
         assert np.array_equal(_bits(z2), _bits(k))
+        uo, ul = rd.usp_attn_fwd_dist(q.cuda(), k.cuda(), v.cuda(), True, D ** -0.5)
+        assert max_abs(f64(uo), want_o) <= 1e-2 and max_abs(f64(ul), want_l) <= 1e-3
         torch.cuda.synchronize()
     finally:
         dist.destroy_process_group()

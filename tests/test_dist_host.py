@@ -223,6 +223,48 @@ def test_ulysses_pack_all_to_all_unpack_bit_exact(world, B):
         assert ok == (True, True), (rank, ok)
 
 
+# ------------------------------------------------------------------ ring x Ulysses (USP)
+def _usp(rank, world, P_u, causal):
+    import torch.distributed as dist
+    from sequence_parallelism_attn_b200 import dist as rd
+    import oracle
+    P_r = world // P_u
+    # every rank creates every group, in the same order
+    ulysses = [dist.new_group([g * P_u + u for u in range(P_u)]) for g in range(P_r)]
+    rings = [dist.new_group([g * P_u + u for g in range(P_r)]) for u in range(P_u)]
+    B, Ls, H_q, H_kv, D = 2, 5, 4, 1, 8
+    rng = np.random.default_rng(21)
+    q = rng.standard_normal((world, B, Ls, H_q, D)) * 2.0
+    k = rng.standard_normal((world, B, Ls, H_kv, D))
+    v = rng.standard_normal((world, B, Ls, H_kv, D))
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x[rank]))
+    out, lse = rd.usp_attn_fwd_dist(t(q), t(k), t(v), causal, 0.3,
+                                    ulysses_group=ulysses[rank // P_u],
+                                    ring_group=rings[rank % P_u], ops=OracleOps)
+    seq = lambda x: np.concatenate(list(x), axis=1)  # [B, world * Ls, H, D]
+    want_o, want_l = oracle.attention(seq(q), seq(k), seq(v), 0.3, causal)
+    sl = slice(rank * Ls, (rank + 1) * Ls)
+    u = rank % P_u
+    Hl = H_q // P_u
+    eo = float(np.abs(out.numpy() - want_o[:, sl]).max())
+    g = rank // P_u  # the Ulysses group's tokens: the ring chunk g
+    gsl = slice(g * P_u * Ls, (g + 1) * P_u * Ls)
+    el = float(np.abs(lse.numpy() - want_l[:, u * Hl:(u + 1) * Hl, gsl]).max())
+    return eo, el
+
+
+@pytest.mark.parametrize("P_u,causal", [(2, True), (2, False), (4, True), (1, True)])
+def test_usp_across_ranks_equals_whole_sequence(P_u, causal):
+    """4 ranks as P_r ring groups x P_u Ulysses ranks (2 x 2, 1 x 4, 4 x 1): each rank's
+    output rows, and its head block's LSE over its group's tokens, equal attention over the
+    whole sequence (one KV head copied up to P_u)."""
+    res = run_ranks(4, _usp, P_u, causal)
+    for rank in range(4):
+        status, errs = res[rank]
+        assert status == "ok", errs
+        assert errs[0] <= 1e-12 and errs[1] <= 1e-12, (rank, errs)
+
+
 # ------------------------------------------------------------------ a rank that leaves
 def _leaver(rank, world, leave_rank):
     from sequence_parallelism_attn_b200 import dist as rd

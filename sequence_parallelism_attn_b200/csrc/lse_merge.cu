@@ -8,19 +8,29 @@
 // A row is handled by TPR threads of one warp (TPR = the power of two >= D/4, at most
 // 32), each moving float4s; every thread of a row reads both LSEs before the row's
 // first thread overwrites lse_a, separated by __syncwarp, so the in-place update has no
-// race.  The grid is a multiple of the SM count and strides over rows.
+// race.  The grid is one wave of 256-thread blocks (a multiple of the SM count) and strides
+// over rows.
 #include "ra_internal.h"
+#include "permute_index.cuh"
 #include <cmath>
 
 namespace ra {
 namespace {
 
+// Two rows per warp slot per iteration, and every load of both rows (the two LSEs and the
+// first float4 of O_a and O_b) issued before any arithmetic: the row's addresses do not
+// depend on the LSE values, so a warp keeps four independent loads per lane in flight
+// instead of waiting for the LSEs before it asks for O.
+// FAST: every row index fits in 32 bits, so the row's (b, t, h) come from two
+// invariant-divisor multiplications (by H, then by L) instead of 64-bit divisions, which
+// would cost more instructions per row than the row's loads and stores.
+template <bool FAST>
 __global__ void __launch_bounds__(256) lse_merge_kernel(float* __restrict__ o_a,
                                                         float* __restrict__ lse_a,
                                                         const float* __restrict__ o_b,
                                                         const float* __restrict__ lse_b,
                                                         int B, int H, long long L, int D,
-                                                        int tpr_log2) {
+                                                        int tpr_log2, FastDiv fH, FastDiv fL) {
     const int tpr = 1 << tpr_log2;
     const int rows_per_warp = 32 >> tpr_log2;
     const int lane = threadIdx.x & 31;
@@ -29,56 +39,85 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(float* __restrict__ o_a,
     const long long n_rows = (long long)B * L * H;
     const long long warp_global = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const long long n_warps = ((long long)gridDim.x * blockDim.x) >> 5;
+    const long long step = n_warps * rows_per_warp;  // rows between a warp's two rows
     const int D4 = D >> 2;
+    const bool has_c = li < D4;  // this lane owns float4 li of each row
     // Every lane of the warp runs the same number of iterations so that __syncwarp is legal.
-    for (long long base = warp_global * rows_per_warp; base < n_rows;
-         base += n_warps * rows_per_warp) {
-        const long long row = base + sub;  // row in [B][L][H] order
-        const bool active = row < n_rows;
-        long long li_idx = 0;
-        float la = -INFINITY, lb = -INFINITY;
-        if (active) {
-            const long long h = row % H;
-            const long long t = (row / H) % L;
-            const long long b = row / H / L;
-            li_idx = (b * H + h) * L + t;
-            la = lse_a[li_idx];
-            lb = lse_b[li_idx];
+    for (long long base = warp_global * rows_per_warp; base < n_rows; base += 2 * step) {
+        long long row[2], li_idx[2] = {0, 0};
+        bool active[2];
+        float la[2] = {-INFINITY, -INFINITY}, lb[2] = {-INFINITY, -INFINITY};
+        float4 x[2], y[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            row[u] = base + u * step + sub;  // row in [B][L][H] order
+            active[u] = row[u] < n_rows;
+            if (active[u]) {
+                long long h, t, b;
+                if (FAST) {
+                    const uint32_t r = (uint32_t)row[u];
+                    const uint32_t tok = fdiv(r, fH);  // b * L + t
+                    const uint32_t bb = fdiv(tok, fL);
+                    h = r - tok * (uint32_t)H;
+                    t = tok - bb * (uint32_t)L;
+                    b = bb;
+                } else {
+                    h = row[u] % H;
+                    t = (row[u] / H) % L;
+                    b = row[u] / H / L;
+                }
+                li_idx[u] = (b * H + h) * L + t;
+                la[u] = lse_a[li_idx[u]];
+                lb[u] = lse_b[li_idx[u]];
+                if (has_c) {
+                    x[u] = reinterpret_cast<const float4*>(o_a + row[u] * D)[li];
+                    y[u] = __ldg(reinterpret_cast<const float4*>(o_b + row[u] * D) + li);
+                }
+            }
         }
         __syncwarp();
-        const float m = fmaxf(la, lb);
-        float wa = 0.f, wb = 0.f, lse = -INFINITY;
-        if (m != -INFINITY) {
-            const float ea = expf(la - m), eb = expf(lb - m);
-            const float z = ea + eb;
-            lse = m + logf(z);
-            wa = ea / z;
-            wb = eb / z;
-        }
-        if (active) {
-            float4* pa = reinterpret_cast<float4*>(o_a + row * D);
-            const float4* pb = reinterpret_cast<const float4*>(o_b + row * D);
-            for (int c = li; c < D4; c += tpr) {
-                const float4 x = pa[c], y = __ldg(pb + c);
-                float4 r;
-                r.x = wa * x.x + wb * y.x;
-                r.y = wa * x.y + wb * y.y;
-                r.z = wa * x.z + wb * y.z;
-                r.w = wa * x.w + wb * y.w;
-                pa[c] = r;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const float m = fmaxf(la[u], lb[u]);
+            float wa = 0.f, wb = 0.f, lse = -INFINITY;
+            if (m != -INFINITY) {
+                const float ea = expf(la[u] - m), eb = expf(lb[u] - m);
+                const float z = ea + eb;
+                lse = m + logf(z);
+                wa = ea / z;
+                wb = eb / z;
             }
-            if (li == 0) lse_a[li_idx] = lse;
+            if (active[u]) {
+                float4* pa = reinterpret_cast<float4*>(o_a + row[u] * D);
+                const float4* pb = reinterpret_cast<const float4*>(o_b + row[u] * D);
+                if (has_c)
+                    pa[li] = make_float4(wa * x[u].x + wb * y[u].x, wa * x[u].y + wb * y[u].y,
+                                         wa * x[u].z + wb * y[u].z, wa * x[u].w + wb * y[u].w);
+                for (int c = li + tpr; c < D4; c += tpr) {  // rows wider than 32 float4s
+                    const float4 xc = pa[c], yc = __ldg(pb + c);
+                    pa[c] = make_float4(wa * xc.x + wb * yc.x, wa * xc.y + wb * yc.y,
+                                        wa * xc.z + wb * yc.z, wa * xc.w + wb * yc.w);
+                }
+                if (li == 0) lse_a[li_idx[u]] = lse;
+            }
         }
     }
 }
 
-int sm_count_merge() {
+// Blocks of one full wave: SMs x resident 256-thread blocks per SM.
+int wave_blocks_merge() {
     static int n = 0;
     if (n == 0) {
-        int dev = 0;
+        int dev = 0, sms = 0, per_sm = 0;
         if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-            n = 148;
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            sms <= 0)
+            sms = 148;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, lse_merge_kernel<true>, 256, 0) !=
+                cudaSuccess ||
+            per_sm <= 0)
+            per_sm = 4;
+        n = sms * per_sm;
     }
     return n;
 }
@@ -92,10 +131,18 @@ cudaError_t launch_lse_merge(float* o_a, float* lse_a, const float* o_b, const f
     const long long n_rows = (long long)B * L * H;
     const long long rows_per_block = (256 / 32) * (32 >> tpr_log2);
     long long blocks = (n_rows + rows_per_block - 1) / rows_per_block;
-    const long long cap = (long long)sm_count_merge() * 8 * 4;
+    const long long cap = wave_blocks_merge();
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    lse_merge_kernel<<<(unsigned)blocks, 256, 0, s>>>(o_a, lse_a, o_b, lse_b, B, H, L, D, tpr_log2);
+    const FastDiv fH = make_fastdiv((uint32_t)H);
+    const bool fast = n_rows <= 0xffffffffLL && L <= 0xffffffffLL;
+    const FastDiv fL = make_fastdiv(fast ? (uint32_t)L : 1u);
+    if (fast)
+        lse_merge_kernel<true><<<(unsigned)blocks, 256, 0, s>>>(o_a, lse_a, o_b, lse_b, B, H, L,
+                                                                 D, tpr_log2, fH, fL);
+    else
+        lse_merge_kernel<false><<<(unsigned)blocks, 256, 0, s>>>(o_a, lse_a, o_b, lse_b, B, H, L,
+                                                                  D, tpr_log2, fH, fL);
     return cudaGetLastError();
 }
 

@@ -19,7 +19,11 @@
 // The compute warps publish P / dS in two 64-column halves (the MMAs over the first half
 // run while the second is formed) and signal when they have read dP, so that the next
 // tile's S (dQ kernel: into the spare region) and dP (dK/dV: S^T into the freed dP^T
-// region) are computed while they work.
+// region) are computed while they work.  Each MMA thread commits its own ready barrier (S
+// or S^T; dP or dP^T): in the dK/dV kernel the compute warps form and publish P^T from S^T
+// before they wait for dP^T, whose region frees only when dK of the previous tile is done,
+// so the exponentials overlap that chain; in the dQ kernel the S-ready commit waits for S
+// alone, not for the previous tile's dQ.
 // Roles (dQ kernel 352 threads, dK/dV 384 with an idle warp 11 and a setmaxnreg split):
 // warps 0-7 compute P, dS (one TMEM lane = one row; warps 0-3 the first 64 columns of a
 // tile, 4-7 the second), warp 8 loads (TMA, and in dK/dV the per-row LSE, Delta,
@@ -101,10 +105,12 @@ struct BCfg {
     static constexpr int ROWS_BYTES = 4 * kBM * 4 + 4 * 4;
     static constexpr int STAGE = 2 * TILE + ((ROWS_BYTES + 1023) / 1024) * 1024;
     static constexpr int OFF_BAR = OFF_RING + NS * STAGE;
-    // barriers: fixed_full, full[NS], empty[NS], sd_full, ds_full[2] (one per 64-column
-    // half of dS / P^T), acc_done, drain, dp_free (the compute warps have read all of dP),
-    // x_free (dK/dV kernel: the MMAs reading P^T / dS^T of a tile are done)
-    static constexpr int N_BARS = 1 + 2 * NS + 7;
+    // barriers: fixed_full, full[NS], empty[NS], s_ready (S / S^T of a tile complete),
+    // dp_ready (dP / dP^T complete), ds_full[2][2] (dS / dS^T of each 64-column half stored;
+    // two per half, by tile parity), p_full[2][2] (dK/dV kernel: P^T of each half stored; by
+    // tile parity), acc_done, drain, dp_free (the compute warps have read all of dP), x_free
+    // (dK/dV kernel: the MMAs reading P^T / dS^T of a tile are done)
+    static constexpr int N_BARS = 1 + 2 * NS + 14;
     static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem base, abort flag, n
     static constexpr int OFF_SCHED = OFF_MISC + 16;
     // dK/dV kernel, zigzag / packed: ascending query-tile ranges [lo, hi), at most 2 per rank
@@ -113,12 +119,17 @@ struct BCfg {
     static constexpr int BAR_FIXED = 0;
     __host__ __device__ static constexpr int bar_full(int s) { return 1 + s; }
     __host__ __device__ static constexpr int bar_empty(int s) { return 1 + NS + s; }
-    static constexpr int BAR_SD = 1 + 2 * NS;
-    __host__ __device__ static constexpr int bar_ds(int half) { return 2 + 2 * NS + half; }
-    static constexpr int BAR_ACC = 4 + 2 * NS;
-    static constexpr int BAR_DRAIN = 5 + 2 * NS;
-    static constexpr int BAR_DPFREE = 6 + 2 * NS;
-    static constexpr int BAR_XFREE = 7 + 2 * NS;
+    static constexpr int BAR_SREADY = 1 + 2 * NS;
+    static constexpr int BAR_DPREADY = 2 + 2 * NS;
+    // tile i's barrier of a half and its wait parity: the k-th phase of ds(half, par) (or
+    // p(half, par)) belongs to tile 2k + par
+    __host__ __device__ static constexpr int bar_ds(int half, int i) { return 3 + 2 * NS + 2 * half + (i & 1); }
+    __host__ __device__ static constexpr int bar_p(int half, int i) { return 7 + 2 * NS + 2 * half + (i & 1); }
+    __host__ __device__ static constexpr uint32_t par2(int i) { return (uint32_t)(i >> 1) & 1u; }
+    static constexpr int BAR_ACC = 11 + 2 * NS;
+    static constexpr int BAR_DRAIN = 12 + 2 * NS;
+    static constexpr int BAR_DPFREE = 13 + 2 * NS;
+    static constexpr int BAR_XFREE = 14 + 2 * NS;
     // dQ kernel TMEM: S of even key tiles at column 0, of odd ones at S_ODD (S of the next
     // tile is computed while this tile's dS is formed), dP at 128, dQ at 256.
     static constexpr uint32_t S_ODD = 384;
@@ -252,27 +263,38 @@ __device__ __forceinline__ void tmem_ld64_pairs(uint32_t taddr, uint64_t (&o)[32
         : "memory");
 }
 
-// One column pair of the backward's elementwise step, on packed fp32 pairs:
+// The backward's elementwise step on packed fp32 pairs, in two parts so that P can be
+// formed before dP is ready:
 //   p  = 2^(s * scale_log2 + neg_lse)     (one packed fma, two MUFU ex2)
 //   ds = p * (dp + neg_delta)             (one packed add, one packed multiply)
-// Returns bf16x2(p) in pp and bf16x2(ds) in pd (lane 0 in the low half).  The roundings are
-// those of the scalar fma, add and multiply.
-__device__ __forceinline__ void p_ds_pair(uint64_t s2, uint64_t dp2, uint64_t sl2x2,
-                                          uint64_t nlse2, uint64_t ndelta2, uint32_t& pp,
-                                          uint32_t& pd) {
-    asm("{\n\t.reg .b32 x0, x1, p0, p1, d0, d1;\n\t.reg .b64 x, p, t, d;\n\t"
-        "fma.rn.f32x2 x, %2, %4, %5;\n\t"
+// p_pair returns bf16x2(p) (lane 0 in the low half) and the fp32 pair in p2; the roundings
+// are those of the scalar fma, add and multiply.
+__device__ __forceinline__ uint32_t p_pair(uint64_t s2, uint64_t sl2x2, uint64_t nlse2,
+                                           uint64_t& p2) {
+    uint32_t pp;
+    asm("{\n\t.reg .b32 x0, x1, p0, p1;\n\t.reg .b64 x;\n\t"
+        "fma.rn.f32x2 x, %2, %3, %4;\n\t"
         "mov.b64 {x0, x1}, x;\n\t"
         "ex2.approx.ftz.f32 p0, x0;\n\t"
         "ex2.approx.ftz.f32 p1, x1;\n\t"
         "cvt.rn.bf16x2.f32 %0, p1, p0;\n\t"
-        "mov.b64 p, {p0, p1};\n\t"
-        "add.rn.f32x2 t, %3, %6;\n\t"
-        "mul.rn.f32x2 d, p, t;\n\t"
+        "mov.b64 %1, {p0, p1};\n\t}"
+        : "=r"(pp), "=l"(p2)
+        : "l"(s2), "l"(sl2x2), "l"(nlse2));
+    return pp;
+}
+
+// The second part: bf16x2(p * (dp + neg_delta)) from the fp32 pair p2 of p_pair.
+__device__ __forceinline__ uint32_t ds_from_p(uint64_t p2, uint64_t dp2, uint64_t ndelta2) {
+    uint32_t pd;
+    asm("{\n\t.reg .b32 d0, d1;\n\t.reg .b64 t, d;\n\t"
+        "add.rn.f32x2 t, %2, %3;\n\t"
+        "mul.rn.f32x2 d, %1, t;\n\t"
         "mov.b64 {d0, d1}, d;\n\t"
-        "cvt.rn.bf16x2.f32 %1, d1, d0;\n\t}"
-        : "=r"(pp), "=r"(pd)
-        : "l"(s2), "l"(dp2), "l"(sl2x2), "l"(nlse2), "l"(ndelta2));
+        "cvt.rn.bf16x2.f32 %0, d1, d0;\n\t}"
+        : "=r"(pd)
+        : "l"(p2), "l"(dp2), "l"(ndelta2));
+    return pd;
 }
 
 // The same without bf16(p): the dQ kernel needs only dS.
@@ -389,9 +411,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
             mbar_init(bar(C::bar_full(s)), 1);
             mbar_init(bar(C::bar_empty(s)), 1);
         }
-        mbar_init(bar(C::BAR_SD), 2);  // one commit from each MMA thread
-        mbar_init(bar(C::bar_ds(0)), 4 * 32);
-        mbar_init(bar(C::bar_ds(1)), 4 * 32);
+        mbar_init(bar(C::BAR_SREADY), 1);   // thread A's commit after S
+        mbar_init(bar(C::BAR_DPREADY), 1);  // thread B's commit after dP
+        for (int hf = 0; hf < 2; ++hf)
+            for (int par = 0; par < 2; ++par) mbar_init(bar(C::bar_ds(hf, par)), 4 * 32);
         mbar_init(bar(C::BAR_ACC), 1);
         mbar_init(bar(C::BAR_DRAIN), 2);
         mbar_init(bar(C::BAR_DPFREE), kComputeWarps * 32);
@@ -490,40 +513,44 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
             };
             // Two issuing threads (one thread cannot issue 128-wide MMAs fast enough to keep
             // the tensor core busy).  A issues S and dQ, B issues dP; no MMA reads the other
-            // thread's output columns, so they share only SD (one commit from each) and the
-            // drain.  A, per key tile jt: S(jt+1) into the other S region; dQ over each
-            // 64-key half as the compute warps publish it; after the second half, its share
-            // of SD(jt+1), then that half's dQ (it overlaps their next tile).  B, per key
-            // tile jt: dP(jt+1) once the compute warps have read dP(jt), and its share of
-            // SD(jt+1): dP(jt+1) overlaps their work on tile jt.
+            // thread's output columns.  A, per key tile jt: S(jt+1) into the other S region as
+            // soon as K(jt+1) has landed, committed to s_ready once every compute warp has
+            // read tile jt (dp_free) -- so the commit waits for S(jt+1) alone, not for dQ(jt),
+            // and s_ready cannot complete a phase before the compute warps have waited for
+            // the previous one; then dQ over each 64-key half as the compute warps publish it.
+            // B, per key tile jt: dP(jt+1) once the compute warps have read dP(jt), committed
+            // to dp_ready.  The compute warps can then finish tile jt+1 before A has waited for
+            // tile jt's dS, which is why each half's ds barrier alternates by tile parity.
             if (wait1(bar(C::BAR_FIXED), 0, abort_flag, lim, kErrMma) && n > 0 &&
                 wait1(bar(C::bar_full(0)), 0, abort_flag, lim, kErrMma)) {
                 tc_fence_after();
                 if (thread_a) {
                     issue_s(0);
-                    tc_commit(bar(C::BAR_SD));
+                    tc_commit(bar(C::BAR_SREADY));
                     for (int jt = 0; jt < n; ++jt) {
                         const bool more = jt + 1 < n;
-                        const uint32_t ph = jt & 1;
                         if (more) {
                             if (!wait1(bar(C::bar_full((jt + 1) % C::NS)), ((jt + 1) / C::NS) & 1,
                                        abort_flag, lim, kErrMma))
                                 break;
                             tc_fence_after();
                             issue_s(jt + 1);
+                            if (!wait1(bar(C::BAR_DPFREE), jt & 1, abort_flag, lim, kErrMma)) break;
+                            tc_commit(bar(C::BAR_SREADY));
                         }
-                        if (!wait1(bar(C::bar_ds(0)), ph, abort_flag, lim, kErrMma)) break;
+                        if (!wait1(bar(C::bar_ds(0, jt)), C::par2(jt), abort_flag, lim, kErrMma))
+                            break;
                         tc_fence_after();
                         dq_half(jt, 0);
-                        if (!wait1(bar(C::bar_ds(1)), ph, abort_flag, lim, kErrMma)) break;
+                        if (!wait1(bar(C::bar_ds(1, jt)), C::par2(jt), abort_flag, lim, kErrMma))
+                            break;
                         tc_fence_after();
-                        if (more) tc_commit(bar(C::BAR_SD));
                         dq_half(jt, 1);
                         tc_commit(bar(C::bar_empty(jt % C::NS)));
                     }
                 } else {
                     issue_dp(0);
-                    tc_commit(bar(C::BAR_SD));
+                    tc_commit(bar(C::BAR_DPREADY));
                     for (int jt = 0; jt + 1 < n; ++jt) {
                         if (!wait1(bar(C::BAR_DPFREE), jt & 1, abort_flag, lim, kErrMma)) break;
                         if (!wait1(bar(C::bar_full((jt + 1) % C::NS)), ((jt + 1) / C::NS) & 1,
@@ -531,7 +558,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
                             break;
                         tc_fence_after();
                         issue_dp(jt + 1);
-                        tc_commit(bar(C::BAR_SD));
+                        tc_commit(bar(C::BAR_DPREADY));
                     }
                 }
             }
@@ -565,7 +592,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
         SchedIter it;
         it.begin(sched);
         for (int jt = 0; jt < n; ++jt, it.next()) {
-            if (!wait_warp(bar(C::BAR_SD), jt & 1, abort_flag, lim, kErrCompute)) {
+            if (!wait_warp(bar(C::BAR_SREADY), jt & 1, abort_flag, lim, kErrCompute) ||
+                !wait_warp(bar(C::BAR_DPREADY), jt & 1, abort_flag, lim, kErrCompute)) {
                 ok = false;
                 break;
             }
@@ -617,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_sm100(const __grid_constan
             tmem_st32(tmem + lane_off + scol + 64 * c, pk);
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(C::bar_ds(c)));
+            mbar_arrive(bar(C::bar_ds(c, jt)));
         }
         if (ok && n > 0 && wait_warp(bar(C::BAR_ACC), 0, abort_flag, lim, kErrCompute)) {
             __syncwarp();
@@ -700,9 +728,12 @@ __global__ void __launch_bounds__(kThreadsKV, 1) bwd_dkdv_sm100(const __grid_con
             mbar_init(bar(C::bar_full(s)), 1 + 1);  // the load thread's expect_tx + the per-row values
             mbar_init(bar(C::bar_empty(s)), 1);
         }
-        mbar_init(bar(C::BAR_SD), 1);
-        mbar_init(bar(C::bar_ds(0)), 4 * 32);
-        mbar_init(bar(C::bar_ds(1)), 4 * 32);
+        mbar_init(bar(C::BAR_SREADY), 1);   // thread B's commit after S^T
+        mbar_init(bar(C::BAR_DPREADY), 1);  // thread A's commit after dP^T
+        mbar_init(bar(C::bar_ds(0, 0)), 4 * 32);
+        mbar_init(bar(C::bar_ds(1, 0)), 4 * 32);
+        for (int hf = 0; hf < 2; ++hf)
+            for (int par = 0; par < 2; ++par) mbar_init(bar(C::bar_p(hf, par)), 4 * 32);
         mbar_init(bar(C::BAR_ACC), 2);  // dV from thread A, dK from thread B
         mbar_init(bar(C::BAR_DRAIN), 2);
         mbar_init(bar(C::BAR_XFREE), 1);
@@ -852,41 +883,44 @@ __global__ void __launch_bounds__(kThreadsKV, 1) bwd_dkdv_sm100(const __grid_con
                     mma_ts(tmem + 256 + acc * D, a0 + (kk % 4) * 8, bm + (uint64_t)((kk * 2048) >> 4),
                            IDESC_O, (i > 0 || kk > 0) ? 1u : 0u);
             };
-            // Two issuing threads.  A issues dP^T and dV, B issues S^T and dK.  dP^T(i+1)
-            // overwrites the region that dK(i) reads, so A first waits for B's x_free commit
-            // (after dK(i)); that commit also covers S^T(i+1), so A's commit of SD(i+1)
-            // alone tells the compute warps that the next tile's S^T and dP^T are ready.
-            // B, per query tile i: S^T(i+1) into the dP^T region once the compute warps have
-            // read dP^T(i) (it overlaps their work on tile i); dK over each half as they
-            // publish it; x_free.  A: dV over each half; then dP^T(i+1) into the S^T region
-            // and SD(i+1).
+            // Two issuing threads.  A issues dP^T and dV, B issues S^T and dK, each committing
+            // its own ready barrier, so that the compute warps can form P^T of tile i+1 from
+            // S^T(i+1) while dP^T(i+1) waits for the end of tile i: dP^T(i+1) overwrites the
+            // region whose P^T / dS^T(i) dV(i) and dK(i) read, so A first waits for B's
+            // x_free commit (after dK(i)).  B, per query tile i: S^T(i+1) into the dP^T(i)
+            // region once every compute warp has read dP^T(i), s_ready; dK over each half as
+            // its dS^T is published; x_free.  A: dV over each half as its P^T is published
+            // (p_full alternates by tile parity: A's wait for tile i may come after the
+            // warpgroup's arrival for tile i+1); then dP^T(i+1) and dp_ready.
             if (wait1(bar(C::BAR_FIXED), 0, abort_flag, lim, kErrMma) && n > 0 &&
                 wait1(bar(C::bar_full(0)), 0, abort_flag, lim, kErrMma)) {
                 tc_fence_after();
                 if (thread_a) {
-                    issue_st(0);  // tile 0's S^T as well, so that SD has one committer
                     issue_dpt(0);
-                    tc_commit(bar(C::BAR_SD));
+                    tc_commit(bar(C::BAR_DPREADY));
                     for (int it = 0; it < n; ++it) {
                         const bool more = it + 1 < n;
-                        const uint32_t ph = it & 1;
-                        if (!wait1(bar(C::bar_ds(0)), ph, abort_flag, lim, kErrMma)) break;
+                        if (!wait1(bar(C::bar_p(0, it)), C::par2(it), abort_flag, lim, kErrMma))
+                            break;
                         tc_fence_after();
                         acc_half(it, 0, 0);
-                        if (!wait1(bar(C::bar_ds(1)), ph, abort_flag, lim, kErrMma)) break;
+                        if (!wait1(bar(C::bar_p(1, it)), C::par2(it), abort_flag, lim, kErrMma))
+                            break;
                         tc_fence_after();
                         acc_half(it, 1, 0);
                         if (more) {
-                            if (!wait1(bar(C::BAR_XFREE), ph, abort_flag, lim, kErrMma)) break;
+                            if (!wait1(bar(C::BAR_XFREE), it & 1, abort_flag, lim, kErrMma)) break;
                             tc_fence_after();
                         }
                         tc_commit(bar(C::bar_empty(it % C::NS)));
                         if (more) {
                             issue_dpt(it + 1);
-                            tc_commit(bar(C::BAR_SD));
+                            tc_commit(bar(C::BAR_DPREADY));
                         }
                     }
                 } else {
+                    issue_st(0);
+                    tc_commit(bar(C::BAR_SREADY));
                     for (int it = 0; it < n; ++it) {
                         const uint32_t ph = it & 1;
                         if (it + 1 < n) {
@@ -896,11 +930,12 @@ __global__ void __launch_bounds__(kThreadsKV, 1) bwd_dkdv_sm100(const __grid_con
                                 break;
                             tc_fence_after();
                             issue_st(it + 1);
+                            tc_commit(bar(C::BAR_SREADY));
                         }
-                        if (!wait1(bar(C::bar_ds(0)), ph, abort_flag, lim, kErrMma)) break;
+                        if (!wait1(bar(C::bar_ds(0, 0)), ph, abort_flag, lim, kErrMma)) break;
                         tc_fence_after();
                         acc_half(it, 0, 1);
-                        if (!wait1(bar(C::bar_ds(1)), ph, abort_flag, lim, kErrMma)) break;
+                        if (!wait1(bar(C::bar_ds(1, 0)), ph, abort_flag, lim, kErrMma)) break;
                         tc_fence_after();
                         acc_half(it, 1, 1);
                         tc_commit(bar(C::BAR_XFREE));
@@ -932,7 +967,9 @@ __global__ void __launch_bounds__(kThreadsKV, 1) bwd_dkdv_sm100(const __grid_con
         for (int it = 0; it < n; ++it) {
             const int slot = it % C::NS;
             const int q0 = (qt0 + it % n_qt) * kBM;
-            if (!wait_warp(bar(C::BAR_SD), it & 1, abort_flag, lim, kErrCompute)) {
+            // P^T first, from S^T alone (the exponentials), then dS^T once dP^T is ready: the
+            // exponentials of this tile overlap dK of the previous one and this tile's dP^T
+            if (!wait_warp(bar(C::BAR_SREADY), it & 1, abort_flag, lim, kErrCompute)) {
                 ok = false;
                 break;
             }
@@ -949,54 +986,85 @@ __global__ void __launch_bounds__(kThreadsKV, 1) bwd_dkdv_sm100(const __grid_con
                 CONTIG ? lo_c <= 64 * c
                        : (my_kpos <= posv[2 * kBM + c] && my_kpos >= posv[2 * kBM + 2 + c]);
             const uint32_t xs = C::st_col(it), yd = C::dpt_col(it);
-            uint32_t pp[32], pd[32];
             // warp-uniform: the TMEM loads below are warp-collective
-            if (__all_sync(0xffffffffu, key_ok && half_visible)) {
+            const bool packed = __all_sync(0xffffffffu, key_ok && half_visible);
+            uint32_t pp[32];
+            uint64_t p2[32];  // the fp32 probabilities as pairs (column 2i low), kept for dS
+            if (packed) {
                 // every query of this half sees every key of the warp: packed pairs
-                uint64_t s2[32], d2[32];
+                uint64_t s2[32];
                 tmem_ld64_pairs(tmem + lane_off + xs + 64 * c, s2);
-                tmem_ld64_pairs(tmem + lane_off + yd + 64 * c, d2);
-                // dP^T is in registers: once both halves are, its region may take S^T(it+1)
-                tc_fence_before();
-                mbar_arrive(bar(C::BAR_DPFREE));
                 const ulonglong2* nl = reinterpret_cast<const ulonglong2*>(rows + 64 * c);
-                const ulonglong2* nd = reinterpret_cast<const ulonglong2*>(rows + kBM + 64 * c);
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
-                    const ulonglong2 a = nl[k], d = nd[k];
-                    p_ds_pair(s2[2 * k], d2[2 * k], sl2x2, a.x, d.x, pp[2 * k], pd[2 * k]);
-                    p_ds_pair(s2[2 * k + 1], d2[2 * k + 1], sl2x2, a.y, d.y, pp[2 * k + 1],
-                              pd[2 * k + 1]);
+                    const ulonglong2 a = nl[k];
+                    pp[2 * k] = p_pair(s2[2 * k], sl2x2, a.x, p2[2 * k]);
+                    pp[2 * k + 1] = p_pair(s2[2 * k + 1], sl2x2, a.y, p2[2 * k + 1]);
                 }
             } else {
-                float s[64], dp[64];
+                float s[64];
                 tmem_ld64(tmem + lane_off + xs + 64 * c, s);
-                tmem_ld64(tmem + lane_off + yd + 64 * c, dp);
-                tc_fence_before();
-                mbar_arrive(bar(C::BAR_DPFREE));
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    float pr2[2], ds2[2];
+                    float pr2[2];
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         const int col = 64 * c + 2 * i + e;
                         const bool vis =
                             key_ok && (CONTIG ? col >= lo_c
                                               : (my_kpos <= posv[col] && my_kpos >= startv[col]));
-                        const float pr = vis ? ex2_approx(s[2 * i + e] * sl2 + rows[col]) : 0.f;
-                        pr2[e] = pr;
-                        ds2[e] = pr * (dp[2 * i + e] + rows[kBM + col]);
+                        pr2[e] = vis ? ex2_approx(s[2 * i + e] * sl2 + rows[col]) : 0.f;
                     }
                     pp[i] = pack_bf16x2(pr2[0], pr2[1]);
+                    p2[i] = f2_pack(pr2[0], pr2[1]);
+                }
+            }
+            // publish P^T of this 64-query half over the S^T columns just read
+            tmem_st32(tmem + lane_off + xs + 64 * c, pp);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(C::bar_p(c, it)));
+
+            if (!wait_warp(bar(C::BAR_DPREADY), it & 1, abort_flag, lim, kErrCompute)) {
+                ok = false;
+                break;
+            }
+            __syncwarp();
+            tc_fence_after();
+            uint32_t pd[32];
+            if (packed) {
+                uint64_t d2[32];
+                tmem_ld64_pairs(tmem + lane_off + yd + 64 * c, d2);
+                // dP^T is in registers: once every warp's is, its region may take S^T(it+1)
+                tc_fence_before();
+                mbar_arrive(bar(C::BAR_DPFREE));
+                const ulonglong2* nd = reinterpret_cast<const ulonglong2*>(rows + kBM + 64 * c);
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const ulonglong2 d = nd[k];
+                    pd[2 * k] = ds_from_p(p2[2 * k], d2[2 * k], d.x);
+                    pd[2 * k + 1] = ds_from_p(p2[2 * k + 1], d2[2 * k + 1], d.y);
+                }
+            } else {
+                float dp[64];
+                tmem_ld64(tmem + lane_off + yd + 64 * c, dp);
+                tc_fence_before();
+                mbar_arrive(bar(C::BAR_DPFREE));
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    float pr2[2], ds2[2];
+                    f2_unpack(p2[i], pr2[0], pr2[1]);
+#pragma unroll
+                    for (int e = 0; e < 2; ++e)
+                        ds2[e] = pr2[e] * (dp[2 * i + e] + rows[kBM + 64 * c + 2 * i + e]);
                     pd[i] = pack_bf16x2(ds2[0], ds2[1]);
                 }
             }
-            // publish this 64-query half over the S^T columns just read
-            tmem_st32(tmem + lane_off + xs + 64 * c, pp);
+            // publish dS^T of this half beside its P^T
             tmem_st32(tmem + lane_off + xs + 64 * c + 32, pd);
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(C::bar_ds(c)));
+            mbar_arrive(bar(C::bar_ds(c, 0)));
         }
         if (ok && n > 0 && wait_warp(bar(C::BAR_ACC), 0, abort_flag, lim, kErrCompute)) {
             __syncwarp();

@@ -21,8 +21,8 @@ namespace {
 // first float4 of O_a and O_b) issued before any arithmetic: the row's addresses do not
 // depend on the LSE values, so a warp keeps four independent loads per lane in flight
 // instead of waiting for the LSEs before it asks for O.
-// FAST: every row index fits in 32 bits, so the row's (b, t, h) come from two
-// invariant-divisor multiplications (by H, then by L) instead of 64-bit divisions, which
+// FAST: every row index fits in 32 bits, so the row's (b, h, t) come from two
+// invariant-divisor multiplications (by L, then by H) instead of 64-bit divisions, which
 // would cost more instructions per row than the row's loads and stores.
 template <bool FAST>
 __global__ void __launch_bounds__(256) lse_merge_kernel(float* __restrict__ o_a,
@@ -44,34 +44,38 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(float* __restrict__ o_a,
     const bool has_c = li < D4;  // this lane owns float4 li of each row
     // Every lane of the warp runs the same number of iterations so that __syncwarp is legal.
     for (long long base = warp_global * rows_per_warp; base < n_rows; base += 2 * step) {
-        long long row[2], li_idx[2] = {0, 0};
+        long long orow[2], li_idx[2] = {0, 0};
         bool active[2];
         float la[2] = {-INFINITY, -INFINITY}, lb[2] = {-INFINITY, -INFINITY};
         float4 x[2], y[2];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-            row[u] = base + u * step + sub;  // row in [B][L][H] order
-            active[u] = row[u] < n_rows;
+            // rows in LSE order [B][H][L]: neighbouring warps read and write neighbouring
+            // LSE entries (one 32-byte sector serves eight rows), while each row of O is one
+            // contiguous D-float segment of the [B][L][H][D] tensor
+            li_idx[u] = base + u * step + sub;
+            active[u] = li_idx[u] < n_rows;
+            orow[u] = 0;
             if (active[u]) {
                 long long h, t, b;
                 if (FAST) {
-                    const uint32_t r = (uint32_t)row[u];
-                    const uint32_t tok = fdiv(r, fH);  // b * L + t
-                    const uint32_t bb = fdiv(tok, fL);
-                    h = r - tok * (uint32_t)H;
-                    t = tok - bb * (uint32_t)L;
+                    const uint32_t r = (uint32_t)li_idx[u];
+                    const uint32_t bh = fdiv(r, fL);  // b * H + h
+                    const uint32_t bb = fdiv(bh, fH);
+                    t = r - bh * (uint32_t)L;
+                    h = bh - bb * (uint32_t)H;
                     b = bb;
                 } else {
-                    h = row[u] % H;
-                    t = (row[u] / H) % L;
-                    b = row[u] / H / L;
+                    t = li_idx[u] % L;
+                    h = (li_idx[u] / L) % H;
+                    b = li_idx[u] / L / H;
                 }
-                li_idx[u] = (b * H + h) * L + t;
+                orow[u] = (b * L + t) * H + h;
                 la[u] = lse_a[li_idx[u]];
                 lb[u] = lse_b[li_idx[u]];
                 if (has_c) {
-                    x[u] = reinterpret_cast<const float4*>(o_a + row[u] * D)[li];
-                    y[u] = __ldg(reinterpret_cast<const float4*>(o_b + row[u] * D) + li);
+                    x[u] = reinterpret_cast<const float4*>(o_a + orow[u] * D)[li];
+                    y[u] = __ldg(reinterpret_cast<const float4*>(o_b + orow[u] * D) + li);
                 }
             }
         }
@@ -88,8 +92,8 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(float* __restrict__ o_a,
                 wb = eb / z;
             }
             if (active[u]) {
-                float4* pa = reinterpret_cast<float4*>(o_a + row[u] * D);
-                const float4* pb = reinterpret_cast<const float4*>(o_b + row[u] * D);
+                float4* pa = reinterpret_cast<float4*>(o_a + orow[u] * D);
+                const float4* pb = reinterpret_cast<const float4*>(o_b + orow[u] * D);
                 if (has_c)
                     pa[li] = make_float4(wa * x[u].x + wb * y[u].x, wa * x[u].y + wb * y[u].y,
                                          wa * x[u].z + wb * y[u].z, wa * x[u].w + wb * y[u].w);

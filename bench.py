@@ -319,12 +319,17 @@ class DistUlyssesPath:
     whole sequence (the attention kernel over the workload's chunk count) -> head->seq
     all-to-all of O.  The total problem is the one-GPU workload's (strong scaling)."""
 
+    @staticmethod
+    def splits(w, world) -> bool:
+        """The workload's query heads and sequence divide over `world` ranks."""
+        return w.H_q % world == 0 and (w.P * w.Lc) % world == 0 and w.G == w.P
+
     def __init__(self, w, device, rank, world):
         import torch
         from sequence_parallelism_attn_b200 import dist as rd, ra
         self.ra, self.rd, self.kind, self.w, self.dev = ra, rd, "ulysses_dist", w, device
         L = w.P * w.Lc
-        if w.H_q % world or L % world or w.G != w.P:
+        if not self.splits(w, world):
             raise ValueError(f"{w.name} does not split over {world} ranks")
         self.world, self.Ls, self.L = world, L // world, L
         self.H_kv_rep = math.lcm(w.H_kv, world)
@@ -577,10 +582,12 @@ def main():
                                 device_id=device)
     peaks, peaks_src = load_peaks()
 
-    if world > 1 and kind == "ulysses":
+    if world > 1 and kind == "ulysses" and DistUlyssesPath.splits(w, world):
         # N GPUs: the Ulysses layer with real all-to-alls between the ranks
         path = DistUlyssesPath(w, device, rank, world)
     else:
+        # one GPU, a workload without an exchange, or heads that do not split over N:
+        # independent replicas
         path = Path(kind, w, device)
     for _ in range(args.warmup):
         path.step()

@@ -119,3 +119,15 @@ def test_reference_arm_backward_times_the_oracle_gradients():
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["config"]["workload"].endswith("_backward")
     assert "gradients" in line["cpu_baseline"]["sample"]
+
+
+def test_multi_gpu_step_splits_heads_or_falls_back():
+    """bench --gpus N runs the Ulysses step across N GPUs when the workload's query heads
+    and sequence divide over N (the driver's 1, 2, 4, 8), otherwise independent replicas."""
+    import bench
+    from sequence_parallelism_attn_b200 import synth
+    w = synth.ULYSSES_128K
+    assert [n for n in (1, 2, 3, 4, 5, 8, 16) if bench.DistUlyssesPath.splits(w, n)] == \
+        [1, 2, 4, 8, 16]
+    # the hybrid workload (head groups fewer than ranks) keeps replicas
+    assert not bench.DistUlyssesPath.splits(synth.USP_128K, 2)

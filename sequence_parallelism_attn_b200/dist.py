@@ -145,17 +145,12 @@ class RingAccumulator:
         self.visited += 1
 
 
-def ring_attn_fwd_dist(q, k, v, causal: bool, scale: float | None = None, group=None,
-                       out=None, lse=None, ops=DeviceOps):
-    """Ring attention across the ranks of `group`: q [B, Lc, H_q, D] is this rank's query
-    chunk, k/v [B, Lc, H_kv, D] its K/V chunk (contiguous), rank i holding tokens
-    i*Lc .. i*Lc+Lc-1 of the sequence.  Returns this rank's (out [B, Lc, H_q, D] fp32,
-    lse [B, H_q, Lc] fp32), equal to attention of its queries over the whole sequence.
-    The chunk received during step s is sent on during step s + 1; two receive buffers
-    alternate, and a buffer is received into only after the step that read it has been
-    enqueued (NCCL's stream waits for it) and its own send has completed."""
+def _ring_exchange(k, v, group, visit):
+    """The ring's exchange loop: visit(j, k_j, v_j) for the chunk held at each step, while
+    the held chunk travels to rank i + 1 and the next arrives from rank i - 1 into the
+    second of two receive buffers.  A buffer is received into only after the step that
+    read it has been enqueued (NCCL's stream waits for it) and its own send has completed."""
     rank, world = _group_info(group)
-    acc = RingAccumulator(q, rank, causal, scale, out, lse, ops)
     bufs = [(torch.empty_like(k), torch.empty_like(v)) for _ in range(2)] if world > 1 else []
     held = (k, v)
     nxt_rank, prv_rank = _peer(group, (rank + 1) % world), _peer(group, (rank - 1) % world)
@@ -172,11 +167,77 @@ def ring_attn_fwd_dist(q, k, v, causal: bool, scale: float | None = None, group=
             except Exception as e:
                 raise ExchangeError(f"ring step {s}: posting the exchange with ranks "
                                     f"{(rank + 1) % world} / {(rank - 1) % world}: {e}") from e
-        acc.visit(j, held[0], held[1])
+        visit(j, held[0], held[1])
         if works:
             _wait(works, f"ring step {s}: chunk from rank {(rank - 1) % world}")
             held = nxt
+
+
+def ring_attn_fwd_dist(q, k, v, causal: bool, scale: float | None = None, group=None,
+                       out=None, lse=None, ops=DeviceOps):
+    """Ring attention across the ranks of `group`: q [B, Lc, H_q, D] is this rank's query
+    chunk, k/v [B, Lc, H_kv, D] its K/V chunk (contiguous), rank i holding tokens
+    i*Lc .. i*Lc+Lc-1 of the sequence.  Returns this rank's (out [B, Lc, H_q, D] fp32,
+    lse [B, H_q, Lc] fp32), equal to attention of its queries over the whole sequence."""
+    rank, _ = _group_info(group)
+    acc = RingAccumulator(q, rank, causal, scale, out, lse, ops)
+    _ring_exchange(k, v, group, acc.visit)
     return acc.out, acc.lse
+
+
+class ZigzagRingAccumulator:
+    """Rank i's causal attention over the zigzag layout's chunks (the load-balanced layout
+    named beside the ring in "Метод контекстного параллелизма Ulysses"; rank i holds the
+    segments i and 2P-1-i of 2P segments of h = Lc/2 tokens).  The two query halves keep
+    separate running results; against rank j's shard (segments j and 2P-1-j, key halves
+    K0 and K1):
+      j == i: half 0 sees K0 causally; half 1 sees K0 wholly and K1 causally;
+      j <  i: both halves see K0 wholly and nothing of K1;
+      j >  i: half 0 sees nothing; half 1 sees K0 and K1 wholly.
+    Every rank does the same work at every step but the first."""
+
+    def __init__(self, q, rank: int, world: int, scale: float | None = None, ops=DeviceOps):
+        B, Lc, H_q, D = q.shape
+        if Lc % 2:
+            raise ValueError("the zigzag layout needs an even chunk length")
+        self.h, self.rank, self.world = Lc // 2, rank, world
+        self.q = (q[:, :self.h], q[:, self.h:])
+        self.acc = tuple(RingAccumulator(qq, 0, False, scale, ops=ops) for qq in self.q)
+
+    def _add(self, half, k, v, causal_diagonal):
+        a = self.acc[half]
+        a.causal = causal_diagonal  # the pair decides: "diagonal" when causal, else "full"
+        a.visit(0, k, v)
+
+    def visit(self, j: int, k, v):
+        K = ((k[:, :self.h], v[:, :self.h]), (k[:, self.h:], v[:, self.h:]))
+        if j == self.rank:
+            self._add(0, *K[0], True)
+            self._add(1, *K[0], False)
+            self._add(1, *K[1], True)
+        elif j < self.rank:
+            self._add(0, *K[0], False)
+            self._add(1, *K[0], False)
+        else:
+            self._add(1, *K[0], False)
+            self._add(1, *K[1], False)
+
+    def result(self):
+        """(out [B, Lc, H_q, D], lse [B, H_q, Lc]) in the shard's token order."""
+        out = torch.cat([self.acc[0].out, self.acc[1].out], dim=1)
+        lse = torch.cat([self.acc[0].lse, self.acc[1].lse], dim=2)
+        return out, lse
+
+
+def ring_attn_fwd_zigzag_dist(q, k, v, scale: float | None = None, group=None, ops=DeviceOps):
+    """Causal ring attention across the ranks of `group` over shards in the zigzag layout:
+    q [B, Lc, H_q, D] and k/v [B, Lc, H_kv, D] are this rank's shard (its segments i and
+    2P-1-i, Lc even).  Returns this rank's (out [B, Lc, H_q, D], lse [B, H_q, Lc]) in shard
+    order, equal to causal attention of its queries over the sequence in natural order."""
+    rank, world = _group_info(group)
+    acc = ZigzagRingAccumulator(q, rank, world, scale, ops)
+    _ring_exchange(k, v, group, acc.visit)
+    return acc.result()
 
 
 def _all_to_all(send, group, what):

@@ -55,6 +55,42 @@ def test_ring_steps_equal_whole_sequence(ra_lib, oracle_mod, P, causal):
         assert eo <= TOL[torch.bfloat16][0] and el <= TOL[torch.bfloat16][1]
 
 
+@pytest.mark.parametrize("B,P,Lc", [(1, 4, 256), (2, 3, 200)])
+def test_zigzag_ring_steps_equal_causal_attention(ra_lib, oracle_mod, B, P, Lc):
+    """Every virtual rank's zigzag accumulator over its ring steps (attention launches on
+    shard halves, merges by ra_lse_merge) equals causal attention over the natural-order
+    sequence, every row; and agrees with the one-launch zigzag kernel on the same shards."""
+    H_q, H_kv, D = 4, 2, 128
+    g = torch.Generator().manual_seed(600 + P)
+    L = P * Lc
+    q = (torch.randn(B, L, H_q, D, generator=g) * 2).to(torch.bfloat16)  # natural order
+    k = torch.randn(B, L, H_kv, D, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, L, H_kv, D, generator=g).to(torch.bfloat16)
+    scale = D ** -0.5
+    want_o, want_l = oracle_mod.attention(f64(q), f64(k), f64(v), scale, True)
+    pos = oracle_mod.zigzag_positions(P, Lc)
+    shard = lambda x, i: x[:, torch.from_numpy(pos[i * Lc:(i + 1) * Lc])].contiguous().cuda()
+    qz = torch.cat([shard(q, i) for i in range(P)], dim=1)  # rank-major zigzag shards
+    kz = torch.stack([shard(k, i) for i in range(P)])
+    vz = torch.stack([shard(v, i) for i in range(P)])
+    one_o, one_l = ra_lib.ring_attn_fwd(qz, kz, vz, True, scale, layout="zigzag")
+    for i in range(P):
+        acc = rd.ZigzagRingAccumulator(shard(q, i), i, P, scale)
+        for j in rd.ring_schedule(i, P):
+            acc.visit(j, shard(k, j), shard(v, j))
+        out, lse = acc.result()
+        assert ra_lib.ra_sync_status() == 0, ra_lib.ra_last_error()
+        p_i = pos[i * Lc:(i + 1) * Lc]
+        eo = max_abs(f64(out), want_o[:, p_i])
+        el = max_abs(f64(lse), want_l[:, :, p_i])
+        print(f"[parity] zigzag ring steps P={P} B={B} rank {i}: max|dO|={eo:.3e} "
+              f"max|dLSE|={el:.3e}")
+        assert eo <= TOL[torch.bfloat16][0] and el <= TOL[torch.bfloat16][1]
+        sl = slice(i * Lc, (i + 1) * Lc)
+        assert max_abs(f64(out), f64(one_o[:, sl])) <= 2e-2
+        assert max_abs(f64(lse), f64(one_l[:, :, sl])) <= 2e-3
+
+
 @pytest.mark.parametrize("B,dtype", [(1, torch.bfloat16), (2, torch.bfloat16),
                                      (2, torch.float32)])
 def test_ulysses_pack_unpack_bit_exact(ra_lib, oracle_mod, B, dtype):

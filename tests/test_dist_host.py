@@ -194,6 +194,33 @@ def test_ring_attention_equals_whole_sequence(world, causal):
         assert errs[0] <= 1e-12 and errs[1] <= 1e-12, (rank, errs)
 
 
+def _zigzag_ring(rank, world, B, Lc, H_q, H_kv, D):
+    from sequence_parallelism_attn_b200 import dist as rd
+    import oracle
+    g = np.random.default_rng(17)
+    L = world * Lc
+    q = g.standard_normal((B, L, H_q, D)) * 2.0   # natural (sequence) order
+    k = g.standard_normal((B, L, H_kv, D))
+    v = g.standard_normal((B, L, H_kv, D))
+    pos = oracle.zigzag_positions(world, Lc)[rank * Lc:(rank + 1) * Lc]  # this shard's tokens
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x[:, pos]))
+    out, lse = rd.ring_attn_fwd_zigzag_dist(t(q), t(k), t(v), 0.3, ops=OracleOps)
+    want_o, want_l = oracle.attention(q, k, v, 0.3, True)
+    return (float(np.abs(out.numpy() - want_o[:, pos]).max()),
+            float(np.abs(lse.numpy() - want_l[:, :, pos]).max()))
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_zigzag_ring_equals_causal_attention(world):
+    """Shards in the zigzag layout (rank i holds segments i and 2P-1-i): each rank's rows
+    equal causal attention over the sequence in natural order (GQA 4:2, B = 2)."""
+    res = run_ranks(world, _zigzag_ring, 2, 6, 4, 2, 8)
+    for rank in range(world):
+        status, errs = res[rank]
+        assert status == "ok", errs
+        assert errs[0] <= 1e-12 and errs[1] <= 1e-12, (rank, errs)
+
+
 # ------------------------------------------------------------------ Ulysses
 def _ulysses(rank, world, B, Lc, H_q, H_kv, D):
     from sequence_parallelism_attn_b200 import dist as rd

@@ -259,7 +259,7 @@ class Path:
                 self.dv = torch.empty_like(self.dk)
                 self.ws = torch.empty((w.B, w.H_q, w.L), dtype=torch.float32, device=device)
                 self.flops = 2.5 * self.flops
-                self.launches_per_step = 3
+                self.launches_per_step = 2  # Delta (and dQ zeroing), then dQ / dK / dV
             self.permute_bytes = 0
             self.in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
             self.out_bytes = self.o.numel() * self.o.element_size()
@@ -639,7 +639,7 @@ def main():
                        "peak": sustained, "unit": "TFLOP/s",
                        "frac": round(attn_tflops / sustained, 4),
                        "traffic": traffic,
-                       "kernel": ("bwd_delta + bwd_dq_sm100 + bwd_dkdv_sm100, D=128"
+                       "kernel": ("bwd_delta + bwd_sm100 (dQ, dK, dV), D=128"
                                   if kind.startswith("attn_bwd") else "attn_fwd_sm100<128>"),
                        "peak_source": f"{peaks_src} bf16_tflops_sustained",
                        "frac_of_burst": round(attn_tflops / peaks.get("bf16_tflops", 1590.0), 4),

@@ -178,16 +178,21 @@ RA_API ra_status ra_ring_attn_fwd_packed(const void* q, const void* const* k_chu
  *   dS_ij = P_ij * (dout_i . v_j - Delta_i)
  *   dq_i = scale * sum_j dS_ij k_j;  dk_j = scale * sum_i dS_ij q_i;  dv_j = sum_i P_ij dout_i
  * with i over the query rows (of every query head sharing the kv head) that see
- * key j.  Computed on the tensor cores: a row reduction for Delta, then dq with
- * the query tile stationary (the chunks in the forward's ring order, causal
- * tiles skipped), then dk, dv with the key tile stationary.
+ * key j.  Computed on the tensor cores: a row reduction for Delta (which also
+ * zeroes dq), then one kernel with the key tile stationary that visits the query
+ * tiles seeing its keys (causal tiles skipped), accumulates dk and dv, and adds
+ * each tile pair's share of dq into dq in global memory (fp32 reduce-adds).
+ * Reproducibility: dk and dv are the same bits on every call with the same
+ * inputs; dq is the same up to the rounding of its fp32 sum, whose order of
+ * additions across key tiles varies from call to call.
  * Arguments
  *   q, k_chunks, v_chunks, P, B, H_q, H_kv, Lc, D, q_bstride, kv_bstride,
  *   scale, causal   exactly as given to ra_ring_attn_fwd (bf16, D in {64,128}).
  *   out        device, bf16, dense [B][P*Lc][H_q][D]: the forward's output.
  *   lse        device, fp32, dense [B][H_q][P*Lc]: the forward's log-sum-exp.
  *   dout       device, bf16, dense [B][P*Lc][H_q][D].
- *   dq         device, fp32, dense [B][P*Lc][H_q][D] (written).
+ *   dq         device, fp32, dense [B][P*Lc][H_q][D] (written; its prior contents
+ *              are never read).
  *   dk_chunks, dv_chunks  host arrays of P device pointers, chunk j fp32 dense
  *              [B][Lc][H_kv][D] (written).
  *   workspace  device, fp32, [B][H_q][P*Lc] scratch owned by the caller (holds

@@ -7,7 +7,7 @@
 // and kernels are used unchanged.
 //
 // Nothing in the scratch has to start at zero: the Delta kernel writes every row that the
-// dQ and dK/dV kernels read, earlier on the same stream.  The one array is shared by every
+// gradient kernel reads, earlier on the same stream.  The one array is shared by every
 // call on a device, so calls that overlap in time (different streams, or different host
 // threads without ordering) race on it.
 #include <cuda_runtime.h>

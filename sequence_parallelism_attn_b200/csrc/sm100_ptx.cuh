@@ -85,6 +85,23 @@ __device__ __forceinline__ void tma_store_5d(const void* tmap, uint32_t src, int
         "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
         : "memory");
 }
+// 4-D tiled reduce-add shared -> global (bulk-group completion): every element of the box is
+// added to the global element in the tensor map's type (fp32 here); elements past the
+// tensor's extent are skipped.  Coordinates are never negative.
+__device__ __forceinline__ void tma_reduce_add_4d(const void* tmap, uint32_t src, int c0, int c1,
+                                                  int c2, int c3) {
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group"
+        " [%0, {%2, %3, %4, %5}], [%1];" ::"l"(reinterpret_cast<uint64_t>(tmap)),
+        "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+                 "r"(d)
+                 : "memory");
+}
 __device__ __forceinline__ void bulk_commit() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -364,6 +381,13 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t smem_addr, uint32_t lbo_
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int b_mn_major) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn_major << 16) |
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// The same with A also MN-major (bit 15): both operands with their M / N dimension
+// contiguous in shared memory.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_ab(int M, int N, int a_mn_major,
+                                                         int b_mn_major) {
+    return idesc_bf16_f32(M, N, b_mn_major) | ((uint32_t)a_mn_major << 15);
 }
 
 }  // namespace ra

@@ -48,7 +48,8 @@ class Sim:
         # from then on every abortable wait returns False (the CTA abort flag)
         self.abort_after, self.aborted, self.steps = abort_after, False, 0
         self.bars, self.mem, self.queues, self.tma = {}, {}, {}, []
-        self.bulk, self.bulk_seq = [], 0  # bulk store groups: (seq, reads, who)
+        self.bulk, self.bulk_seq = [], 0  # bulk store groups: (seq, reads, who, owner)
+        self.bulk_issued = {}  # per owner: sequence numbers of its groups, in issue order
 
     def bar(self, name, count):
         self.bars[name] = Barrier(name, count)
@@ -75,15 +76,20 @@ class Sim:
     def tma_load(self, barrier, region, label):
         self.tma.append((barrier, region, label))
 
-    def bulk_group(self, reads, who):
-        """A committed group of bulk (TMA) stores: it reads its source regions when it
-        executes; groups execute in any order."""
+    def bulk_group(self, reads, who, owner=None):
+        """A committed group of bulk (TMA) stores or reduces, issued by thread `owner`: it
+        reads its source regions when it executes; groups execute in any order."""
         self.bulk_seq += 1
-        self.bulk.append((self.bulk_seq, reads, who))
+        self.bulk.append((self.bulk_seq, reads, who, owner))
+        self.bulk_issued.setdefault(owner, []).append(self.bulk_seq)
 
-    def bulk_read_done_but(self, k):
-        """cp.async.bulk.wait_group.read k: every group but the k most recent has read."""
-        return all(seq > self.bulk_seq - k for seq, _, _ in self.bulk)
+    def bulk_read_done_but(self, k, owner=None):
+        """cp.async.bulk.wait_group.read k by thread `owner` (bulk groups are per thread):
+        every group of that thread but its k most recent has read its source."""
+        mine = [seq for seq, _, _, o in self.bulk if o == owner]
+        issued = self.bulk_issued.get(owner, [])
+        recent = set(issued[-k:]) if k > 0 else set()
+        return all(seq in recent for seq in mine)
 
     def _step_async(self):
         choices = [q for q in self.queues.values() if q]
@@ -95,7 +101,7 @@ class Sim:
             return False
         q = self.rng.choice(choices)
         if q is self.bulk:
-            _, reads, who = self.bulk.pop(self.rng.randrange(len(self.bulk)))
+            _, reads, who, _ = self.bulk.pop(self.rng.randrange(len(self.bulk)))
             for region, want in reads:
                 self.read(region, want, who)
         elif q is self.tma:

@@ -441,39 +441,53 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_sm100(const __grid_constant__
         for (int s = 0; s < C::NS; ++s) armed[s] = -1;
         for_items([&](int it, int h, int q0) -> bool {
             const int slot = it % C::NS;
+            // the item's per-row values into registers first: their global loads are in
+            // flight while the warp waits for a free stage.  Negated: the compute warps add
+            // them (rows past L give P = 0, dS = 0).  Zigzag / packed: the row's sequence
+            // position and sample start (it sees the keys at positions start .. pos; every
+            // key when not causal).
+            const long long lbase = ((long long)b * p.H_q + h) * p.L;
+            float vl[4], vd[4];
+            int vp[4], vs[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const long long row = (long long)q0 + lane + 32 * k;
+                vl[k] = row < p.L ? -(p.lse[lbase + row] * 1.4426950408889634f) : -INFINITY;
+                vd[k] = row < p.L ? -p.delta[lbase + row] : 0.f;
+                vp[k] = INT_MAX;
+                vs[k] = 0;
+                if (!CONTIG && row < p.L && p.causal) {
+                    const int ri = (int)row;  // L <= 2^30
+                    vp[k] = (int)shard_pos(LAYOUT == kLayoutZigzag ? 1 : 0, p.P, p.Lc, ri / p.Lc,
+                                           ri % p.Lc);
+                    if (LAYOUT == kLayoutPacked) vs[k] = sample_start(p, b, ri);
+                }
+            }
             if (it >= C::NS &&
                 !wait_warp(bar(C::bar_empty(slot)), ((it / C::NS) - 1) & 1, abort_flag, lim, kErrLoad))
                 return false;
             const uint32_t st = stage(it);
             if (lane == 0) {
                 mbar_arrive_expect_tx(bar(C::bar_full(slot)), 2 * C::TILE);
-                for (int kb = 0; kb < C::NKB; ++kb) {
+                for (int kb = 0; kb < C::NKB; ++kb)
                     tma_load_4d(st + kb * C::BLK, &p.tm_q, bar(C::bar_full(slot)), kb * 64, h, q0, b);
+                for (int kb = 0; kb < C::NKB; ++kb)
                     tma_load_4d(st + C::TILE + kb * C::BLK, &p.tm_do, bar(C::bar_full(slot)), kb * 64, h, q0, b);
-                }
             }
             float* rows = rows_of(it);
-            const long long lbase = ((long long)b * p.H_q + h) * p.L;
-            int pmin0 = INT_MAX, pmin1 = INT_MAX, smax0 = 0, smax1 = 0;
-            for (int r = lane; r < kBM; r += 32) {
-                const long long row = (long long)q0 + r;
-                rows[r] = row < p.L ? -(p.lse[lbase + row] * 1.4426950408889634f) : -INFINITY;
-                rows[kBM + r] = row < p.L ? -p.delta[lbase + row] : 0.f;
-                if (!CONTIG) {
-                    int pos = INT_MAX, start = 0;
-                    if (row < p.L && p.causal) {
-                        const int ri = (int)row;
-                        pos = (int)shard_pos(LAYOUT == kLayoutZigzag ? 1 : 0, p.P, p.Lc,
-                                             ri / p.Lc, ri % p.Lc);
-                        if (LAYOUT == kLayoutPacked) start = sample_start(p, b, (int)row);
-                    }
-                    reinterpret_cast<int*>(rows)[2 * kBM + r] = pos;
-                    reinterpret_cast<int*>(rows)[3 * kBM + r] = start;
-                    if (r < kBM / 2) { pmin0 = min(pmin0, pos); smax0 = max(smax0, start); }
-                    else { pmin1 = min(pmin1, pos); smax1 = max(smax1, start); }
-                }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                rows[lane + 32 * k] = vl[k];
+                rows[kBM + lane + 32 * k] = vd[k];
             }
             if (!CONTIG) {
+                int pmin0 = min(vp[0], vp[1]), pmin1 = min(vp[2], vp[3]);
+                int smax0 = max(vs[0], vs[1]), smax1 = max(vs[2], vs[3]);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    reinterpret_cast<int*>(rows)[2 * kBM + lane + 32 * k] = vp[k];
+                    reinterpret_cast<int*>(rows)[3 * kBM + lane + 32 * k] = vs[k];
+                }
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1) {
                     pmin0 = min(pmin0, __shfl_xor_sync(0xffffffffu, pmin0, off));

@@ -60,9 +60,12 @@ def _load():
     lib.ora_packed_lower_bounds.argtypes = [P, i32, i64, P]
     lib.ora_attention_backward_rows.argtypes = [P, P, P, P, i32, i64, i32, i32, i32, f64, i32, P,
                                                 P, i64, P, P, P, i64, P, P, P, P, P, P, i32]
+    lib.ora_attention_backward_pair.argtypes = [P, P, P, P, P, P, i32, i64, i64, i32, i32, i32,
+                                                f64, i32, P, P, P, i32]
     for f in ("ora_attention", "ora_attention_rows", "ora_ring_attention", "ora_lse_merge",
               "ora_seq2head", "ora_head2seq", "ora_zigzag_positions", "ora_packed_lower_bounds",
-              "ora_attention_backward", "ora_attention_backward_rows"):
+              "ora_attention_backward", "ora_attention_backward_rows",
+              "ora_attention_backward_pair"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -107,6 +110,26 @@ def attention_backward(q, k, v, dout, scale: float, causal: bool, nthreads: int 
                                         D, float(scale), int(bool(causal)), _ptr(dq), _ptr(dk),
                                         _ptr(dv), nthreads)
     _check(rc, "attention_backward")
+    return dq, dk, dv
+
+
+def attention_backward_pair(q, k, v, out, lse, dout, scale: float, causal: bool,
+                            nthreads: int = 0):
+    """One ring step's share of the gradients: queries q [B,Lq,H_q,D] (with the forward's
+    final out [B,Lq,H_q,D] and lse [B,H_q,Lq] over the whole sequence, and dout) against the
+    keys of one chunk k/v [B,Lk,H_kv,D]; causal: the chunk's own keys (Lq == Lk), key j
+    seen by query i only when j <= i.  Returns (dq [B,Lq,H_q,D], dk, dv [B,Lk,H_kv,D])."""
+    q, k, v, out, lse, dout = _f64(q), _f64(k), _f64(v), _f64(out), _f64(lse), _f64(dout)
+    B, Lq, H_q, D = q.shape
+    _, Lk, H_kv, _ = k.shape
+    assert k.shape == (B, Lk, H_kv, D) and v.shape == k.shape
+    assert out.shape == q.shape and dout.shape == q.shape and lse.shape == (B, H_q, Lq)
+    dq, dk, dv = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+    rc = _load().ora_attention_backward_pair(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                             _ptr(dout), B, Lq, Lk, H_q, H_kv, D, float(scale),
+                                             int(bool(causal)), _ptr(dq), _ptr(dk), _ptr(dv),
+                                             nthreads)
+    _check(rc, "attention_backward_pair")
     return dq, dk, dv
 
 

@@ -366,6 +366,80 @@ int ora_attention_backward(const double* q, const double* k, const double* v,
     return 0;
 }
 
+// One ring step's share of the gradients: the query rows of one chunk (Lq tokens) against the
+// keys of one chunk (Lk tokens), with the softmax statistics of the WHOLE sequence given --
+// out and lse are the forward's final output rows and log-sum-exps of these queries (the
+// ring backward of "Как работает sequence parallelism в контексте LLM?", section 5, carried
+// to the gradient: each step reuses the final LSE instead of recomputing a softmax).
+//   P_ij = exp(scale q_i.k_j - lse_i),  Delta_i = dout_i . out_i,
+//   dS_ij = P_ij (dout_i . v_j - Delta_i),
+//   dq_i = scale sum_j dS_ij k_j,  dk_j = scale sum_i dS_ij q_i,  dv_j = sum_i P_ij dout_i
+// over the pairs (i, j) the step attends: every pair, or with causal (the chunk's own keys,
+// Lq == Lk) only j <= i.  q, out, dout [B][Lq][H_q][D], lse [B][H_q][Lq], k, v
+// [B][Lk][H_kv][D]; dq [B][Lq][H_q][D], dk, dv [B][Lk][H_kv][D] are written.  Summed over
+// the chunks of the sequence, the shares are the gradients of ora_attention_backward.
+int ora_attention_backward_pair(const double* q, const double* k, const double* v,
+                                const double* out, const double* lse, const double* dout, int B,
+                                long long Lq, long long Lk, int H_q, int H_kv, int D,
+                                double scale, int causal, double* dq, double* dk, double* dv,
+                                int nthreads) {
+    if (B < 1 || Lq < 1 || Lk < 1 || H_q < 1 || H_kv < 1 || D < 1 || H_q % H_kv != 0) return 1;
+    if (causal && Lq != Lk) return 1;
+    const int group = H_q / H_kv;
+    auto qoff = [&](int b, long long t, int h) { return (((long long)b * Lq + t) * H_q + h) * D; };
+    auto koff = [&](int b, long long t, int g) { return (((long long)b * Lk + t) * H_kv + g) * D; };
+    auto dot = [&](const double* a, const double* c) {
+        double r = 0.0;
+        for (int d = 0; d < D; ++d) r += a[d] * c[d];
+        return r;
+    };
+    auto delta = [&](int b, long long t, int h) { return dot(dout + qoff(b, t, h), out + qoff(b, t, h)); };
+    auto lse_of = [&](int b, long long t, int h) { return lse[((long long)b * H_q + h) * Lq + t]; };
+    // dQ per query row
+    const long long n_rows = (long long)B * Lq * H_q;
+    parallel_for(n_rows, nthreads, [&](long long row) {
+        const int h = (int)(row % H_q);
+        const long long t = (row / H_q) % Lq;
+        const int b = (int)(row / H_q / Lq), g = h / group;
+        const double* qv = q + qoff(b, t, h);
+        const double* dov = dout + qoff(b, t, h);
+        const double dl = delta(b, t, h), l = lse_of(b, t, h);
+        double* dqv = dq + qoff(b, t, h);
+        for (int d = 0; d < D; ++d) dqv[d] = 0.0;
+        const long long jend = causal ? t + 1 : Lk;
+        for (long long j = 0; j < jend; ++j) {
+            const double* kj = k + koff(b, j, g);
+            const double p = std::exp(scale * dot(qv, kj) - l);
+            const double ds = p * (dot(dov, v + koff(b, j, g)) - dl);
+            for (int d = 0; d < D; ++d) dqv[d] += scale * ds * kj[d];
+        }
+    });
+    // dK, dV per key row, summed over the query heads of its group
+    const long long n_keys = (long long)B * Lk * H_kv;
+    parallel_for(n_keys, nthreads, [&](long long kr) {
+        const int g = (int)(kr % H_kv);
+        const long long j = (kr / H_kv) % Lk;
+        const int b = (int)(kr / H_kv / Lk);
+        const double* kj = k + koff(b, j, g);
+        const double* vj = v + koff(b, j, g);
+        double* dkv = dk + koff(b, j, g);
+        double* dvv = dv + koff(b, j, g);
+        for (int d = 0; d < D; ++d) dkv[d] = dvv[d] = 0.0;
+        for (int h = g * group; h < (g + 1) * group; ++h)
+            for (long long t = causal ? j : 0; t < Lq; ++t) {
+                const double* qv = q + qoff(b, t, h);
+                const double* dov = dout + qoff(b, t, h);
+                const double p = std::exp(scale * dot(qv, kj) - lse_of(b, t, h));
+                const double ds = p * (dot(dov, vj) - delta(b, t, h));
+                for (int d = 0; d < D; ++d) {
+                    dkv[d] += scale * ds * qv[d];
+                    dvv[d] += p * dov[d];
+                }
+            }
+    });
+    return 0;
+}
+
 // The same gradients for a sample of rows, at sizes where every row is too slow: dQ of
 // the query rows (qb, qt, qh) and dK, dV of the key rows (kb, kt, kg).  Tokens are given
 // in storage order; `pos` (NULL: pos[t] = t) gives the sequence position of each stored

@@ -690,3 +690,60 @@ def test_backward_rows_invalid_arguments(oracle_mod):
     with pytest.raises(ValueError):
         oracle_mod.attention_backward_rows(z, z, z, z, 1.0, True, ([0], [0], [0]), ([], [], []),
                                            positions=[0, 1, 1, 3])
+
+
+# ---------------------------------------------------------------- one ring step's gradients
+# The ring backward reuses the forward's final LSE ("Как работает sequence parallelism в
+# контексте LLM?", section 5, taken to the gradient): each step's share is pinned by summing
+# the shares of every chunk pair and comparing with the whole-sequence gradients (pinned
+# against torch autograd above), by the one-chunk case, and by a closed form.
+
+def _pair_shares(oracle_mod, q, k, v, dout, P, scale, causal):
+    """Sum over every (query chunk i, key chunk j) pair of the oracle's one-step shares, with
+    the whole sequence's out / lse; causal pairs: j < i whole, j == i causal, j > i none."""
+    B, L, H_q, D = q.shape
+    Lc = L // P
+    out, lse = oracle_mod.attention(q, k, v, scale, causal)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for i in range(P):
+        qi = slice(i * Lc, (i + 1) * Lc)
+        for j in range(P):
+            if causal and j > i:
+                continue
+            kj = slice(j * Lc, (j + 1) * Lc)
+            a, b_, c = oracle_mod.attention_backward_pair(
+                q[:, qi], k[:, kj], v[:, kj], out[:, qi], lse[:, :, qi], dout[:, qi], scale,
+                causal and j == i)
+            dq[:, qi] += a
+            dk[:, kj] += b_
+            dv[:, kj] += c
+    return dq, dk, dv
+
+
+@pytest.mark.parametrize("P,causal", [(1, True), (3, True), (4, False), (3, False)])
+def test_backward_pair_shares_sum_to_whole_sequence(oracle_mod, P, causal):
+    B, Lc, H_q, H_kv, D = 2, 5, 4, 2, 8
+    L = P * Lc
+    q, k, v = rnd((B, L, H_q, D), 110, 1.5), rnd((B, L, H_kv, D), 111), rnd((B, L, H_kv, D), 112)
+    dout = rnd((B, L, H_q, D), 113)
+    got = _pair_shares(oracle_mod, q, k, v, dout, P, 0.41, causal)
+    want = oracle_mod.attention_backward(q, k, v, dout, 0.41, causal)
+    for g, w in zip(got, want):
+        np.testing.assert_allclose(g, w, atol=1e-12)
+
+
+def test_backward_pair_one_query_one_key_closed_form(oracle_mod):
+    """One query, one key: P = 1, so dS = dO.v - dO.O = 0 (O = v): dq = dk = 0, dv = dO."""
+    q, k, v = rnd((1, 1, 2, 4), 114), rnd((1, 1, 1, 4), 115), rnd((1, 1, 1, 4), 116)
+    dout = rnd((1, 1, 2, 4), 117)
+    out, lse = oracle_mod.attention(q, k, v, 0.7, True)
+    dq, dk, dv = oracle_mod.attention_backward_pair(q, k, v, out, lse, dout, 0.7, True)
+    assert np.abs(dq).max() < 1e-15 and np.abs(dk).max() < 1e-15
+    np.testing.assert_allclose(dv[0, 0, 0], dout[0, 0].sum(axis=0), atol=1e-15)
+
+
+def test_backward_pair_rejects_causal_between_unequal_chunks(oracle_mod):
+    z, zl = np.zeros((1, 4, 2, 8)), np.zeros((1, 2, 4))
+    with pytest.raises(ValueError):
+        oracle_mod.attention_backward_pair(z, np.zeros((1, 3, 2, 8)), np.zeros((1, 3, 2, 8)), z,
+                                           zl, z, 1.0, True)

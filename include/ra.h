@@ -211,6 +211,30 @@ RA_API ra_status ra_ring_attn_bwd(const void* q, const void* const* k_chunks,
                                   float* workspace, void* stream);
 
 /*
+ * ra_ring_attn_bwd_accumulate -- ra_ring_attn_bwd that adds this call's gradients into dq,
+ * dk_chunks and dv_chunks instead of overwriting them.  It is the per-step call of a ring
+ * backward across devices ([SP-QA] section 5, carried to the gradient): each step adds the
+ * share of one K/V chunk, computed with the forward's FINAL out and lse (those of the whole
+ * sequence), into the query chunk's dq and into the dk, dv accumulators that travel with
+ * the K/V chunk; summed over the chunks, the shares are the gradients.
+ * Arguments as ra_ring_attn_bwd, except: dq, dk_chunks, dv_chunks hold valid fp32 values on
+ * entry (zeros, or earlier shares) and receive the sums.  With causal = 1 the call is one
+ * chunk's own (diagonal) step; a wholly visible chunk is causal = 0.  out and lse are the
+ * forward's results over the whole sequence for these query rows.
+ * Reproducibility: as ra_ring_attn_bwd (dk, dv: fixed order; dq: the order of its fp32
+ * additions across key tiles varies).
+ * Errors: as ra_ring_attn_bwd.
+ */
+RA_API ra_status ra_ring_attn_bwd_accumulate(const void* q, const void* const* k_chunks,
+                                             const void* const* v_chunks, const void* out,
+                                             const float* lse, const void* dout, int P, int B,
+                                             int H_q, int H_kv, int Lc, int D,
+                                             long long q_bstride, long long kv_bstride,
+                                             float scale, int causal, float* dq,
+                                             float* const* dk_chunks, float* const* dv_chunks,
+                                             float* workspace, void* stream);
+
+/*
  * ra_ring_attn_bwd_zigzag -- ra_ring_attn_bwd for shards in the zigzag layout: the
  * gradients of ra_ring_attn_fwd_zigzag.  The same definition with every token at its
  * sequence position (the layout of ra_ring_attn_fwd_zigzag); dq, dk_chunks and

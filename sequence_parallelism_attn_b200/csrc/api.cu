@@ -147,7 +147,7 @@ static ra_status ring_attn_bwd(const void* q, const void* const* k_chunks,
                                long long q_bstride, long long kv_bstride, float scale, int causal,
                                float* dq, float* const* dk_chunks, float* const* dv_chunks,
                                float* workspace, void* stream, int zigzag,
-                               const int* position_ids) {
+                               const int* position_ids, int accumulate = 0) {
     if (P < 1 || P > RA_MAX_P) return fail(RA_ERR_INVALID, "P must be in [1, RA_MAX_P]");
     if (zigzag && Lc % 2 != 0)
         return fail(RA_ERR_INVALID, "the zigzag layout needs an even chunk length Lc");
@@ -201,6 +201,7 @@ static ra_status ring_attn_bwd(const void* q, const void* const* k_chunks,
     a.workspace = workspace;
     a.zigzag = zigzag;
     a.pid = position_ids;
+    a.accumulate = accumulate;
     a.stream = (cudaStream_t)stream;
     const char* why = "launch failed";
     cudaError_t e = ra::launch_attn_bwd_sm100(a, g_wait_limit_ns.load(), &why);
@@ -217,6 +218,18 @@ ra_status ra_ring_attn_bwd(const void* q, const void* const* k_chunks, const voi
     return ring_attn_bwd(q, k_chunks, v_chunks, out, lse, dout, P, B, H_q, H_kv, Lc, D, q_bstride,
                          kv_bstride, scale, causal, dq, dk_chunks, dv_chunks, workspace, stream, 0,
                          nullptr);
+}
+
+ra_status ra_ring_attn_bwd_accumulate(const void* q, const void* const* k_chunks,
+                                      const void* const* v_chunks, const void* out,
+                                      const float* lse, const void* dout, int P, int B, int H_q,
+                                      int H_kv, int Lc, int D, long long q_bstride,
+                                      long long kv_bstride, float scale, int causal, float* dq,
+                                      float* const* dk_chunks, float* const* dv_chunks,
+                                      float* workspace, void* stream) {
+    return ring_attn_bwd(q, k_chunks, v_chunks, out, lse, dout, P, B, H_q, H_kv, Lc, D, q_bstride,
+                         kv_bstride, scale, causal, dq, dk_chunks, dv_chunks, workspace, stream, 0,
+                         nullptr, 1);
 }
 
 ra_status ra_ring_attn_bwd_zigzag(const void* q, const void* const* k_chunks,

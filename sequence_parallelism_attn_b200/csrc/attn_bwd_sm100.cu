@@ -67,6 +67,7 @@ struct __align__(64) BwdParams {
     int zigzag;       // shards in the zigzag layout
     int position_order;  // zigzag, causal, Lc/2 a multiple of 128: grids by sequence position
     const int* pid;   // packed samples: position_ids [B][L] (else null)
+    int accumulate;   // dK, dV added to the values in memory (dQ: not zeroed by Delta)
     float scale, scale_log2;
     unsigned long long wait_limit_ns;
 };
@@ -241,14 +242,14 @@ template <int D>
 __global__ void __launch_bounds__(256) bwd_delta_kernel(const uint16_t* __restrict__ out,
                                                         const uint16_t* __restrict__ dout,
                                                         float* __restrict__ delta,
-                                                        float* __restrict__ dq, int B, int L,
-                                                        int H) {
+                                                        float* __restrict__ dq, int zero_dq,
+                                                        int B, int L, int H) {
     const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= (long long)B * L * H) return;
     const uint16_t* o = out + row * D;
     const uint16_t* g = dout + row * D;
-    if (4 * lane < D)
+    if (zero_dq && 4 * lane < D)
         reinterpret_cast<float4*>(dq + row * D)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
     float acc = 0.f;
 #pragma unroll
@@ -825,14 +826,23 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_sm100(const __grid_constant__
                 if (key_ok) {
                     float4* dst = reinterpret_cast<float4*>(outp + orow + cb * 32);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        dst[i] = make_float4(__uint_as_float(o[4 * i]) * mul,
-                                             __uint_as_float(o[4 * i + 1]) * mul,
-                                             __uint_as_float(o[4 * i + 2]) * mul,
-                                             __uint_as_float(o[4 * i + 3]) * mul);
+                    for (int i = 0; i < 8; ++i) {
+                        float4 r = make_float4(__uint_as_float(o[4 * i]) * mul,
+                                               __uint_as_float(o[4 * i + 1]) * mul,
+                                               __uint_as_float(o[4 * i + 2]) * mul,
+                                               __uint_as_float(o[4 * i + 3]) * mul);
+                        if (p.accumulate) {  // this CTA alone owns the key's row
+                            const float4 was = dst[i];
+                            r.x += was.x;
+                            r.y += was.y;
+                            r.z += was.z;
+                            r.w += was.w;
+                        }
+                        dst[i] = r;
+                    }
                 }
             }
-        } else if (ok && n == 0 && key_ok) {
+        } else if (ok && n == 0 && key_ok && !p.accumulate) {  // no query sees the key
             const long long orow = (((long long)b * p.Lc + t * kBN + key_t) * p.H_kv + g) * D;
             float* outp = c ? p.dk[j] : p.dv[j];
             for (int i = 0; i < D; ++i) outp[orow + i] = 0.f;
@@ -919,7 +929,8 @@ cudaError_t launch_bwd_d(const BwdParams& p, const AttnBwdArgs& a, const char** 
     const int layout = p.pid ? kLayoutPacked : (p.zigzag ? kLayoutZigzag : kLayoutContiguous);
     const long long rows = (long long)a.B * p.L * a.H_q;
     bwd_delta_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, a.stream>>>(
-        (const uint16_t*)a.out, (const uint16_t*)a.dout, a.workspace, a.dq, a.B, p.L, a.H_q);
+        (const uint16_t*)a.out, (const uint16_t*)a.dout, a.workspace, a.dq, !a.accumulate, a.B,
+        p.L, a.H_q);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const long long grid_k = (long long)a.B * a.H_kv * a.P * p.ntc;
@@ -964,6 +975,7 @@ cudaError_t launch_attn_bwd_sm100(const AttnBwdArgs& a, unsigned long long wait_
     p.zigzag = a.zigzag;
     p.position_order = a.zigzag && a.causal && (a.Lc / 2) % kBM == 0;
     p.pid = a.pid;
+    p.accumulate = a.accumulate;
     p.group = a.H_q / a.H_kv;
     p.n_qblocks = (int)((L + kBM - 1) / kBM);
     p.ntc = (a.Lc + kBN - 1) / kBN;

@@ -58,6 +58,7 @@ struct AttnBwdArgs {
     float* workspace;             // [B][H_q][P*Lc] fp32 (rowsum(dO * O))
     int zigzag = 0;               // shards in the zigzag layout
     const int* pid = nullptr;     // packed samples: position_ids [B][P*Lc] (causal), else null
+    int accumulate = 0;           // add into dq, dk, dv instead of overwriting them
     cudaStream_t stream;
 };
 

@@ -19,6 +19,10 @@ the P received token blocks in source-rank order (a view when B = 1).  head->seq
 inverse.  No kernel reads another GPU's memory: every remote block lands in this GPU's
 own buffers through NCCL before a kernel touches it.
 
+The ring backward (ring_attn_bwd_dist) moves each K/V chunk the same way, with fp32 dK, dV
+accumulators that every rank adds its share into before passing them on; the last pass
+returns them to the chunk's own rank.
+
 Every rank takes the same collective steps in the same order.  A peer that leaves between
 steps ends the next exchange with an error (the process group's timeout bounds the wait),
 raised here as ExchangeError naming the step and the peers.
@@ -60,6 +64,14 @@ class DeviceOps:
     def merge(o_a, lse_a, o_b, lse_b):
         from . import ra
         ra.ra_lse_merge(o_a, lse_a, o_b, lse_b)
+
+    @staticmethod
+    def attend_bwd(q, k, v, out, lse, dout, causal_diagonal, scale, dq, dk, dv):
+        """Add the gradient share of (these queries, one K/V chunk) into dq, dk, dv, with the
+        forward's final out and lse (ra_ring_attn_bwd_accumulate)."""
+        from . import ra
+        ra.ring_attn_bwd(q, k.unsqueeze(0), v.unsqueeze(0), out, lse, dout, causal_diagonal,
+                         scale, dq=dq, dk=dk.unsqueeze(0), dv=dv.unsqueeze(0), accumulate=True)
 
     @staticmethod
     def seq2head_pack(x, H_out, P):
@@ -183,6 +195,72 @@ def ring_attn_fwd_dist(q, k, v, causal: bool, scale: float | None = None, group=
     acc = RingAccumulator(q, rank, causal, scale, out, lse, ops)
     _ring_exchange(k, v, group, acc.visit)
     return acc.out, acc.lse
+
+
+def ring_attn_bwd_dist(q, k, v, out, lse, dout, causal: bool, scale: float | None = None,
+                       group=None, ops=DeviceOps):
+    """The backward of ring_attn_fwd_dist across the ranks of `group`: q, dout and out
+    [B, Lc, H_q, D] are this rank's query chunk, its output gradient and the forward's
+    output (bf16 on the GPU), lse [B, H_q, Lc] the forward's log-sum-exps over the whole
+    sequence, k/v [B, Lc, H_kv, D] this rank's K/V chunk.  Returns (dq [B, Lc, H_q, D],
+    dk, dv [B, Lc, H_kv, D]) in fp32: the gradients of the loss with respect to this rank's
+    chunks.
+
+    The K/V chunks travel the ring as in the forward (rank i holds chunk (i - s) mod P at
+    step s, the next one arriving while the step computes), and each carries fp32 dK, dV
+    accumulators: rank i adds the share of its queries against the held chunk into dq and
+    into those accumulators (one ra_ring_attn_bwd_accumulate, with the forward's final LSE),
+    then passes them on with the chunk.  After P steps every chunk's accumulators have met
+    every query chunk and the last pass lands them on the chunk's own rank.  Causal: chunk
+    pairs j > i add nothing, though the chunk and its accumulators still travel.  The
+    accumulators move after the step that adds into them (P passes, each after its step's
+    computation); the K/V chunks move during it (P - 1 passes)."""
+    rank, world = _group_info(group)
+    B, Lc, H_q, D = q.shape
+    scale = D ** -0.5 if scale is None else scale
+    gdt = torch.float64 if q.dtype == torch.float64 else torch.float32
+    dq = torch.zeros(q.shape, dtype=gdt, device=q.device)
+    acc = (torch.zeros(k.shape, dtype=gdt, device=k.device),
+           torch.zeros(v.shape, dtype=gdt, device=v.device))
+    if world > 1:
+        kv_bufs = [(torch.empty_like(k), torch.empty_like(v)) for _ in range(2)]
+        acc_bufs = [(torch.empty_like(acc[0]), torch.empty_like(acc[1])) for _ in range(2)]
+    held = (k, v)
+    nxt_rank, prv_rank = _peer(group, (rank + 1) % world), _peer(group, (rank - 1) % world)
+    for s, j in enumerate(ring_schedule(rank, world)):
+        works = []
+        if s < world - 1:
+            nxt = kv_bufs[s % 2]
+            p2p = [dist.P2POp(dist.isend, held[0], nxt_rank, group),
+                   dist.P2POp(dist.isend, held[1], nxt_rank, group),
+                   dist.P2POp(dist.irecv, nxt[0], prv_rank, group),
+                   dist.P2POp(dist.irecv, nxt[1], prv_rank, group)]
+            try:
+                works = dist.batch_isend_irecv(p2p)
+            except Exception as e:
+                raise ExchangeError(f"ring backward step {s}: posting the K/V exchange with "
+                                    f"ranks {(rank + 1) % world} / {(rank - 1) % world}: {e}") from e
+        kind = chunk_pair(rank, j, causal)
+        if kind != "skip":
+            ops.attend_bwd(q, held[0], held[1], out, lse, dout, kind == "diagonal", scale, dq,
+                           acc[0], acc[1])
+        if world > 1:  # the held chunk's accumulators move on; the next chunk's arrive
+            racc = acc_bufs[s % 2]
+            p2p = [dist.P2POp(dist.isend, acc[0], nxt_rank, group),
+                   dist.P2POp(dist.isend, acc[1], nxt_rank, group),
+                   dist.P2POp(dist.irecv, racc[0], prv_rank, group),
+                   dist.P2POp(dist.irecv, racc[1], prv_rank, group)]
+            try:
+                awork = dist.batch_isend_irecv(p2p)
+            except Exception as e:
+                raise ExchangeError(f"ring backward step {s}: posting the dK/dV exchange: "
+                                    f"{e}") from e
+            _wait(awork, f"ring backward step {s}: dK/dV from rank {(rank - 1) % world}")
+            acc = racc
+        if works:
+            _wait(works, f"ring backward step {s}: chunk from rank {(rank - 1) % world}")
+            held = nxt
+    return dq, acc[0], acc[1]
 
 
 class ZigzagRingAccumulator:

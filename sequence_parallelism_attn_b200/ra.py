@@ -20,7 +20,7 @@ RA_BF16, RA_FP32 = 0, 1
 RA_MAX_P = 64
 EXPORTED = ("ra_ring_attn_fwd", "ra_ring_attn_fwd_zigzag", "ra_ring_attn_fwd_packed",
             "ra_ring_attn_bwd", "ra_ring_attn_bwd_zigzag", "ra_ring_attn_bwd_packed",
-            "ra_ring_attn_bwd_static",
+            "ra_ring_attn_bwd_static", "ra_ring_attn_bwd_accumulate",
             "ra_lse_merge", "ra_ulysses_seq2head", "ra_ulysses_head2seq",
             "ra_ulysses_seq2head_grouped", "ra_ulysses_head2seq_grouped",
             "ra_sync_status", "ra_last_error", "ra_set_wait_limit_ns", "ra_debug_inject_stall",
@@ -53,6 +53,7 @@ def load() -> ctypes.CDLL:
                                      i64, f32, i32, vp, vp, vp, vp, vp]
     lib.ra_ring_attn_bwd_static.argtypes = lib.ra_ring_attn_bwd.argtypes[:19] + [vp]
     lib.ra_ring_attn_bwd_zigzag.argtypes = lib.ra_ring_attn_bwd.argtypes
+    lib.ra_ring_attn_bwd_accumulate.argtypes = lib.ra_ring_attn_bwd.argtypes
     lib.ra_ring_attn_bwd_packed.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
                                             i32, i64, i64, f32, vp, vp, vp, vp, vp]
     lib.ra_ring_attn_fwd_packed.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i64, i64,
@@ -65,7 +66,7 @@ def load() -> ctypes.CDLL:
     lib.ra_sync_status.argtypes = [vp]
     for f in ("ra_ring_attn_fwd", "ra_ring_attn_fwd_zigzag", "ra_ring_attn_fwd_packed",
               "ra_ring_attn_bwd", "ra_ring_attn_bwd_zigzag", "ra_ring_attn_bwd_packed",
-              "ra_ring_attn_bwd_static", "ra_lse_merge",
+              "ra_ring_attn_bwd_static", "ra_ring_attn_bwd_accumulate", "ra_lse_merge",
               "ra_ulysses_seq2head", "ra_ulysses_head2seq", "ra_ulysses_seq2head_grouped",
               "ra_ulysses_head2seq_grouped", "ra_sync_status"):
         getattr(lib, f).restype = ctypes.c_int
@@ -155,6 +156,17 @@ def ra_ring_attn_bwd_zigzag(q_ptr, k_ptrs, v_ptrs, out_ptr, lse_ptr, dout_ptr, P
                                           arr(*dv_ptrs), ws_ptr, stream))
 
 
+def ra_ring_attn_bwd_accumulate(q_ptr, k_ptrs, v_ptrs, out_ptr, lse_ptr, dout_ptr, P, B, H_q,
+                                H_kv, Lc, D, q_bstride, kv_bstride, scale, causal, dq_ptr, dk_ptrs,
+                                dv_ptrs, ws_ptr, stream):
+    """The backward C entry point that adds into dq / dk / dv (raw pointers)."""
+    arr = ctypes.c_void_p * P
+    _check(load().ra_ring_attn_bwd_accumulate(q_ptr, arr(*k_ptrs), arr(*v_ptrs), out_ptr,
+                                              lse_ptr, dout_ptr, P, B, H_q, H_kv, Lc, D,
+                                              q_bstride, kv_bstride, scale, int(causal), dq_ptr,
+                                              arr(*dk_ptrs), arr(*dv_ptrs), ws_ptr, stream))
+
+
 def ra_ring_attn_bwd_packed(q_ptr, k_ptrs, v_ptrs, pid_ptr, out_ptr, lse_ptr, dout_ptr, P, B, H_q,
                             H_kv, Lc, D, q_bstride, kv_bstride, scale, dq_ptr, dk_ptrs, dv_ptrs,
                             ws_ptr, stream):
@@ -183,16 +195,21 @@ def ring_attn_bwd(q: torch.Tensor, k_chunks: torch.Tensor, v_chunks: torch.Tenso
                   scale: float | None = None, dq: torch.Tensor | None = None,
                   dk: torch.Tensor | None = None, dv: torch.Tensor | None = None,
                   workspace: torch.Tensor | None = None, stream=None,
-                  layout: str = "contiguous", position_ids: torch.Tensor | None = None):
+                  layout: str = "contiguous", position_ids: torch.Tensor | None = None,
+                  accumulate: bool = False):
     """Gradients of ring_attn_fwd: q/out/dout [B, P*Lc, H_q, D] bf16 (dense), k/v chunks
     [P, B, Lc, H_kv, D] bf16, lse [B, H_q, P*Lc] fp32.  Returns (dq [B, P*Lc, H_q, D],
     dk, dv [P, B, Lc, H_kv, D]) in fp32; the fp32 workspace [B, H_q, P*Lc] is allocated
     here when not given (the library itself allocates nothing).  layout and position_ids
-    as for ring_attn_fwd (the forward's)."""
+    as for ring_attn_fwd (the forward's).  accumulate: add into the given dq / dk / dv
+    (ra_ring_attn_bwd_accumulate; contiguous layout)."""
     if layout not in ("contiguous", "zigzag"):
         raise ValueError(f"unknown layout {layout!r}")
     if position_ids is not None and (layout != "contiguous" or not causal):
         raise ValueError("packed samples need the contiguous layout and causal=True")
+    if accumulate and (dq is None or dk is None or dv is None or layout != "contiguous"
+                       or position_ids is not None):
+        raise ValueError("accumulate needs dq, dk and dv to add into, and the contiguous layout")
     P, B, Lc, H_kv, D = k_chunks.shape
     _, L, H_q, _ = q.shape
     assert L == P * Lc and q.is_contiguous() and out.is_contiguous() and dout.is_contiguous()
@@ -219,6 +236,8 @@ def ring_attn_bwd(q: torch.Tensor, k_chunks: torch.Tensor, v_chunks: torch.Tenso
                                 workspace.data_ptr(), _stream(stream))
     else:
         entry = ra_ring_attn_bwd_zigzag if layout == "zigzag" else ra_ring_attn_bwd
+        if accumulate:
+            entry = ra_ring_attn_bwd_accumulate
         entry(q.data_ptr(), kp, vp_, out.data_ptr(), lse.data_ptr(), dout.data_ptr(), P, B, H_q,
               H_kv, Lc, D, L * H_q * D, Lc * H_kv * D, float(scale), causal, dq.data_ptr(), dkp,
               dvp, workspace.data_ptr(), _stream(stream))

@@ -133,7 +133,7 @@ def _bwd(lib, entry="ra_ring_attn_bwd", **kw):
 
 
 @pytest.mark.parametrize("entry", ["ra_ring_attn_bwd", "ra_ring_attn_bwd_zigzag",
-                                   "ra_ring_attn_bwd_packed"])
+                                   "ra_ring_attn_bwd_packed", "ra_ring_attn_bwd_accumulate"])
 @pytest.mark.parametrize("kw,status", [
     (dict(P=0), 1), (dict(P=65), 1), (dict(H_q=3, H_kv=2), 1), (dict(scale=0.0), 1),
     (dict(D=32), 2), (dict(D=96), 2), (dict(q=FAKE + 8), 1), (dict(out=0), 1),

@@ -1,6 +1,7 @@
 """The multi-GPU data plane's computations on one GPU: the ring's per-step attention and
 merge (RingAccumulator with the library's kernels) for P virtual ranks visiting the chunks
-in ring order, against the oracle's attention over the whole sequence; the Ulysses pack and
+in ring order, against the oracle's attention over the whole sequence; the ring backward's
+per-step accumulating calls against the oracle's gradients; the Ulysses pack and
 unpack kernels around an all-to-all emulated on the device, bit for bit against the
 oracle's seq->head / head->seq; and the distributed functions themselves through a
 one-rank NCCL process group.  The exchanges between ranks are tested on CPU ranks
@@ -15,7 +16,7 @@ import pytest
 import torch
 
 from sequence_parallelism_attn_b200 import dist as rd
-from _util import TOL, f64, max_abs
+from _util import TOL, check_grad, f64, max_abs
 
 pytestmark = pytest.mark.gpu
 
@@ -53,6 +54,49 @@ def test_ring_steps_equal_whole_sequence(ra_lib, oracle_mod, P, causal):
         print(f"[parity] ring steps P={P} causal={causal} rank {i}: max|dO|={eo:.3e} "
               f"max|dLSE|={el:.3e}")
         assert eo <= TOL[torch.bfloat16][0] and el <= TOL[torch.bfloat16][1]
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("P", [1, 3])
+def test_ring_backward_steps_equal_whole_sequence_gradients(ra_lib, oracle_mod, P, causal):
+    """The ring backward's per-step calls (ra_ring_attn_bwd_accumulate: each virtual rank's
+    queries against every K/V chunk it visits, with the forward's final out and LSE, adding
+    into its dq and into the chunk's dK, dV accumulators) sum to the gradients of attention
+    over the whole sequence, every element (B = 2, ragged chunks of 200 tokens, GQA 4:2,
+    bf16 in, fp32 gradients)."""
+    B, Lc, H_q, H_kv, D = 2, 200, 4, 2, 128
+    g = torch.Generator().manual_seed(700 + P)
+    L = P * Lc
+    q = (torch.randn(B, L, H_q, D, generator=g) * 2).to(torch.bfloat16)
+    k = torch.randn(B, L, H_kv, D, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, L, H_kv, D, generator=g).to(torch.bfloat16)
+    dout = torch.randn(B, L, H_q, D, generator=g).to(torch.bfloat16)
+    scale = D ** -0.5
+    # the forward over the whole sequence gives each chunk's final out (bf16) and LSE
+    kc = k.view(B, P, Lc, H_kv, D).transpose(0, 1).contiguous().cuda()
+    vc = v.view(B, P, Lc, H_kv, D).transpose(0, 1).contiguous().cuda()
+    o, l = ra_lib.ring_attn_fwd(q.cuda(), kc, vc, causal, scale, out_dtype=torch.bfloat16)
+    shard = lambda x, i: x[:, i * Lc:(i + 1) * Lc].contiguous().cuda()
+    dq = torch.zeros(B, L, H_q, D, device="cuda")
+    dk = torch.zeros(P, B, Lc, H_kv, D, device="cuda")
+    dv = torch.zeros_like(dk)
+    for i in range(P):
+        dqi = torch.zeros(B, Lc, H_q, D, device="cuda")
+        for j in rd.ring_schedule(i, P):
+            kind = rd.chunk_pair(i, j, causal)
+            if kind == "skip":
+                continue
+            rd.DeviceOps.attend_bwd(shard(q, i), kc[j, :], vc[j, :], o[:, i * Lc:(i + 1) * Lc].contiguous(),
+                                    l[:, :, i * Lc:(i + 1) * Lc].contiguous(), shard(dout, i),
+                                    kind == "diagonal", scale, dqi, dk[j], dv[j])
+        dq[:, i * Lc:(i + 1) * Lc] = dqi
+    assert ra_lib.ra_sync_status() == 0, ra_lib.ra_last_error()
+    rq, rk, rv = oracle_mod.attention_backward(f64(q), f64(k), f64(v), f64(dout), scale, causal)
+    seq = lambda x: x.transpose(0, 1).reshape(B, L, H_kv, D)
+    name = f"ring backward steps P={P} causal={causal}"
+    check_grad(name, "dq", f64(dq), rq)
+    check_grad(name, "dk", f64(seq(dk)), rk)
+    check_grad(name, "dv", f64(seq(dv)), rv)
 
 
 @pytest.mark.parametrize("B,P,Lc", [(1, 4, 256), (2, 3, 200)])
@@ -148,6 +192,16 @@ def test_distributed_functions_on_one_rank(ra_lib, oracle_mod):
         assert np.array_equal(_bits(z2), _bits(k))
         uo, ul = rd.usp_attn_fwd_dist(q.cuda(), k.cuda(), v.cuda(), True, D ** -0.5)
         assert max_abs(f64(uo), want_o) <= 1e-2 and max_abs(f64(ul), want_l) <= 1e-3
+        # the ring backward on one rank: one diagonal step, the accumulators' one pass home
+        dout = torch.randn(B, Lc, H_q, D, generator=g).to(torch.bfloat16)
+        ob = o.to(torch.bfloat16)
+        gq, gk, gv = rd.ring_attn_bwd_dist(q.cuda(), k.cuda(), v.cuda(), ob, l, dout.cuda(), True,
+                                           D ** -0.5)
+        rq, rk, rv = oracle_mod.attention_backward(f64(q), f64(k), f64(v), f64(dout), D ** -0.5,
+                                                   True)
+        check_grad("ring backward, one rank", "dq", f64(gq), rq)
+        check_grad("ring backward, one rank", "dk", f64(gk), rk)
+        check_grad("ring backward, one rank", "dv", f64(gv), rv)
         torch.cuda.synchronize()
     finally:
         dist.destroy_process_group()

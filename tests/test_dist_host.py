@@ -1,6 +1,7 @@
 """The multi-GPU data plane's exchange logic on CPU ranks (gloo, world sizes 2 and 4): the
 ring schedule and its double-buffered K/V exchange, ring attention across ranks equal to
-attention over the whole sequence, the Ulysses pack -> all-to-all -> unpack equal to the
+attention over the whole sequence, the ring backward (dK, dV accumulators travelling with
+their chunks) equal to the whole sequence's gradients, the Ulysses pack -> all-to-all -> unpack equal to the
 oracle's seq->head / head->seq bit for bit, and a rank that leaves between steps reported
 as an error rather than a hang.
 
@@ -121,6 +122,17 @@ class OracleOps:
         return torch.from_numpy(oracle.head2seq(recv.numpy(), P=1)).view(B, Lc, P * Hl, D)
 
 
+    @staticmethod
+    def attend_bwd(q, k, v, out, lse, dout, causal_diagonal, scale, dq, dk, dv):
+        import oracle
+        a, b, c = oracle.attention_backward_pair(q.numpy(), k.numpy(), v.numpy(), out.numpy(),
+                                                 lse.numpy(), dout.numpy(), scale,
+                                                 causal_diagonal)
+        dq += torch.from_numpy(a)
+        dk += torch.from_numpy(b)
+        dv += torch.from_numpy(c)
+
+
 class RecordingOps(OracleOps):
     """Records the first element of every chunk a rank attends to (each rank's K/V is
     filled with its own rank index)."""
@@ -192,6 +204,76 @@ def test_ring_attention_equals_whole_sequence(world, causal):
         status, errs = res[rank]
         assert status == "ok", errs
         assert errs[0] <= 1e-12 and errs[1] <= 1e-12, (rank, errs)
+
+
+def _ring_backward(rank, world, causal, B, Lc, H_q, H_kv, D):
+    from sequence_parallelism_attn_b200 import dist as rd
+    import oracle
+    g = np.random.default_rng(23)
+    L = world * Lc
+    q = g.standard_normal((B, L, H_q, D)) * 2.0
+    k = g.standard_normal((B, L, H_kv, D))
+    v = g.standard_normal((B, L, H_kv, D))
+    dout = g.standard_normal((B, L, H_q, D))
+    out, lse = oracle.attention(q, k, v, 0.3, causal)  # the forward over the whole sequence
+    sl = slice(rank * Lc, (rank + 1) * Lc)
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x[:, sl]))
+    dq, dk, dv = rd.ring_attn_bwd_dist(t(q), t(k), t(v), t(out),
+                                       torch.from_numpy(np.ascontiguousarray(lse[:, :, sl])),
+                                       t(dout), causal, 0.3, ops=OracleOps)
+    want = oracle.attention_backward(q, k, v, dout, 0.3, causal)
+    return [float(np.abs(got.numpy() - w[:, sl]).max()) for got, w in zip((dq, dk, dv), want)]
+
+
+@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("causal", [False, True])
+def test_ring_backward_equals_whole_sequence_gradients(world, causal):
+    """The ring backward across ranks (K/V chunks travelling with their dK, dV accumulators,
+    every rank adding its queries' share, the last pass returning them home) gives each
+    rank the gradients of its chunks of the whole-sequence attention (GQA 4:2, B = 2)."""
+    res = run_ranks(world, _ring_backward, causal, 2, 6, 4, 2, 8)
+    for rank in range(world):
+        status, errs = res[rank]
+        assert status == "ok", errs
+        assert max(errs) <= 1e-12, (rank, errs)
+
+
+def _ring_backward_accumulators(rank, world, causal):
+    """Each rank's chunk of K and V filled with the rank index + 1; the attend hook adds 1
+    to every accumulator it receives and records the chunk's first K value."""
+    from sequence_parallelism_attn_b200 import dist as rd
+    seen = []
+
+    class Ops(OracleOps):
+        @staticmethod
+        def attend_bwd(q, k, v, out, lse, dout, causal_diagonal, scale, dq, dk, dv):
+            seen.append((int(k.flatten()[0].item()), bool(causal_diagonal)))
+            dk += 1.0
+            dv += 2.0
+
+    z = torch.zeros(1, 3, 2, 4, dtype=torch.float64)
+    k = torch.full((1, 3, 1, 4), float(rank + 1), dtype=torch.float64)
+    _, dk, dv = rd.ring_attn_bwd_dist(z, k, k.clone(), z, torch.zeros(1, 2, 3, dtype=torch.float64),
+                                      z, causal, 0.5, ops=Ops)
+    return seen, float(dk.flatten()[0]), float(dv.flatten()[0])
+
+
+@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("causal", [False, True])
+def test_ring_backward_accumulators_visit_every_rank_and_return(world, causal):
+    """A chunk's accumulators come back to its own rank having collected one share from
+    every rank that attends to it: all P ranks when not causal, ranks j .. P-1 for chunk j
+    when causal (the chunk's own rank on the diagonal)."""
+    res = run_ranks(world, _ring_backward_accumulators, causal)
+    for rank in range(world):
+        status, val = res[rank]
+        assert status == "ok", val
+        seen, dk0, dv0 = val
+        want_seen = [(j + 1, causal and j == rank) for j in
+                     [(rank - s) % world for s in range(world)] if not (causal and j > rank)]
+        assert seen == want_seen, (rank, seen, want_seen)
+        visits = world - rank if causal else world
+        assert (dk0, dv0) == (float(visits), 2.0 * visits), (rank, dk0, dv0)
 
 
 def _zigzag_ring(rank, world, B, Lc, H_q, H_kv, D):
@@ -306,6 +388,29 @@ def _leaver(rank, world, leave_rank):
     except rd.ExchangeError as e:
         return "ExchangeError: " + str(e)[:200]
     return "completed"
+
+
+def _leaver_bwd(rank, world, leave_rank):
+    from sequence_parallelism_attn_b200 import dist as rd
+    if rank == leave_rank:
+        os._exit(0)  # leaves between steps: never posts its exchange
+    z = torch.zeros(1, 4, 2, 8, dtype=torch.float64)
+    k = torch.zeros(1, 4, 1, 8, dtype=torch.float64)
+    try:
+        rd.ring_attn_bwd_dist(z, k, k.clone(), z, torch.zeros(1, 2, 4, dtype=torch.float64), z,
+                              True, 0.5, ops=RecordingOps)
+    except rd.ExchangeError as e:
+        return "ExchangeError: " + str(e)[:200]
+    return "completed"
+
+
+def test_rank_leaving_the_ring_backward_is_reported_not_hung():
+    """Rank 1 of 2 exits before the ring backward's first exchange: rank 0 gets an
+    ExchangeError within the process group's timeout."""
+    res = run_ranks(2, _leaver_bwd, 1, timeout=90)
+    assert 1 not in res
+    status, msg = res[0]
+    assert status == "ok" and msg.startswith("ExchangeError"), msg
 
 
 def test_rank_leaving_is_reported_not_hung():

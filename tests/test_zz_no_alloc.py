@@ -5,6 +5,7 @@ give the existing entry point's gradients (dK and dV bit for bit, dQ up to the o
 fp32 reduce-adds across CTAs); the second call must leave the
 device's free memory and torch's allocated and reserved memory unchanged; sizes beyond
 RA_BWD_STATIC_MAX_ROWS are refused before anything is enqueued.  The pages have no counterpart to this entry point."""
+import gc
 import zlib
 
 import pytest
@@ -42,14 +43,20 @@ def _static_call(ra, w, q, k, v, o, lse, dout):
 
 def _memory_around(ra, call):
     """Run one static call; return (device free memory, torch allocated, torch reserved)
-    before and after it."""
-    torch.cuda.synchronize()
-    before = (torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated(),
-              torch.cuda.memory_reserved())
-    call()
-    assert ra.ra_sync_status() == 0, ra.ra_last_error()
-    after = (torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated(),
-             torch.cuda.memory_reserved())
+    before and after it.  Python's cyclic garbage collector is run first and paused during
+    the call, so that no tensor left over from earlier tests is freed inside the window."""
+    gc.collect()
+    gc.disable()
+    try:
+        torch.cuda.synchronize()
+        before = (torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated(),
+                  torch.cuda.memory_reserved())
+        call()
+        assert ra.ra_sync_status() == 0, ra.ra_last_error()
+        after = (torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated(),
+                 torch.cuda.memory_reserved())
+    finally:
+        gc.enable()
     return before, after
 
 

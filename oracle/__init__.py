@@ -62,10 +62,11 @@ def _load():
                                                 P, i64, P, P, P, i64, P, P, P, P, P, P, i32]
     lib.ora_attention_backward_pair.argtypes = [P, P, P, P, P, P, i32, i64, i64, i32, i32, i32,
                                                 f64, i32, P, P, P, i32]
+    lib.ora_replica_sum.argtypes = [P, P, i64, i32, i32, i32]
     for f in ("ora_attention", "ora_attention_rows", "ora_ring_attention", "ora_lse_merge",
               "ora_seq2head", "ora_head2seq", "ora_zigzag_positions", "ora_packed_lower_bounds",
               "ora_attention_backward", "ora_attention_backward_rows",
-              "ora_attention_backward_pair"):
+              "ora_attention_backward_pair", "ora_replica_sum"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -292,6 +293,17 @@ def head2seq(x: np.ndarray, P: int | None = None) -> np.ndarray:
     out = np.empty((P, B, Lc, Hl * G, D), x.dtype)
     _check(_load().ora_head2seq(_ptr(x), _ptr(out), P, G, B, Lc, Hl * G, D, x.itemsize),
            "head2seq")
+    return out
+
+
+def replica_sum(x, H_out: int) -> np.ndarray:
+    """The gradient of the GQA copy: x [..., H_in, D] (H_in = H_out * rep, replica j a copy
+    of head j // rep) -> [..., H_out, D], each head the sum of its replicas (fp64)."""
+    x = _f64(x)
+    *lead, H_in, D = x.shape
+    rows = int(np.prod(lead)) if lead else 1
+    out = np.empty((*lead, H_out, D), np.float64)
+    _check(_load().ora_replica_sum(_ptr(x), _ptr(out), rows, H_in, H_out, D), "replica_sum")
     return out
 
 

@@ -673,4 +673,21 @@ int ora_head2seq(const void* in, void* out, int P, int G, int B, long long Lc, i
     return 0;
 }
 
+// The adjoint of the GQA copy in seq->head ("Метод контекстного параллелизма Ulysses": KV
+// heads are copied so that every rank has one; H_in = H_out * rep replicas, replica j a copy
+// of head j / rep): the gradient of a KV head is the sum of its replicas' gradients.
+// in [rows][H_in][D], out [rows][H_out][D], out[r][g][d] = sum_{k < rep} in[r][g rep + k][d].
+int ora_replica_sum(const double* in, double* out, long long rows, int H_in, int H_out, int D) {
+    if (rows < 1 || H_in < 1 || H_out < 1 || D < 1 || H_in % H_out != 0) return 1;
+    const int rep = H_in / H_out;
+    for (long long r = 0; r < rows; ++r)
+        for (int g = 0; g < H_out; ++g)
+            for (int d = 0; d < D; ++d) {
+                double acc = 0.0;
+                for (int kk = 0; kk < rep; ++kk) acc += in[(r * H_in + g * rep + kk) * D + d];
+                out[(r * H_out + g) * D + d] = acc;
+            }
+    return 0;
+}
+
 }  // extern "C"

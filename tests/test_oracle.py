@@ -747,3 +747,26 @@ def test_backward_pair_rejects_causal_between_unequal_chunks(oracle_mod):
     with pytest.raises(ValueError):
         oracle_mod.attention_backward_pair(z, np.zeros((1, 3, 2, 8)), np.zeros((1, 3, 2, 8)), z,
                                            zl, z, 1.0, True)
+
+
+# ---------------------------------------------------------------- the GQA copy's gradient
+def test_replica_sum_is_the_adjoint_of_the_copy(oracle_mod):
+    """<copy(x), y> = <x, replica_sum(y)> for the repeat-interleave copy of seq->head (numpy's
+    repeat as the copy), so replica_sum is the copy's transpose: the gradient rule."""
+    x = rnd((3, 5, 2, 8), 120)
+    y = rnd((3, 5, 6, 8), 121)
+    copy = np.repeat(x, 3, axis=2)  # replica j of head j // 3
+    lhs = float(np.sum(copy * y))
+    rhs = float(np.sum(x * oracle_mod.replica_sum(y, 2)))
+    assert abs(lhs - rhs) < 1e-12 * max(1.0, abs(lhs))
+
+
+def test_replica_sum_closed_forms(oracle_mod):
+    y = rnd((2, 4, 3, 4), 122)
+    np.testing.assert_array_equal(oracle_mod.replica_sum(y, 3), y)      # one replica each
+    c = np.full((2, 4, 8, 4), 0.25)
+    np.testing.assert_array_equal(oracle_mod.replica_sum(c, 2), np.full((2, 4, 2, 4), 1.0))
+    h = np.arange(2 * 4 * 1, dtype=np.float64).reshape(1, 1, 8, 1)      # heads 0..7, 2 groups
+    np.testing.assert_array_equal(oracle_mod.replica_sum(h, 2).ravel(), [0 + 1 + 2 + 3, 4 + 5 + 6 + 7])
+    with pytest.raises(ValueError):
+        oracle_mod.replica_sum(rnd((1, 1, 6, 4), 123), 4)

@@ -346,6 +346,21 @@ RA_API ra_status ra_ulysses_head2seq(const void* in, void* out, int P, int B, in
                               int H, int D, ra_dtype dt, void* stream);
 
 /*
+ * ra_ulysses_replica_sum -- the gradient of seq->head's GQA copy ([ULYSSES]: KV heads are
+ * copied so that every rank holds one): replica j of H_in = H_out * rep heads is a copy of
+ * head j / rep, so the gradient of head g is the sum of the gradients of its rep replicas.
+ *   in   device, fp32, [rows][H_in][D] (for example dK of the replicated heads, after
+ *        head->seq: rows = B * Lc)
+ *   out  device, fp32, [rows][H_out][D]
+ *   out[r][g][:] = sum_{k < rep} in[r][g*rep + k][:], the replicas added in ascending k
+ *   (the same bits on every call).  Caller-owned buffers; asynchronous on stream.
+ * Errors: RA_ERR_INVALID for sizes < 1, H_in % H_out != 0, D % 4 != 0, null or
+ *   misaligned (16-byte) pointers, in == out.
+ */
+RA_API ra_status ra_ulysses_replica_sum(const float* in, float* out, long long rows, int H_in,
+                                        int H_out, int D, void* stream);
+
+/*
  * ra_ulysses_seq2head_grouped / ra_ulysses_head2seq_grouped -- the two
  * transforms above with the head groups counted apart from the shards: G
  * groups of H_out/G heads, each receiving the tokens of all P shards.  G = P is

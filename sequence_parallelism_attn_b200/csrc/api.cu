@@ -309,6 +309,21 @@ ra_status ra_ulysses_head2seq_grouped(const void* in, void* out, int P, int G, i
     return RA_OK;
 }
 
+ra_status ra_ulysses_replica_sum(const float* in, float* out, long long rows, int H_in, int H_out,
+                                 int D, void* stream) {
+    if (rows < 1 || H_in < 1 || H_out < 1 || D < 1)
+        return fail(RA_ERR_INVALID, "sizes must be >= 1");
+    if (H_in % H_out != 0) return fail(RA_ERR_INVALID, "H_in must be a multiple of H_out");
+    if (D % 4 != 0) return fail(RA_ERR_INVALID, "D must be a multiple of 4 (16-byte rows)");
+    if (!aligned16(in) || !aligned16(out))
+        return fail(RA_ERR_INVALID, "pointers must be non-null and 16-byte aligned");
+    if (static_cast<const void*>(in) == static_cast<const void*>(out))
+        return fail(RA_ERR_INVALID, "in and out must not alias");
+    cudaError_t e = ra::launch_replica_sum(in, out, rows, H_in, H_out, D, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "replica sum launch");
+    return RA_OK;
+}
+
 ra_status ra_ulysses_seq2head(const void* in, void* out, int P, int B, int Lc, int H_in, int H_out,
                               int D, ra_dtype dt, void* stream) {
     return ra_ulysses_seq2head_grouped(in, out, P, P, B, Lc, H_in, H_out, D, dt, stream);

@@ -351,6 +351,49 @@ cudaError_t launch_head2seq(const void* in, void* out, int P, int G, int B, int 
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ the GQA copy's gradient
+// out[r][g][:] = sum_{k < rep} in[r][g rep + k][:] over fp32 rows of H_in = H_out * rep heads:
+// the adjoint of seq->head's repeat-interleave copy, so the gradient of a KV head is the sum
+// of its replicas'.  HBM-bound: every input element read once, every output written once;
+// one thread per 16-byte vector of out, the replicas added in ascending order (the same bits
+// on every call).
+__global__ void __launch_bounds__(256) replica_sum_kernel(const float4* __restrict__ in,
+                                                          float4* __restrict__ out,
+                                                          unsigned long long n_out, int H_out,
+                                                          int rep, int D4) {
+    const unsigned long long stride = (unsigned long long)gridDim.x * blockDim.x;
+    for (unsigned long long i = (unsigned long long)blockIdx.x * blockDim.x + threadIdx.x; i < n_out;
+         i += stride) {
+        const unsigned long long row_g = i / (unsigned)D4;  // (row, g) pair
+        const unsigned d4 = (unsigned)(i - row_g * (unsigned)D4);
+        const unsigned long long r = row_g / (unsigned)H_out;
+        const unsigned g = (unsigned)(row_g - r * (unsigned)H_out);
+        const float4* src = in + ((r * (unsigned)H_out + g) * (unsigned)rep) * (unsigned)D4 + d4;
+        float4 acc = src[0];
+        for (int k = 1; k < rep; ++k) {
+            const float4 x = src[(unsigned long long)k * (unsigned)D4];
+            acc.x += x.x;
+            acc.y += x.y;
+            acc.z += x.z;
+            acc.w += x.w;
+        }
+        out[i] = acc;
+    }
+}
+
+cudaError_t launch_replica_sum(const float* in, float* out, long long rows, int H_in, int H_out,
+                               int D, cudaStream_t s) {
+    const int D4 = D / 4, rep = H_in / H_out;
+    const unsigned long long n_out = (unsigned long long)rows * H_out * D4;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const unsigned long long want = (n_out + 255) / 256;
+    const unsigned grid = (unsigned)(want < (unsigned long long)sms * 8 ? (want ? want : 1) : (unsigned long long)sms * 8);
+    replica_sum_kernel<<<grid, 256, 0, s>>>((const float4*)in, (float4*)out, n_out, H_out, rep, D4);
+    return cudaGetLastError();
+}
+
 cudaError_t read_and_clear_permute_error(unsigned int* value) {
     cudaError_t e = cudaMemcpyFromSymbol(value, g_permute_error_word, sizeof(unsigned int));
     if (e != cudaSuccess) return e;

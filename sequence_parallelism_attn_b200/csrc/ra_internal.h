@@ -188,6 +188,8 @@ cudaError_t launch_lse_merge(float* o_a, float* lse_a, const float* o_b, const f
 cudaError_t launch_seq2head(const void* in, void* out, int P, int G, int B, int Lc, int H_in,
                             int H_out, int D, int esize, cudaStream_t s,
                             unsigned long long wait_limit_ns);
+cudaError_t launch_replica_sum(const float* in, float* out, long long rows, int H_in, int H_out,
+                               int D, cudaStream_t s);
 cudaError_t launch_head2seq(const void* in, void* out, int P, int G, int B, int Lc, int H, int D,
                             int esize, cudaStream_t s, unsigned long long wait_limit_ns);
 // Tensor-core backward for bf16 inputs, D in {64, 128}: Delta, dQ, then dK/dV.

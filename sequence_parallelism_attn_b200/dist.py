@@ -21,7 +21,8 @@ own buffers through NCCL before a kernel touches it.
 
 The ring backward (ring_attn_bwd_dist) moves each K/V chunk the same way, with fp32 dK, dV
 accumulators that every rank adds its share into before passing them on; the last pass
-returns them to the chunk's own rank.
+returns them to the chunk's own rank.  The Ulysses / USP backward (usp_attn_bwd_dist) wraps
+it in the same all-to-alls, and sums the GQA replicas' dK, dV back onto their heads.
 
 Every rank takes the same collective steps in the same order.  A peer that leaves between
 steps ends the next exchange with an error (the process group's timeout bounds the wait),
@@ -72,6 +73,13 @@ class DeviceOps:
         from . import ra
         ra.ring_attn_bwd(q, k.unsqueeze(0), v.unsqueeze(0), out, lse, dout, causal_diagonal,
                          scale, dq=dq, dk=dk.unsqueeze(0), dv=dv.unsqueeze(0), accumulate=True)
+
+    @staticmethod
+    def replica_sum(x, H_out):
+        """[B, Lc, H_in, D] fp32 -> [B, Lc, H_out, D]: the gradient of the GQA copy, each
+        head the sum of its replicas."""
+        from . import ra
+        return ra.ra_ulysses_replica_sum(x, H_out)
 
     @staticmethod
     def seq2head_pack(x, H_out, P):
@@ -373,3 +381,38 @@ def usp_attn_fwd_dist(q, k, v, causal: bool, scale: float | None = None, ulysses
     vh = ulysses_seq2head_dist(v, H_rep, group=ulysses_group, ops=ops)
     o, lse = ring_attn_fwd_dist(qh, kh, vh, causal, scale, group=ring_group, ops=ops)
     return ulysses_head2seq_dist(o, group=ulysses_group, ops=ops), lse
+
+
+def usp_attn_bwd_dist(q, k, v, out, lse, dout, causal: bool, scale: float | None = None,
+                      ulysses_group=None, ring_group=None, ops=DeviceOps):
+    """The backward of usp_attn_fwd_dist (and of plain Ulysses: a ring group of one rank).
+    q, dout and out [B, Ls, H_q, D] (the forward's output, bf16 on the GPU) and k/v
+    [B, Ls, H_kv, D] are this rank's sequence shard with every head; lse is the one
+    usp_attn_fwd_dist returned (this rank's head block over its Ulysses group's tokens).
+    Returns (dq [B, Ls, H_q, D], dk, dv [B, Ls, H_kv, D]) in fp32, the gradients of this
+    rank's shard.
+
+    Inside the Ulysses group: seq->head of q, k, v (the GQA copy to lcm(H_kv, P_u) heads),
+    out and dout; across the ring group: the ring backward on the head blocks
+    (ring_attn_bwd_dist); inside the Ulysses group again: head->seq of the three gradients,
+    and the replicas' dK, dV summed back onto the H_kv heads (the copy's gradient,
+    ra_ulysses_replica_sum).  The forward's head-layout tensors are exchanged again here
+    rather than kept from the forward."""
+    import math
+    P_u = dist.get_world_size(ulysses_group)
+    H_q, H_kv = q.shape[2], k.shape[2]
+    H_rep = H_kv * P_u // math.gcd(H_kv, P_u)
+    qh = ulysses_seq2head_dist(q, H_q, group=ulysses_group, ops=ops)
+    kh = ulysses_seq2head_dist(k, H_rep, group=ulysses_group, ops=ops)
+    vh = ulysses_seq2head_dist(v, H_rep, group=ulysses_group, ops=ops)
+    oh = ulysses_seq2head_dist(out, H_q, group=ulysses_group, ops=ops)
+    doh = ulysses_seq2head_dist(dout, H_q, group=ulysses_group, ops=ops)
+    dqh, dkh, dvh = ring_attn_bwd_dist(qh, kh, vh, oh, lse, doh, causal, scale, group=ring_group,
+                                       ops=ops)
+    dq = ulysses_head2seq_dist(dqh, group=ulysses_group, ops=ops)
+    dk = ulysses_head2seq_dist(dkh, group=ulysses_group, ops=ops)
+    dv = ulysses_head2seq_dist(dvh, group=ulysses_group, ops=ops)
+    if H_rep != H_kv:
+        dk, dv = ops.replica_sum(dk, H_kv), ops.replica_sum(dv, H_kv)
+    return dq, dk, dv
+

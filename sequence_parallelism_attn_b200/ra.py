@@ -23,7 +23,7 @@ EXPORTED = ("ra_ring_attn_fwd", "ra_ring_attn_fwd_zigzag", "ra_ring_attn_fwd_pac
             "ra_ring_attn_bwd_static", "ra_ring_attn_bwd_accumulate",
             "ra_lse_merge", "ra_ulysses_seq2head", "ra_ulysses_head2seq",
             "ra_ulysses_seq2head_grouped", "ra_ulysses_head2seq_grouped",
-            "ra_sync_status", "ra_last_error", "ra_set_wait_limit_ns", "ra_debug_inject_stall",
+            "ra_ulysses_replica_sum", "ra_sync_status", "ra_last_error", "ra_set_wait_limit_ns", "ra_debug_inject_stall",
             "ra_version")
 
 
@@ -63,12 +63,13 @@ def load() -> ctypes.CDLL:
     lib.ra_ulysses_head2seq.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp]
     lib.ra_ulysses_seq2head_grouped.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp]
     lib.ra_ulysses_head2seq_grouped.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, vp]
+    lib.ra_ulysses_replica_sum.argtypes = [vp, vp, i64, i32, i32, i32, vp]
     lib.ra_sync_status.argtypes = [vp]
     for f in ("ra_ring_attn_fwd", "ra_ring_attn_fwd_zigzag", "ra_ring_attn_fwd_packed",
               "ra_ring_attn_bwd", "ra_ring_attn_bwd_zigzag", "ra_ring_attn_bwd_packed",
               "ra_ring_attn_bwd_static", "ra_ring_attn_bwd_accumulate", "ra_lse_merge",
               "ra_ulysses_seq2head", "ra_ulysses_head2seq", "ra_ulysses_seq2head_grouped",
-              "ra_ulysses_head2seq_grouped", "ra_sync_status"):
+              "ra_ulysses_head2seq_grouped", "ra_ulysses_replica_sum", "ra_sync_status"):
         getattr(lib, f).restype = ctypes.c_int
     lib.ra_last_error.restype = ctypes.c_char_p
     lib.ra_version.restype = ctypes.c_char_p
@@ -253,6 +254,23 @@ def ra_lse_merge(o_a: torch.Tensor, lse_a: torch.Tensor, o_b: torch.Tensor, lse_
     assert o_b.shape == o_a.shape and lse_a.shape == lse_b.shape == (B, H, L)
     _check(load().ra_lse_merge(o_a.data_ptr(), lse_a.data_ptr(), o_b.data_ptr(), lse_b.data_ptr(),
                                B, H, L, D, _stream(stream)))
+
+
+def ra_ulysses_replica_sum(x: torch.Tensor, H_out: int, out: torch.Tensor | None = None,
+                           stream=None) -> torch.Tensor:
+    """The gradient of the GQA copy: x [..., H_in, D] fp32 (H_in = H_out * rep) ->
+    [..., H_out, D], each head the sum of its rep replicas."""
+    assert x.is_cuda and x.dtype == torch.float32 and x.is_contiguous()
+    *lead, H_in, D = x.shape
+    rows = 1
+    for n in lead:
+        rows *= n
+    if out is None:
+        out = torch.empty((*lead, H_out, D), dtype=torch.float32, device=x.device)
+    assert out.is_contiguous() and out.dtype == torch.float32 and out.shape == (*lead, H_out, D)
+    _check(load().ra_ulysses_replica_sum(x.data_ptr(), out.data_ptr(), rows, H_in, H_out, D,
+                                         _stream(stream)))
+    return out
 
 
 def ra_ulysses_seq2head(x: torch.Tensor, H_out: int | None = None, out: torch.Tensor | None = None,

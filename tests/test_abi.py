@@ -96,6 +96,17 @@ def test_permute_argument_validation(lib):
     assert h2s(FAKE, FAKE * 2, 2, 1, 16, 4, 64, 7, None) == 1       # bad dtype
 
 
+def test_replica_sum_argument_validation(lib):
+    """ra_ulysses_replica_sum refuses bad arguments on the host, before any CUDA call."""
+    f = lambda i=FAKE, o=FAKE + 4096, rows=4, H_in=8, H_out=2, D=128: (
+        lib.ra_ulysses_replica_sum(i, o, rows, H_in, H_out, D, None))
+    assert f(rows=0) == 1 and f(H_out=0) == 1 and f(D=0) == 1
+    assert f(H_in=6, H_out=4) == 1 and b"multiple" in lib.ra_last_error()
+    assert f(D=66) == 1 and b"multiple of 4" in lib.ra_last_error()
+    assert f(i=FAKE + 8) == 1 and f(o=0) == 1
+    assert f(o=FAKE) == 1 and b"alias" in lib.ra_last_error()
+
+
 def test_merge_argument_validation(lib):
     m = lib.ra_lse_merge
     assert m(FAKE, FAKE * 2, FAKE * 3, FAKE * 4, 1, 1, 8, 6, None) == 2  # D % 4

@@ -202,6 +202,13 @@ def test_distributed_functions_on_one_rank(ra_lib, oracle_mod):
         check_grad("ring backward, one rank", "dq", f64(gq), rq)
         check_grad("ring backward, one rank", "dk", f64(gk), rk)
         check_grad("ring backward, one rank", "dv", f64(gv), rv)
+        # the Ulysses / USP backward on one rank: transforms of one block, one ring step
+        ub = uo.to(torch.bfloat16)
+        uq, uk, uv = rd.usp_attn_bwd_dist(q.cuda(), k.cuda(), v.cuda(), ub, ul, dout.cuda(), True,
+                                          D ** -0.5)
+        check_grad("USP backward, one rank", "dq", f64(uq), rq)
+        check_grad("USP backward, one rank", "dk", f64(uk), rk)
+        check_grad("USP backward, one rank", "dv", f64(uv), rv)
         torch.cuda.synchronize()
     finally:
         dist.destroy_process_group()

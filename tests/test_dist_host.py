@@ -133,6 +133,12 @@ class OracleOps:
         dv += torch.from_numpy(c)
 
 
+    @staticmethod
+    def replica_sum(x, H_out):
+        import oracle
+        return torch.from_numpy(oracle.replica_sum(x.numpy(), H_out))
+
+
 class RecordingOps(OracleOps):
     """Records the first element of every chunk a rank attends to (each rank's K/V is
     filled with its own rank index)."""
@@ -372,6 +378,44 @@ def test_usp_across_ranks_equals_whole_sequence(P_u, causal):
         status, errs = res[rank]
         assert status == "ok", errs
         assert errs[0] <= 1e-12 and errs[1] <= 1e-12, (rank, errs)
+
+
+def _usp_backward(rank, world, P_u, causal, H_kv):
+    import torch.distributed as dist
+    from sequence_parallelism_attn_b200 import dist as rd
+    import oracle
+    P_r = world // P_u
+    ulysses = [dist.new_group([g * P_u + u for u in range(P_u)]) for g in range(P_r)]
+    rings = [dist.new_group([g * P_u + u for g in range(P_r)]) for u in range(P_u)]
+    B, Ls, H_q, D = 2, 5, 4, 8
+    rng = np.random.default_rng(31)
+    q = rng.standard_normal((world, B, Ls, H_q, D)) * 2.0
+    k = rng.standard_normal((world, B, Ls, H_kv, D))
+    v = rng.standard_normal((world, B, Ls, H_kv, D))
+    do = rng.standard_normal((world, B, Ls, H_q, D))
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x[rank]))
+    kw = dict(ulysses_group=ulysses[rank // P_u], ring_group=rings[rank % P_u], ops=OracleOps)
+    out, lse = rd.usp_attn_fwd_dist(t(q), t(k), t(v), causal, 0.3, **kw)
+    dq, dk, dv = rd.usp_attn_bwd_dist(t(q), t(k), t(v), out, lse, t(do), causal, 0.3, **kw)
+    seq = lambda x: np.concatenate(list(x), axis=1)  # [B, world * Ls, H, D]
+    want = oracle.attention_backward(seq(q), seq(k), seq(v), seq(do), 0.3, causal)
+    sl = slice(rank * Ls, (rank + 1) * Ls)
+    return [float(np.abs(g.numpy() - w[:, sl]).max()) for g, w in zip((dq, dk, dv), want)]
+
+
+@pytest.mark.parametrize("P_u,causal,H_kv", [(2, True, 1), (2, False, 2), (4, True, 1),
+                                             (4, True, 4), (1, True, 1)])
+def test_usp_backward_across_ranks_equals_whole_sequence_gradients(P_u, causal, H_kv):
+    """The backward of the ring x Ulysses hybrid at four ranks (2 x 2, 1 x 4 = plain
+    Ulysses, 4 x 1 = plain ring): seq->head of q, k, v, out, dout, the ring backward on the
+    head blocks, head->seq of the gradients and the sum of each KV head's replicas give every
+    rank its shard's gradients of whole-sequence attention (one, two or four KV heads: copied
+    up to P_u or not at all)."""
+    res = run_ranks(4, _usp_backward, P_u, causal, H_kv)
+    for rank in range(4):
+        status, errs = res[rank]
+        assert status == "ok", errs
+        assert max(errs) <= 1e-12, (rank, errs)
 
 
 # ------------------------------------------------------------------ a rank that leaves

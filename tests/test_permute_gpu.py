@@ -75,3 +75,23 @@ def test_full_size_ulysses_transforms_bit_exact(ra_lib, oracle_mod):
         torch.from_numpy(yq.view(np.int16)).view(torch.bfloat16).cuda())
     torch.cuda.synchronize()
     assert np.array_equal(_bits(back), _bits(q))
+
+
+@pytest.mark.parametrize("lead,H_in,H_out,D", [((2, 300), 8, 2, 128), ((1, 1000), 6, 3, 64),
+                                               ((3, 7), 4, 4, 32), ((1, 4096), 32, 1, 128)])
+def test_replica_sum_matches_oracle(ra_lib, oracle_mod, lead, H_in, H_out, D):
+    """The GQA copy's gradient (each head the sum of its replicas) against the oracle's fp64
+    sum: every element within the rounding of an fp32 sum of rep terms, (rep - 1) 2^-24
+    times the sum of their magnitudes; two calls give the same bits."""
+    g = torch.Generator().manual_seed(sum(lead) + H_in)
+    x = torch.randn(*lead, H_in, D, generator=g)
+    got = ra_lib.ra_ulysses_replica_sum(x.cuda(), H_out)
+    again = ra_lib.ra_ulysses_replica_sum(x.cuda(), H_out)
+    assert ra_lib.ra_sync_status() == 0, ra_lib.ra_last_error()
+    assert torch.equal(got, again)
+    want = oracle_mod.replica_sum(x.double().numpy(), H_out)
+    rep = H_in // H_out
+    mag = np.abs(x.double().numpy()).reshape(*lead, H_out, rep, D).sum(axis=-2)
+    err = np.abs(got.double().cpu().numpy() - want)
+    assert np.all(err <= (rep - 1) * 2.0 ** -24 * mag + 1e-30), float((err - (rep - 1) * 2.0 ** -24 * mag).max())
+

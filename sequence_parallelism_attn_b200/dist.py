@@ -326,6 +326,79 @@ def ring_attn_fwd_zigzag_dist(q, k, v, scale: float | None = None, group=None, o
     return acc.result()
 
 
+def ring_attn_bwd_zigzag_dist(q, k, v, out, lse, dout, scale: float | None = None, group=None,
+                              ops=DeviceOps):
+    """The backward of ring_attn_fwd_zigzag_dist (causal): q, out, dout [B, Lc, H_q, D] and
+    k/v [B, Lc, H_kv, D] are this rank's shard in the zigzag layout (segments i and 2P-1-i,
+    Lc even), lse [B, H_q, Lc] the forward's, in shard order.  Returns (dq, dk, dv) of the
+    shard in fp32, in shard order.
+
+    The ring backward of ring_attn_bwd_dist over the shard's halves: the K/V shards travel
+    with fp32 dK, dV accumulators kept as two halves (one per segment), and against rank j's
+    shard rank i adds the shares of the half-pairs that the forward attended --
+      j == i: (Q0, K0) causally, (Q1, K0) wholly, (Q1, K1) causally;
+      j <  i: (Q0, K0) and (Q1, K0) wholly;
+      j >  i: (Q1, K0) and (Q1, K1) wholly."""
+    rank, world = _group_info(group)
+    B, Lc, H_q, D = q.shape
+    if Lc % 2:
+        raise ValueError("the zigzag layout needs an even chunk length")
+    h = Lc // 2
+    scale = D ** -0.5 if scale is None else scale
+    gdt = torch.float64 if q.dtype == torch.float64 else torch.float32
+    half = lambda x, c: x[:, c * h:(c + 1) * h].contiguous()
+    Q = [half(q, c) for c in (0, 1)]
+    O = [half(out, c) for c in (0, 1)]
+    dO = [half(dout, c) for c in (0, 1)]
+    LSE = [lse[:, :, c * h:(c + 1) * h].contiguous() for c in (0, 1)]
+    dq = [torch.zeros(Q[c].shape, dtype=gdt, device=q.device) for c in (0, 1)]
+    zero = lambda: torch.zeros((B, h, k.shape[2], k.shape[3]), dtype=gdt, device=k.device)
+    acc = [zero(), zero(), zero(), zero()]  # dK0, dK1, dV0, dV1 of the held shard
+    acc_bufs = [[torch.empty_like(a) for a in acc] for _ in range(2)] if world > 1 else []
+    kv_bufs = [(torch.empty_like(k), torch.empty_like(v)) for _ in range(2)] if world > 1 else []
+    held = (k, v)
+    nxt_rank, prv_rank = _peer(group, (rank + 1) % world), _peer(group, (rank - 1) % world)
+    for s, j in enumerate(ring_schedule(rank, world)):
+        works = []
+        if s < world - 1:
+            nxt = kv_bufs[s % 2]
+            p2p = [dist.P2POp(dist.isend, held[0], nxt_rank, group),
+                   dist.P2POp(dist.isend, held[1], nxt_rank, group),
+                   dist.P2POp(dist.irecv, nxt[0], prv_rank, group),
+                   dist.P2POp(dist.irecv, nxt[1], prv_rank, group)]
+            try:
+                works = dist.batch_isend_irecv(p2p)
+            except Exception as e:
+                raise ExchangeError(f"zigzag ring backward step {s}: posting the K/V exchange: "
+                                    f"{e}") from e
+        K = [half(held[0], c) for c in (0, 1)]
+        V = [half(held[1], c) for c in (0, 1)]
+        if j == rank:
+            pairs = ((0, 0, True), (1, 0, False), (1, 1, True))
+        elif j < rank:
+            pairs = ((0, 0, False), (1, 0, False))
+        else:
+            pairs = ((1, 0, False), (1, 1, False))
+        for qc, kc, diag in pairs:
+            ops.attend_bwd(Q[qc], K[kc], V[kc], O[qc], LSE[qc], dO[qc], diag, scale, dq[qc],
+                           acc[kc], acc[2 + kc])
+        if world > 1:
+            racc = acc_bufs[s % 2]
+            p2p = ([dist.P2POp(dist.isend, a, nxt_rank, group) for a in acc] +
+                   [dist.P2POp(dist.irecv, r, prv_rank, group) for r in racc])
+            try:
+                awork = dist.batch_isend_irecv(p2p)
+            except Exception as e:
+                raise ExchangeError(f"zigzag ring backward step {s}: posting the dK/dV "
+                                    f"exchange: {e}") from e
+            _wait(awork, f"zigzag ring backward step {s}: dK/dV from rank {(rank - 1) % world}")
+            acc = racc
+        if works:
+            _wait(works, f"zigzag ring backward step {s}: shard from rank {(rank - 1) % world}")
+            held = nxt
+    return (torch.cat(dq, dim=1), torch.cat(acc[:2], dim=1), torch.cat(acc[2:], dim=1))
+
+
 def _all_to_all(send, group, what):
     recv = torch.empty_like(send)
     try:

@@ -209,6 +209,13 @@ def test_distributed_functions_on_one_rank(ra_lib, oracle_mod):
         check_grad("USP backward, one rank", "dq", f64(uq), rq)
         check_grad("USP backward, one rank", "dk", f64(uk), rk)
         check_grad("USP backward, one rank", "dv", f64(uv), rv)
+        # the zigzag ring backward on one rank (its shard is the natural order): the three
+        # half-pairs of the diagonal step
+        zq, zk, zv = rd.ring_attn_bwd_zigzag_dist(q.cuda(), k.cuda(), v.cuda(), ob, l,
+                                                  dout.cuda(), D ** -0.5)
+        check_grad("zigzag ring backward, one rank", "dq", f64(zq), rq)
+        check_grad("zigzag ring backward, one rank", "dk", f64(zk), rk)
+        check_grad("zigzag ring backward, one rank", "dv", f64(zv), rv)
         torch.cuda.synchronize()
     finally:
         dist.destroy_process_group()

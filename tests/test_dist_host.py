@@ -298,6 +298,37 @@ def _zigzag_ring(rank, world, B, Lc, H_q, H_kv, D):
             float(np.abs(lse.numpy() - want_l[:, :, pos]).max()))
 
 
+def _zigzag_ring_backward(rank, world, B, Lc, H_q, H_kv, D):
+    from sequence_parallelism_attn_b200 import dist as rd
+    import oracle
+    g = np.random.default_rng(29)
+    L = world * Lc
+    q = g.standard_normal((B, L, H_q, D)) * 2.0   # natural (sequence) order
+    k = g.standard_normal((B, L, H_kv, D))
+    v = g.standard_normal((B, L, H_kv, D))
+    do = g.standard_normal((B, L, H_q, D))
+    out, lse = oracle.attention(q, k, v, 0.3, True)
+    pos = oracle.zigzag_positions(world, Lc)[rank * Lc:(rank + 1) * Lc]  # this shard's tokens
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x[:, pos]))
+    dq, dk, dv = rd.ring_attn_bwd_zigzag_dist(
+        t(q), t(k), t(v), t(out), torch.from_numpy(np.ascontiguousarray(lse[:, :, pos])), t(do),
+        0.3, ops=OracleOps)
+    want = oracle.attention_backward(q, k, v, do, 0.3, True)
+    return [float(np.abs(got.numpy() - w[:, pos]).max()) for got, w in zip((dq, dk, dv), want)]
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_zigzag_ring_backward_equals_causal_gradients(world):
+    """The zigzag ring's backward (shard halves, dK / dV accumulators travelling with the
+    shards): each rank's gradients equal those of causal attention over the sequence in
+    natural order, mapped to its shard (GQA 4:2, B = 2)."""
+    res = run_ranks(world, _zigzag_ring_backward, 2, 6, 4, 2, 8)
+    for rank in range(world):
+        status, errs = res[rank]
+        assert status == "ok", errs
+        assert max(errs) <= 1e-12, (rank, errs)
+
+
 @pytest.mark.parametrize("world", [2, 4])
 def test_zigzag_ring_equals_causal_attention(world):
     """Shards in the zigzag layout (rank i holds segments i and 2P-1-i): each rank's rows

@@ -464,12 +464,14 @@ def e2e_region(paths, steps, torch, dist, device):
     return max_over_ranks(ms, dist, torch, device)
 
 
-def attn_traffic(path_kind):
-    """DRAM bytes per attention launch from the committed ncu summary, if it was taken on
-    the current kernel source (else None)."""
+def attn_traffic(path_kind, backward=False):
+    """DRAM bytes per launch of the dominant kernel (the attention kernel, or the backward
+    kernel) from the committed ncu summary, if it was taken on the current kernel source
+    (else None)."""
     import hashlib
-    src = os.path.join(ROOT, "sequence_parallelism_attn_b200", "csrc", "attn_sm100.cu")
-    prof = os.path.join(ROOT, "profiles", "attn_sm100_traffic.json")
+    name = "attn_bwd_sm100" if backward else "attn_sm100"
+    src = os.path.join(ROOT, "sequence_parallelism_attn_b200", "csrc", name + ".cu")
+    prof = os.path.join(ROOT, "profiles", name + "_traffic.json")
     if not os.path.exists(prof):
         return None
     with open(prof) as f:
@@ -634,7 +636,8 @@ def main():
     sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     # DRAM bytes from the committed capture of the one-GPU launch (another launch shape
     # when the heads are split over several GPUs)
-    traffic = None if dist_ulysses else attn_traffic(args.workload)
+    traffic = None if dist_ulysses else attn_traffic(args.workload,
+                                                       backward=kind.startswith("attn_bwd"))
     out["roofline"] = {"bound": "tensor", "achieved": round(attn_tflops, 2),
                        "peak": sustained, "unit": "TFLOP/s",
                        "frac": round(attn_tflops / sustained, 4),

@@ -409,6 +409,12 @@ def max_over_ranks(x, dist, torch, device):
     return float(t.item())
 
 
+def any_over_ranks(flag: bool, dist, torch, device) -> bool:
+    """True on every rank when it is True on any: a decision that changes which collectives
+    follow (a retried timing region) must be the same on all ranks."""
+    return max_over_ranks(1.0 if flag else 0.0, dist, torch, device) > 0.5
+
+
 def e2e_region(paths, steps, torch, dist, device):
     """The step through the public API, end to end: every step copies its inputs from
     pinned host memory to the device and reads its result back to pinned host memory.
@@ -598,7 +604,8 @@ def main():
     for attempt in range(2):
         with ClockSampler(local_rank) as clk:
             total_ms, stage_ms = time_region(path, args.steps, torch, dist, stages)
-        if not clk.rejected():
+        # retaken on every rank or on none: the retry runs collectives (barrier, all-reduce)
+        if not any_over_ranks(clk.rejected(), dist, torch, device):
             break
     st = path.ra.ra_sync_status()
     if st != 0:

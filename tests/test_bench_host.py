@@ -1,5 +1,6 @@
 """Host logic of bench.py on the CPU: the N-rank timing reduction (max over ranks, gloo with
-two ranks), the reference arm's rank-0-only rule, and the clock-sample rejection rules."""
+two ranks) and the all-rank agreement on retaking a clock-rejected timing region, the
+reference arm's rank-0-only rule, and the clock-sample rejection rules."""
 import json
 import os
 import socket
@@ -31,8 +32,11 @@ def _rank_main(rank, world, port, values, out_q):
     dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=datetime.timedelta(seconds=60))
     got = bench.max_over_ranks(values[rank], dist, torch, "cpu")
+    # a clock rejection seen on one rank only: both ranks retake the timing region
+    agree = bench.any_over_ranks(rank == 1, dist, torch, "cpu")
+    none = bench.any_over_ranks(False, dist, torch, "cpu")
     dist.barrier()
-    out_q.put((rank, got))
+    out_q.put((rank, (got, agree, none)))
     dist.destroy_process_group()
 
 
@@ -48,7 +52,7 @@ def test_max_over_ranks_gloo_two_ranks():
         p.join(120)
         assert p.exitcode == 0
     got = dict(q.get(timeout=10) for _ in range(2))
-    assert got == {0: 40.25, 1: 40.25}
+    assert got == {0: (40.25, True, False), 1: (40.25, True, False)}
 
 
 def test_max_over_ranks_single_process_is_identity():

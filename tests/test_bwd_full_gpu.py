@@ -1,6 +1,7 @@
-"""GPU parity of the backward pass at the benchmarked size: L = 131072 (16 ranks x 8192
+"""GPU parity of the backward pass at the benchmarked sizes: L = 131072 (16 ranks x 8192
 tokens), H = 8, D = 128, causal, bf16 O from the forward (as the benchmark feeds it), in
-each shard layout -- contiguous, zigzag and 20 packed documents of 512..32768 tokens.
+each shard layout -- contiguous, zigzag and 20 packed documents of 512..32768 tokens -- and
+the Llama-8B-shaped GQA workload (L = 32768, H_q = 32 over H_kv = 8).
 
 Sampled rows against the fp64 oracle's gradients over the full visible key or query range
 (oracle.attention_backward_rows): dQ of >= 2048 query rows (every chunk's and, for the
@@ -99,3 +100,31 @@ def test_bwd_128k_sampled(ra_lib, oracle_mod, layout):
     check_grad(f"full {layout}", "dq", tq(dq, qr), rq)
     check_grad(f"full {layout}", "dk", tq(dk, kr), rk)
     check_grad(f"full {layout}", "dv", tq(dv, kr), rv)
+
+
+def test_bwd_32k_gqa_sampled(ra_lib, oracle_mod):
+    """The backward of the Llama-8B-shaped GQA workload at its benchmarked size (B = 1,
+    L = 32768 as 8 ranks x 4096 tokens, H_q = 32 over H_kv = 8, D = 128, causal, Q x 4):
+    sampled dQ rows of every head and dK, dV rows of one kv head, each summing the four
+    query heads of its group, against the oracle over the full visible range."""
+    w = synth.LLAMA8B_GQA
+    q, k, v = synth.attention_inputs(w)
+    g = torch.Generator().manual_seed(w.seed + 1)
+    dout = torch.randn(q.shape, generator=g).to(torch.bfloat16)
+    qc, kc, vc, doc = q.cuda(), k.cuda(), v.cuda(), dout.cuda()
+    o, lse = ra_lib.ring_attn_fwd(qc, kc, vc, True, w.scale, out_dtype=torch.bfloat16)
+    dq, dk, dv = ra_lib.ring_attn_bwd(qc, kc, vc, o, lse, doc, True, w.scale)
+    assert ra_lib.ra_sync_status() == 0, ra_lib.ra_last_error()
+    assert torch.isfinite(dq).all() and torch.isfinite(dk).all() and torch.isfinite(dv).all()
+    dq, dk, dv = dq.cpu(), chunks_to_seq(dk.cpu()), chunks_to_seq(dv.cpu())
+    del qc, kc, vc, doc, o, lse
+    edges = _edges(w.L, range(0, w.L, w.Lc))
+    qr = _rows(w.B, w.H_q, w.L, N_Q_ROWS, w.seed + 41, edges)
+    kr = _rows(w.B, w.H_kv, w.L, N_K_ROWS, w.seed + 43, edges, head=w.H_kv - 1)
+    rq, rk, rv = oracle_mod.attention_backward_rows(
+        f64(q), f64(chunks_to_seq(k)), f64(chunks_to_seq(v)), f64(dout), w.scale, True, qr, kr)
+    tq = lambda x, r: f64(x[torch.from_numpy(r[0]), torch.from_numpy(r[1]),
+                            torch.from_numpy(r[2])])
+    check_grad("full 32k GQA", "dq", tq(dq, qr), rq)
+    check_grad("full 32k GQA", "dk", tq(dk, kr), rk)
+    check_grad("full 32k GQA", "dv", tq(dv, kr), rv)

@@ -184,7 +184,10 @@ RA_API ra_status ra_ring_attn_fwd_packed(const void* q, const void* const* k_chu
  * each tile pair's share of dq into dq in global memory (fp32 reduce-adds).
  * Reproducibility: dk and dv are the same bits on every call with the same
  * inputs; dq is the same up to the rounding of its fp32 sum, whose order of
- * additions across key tiles varies from call to call.
+ * additions across key tiles varies from call to call.  With
+ * ra_set_bwd_deterministic(1) dq is computed instead by a second kernel with the
+ * query tile stationary (every element summed in one fixed order and written
+ * once), so that all three gradients are the same bits on every call.
  * Arguments
  *   q, k_chunks, v_chunks, P, B, H_q, H_kv, Lc, D, q_bstride, kv_bstride,
  *   scale, causal   exactly as given to ra_ring_attn_fwd (bf16, D in {64,128}).
@@ -399,6 +402,20 @@ RA_API const char* ra_last_error(void);
  * launch.  Returns the previous value.  ns == 0 restores the default.
  */
 RA_API unsigned long long ra_set_wait_limit_ns(unsigned long long ns);
+
+/*
+ * ra_set_bwd_deterministic -- process-wide switch of every backward entry point
+ * (ra_ring_attn_bwd and its _accumulate, _static, _zigzag and _packed forms).  With on != 0
+ * the gradients are bitwise reproducible: dq comes from a kernel that keeps a query
+ * tile stationary, visits the key tiles it sees in one fixed order and writes each dq
+ * element once (adding it into dq in the _accumulate form), and the key-stationary
+ * kernel computes dk and dv only.  It costs a second pass over the score tiles (about
+ * half as much again as the default backward).  With on == 0 (the default) dq is
+ * reduce-added from the key-stationary kernel, reproducible up to the rounding of
+ * its fp32 sum.  Returns the previous setting (0 or 1).  Thread-safe; a call in
+ * flight keeps the setting it started with.
+ */
+RA_API int ra_set_bwd_deterministic(int on);
 
 /*
  * ra_debug_inject_stall -- test hook.  With on != 0 the next tensor-core

@@ -16,6 +16,7 @@ thread_local std::string g_last_error;
 thread_local int g_inject_stall = 0;
 constexpr unsigned long long kDefaultWaitLimitNs = 4000000000ull;
 std::atomic<unsigned long long> g_wait_limit_ns{kDefaultWaitLimitNs};
+std::atomic<int> g_bwd_deterministic{0};
 
 ra_status fail(ra_status s, const std::string& msg) {
     g_last_error = msg;
@@ -202,6 +203,7 @@ static ra_status ring_attn_bwd(const void* q, const void* const* k_chunks,
     a.zigzag = zigzag;
     a.pid = position_ids;
     a.accumulate = accumulate;
+    a.deterministic = g_bwd_deterministic.load();
     a.stream = (cudaStream_t)stream;
     const char* why = "launch failed";
     cudaError_t e = ra::launch_attn_bwd_sm100(a, g_wait_limit_ns.load(), &why);
@@ -360,6 +362,8 @@ unsigned long long ra_set_wait_limit_ns(unsigned long long ns) {
 }
 
 void ra_debug_inject_stall(int on) { g_inject_stall = on ? 1 : 0; }
+
+int ra_set_bwd_deterministic(int on) { return g_bwd_deterministic.exchange(on ? 1 : 0); }
 
 const char* ra_version(void) { return "ra_b200 0.1 (sm_100a: tcgen05/TMEM/TMA attention)"; }
 

@@ -35,6 +35,7 @@ __device__ unsigned int g_bwd_error_word = 0;
 namespace {
 
 constexpr int kThreads = 512;
+constexpr int kThreadsQ = 352;  // the deterministic mode's dQ kernel
 constexpr int kComputeWarps = 8;  // two warpgroups: one per 64-query half of every item
 constexpr int kWarpLoad = 8;
 constexpr int kWarpMma = 9;    // MMA-issuing thread A: S^T, dV (owns tensor memory)
@@ -68,6 +69,7 @@ struct __align__(64) BwdParams {
     int position_order;  // zigzag, causal, Lc/2 a multiple of 128: grids by sequence position
     const int* pid;   // packed samples: position_ids [B][L] (else null)
     int accumulate;   // dK, dV added to the values in memory (dQ: not zeroed by Delta)
+    int skip_dq;      // deterministic mode: the key-stationary kernel leaves dQ alone
     float scale, scale_log2;
     unsigned long long wait_limit_ns;
 };
@@ -229,10 +231,54 @@ __device__ __forceinline__ uint32_t ds_from_p(uint64_t p2, uint64_t dp2, uint64_
     return pd;
 }
 
+// The same without bf16(p): the dQ kernel needs only dS.
+__device__ __forceinline__ uint32_t ds_pair(uint64_t s2, uint64_t dp2, uint64_t sl2x2,
+                                            uint64_t nlse2, uint64_t ndelta2) {
+    uint32_t pd;
+    asm("{\n\t.reg .b32 x0, x1, p0, p1, d0, d1;\n\t.reg .b64 x, p, t, d;\n\t"
+        "fma.rn.f32x2 x, %1, %3, %4;\n\t"
+        "mov.b64 {x0, x1}, x;\n\t"
+        "ex2.approx.ftz.f32 p0, x0;\n\t"
+        "ex2.approx.ftz.f32 p1, x1;\n\t"
+        "mov.b64 p, {p0, p1};\n\t"
+        "add.rn.f32x2 t, %2, %5;\n\t"
+        "mul.rn.f32x2 d, p, t;\n\t"
+        "mov.b64 {d0, d1}, d;\n\t"
+        "cvt.rn.bf16x2.f32 %0, d1, d0;\n\t}"
+        : "=r"(pd)
+        : "l"(s2), "l"(dp2), "l"(sl2x2), "l"(nlse2), "l"(ndelta2));
+    return pd;
+}
+
 // ------------------------------------------------------------------ layout helpers
 // Sample start of row r of batch row b (packed samples).
 __device__ __forceinline__ int sample_start(const BwdParams& p, int b, int r) {
     return ra::sample_start(p.pid + (long long)b * p.L, r);
+}
+
+// The keys of tile (chunk j, local keys key0 .. key0 + kvalid - 1) that a query at sequence
+// position my_pos with sample start my_start sees form one interval [c_lo, c_hi] of tile
+// columns (empty when c_lo > c_hi).  Key c sits at position kpos0 + c, except that a zigzag
+// tile straddling the shard's two segments continues from c = cs at the second segment's
+// start, and a query that sees a key of the second segment sees all of the first.
+template <int LAYOUT>
+__device__ __forceinline__ void key_interval(const BwdParams& p, int j, int key0, int kvalid,
+                                             int my_pos, int my_start, int& c_lo, int& c_hi) {
+    constexpr int ZZ = LAYOUT == kLayoutZigzag ? 1 : 0;
+    const int kpos0 = (int)shard_pos(ZZ, p.P, p.Lc, j, key0);
+    auto clamp_c = [](int x) { return x < -1 ? -1 : (x > kBN ? kBN : x); };
+    c_hi = kvalid - 1;
+    if (p.causal) {
+        int hi = clamp_c(my_pos - kpos0);
+        const int hseg = p.Lc / 2;
+        if (ZZ && key0 < hseg && key0 + kBN > hseg) {
+            const int cs = hseg - key0;
+            const int hi2 = clamp_c(my_pos - (int)shard_pos(1, p.P, p.Lc, j, hseg) + cs);
+            hi = hi2 >= cs ? hi2 : min(hi, cs - 1);
+        }
+        c_hi = min(c_hi, hi);
+    }
+    c_lo = LAYOUT == kLayoutPacked ? clamp_c(my_start - kpos0) : -1;
 }
 
 // ------------------------------------------------------------------ Delta = rowsum(dO * O)
@@ -262,6 +308,375 @@ __global__ void __launch_bounds__(256) bwd_delta_kernel(const uint16_t* __restri
         delta[(b * H + h) * L + t] = acc;
     }
 }
+
+template <int D>
+struct QCfg {
+    static constexpr int TILE = kBM * D * 2;  // bytes of a 128 x D bf16 tile
+    static constexpr int NKB = D / 64;        // 64-column (128-byte) swizzle blocks per tile
+    static constexpr int BLK = kBM * 128;     // bytes of one swizzle block
+    static constexpr int NS = 2;              // ring stages
+    // Q and dO once; a ring of (K, V) stages
+    static constexpr int OFF_A = 0;                      // Q
+    static constexpr int OFF_B = TILE;                   // dO
+    static constexpr int OFF_RING = 2 * TILE;            // NS x (K, V) stages
+    static constexpr int STAGE = 2 * TILE;
+    static constexpr int OFF_BAR = OFF_RING + NS * STAGE;
+    // barriers: fixed_full, full[NS], empty[NS], s_ready (S of a tile complete), dp_ready
+    // (dP complete), ds_full[2][2] (dS of each 64-column half stored; two per half, by tile
+    // parity), acc_done, drain, dp_free (the compute warps have read all of dP); the indices
+    // between are unused
+    static constexpr int N_BARS = 1 + 2 * NS + 14;
+    static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;  // tmem base, abort flag, n
+    static constexpr int OFF_SCHED = OFF_MISC + 16;   // per-chunk tile ranges
+    static constexpr int SMEM = OFF_SCHED + 2 * RA_MAX_P * 4 + 1024;
+    static constexpr int BAR_FIXED = 0;
+    __host__ __device__ static constexpr int bar_full(int s) { return 1 + s; }
+    __host__ __device__ static constexpr int bar_empty(int s) { return 1 + NS + s; }
+    static constexpr int BAR_SREADY = 1 + 2 * NS;
+    static constexpr int BAR_DPREADY = 2 + 2 * NS;
+    // tile i's barrier of a half and its wait parity: the k-th phase of ds(half, par)
+    // belongs to tile 2k + par
+    __host__ __device__ static constexpr int bar_ds(int half, int i) { return 3 + 2 * NS + 2 * half + (i & 1); }
+    __host__ __device__ static constexpr uint32_t par2(int i) { return (uint32_t)(i >> 1) & 1u; }
+    static constexpr int BAR_ACC = 11 + 2 * NS;
+    static constexpr int BAR_DRAIN = 12 + 2 * NS;
+    static constexpr int BAR_DPFREE = 13 + 2 * NS;
+    // TMEM: S of even key tiles at column 0, of odd ones at S_ODD (S of the next tile is
+    // computed while this tile's dS is formed), dP at 128, dQ at 256.
+    static constexpr uint32_t S_ODD = 384;
+    __host__ __device__ static constexpr uint32_t s_col(int jt) { return (jt & 1) ? S_ODD : 0u; }
+    static_assert(SMEM <= 232448, "shared memory budget");
+    static_assert(STAGE % 1024 == 0, "TMA destinations of every stage stay 1024-byte aligned");
+    static_assert(256 + D <= (int)S_ODD && S_ODD + kBN <= kTmemCols, "dQ kernel columns");
+};
+
+// ------------------------------------------------------------------ dQ, deterministic
+// The deterministic mode's dQ: one CTA per 128 query rows of one (batch, head), 352 threads
+// (warps 0-7 compute, warp 8 loads, warps 9 and 10 one MMA-issuing thread each).  Q and dO
+// stay in shared memory; K and V stream through a two-stage ring in the forward's chunk
+// order (causal tiles skipped by the shared schedule).  Per key tile: S = Q K^T and
+// dP = dO V^T, dS formed in registers and stored as bf16 over S, dQ += dS K; every dQ
+// element is written once, by its CTA, after all key tiles in one fixed order.  The
+// key-stationary kernel then runs with its dQ share skipped.
+template <int D, int LAYOUT>
+__global__ void __launch_bounds__(kThreadsQ, 1) bwd_dq_sm100(const __grid_constant__ BwdParams p) {
+    using C = QCfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint32_t base = smem_u32(smem_raw);
+    const uint32_t pad = (1024u - (base & 1023u)) & 1023u;
+    base += pad;
+    uint8_t* smem = smem_raw + pad;
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+    volatile int* n_slot = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
+    uint32_t* sched_range = reinterpret_cast<uint32_t*>(smem + C::OFF_SCHED);
+    auto bar = [&](int i) { return base + C::OFF_BAR + 8u * (uint32_t)i; };
+    const unsigned long long lim = p.wait_limit_ns;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // grid: (batch, kv head) outermost, then row blocks heaviest first, then the query
+    // heads of the group (they read the same K/V tiles)
+    const int per_bg = p.n_qblocks * p.group;
+    const int bg = (int)(blockIdx.x / per_bg), rem = (int)(blockIdx.x % per_bg);
+    const int b = bg / p.H_kv, g = bg % p.H_kv;
+    const int h = g * p.group + rem % p.group;
+    int r0 = (p.n_qblocks - 1 - rem / p.group) * kBM;
+    if (LAYOUT == kLayoutZigzag && p.position_order) {
+        // the k-th block visited is the one at the k-th latest position: segments 2P-1 down
+        // to 0 (segment s >= P is the second half of rank 2P-1-s, s < P the first of rank s)
+        const int kvis = rem / p.group, hseg = p.Lc / 2, seg_blocks = hseg / kBM;
+        const int seg = 2 * p.P - 1 - kvis / seg_blocks;
+        const int bis = seg_blocks - 1 - kvis % seg_blocks;
+        const int rank = seg < p.P ? seg : 2 * p.P - 1 - seg;
+        r0 = rank * p.Lc + (seg < p.P ? 0 : hseg) + bis * kBM;
+    }
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(C::BAR_FIXED), 1);
+        for (int s = 0; s < C::NS; ++s) {
+            mbar_init(bar(C::bar_full(s)), 1);
+            mbar_init(bar(C::bar_empty(s)), 1);
+        }
+        mbar_init(bar(C::BAR_SREADY), 1);   // thread A's commit after S
+        mbar_init(bar(C::BAR_DPREADY), 1);  // thread B's commit after dP
+        for (int hf = 0; hf < 2; ++hf)
+            for (int par = 0; par < 2; ++par) mbar_init(bar(C::bar_ds(hf, par)), 4 * 32);
+        mbar_init(bar(C::BAR_ACC), 1);
+        mbar_init(bar(C::BAR_DRAIN), 2);
+        mbar_init(bar(C::BAR_DPFREE), kComputeWarps * 32);
+        *abort_flag = 0;
+        fence_mbar_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == kWarpLoad) {
+        SchedArgs sa;
+        sa.P = p.P; sa.Lc = p.Lc; sa.L = p.L; sa.causal = p.causal;
+        sa.zigzag = LAYOUT == kLayoutZigzag ? 1 : 0;
+        sa.pid = LAYOUT == kLayoutPacked ? p.pid : nullptr;
+        const long long last_row = min((long long)r0 + kBM - 1, (long long)p.L - 1);
+        const int nt = make_schedule(sa, b, r0, last_row, sched_range);
+        if (lane == 0) *n_slot = nt;
+    }
+    if (warp == kWarpMma) {
+        __syncwarp();
+        tmem_alloc(base + C::OFF_MISC, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    Sched sched;
+    sched.range = sched_range;
+    sched.P = p.P;
+    sched.i0 = r0 / p.Lc;
+    const int n = *n_slot;
+
+    if (warp == kWarpLoad) {
+        if (lane == 0) {
+            // Q and dO once; K and V of each visited tile through an NS-deep ring
+            mbar_arrive_expect_tx(bar(C::BAR_FIXED), 2 * C::TILE);
+            for (int kb = 0; kb < C::NKB; ++kb) {
+                tma_load_4d(base + C::OFF_A + kb * C::BLK, &p.tm_q, bar(C::BAR_FIXED), kb * 64, h, r0, b);
+                tma_load_4d(base + C::OFF_B + kb * C::BLK, &p.tm_do, bar(C::BAR_FIXED), kb * 64, h, r0, b);
+            }
+            int armed[C::NS];
+            for (int s = 0; s < C::NS; ++s) armed[s] = -1;
+            SchedIter it;
+            it.begin(sched);
+            for (int jt = 0; jt < n; ++jt, it.next()) {
+                const int slot = jt % C::NS;
+                if (jt >= C::NS &&
+                    !wait1(bar(C::bar_empty(slot)), ((jt / C::NS) - 1) & 1, abort_flag, lim, kErrLoad))
+                    break;
+                const uint32_t st = base + C::OFF_RING + slot * C::STAGE;
+                mbar_arrive_expect_tx(bar(C::bar_full(slot)), 2 * C::TILE);
+                for (int kb = 0; kb < C::NKB; ++kb) {
+                    tma_load_4d(st + kb * C::BLK, &p.tm_k[it.chunk()], bar(C::bar_full(slot)),
+                                kb * 64, g, it.t * kBN, b);
+                    tma_load_4d(st + C::TILE + kb * C::BLK, &p.tm_v[it.chunk()],
+                                bar(C::bar_full(slot)), kb * 64, g, it.t * kBN, b);
+                }
+                armed[slot] = jt;
+            }
+            wait_drain(bar(C::BAR_FIXED), 0, abort_flag, lim);
+            for (int s = 0; s < C::NS; ++s)
+                if (armed[s] >= 0) wait_drain(bar(C::bar_full(s)), (armed[s] / C::NS) & 1, abort_flag, lim);
+        }
+    } else if (warp == kWarpMma || warp == kWarpMma2) {
+        if (lane == 0) {
+            const bool thread_a = warp == kWarpMma;
+            constexpr uint32_t IDESC_S = idesc_bf16_f32(kBM, kBN, 0);  // K-major A and B
+            constexpr uint32_t IDESC_O = idesc_bf16_f32(kBM, D, 1);    // B MN-major (D contiguous)
+            const uint64_t dq_ = desc_sw128(base + C::OFF_A, 16, 1024);
+            const uint64_t ddo = desc_sw128(base + C::OFF_B, 16, 1024);
+            auto stage = [&](int jt) { return base + C::OFF_RING + (uint32_t)(jt % C::NS) * C::STAGE; };
+            auto issue_s = [&](int jt) {  // S(jt) = Q K(jt)^T into its column region
+                const uint64_t dk = desc_sw128(stage(jt), 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = ((kk / 4) * C::BLK + (kk % 4) * 32) >> 4;
+                    mma_ss(tmem + C::s_col(jt), dq_ + off, dk + off, IDESC_S, kk > 0 ? 1u : 0u);
+                }
+            };
+            auto issue_dp = [&](int jt) {  // dP(jt) = dO V(jt)^T
+                const uint64_t dv = desc_sw128(stage(jt) + C::TILE, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = ((kk / 4) * C::BLK + (kk % 4) * 32) >> 4;
+                    mma_ss(tmem + 128, ddo + off, dv + off, IDESC_S, kk > 0 ? 1u : 0u);
+                }
+            };
+            auto dq_half = [&](int jt, int half) {  // dQ += dS(jt) K(jt) over 64 keys
+                // dS (bf16 pairs) of the half over the first 32 of its 64 S columns, K as
+                // MN-major B
+                const uint64_t dkm = desc_sw128(stage(jt), C::BLK, 1024);
+#pragma unroll
+                for (int kk = 4 * half; kk < 4 * half + 4; ++kk)
+                    mma_ts(tmem + 256, tmem + C::s_col(jt) + 64 * half + (kk % 4) * 8,
+                           dkm + (uint64_t)((kk * 2048) >> 4), IDESC_O,
+                           (jt > 0 || kk > 0) ? 1u : 0u);
+            };
+            // Two issuing threads (one thread cannot issue 128-wide MMAs fast enough to keep
+            // the tensor core busy).  A issues S and dQ, B issues dP; no MMA reads the other
+            // thread's output columns.  A, per key tile jt: S(jt+1) into the other S region as
+            // soon as K(jt+1) has landed, committed to s_ready once every compute warp has
+            // read tile jt (dp_free) -- so the commit waits for S(jt+1) alone, not for dQ(jt),
+            // and s_ready cannot complete a phase before the compute warps have waited for
+            // the previous one; then dQ over each 64-key half as the compute warps publish it.
+            // B, per key tile jt: dP(jt+1) once the compute warps have read dP(jt), committed
+            // to dp_ready.  The compute warps can then finish tile jt+1 before A has waited for
+            // tile jt's dS, which is why each half's ds barrier alternates by tile parity.
+            if (wait1(bar(C::BAR_FIXED), 0, abort_flag, lim, kErrMma) && n > 0 &&
+                wait1(bar(C::bar_full(0)), 0, abort_flag, lim, kErrMma)) {
+                tc_fence_after();
+                if (thread_a) {
+                    issue_s(0);
+                    tc_commit(bar(C::BAR_SREADY));
+                    for (int jt = 0; jt < n; ++jt) {
+                        const bool more = jt + 1 < n;
+                        if (more) {
+                            if (!wait1(bar(C::bar_full((jt + 1) % C::NS)), ((jt + 1) / C::NS) & 1,
+                                       abort_flag, lim, kErrMma))
+                                break;
+                            tc_fence_after();
+                            issue_s(jt + 1);
+                            if (!wait1(bar(C::BAR_DPFREE), jt & 1, abort_flag, lim, kErrMma)) break;
+                            tc_commit(bar(C::BAR_SREADY));
+                        }
+                        if (!wait1(bar(C::bar_ds(0, jt)), C::par2(jt), abort_flag, lim, kErrMma))
+                            break;
+                        tc_fence_after();
+                        dq_half(jt, 0);
+                        if (!wait1(bar(C::bar_ds(1, jt)), C::par2(jt), abort_flag, lim, kErrMma))
+                            break;
+                        tc_fence_after();
+                        dq_half(jt, 1);
+                        tc_commit(bar(C::bar_empty(jt % C::NS)));
+                    }
+                } else {
+                    issue_dp(0);
+                    tc_commit(bar(C::BAR_DPREADY));
+                    for (int jt = 0; jt + 1 < n; ++jt) {
+                        if (!wait1(bar(C::BAR_DPFREE), jt & 1, abort_flag, lim, kErrMma)) break;
+                        if (!wait1(bar(C::bar_full((jt + 1) % C::NS)), ((jt + 1) / C::NS) & 1,
+                                   abort_flag, lim, kErrMma))
+                            break;
+                        tc_fence_after();
+                        issue_dp(jt + 1);
+                        tc_commit(bar(C::BAR_DPREADY));
+                    }
+                }
+            }
+            if (n > 0) {  // a commit with nothing outstanding arrives at once
+                if (thread_a) tc_commit(bar(C::BAR_ACC));
+                tc_commit(bar(C::BAR_DRAIN));
+                wait_drain(bar(C::BAR_DRAIN), 0, abort_flag, lim);
+            }
+        }
+    } else {
+        // compute warps: P and dS for this thread's row over its warpgroup's 64-key half
+        // (a warp reaches TMEM lanes 32 (warp % 4) .. + 31)
+        const int quarter = warp & 3, c = warp >> 2;
+        const int row_t = quarter * 32 + lane;
+        const long long my_row = (long long)r0 + row_t;
+        const bool row_ok = my_row < p.L;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const long long lrow = ((long long)b * p.H_q + h) * p.L + (row_ok ? my_row : 0);
+        // rows past L see nothing (lse2 = +inf makes every probability 0)
+        const float lse2 = row_ok ? p.lse[lrow] * 1.4426950408889634f : INFINITY;
+        const float dlt = row_ok ? p.delta[lrow] : 0.f;
+        const float sl2 = p.scale_log2;
+        const uint64_t sl2x2 = f2_pack(sl2, sl2), nlse2 = f2_pack(-lse2, -lse2),
+                       nd2 = f2_pack(-dlt, -dlt);
+        // zigzag / packed: this row's sequence position and sample start (L <= 2^30)
+        constexpr int ZZ = LAYOUT == kLayoutZigzag ? 1 : 0;
+        const int my_pos = row_ok ? (int)shard_pos(ZZ, p.P, p.Lc, (int)(my_row / p.Lc), my_row % p.Lc)
+                                  : p.L;
+        const int my_start = (LAYOUT == kLayoutPacked && row_ok) ? sample_start(p, b, (int)my_row) : 0;
+        bool ok = true;
+        SchedIter it;
+        it.begin(sched);
+        for (int jt = 0; jt < n; ++jt, it.next()) {
+            if (!wait_warp(bar(C::BAR_SREADY), jt & 1, abort_flag, lim, kErrCompute) ||
+                !wait_warp(bar(C::BAR_DPREADY), jt & 1, abort_flag, lim, kErrCompute)) {
+                ok = false;
+                break;
+            }
+            __syncwarp();
+            tc_fence_after();
+            const int kvalid = min(kBN, p.Lc - it.t * kBN);
+            // this row sees the tile's keys c with c_lo <= c <= c_hi
+            int c_lo = -1, c_hi;
+            if (LAYOUT == kLayoutContiguous) {
+                const long long k0 = (long long)it.chunk() * p.Lc + (long long)it.t * kBN;
+                const long long lim = p.causal ? my_row - k0 : (long long)kBN;
+                c_hi = (int)min((long long)(kvalid - 1), lim < -1 ? -1LL : lim);
+            } else {
+                key_interval<LAYOUT>(p, it.chunk(), it.t * kBN, kvalid, my_pos, my_start, c_lo, c_hi);
+            }
+            const uint32_t scol = C::s_col(jt);
+            uint32_t pk[32];
+            // warp-uniform: the TMEM loads below are warp-collective
+            if (__all_sync(0xffffffffu, 64 * c >= c_lo && 64 * c + 63 <= c_hi)) {
+                // every key of this half is visible to every row of the warp: packed pairs
+                uint64_t s2[32], d2[32];
+                tmem_ld64_pairs(tmem + lane_off + scol + 64 * c, s2);
+                tmem_ld64_pairs(tmem + lane_off + 128 + 64 * c, d2);
+                // dP is in registers: once both halves are, its columns may take dP(jt+1)
+                tc_fence_before();
+                mbar_arrive(bar(C::BAR_DPFREE));
+#pragma unroll
+                for (int i = 0; i < 32; ++i) pk[i] = ds_pair(s2[i], d2[i], sl2x2, nlse2, nd2);
+            } else {
+                float s[64], dp[64];
+                tmem_ld64(tmem + lane_off + scol + 64 * c, s);
+                tmem_ld64(tmem + lane_off + 128 + 64 * c, dp);
+                tc_fence_before();
+                mbar_arrive(bar(C::BAR_DPFREE));
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    float ds2[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int col = 64 * c + 2 * i + e;
+                        const bool vis = col >= c_lo && col <= c_hi;
+                        const float pr = vis ? ex2_approx(s[2 * i + e] * sl2 - lse2) : 0.f;
+                        ds2[e] = pr * (dp[2 * i + e] - dlt);
+                    }
+                    pk[i] = pack_bf16x2(ds2[0], ds2[1]);
+                }
+            }
+            // publish this 64-key half over its own S columns (already read)
+            tmem_st32(tmem + lane_off + scol + 64 * c, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(C::bar_ds(c, jt)));
+        }
+        if (ok && n > 0 && wait_warp(bar(C::BAR_ACC), 0, abort_flag, lim, kErrCompute)) {
+            __syncwarp();
+            tc_fence_after();
+#pragma unroll
+            for (int cb = c * (D / 64); cb < (c + 1) * (D / 64); ++cb) {  // this half's columns
+                uint32_t o[32];
+                tmem_ld32(tmem + lane_off + 256 + cb * 32, o);
+                tmem_wait_ld();
+                if (row_ok) {
+                    float4* dst = reinterpret_cast<float4*>(
+                        p.dq + (((long long)b * p.L + my_row) * p.H_q + h) * D + cb * 32);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        float4 r = make_float4(__uint_as_float(o[4 * i]) * p.scale,
+                                               __uint_as_float(o[4 * i + 1]) * p.scale,
+                                               __uint_as_float(o[4 * i + 2]) * p.scale,
+                                               __uint_as_float(o[4 * i + 3]) * p.scale);
+                        if (p.accumulate) {  // this CTA alone owns the row
+                            const float4 was = dst[i];
+                            r.x += was.x;
+                            r.y += was.y;
+                            r.z += was.z;
+                            r.w += was.w;
+                        }
+                        dst[i] = r;
+                    }
+                }
+            }
+        } else if (ok && n == 0 && row_ok && !p.accumulate) {  // the row sees no key
+            float4* dst = reinterpret_cast<float4*>(
+                p.dq + (((long long)b * p.L + my_row) * p.H_q + h) * D + c * (D / 2));
+            for (int i = 0; i < D / 8; ++i) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kWarpMma) {
+        __syncwarp();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
 
 // ------------------------------------------------------------------ dQ, dK, dV (key tile stationary)
 // Per (head, query tile) item i of the CTA, tensor memory holds
@@ -601,7 +1016,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_sm100(const __grid_constant__
                     issue_dk(it, 0);
                     if (!wait1(bar(C::bar_ds(1)), ph, abort_flag, lim, kErrMma)) break;
                     tc_fence_after();
-                    issue_dq(it);
+                    if (!p.skip_dq) issue_dq(it);
                     tc_commit(bar(C::BAR_DQREADY));
                     issue_dk(it, 1);
                     tc_commit(bar(C::bar_empty(it % C::NS)));
@@ -656,6 +1071,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_sm100(const __grid_constant__
             const bool rows_in = row0 < p.L;  // warp-uniform; rows past L are clipped by TMA
 #pragma unroll
             for (int hf = 0; hf < (D + 63) / 64; ++hf) {
+                if (p.skip_dq) {  // no dQ share was computed: only free the columns
+                    mbar_arrive(bar(C::bar_rfree(hf)));
+                    if (D == 64) mbar_arrive(bar(C::bar_rfree(1)));
+                    continue;
+                }
                 uint32_t va[32], vb[32];
                 tmem_ld32(tmem + lane_off + C::R_DP + 64 * hf, va);
                 tmem_ld32(tmem + lane_off + C::R_DP + 64 * hf + 32, vb);
@@ -909,6 +1329,9 @@ cudaError_t launch_bwd_d(const BwdParams& p, const AttnBwdArgs& a, const char** 
     decltype(&bwd_sm100<D, kLayoutContiguous>) kern[3] = {
         bwd_sm100<D, kLayoutContiguous>, bwd_sm100<D, kLayoutZigzag>,
         bwd_sm100<D, kLayoutPacked>};
+    decltype(&bwd_dq_sm100<D, kLayoutContiguous>) kern_dq[3] = {
+        bwd_dq_sm100<D, kLayoutContiguous>, bwd_dq_sm100<D, kLayoutZigzag>,
+        bwd_dq_sm100<D, kLayoutPacked>};
     if (configured_for != dev) {
         for (int l = 0; l < 3; ++l) {
             // the register split assumes the launch allocation: a raise beyond it would
@@ -923,18 +1346,26 @@ cudaError_t launch_bwd_d(const BwdParams& p, const AttnBwdArgs& a, const char** 
             e = cudaFuncSetAttribute(kern[l], cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      BCfg<D>::SMEM);
             if (e != cudaSuccess) return e;
+            e = cudaFuncSetAttribute(kern_dq[l], cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     QCfg<D>::SMEM);
+            if (e != cudaSuccess) return e;
         }
         configured_for = dev;
     }
     const int layout = p.pid ? kLayoutPacked : (p.zigzag ? kLayoutZigzag : kLayoutContiguous);
     const long long rows = (long long)a.B * p.L * a.H_q;
     bwd_delta_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, a.stream>>>(
-        (const uint16_t*)a.out, (const uint16_t*)a.dout, a.workspace, a.dq, !a.accumulate, a.B,
-        p.L, a.H_q);
+        (const uint16_t*)a.out, (const uint16_t*)a.dout, a.workspace, a.dq,
+        !a.accumulate && !p.skip_dq, a.B, p.L, a.H_q);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const long long grid_k = (long long)a.B * a.H_kv * a.P * p.ntc;
     kern[layout]<<<(unsigned)grid_k, kThreads, BCfg<D>::SMEM, a.stream>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || !p.skip_dq) return e;
+    // deterministic mode: dQ from the query-stationary kernel, each element written once
+    const long long grid_q = (long long)p.n_qblocks * a.B * a.H_q;
+    kern_dq[layout]<<<(unsigned)grid_q, kThreadsQ, QCfg<D>::SMEM, a.stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -976,6 +1407,7 @@ cudaError_t launch_attn_bwd_sm100(const AttnBwdArgs& a, unsigned long long wait_
     p.position_order = a.zigzag && a.causal && (a.Lc / 2) % kBM == 0;
     p.pid = a.pid;
     p.accumulate = a.accumulate;
+    p.skip_dq = a.deterministic ? 1 : 0;
     p.group = a.H_q / a.H_kv;
     p.n_qblocks = (int)((L + kBM - 1) / kBM);
     p.ntc = (a.Lc + kBN - 1) / kBN;

@@ -59,6 +59,7 @@ struct AttnBwdArgs {
     int zigzag = 0;               // shards in the zigzag layout
     const int* pid = nullptr;     // packed samples: position_ids [B][P*Lc] (causal), else null
     int accumulate = 0;           // add into dq, dk, dv instead of overwriting them
+    int deterministic = 0;        // dq from the query-stationary kernel (fixed order)
     cudaStream_t stream;
 };
 

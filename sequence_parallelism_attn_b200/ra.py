@@ -23,8 +23,8 @@ EXPORTED = ("ra_ring_attn_fwd", "ra_ring_attn_fwd_zigzag", "ra_ring_attn_fwd_pac
             "ra_ring_attn_bwd_static", "ra_ring_attn_bwd_accumulate",
             "ra_lse_merge", "ra_ulysses_seq2head", "ra_ulysses_head2seq",
             "ra_ulysses_seq2head_grouped", "ra_ulysses_head2seq_grouped",
-            "ra_ulysses_replica_sum", "ra_sync_status", "ra_last_error", "ra_set_wait_limit_ns", "ra_debug_inject_stall",
-            "ra_version")
+            "ra_ulysses_replica_sum", "ra_sync_status", "ra_last_error", "ra_set_wait_limit_ns",
+            "ra_set_bwd_deterministic", "ra_debug_inject_stall", "ra_version")
 
 
 class RaError(RuntimeError):
@@ -75,6 +75,8 @@ def load() -> ctypes.CDLL:
     lib.ra_version.restype = ctypes.c_char_p
     lib.ra_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
     lib.ra_set_wait_limit_ns.restype = ctypes.c_ulonglong
+    lib.ra_set_bwd_deterministic.argtypes = [i32]
+    lib.ra_set_bwd_deterministic.restype = i32
     lib.ra_debug_inject_stall.argtypes = [i32]
     lib.ra_debug_inject_stall.restype = None
     _lib = lib
@@ -320,6 +322,12 @@ def ra_last_error() -> str:
 
 def ra_set_wait_limit_ns(ns: int) -> int:
     return load().ra_set_wait_limit_ns(ns)
+
+
+def ra_set_bwd_deterministic(on: bool) -> bool:
+    """Bitwise-reproducible backward (dq from the query-stationary kernel) on or off for
+    every later backward call of the process; returns the previous setting."""
+    return bool(load().ra_set_bwd_deterministic(1 if on else 0))
 
 
 def ra_debug_inject_stall(on: bool):

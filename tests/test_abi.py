@@ -121,6 +121,15 @@ def test_wait_limit_roundtrip(lib):
     assert lib.ra_set_wait_limit_ns(old) == 4000000000
 
 
+def test_bwd_deterministic_roundtrip(lib):
+    """The process-wide switch of the backward: host state only, returns the previous value
+    (any non-zero argument reads as on)."""
+    old = lib.ra_set_bwd_deterministic(7)
+    assert old in (0, 1)
+    assert lib.ra_set_bwd_deterministic(0) == 1
+    assert lib.ra_set_bwd_deterministic(old) == 0
+
+
 def _bwd(lib, entry="ra_ring_attn_bwd", **kw):
     """One backward call with fake pointers (every case below fails validation first)."""
     a = dict(q=FAKE, k=[FAKE], v=[FAKE], pid=FAKE, out=FAKE, lse=FAKE, dout=FAKE, P=1, B=1,

@@ -1,4 +1,5 @@
-"""A model of the synchronisation protocol of the tensor-core backward kernel (bwd_sm100 in
+"""A model of the synchronisation protocol of the tensor-core backward kernels (bwd_sm100,
+and bwd_dq_sm100 of the deterministic mode, in
 sequence_parallelism_attn_b200/csrc/attn_bwd_sm100.cu), run under random latencies on the
 CPU.
 
@@ -42,7 +43,9 @@ from _protocol_sim import Sim, Violation
 #   reduce warps (one per TMEM lane quarter): dqready; per 64-column half of dQ(i): load
 #      it, rfree of that half, then 16-column chunks through three staging buffers per warp
 #      into bulk reduce-adds (wait_group.read 2 before a buffer is reused).
-def fused_roles(sim, n, ds_in_do=True, mutation=None):
+# In the deterministic mode (skip_dq) B issues no dQ MMA but still commits dqready, and the
+# reduce warps only arrive on rfree0 / rfree1 after it: the same barriers in the same order.
+def fused_roles(sim, n, ds_in_do=True, mutation=None, skip_dq=False):
     NS, NRED = 2, 4
     for name, count in (("fixed", 1), ("sready", 1), ("dpready0", 1), ("dpready1", 1),
                         ("dvdone", 1), ("p0", 1), ("p1", 1), ("ds0", 1), ("ds1", 1),
@@ -145,9 +148,10 @@ def fused_roles(sim, n, ds_in_do=True, mutation=None):
                 sim.mma("B", [(ds_block(s, 0), ("dS", it)), q(it)], [], f"dK h0({it})")
                 if mutation != "no_ds1_wait" and not (yield ("wait", "ds1", it)):
                     break
-                sim.mma("B", [(ds_block(s, 0), ("dS", it)), (ds_block(s, 1), ("dS", it)),
-                              ("KV", "KV")], [("RdPh0", ("dQ", it)), ("RdPh1", ("dQ", it))],
-                        f"dQ({it})")
+                if not skip_dq:
+                    sim.mma("B", [(ds_block(s, 0), ("dS", it)), (ds_block(s, 1), ("dS", it)),
+                                  ("KV", "KV")], [("RdPh0", ("dQ", it)), ("RdPh1", ("dQ", it))],
+                            f"dQ({it})")
                 sim.commit("B", "dqready")
                 sim.mma("B", [(ds_block(s, 1), ("dS", it)), q(it)], [], f"dK h1({it})")
                 sim.commit("B", f"empty{s}")
@@ -194,6 +198,9 @@ def fused_roles(sim, n, ds_in_do=True, mutation=None):
             if not (yield ("wait", "dqready", it)):
                 break
             for h in (0, 1):
+                if skip_dq:
+                    sim.bars[f"rfree{h}"].arrive()
+                    continue
                 sim.read(f"RdPh{h}", ("dQ", it), f"RED{w} dQ h{h}({it})")
                 yield None
                 sim.bars[f"rfree{h}"].arrive()
@@ -215,11 +222,122 @@ def fused_roles(sim, n, ds_in_do=True, mutation=None):
     return roles
 
 
+# The deterministic mode's dQ kernel (bwd_dq_sm100, one CTA per query tile).  Per key tile
+# j: S(j) (thread A) into one of two S regions, dP(j) (thread B).  The compute warps wait
+# S(j) (sready) and dP(j) (dpready), read both (dpfree), and store dS over their half of
+# S(j) (ds0 / ds1).  A issues S(j+1) as soon as K(j+1) has landed and commits sready once
+# every compute warp has read tile j (dpfree), so that the commit waits for S(j+1) alone and
+# never for dQ(j); then dQ per half after ds0 / ds1.  B issues dP(j+1) once dP(j) has been
+# read.  The compute warps may then finish tile j+1 before A has waited for tile j's dS, so
+# ds0 / ds1 alternate between two barriers each by tile parity.
+def dq_roles(sim, n, mutation=None):
+    NS = 2
+    s_col = lambda j: "S1" if j & 1 else "S0"
+    for name, count in (("fixed", 1), ("sready", 1), ("dpready", 1), ("ds00", 1), ("ds01", 1),
+                        ("ds10", 1), ("ds11", 1), ("acc", 1), ("drain", 2), ("dpfree", 2)):
+        sim.bar(name, count)
+    for s in range(NS):
+        sim.bar(f"full{s}", 1)
+        sim.bar(f"empty{s}", 1)
+
+    def loader():
+        sim.bars["fixed"].arrive(tx=1)
+        sim.tma_load("fixed", "QdO", "QdO")
+        yield None
+        armed = {}
+        for jt in range(n):
+            slot = jt % NS
+            if jt >= NS and not (yield ("wait", f"empty{slot}", jt // NS - 1)):
+                break
+            sim.bars[f"full{slot}"].arrive(tx=1)
+            sim.tma_load(f"full{slot}", f"stage{slot}", ("KV", jt))
+            armed[slot] = jt
+            yield None
+        yield ("drain", "fixed", 0)
+        for slot, jt in armed.items():
+            yield ("drain", f"full{slot}", jt // NS)
+
+    kv = lambda j: [(f"stage{j % NS}", ("KV", j)), ("QdO", "QdO")]
+    ds = lambda c, j: f"ds{c}{j & 1}"
+
+    def mma_a():  # S and dQ
+        if (yield ("wait", "fixed", 0)) and (yield ("wait", "full0", 0)):
+            sim.mma("A", kv(0), [(s_col(0) + "h0", ("S", 0)), (s_col(0) + "h1", ("S", 0))],
+                    "S(0)")
+            sim.commit("A", "sready")
+            for jt in range(n):
+                more = jt + 1 < n
+                if more:
+                    if not (yield ("wait", f"full{(jt + 1) % NS}", (jt + 1) // NS)):
+                        break
+                    sim.mma("A", kv(jt + 1), [(s_col(jt + 1) + "h0", ("S", jt + 1)),
+                                              (s_col(jt + 1) + "h1", ("S", jt + 1))],
+                            f"S({jt + 1})")
+                    if mutation != "no_sready_gate" and not (yield ("wait", "dpfree", jt)):
+                        break
+                    sim.commit("A", "sready")
+                if not (yield ("wait", ds(0, jt), jt // 2)):
+                    break
+                sim.mma("A", [(s_col(jt) + "h0", ("dS", jt))] + kv(jt), [], f"dQ h0({jt})")
+                if mutation != "no_ds1_wait" and not (yield ("wait", ds(1, jt), jt // 2)):
+                    break
+                sim.mma("A", [(s_col(jt) + "h1", ("dS", jt))] + kv(jt), [], f"dQ h1({jt})")
+                sim.commit("A", f"empty{jt % NS}")
+        sim.commit("A", "acc")
+        sim.commit("A", "drain")
+        if mutation != "no_mma_drain":
+            yield ("drain", "drain", 0)
+
+    def mma_b():  # dP
+        if (yield ("wait", "fixed", 0)) and (yield ("wait", "full0", 0)):
+            sim.mma("B", kv(0), [("dPh0", ("dP", 0)), ("dPh1", ("dP", 0))], "dP(0)")
+            sim.commit("B", "dpready")
+            for jt in range(n - 1):
+                if mutation != "no_dpfree_wait" and not (yield ("wait", "dpfree", jt)):
+                    break
+                if not (yield ("wait", f"full{(jt + 1) % NS}", (jt + 1) // NS)):
+                    break
+                sim.mma("B", kv(jt + 1), [("dPh0", ("dP", jt + 1)), ("dPh1", ("dP", jt + 1))],
+                        f"dP({jt + 1})")
+                sim.commit("B", "dpready")
+        sim.commit("B", "drain")
+        if mutation != "no_mma_drain":
+            yield ("drain", "drain", 0)
+
+    def compute(c):
+        ok = True
+        for jt in range(n):
+            if not (yield ("wait", "sready", jt)):
+                ok = False
+                break
+            if not (yield ("wait", "dpready", jt)):
+                ok = False
+                break
+            sim.read(f"{s_col(jt)}h{c}", ("S", jt), f"WG{c} S({jt})")
+            sim.read(f"dPh{c}", ("dP", jt), f"WG{c} dP({jt})")
+            yield None
+            sim.bars["dpfree"].arrive()
+            yield None
+            sim.write(f"{s_col(jt)}h{c}", ("dS", jt))
+            yield None
+            sim.bars[ds(c, jt)].arrive()
+        if ok and n > 0:
+            yield ("wait", "acc", 0)
+
+    return {"load": loader(), "A": mma_a(), "B": mma_b(), "WG0": compute(0), "WG1": compute(1)}
+
+
 KERNELS = {"d128": lambda sim, n, mutation=None: fused_roles(sim, n, True, mutation),
-           "d64": lambda sim, n, mutation=None: fused_roles(sim, n, False, mutation)}
+           "d64": lambda sim, n, mutation=None: fused_roles(sim, n, False, mutation),
+           "d128_skip_dq": lambda sim, n, mutation=None: fused_roles(sim, n, True, mutation,
+                                                                     skip_dq=True),
+           "d64_skip_dq": lambda sim, n, mutation=None: fused_roles(sim, n, False, mutation,
+                                                                    skip_dq=True),
+           "dq": dq_roles}
+ALL = ["d128", "d64", "d128_skip_dq", "d64_skip_dq", "dq"]
 
 
-@pytest.mark.parametrize("kernel", ["d128", "d64"])
+@pytest.mark.parametrize("kernel", ALL)
 @pytest.mark.parametrize("n", [1, 2, 3, 4, 7])
 def test_protocol_holds_under_random_latencies(kernel, n):
     for seed in range(300):
@@ -232,7 +350,13 @@ def test_protocol_holds_under_random_latencies(kernel, n):
                                              ("d128", "no_ds1_wait"),
                                              ("d128", "no_stage_wait"),
                                              ("d64", "no_a_release"),
-                                             ("d64", "no_rfree_wait")])
+                                             ("d64", "no_rfree_wait"),
+                                             ("d128_skip_dq", "no_do_wait"),
+                                             ("d128_skip_dq", "no_ds1_wait"),
+                                             ("d64_skip_dq", "no_a_release"),
+                                             ("dq", "no_dpfree_wait"),
+                                             ("dq", "no_ds1_wait"),
+                                             ("dq", "no_sready_gate")])
 def test_mutated_protocols_are_caught(kernel, mutation):
     caught = 0
     for seed in range(300):
@@ -244,7 +368,7 @@ def test_mutated_protocols_are_caught(kernel, mutation):
     assert caught > 0, f"{kernel} with {mutation} was never flagged"
 
 
-@pytest.mark.parametrize("kernel", ["d128", "d64"])
+@pytest.mark.parametrize("kernel", ALL)
 @pytest.mark.parametrize("n", [1, 3, 6])
 def test_abort_at_any_point_tears_down_cleanly(kernel, n):
     """A bounded wait that gives up at any step: every role stops, drains only its own
@@ -268,3 +392,15 @@ def test_teardown_without_a_drain_is_caught(mutation):
         except Violation:
             caught += 1
     assert caught > 0, f"{mutation} was never flagged"
+
+
+def test_dq_kernel_teardown_without_a_drain_is_caught():
+    """The deterministic mode's dQ kernel: both MMA threads skipping their drain wait."""
+    caught = 0
+    for seed in range(400):
+        sim = Sim(seed, abort_after=1 + seed % 200)
+        try:
+            sim.run(dq_roles(sim, 5, "no_mma_drain"))
+        except Violation:
+            caught += 1
+    assert caught > 0

@@ -69,7 +69,8 @@ struct __align__(64) BwdParams {
     int position_order;  // zigzag, causal, Lc/2 a multiple of 128: grids by sequence position
     const int* pid;   // packed samples: position_ids [B][L] (else null)
     int accumulate;   // dK, dV added to the values in memory (dQ: not zeroed by Delta)
-    int skip_dq;      // deterministic mode: the key-stationary kernel leaves dQ alone
+    int skip_dq;      // deterministic mode: dQ from bwd_dq_sm100 (the key-stationary kernel
+                      // is then its SKIP_DQ instance)
     float scale, scale_log2;
     unsigned long long wait_limit_ns;
 };
@@ -746,7 +747,7 @@ struct BCfg {
     static_assert(D <= 128, "dQ of one item fits in the dP^T region");
 };
 
-template <int D, int LAYOUT>
+template <int D, int LAYOUT, bool SKIP_DQ>
 __global__ void __launch_bounds__(kThreads, 1) bwd_sm100(const __grid_constant__ BwdParams p) {
     using C = BCfg<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -1016,7 +1017,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_sm100(const __grid_constant__
                     issue_dk(it, 0);
                     if (!wait1(bar(C::bar_ds(1)), ph, abort_flag, lim, kErrMma)) break;
                     tc_fence_after();
-                    if (!p.skip_dq) issue_dq(it);
+                    if (!SKIP_DQ) issue_dq(it);
                     tc_commit(bar(C::BAR_DQREADY));
                     issue_dk(it, 1);
                     tc_commit(bar(C::bar_empty(it % C::NS)));
@@ -1071,7 +1072,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_sm100(const __grid_constant__
             const bool rows_in = row0 < p.L;  // warp-uniform; rows past L are clipped by TMA
 #pragma unroll
             for (int hf = 0; hf < (D + 63) / 64; ++hf) {
-                if (p.skip_dq) {  // no dQ share was computed: only free the columns
+                if (SKIP_DQ) {  // no dQ share was computed: only free the columns
                     mbar_arrive(bar(C::bar_rfree(hf)));
                     if (D == 64) mbar_arrive(bar(C::bar_rfree(1)));
                     continue;
@@ -1326,26 +1327,32 @@ cudaError_t launch_bwd_d(const BwdParams& p, const AttnBwdArgs& a, const char** 
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    decltype(&bwd_sm100<D, kLayoutContiguous>) kern[3] = {
-        bwd_sm100<D, kLayoutContiguous>, bwd_sm100<D, kLayoutZigzag>,
-        bwd_sm100<D, kLayoutPacked>};
+    // [skip dQ][layout]: the deterministic mode's key-stationary kernel is compiled apart,
+    // so that the default one carries no test of it
+    decltype(&bwd_sm100<D, kLayoutContiguous, false>) kern[2][3] = {
+        {bwd_sm100<D, kLayoutContiguous, false>, bwd_sm100<D, kLayoutZigzag, false>,
+         bwd_sm100<D, kLayoutPacked, false>},
+        {bwd_sm100<D, kLayoutContiguous, true>, bwd_sm100<D, kLayoutZigzag, true>,
+         bwd_sm100<D, kLayoutPacked, true>}};
     decltype(&bwd_dq_sm100<D, kLayoutContiguous>) kern_dq[3] = {
         bwd_dq_sm100<D, kLayoutContiguous>, bwd_dq_sm100<D, kLayoutZigzag>,
         bwd_dq_sm100<D, kLayoutPacked>};
     if (configured_for != dev) {
         for (int l = 0; l < 3; ++l) {
-            // the register split assumes the launch allocation: a raise beyond it would
-            // never complete
-            cudaFuncAttributes fa;
-            e = cudaFuncGetAttributes(&fa, kern[l]);
-            if (e != cudaSuccess) return e;
-            if (fa.numRegs != (int)kRegsLaunch) {
-                *why = "backward kernel compiled with a register count its register split does not assume";
-                return cudaErrorInvalidKernelImage;
+            for (int sk = 0; sk < 2; ++sk) {
+                // the register split assumes the launch allocation: a raise beyond it
+                // would never complete
+                cudaFuncAttributes fa;
+                e = cudaFuncGetAttributes(&fa, kern[sk][l]);
+                if (e != cudaSuccess) return e;
+                if (fa.numRegs != (int)kRegsLaunch) {
+                    *why = "backward kernel compiled with a register count its register split does not assume";
+                    return cudaErrorInvalidKernelImage;
+                }
+                e = cudaFuncSetAttribute(kern[sk][l], cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         BCfg<D>::SMEM);
+                if (e != cudaSuccess) return e;
             }
-            e = cudaFuncSetAttribute(kern[l], cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     BCfg<D>::SMEM);
-            if (e != cudaSuccess) return e;
             e = cudaFuncSetAttribute(kern_dq[l], cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      QCfg<D>::SMEM);
             if (e != cudaSuccess) return e;
@@ -1360,7 +1367,7 @@ cudaError_t launch_bwd_d(const BwdParams& p, const AttnBwdArgs& a, const char** 
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const long long grid_k = (long long)a.B * a.H_kv * a.P * p.ntc;
-    kern[layout]<<<(unsigned)grid_k, kThreads, BCfg<D>::SMEM, a.stream>>>(p);
+    kern[p.skip_dq ? 1 : 0][layout]<<<(unsigned)grid_k, kThreads, BCfg<D>::SMEM, a.stream>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess || !p.skip_dq) return e;
     // deterministic mode: dQ from the query-stationary kernel, each element written once

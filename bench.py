@@ -15,8 +15,11 @@ the steps (max over ranks), in TFLOP/s.  With --gpus N every rank runs its own r
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload ulysses_e2e|ulysses_32k|usp_e2e|long_128k|long_128k_zigzag|long_128k_packed|
                               long_128k_bwd|long_128k_bwd_zigzag|long_128k_bwd_packed|
-                              llama8b_32k_bwd|
+                              long_128k_bwd_det|llama8b_32k_bwd|
                               llama8b_32k|small_4k|merge_128k]
+
+long_128k_bwd_det times the backward with ra_set_bwd_deterministic(1) (dQ from the
+query-stationary kernel: bit-reproducible gradients).
 
 merge_128k times the log-sum-exp merge alone (ra_lse_merge, B=1, H=8, L=131072, D=128,
 fp32): one step = one merge of two partials, reported in GB/s of 3*D*4 + 12 bytes per row
@@ -44,7 +47,8 @@ DATASHEET_BF16_TFLOPS = 2250.0
 DATASHEET_HBM_GBS = 8000.0
 # workload name suffix of each path kind
 SUFFIX = {"attn_zigzag": "_zigzag", "attn_packed": "_packed", "attn_bwd": "_backward",
-          "attn_bwd_zigzag": "_zigzag_backward", "attn_bwd_packed": "_packed_backward"}
+          "attn_bwd_zigzag": "_zigzag_backward", "attn_bwd_packed": "_packed_backward",
+          "attn_bwd_det": "_deterministic_backward"}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -70,6 +74,7 @@ def workloads():
         "long_128k_bwd": ("attn_bwd", synth.LONG_128K),
         "long_128k_bwd_zigzag": ("attn_bwd_zigzag", synth.LONG_128K),
         "long_128k_bwd_packed": ("attn_bwd_packed", synth.LONG_128K),
+        "long_128k_bwd_det": ("attn_bwd_det", synth.LONG_128K),
         "llama8b_32k": ("attn", synth.LLAMA8B_GQA),
         "llama8b_32k_bwd": ("attn_bwd", synth.LLAMA8B_GQA),
         "small_4k": ("attn", synth.SMALL_BF16),
@@ -260,6 +265,12 @@ class Path:
                 self.ws = torch.empty((w.B, w.H_q, w.L), dtype=torch.float32, device=device)
                 self.flops = 2.5 * self.flops
                 self.launches_per_step = 2  # Delta (and dQ zeroing), then dQ / dK / dV
+                # the deterministic mode: Delta, dK / dV, then dQ by the query-stationary
+                # kernel (a process-wide switch of the library, set once here)
+                det = kind == "attn_bwd_det"
+                ra.ra_set_bwd_deterministic(det)
+                if det:
+                    self.launches_per_step = 3
             self.permute_bytes = 0
             self.in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
             self.out_bytes = self.o.numel() * self.o.element_size()
@@ -649,7 +660,9 @@ def main():
                        "peak": sustained, "unit": "TFLOP/s",
                        "frac": round(attn_tflops / sustained, 4),
                        "traffic": traffic,
-                       "kernel": ("bwd_delta + bwd_sm100 (dQ, dK, dV), D=128"
+                       "kernel": ("bwd_delta + bwd_sm100 (dK, dV) + bwd_dq_sm100 (dQ), D=128"
+                                  if kind == "attn_bwd_det" else
+                                  "bwd_delta + bwd_sm100 (dQ, dK, dV), D=128"
                                   if kind.startswith("attn_bwd") else "attn_fwd_sm100<128>"),
                        "peak_source": f"{peaks_src} bf16_tflops_sustained",
                        "frac_of_burst": round(attn_tflops / peaks.get("bf16_tflops", 1590.0), 4),

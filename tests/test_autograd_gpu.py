@@ -105,3 +105,25 @@ def test_distributed_backward_through_autograd(ra_lib, oracle_mod):
         torch.cuda.synchronize()
     finally:
         dist.destroy_process_group()
+
+
+def test_ring_attention_deterministic_training_step(ra_lib):
+    """With ra_set_bwd_deterministic(1), two identical loss.backward() passes through
+    ring_attention give the same gradient bits (dq included)."""
+    w = synth.AttnWorkload("autograd_det", B=1, H_q=8, H_kv=2, D=128, P=4, Lc=512,
+                           dtype=torch.bfloat16, causal=True, seed=813)
+    q, k, v = synth.attention_inputs(w)
+    wt = torch.randn(q.shape, generator=torch.Generator().manual_seed(814)).to(torch.bfloat16)
+    old = ra_lib.ra_set_bwd_deterministic(True)
+    try:
+        grads = []
+        for _ in range(2):
+            ql, kl, vl = _leaf(q), _leaf(k), _leaf(v)
+            o = rag.ring_attention(ql, kl, vl, True, w.scale)
+            (o.float() * wt.cuda().float()).sum().backward()
+            assert ra_lib.ra_sync_status() == 0, ra_lib.ra_last_error()
+            grads.append((ql.grad, kl.grad, vl.grad))
+    finally:
+        ra_lib.ra_set_bwd_deterministic(old)
+    for nm, a, b in zip(("dq", "dk", "dv"), grads[0], grads[1]):
+        assert torch.equal(a, b), f"{nm} differs between two deterministic passes"

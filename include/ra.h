@@ -349,6 +349,39 @@ RA_API ra_status ra_ulysses_head2seq(const void* in, void* out, int P, int B, in
                               int H, int D, ra_dtype dt, void* stream);
 
 /*
+ * ra_ulysses_seq2head_scatter / ra_ulysses_head2seq_scatter -- one rank's share of
+ * the Ulysses all-to-all ([ULYSSES]: the exchange before attention and the one after
+ * it) as a single kernel that stores each destination rank's block straight into that
+ * rank's buffer: the pack, the all-to-all and the unpack in one pass.  Across GPUs the
+ * dst pointers are the peers' buffers mapped into this process (symmetric memory);
+ * on one GPU they may be local buffers.  After every rank r of the P has made its call
+ * and a cross-rank barrier ordered after those calls has completed, rank r's buffer
+ * holds exactly what ra_ulysses_seq2head / ra_ulysses_head2seq would give rank r.
+ *   seq2head: in  device, dt, [B][Lc][H_in][D]: this rank's sequence shard s = rank.
+ *             dst host array of P device pointers; dst[r] is rank r's [B][P*Lc][H_out/P][D]
+ *             buffer, of which this call writes tokens rank*Lc .. rank*Lc + Lc - 1:
+ *             dst[r][b][rank*Lc+t][h'][:] = in[b][t][floor((r*H_out/P + h')*H_in/H_out)][:]
+ *   head2seq: in  device, dt, [B][P*Lc][H/P][D]: this rank's head group g = rank.
+ *             dst[r] is rank r's [B][Lc][H][D] buffer, of which this call writes heads
+ *             rank*H/P .. rank*H/P + H/P - 1:
+ *             dst[r][b][t][rank*H/P + h'][:] = in[b][r*Lc+t][h'][:]
+ * Plain 16-byte loads and stores (no TMA, no multicast); the kernel ends with a
+ * system-scope fence.  Bit-exact.  The buffers are the caller's; the library frees and
+ * synchronises nothing across ranks: the caller orders the calls against the readers
+ * of the buffers (a barrier before, so that no rank is still reading its buffer, and one
+ * after).  Asynchronous on stream.
+ * Errors: as ra_ulysses_seq2head / ra_ulysses_head2seq with P ranks, and RA_ERR_INVALID
+ *   for P outside [1, RA_MAX_P], rank outside [0, P), a null dst array, a null or
+ *   misaligned dst[r], a dst[r] equal to in, or two equal dst pointers.
+ */
+RA_API ra_status ra_ulysses_seq2head_scatter(const void* in, void* const* dst, int P, int rank,
+                                             int B, int Lc, int H_in, int H_out, int D,
+                                             ra_dtype dt, void* stream);
+RA_API ra_status ra_ulysses_head2seq_scatter(const void* in, void* const* dst, int P, int rank,
+                                             int B, int Lc, int H, int D, ra_dtype dt,
+                                             void* stream);
+
+/*
  * ra_ulysses_replica_sum -- the gradient of seq->head's GQA copy ([ULYSSES]: KV heads are
  * copied so that every rank holds one): replica j of H_in = H_out * rep heads is a copy of
  * head j / rep, so the gradient of head g is the sum of the gradients of its rep replicas.

@@ -311,6 +311,38 @@ ra_status ra_ulysses_head2seq_grouped(const void* in, void* out, int P, int G, i
     return RA_OK;
 }
 
+static ra_status ulysses_scatter(int mode, const void* in, void* const* dst, int P, int rank,
+                                 int B, int Lc, int H_in, int H_out, int D, ra_dtype dt,
+                                 void* stream) {
+    if (P < 1 || P > RA_MAX_P) return fail(RA_ERR_INVALID, "P must be in [1, RA_MAX_P]");
+    if (rank < 0 || rank >= P) return fail(RA_ERR_INVALID, "rank must be in [0, P)");
+    if (!dst) return fail(RA_ERR_INVALID, "dst must be a host array of P device pointers");
+    ra_status s = check_permute(in, dst[0], P, P, B, Lc, H_in, H_out, D, dt);
+    if (s != RA_OK) return s;
+    for (int r = 0; r < P; ++r) {
+        if (!aligned16(dst[r]))
+            return fail(RA_ERR_INVALID, "every dst pointer must be non-null and 16-byte aligned");
+        if (dst[r] == in) return fail(RA_ERR_INVALID, "in and a dst buffer must not alias");
+        for (int q = 0; q < r; ++q)
+            if (dst[q] == dst[r]) return fail(RA_ERR_INVALID, "dst buffers must be distinct");
+    }
+    cudaError_t e = ra::launch_ulysses_scatter(mode, in, dst, P, rank, B, Lc, H_in, H_out, D,
+                                               elem_size(dt), (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "Ulysses scatter launch");
+    return RA_OK;
+}
+
+ra_status ra_ulysses_seq2head_scatter(const void* in, void* const* dst, int P, int rank, int B,
+                                      int Lc, int H_in, int H_out, int D, ra_dtype dt,
+                                      void* stream) {
+    return ulysses_scatter(0, in, dst, P, rank, B, Lc, H_in, H_out, D, dt, stream);
+}
+
+ra_status ra_ulysses_head2seq_scatter(const void* in, void* const* dst, int P, int rank, int B,
+                                      int Lc, int H, int D, ra_dtype dt, void* stream) {
+    return ulysses_scatter(1, in, dst, P, rank, B, Lc, H, H, D, dt, stream);
+}
+
 ra_status ra_ulysses_replica_sum(const float* in, float* out, long long rows, int H_in, int H_out,
                                  int D, void* stream) {
     if (rows < 1 || H_in < 1 || H_out < 1 || D < 1)

@@ -15,6 +15,7 @@
 #include "ra_internal.h"
 #include "permute_index.cuh"
 #include "sm100_ptx.cuh"
+#include "../../include/ra.h"
 
 namespace ra {
 
@@ -391,6 +392,60 @@ cudaError_t launch_replica_sum(const float* in, float* out, long long rows, int 
     const unsigned long long want = (n_out + 255) / 256;
     const unsigned grid = (unsigned)(want < (unsigned long long)sms * 8 ? (want ? want : 1) : (unsigned long long)sms * 8);
     replica_sum_kernel<<<grid, 256, 0, s>>>((const float4*)in, (float4*)out, n_out, H_out, rep, D4);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ one rank's all-to-all share
+// The Ulysses exchange as one kernel: rank `me` reads its own tensor and stores each
+// destination rank's block straight into that rank's buffer (dst[r]: peer memory mapped
+// into this process, or local memory), so the pack, the all-to-all and the unpack become one
+// pass.  Plain 16-byte loads from local memory and 16-byte stores; consecutive threads
+// store consecutive addresses of one destination (a whole head segment, or Hl of them).
+// The kernel ends with a system-scope fence, so that its stores to peers are performed
+// before work ordered after the kernel (the caller's cross-rank barrier) signals anyone.
+struct ScatterParams {
+    int4* dst[RA_MAX_P];
+    const int4* in;
+    uint32_t n_groups;
+    ScatterGeom geo;
+};
+
+namespace {
+template <int MODE, int U>  // MODE 0: seq2head, 1: head2seq
+__global__ void __launch_bounds__(256) scatter_kernel(const __grid_constant__ ScatterParams p) {
+    const uint32_t stride = gridDim.x * blockDim.x;
+    for (uint32_t g = blockIdx.x * blockDim.x + threadIdx.x; g < p.n_groups; g += stride) {
+        const uint32_t vec = g * U;  // U vectors of one head segment (VD % U == 0)
+        const ScatterVec sv =
+            MODE == 0 ? seq2head_scatter_vec(p.geo, vec) : head2seq_scatter_vec(p.geo, vec);
+        int4 v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) v[u] = __ldg(p.in + sv.src + u);
+        int4* d = p.dst[sv.r] + sv.dst;
+#pragma unroll
+        for (int u = 0; u < U; ++u) d[u] = v[u];
+    }
+    __threadfence_system();
+}
+}  // namespace
+
+cudaError_t launch_ulysses_scatter(int mode, const void* in, void* const* dst, int P, int me,
+                                   int B, int Lc, int H_in, int H_out, int D, int esize,
+                                   cudaStream_t s) {
+    static thread_local ScatterParams p;
+    const int Hl = H_out / P;
+    for (int r = 0; r < P; ++r) p.dst[r] = (int4*)dst[r];
+    p.in = (const int4*)in;
+    p.geo = make_scatter_geom(P, me, B, Lc, H_in, H_out, Hl, D, esize);
+    const uint64_t n_vec = (uint64_t)P * B * Lc * (uint64_t)Hl * p.geo.VD.div;
+    const int U = p.geo.VD.div % 4 == 0 ? 4 : 1;
+    p.n_groups = (uint32_t)(n_vec / U);
+    if (p.n_groups == 0) return cudaSuccess;
+    const unsigned grid = grid_for(p.n_groups);
+    if (mode == 0 && U == 4) scatter_kernel<0, 4><<<grid, 256, 0, s>>>(p);
+    else if (mode == 0) scatter_kernel<0, 1><<<grid, 256, 0, s>>>(p);
+    else if (U == 4) scatter_kernel<1, 4><<<grid, 256, 0, s>>>(p);
+    else scatter_kernel<1, 1><<<grid, 256, 0, s>>>(p);
     return cudaGetLastError();
 }
 

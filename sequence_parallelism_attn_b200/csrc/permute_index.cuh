@@ -100,4 +100,74 @@ RA_HD uint64_t head2seq_src_vec(const PermuteGeom& g, uint32_t vec) {
             hh) * g.VD.div + dv;
 }
 
+// ------------------------------------------------------------------ scatter (one rank's share)
+// One rank `me` of P writes its share of the Ulysses all-to-all straight into the P
+// destination buffers (peer memory or local).  The share is enumerated as vectors over
+// [P (destination r)][B][Lc][Hl][VD]; every vector has one source and one destination.
+//   seq2head: in [B][Lc][H_in][VD] (this rank's sequence shard) -> dst[r] [B][P*Lc][Hl][VD]
+//     at token me*Lc + t, head hh of group r (source head hs by the GQA copy).
+//   head2seq: in [B][P*Lc][Hl][VD] (this rank's head group) -> dst[r] [B][Lc][P*Hl][VD]
+//     (rank r's sequence shard) at head me*Hl + hh, from token r*Lc + t.
+struct ScatterGeom {
+    FastDiv VD, Hl, Lc, B, H_out;
+    uint32_t P, me, H_in;
+};
+
+struct ScatterVec {
+    uint32_t r;    // destination rank
+    uint64_t src;  // vector index into in
+    uint64_t dst;  // vector index into dst[r]
+};
+
+inline ScatterGeom make_scatter_geom(int P, int me, int B, int Lc, int H_in, int H_out, int Hl,
+                                     int D, int esize) {
+    ScatterGeom g;
+    g.VD = make_fastdiv((uint32_t)(D * esize / 16));
+    g.Hl = make_fastdiv((uint32_t)Hl);
+    g.Lc = make_fastdiv((uint32_t)Lc);
+    g.B = make_fastdiv((uint32_t)B);
+    g.H_out = make_fastdiv((uint32_t)H_out);
+    g.P = (uint32_t)P;
+    g.me = (uint32_t)me;
+    g.H_in = (uint32_t)H_in;
+    return g;
+}
+
+// coordinates (r, b, t, hh, dv) of share vector `vec`
+RA_HD void scatter_coords(const ScatterGeom& g, uint32_t vec, uint32_t& r, uint32_t& b,
+                          uint32_t& t, uint32_t& hh, uint32_t& dv) {
+    const uint32_t seg = fdiv(vec, g.VD);
+    dv = vec - seg * g.VD.div;
+    const uint32_t row = fdiv(seg, g.Hl);
+    hh = seg - row * g.Hl.div;
+    const uint32_t rb = fdiv(row, g.Lc);
+    t = row - rb * g.Lc.div;
+    r = fdiv(rb, g.B);
+    b = rb - r * g.B.div;
+}
+
+RA_HD ScatterVec seq2head_scatter_vec(const ScatterGeom& g, uint32_t vec) {
+    uint32_t r, b, t, hh, dv;
+    scatter_coords(g, vec, r, b, t, hh, dv);
+    const uint32_t hs = fdiv((r * g.Hl.div + hh) * g.H_in, g.H_out);
+    const uint64_t PLc = (uint64_t)g.P * g.Lc.div;
+    ScatterVec o;
+    o.r = r;
+    o.src = (((uint64_t)b * g.Lc.div + t) * g.H_in + hs) * g.VD.div + dv;
+    o.dst = (((uint64_t)b * PLc + (uint64_t)g.me * g.Lc.div + t) * g.Hl.div + hh) * g.VD.div + dv;
+    return o;
+}
+
+RA_HD ScatterVec head2seq_scatter_vec(const ScatterGeom& g, uint32_t vec) {
+    uint32_t r, b, t, hh, dv;
+    scatter_coords(g, vec, r, b, t, hh, dv);
+    const uint64_t PLc = (uint64_t)g.P * g.Lc.div;
+    const uint64_t H = (uint64_t)g.P * g.Hl.div;
+    ScatterVec o;
+    o.r = r;
+    o.src = (((uint64_t)b * PLc + (uint64_t)r * g.Lc.div + t) * g.Hl.div + hh) * g.VD.div + dv;
+    o.dst = (((uint64_t)b * g.Lc.div + t) * H + (uint64_t)g.me * g.Hl.div + hh) * g.VD.div + dv;
+    return o;
+}
+
 }  // namespace ra

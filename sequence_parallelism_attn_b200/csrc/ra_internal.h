@@ -193,6 +193,11 @@ cudaError_t launch_replica_sum(const float* in, float* out, long long rows, int 
                                int D, cudaStream_t s);
 cudaError_t launch_head2seq(const void* in, void* out, int P, int G, int B, int Lc, int H, int D,
                             int esize, cudaStream_t s, unsigned long long wait_limit_ns);
+// One rank's share of the Ulysses all-to-all stored straight into the P destination buffers
+// (mode 0: seq2head with the GQA copy H_in -> H_out; mode 1: head2seq, H_in = H_out = H).
+cudaError_t launch_ulysses_scatter(int mode, const void* in, void* const* dst, int P, int me,
+                                   int B, int Lc, int H_in, int H_out, int D, int esize,
+                                   cudaStream_t s);
 // Tensor-core backward for bf16 inputs, D in {64, 128}: Delta, dQ, then dK/dV.
 cudaError_t launch_attn_bwd_sm100(const AttnBwdArgs& a, unsigned long long wait_limit_ns,
                                   const char** why);

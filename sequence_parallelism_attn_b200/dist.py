@@ -17,7 +17,10 @@ destination blocks of H_out / P heads (with the GQA copy), so each peer's slice 
 contiguous block; the all-to-all swaps block r of every rank into rank r; the unpack puts
 the P received token blocks in source-rank order (a view when B = 1).  head->seq is the
 inverse.  No kernel reads another GPU's memory: every remote block lands in this GPU's
-own buffers through NCCL before a kernel touches it.
+own buffers through NCCL before a kernel touches it.  ulysses_seq2head_p2p /
+ulysses_head2seq_p2p do the same exchange with one kernel per rank that stores its share
+straight into the peers' symmetric-memory buffers (PeerBuffers), between two cross-rank
+barriers.
 
 The ring backward (ring_attn_bwd_dist) moves each K/V chunk the same way, with fp32 dK, dV
 accumulators that every rank adds its share into before passing them on; the last pass
@@ -432,6 +435,73 @@ def ulysses_head2seq_dist(y, group=None, ops=DeviceOps, out=None):
     send = ops.head2seq_pack(y, world)
     recv = _all_to_all(send, group, f"head2seq all-to-all on rank {rank}")
     return ops.head2seq_unpack(recv) if out is None else ops.head2seq_unpack(recv, out=out)
+
+
+# ------------------------------------------------------------------ one-kernel exchange
+class PeerBuffers:
+    """A buffer of one shape on every rank of `group`, each mapped into every rank's address
+    space (torch symmetric memory), for the one-kernel Ulysses exchange: each rank's scatter
+    kernel (ra_ulysses_*_scatter) stores its share straight into the peers' buffers over
+    NVLink, in place of pack -> all_to_all -> unpack.  The kernel is handed peer addresses
+    for plain 16-byte stores only; nothing reads a peer's memory.
+
+    sync() is the cross-rank barrier around a scatter: an all-reduce of one element on the
+    current stream (NCCL), so it is ordered after this rank's kernels and the process
+    group's timeout bounds the wait."""
+
+    def __init__(self, shape, dtype, group=None, device=None):
+        from torch.distributed import _symmetric_memory as symm
+        self.group = group
+        self.rank, self.world = _group_info(group)
+        pg = group if group is not None else dist.group.WORLD
+        self.buf = symm.empty(*shape, dtype=dtype, device=device)
+        self.handle = symm.rendezvous(self.buf, pg)
+        self.ptrs = [int(a) for a in self.handle.buffer_ptrs]
+        if len(self.ptrs) != self.world:
+            raise RuntimeError(f"symmetric memory gave {len(self.ptrs)} buffers for "
+                               f"{self.world} ranks")
+        self._token = torch.zeros(1, dtype=torch.float32, device=self.buf.device)
+
+    def sync(self, what):
+        try:
+            dist.all_reduce(self._token, group=self.group)
+        except Exception as e:  # a peer left or the process group timed out
+            raise ExchangeError(f"{what}: {e}") from e
+
+
+def ulysses_seq2head_p2p(x, peer: PeerBuffers, H_out: int | None = None):
+    """ulysses_seq2head_dist with the exchange done by one kernel per rank: x [B, Lc, H_in, D]
+    is this rank's sequence shard; every rank stores its share into every rank's buffer of
+    `peer` ([B, P*Lc, H_out/P, D]), which is returned.  It stays valid until the next
+    exchange through the same buffers."""
+    from . import ra
+    B, Lc, H_in, D = x.shape
+    H_out = H_in if H_out is None else H_out
+    want = (B, peer.world * Lc, H_out // peer.world, D)
+    if H_out % peer.world or H_out % H_in or tuple(peer.buf.shape) != want \
+            or peer.buf.dtype != x.dtype:
+        raise ValueError(f"peer buffers {tuple(peer.buf.shape)} {peer.buf.dtype} do not hold "
+                         f"{want} {x.dtype}")
+    peer.sync(f"seq2head scatter on rank {peer.rank}: buffers free")
+    ra.ra_ulysses_seq2head_scatter(x.contiguous(), peer.ptrs, peer.rank, H_out)
+    peer.sync(f"seq2head scatter on rank {peer.rank}: shares stored")
+    return peer.buf
+
+
+def ulysses_head2seq_p2p(y, peer: PeerBuffers):
+    """ulysses_head2seq_dist with the exchange done by one kernel per rank: y [B, P*Lc, Hl, D]
+    is this rank's head group; every rank stores its share into every rank's buffer of
+    `peer` ([B, Lc, P*Hl, D]), which is returned (valid until the next exchange)."""
+    from . import ra
+    B, L, Hl, D = y.shape
+    want = (B, L // peer.world, peer.world * Hl, D)
+    if L % peer.world or tuple(peer.buf.shape) != want or peer.buf.dtype != y.dtype:
+        raise ValueError(f"peer buffers {tuple(peer.buf.shape)} {peer.buf.dtype} do not hold "
+                         f"{want} {y.dtype}")
+    peer.sync(f"head2seq scatter on rank {peer.rank}: buffers free")
+    ra.ra_ulysses_head2seq_scatter(y.contiguous(), peer.ptrs, peer.rank)
+    peer.sync(f"head2seq scatter on rank {peer.rank}: shares stored")
+    return peer.buf
 
 
 def usp_attn_fwd_dist(q, k, v, causal: bool, scale: float | None = None, ulysses_group=None,

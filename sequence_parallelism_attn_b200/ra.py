@@ -23,6 +23,7 @@ EXPORTED = ("ra_ring_attn_fwd", "ra_ring_attn_fwd_zigzag", "ra_ring_attn_fwd_pac
             "ra_ring_attn_bwd_static", "ra_ring_attn_bwd_accumulate",
             "ra_lse_merge", "ra_ulysses_seq2head", "ra_ulysses_head2seq",
             "ra_ulysses_seq2head_grouped", "ra_ulysses_head2seq_grouped",
+            "ra_ulysses_seq2head_scatter", "ra_ulysses_head2seq_scatter",
             "ra_ulysses_replica_sum", "ra_sync_status", "ra_last_error", "ra_set_wait_limit_ns",
             "ra_set_bwd_deterministic", "ra_debug_inject_stall", "ra_version")
 
@@ -64,12 +65,15 @@ def load() -> ctypes.CDLL:
     lib.ra_ulysses_seq2head_grouped.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp]
     lib.ra_ulysses_head2seq_grouped.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, vp]
     lib.ra_ulysses_replica_sum.argtypes = [vp, vp, i64, i32, i32, i32, vp]
+    lib.ra_ulysses_seq2head_scatter.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp]
+    lib.ra_ulysses_head2seq_scatter.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, vp]
     lib.ra_sync_status.argtypes = [vp]
     for f in ("ra_ring_attn_fwd", "ra_ring_attn_fwd_zigzag", "ra_ring_attn_fwd_packed",
               "ra_ring_attn_bwd", "ra_ring_attn_bwd_zigzag", "ra_ring_attn_bwd_packed",
               "ra_ring_attn_bwd_static", "ra_ring_attn_bwd_accumulate", "ra_lse_merge",
               "ra_ulysses_seq2head", "ra_ulysses_head2seq", "ra_ulysses_seq2head_grouped",
-              "ra_ulysses_head2seq_grouped", "ra_ulysses_replica_sum", "ra_sync_status"):
+              "ra_ulysses_head2seq_grouped", "ra_ulysses_replica_sum", "ra_sync_status",
+              "ra_ulysses_seq2head_scatter", "ra_ulysses_head2seq_scatter"):
         getattr(lib, f).restype = ctypes.c_int
     lib.ra_last_error.restype = ctypes.c_char_p
     lib.ra_version.restype = ctypes.c_char_p
@@ -309,6 +313,32 @@ def ra_ulysses_head2seq(x: torch.Tensor, out: torch.Tensor | None = None,
         _check(load().ra_ulysses_head2seq_grouped(x.data_ptr(), out.data_ptr(), P, G, B, Lc,
                                                   Hl * G, D, _dt(x.dtype), _stream(stream)))
     return out
+
+
+def ra_ulysses_seq2head_scatter(x: torch.Tensor, dst_ptrs, rank: int, H_out: int | None = None,
+                                stream=None) -> None:
+    """This rank's share of the Ulysses seq->head all-to-all, stored straight into the P
+    destination buffers: x [B, Lc, H_in, D] (this rank's sequence shard), dst_ptrs = P device
+    addresses (ints) of the ranks' [B, P*Lc, H_out/P, D] buffers (peer or local memory)."""
+    assert x.is_cuda and x.is_contiguous() and x.dim() == 4
+    B, Lc, H_in, D = x.shape
+    P = len(dst_ptrs)
+    H_out = H_in if H_out is None else H_out
+    arr = (ctypes.c_void_p * P)(*dst_ptrs)
+    _check(load().ra_ulysses_seq2head_scatter(x.data_ptr(), arr, P, rank, B, Lc, H_in, H_out, D,
+                                              _dt(x.dtype), _stream(stream)))
+
+
+def ra_ulysses_head2seq_scatter(y: torch.Tensor, dst_ptrs, rank: int, stream=None) -> None:
+    """This rank's share of the Ulysses head->seq all-to-all: y [B, P*Lc, H/P, D] (this rank's
+    head group over the whole sequence), dst_ptrs = P device addresses (ints) of the ranks'
+    [B, Lc, H, D] buffers."""
+    assert y.is_cuda and y.is_contiguous() and y.dim() == 4
+    B, L, Hl, D = y.shape
+    P = len(dst_ptrs)
+    arr = (ctypes.c_void_p * P)(*dst_ptrs)
+    _check(load().ra_ulysses_head2seq_scatter(y.data_ptr(), arr, P, rank, B, L // P, Hl * P, D,
+                                              _dt(y.dtype), _stream(stream)))
 
 
 def ra_sync_status(stream=None) -> int:

@@ -3,10 +3,12 @@
 // (Granlund-Montgomery) against the / operator, and the source vector of every output
 // vector of seq2head and head2seq against the coordinates written out directly, for G head
 // groups over P shards with the GQA copy ("Метод контекстного параллелизма Ulysses": the
-// seq<->head all-to-all; G = P is Ulysses, G < P the ring x Ulysses hybrid's head split).
+// seq<->head all-to-all; G = P is Ulysses, G < P the ring x Ulysses hybrid's head split),
+// and the one-rank shares of the scatter kernels against the whole transforms.
 #include <cstdint>
 #include <cstdio>
 #include <random>
+#include <vector>
 #include "permute_index.cuh"
 
 int main() {
@@ -71,6 +73,47 @@ int main() {
                 ((((uint64_t)r * B + b) * ((uint64_t)P * Lc) + (uint64_t)s * Lc + t) * Hl + hh) * VD + dv;
             if (head2seq_src_vec(gh, (uint32_t)v) != want) ++bad;
         }
+    }
+    // One rank's share of the all-to-all (G = P): every destination vector of every rank's
+    // buffer is written exactly once over the P ranks' shares, from the source vector that
+    // the whole-tensor transform reads for it.
+    for (const auto& g0 : geos) {
+        const int P = g0[0], G = g0[1], B = g0[2], Lc = g0[3], Hi = g0[4], Ho = g0[5], D = g0[6],
+                  es = g0[7];
+        if (G != P) continue;
+        const int VD = D * es / 16, Hl = Ho / P;
+        const uint64_t share = (uint64_t)P * B * Lc * Hl * VD;
+        // seq2head: dst[r] [B][P*Lc][Hl][VD] is block r of the whole output
+        const PermuteGeom gs = make_seq2head_geom(P, P, B, Lc, Hi, Ho, D, es);
+        const uint64_t blk_out = (uint64_t)B * P * Lc * Hl * VD, blk_in = (uint64_t)B * Lc * Hi * VD;
+        std::vector<int> seen(P * blk_out, 0);
+        for (int me = 0; me < P; ++me) {
+            const ScatterGeom sg = make_scatter_geom(P, me, B, Lc, Hi, Ho, Hl, D, es);
+            for (uint64_t v = 0; v < share; ++v, ++checked) {
+                const ScatterVec sv = seq2head_scatter_vec(sg, (uint32_t)v);
+                if (sv.r >= (uint32_t)P || sv.dst >= blk_out || sv.src >= blk_in) { ++bad; continue; }
+                const uint64_t gout = sv.r * blk_out + sv.dst;
+                ++seen[gout];
+                if (seq2head_src_vec(gs, (uint32_t)gout) != me * blk_in + sv.src) ++bad;
+            }
+        }
+        for (int c : seen) if (c != 1) ++bad;
+        // head2seq: dst[r] [B][Lc][P*Hl][VD] is shard r of the whole output; rank me's input is
+        // head group me [B][P*Lc][Hl][VD]
+        const PermuteGeom gh = make_head2seq_geom(P, P, B, Lc, Ho, D, es);
+        const uint64_t shard = (uint64_t)B * Lc * Ho * VD, grp = (uint64_t)B * P * Lc * Hl * VD;
+        std::vector<int> seen2(P * shard, 0);
+        for (int me = 0; me < P; ++me) {
+            const ScatterGeom sg = make_scatter_geom(P, me, B, Lc, Ho, Ho, Hl, D, es);
+            for (uint64_t v = 0; v < share; ++v, ++checked) {
+                const ScatterVec sv = head2seq_scatter_vec(sg, (uint32_t)v);
+                if (sv.r >= (uint32_t)P || sv.dst >= shard || sv.src >= grp) { ++bad; continue; }
+                const uint64_t gout = sv.r * shard + sv.dst;
+                ++seen2[gout];
+                if (head2seq_src_vec(gh, (uint32_t)gout) != me * grp + sv.src) ++bad;
+            }
+        }
+        for (int c : seen2) if (c != 1) ++bad;
     }
     std::printf("vectors checked: %lld\nmismatches: %d\n", checked, bad);
     return bad != 0;

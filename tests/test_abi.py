@@ -107,6 +107,32 @@ def test_replica_sum_argument_validation(lib):
     assert f(o=FAKE) == 1 and b"alias" in lib.ra_last_error()
 
 
+def test_scatter_argument_validation(lib):
+    """The one-kernel Ulysses exchange refuses bad arguments on the host, before any CUDA
+    call: the rank, the destination table (null, misaligned, aliasing the input, repeated)
+    and the permute's own rules."""
+    def arr(*ptrs):
+        return (ctypes.c_void_p * len(ptrs))(*ptrs)
+    good = arr(FAKE * 2, FAKE * 3)
+    s2h = lambda i=FAKE, d=good, P=2, rank=0, B=1, Lc=16, Hi=2, Ho=4, D=64, dt=0: (
+        lib.ra_ulysses_seq2head_scatter(i, d, P, rank, B, Lc, Hi, Ho, D, dt, None))
+    h2s = lambda i=FAKE, d=good, P=2, rank=1, B=1, Lc=16, H=4, D=64, dt=0: (
+        lib.ra_ulysses_head2seq_scatter(i, d, P, rank, B, Lc, H, D, dt, None))
+    assert s2h(rank=2) == 1 and b"rank" in lib.ra_last_error()
+    assert s2h(rank=-1) == 1 and h2s(rank=2) == 1
+    assert s2h(d=None) == 1 and h2s(d=None) == 1
+    assert s2h(d=arr(FAKE * 2, FAKE * 3 + 8)) == 1 and b"aligned" in lib.ra_last_error()
+    assert s2h(d=arr(FAKE * 2, 0)) == 1
+    assert s2h(d=arr(FAKE * 2, FAKE)) == 1 and b"alias" in lib.ra_last_error()
+    assert h2s(d=arr(FAKE * 2, FAKE * 2)) == 1 and b"distinct" in lib.ra_last_error()
+    assert s2h(Ho=6, Hi=2, P=4, d=arr(FAKE * 2, FAKE * 3, FAKE * 4, FAKE * 5)) == 1  # 6 % 4
+    assert s2h(Hi=3) == 1                       # H_out % H_in
+    assert s2h(D=4) == 1                        # D * 2 bytes % 16
+    assert s2h(P=0) == 1 and s2h(P=65) == 1
+    assert h2s(H=3) == 1 and h2s(dt=7) == 1
+    assert s2h(i=FAKE + 4) == 1
+
+
 def test_merge_argument_validation(lib):
     m = lib.ra_lse_merge
     assert m(FAKE, FAKE * 2, FAKE * 3, FAKE * 4, 1, 1, 8, 6, None) == 2  # D % 4

@@ -219,3 +219,35 @@ def test_distributed_functions_on_one_rank(ra_lib, oracle_mod):
         torch.cuda.synchronize()
     finally:
         dist.destroy_process_group()
+
+
+def test_peer_exchange_on_one_rank(ra_lib, oracle_mod):
+    """The one-kernel Ulysses exchange (symmetric-memory buffers, the scatter kernels, the
+    barriers around them) through a one-rank NCCL process group: the buffers are set up and
+    mapped, and seq->head / head->seq give the bits of the NCCL path's functions."""
+    import torch.distributed as dist
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0,
+                            world_size=1, device_id=torch.device("cuda", 0))
+    try:
+        B, Lc, H_in, H_out, D = 2, 300, 2, 4, 128
+        g = torch.Generator().manual_seed(502)
+        x = torch.randn(B, Lc, H_in, D, generator=g).to(torch.bfloat16).cuda()
+        heads = rd.PeerBuffers((B, Lc, H_out, D), torch.bfloat16, device="cuda")
+        seq = rd.PeerBuffers((B, Lc, H_out, D), torch.bfloat16, device="cuda")
+        assert heads.ptrs == [heads.buf.data_ptr()]
+        for _ in range(2):  # the buffers are reused across exchanges
+            y = rd.ulysses_seq2head_p2p(x, heads, H_out)
+            assert np.array_equal(_bits(y), _bits(rd.ulysses_seq2head_dist(x, H_out)))
+            assert np.array_equal(_bits(y), oracle_mod.seq2head(_bits(x)[None], H_out)[0])
+            z = rd.ulysses_head2seq_p2p(y, seq)
+            assert np.array_equal(_bits(z), _bits(rd.ulysses_head2seq_dist(y)))
+        with pytest.raises(ValueError):
+            rd.ulysses_seq2head_p2p(x, seq, 8)  # buffers of another shape
+        torch.cuda.synchronize()
+        del heads, seq, y, z
+    finally:
+        dist.destroy_process_group()

@@ -335,10 +335,11 @@ class DistUlyssesPath:
         """The workload's query heads and sequence divide over `world` ranks."""
         return w.H_q % world == 0 and (w.P * w.Lc) % world == 0 and w.G == w.P
 
-    def __init__(self, w, device, rank, world):
+    def __init__(self, w, device, rank, world, exchange="nccl"):
         import torch
         from sequence_parallelism_attn_b200 import dist as rd, ra
         self.ra, self.rd, self.kind, self.w, self.dev = ra, rd, "ulysses_dist", w, device
+        self.exchange = exchange
         L = w.P * w.Lc
         if not self.splits(w, world):
             raise ValueError(f"{w.name} does not split over {world} ranks")
@@ -354,6 +355,14 @@ class DistUlyssesPath:
         self.o = torch.empty((w.B, L, self.Hq_l, w.D), dtype=torch.bfloat16, device=device)
         self.lse = torch.empty((w.B, self.Hq_l, L), dtype=torch.float32, device=device)
         self.o_seq = torch.empty((w.B, self.Ls, w.H_q, w.D), dtype=w.dtype, device=device)
+        if exchange == "p2p":
+            # the one-kernel exchange: every rank's scatter stores into these symmetric
+            # buffers (the head blocks of Q, K, V and this rank's shard of O)
+            pb = lambda *shape: rd.PeerBuffers(shape, w.dtype, device=device)
+            self.pq = pb(w.B, L, self.Hq_l, w.D)
+            self.pk, self.pv = pb(w.B, L, self.Hkv_l, w.D), pb(w.B, L, self.Hkv_l, w.D)
+            self.po = pb(w.B, self.Ls, w.H_q, w.D)
+            self.o_seq = self.po.buf
         self.scale = w.D ** -0.5
         self.flops = 4.0 * w.B * self.Hq_l * float(L) ** 2 * w.D / 2
         self.launches_per_step = 3 + 1 + (1 if w.B == 1 else 2) + (3 if w.B > 1 else 0)
@@ -369,9 +378,14 @@ class DistUlyssesPath:
         rd, w = self.rd, self.w
         rec = (lambda name, i: ev[name][i].record()) if ev is not None else (lambda *_: None)
         rec("permute_in", 0)
-        qh = rd.ulysses_seq2head_dist(self.q, w.H_q)
-        kh = rd.ulysses_seq2head_dist(self.k, self.H_kv_rep)
-        vh = rd.ulysses_seq2head_dist(self.v, self.H_kv_rep)
+        if self.exchange == "p2p":
+            qh, kh, vh = rd.ulysses_seq2head_p2p_many([(self.q, self.pq, w.H_q),
+                                                       (self.k, self.pk, self.H_kv_rep),
+                                                       (self.v, self.pv, self.H_kv_rep)])
+        else:
+            qh = rd.ulysses_seq2head_dist(self.q, w.H_q)
+            kh = rd.ulysses_seq2head_dist(self.k, self.H_kv_rep)
+            vh = rd.ulysses_seq2head_dist(self.v, self.H_kv_rep)
         rec("permute_in", 1)
         rec("attn", 0)
         C, Lc = self.chunks, self.L // self.chunks
@@ -380,7 +394,10 @@ class DistUlyssesPath:
         rec("attn", 1)
         rec("permute_out", 0)
         # into the same buffer every step: the end-to-end leg reads it on another stream
-        rd.ulysses_head2seq_dist(self.o, out=self.o_seq)
+        if self.exchange == "p2p":
+            rd.ulysses_head2seq_p2p(self.o, self.po)
+        else:
+            rd.ulysses_head2seq_dist(self.o, out=self.o_seq)
         rec("permute_out", 1)
 
     def result(self):
@@ -574,6 +591,10 @@ def main():
     ap.add_argument("--workload", default="ulysses_e2e")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--exchange", choices=["nccl", "p2p"], default="nccl",
+                    help="N > 1 Ulysses step: NCCL all-to-alls with pack / unpack kernels, "
+                         "or one scatter kernel per rank into symmetric-memory buffers "
+                         "(the end-to-end leg is then skipped)")
     ap.add_argument("--ref-step-seconds", type=float, default=None,
                     help="reference arm: target seconds of oracle work per step")
     args = ap.parse_args()
@@ -603,7 +624,7 @@ def main():
 
     if world > 1 and kind == "ulysses" and DistUlyssesPath.splits(w, world):
         # N GPUs: the Ulysses layer with real all-to-alls between the ranks
-        path = DistUlyssesPath(w, device, rank, world)
+        path = DistUlyssesPath(w, device, rank, world, exchange=args.exchange)
     else:
         # one GPU, a workload without an exchange, or heads that do not split over N:
         # independent replicas
@@ -643,8 +664,11 @@ def main():
         out["config"].update({"global_batch": w.B, "seq_len": path.L, "heads_q": w.H_q,
                               "heads_kv": w.H_kv, "tokens_per_rank": path.Ls,
                               "heads_q_per_rank": path.Hq_l, "heads_kv_per_rank": path.Hkv_l,
-                              "exchange": "NCCL all-to-all between the ranks, pack/unpack "
-                                          "kernels around it"})
+                              "exchange": ("one scatter kernel per rank into the peers' "
+                                           "symmetric-memory buffers, a barrier on each side"
+                                           if args.exchange == "p2p" else
+                                           "NCCL all-to-all between the ranks, pack/unpack "
+                                           "kernels around it")})
     if kind == "ulysses":
         # Ulysses: P head groups; the ring x Ulysses hybrid: fewer, each with a ring
         out["config"]["head_groups"] = w.G
@@ -690,6 +714,11 @@ def main():
         # v, O, LSE, dO) and results (dq, dk, dv) are not what it moves, so no number
         out["e2e"] = None
         out["e2e_note"] = "not measured for backward workloads"
+    elif not args.no_e2e and dist_ulysses and args.exchange == "p2p":
+        # the peers store into this rank's output buffer during their next step, which the
+        # pipelined leg's copy stream would race
+        out["e2e"] = None
+        out["e2e_note"] = "not measured with the one-kernel exchange (--exchange p2p)"
     elif not args.no_e2e:
         # second buffer set for the pipelined end-to-end leg
         path2 = DistUlyssesPath(w, device, rank, world) if dist_ulysses else Path(kind, w, device)

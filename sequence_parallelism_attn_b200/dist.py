@@ -474,18 +474,28 @@ def ulysses_seq2head_p2p(x, peer: PeerBuffers, H_out: int | None = None):
     is this rank's sequence shard; every rank stores its share into every rank's buffer of
     `peer` ([B, P*Lc, H_out/P, D]), which is returned.  It stays valid until the next
     exchange through the same buffers."""
+    return ulysses_seq2head_p2p_many([(x, peer, H_out)])[0]
+
+
+def ulysses_seq2head_p2p_many(jobs):
+    """Several seq->head exchanges (Q, K, V) between one pair of barriers: jobs is a list of
+    (x, peer, H_out); returns the peers' buffers in order."""
     from . import ra
-    B, Lc, H_in, D = x.shape
-    H_out = H_in if H_out is None else H_out
-    want = (B, peer.world * Lc, H_out // peer.world, D)
-    if H_out % peer.world or H_out % H_in or tuple(peer.buf.shape) != want \
-            or peer.buf.dtype != x.dtype:
-        raise ValueError(f"peer buffers {tuple(peer.buf.shape)} {peer.buf.dtype} do not hold "
-                         f"{want} {x.dtype}")
-    peer.sync(f"seq2head scatter on rank {peer.rank}: buffers free")
-    ra.ra_ulysses_seq2head_scatter(x.contiguous(), peer.ptrs, peer.rank, H_out)
-    peer.sync(f"seq2head scatter on rank {peer.rank}: shares stored")
-    return peer.buf
+    for x, peer, H_out in jobs:
+        B, Lc, H_in, D = x.shape
+        H_out = H_in if H_out is None else H_out
+        want = (B, peer.world * Lc, H_out // peer.world, D)
+        if H_out % peer.world or H_out % H_in or tuple(peer.buf.shape) != want \
+                or peer.buf.dtype != x.dtype:
+            raise ValueError(f"peer buffers {tuple(peer.buf.shape)} {peer.buf.dtype} do not "
+                             f"hold {want} {x.dtype}")
+    first = jobs[0][1]
+    first.sync(f"seq2head scatter on rank {first.rank}: buffers free")
+    for x, peer, H_out in jobs:
+        ra.ra_ulysses_seq2head_scatter(x.contiguous(), peer.ptrs, peer.rank,
+                                       x.shape[2] if H_out is None else H_out)
+    first.sync(f"seq2head scatter on rank {first.rank}: shares stored")
+    return [peer.buf for _, peer, _ in jobs]
 
 
 def ulysses_head2seq_p2p(y, peer: PeerBuffers):

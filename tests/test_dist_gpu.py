@@ -251,3 +251,39 @@ def test_peer_exchange_on_one_rank(ra_lib, oracle_mod):
         del heads, seq, y, z
     finally:
         dist.destroy_process_group()
+
+
+def test_bench_dist_path_exchanges_agree_on_one_rank(ra_lib):
+    """bench.py's multi-GPU Ulysses step through a one-rank NCCL group with either exchange
+    (NCCL all-to-alls with pack / unpack, or the scatter kernels into symmetric memory):
+    the same bits of O in the sequence layout."""
+    import importlib.util
+    import os
+    import torch.distributed as dist
+    from sequence_parallelism_attn_b200 import synth
+    spec = importlib.util.spec_from_file_location(
+        "bench", os.path.join(os.path.dirname(os.path.dirname(__file__)), "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0,
+                            world_size=1, device_id=torch.device("cuda", 0))
+    try:
+        w = synth.UlyssesWorkload("dist_path_small", P=4, B=1, Lc=256, H_q=8, H_kv=2, D=128,
+                                  dtype=torch.bfloat16, causal=True, seed=77)
+        dev = torch.device("cuda", 0)
+        outs = []
+        for ex in ("nccl", "p2p"):
+            path = bench.DistUlyssesPath(w, dev, 0, 1, exchange=ex)
+            for _ in range(2):
+                path.step()
+            torch.cuda.synchronize()
+            outs.append(path.result().clone())
+            del path
+        assert ra_lib.ra_sync_status() == 0, ra_lib.ra_last_error()
+        assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+    finally:
+        dist.destroy_process_group()

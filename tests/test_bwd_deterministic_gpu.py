@@ -152,3 +152,36 @@ def test_det_setter_returns_previous(ra_lib):
     assert ra_lib.ra_set_bwd_deterministic(True) is True
     assert ra_lib.ra_set_bwd_deterministic(False) is True
     assert ra_lib.ra_set_bwd_deterministic(True) is False
+
+
+@pytest.mark.parametrize("layout", ["contiguous", "zigzag", "packed"])
+def test_det_full_size_matches_default_mode(ra_lib, layout):
+    """The bench's backward workload at full size (B = 1, L = 131072, H = 8, D = 128, causal;
+    zigzag shards; 20 packed documents): the deterministic mode's dK, dV are the default
+    mode's bits and its dQ the default mode's sum up to the order of its additions (the
+    default mode is checked against the oracle at this size in test_bwd_full_gpu.py); two
+    deterministic calls agree bit for bit."""
+    W = synth.LONG_128K
+    q, k, v = synth.attention_inputs(W, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(W.seed + 2)
+    dout = torch.randn(q.shape, generator=g, device="cuda").to(torch.bfloat16)
+    kw = {}
+    if layout == "zigzag":
+        kw["layout"] = "zigzag"
+    elif layout == "packed":
+        lens = synth.packed_lengths(W.L, W.seed + 21, 512, 32768)
+        kw["position_ids"] = synth.position_ids_from_lengths([lens]).cuda()
+    o, l = ra_lib.ring_attn_fwd(q, k, v, True, W.scale, out_dtype=torch.bfloat16, **kw)
+    det = ra_lib.ring_attn_bwd(q, k, v, o, l, dout, True, W.scale, **kw)
+    det2 = ra_lib.ring_attn_bwd(q, k, v, o, l, dout, True, W.scale, **kw)
+    assert ra_lib.ra_sync_status() == 0, ra_lib.ra_last_error()
+    for nm, a, b in zip(("dq", "dk", "dv"), det, det2):
+        assert torch.equal(a, b), f"{nm} differs between two deterministic calls"
+    del det2
+    ra_lib.ra_set_bwd_deterministic(False)
+    try:
+        fast = ra_lib.ring_attn_bwd(q, k, v, o, l, dout, True, W.scale, **kw)
+        assert ra_lib.ra_sync_status() == 0, ra_lib.ra_last_error()
+    finally:
+        ra_lib.ra_set_bwd_deterministic(True)
+    assert_same_grads(fast, det, f"full size, {layout}")

@@ -479,8 +479,10 @@ def ulysses_seq2head_p2p(x, peer: PeerBuffers, H_out: int | None = None):
 
 def ulysses_seq2head_p2p_many(jobs):
     """Several seq->head exchanges (Q, K, V) between one pair of barriers: jobs is a list of
-    (x, peer, H_out); returns the peers' buffers in order."""
+    (x, peer, H_out), every peer over the same group; returns the peers' buffers in order."""
     from . import ra
+    if any(peer.group is not jobs[0][1].group for _, peer, _ in jobs):
+        raise ValueError("the exchanges of one barrier pair must use one process group")
     for x, peer, H_out in jobs:
         B, Lc, H_in, D = x.shape
         H_out = H_in if H_out is None else H_out

@@ -500,3 +500,32 @@ def test_rank_leaving_is_reported_not_hung():
     # neighbour rank 0 gave up), never by waiting for good
     status, msg = res[1]
     assert status == "ok" and msg.startswith("ExchangeError"), msg
+
+
+def test_peer_exchange_rejects_mismatched_buffers():
+    """The one-kernel exchange checks its buffers before any barrier or kernel: a buffer of
+    another shape or dtype, heads that do not split over the ranks, or exchanges over two
+    groups in one barrier pair are refused (no process group, no GPU needed)."""
+    from types import SimpleNamespace
+    import torch
+    from sequence_parallelism_attn_b200 import dist as rd
+
+    def peer(shape, dtype=torch.bfloat16, world=2, group=None):
+        def sync(what):
+            raise AssertionError("no barrier may run for refused arguments")
+        return SimpleNamespace(buf=torch.empty(shape, dtype=dtype), world=world, rank=0,
+                               ptrs=[0] * world, group=group, sync=sync)
+
+    x = torch.empty(1, 16, 2, 64, dtype=torch.bfloat16)       # B, Lc, H_in, D
+    with pytest.raises(ValueError):
+        rd.ulysses_seq2head_p2p(x, peer((1, 32, 1, 64)), 4)   # wants (1, 32, 2, 64)
+    with pytest.raises(ValueError):
+        rd.ulysses_seq2head_p2p(x, peer((1, 32, 2, 64), torch.float32), 4)
+    with pytest.raises(ValueError):
+        rd.ulysses_seq2head_p2p(x, peer((1, 32, 1, 64)), 3)   # 3 heads over 2 ranks
+    with pytest.raises(ValueError):
+        rd.ulysses_seq2head_p2p_many([(x, peer((1, 32, 2, 64), group="a"), 4),
+                                      (x, peer((1, 32, 2, 64), group="b"), 4)])
+    y = torch.empty(1, 32, 2, 64, dtype=torch.bfloat16)       # B, P*Lc, Hl, D
+    with pytest.raises(ValueError):
+        rd.ulysses_head2seq_p2p(y, peer((1, 16, 2, 64)))      # wants (1, 16, 4, 64)

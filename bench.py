@@ -354,8 +354,9 @@ class DistUlyssesPath:
         self.chunks = w.P  # the attention walks the same chunk count as on one GPU
         self.o = torch.empty((w.B, L, self.Hq_l, w.D), dtype=torch.bfloat16, device=device)
         self.lse = torch.empty((w.B, self.Hq_l, L), dtype=torch.float32, device=device)
-        self.o_seq = torch.empty((w.B, self.Ls, w.H_q, w.D), dtype=w.dtype, device=device)
-        if exchange == "p2p":
+        if exchange != "p2p":
+            self.o_seq = torch.empty((w.B, self.Ls, w.H_q, w.D), dtype=w.dtype, device=device)
+        else:
             # the one-kernel exchange: every rank's scatter stores into these symmetric
             # buffers (the head blocks of Q, K, V and this rank's shard of O)
             pb = lambda *shape: rd.PeerBuffers(shape, w.dtype, device=device)
@@ -366,6 +367,8 @@ class DistUlyssesPath:
         self.scale = w.D ** -0.5
         self.flops = 4.0 * w.B * self.Hq_l * float(L) ** 2 * w.D / 2
         self.launches_per_step = 3 + 1 + (1 if w.B == 1 else 2) + (3 if w.B > 1 else 0)
+        if exchange == "p2p":
+            self.launches_per_step = 3 + 1 + 1  # Q, K, V scatters, attention, O scatter
         es = torch.tensor([], dtype=w.dtype).element_size()
         part = (world - 1) / world
         self.bytes_sent = int(es * w.B * self.Ls * w.D * part *
